@@ -1,0 +1,226 @@
+"""Plain, slow fp64 CPU oracle for Sketch Attention (SA) and STCA.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+benchmark's CPU-baseline leg may import this package.  The product path (the
+C-ABI library and its Python binding) never calls it, and it shares no code
+with the CUDA kernels: it reads plain arrays and writes plain arrays.
+
+Citations name the SequenceO1 paper ("SequenceO1: End-to-End Ultra-Long
+(100K) Sequence Modeling in Recommendation with Low-Rank Caching"), as given
+by its reading-note page (equations (1)-(36)) and its arXiv HTML text, by
+section and equation number.
+
+Readings where the pages leave a step open (each is an explicit choice):
+* SA value projection and per-prototype normalisation: the pages aggregate
+  raw X (eq. 9).  Here S = diag(1/(m+eps)) (A X) W_V with m_j = sum_i A_ji;
+  H = A X (the pages' X-tilde) is returned as well.
+* Softmax stabiliser: the per-token maximum over prototypes is subtracted
+  ("numerically robust softmax", Sec. 4.4 FlashSA); the result is unchanged.
+* STCA layer body: attention, optional output projection W_O, residual add
+  to the query (eq. 4 plus the W_O term of eq. 26); no FFN, no LayerNorm.
+* STCA over an empty key range: the attention output is zero.
+* Fusion: a linear map [z_r; z_u] W_F + b_F (Sec. 3.4 leaves the fusion open).
+
+Parity pins (tests/test_oracle_*.py): per-token column sums, total mass,
+permutation invariance, k = 1 mean, uniform assignment at zero logits,
+identical tokens, a two-prototype closed form that fixes the 1/sqrt(d) scale
+and the operand order, central finite differences for every gradient, STCA at
+L = 1, identical keys, torch SDPA in fp64, the eq. (24) reordering, and the
+analytic FLOP numbers the pages print.  No function here is "parity
+unpinned".
+"""
+from __future__ import annotations
+
+import math
+from typing import Optional, Sequence
+
+import numpy as np
+
+__all__ = [
+    "sa_forward", "sa_user", "sa_backward", "stca_branch", "stca_branch_reordered",
+    "stca_fuse", "assignment",
+]
+
+
+def _f64(a) -> np.ndarray:
+    return np.asarray(a, dtype=np.float64)
+
+
+def assignment(Xu, P, W_Q, W_K) -> np.ndarray:
+    """A in R^{k x n}: prototype-wise softmax of the affinities.
+
+    Affinities S = (P W_Q)(X W_K)^T / sqrt(d)            -- Sec. 3.1, eq. (6)
+    A_{j,i} = exp S_{j,i} / sum_j' exp S_{j',i}           -- eqs. (7)-(8)
+    so each token's column of A sums to one over the k prototypes.
+    """
+    Xu, P, W_Q, W_K = _f64(Xu), _f64(P), _f64(W_Q), _f64(W_K)
+    d = P.shape[1]
+    Q = P @ W_Q                       # k x d
+    K = Xu @ W_K                      # n x d
+    Z = (Q @ K.T) / math.sqrt(d)      # k x n, eq. (6)
+    Zc = Z - Z.max(axis=0, keepdims=True)
+    E = np.exp(Zc)
+    return E / E.sum(axis=0, keepdims=True)   # softmax over prototypes, eq. (8)
+
+
+def sa_user(Xu, P, W_Q, W_K, W_V, eps: float):
+    """One user's sketch.  Returns (S, m, H) with
+    H = A X (eq. 9), m_j = sum_i A_{j,i}, S = diag(1/(m+eps)) H W_V."""
+    Xu = _f64(Xu)
+    k, d = np.shape(P)
+    if Xu.shape[0] == 0:
+        return np.zeros((k, d)), np.zeros(k), np.zeros((k, d))
+    A = assignment(Xu, P, W_Q, W_K)
+    m = A.sum(axis=1)
+    H = A @ Xu                                  # eq. (9)
+    S = (H / (m + eps)[:, None]) @ _f64(W_V)
+    return S, m, H
+
+
+def sa_forward(X, offsets: Sequence[int], P, W_Q, W_K, W_V, eps: float):
+    """Sketches of a ragged batch: users own rows [offsets[u], offsets[u+1]).
+
+    Returns S [B,k,d], mass [B,k], H [B,k,d] in fp64.
+    """
+    offsets = np.asarray(offsets, np.int64)
+    B = len(offsets) - 1
+    k, d = np.shape(P)
+    S = np.zeros((B, k, d))
+    mass = np.zeros((B, k))
+    H = np.zeros((B, k, d))
+    for u in range(B):
+        S[u], mass[u], H[u] = sa_user(X[offsets[u]:offsets[u + 1]], P, W_Q, W_K, W_V, eps)
+    return S, mass, H
+
+
+def sa_backward(X, offsets, P, W_Q, W_K, W_V, eps: float, dS, dmass=None):
+    """Gradients of sum_u <dS_u, S_u> + <dmass_u, m_u> with respect to
+    X, P, W_Q, W_K, W_V (weights are shared, so their gradients sum over users).
+
+    The pages state that SA is differentiable end to end (Sec. 3.1) but print
+    no backward; these are the chain-rule derivatives of the forward above,
+    written out step by step:
+        Hh = H/(m+eps),  dW_V += Hh^T G,  dHh = G W_V^T
+        dH_j = dHh_j/(m_j+eps),  dm_j = -(dHh_j . H_j)/(m_j+eps)^2 + dmass_j
+        dA_ji = dH_j . x_i + dm_j,  c_i = sum_j A_ji dA_ji
+        dZ_ji = A_ji (dA_ji - c_i)
+        dQ = dZ K/sqrt(d),  dK = dZ^T Q/sqrt(d)
+        dX = A^T dH + dK W_K^T,  dP += dQ W_Q^T,  dW_Q += P^T dQ,  dW_K += X^T dK
+    """
+    X = _f64(X)
+    P, W_Q, W_K, W_V = _f64(P), _f64(W_Q), _f64(W_K), _f64(W_V)
+    offsets = np.asarray(offsets, np.int64)
+    B = len(offsets) - 1
+    k, d = P.shape
+    dX = np.zeros_like(X)
+    dP = np.zeros_like(P)
+    dW_Q = np.zeros_like(W_Q)
+    dW_K = np.zeros_like(W_K)
+    dW_V = np.zeros_like(W_V)
+    Q = P @ W_Q
+    for u in range(B):
+        lo, hi = int(offsets[u]), int(offsets[u + 1])
+        if hi == lo:
+            continue
+        Xu = X[lo:hi]
+        G = _f64(dS[u])
+        A = assignment(Xu, P, W_Q, W_K)
+        m = A.sum(axis=1)
+        H = A @ Xu
+        Hh = H / (m + eps)[:, None]
+        dW_V += Hh.T @ G
+        dHh = G @ W_V.T
+        dH = dHh / (m + eps)[:, None]
+        dm = -np.sum(dHh * H, axis=1) / (m + eps) ** 2
+        if dmass is not None:
+            dm = dm + _f64(dmass[u])
+        dA = dH @ Xu.T + dm[:, None]               # k x n
+        c = np.sum(A * dA, axis=0, keepdims=True)  # 1 x n
+        dZ = A * (dA - c)
+        K = Xu @ W_K
+        dQ = dZ @ K / math.sqrt(d)
+        dK = dZ.T @ Q / math.sqrt(d)
+        dX[lo:hi] = A.T @ dH + dK @ W_K.T
+        dP += dQ @ W_Q.T
+        dW_Q += P.T @ dQ
+        dW_K += Xu.T @ dK
+    return dX, dP, dW_Q, dW_K, dW_V
+
+
+# --------------------------------------------------------------------------
+# STCA
+# --------------------------------------------------------------------------
+def _softmax_rows(s: np.ndarray) -> np.ndarray:
+    s = s - s.max(axis=1, keepdims=True)
+    e = np.exp(s)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def stca_branch(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: int, d_h: int):
+    """Stacked target-to-history single-query cross attention, direct form.
+
+    One layer (Sec. 2.3, eq. (4)), per head h:
+        alpha = softmax((q W_Q^h)(X W_K^h)^T / sqrt(d_h))   over the L keys
+        o_h   = alpha (X W_V^h)
+    then q <- q + concat_h(o_h) W_O (W_O = identity when absent).
+    Candidates of user u are rows [cand_offsets[u], cand_offsets[u+1]) of q;
+    their keys/values are rows [kv_begin[u], kv_end[u]) of kv.
+    ``layers`` is a list of objects with W_Q, W_K, W_V ([heads, D, d_h]) and
+    W_O ([heads*d_h, D] or None).
+    """
+    out = _f64(q).copy()
+    kv = _f64(kv)
+    cand_offsets = np.asarray(cand_offsets, np.int64)
+    for u in range(len(cand_offsets) - 1):
+        c0, c1 = int(cand_offsets[u]), int(cand_offsets[u + 1])
+        if c1 == c0:
+            continue
+        Xu = kv[int(kv_begin[u]):int(kv_end[u])]
+        qu = out[c0:c1]
+        for lay in layers:
+            o = np.zeros((c1 - c0, heads * d_h))
+            if Xu.shape[0] > 0:
+                for h in range(heads):
+                    Wq, Wk, Wv = _f64(lay.W_Q[h]), _f64(lay.W_K[h]), _f64(lay.W_V[h])
+                    scores = (qu @ Wq) @ (Xu @ Wk).T / math.sqrt(d_h)
+                    alpha = _softmax_rows(scores)
+                    o[:, h * d_h:(h + 1) * d_h] = alpha @ (Xu @ Wv)
+            qu = qu + (o if lay.W_O is None else o @ _f64(lay.W_O))
+        out[c0:c1] = qu
+    return out
+
+
+def stca_branch_reordered(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: int, d_h: int):
+    """The same layers in the single-query reordering of Sec. 5.1, eq. (24):
+        u = (q W_Q^h) W_K^h^T,  alpha = softmax(u X^T / sqrt(d_h)),  o = (alpha X) W_V^h.
+    Keys and values are the raw history rows.  Used only as a cross-check of
+    ``stca_branch``."""
+    out = _f64(q).copy()
+    kv = _f64(kv)
+    cand_offsets = np.asarray(cand_offsets, np.int64)
+    for u in range(len(cand_offsets) - 1):
+        c0, c1 = int(cand_offsets[u]), int(cand_offsets[u + 1])
+        if c1 == c0:
+            continue
+        Xu = kv[int(kv_begin[u]):int(kv_end[u])]
+        qu = out[c0:c1]
+        for lay in layers:
+            o = np.zeros((c1 - c0, heads * d_h))
+            if Xu.shape[0] > 0:
+                for h in range(heads):
+                    Wq, Wk, Wv = _f64(lay.W_Q[h]), _f64(lay.W_K[h]), _f64(lay.W_V[h])
+                    uvec = (qu @ Wq) @ Wk.T
+                    alpha = _softmax_rows(uvec @ Xu.T / math.sqrt(d_h))
+                    o[:, h * d_h:(h + 1) * d_h] = (alpha @ Xu) @ Wv
+            qu = qu + (o if lay.W_O is None else o @ _f64(lay.W_O))
+        out[c0:c1] = qu
+    return out
+
+
+def stca_fuse(z_r, z_u, W_F, b_F=None):
+    """Linear fusion of the two branches: [z_r ; z_u] W_F + b_F (Sec. 3.4)."""
+    z = np.concatenate([_f64(z_r), _f64(z_u)], axis=1)
+    out = z @ _f64(W_F)
+    if b_F is not None:
+        out = out + _f64(b_F)[None, :]
+    return out
