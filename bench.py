@@ -1,0 +1,441 @@
+#!/usr/bin/env python
+"""Benchmark of the SA / STCA hot path on B200.
+
+A step is one pass of the whole hot path over one batch: sa_forward and
+sa_backward over 64 ragged users (mean 85K events, k=1024, d=128, bf16), then
+STCA on the produced sketches and on each user's last 10K events against 256
+candidates per user, then the linear fusion.  The headline metric is SA
+history tokens per second (k=1024, d=128); STCA candidates per second and the
+per-phase rates are reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun, one process per GPU, NCCL) every rank runs its own
+batch (weak scaling) and the weight gradients are all-reduced, the one
+exchange step of data-parallel SA training.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SA history-tokens/s (k=1024,d=128) + % of roofline; STCA candidates/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SMS, FP32_LANES = 148, 128
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"sa_bench_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
+                "samples": len(rows), "reasons": reasons}
+
+
+# --------------------------------------------------------------------------
+# workloads on the device
+def _dev_bf16(bits, device):
+    return torch.from_numpy(bits.view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def _f32(a, device):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+
+
+class TrainStepRunner:
+    """Device buffers and the step of the end-to-end training workload."""
+
+    def __init__(self, w, device, world):
+        import sketch_attention_b200 as sab
+        self.sab, self.w, self.dev, self.world = sab, w, device, world
+        sa = w.sa
+        self.B, self.k, self.d = sa.B, sa.k, sa.d
+        self.off = sa.offsets
+        self.X = _dev_bf16(sa.X, device)
+        self.offd = torch.from_numpy(self.off).to(device)
+        self.P, self.WQ, self.WK, self.WV = (_f32(a, device) for a in (sa.P, sa.W_Q, sa.W_K, sa.W_V))
+        self.dS = _f32(sa.dS, device)
+        self.q = _dev_bf16(w.q, device)
+        self.cand = w.cand_offsets
+        self.candd = torch.from_numpy(self.cand).to(device)
+        self.rb, self.re = w.recent_begin, w.recent_end
+        self.rbd, self.red = torch.from_numpy(self.rb).to(device), torch.from_numpy(self.re).to(device)
+        self.sb = np.arange(self.B, dtype=np.int64) * self.k
+        self.se = self.sb + self.k
+        self.sbd, self.sed = torch.from_numpy(self.sb).to(device), torch.from_numpy(self.se).to(device)
+        lay = lambda L: dict(W_Q=_f32(L.W_Q, device), W_K=_f32(L.W_K, device),
+                             W_V=_f32(L.W_V, device), W_O=_f32(L.W_O, device))
+        self.layers_r = [lay(L) for L in w.layers_r]
+        self.layers_u = [lay(L) for L in w.layers_u]
+        self.WF, self.bF = _f32(w.W_F, device), _f32(w.b_F, device)
+        B, k, d, C = self.B, self.k, self.d, int(self.cand[-1])
+        n = sa.n_total
+        e = lambda *s, dt=torch.float32: torch.empty(*s, device=device, dtype=dt)
+        self.fo = {"S": e(B, k, d), "mass": e(B, k), "H": e(B, k, d), "S_bf16": e(B, k, d, dt=torch.bfloat16)}
+        self.go = {"dX": e(n, d, dt=torch.bfloat16), "dP": e(k, d), "dW_Q": e(d, d), "dW_K": e(d, d), "dW_V": e(d, d)}
+        self.zr, self.zu, self.z = e(C, d), e(C, d), e(C, d)
+        sab_ws = lambda nbytes: torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+        self.ws_f = sab_ws(sab.sa_forward_workspace(B, n, k, d, sab.SA_BF16))
+        self.ws_b = sab_ws(sab.sa_backward_workspace(B, n, k, d, sab.SA_BF16))
+        self.ws_s = sab_ws(sab.stca_forward_workspace(B, C, d, w.heads, w.d_h, sab.SA_BF16))
+        self.tokens = n
+        self.cands = C
+        self.phase_events = None
+
+    def step(self, phases=None):
+        sab, w = self.sab, self.w
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if phases is not None else None
+        if ev: ev[0].record()
+        fwd = sab.sa_forward(self.X, self.off, self.P, self.WQ, self.WK, self.WV, w.sa.eps,
+                             offsets_dev=self.offd, out=self.fo, workspace=self.ws_f)
+        if ev: ev[1].record()
+        g = sab.sa_backward(self.X, self.off, self.P, self.WQ, self.WK, self.WV, w.sa.eps,
+                            fwd["H"], fwd["mass"], self.dS, offsets_dev=self.offd, out=self.go,
+                            workspace=self.ws_b)
+        if self.world > 1:
+            for name in ("dP", "dW_Q", "dW_K", "dW_V"):
+                torch.distributed.all_reduce(g[name])
+        if ev: ev[2].record()
+        sab.stca_forward(self.q, self.cand, self.X, self.rb, self.re, self.layers_r, w.heads, w.d_h,
+                         cand_offsets_dev=self.candd, kv_begin_dev=self.rbd, kv_end_dev=self.red,
+                         out=self.zr, workspace=self.ws_s)
+        sk = fwd["S_bf16"].view(self.B * self.k, self.d)
+        sab.stca_forward(self.q, self.cand, sk, self.sb, self.se, self.layers_u, w.heads, w.d_h,
+                         cand_offsets_dev=self.candd, kv_begin_dev=self.sbd, kv_end_dev=self.sed,
+                         out=self.zu, workspace=self.ws_s)
+        sab.stca_fuse(self.zr, self.zu, self.WF, self.bF, out=self.z)
+        if ev:
+            ev[3].record()
+            phases.append(ev)
+        return self.z, g
+
+    def results_nbytes(self):
+        return self.z.numel() * 4 + sum(self.go[n].numel() * 4 for n in ("dP", "dW_Q", "dW_K", "dW_V"))
+
+
+# Per-kernel algorithmic work (flops) per launch, for the roofline of the
+# dominant kernel.  tokens = history tokens of the call.
+def kernel_model(name, w):
+    k, d = w.sa.k, w.sa.d
+    n = w.sa.n_total
+    if name in ("sa_fwd_tc_kernel",):
+        return "tensor", 4.0 * k * d * n
+    if name == "sa_lse_kernel":
+        return "alu", 2.0 * k * d * n
+    if name == "sa_agg_kernel":
+        return "alu", 2.0 * k * d * n
+    if name == "sa_bwd_token_kernel":
+        return "alu", 8.0 * k * d * n
+    if name == "sa_bwd_E_kernel":
+        return "alu", 2.0 * k * d * n
+    if name.startswith("sa_bwd_tc"):
+        return "tensor", 10.0 * k * d * n
+    if name.startswith("stca_attn"):
+        # one launch: one layer of one branch; the two branches differ in L
+        C = int(w.cand_offsets[-1])
+        L_avg = 0.5 * (float(np.mean(w.recent_end - w.recent_begin)) + k)
+        return ("tensor" if "tc" in name else "alu"), 4.0 * L_avg * d * C * w.heads
+    return None, None
+
+
+def run_ours(args, rank, world, device):
+    import sketch_attention_b200 as sab
+    from sketch_attention_b200 import build as _b
+    if rank == 0 or not os.path.exists(_b.LIB):
+        _b.build()
+    if world > 1:
+        torch.distributed.barrier()
+    sab.load()
+    from sa_inputs import TRAIN_STEP_WORKLOAD, train_step_workload
+    t0 = time.time()
+    w = train_step_workload()
+    gen_s = time.time() - t0
+    R = TrainStepRunner(w, device, world)
+    peaks, peaks_src = load_peaks()
+
+    for _ in range(args.warmup):
+        R.step()
+    torch.cuda.synchronize()
+    phases = []
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sab.profile(True)
+    launches0 = sab.launch_count()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        start.record()
+        for _ in range(args.steps):
+            R.step(phases)
+        end.record()
+        torch.cuda.synchronize()
+    launches = sab.launch_count() - launches0
+    prof = sab.profile_read()
+    sab.profile(False)
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end) / args.steps
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms = float(t.item())
+    ph = np.array([[a.elapsed_time(b) for a, b in zip(e[:-1], e[1:])] for e in phases])
+    ph_ms = ph.mean(axis=0) if len(ph) else np.zeros(3)
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hX = torch.empty(R.X.shape, dtype=torch.bfloat16, pin_memory=True)
+        hX.copy_(R.X)
+        hq = torch.empty(R.q.shape, dtype=torch.bfloat16, pin_memory=True)
+        hq.copy_(R.q)
+        hdS = torch.empty(R.dS.shape, dtype=torch.float32, pin_memory=True)
+        hdS.copy_(R.dS)
+        hz = torch.empty(R.z.shape, dtype=torch.float32, pin_memory=True)
+        hg = {n: torch.empty(R.go[n].shape, dtype=torch.float32, pin_memory=True)
+              for n in ("dP", "dW_Q", "dW_K", "dW_V")}
+        torch.cuda.synchronize()
+
+        def e2e_step():
+            R.X.copy_(hX, non_blocking=True)
+            R.q.copy_(hq, non_blocking=True)
+            R.dS.copy_(hdS, non_blocking=True)
+            z, g = R.step()
+            hz.copy_(z, non_blocking=True)
+            for n in hg:
+                hg[n].copy_(g[n], non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e2.record()
+        torch.cuda.synchronize()
+        e2e_ms = s2.elapsed_time(e2) / args.steps
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        if world > 1:
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        h2d = hX.numel() * 2 + hq.numel() * 2 + hdS.numel() * 4
+        d2h = R.results_nbytes()
+        e2e = {"value": world * R.tokens / (e2e_ms / 1e3), "unit": "history-tokens/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    # ---- roofline of the dominant kernel
+    roof = None
+    if prof:
+        dom = max(prof.items(), key=lambda kv: kv[1][0])
+        name, (tot_ms, cnt) = dom
+        bound, flops = kernel_model(name, w)
+        if bound is not None:
+            avg_s = tot_ms / cnt / 1e3
+            achieved = flops / avg_s / 1e12
+            if bound == "tensor":
+                peak = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+                peak_note = f"bf16 dense, sustained ({peaks_src})"
+            else:
+                mhz = peaks.get("sm_max_mhz", 1965.0)
+                peak = SMS * FP32_LANES * 2 * mhz * 1e6 / 1e12
+                peak_note = f"fp32 FMA: {SMS} SMs x {FP32_LANES} lanes x 2 x {mhz:.0f} MHz"
+            roof = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak,
+                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                    "peak_source": peak_note, "avg_launch_ms": tot_ms / cnt,
+                    "launches": cnt, "share_of_step": tot_ms / (ms * args.steps)}
+    kernels = {n: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+               for n, v in sorted(prof.items(), key=lambda kv: -kv[1][0])}
+
+    tokens = R.tokens
+    value = world * tokens / (ms / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "history-tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded item+action events (Zipf(1.1) ids over 1M items), lognormal lengths",
+        "config": {"workload": TRAIN_STEP_WORKLOAD, "users_per_gpu": R.B,
+                   "history_tokens_per_gpu": tokens, "k": R.k, "d": R.d,
+                   "stca_candidates_per_gpu": R.cands, "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (X is %.2f GB per GPU)" % (R.X.numel() * 2 / 1e9)},
+        "phases": {"sa_forward_ms": float(ph_ms[0]), "sa_backward_ms": float(ph_ms[1]),
+                   "stca_fuse_ms": float(ph_ms[2]),
+                   "sa_forward_tokens_per_s": tokens / (ph_ms[0] / 1e3) if ph_ms[0] else None,
+                   "sa_backward_tokens_per_s": tokens / (ph_ms[1] / 1e3) if ph_ms[1] else None,
+                   "stca_candidates_per_s": R.cands / (ph_ms[2] / 1e3) if ph_ms[2] else None},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": int(launches),
+        "e2e": e2e,
+        "clocks": clk.summary(),
+        "input_generation_s": gen_s,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, 30_000)
+    return line
+
+
+# --------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and the reference arm)
+def _oracle_sample(w, n_tokens=None):
+    """One bounded sample of the step: user 0's forward and backward (its first
+    n_tokens events) plus STCA of its 256 candidates on both branches and the
+    fusion, all by the fp64 oracle."""
+    import oracle
+    from sa_inputs import bf16_to_f64
+    sa = w.sa
+    lo, hi = int(sa.offsets[0]), int(sa.offsets[1])
+    if n_tokens is not None:
+        hi = min(hi, lo + n_tokens)
+    X = sa.x_f64(lo, hi)
+    t0 = time.perf_counter()
+    S, m, H = oracle.sa_forward(X, [0, hi - lo], sa.P, sa.W_Q, sa.W_K, sa.W_V, sa.eps)
+    oracle.sa_backward(X, [0, hi - lo], sa.P, sa.W_Q, sa.W_K, sa.W_V, sa.eps, sa.dS[:1])
+    c0, c1 = int(w.cand_offsets[0]), int(w.cand_offsets[1])
+    q = bf16_to_f64(w.q[c0:c1])
+    rb = max(lo, hi - 10_000)
+    zr = oracle.stca_branch(q, [0, c1 - c0], X, [rb - lo], [hi - lo], w.layers_r, w.heads, w.d_h)
+    zu = oracle.stca_branch(q, [0, c1 - c0], S[0], [0], [sa.k], w.layers_u, w.heads, w.d_h)
+    oracle.stca_fuse(zr, zu, w.W_F, w.b_F)
+    return hi - lo, time.perf_counter() - t0
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, n_tokens=None):
+    n, secs = _oracle_sample(w, n_tokens)
+    return {"value": n / secs, "unit": "history-tokens/s", "cores": _cores(), "kind": "oracle",
+            "sample": f"user 0 ({n} events) forward+backward, STCA on its 256 candidates "
+                      f"(both branches), fusion; fp64 numpy, {secs:.1f} s"}
+
+
+def run_reference(args):
+    from sa_inputs import TRAIN_STEP_WORKLOAD, train_step_workload
+    w = train_step_workload(users=1)
+    for _ in range(args.warmup):
+        _oracle_sample(w, 20_000)
+    times, n = [], 0
+    for _ in range(args.steps):
+        n, s = _oracle_sample(w, 20_000)
+        times.append(s)
+    ms = 1e3 * float(np.mean(times))
+    value = n / (ms / 1e3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "history-tokens/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same generator as the GPU arm)",
+        "config": {"workload": TRAIN_STEP_WORKLOAD, "sample": "user 0, first 20000 events"},
+        "cpu_baseline": {"value": value, "unit": "history-tokens/s", "cores": _cores(),
+                         "kind": "oracle",
+                         "sample": "per step: user 0's first 20000 events forward+backward, STCA "
+                                   "on its 256 candidates (both branches), fusion"},
+        "e2e": {"value": value, "unit": "history-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=device)
+    try:
+        line = run_ours(args, rank, world, device)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * sketch_attn.h -- C ABI of the Sketch Attention (SA) / STCA library for one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operations are those of the SequenceO1 paper ("SequenceO1: End-to-End
+ * Ultra-Long (100K) Sequence Modeling in Recommendation with Low-Rank
+ * Caching"); each entry point cites the section and equation it computes.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Row-major arrays, row-vector convention (x W).
+ *  - Pointers named *_host are host memory and are read during the call only;
+ *    every other pointer is device memory owned by the caller.  The library
+ *    allocates nothing: scratch memory is the caller's `workspace`, whose size
+ *    the matching *_workspace() query returns for the current device.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Outputs are fully overwritten, never accumulated into.
+ *  - Ragged users: user u owns rows [offsets[u], offsets[u+1]) of X;
+ *    offsets[0] = 0, offsets non-decreasing, offsets[B] = total rows.  Both a
+ *    host copy (validated, used for sizes) and a device copy (read by the
+ *    kernels) are passed; they must hold the same values.
+ *  - Errors are status codes.  Nothing is thrown across the ABI, nothing
+ *    aborts, and no kernel traps.  sa_last_error() returns a message for the
+ *    calling thread's last failing call.  Device pointers must be 16-byte
+ *    aligned.
+ *  - Numbers: weights and outputs are fp32.  X, STCA queries and keys are
+ *    fp32 (SA_F32) or bf16 (SA_BF16).  bf16 paths multiply bf16 operands on
+ *    the tensor cores with fp32 accumulation; fp32 paths use fp32 FMA.
+ */
+#ifndef SKETCH_ATTN_H
+#define SKETCH_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,   /* bad pointer, size, offsets or alignment     */
+  SA_ERR_UNSUPPORTED = 2,   /* valid but outside the supported shapes      */
+  SA_ERR_CUDA = 3,          /* a CUDA runtime call failed                  */
+  SA_ERR_TIMEOUT = 4,       /* a device-side wait gave up (see poll below) */
+  SA_ERR_WORKSPACE = 5      /* workspace NULL or smaller than the query    */
+} sa_status;
+
+typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
+
+/* cudaStream_t without including the CUDA headers. */
+typedef struct CUstream_st* sa_stream_t;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int sa_version(void);
+
+/* Message describing the calling thread's last non-OK status. */
+const char* sa_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word.  Returns SA_ERR_TIMEOUT if a kernel's bounded wait expired since the
+ * last poll, SA_ERR_CUDA on a CUDA error, else SA_OK.
+ */
+sa_status sa_poll_device_status(sa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Sketch Attention forward                                                  */
+/* ------------------------------------------------------------------------ */
+/*
+ * Bytes of workspace sa_forward needs for these sizes on the current device.
+ */
+size_t sa_forward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype);
+
+/*
+ * sa_forward -- the sketch of every user (paper Sec. 3.1, eqs. (6)-(9)).
+ *
+ * Per user u with history X_u (n_u x d):
+ *   Z   = (P W_Q)(X_u W_K)^T / sqrt(d)                    eq. (6), k x n_u
+ *   A   = softmax over the k prototypes of each column    eqs. (7)-(8)
+ *   H_u = A X_u                                           eq. (9)
+ *   m_u = row sums of A (mass of each prototype)
+ *   S_u = diag(1/(m_u + eps)) H_u W_V
+ * The value projection W_V and the division by (m + eps) are this library's
+ * reading; with W_V = I and eps = 0 the pages' sketch is H = S diag(m).
+ * The k x n_u matrices Z and A are never written to memory.
+ *
+ * X        [n_total, d] x_dtype; n_total = offsets_host[B].
+ * P        [k, d] fp32 prototypes; W_Q, W_K, W_V [d, d] fp32.
+ * S        [B, k, d] fp32 out.   mass [B, k] fp32 out.
+ * H        [B, k, d] fp32 out, optional (NULL): the unnormalised A X, which
+ *          sa_backward needs.
+ * S_bf16   [B, k, d] bf16 out, optional (NULL): S rounded to bf16 (for STCA).
+ * A user with n_u = 0 gets S = 0, mass = 0, H = 0.
+ * Supported: 1 <= k <= 4096, d in {64, 128}, B >= 1, eps >= 0.
+ */
+sa_status sa_forward(const void* X, sa_dtype x_dtype,
+                     const int64_t* offsets_host, const int64_t* offsets_dev, int B,
+                     int k, int d,
+                     const float* P, const float* W_Q, const float* W_K, const float* W_V,
+                     float eps,
+                     float* S, float* mass, float* H, void* S_bf16,
+                     void* workspace, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Sketch Attention backward                                                 */
+/* ------------------------------------------------------------------------ */
+size_t sa_backward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype);
+
+/*
+ * sa_backward -- gradients of L = sum_u <dS_u, S_u> + <dmass_u, m_u> through
+ * sa_forward (the pages call SA fully differentiable, Sec. 3.1, and print no
+ * backward; these are the chain-rule derivatives of the forward above):
+ *   Hh = H/(m+eps); dW_V = sum_u Hh^T dS; dHh = dS W_V^T
+ *   dH = dHh/(m+eps); dm = -(dHh . Hh)/(m+eps) + dmass
+ *   dA_ji = dH_j . x_i + dm_j;  c_i = sum_j A_ji dA_ji;  dZ = A o (dA - c)
+ *   dX_i = sum_j A_ji dH_j + sum_j dZ_ji p'_j,  p'_j = row j of P W_Q W_K^T / sqrt(d)
+ *   E = sum_u dZ_u X_u;  dP = E W_K W_Q^T/sqrt(d);  dW_Q = P^T E W_K/sqrt(d);
+ *   dW_K = E^T P W_Q/sqrt(d)
+ *
+ * Inputs as sa_forward, plus H and mass from sa_forward, dS [B,k,d] fp32 and
+ * dmass [B,k] fp32 (NULL = zero).
+ * dX [n_total, d] x_dtype out; dP [k,d], dW_Q, dW_K, dW_V [d,d] fp32 out
+ * (sums over the batch).
+ */
+sa_status sa_backward(const void* X, sa_dtype x_dtype,
+                      const int64_t* offsets_host, const int64_t* offsets_dev, int B,
+                      int k, int d,
+                      const float* P, const float* W_Q, const float* W_K, const float* W_V,
+                      float eps,
+                      const float* H, const float* mass, const float* dS, const float* dmass,
+                      void* dX, float* dP, float* dW_Q, float* dW_K, float* dW_V,
+                      void* workspace, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* STCA: stacked target-to-history single-query cross attention             */
+/* ------------------------------------------------------------------------ */
+/* Weights of one STCA layer (device pointers). */
+typedef struct {
+  const float* W_Q;   /* [heads, D, d_h] */
+  const float* W_K;   /* [heads, D, d_h] */
+  const float* W_V;   /* [heads, D, d_h] */
+  const float* W_O;   /* [heads*d_h, D], or NULL for the identity (needs heads*d_h == D) */
+} stca_layer;
+
+size_t stca_forward_workspace(int B, int64_t C_total, int D, int heads, int d_h, sa_dtype dtype);
+
+/*
+ * stca_forward -- one STCA branch over a batch of users (paper Sec. 2.3
+ * eq. (4), evaluated in the single-query reordering of Sec. 5.1 eq. (24)).
+ * For every candidate query q of user u and every layer:
+ *   for each head h:  u_h = (q W_Q^h) W_K^h^T
+ *                     alpha = softmax_i(u_h . x_i / sqrt(d_h)),  i in [kv_begin[u], kv_end[u])
+ *                     o_h = (sum_i alpha_i x_i) W_V^h
+ *   q <- q + concat_h(o_h) W_O
+ * Keys and values are the raw history rows x_i.  An empty key range gives
+ * o = 0.  The recent branch passes the last L_r events of each history
+ * (eq. 3); the sketch branch passes the sketches (eq. 19).
+ *
+ * q       [C_total, D] dtype: candidate targets, user u owns rows
+ *         [cand_offsets[u], cand_offsets[u+1]).
+ * kv      [kv_rows, D] dtype; 0 <= kv_begin[u] <= kv_end[u] <= kv_rows.
+ * layers  host array of n_layers weight sets (device pointers inside).
+ * out     [C_total, D] fp32: the query after the last layer.
+ * Supported: D == 128, heads*d_h <= 4096, n_layers >= 1.
+ */
+sa_status stca_forward(const void* q, sa_dtype dtype,
+                       const int64_t* cand_offsets_host, const int64_t* cand_offsets_dev, int B,
+                       const void* kv, int64_t kv_rows,
+                       const int64_t* kv_begin_host, const int64_t* kv_end_host,
+                       const int64_t* kv_begin_dev, const int64_t* kv_end_dev,
+                       int D, int heads, int d_h, int n_layers, const stca_layer* layers,
+                       float* out, void* workspace, size_t ws_bytes, sa_stream_t stream);
+
+/*
+ * stca_fuse -- linear fusion of the two branches (paper Sec. 3.4 leaves the
+ * fusion to a light MLP or gate; this library applies one linear layer):
+ *   out = [z_r ; z_u] W_F + b_F
+ * z_r, z_u [C, D] fp32; W_F [2D, D] fp32; b_F [D] fp32 or NULL; out [C, D].
+ */
+sa_status stca_fuse(const float* z_r, const float* z_u, const float* W_F, const float* b_F,
+                    int64_t C, int D, float* out, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Measurement support (not part of the method)                              */
+/* ------------------------------------------------------------------------ */
+/* Number of kernels this library has launched in this process. */
+long long sa_launch_count(void);
+
+/*
+ * enable = 1 clears the kernel timers and starts recording a CUDA event pair
+ * on the launch stream around each launch of the library's kernels; 0 stops.
+ * Costs one event record per launch boundary; results are read below.
+ */
+sa_status sa_profile(int enable);
+
+/*
+ * Per-kernel device time since sa_profile(1), summed from the event pairs
+ * (synchronises on them).  Fills entry i (0-based) and returns 1, or returns
+ * 0 when i is past the last kernel.  `name` receives at most name_len bytes.
+ */
+int sa_profile_read(int i, char* name, int name_len, double* total_ms, long long* launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKETCH_ATTN_H */

@@ -13,7 +13,8 @@ section and equation number.
 Readings where the pages leave a step open (each is an explicit choice):
 * SA value projection and per-prototype normalisation: the pages aggregate
   raw X (eq. 9).  Here S = diag(1/(m+eps)) (A X) W_V with m_j = sum_i A_ji;
-  H = A X (the pages' X-tilde) is returned as well.
+  H = A X (the pages' X-tilde) is returned as well.  A prototype whose
+  m_j + eps is zero (eps = 0 and no mass) gets S_j = 0.
 * Softmax stabiliser: the per-token maximum over prototypes is subtracted
   ("numerically robust softmax", Sec. 4.4 FlashSA); the result is unchanged.
 * STCA layer body: attention, optional output projection W_O, residual add
@@ -73,7 +74,9 @@ def sa_user(Xu, P, W_Q, W_K, W_V, eps: float):
     A = assignment(Xu, P, W_Q, W_K)
     m = A.sum(axis=1)
     H = A @ Xu                                  # eq. (9)
-    S = (H / (m + eps)[:, None]) @ _f64(W_V)
+    denom = (m + eps)[:, None]
+    Hh = np.divide(H, denom, out=np.zeros_like(H), where=denom > 0)   # empty prototype -> 0
+    S = Hh @ _f64(W_V)
     return S, m, H
 
 

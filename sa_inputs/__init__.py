@@ -39,8 +39,10 @@ N_ACTIONS = 8              # action types per event
 def bf16_bits(a: np.ndarray) -> np.ndarray:
     """fp32 -> bf16 bit patterns (uint16), round to nearest even."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    assert np.isfinite(a).all()
+    u = a.view(np.uint32)
+    # finite values: the sum stays below 2^32
+    rounded = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
     return rounded.astype(np.uint16)
 
 
@@ -67,7 +69,9 @@ def rng_for(seed: int) -> np.random.Generator:
 
 
 def gauss(rng, shape, std: float) -> np.ndarray:
-    return (rng.standard_normal(shape, dtype=np.float32) * np.float32(std)).astype(np.float32)
+    a = rng.standard_normal(shape, dtype=np.float32)
+    a *= np.float32(std)
+    return a
 
 
 class ZipfSampler:
@@ -167,7 +171,7 @@ class SAProblem:
 
 def _weights(rng, k: int, d: int, p_scale: float = 1.0):
     std = 1.0 / math.sqrt(d)           # variance 1/d
-    P = gauss(rng, (k, d), std) * np.float32(p_scale)
+    P = gauss(rng, (k, d), std * p_scale)
     W_Q = gauss(rng, (d, d), std)
     W_K = gauss(rng, (d, d), std)
     W_V = gauss(rng, (d, d), std)
@@ -233,7 +237,8 @@ SA_WORKLOADS = {
 }
 
 
-def sa_workload(cfg: int, vocab: int = 1_000_000, users: Optional[int] = None) -> SAProblem:
+def sa_workload(cfg: int, vocab: int = 1_000_000, users: Optional[int] = None,
+                with_tables: bool = False):
     """SA inputs for workload ``cfg`` (1, 2, 3 or 5).
 
     ``users`` truncates the batch to its first users (same random stream for
@@ -261,7 +266,10 @@ def sa_workload(cfg: int, vocab: int = 1_000_000, users: Optional[int] = None) -
         rows = gauss(rng, (n, d), 1.0 / math.sqrt(d)) if kind == "gauss" else tables.events(rng, n)
         X[offsets[u]:offsets[u + 1]] = _pack(dtype, rows)
     dS = gauss(rng, (len(lengths), k, d), 1.0) if cfg == 5 else None
-    return SAProblem(SA_WORKLOADS[cfg], dtype, offsets, X, P, W_Q, W_K, W_V, 1e-6, dS)
+    prob = SAProblem(SA_WORKLOADS[cfg], dtype, offsets, X, P, W_Q, W_K, W_V, 1e-6, dS)
+    if with_tables:
+        return prob, tables, rng
+    return prob
 
 
 # --------------------------------------------------------------------------
@@ -361,3 +369,40 @@ def stca_workload(vocab: int = 1_000_000, users: int = 16, cands: int = 512) -> 
     512 candidates per user, 2 layers x 4 heads x d_h 32, bf16."""
     return make_stca_problem(users, [cands] * users, [L_RECENT] * users, 1024, 128, 4, 32, 2,
                              "bf16", 1004, vocab=vocab, name=STCA_WORKLOAD_4)
+
+
+@dataclasses.dataclass
+class TrainStep:
+    """The end-to-end step: SA forward and backward over the batch, then STCA on
+    the sketches and on each user's last L_r events against its candidates,
+    then the linear fusion."""
+    sa: SAProblem
+    cand_offsets: np.ndarray     # int64 [B+1]
+    q: np.ndarray                # bf16 bits [C_total, d] candidate targets
+    recent_begin: np.ndarray     # int64 [B] rows of sa.X
+    recent_end: np.ndarray
+    heads: int
+    d_h: int
+    layers_r: list
+    layers_u: list
+    W_F: np.ndarray
+    b_F: np.ndarray
+
+
+TRAIN_STEP_WORKLOAD = ("train step bf16 B=64 n~lognormal(mean 85K) d=128 k=1024: sa_fwd+sa_bwd, "
+                       "then STCA (2 layers x 4 heads x d_h 32) on sketches and 10K suffixes, "
+                       "256 candidates/user, fuse")
+
+
+def train_step_workload(vocab: int = 1_000_000, users: Optional[int] = None,
+                        cands: int = 256) -> TrainStep:
+    sa, tables, rng = sa_workload(5, vocab=vocab, users=users, with_tables=True)
+    D, heads, d_h = sa.d, 4, 32
+    layers_r = stca_layers(rng, 2, D, heads, d_h)
+    layers_u = stca_layers(rng, 2, D, heads, d_h)
+    W_F = gauss(rng, (2 * D, D), 1.0 / math.sqrt(2 * D))
+    b_F = np.zeros(D, np.float32)
+    cand_off = np.arange(sa.B + 1, dtype=np.int64) * cands
+    q = bf16_bits(tables.targets(rng, int(cand_off[-1])))
+    rb, re = suffix_ranges(sa.offsets)
+    return TrainStep(sa, cand_off, q, rb, re, heads, d_h, layers_r, layers_u, W_F, b_F)

@@ -1,0 +1,286 @@
+"""Python binding of libsketchattn.so (include/sketch_attn.h).
+
+Argument marshalling only: PyTorch supplies device memory and the current
+stream; every step of SA and STCA runs in the library's CUDA kernels.  There
+is no CPU fallback: if the library is missing or a call fails, an exception
+is raised.
+
+Entry points keep the C names: ``sa_forward``, ``sa_backward``,
+``stca_forward``, ``stca_fuse`` (plus the workspace queries).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libsketchattn.so")
+
+SA_F32, SA_BF16 = 0, 1
+_STATUS = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_ERR_CUDA",
+           4: "SA_ERR_TIMEOUT", 5: "SA_ERR_WORKSPACE"}
+
+# Symbols include/sketch_attn.h declares.
+EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_workspace",
+           "sa_forward", "sa_backward_workspace", "sa_backward", "stca_forward_workspace",
+           "stca_forward", "stca_fuse", "sa_launch_count", "sa_profile", "sa_profile_read")
+
+
+class SAError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class StcaLayerC(ctypes.Structure):
+    _fields_ = [("W_Q", ctypes.c_void_p), ("W_K", ctypes.c_void_p),
+                ("W_V", ctypes.c_void_p), ("W_O", ctypes.c_void_p)]
+
+
+_lib = None
+
+_vp, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+def load(path: Optional[str] = None):
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m sketch_attention_b200.build`")
+    lib = ctypes.CDLL(path)
+    lib.sa_version.restype = _i
+    lib.sa_last_error.restype = ctypes.c_char_p
+    lib.sa_poll_device_status.restype = _i
+    lib.sa_poll_device_status.argtypes = [_vp]
+    lib.sa_forward_workspace.restype = _sz
+    lib.sa_forward_workspace.argtypes = [_i, _i64, _i, _i, _i]
+    lib.sa_forward.restype = _i
+    lib.sa_forward.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
+                               _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.sa_backward_workspace.restype = _sz
+    lib.sa_backward_workspace.argtypes = [_i, _i64, _i, _i, _i]
+    lib.sa_backward.restype = _i
+    lib.sa_backward.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
+                                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.stca_forward_workspace.restype = _sz
+    lib.stca_forward_workspace.argtypes = [_i, _i64, _i, _i, _i, _i]
+    lib.stca_forward.restype = _i
+    lib.stca_forward.argtypes = [_vp, _i, _vp, _vp, _i, _vp, _i64, _vp, _vp, _vp, _vp,
+                                 _i, _i, _i, _i, ctypes.POINTER(StcaLayerC), _vp, _vp, _sz, _vp]
+    lib.stca_fuse.restype = _i
+    lib.stca_fuse.argtypes = [_vp, _vp, _vp, _vp, _i64, _i, _vp, _vp]
+    lib.sa_launch_count.restype = ctypes.c_longlong
+    lib.sa_profile.restype = _i
+    lib.sa_profile.argtypes = [_i]
+    lib.sa_profile_read.restype = _i
+    lib.sa_profile_read.argtypes = [_i, ctypes.c_char_p, _i, ctypes.POINTER(ctypes.c_double),
+                                    ctypes.POINTER(ctypes.c_longlong)]
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise SAError(fn, status, load().sa_last_error().decode())
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SA_F32
+    if t.dtype == torch.bfloat16:
+        return SA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _host_i64(a) -> np.ndarray:
+    if isinstance(a, torch.Tensor):
+        a = a.cpu().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+
+
+def _hp(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dev_i64(host: np.ndarray, device, given: Optional[torch.Tensor]) -> torch.Tensor:
+    if given is not None:
+        return given
+    return torch.from_numpy(host).to(device, non_blocking=False)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+# --------------------------------------------------------------------------
+def sa_forward_workspace(B: int, n_total: int, k: int, d: int, dtype: int) -> int:
+    return int(load().sa_forward_workspace(B, n_total, k, d, dtype))
+
+
+def sa_forward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
+               offsets_dev: Optional[torch.Tensor] = None, want_H: bool = False,
+               want_bf16: bool = False, out: Optional[dict] = None,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Sketches of a ragged batch.  Returns {"S", "mass"[, "H"][, "S_bf16"]}."""
+    lib = load()
+    _need_cuda(X, P, W_Q, W_K, W_V)
+    off = _host_i64(offsets)
+    B = len(off) - 1
+    k, d = P.shape
+    dev = X.device
+    dt = _dtype_code(X)
+    o = dict(out or {})
+    S = o.get("S") if o.get("S") is not None else torch.empty(B, k, d, device=dev)
+    mass = o.get("mass") if o.get("mass") is not None else torch.empty(B, k, device=dev)
+    H = o.get("H") if o.get("H") is not None else (torch.empty(B, k, d, device=dev) if want_H else None)
+    Sb = o.get("S_bf16") if o.get("S_bf16") is not None else (
+        torch.empty(B, k, d, device=dev, dtype=torch.bfloat16) if want_bf16 else None)
+    ws_bytes = lib.sa_forward_workspace(B, int(off[-1]), k, d, dt)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    offd = _dev_i64(off, dev, offsets_dev)
+    st = lib.sa_forward(_p(X), dt, _hp(off), _p(offd), B, k, d, _p(P), _p(W_Q), _p(W_K), _p(W_V),
+                        float(eps), _p(S), _p(mass), _p(H), _p(Sb), _p(workspace),
+                        workspace.numel(), _stream(stream))
+    _check("sa_forward", st)
+    res = {"S": S, "mass": mass}
+    if H is not None:
+        res["H"] = H
+    if Sb is not None:
+        res["S_bf16"] = Sb
+    return res
+
+
+def sa_backward_workspace(B: int, n_total: int, k: int, d: int, dtype: int) -> int:
+    return int(load().sa_backward_workspace(B, n_total, k, d, dtype))
+
+
+def sa_backward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float, H, mass, dS,
+                dmass=None, *, offsets_dev: Optional[torch.Tensor] = None,
+                out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
+                stream=None) -> dict:
+    """Gradients {"dX", "dP", "dW_Q", "dW_K", "dW_V"} of <dS, S> + <dmass, mass>."""
+    lib = load()
+    _need_cuda(X, P, W_Q, W_K, W_V, H, mass, dS, dmass)
+    off = _host_i64(offsets)
+    B = len(off) - 1
+    k, d = P.shape
+    dev = X.device
+    dt = _dtype_code(X)
+    o = dict(out or {})
+    dX = o.get("dX") if o.get("dX") is not None else torch.empty_like(X)
+    dP = o.get("dP") if o.get("dP") is not None else torch.empty(k, d, device=dev)
+    dWQ = o.get("dW_Q") if o.get("dW_Q") is not None else torch.empty(d, d, device=dev)
+    dWK = o.get("dW_K") if o.get("dW_K") is not None else torch.empty(d, d, device=dev)
+    dWV = o.get("dW_V") if o.get("dW_V") is not None else torch.empty(d, d, device=dev)
+    ws_bytes = lib.sa_backward_workspace(B, int(off[-1]), k, d, dt)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    offd = _dev_i64(off, dev, offsets_dev)
+    st = lib.sa_backward(_p(X), dt, _hp(off), _p(offd), B, k, d, _p(P), _p(W_Q), _p(W_K), _p(W_V),
+                         float(eps), _p(H), _p(mass), _p(dS), _p(dmass), _p(dX), _p(dP), _p(dWQ),
+                         _p(dWK), _p(dWV), _p(workspace), workspace.numel(), _stream(stream))
+    _check("sa_backward", st)
+    return {"dX": dX, "dP": dP, "dW_Q": dWQ, "dW_K": dWK, "dW_V": dWV}
+
+
+def stca_forward_workspace(B: int, C_total: int, D: int, heads: int, d_h: int, dtype: int) -> int:
+    return int(load().stca_forward_workspace(B, C_total, D, heads, d_h, dtype))
+
+
+def stca_forward(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin, kv_end,
+                 layers: Sequence[dict], heads: int, d_h: int, *,
+                 cand_offsets_dev=None, kv_begin_dev=None, kv_end_dev=None,
+                 out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """One STCA branch.  ``layers``: dicts with W_Q, W_K, W_V [heads, D, d_h] and
+    W_O [heads*d_h, D] or None (fp32 CUDA tensors).  Returns out [C_total, D] fp32."""
+    lib = load()
+    _need_cuda(q, kv)
+    dt = _dtype_code(q)
+    if kv.dtype != q.dtype:
+        raise TypeError("q and kv must have the same dtype")
+    cand = _host_i64(cand_offsets)
+    kb, ke = _host_i64(kv_begin), _host_i64(kv_end)
+    B = len(cand) - 1
+    D = q.shape[1]
+    dev = q.device
+    C = int(cand[-1])
+    res = out if out is not None else torch.empty(C, D, device=dev)
+    arr = (StcaLayerC * len(layers))()
+    for i, L in enumerate(layers):
+        _need_cuda(L["W_Q"], L["W_K"], L["W_V"], L.get("W_O"))
+        arr[i].W_Q = L["W_Q"].data_ptr()
+        arr[i].W_K = L["W_K"].data_ptr()
+        arr[i].W_V = L["W_V"].data_ptr()
+        arr[i].W_O = L["W_O"].data_ptr() if L.get("W_O") is not None else None
+    ws_bytes = lib.stca_forward_workspace(B, C, D, heads, d_h, dt)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    cd = _dev_i64(cand, dev, cand_offsets_dev)
+    kbd = _dev_i64(kb, dev, kv_begin_dev)
+    ked = _dev_i64(ke, dev, kv_end_dev)
+    st = lib.stca_forward(_p(q), dt, _hp(cand), _p(cd), B, _p(kv), kv.shape[0], _hp(kb), _hp(ke),
+                          _p(kbd), _p(ked), D, heads, d_h, len(layers), arr, _p(res),
+                          _p(workspace), workspace.numel(), _stream(stream))
+    _check("stca_forward", st)
+    return res
+
+
+def stca_fuse(z_r: torch.Tensor, z_u: torch.Tensor, W_F: torch.Tensor, b_F=None, *,
+              out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """[z_r ; z_u] W_F + b_F."""
+    lib = load()
+    _need_cuda(z_r, z_u, W_F, b_F)
+    C, D = z_r.shape
+    res = out if out is not None else torch.empty(C, D, device=z_r.device)
+    st = lib.stca_fuse(_p(z_r), _p(z_u), _p(W_F), _p(b_F), C, D, _p(res), _stream(stream))
+    _check("stca_fuse", st)
+    return res
+
+
+def poll_device_status(stream=None) -> None:
+    _check("sa_poll_device_status", load().sa_poll_device_status(_stream(stream)))
+
+
+# --------------------------------------------------------------------------
+# measurement support
+def launch_count() -> int:
+    """Kernels the library has launched in this process."""
+    return int(load().sa_launch_count())
+
+
+def profile(enable: bool) -> None:
+    """Start (clearing) or stop the library's per-kernel event timers."""
+    load().sa_profile(1 if enable else 0)
+
+
+def profile_read() -> dict:
+    """{kernel name: (total device ms, launches)} since profile(True)."""
+    lib = load()
+    out = {}
+    buf = ctypes.create_string_buffer(128)
+    ms, cnt = ctypes.c_double(), ctypes.c_longlong()
+    i = 0
+    while lib.sa_profile_read(i, buf, 128, ctypes.byref(ms), ctypes.byref(cnt)):
+        out[buf.value.decode()] = (ms.value, cnt.value)
+        i += 1
+    return out

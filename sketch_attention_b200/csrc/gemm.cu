@@ -1,0 +1,78 @@
+// Tiled SIMT fp32 GEMM: 64 x 64 output tile per CTA, 16-deep k slices staged
+// through shared memory, 4 x 4 outputs per thread.  Arbitrary sizes, strides,
+// transposes and batch; used only for the small projection GEMMs.
+#include "gemm.cuh"
+
+namespace sa {
+
+namespace {
+constexpr int TM = 64, TN = 64, TK = 16;
+
+__global__ void __launch_bounds__(256) gemm_kernel(Gemm g) {
+  __shared__ float As[TK][TM + 4];
+  __shared__ float Bs[TK][TN + 4];
+  const int b = blockIdx.z;
+  const float* A = g.A + (int64_t)b * g.sA;
+  const float* Bm = g.B + (int64_t)b * g.sB;
+  const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < g.K; k0 += TK) {
+    // 64 x 16 of A and 16 x 64 of B, 4 elements of each per thread.
+    for (int e = threadIdx.x; e < TM * TK; e += 256) {
+      int mm, kk;
+      if (g.transA) { mm = e % TM; kk = e / TM; } else { kk = e % TK; mm = e / TK; }
+      int m = m0 + mm, k = k0 + kk;
+      float v = 0.f;
+      if (m < g.M && k < g.K) v = g.transA ? A[(int64_t)k * g.lda + m] : A[(int64_t)m * g.lda + k];
+      As[kk][mm] = v;
+    }
+    for (int e = threadIdx.x; e < TN * TK; e += 256) {
+      int nn, kk;
+      if (g.transB) { kk = e % TK; nn = e / TK; } else { nn = e % TN; kk = e / TN; }
+      int n = n0 + nn, k = k0 + kk;
+      float v = 0.f;
+      if (n < g.N && k < g.K) v = g.transB ? Bm[(int64_t)n * g.ldb + k] : Bm[(int64_t)k * g.ldb + n];
+      Bs[kk][nn] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < TK; ++kk) {
+      float a[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bb[j] = Bs[kk][tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int m = m0 + ty + 16 * i;
+    if (m >= g.M) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int n = n0 + tx + 16 * j;
+      if (n >= g.N) continue;
+      float v = g.alpha * acc[i][j];
+      if (g.bias) v += g.bias[n];
+      if (g.Cin) v += g.Cin[(int64_t)b * g.sCin + (int64_t)m * g.ldcin + n];
+      if (g.C) g.C[(int64_t)b * g.sC + (int64_t)m * g.ldc + n] = v;
+      if (g.C16) g.C16[(int64_t)b * g.sC16 + (int64_t)m * g.ldc16 + n] = __float2bfloat16_rn(v);
+    }
+  }
+}
+}  // namespace
+
+sa_status gemm(const Gemm& g, cudaStream_t stream) {
+  if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return SA_OK;
+  dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, g.batch);
+  SA_TIMED("gemm_kernel", stream, (gemm_kernel<<<grid, 256, 0, stream>>>(g)));
+  return SA_OK;
+}
+
+}  // namespace sa

@@ -1,0 +1,25 @@
+// Small fp32 GEMM for the projections around the hot loops (prototype
+// folding, value projection, STCA head projections, weight gradients).
+// These are O(k d^2) or O(C D^2) per call, far below the token loops.
+#pragma once
+#include "common.cuh"
+
+namespace sa {
+
+struct Gemm {
+  // C[m, n] = alpha * sum_k A[m, k] B[k, n] (+ bias[n]) (+ Cin[m, n])
+  int M = 0, N = 0, K = 0;
+  const float* A = nullptr; int64_t lda = 0; bool transA = false;   // A[m*lda+k] or A[k*lda+m]
+  const float* B = nullptr; int64_t ldb = 0; bool transB = false;   // B[k*ldb+n] or B[n*ldb+k]
+  float* C = nullptr; int64_t ldc = 0;                               // fp32 out (may be NULL)
+  __nv_bfloat16* C16 = nullptr; int64_t ldc16 = 0;                   // optional bf16 copy
+  const float* Cin = nullptr; int64_t ldcin = 0;                     // optional addend
+  const float* bias = nullptr;                                        // optional [N]
+  float alpha = 1.f;
+  int batch = 1;
+  int64_t sA = 0, sB = 0, sC = 0, sC16 = 0, sCin = 0;                // batch strides
+};
+
+sa_status gemm(const Gemm& g, cudaStream_t stream);
+
+}  // namespace sa

@@ -1,0 +1,70 @@
+// Internal interfaces between the C-ABI layer (api.cu) and the SA kernels.
+#pragma once
+#include "common.cuh"
+#include "gemm.cuh"
+
+namespace sa {
+
+struct SaFwdArgs {
+  const void* X; sa_dtype x_dtype;
+  const int64_t* off_dev; int B; int64_t n_total;
+  int k, d;
+  const float *P, *W_Q, *W_K, *W_V;
+  float eps;
+  float* S; float* mass; float* H; void* S_bf16;
+};
+
+// Workspace views of sa_forward.
+struct SaFwdWork {
+  Chunking ch;
+  float* T;             // [d, d]   W_Q W_K^T
+  float* Pf;            // [k, d]   folded prototypes, log2 units, fp32
+  __nv_bfloat16* Pb;    // [k, d]   same, bf16 (tensor-core operand)
+  float* lse;           // [n_total] per-token log2-sum-exp (CUDA-core path)
+  float* Muser;         // [B, k]   mass of users that lie in one chunk
+  float* slotH;         // [G, 2, k, d]
+  float* slotM;         // [G, 2, k]
+  float* Hhat;          // [B, k, d] H/(m+eps)
+};
+
+struct SaBwdArgs {
+  const void* X; sa_dtype x_dtype;
+  const int64_t* off_dev; int B; int64_t n_total;
+  int k, d;
+  const float *P, *W_Q, *W_K, *W_V;
+  float eps;
+  const float *H, *mass, *dS, *dmass;
+  void* dX; float *dP, *dW_Q, *dW_K, *dW_V;
+};
+
+struct SaBwdWork {
+  Chunking ch;          // chunks of the per-token kernel
+  Chunking chE;         // chunks of the E = dZ X accumulation
+  float* T;             // [d, d]
+  float* Pf;            // [k, d]
+  __nv_bfloat16* Pb;    // [k, d]
+  float* lse;           // [n_total]
+  float* cbuf;          // [n_total]  c_t
+  float* dHh;           // [B, k, d]  dS W_V^T
+  float* Hhat;          // [B, k, d]
+  float* dH;            // [B, k, d]
+  float* dm;            // [B, k]
+  float* Epart;         // [chE.G, k, d]
+  float* E;             // [k, d]
+  float* dQ;            // [k, d]
+  float* Q;             // [k, d]
+};
+
+sa_status sa_fold(int k, int d, const float* P, const float* W_Q, const float* W_K, float* T,
+                  float* Pf, __nv_bfloat16* Pb, cudaStream_t st);
+sa_status sa_simt_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
+sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
+sa_status sa_simt_backward(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st);
+sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st);
+
+// Tensor-core forward (sa_tc.cu).
+bool sa_tc_supported(sa_dtype x_dtype, int k, int d);
+int sa_tc_num_chunks(int k);       // number of clusters the persistent launch uses
+sa_status sa_tc_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
+
+}  // namespace sa

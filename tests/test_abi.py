@@ -1,0 +1,93 @@
+"""The C-ABI library: it loads, exports every entry point the header declares,
+answers workspace queries and rejects bad arguments with status codes before
+touching the GPU (no compute calls here: these run without a GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import sketch_attention_b200 as sab
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if not fn.endswith(".h"):
+            continue
+        text = open(os.path.join(inc, fn)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M):
+            name = m.group(1)
+            if name not in ("defined",):
+                names.add(name)
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sketch_attention_b200 import build
+    build.build()
+    return sab.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert {"sa_forward", "sa_backward", "stca_forward", "stca_fuse"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), f"library does not export {name}"
+    assert set(sab.EXPORTS) == declared
+
+
+def test_version_and_workspace_queries(lib):
+    assert lib.sa_version() >= 100
+    w = sab.sa_forward_workspace(4, 10_000, 1024, 128, sab.SA_BF16)
+    assert w >= 4 * 1024 * 128 * 4          # at least the H/(m+eps) scratch
+    assert sab.sa_forward_workspace(0, 10, 4, 64, sab.SA_F32) == 0
+    assert sab.sa_backward_workspace(2, 300, 64, 64, sab.SA_F32) > 300 * 4
+    assert sab.stca_forward_workspace(2, 10, 128, 4, 32, sab.SA_BF16) > 0
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def _fwd(lib, offsets, k=64, d=64, x=0x1000, ws_bytes=1 << 40, eps=1e-6):
+    off = np.asarray(offsets, np.int64)
+    B = len(off) - 1
+    p = _fake(0x2000)
+    return lib.sa_forward(_fake(x), sab.SA_F32, off.ctypes.data_as(ctypes.c_void_p), p, B, k, d,
+                          p, p, p, p, eps, p, p, None, None, _fake(0x100000), ws_bytes, None)
+
+
+def test_rejects_bad_arguments_without_touching_the_gpu(lib):
+    assert _fwd(lib, [0, 5, 3]) == 1                   # offsets not monotone
+    assert _fwd(lib, [1, 5]) == 1                      # offsets[0] != 0
+    assert _fwd(lib, [0, 5], k=0) == 2                 # k out of range
+    assert _fwd(lib, [0, 5], k=5000) == 2
+    assert _fwd(lib, [0, 5], d=96) == 2                # d unsupported
+    assert _fwd(lib, [0, 5], x=0x1004) == 1            # misaligned X
+    assert _fwd(lib, [0, 5], x=0) == 1                 # NULL X with rows
+    assert _fwd(lib, [0, 5], ws_bytes=16) == 5         # workspace too small
+    assert _fwd(lib, [0, 5], eps=-1.0) == 1
+    assert "workspace" in lib.sa_last_error().decode() or "eps" in lib.sa_last_error().decode()
+
+
+def test_stca_rejects_bad_ranges(lib):
+    cand = np.array([0, 2], np.int64)
+    kb, ke = np.array([5], np.int64), np.array([3], np.int64)
+    p = _fake(0x2000)
+    lay = (sab.StcaLayerC * 1)()
+    lay[0].W_Q = lay[0].W_K = lay[0].W_V = 0x3000
+    st = lib.stca_forward(p, sab.SA_BF16, cand.ctypes.data_as(ctypes.c_void_p), p, 1, p, 10,
+                          kb.ctypes.data_as(ctypes.c_void_p), ke.ctypes.data_as(ctypes.c_void_p),
+                          p, p, 128, 4, 32, 1, lay, p, p, 1 << 40, None)
+    assert st == 1 and "range" in lib.sa_last_error().decode()
+    st = lib.stca_forward(p, sab.SA_BF16, cand.ctypes.data_as(ctypes.c_void_p), p, 1, p, 10,
+                          kb.ctypes.data_as(ctypes.c_void_p), ke.ctypes.data_as(ctypes.c_void_p),
+                          p, p, 96, 4, 32, 1, lay, p, p, 1 << 40, None)
+    assert st == 2
