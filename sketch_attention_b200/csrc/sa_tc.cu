@@ -1,10 +1,458 @@
-// Tensor-core SA forward (tcgen05 / TMEM / TMA).  Not enabled yet.
+// Tensor-core Sketch Attention forward for sm_100a (SequenceO1 Sec. 3.1,
+// eqs. (6)-(9); the fused streaming operator of Sec. 4.4, re-designed for
+// tcgen05, TMEM and TMA).
+//
+// Work split.  The token stream is cut into G chunks, one per cluster of
+// C = k/128 CTAs.  CTA r of a cluster owns prototypes [128 r, 128 r + 128):
+// its slice of P' (bf16, SMEM-resident) and its accumulator
+// H_slice = [A_slice X | A_slice 1] (128 x 144 fp32 in TMEM; the last 16
+// columns hold the mass).  Every CTA of the cluster streams the same 128-token
+// tiles of X through SMEM with TMA (no multicast: each CTA issues its own
+// loads, the copies after the first come from L2).
+//
+// Per tile (t = 128 tokens of one user):
+//   MMA1   Z^T[t, j] = X_t . P'_j              (M=128 tokens, N=128 prototypes, K=d)
+//   softmax over all k prototypes of each token: each CTA reduces its 128
+//          logits in registers (one TMEM lane = one token = one thread) to a
+//          log2-sum-exp, sends it to every CTA of the cluster (DSMEM bulk
+//          copies), and rescales its exponentials by 2^{m - lse_total}
+//   MMA2   H_slice[j, :] += sum_t p[t, j] [x_t | 1]   (M=128 prototypes, N=144, K=128 tokens)
+// so the k x n assignment matrix never leaves the SM.
+//
+// Warp roles (12 warps): 0 TMA, 1 MMA issue + TMEM owner, 2-3 idle,
+// 4-7 softmax of even tiles (and the H drain at the end of a piece),
+// 8-11 softmax of odd tiles.
+#include <algorithm>
+#include <mutex>
+
 #include "sa_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace sa {
-bool sa_tc_supported(sa_dtype, int, int) { return false; }
-int sa_tc_num_chunks(int) { return 1; }
-sa_status sa_tc_forward(const SaFwdArgs&, const SaFwdWork&, cudaStream_t) {
-  return fail(SA_ERR_UNSUPPORTED, "tensor-core SA forward not built");
+
+namespace {
+using namespace tc;
+
+constexpr int TILE = 128;            // tokens per tile = prototypes per CTA
+constexpr int DD = 128;              // d
+constexpr int NS = 3;                // X pipeline stages
+constexpr int MAXC = 8;              // cluster size limit (k <= 1024)
+constexpr int N2 = DD + 16;          // MMA2 N: d columns + 16 mass columns
+constexpr int THREADS = 384;
+
+// shared-memory layout (offsets from a 1024-aligned base)
+constexpr uint32_t X_BOX = TILE * 32;                  // one [128 x 16] bf16 SW32 box = 4 KB
+constexpr uint32_t X_STAGE = 9 * X_BOX;                // 8 boxes of X + 1 box of ones = 36 KB
+constexpr uint32_t OFF_PQ = 0;                         // P' slice: 2 x [128 x 64] SW128 = 32 KB
+constexpr uint32_t OFF_X = 32768;
+constexpr uint32_t OFF_P = OFF_X + NS * X_STAGE;       // 2 x 32 KB probability tiles
+constexpr uint32_t OFF_XCHG = OFF_P + 2 * 32768;       // [4 slots][MAXC][128] fp32
+constexpr uint32_t OFF_STAGE = OFF_XCHG + 4 * MAXC * TILE * 4;  // [2 wg][2][128] fp32
+constexpr uint32_t OFF_BAR = OFF_STAGE + 2 * 2 * TILE * 4;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
+
+// TMEM columns
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_H = 256, TM_COLS = 512;
+
+struct Bars {
+  uint64_t x_full[NS], x_empty[NS];
+  uint64_t s_full[2], p_full[2], p_empty[2];
+  uint64_t h_full, h_empty, pq_full, mma_done;
+  uint64_t xchg[4];
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+struct Params {
+  const int64_t* off;
+  int B;
+  Chunking ch;
+  int k;
+  float* Huser;
+  float* Muser;
+  float* slotH;
+  float* slotM;
+  int* err;
+};
+
+// Iterates the tiles of chunk g: calls f(tile_index, user, tile_begin,
+// piece_begin, piece_end, first_tile_of_piece, last_tile_of_piece) in order;
+// stops early if f returns false.
+template <class F>
+__device__ __forceinline__ void for_each_tile(const Params& p, int g, F&& f) {
+  const int64_t cb = (int64_t)g * p.ch.T, ce = min(cb + p.ch.T, p.ch.n_total);
+  int t = 0;
+  for (int u = user_of_token(p.off, p.B, cb); u < p.B && p.off[u] < ce; ++u) {
+    const int64_t pb = max(p.off[u], cb), pe = min(p.off[u + 1], ce);
+    for (int64_t tb = pb; tb < pe; tb += TILE, ++t)
+      if (!f(t, u, tb, pb, pe, tb == pb, tb + TILE >= pe)) return;
+  }
 }
+
+__global__ void __launch_bounds__(THREADS, 1)
+    sa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                     const __grid_constant__ CUtensorMap tmP, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Bars* bars = (Bars*)(smem + OFF_BAR);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank(), C = cluster_size();
+  const int g = (int)cluster_id_x();
+  const bool chunk_ok = g < p.ch.G;
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->p_full[b], 128);
+      mbar_init(&bars->p_empty[b], 1);
+    }
+    mbar_init(&bars->h_full, 1);
+    mbar_init(&bars->h_empty, 128);
+    mbar_init(&bars->pq_full, 1);
+    mbar_init(&bars->mma_done, 1);
+    for (int s = 0; s < 4; ++s) mbar_init(&bars->xchg[s], 1);
+    bars->abort = 0;
+    fence_mbar_init();
+    // arm the exchange slots for their first use (tiles 0..3)
+    for (int s = 0; s < 4; ++s) mbar_arrive_expect_tx(&bars->xchg[s], C * TILE * 4);
+  }
+  // constant ones block of every stage (MMA2 columns d..d+15 -> prototype mass)
+  for (int i = threadIdx.x; i < NS * (int)X_BOX / 4; i += THREADS) {
+    const int s = i / (X_BOX / 4), w = i % (X_BOX / 4);
+    ((uint32_t*)(smem + OFF_X + s * X_STAGE + 8 * X_BOX))[w] = 0x3F803F80u;   // bf16 1.0 pairs
+  }
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync();          // peers' barriers are initialised before any exchange
+  const uint32_t tmem = bars->tmem_base;
+
+  if (chunk_ok) {
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      prefetch_tensormap(&tmX);
+      prefetch_tensormap(&tmP);
+      mbar_arrive_expect_tx(&bars->pq_full, 2 * 16384);
+      tma_load_2d(smem + OFF_PQ, &tmP, &bars->pq_full, 0, (int)(rank * TILE));
+      tma_load_2d(smem + OFF_PQ + 16384, &tmP, &bars->pq_full, 64, (int)(rank * TILE));
+      int issued = 0;
+      for_each_tile(p, g, [&](int t, int, int64_t tb, int64_t, int64_t, bool, bool) {
+        const int s = t % NS;
+        if (t >= NS && !mbar_wait(&bars->x_empty[s], ((t / NS) - 1) & 1, abort, p.err)) return false;
+        mbar_arrive_expect_tx(&bars->x_full[s], 8 * X_BOX);
+        uint8_t* dst = smem + OFF_X + s * X_STAGE;
+        for (int b = 0; b < 8; ++b) tma_load_2d(dst + b * X_BOX, &tmX, &bars->x_full[s], 16 * b, (int)tb);
+        issued = t + 1;
+        return true;
+      });
+      if (*abort) {
+        // let the loads still in flight land before the CTA can exit
+        mbar_wait_bounded(&bars->pq_full, 0);
+        for (int t = std::max(0, issued - NS); t < issued; ++t)
+          mbar_wait_bounded(&bars->x_full[t % NS], (t / NS) & 1);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint32_t id1 = idesc_bf16(128, 128, false, false);
+      const uint32_t id2 = idesc_bf16(128, N2, true, true);
+      const uint32_t pq = smem_u32(smem + OFF_PQ);
+      bool ok = mbar_wait(&bars->pq_full, 0, abort, p.err);
+      int piece = -1;
+      int prev_t = -1;
+      bool prev_first = false, prev_last = false;
+      auto mma2 = [&](int t, bool first, bool last) -> bool {
+        const int b = t & 1, s = t % NS;
+        if (first && piece > 0 && !mbar_wait(&bars->h_empty, (piece - 1) & 1, abort, p.err)) return false;
+        if (!mbar_wait(&bars->p_full[b], (t >> 1) & 1, abort, p.err)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(smem + OFF_P + b * 32768);
+        const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t da = smem_desc(pa + ks * 2048, 16384, 1024, SWZ_128B);
+          const uint64_t db = smem_desc(xa + ks * 512, X_BOX, 256, SWZ_32B);
+          mma_ss(tmem + TM_H, da, db, id2, (first && ks == 0) ? 0u : 1u);
+        }
+        mma_commit(&bars->p_empty[b]);
+        mma_commit(&bars->x_empty[s]);
+        if (last) mma_commit(&bars->h_full);
+        return true;
+      };
+      if (ok) {
+        for_each_tile(p, g, [&](int t, int, int64_t, int64_t, int64_t, bool first, bool last) {
+          const int s = t % NS, b = t & 1;
+          if (!mbar_wait(&bars->x_full[s], (t / NS) & 1, abort, p.err)) return false;
+          tc_fence_after();
+          const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t da = smem_desc(xa + ks * X_BOX, 16, 256, SWZ_32B);
+            const uint64_t db = smem_desc(pq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B);
+            mma_ss(tmem + (b ? TM_S1 : TM_S0), da, db, id1, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->s_full[b]);
+          if (prev_t >= 0) {
+            if (prev_first) ++piece;
+            if (!mma2(prev_t, prev_first, prev_last)) return false;
+          }
+          prev_t = t; prev_first = first; prev_last = last;
+          return true;
+        });
+        if (prev_t >= 0 && !*abort) {
+          if (prev_first) ++piece;
+          mma2(prev_t, prev_first, prev_last);
+        }
+      }
+      // every MMA this thread issued has completed before TMEM is released
+      mma_commit(&bars->mma_done);
+      mbar_wait_bounded(&bars->mma_done, 0);
+    } else if (warp >= 4) {
+      // ------------------------------------------------------------ softmax groups
+      const int wg = (warp - 4) / 4;            // 0: even tiles, 1: odd tiles
+      const int q = warp % 4;                   // TMEM lane quarter
+      const int row = q * 32 + lane;            // token within the tile / prototype lane
+      const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+      float* stage = (float*)(smem + OFF_STAGE) + wg * 2 * TILE;
+      const float* xchg = (const float*)(smem + OFF_XCHG);
+      int piece = -1;
+      for_each_tile(p, g, [&](int t, int u, int64_t tb, int64_t pb, int64_t pe, bool first, bool last) {
+        if (first) ++piece;
+        if ((t & 1) == wg) {
+          const int b = t & 1;
+          const bool valid = tb + row < pe;
+          // logits of this token over the CTA's 128 prototypes (base-2 units)
+          if (!mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort, p.err)) return false;
+          tc_fence_after();
+          // Two halves of 64 columns; each half is exponentiated against the
+          // running maximum at that point (mh[h]) and kept as bf16 pairs.
+          uint32_t ep[64];
+          float mh[2];
+          float m = -__builtin_huge_valf(), s = 0.f;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float z[64];
+            tmem_ld32(tmem + lane_addr + (b ? TM_S1 : TM_S0) + 64 * h, z);
+            tmem_ld32(tmem + lane_addr + (b ? TM_S1 : TM_S0) + 64 * h + 32, z + 32);
+            tmem_wait_ld();
+            float cm = z[0];
+#pragma unroll
+            for (int j = 1; j < 64; ++j) cm = fmaxf(cm, z[j]);
+            const float mn = fmaxf(m, cm);
+            s *= ex2(m - mn);
+            m = mn;
+            mh[h] = mn;
+#pragma unroll
+            for (int j = 0; j < 64; j += 2) {
+              const float e0 = ex2(z[j] - mn), e1 = ex2(z[j + 1] - mn);
+              s += e0 + e1;
+              ep[32 * h + j / 2] = pack_bf16x2(e0, e1);
+            }
+          }
+          const float l = valid ? m + lg2(s) : -__builtin_huge_valf();
+          // send this CTA's log2-sum-exp of every token to every CTA of the cluster
+          float* st = stage + ((t >> 1) & 1) * TILE;
+          st[row] = l;
+          fence_proxy_async_smem();
+          named_bar_sync(1 + wg, 128);
+          const int slot = t & 3;
+          if (row == 0) {
+            const uint32_t src = smem_u32(st);
+            const uint32_t dst = smem_u32(smem + OFF_XCHG + (slot * MAXC + rank) * TILE * 4);
+            const uint32_t bar = smem_u32(&bars->xchg[slot]);
+            for (uint32_t c = 0; c < C; ++c)
+              bulk_copy_to_peer(map_to_rank(dst, c), src, TILE * 4, map_to_rank(bar, c));
+          }
+          if (!mbar_wait(&bars->xchg[slot], (t >> 2) & 1, abort, p.err)) return false;
+          uint32_t rr[2] = {0u, 0u};
+          if (valid) {
+            float L = -__builtin_huge_valf();
+            for (uint32_t c = 0; c < C; ++c) L = fmaxf(L, xchg[(slot * MAXC + c) * TILE + row]);
+            float z = 0.f;
+            for (uint32_t c = 0; c < C; ++c) z += ex2(xchg[(slot * MAXC + c) * TILE + row] - L);
+            const float lt = L + lg2(z);
+            const float r0 = ex2(mh[0] - lt), r1 = ex2(mh[1] - lt);
+            rr[0] = pack_bf16x2(r0, r0);
+            rr[1] = pack_bf16x2(r1, r1);
+          }
+          named_bar_sync(1 + wg, 128);      // every thread has read the slot
+          if (row == 0) mbar_arrive_expect_tx(&bars->xchg[slot], C * TILE * 4);   // re-arm for t+4
+          // probabilities p[t, j] = e_j r as bf16 into the MN-major SW128 A tile of MMA2
+          if (t >= 2 && !mbar_wait(&bars->p_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return false;
+          const uint32_t pa = smem_u32(smem + OFF_P + b * 32768) + row * 128;
+#pragma unroll
+          for (int blk = 0; blk < 2; ++blk) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int q4 = blk * 32 + c * 4;        // index of the first bf16 pair
+              st_shared_v4(pa + blk * 16384 + ((c ^ (row & 7)) << 4),
+                           mul_bf16x2(ep[q4], rr[blk]), mul_bf16x2(ep[q4 + 1], rr[blk]),
+                           mul_bf16x2(ep[q4 + 2], rr[blk]), mul_bf16x2(ep[q4 + 3], rr[blk]));
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(&bars->p_full[b]);
+        }
+        if (last && wg == 0) {
+          // ------------------------------------------------------ drain H of the piece
+          if (!mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return false;
+          tc_fence_after();
+          const int64_t ub = p.off[u], ue = p.off[u + 1];
+          const int64_t cb = (int64_t)g * p.ch.T, ce = min(cb + p.ch.T, p.ch.n_total);
+          const int dest = piece_dest(ub, ue, cb, ce);
+          const int j = (int)rank * TILE + row;
+          float* Hrow;
+          float* mrow;
+          if (dest == DEST_USER) {
+            Hrow = p.Huser + ((int64_t)u * p.k + j) * DD;
+            mrow = p.Muser + (int64_t)u * p.k + j;
+          } else {
+            Hrow = p.slotH + (((int64_t)g * 2 + dest) * p.k + j) * DD;
+            mrow = p.slotM + ((int64_t)g * 2 + dest) * p.k + j;
+          }
+          float hv[32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            tmem_ld32(tmem + lane_addr + TM_H + 32 * c, hv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              *(float4*)(Hrow + 32 * c + i) = make_float4(hv[i], hv[i + 1], hv[i + 2], hv[i + 3]);
+          }
+          const float mass = tmem_ld1(tmem + lane_addr + TM_H + DD);
+          tmem_wait_ld();
+          *mrow = mass;
+          tc_fence_before();
+          mbar_arrive(&bars->h_empty);
+        }
+        return true;
+      });
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+  cluster_sync();          // no peer copies may target this CTA after it exits
+}
+
+struct Cached {
+  bool init = false;
+  int clusters[MAXC + 1] = {};
+};
+std::mutex g_mu;
+Cached g_cache[64];
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeFn)p;
+  });
+  return fn;
+}
+
+sa_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                   uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return SA_OK;
+}
+
+int clusters_for(int C) {
+  const DeviceInfo& di = device_info();
+  std::lock_guard<std::mutex> lock(g_mu);
+  Cached& c = g_cache[di.device & 63];
+  if (!c.init) {
+    cudaFuncSetAttribute(sa_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaFuncSetAttribute(sa_fwd_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    for (int cs = 1; cs <= MAXC; ++cs) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = cs;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(cs * (di.sm_count / cs), 1, 1);
+      cfg.blockDim = dim3(THREADS, 1, 1);
+      cfg.dynamicSmemBytes = SMEM_BYTES;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, sa_fwd_tc_kernel, &cfg) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        n = std::max(1, di.sm_count / cs);
+      }
+      c.clusters[cs] = n;
+    }
+    c.init = true;
+  }
+  return c.clusters[C];
+}
+}  // namespace
+
+bool sa_tc_supported(sa_dtype x_dtype, int k, int d) {
+  return x_dtype == SA_BF16 && d == DD && k % TILE == 0 && k / TILE >= 1 && k / TILE <= MAXC;
+}
+
+int sa_tc_num_chunks(int k) { return clusters_for(k / TILE); }
+
+sa_status sa_tc_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st) {
+  const int C = a.k / TILE;
+  if (a.n_total >= (1LL << 31)) return fail(SA_ERR_UNSUPPORTED, "n_total must be < 2^31");
+  CUtensorMap tmX, tmP;
+  sa_status s = make_map(&tmX, a.X, DD, (uint64_t)a.n_total, 16, TILE, CU_TENSOR_MAP_SWIZZLE_32B);
+  if (s != SA_OK) return s;
+  s = make_map(&tmP, w.Pb, DD, (uint64_t)a.k, 64, TILE, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != SA_OK) return s;
+  Params p{a.off_dev, a.B, w.ch, a.k, a.S, w.Muser, w.slotH, w.slotM, device_status_word()};
+  clusters_for(C);   // sets the kernel attributes once per device
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = C;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(C * w.ch.G, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaSuccess;
+  SA_TIMED("sa_fwd_tc_kernel", st, (le = cudaLaunchKernelEx(&cfg, sa_fwd_tc_kernel, tmX, tmP, p)));
+  if (le != cudaSuccess) return cuda_fail(le, "sa_fwd_tc_kernel launch");
+  return SA_OK;
+}
+
 }  // namespace sa

@@ -1,9 +1,309 @@
-// Tensor-core STCA attention (tcgen05 / TMEM / TMA).  Not enabled yet.
+// Tensor-core STCA attention for sm_100a (SequenceO1 Sec. 2.3 eq. (4) in the
+// single-query reordering of Sec. 5.1 eq. (24)).
+//
+// One CTA per tile of 128 query rows of one user; a row is a (candidate,
+// head) pair whose query vector u_h = (q W_Q^h) W_K^h^T * log2(e)/sqrt(d_h) was
+// produced by the projection GEMM (bf16, D = 128 wide).  Keys and values are
+// the same raw history rows x_i, so one SMEM tile per block of 128 keys
+// serves both contractions:
+//   S = U X_blk^T    (M=128 rows, N=128 keys, K=128; X tile K-major)
+//   O += P X_blk     (M=128 rows, N=128, K=128 keys; P from TMEM, X tile MN-major)
+// The softmax over keys is online: each thread owns one query row (one TMEM
+// lane); the running maximum is only raised when a block's maximum exceeds it
+// by more than 8 (base-2 units), so O in TMEM is rarely rescaled.
+//
+// Warp roles (8 warps): 0 TMA, 1 MMA issue + TMEM owner, 2-3 idle,
+// 4-7 softmax and the final normalisation.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
 #include "stca_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace sa {
-bool stca_tc_supported(sa_dtype, int) { return false; }
-sa_status stca_tc_attention(const StcaArgs&, const StcaWork&, cudaStream_t) {
-  return fail(SA_ERR_UNSUPPORTED, "tensor-core STCA attention not built");
+
+namespace {
+using namespace tc;
+
+constexpr int TQ = 128, TKB = 128, DD = 128, NSK = 3, THREADS = 256;
+constexpr uint32_t TILE_BYTES = TQ * DD * 2;                       // 32 KB
+constexpr uint32_t OFF_Q = 0, OFF_KV = TILE_BYTES, OFF_BAR = OFF_KV + NSK * TILE_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
+constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_P0 = 256, TM_P1 = 320, TM_O = 384, TM_COLS = 512;
+constexpr float kRescale = 8.f;      // raise the running max only past this margin
+
+struct Bars {
+  uint64_t q_full, kv_full[NSK], kv_empty[NSK], s_full[2], p_full[2], pv_done[2], o_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct Params {
+  const int* prefix;
+  const int64_t* cand;
+  const int64_t* kvb;
+  const int64_t* kve;
+  int B, heads;
+  float* Y;
+  int* err;
+};
+
+__global__ void __launch_bounds__(THREADS, 1)
+    stca_attn_tc_kernel(const __grid_constant__ CUtensorMap tmU,
+                        const __grid_constant__ CUtensorMap tmK, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Bars* bars = (Bars*)(smem + OFF_BAR);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tile = blockIdx.x;
+  if (tile >= p.prefix[p.B]) return;
+  int lo = 0, hi = p.B - 1;                 // user: largest u with prefix[u] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.prefix[mid] <= tile) lo = mid; else hi = mid - 1;
+  }
+  const int u = lo;
+  const int64_t rend = p.cand[u + 1] * p.heads;
+  const int64_t r0 = p.cand[u] * p.heads + (int64_t)(tile - p.prefix[u]) * TQ;
+  const int64_t kb = p.kvb[u], ke = p.kve[u];
+  const int nblk = (int)((ke - kb + TKB - 1) / TKB);
+  if (nblk == 0) {
+    // no keys: the attention output is zero
+    for (int e = threadIdx.x; e < TQ * DD; e += THREADS) {
+      const int64_t row = r0 + e / DD;
+      if (row < rend) p.Y[row * DD + e % DD] = 0.f;
+    }
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < NSK; ++s) { mbar_init(&bars->kv_full[s], 1); mbar_init(&bars->kv_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->s_full[b], 1);
+      mbar_init(&bars->p_full[b], 128);
+      mbar_init(&bars->pv_done[b], 1);
+    }
+    mbar_init(&bars->o_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA
+    prefetch_tensormap(&tmU);
+    prefetch_tensormap(&tmK);
+    mbar_arrive_expect_tx(&bars->q_full, TILE_BYTES);
+    tma_load_2d(smem + OFF_Q, &tmU, &bars->q_full, 0, (int)r0);
+    tma_load_2d(smem + OFF_Q + TILE_BYTES / 2, &tmU, &bars->q_full, 64, (int)r0);
+    int issued = 0;
+    for (int j = 0; j < nblk; ++j) {
+      const int s = j % NSK;
+      if (j >= NSK && !mbar_wait(&bars->kv_empty[s], ((j / NSK) - 1) & 1, abort, p.err)) break;
+      mbar_arrive_expect_tx(&bars->kv_full[s], TILE_BYTES);
+      uint8_t* dst = smem + OFF_KV + s * TILE_BYTES;
+      const int row = (int)(kb + (int64_t)j * TKB);
+      tma_load_2d(dst, &tmK, &bars->kv_full[s], 0, row);
+      tma_load_2d(dst + TILE_BYTES / 2, &tmK, &bars->kv_full[s], 64, row);
+      issued = j + 1;
+    }
+    if (*abort) {
+      mbar_wait_bounded(&bars->q_full, 0);
+      for (int j = std::max(0, issued - NSK); j < issued; ++j)
+        mbar_wait_bounded(&bars->kv_full[j % NSK], (j / NSK) & 1);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA
+    const uint32_t idS = idesc_bf16(128, 128, false, false);
+    const uint32_t idO = idesc_bf16(128, 128, false, true);
+    const uint32_t qa = smem_u32(smem + OFF_Q);
+    auto pv = [&](int j) -> bool {
+      const int b = j & 1, s = j % NSK;
+      if (!mbar_wait(&bars->p_full[b], (j >> 1) & 1, abort, p.err)) return false;
+      tc_fence_after();
+      const uint32_t va = smem_u32(smem + OFF_KV + s * TILE_BYTES);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ts(tmem + TM_O, tmem + (b ? TM_P1 : TM_P0) + ks * 8,
+               smem_desc(va + ks * 2048, 16384, 1024, SWZ_128B), idO, (j > 0 || ks > 0) ? 1u : 0u);
+      mma_commit(&bars->kv_empty[s]);
+      mma_commit(&bars->pv_done[b]);
+      return true;
+    };
+    bool ok = mbar_wait(&bars->q_full, 0, abort, p.err);
+    for (int j = 0; ok && j < nblk; ++j) {
+      const int s = j % NSK, b = j & 1;
+      if (!mbar_wait(&bars->kv_full[s], (j / NSK) & 1, abort, p.err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t ka = smem_u32(smem + OFF_KV + s * TILE_BYTES);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ss(tmem + (b ? TM_S1 : TM_S0),
+               smem_desc(qa + (ks >> 2) * (TILE_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B),
+               smem_desc(ka + (ks >> 2) * (TILE_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B),
+               idS, ks > 0 ? 1u : 0u);
+      mma_commit(&bars->s_full[b]);
+      if (j > 0 && !pv(j - 1)) { ok = false; break; }
+    }
+    if (ok) pv(nblk - 1);
+    mma_commit(&bars->o_done);
+    mbar_wait_bounded(&bars->o_done, 0);
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- softmax
+    const int q = warp % 4;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    float m = -__builtin_huge_valf(), l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(&bars->s_full[b], (j >> 1) & 1, abort, p.err)) { ok = false; break; }
+      tc_fence_after();
+      float sv[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_addr + (b ? TM_S1 : TM_S0) + 32 * c, sv + 32 * c);
+      tmem_wait_ld();
+      const int64_t kbase = kb + (int64_t)j * TKB;
+      if (kbase + TKB > ke) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (kbase + i >= ke) sv[i] = -__builtin_huge_valf();
+      }
+      float bm = sv[0];
+#pragma unroll
+      for (int i = 1; i < 128; ++i) bm = fmaxf(bm, sv[i]);
+      const bool raise = bm > m + kRescale;
+      if (__any_sync(0xffffffffu, raise)) {
+        const float mn = fmaxf(m, bm);
+        const float corr = ex2(m - mn);        // 0 on the first block, 1 if this row keeps m
+        m = mn;
+        l *= corr;
+        if (j > 0) {
+          // O holds blocks < j: wait for the last of them, then rescale in place
+          if (!mbar_wait(&bars->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort, p.err)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float o[32];
+            tmem_ld32(tmem + lane_addr + TM_O + 32 * c, o);
+            tmem_wait_ld();
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(o[i] * corr);
+            tmem_st32(tmem + lane_addr + TM_O + 32 * c, w);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P buffer b was last read by PV(j-2)
+      if (j >= 2 && !mbar_wait(&bars->pv_done[b], ((j >> 1) - 1) & 1, abort, p.err)) { ok = false; break; }
+      uint32_t pw[64];
+      float ls = 0.f;
+#pragma unroll
+      for (int i = 0; i < 128; i += 2) {
+        const float e0 = ex2(sv[i] - m), e1 = ex2(sv[i + 1] - m);
+        ls += e0 + e1;
+        pw[i / 2] = pack_bf16x2(e0, e1);
+      }
+      l += ls;
+      tmem_st32(tmem + lane_addr + (b ? TM_P1 : TM_P0), pw);
+      tmem_st32(tmem + lane_addr + (b ? TM_P1 : TM_P0) + 32, pw + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[b]);
+    }
+    if (ok && mbar_wait(&bars->o_done, 0, abort, p.err)) {
+      tc_fence_after();
+      const int64_t grow = r0 + row;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_addr + TM_O + 32 * c, o);
+        tmem_wait_ld();
+        if (grow < rend) {
+          float* dst = p.Y + grow * DD + 32 * c;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *(float4*)(dst + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
 }
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* q = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      fn = (EncodeFn)q;
+  });
+  return fn;
+}
+
+sa_status make_map(CUtensorMap* map, const void* base, uint64_t rows) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {DD, rows};
+  cuuint64_t strides[1] = {DD * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return SA_OK;
+}
+}  // namespace
+
+bool stca_tc_supported(sa_dtype dtype, int D) { return dtype == SA_BF16 && D == DD; }
+
+sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(stca_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  });
+  if (a.kv_rows >= (1LL << 31) || a.C_total * a.heads >= (1LL << 31))
+    return fail(SA_ERR_UNSUPPORTED, "row counts must be < 2^31");
+  CUtensorMap tmU, tmK;
+  sa_status s = make_map(&tmU, w.Ub, (uint64_t)(a.C_total * a.heads));
+  if (s != SA_OK) return s;
+  if (a.kv_rows > 0) {
+    s = make_map(&tmK, a.kv, (uint64_t)a.kv_rows);
+    if (s != SA_OK) return s;
+  } else {
+    memset(&tmK, 0, sizeof(tmK));     // never read: every key range is empty
+  }
+  Params p{w.tile_prefix, a.cand_dev, a.kvb_dev, a.kve_dev, a.B, a.heads, w.Y, device_status_word()};
+  SA_TIMED("stca_attn_tc_kernel", st,
+           (stca_attn_tc_kernel<<<w.max_tiles, THREADS, SMEM_BYTES, st>>>(tmU, tmK, p)));
+  return SA_OK;
+}
+
 }  // namespace sa
