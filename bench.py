@@ -135,7 +135,8 @@ class TrainStepRunner:
         B, k, d, C = self.B, self.k, self.d, int(self.cand[-1])
         n = sa.n_total
         e = lambda *s, dt=torch.float32: torch.empty(*s, device=device, dtype=dt)
-        self.fo = {"S": e(B, k, d), "mass": e(B, k), "H": e(B, k, d), "S_bf16": e(B, k, d, dt=torch.bfloat16)}
+        self.fo = {"S": e(B, k, d), "mass": e(B, k), "H": e(B, k, d),
+                   "S_bf16": e(B, k, d, dt=torch.bfloat16), "lse": e(n)}
         self.go = {"dX": e(n, d, dt=torch.bfloat16), "dP": e(k, d), "dW_Q": e(d, d), "dW_K": e(d, d), "dW_V": e(d, d)}
         self.zr, self.zu, self.z = e(C, d), e(C, d), e(C, d)
         sab_ws = lambda nbytes: torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
@@ -154,8 +155,8 @@ class TrainStepRunner:
                              offsets_dev=self.offd, out=self.fo, workspace=self.ws_f)
         if ev: ev[1].record()
         g = sab.sa_backward(self.X, self.off, self.P, self.WQ, self.WK, self.WV, w.sa.eps,
-                            fwd["H"], fwd["mass"], self.dS, offsets_dev=self.offd, out=self.go,
-                            workspace=self.ws_b)
+                            fwd["H"], fwd["mass"], self.dS, None, fwd["lse"],
+                            offsets_dev=self.offd, out=self.go, workspace=self.ws_b)
         if self.world > 1:
             for name in ("dP", "dW_Q", "dW_K", "dW_V"):
                 torch.distributed.all_reduce(g[name])
@@ -406,6 +407,82 @@ def run_reference(args):
     }
 
 
+def run_component(args, rank, world, device):
+    """SA forward alone (32 users x 100K, k=1024) or STCA alone (16 users x 512
+    candidates): for profiling the two tensor-core kernels in isolation."""
+    import sketch_attention_b200 as sab
+    from sketch_attention_b200 import build as _b
+    if rank == 0 or not os.path.exists(_b.LIB):
+        _b.build()
+    sab.load()
+    from sa_inputs import STCA_WORKLOAD_4, sa_workload, stca_workload
+    peaks, peaks_src = load_peaks()
+    if args.workload == "sa_fwd":
+        p = sa_workload(3, users=args.users)
+        X = _dev_bf16(p.X, device)
+        offd = torch.from_numpy(p.offsets).to(device)
+        P, WQ, WK, WV = (_f32(a, device) for a in (p.P, p.W_Q, p.W_K, p.W_V))
+        out = {"S": torch.empty(p.B, p.k, p.d, device=device),
+               "mass": torch.empty(p.B, p.k, device=device),
+               "lse": torch.empty(p.n_total, device=device)}
+        ws = torch.empty(sab.sa_forward_workspace(p.B, p.n_total, p.k, p.d, sab.SA_BF16),
+                         dtype=torch.uint8, device=device)
+        step = lambda: sab.sa_forward(X, p.offsets, P, WQ, WK, WV, p.eps, offsets_dev=offd, out=out,
+                                      workspace=ws)
+        units, unit, name = p.n_total, "history-tokens/s", p.name
+        kname, flops = "sa_fwd_tc_kernel", 4.0 * p.k * p.d * p.n_total
+    else:
+        w = stca_workload(users=args.users or 16)
+        q, kvr, kvs = (_dev_bf16(a, device) for a in (w.recent.q, w.recent.kv, w.sketch.kv))
+        lay = lambda L: dict(W_Q=_f32(L.W_Q, device), W_K=_f32(L.W_K, device),
+                             W_V=_f32(L.W_V, device), W_O=_f32(L.W_O, device))
+        lr, lu = [lay(L) for L in w.layers_r], [lay(L) for L in w.layers_u]
+        WF, bF = _f32(w.W_F, device), _f32(w.b_F, device)
+        C = int(w.recent.cand_offsets[-1])
+        zr, zu, z = (torch.empty(C, 128, device=device) for _ in range(3))
+
+        def step():
+            sab.stca_forward(q, w.recent.cand_offsets, kvr, w.recent.kv_begin, w.recent.kv_end,
+                             lr, w.heads, w.d_h, out=zr)
+            sab.stca_forward(q, w.sketch.cand_offsets, kvs, w.sketch.kv_begin, w.sketch.kv_end,
+                             lu, w.heads, w.d_h, out=zu)
+            sab.stca_fuse(zr, zu, WF, bF, out=z)
+        units, unit, name = C, "candidates/s", STCA_WORKLOAD_4
+        L_avg = 0.5 * (float(np.mean(w.recent.kv_end - w.recent.kv_begin)) + 1024)
+        kname, flops = "stca_attn_tc_kernel", 4.0 * L_avg * 128 * C * w.heads
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sab.profile(True)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index or 0) as clk:
+        start.record()
+        for _ in range(args.steps):
+            step()
+        end.record()
+        torch.cuda.synchronize()
+    prof = sab.profile_read()
+    sab.profile(False)
+    ms = start.elapsed_time(end) / args.steps
+    roof = None
+    if kname in prof:
+        tot, cnt = prof[kname]
+        ach = flops / (tot / cnt / 1e3) / 1e12
+        pk = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+        roof = {"kernel": kname, "bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
+                "frac": ach / pk, "traffic": None,
+                "peak_source": f"bf16 dense, burst ({peaks_src}): the kernel is timed alone",
+                "avg_launch_ms": tot / cnt}
+    return {"metric": unit, "value": world * units / (ms / 1e3), "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": name},
+            "roofline": roof,
+            "kernels": {n: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
+                        for n, v in sorted(prof.items(), key=lambda kv: -kv[1][0])},
+            "clocks": clk.summary()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -414,6 +491,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca"], default="train",
+                    help="train: the full step (default, the headline); sa_fwd: SA forward over "
+                         "32 users x 100K (k=1024); stca: STCA of 16 users x 512 candidates")
+    ap.add_argument("--users", type=int, default=None, help="shrink the batch (profiling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -429,7 +510,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=device)
     try:
-        line = run_ours(args, rank, world, device)
+        if args.workload == "train":
+            line = run_ours(args, rank, world, device)
+        else:
+            line = run_component(args, rank, world, device)
         if rank == 0:
             print(json.dumps(line), flush=True)
     finally:

@@ -91,6 +91,8 @@ size_t sa_forward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dty
  * H        [B, k, d] fp32 out, optional (NULL): the unnormalised A X, which
  *          sa_backward needs.
  * S_bf16   [B, k, d] bf16 out, optional (NULL): S rounded to bf16 (for STCA).
+ * lse      [n_total] fp32 out, optional (NULL): each token's log-sum-exp over
+ *          the k prototypes, ln sum_j exp Z_ji (sa_backward reuses it).
  * A user with n_u = 0 gets S = 0, mass = 0, H = 0.
  * Supported: 1 <= k <= 4096, d in {64, 128}, B >= 1, eps >= 0.
  */
@@ -99,7 +101,7 @@ sa_status sa_forward(const void* X, sa_dtype x_dtype,
                      int k, int d,
                      const float* P, const float* W_Q, const float* W_K, const float* W_V,
                      float eps,
-                     float* S, float* mass, float* H, void* S_bf16,
+                     float* S, float* mass, float* H, void* S_bf16, float* lse,
                      void* workspace, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
@@ -118,8 +120,9 @@ size_t sa_backward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dt
  *   E = sum_u dZ_u X_u;  dP = E W_K W_Q^T/sqrt(d);  dW_Q = P^T E W_K/sqrt(d);
  *   dW_K = E^T P W_Q/sqrt(d)
  *
- * Inputs as sa_forward, plus H and mass from sa_forward, dS [B,k,d] fp32 and
- * dmass [B,k] fp32 (NULL = zero).
+ * Inputs as sa_forward, plus H and mass from sa_forward, dS [B,k,d] fp32,
+ * dmass [B,k] fp32 (NULL = zero) and lse [n_total] from sa_forward (NULL = the
+ * backward recomputes it).
  * dX [n_total, d] x_dtype out; dP [k,d], dW_Q, dW_K, dW_V [d,d] fp32 out
  * (sums over the batch).
  */
@@ -129,7 +132,7 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype,
                       const float* P, const float* W_Q, const float* W_K, const float* W_V,
                       float eps,
                       const float* H, const float* mass, const float* dS, const float* dmass,
-                      void* dX, float* dP, float* dW_Q, float* dW_K, float* dW_V,
+                      const float* lse, void* dX, float* dP, float* dW_Q, float* dW_K, float* dW_V,
                       void* workspace, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */

@@ -39,7 +39,7 @@ import numpy as np
 
 __all__ = [
     "sa_forward", "sa_user", "sa_backward", "stca_branch", "stca_branch_reordered",
-    "stca_fuse", "assignment",
+    "stca_fuse", "assignment", "token_lse",
 ]
 
 
@@ -62,6 +62,16 @@ def assignment(Xu, P, W_Q, W_K) -> np.ndarray:
     Zc = Z - Z.max(axis=0, keepdims=True)
     E = np.exp(Zc)
     return E / E.sum(axis=0, keepdims=True)   # softmax over prototypes, eq. (8)
+
+
+def token_lse(Xu, P, W_Q, W_K) -> np.ndarray:
+    """Each token's log-sum-exp over the prototypes, ln sum_j exp S_{j,i}: the
+    normaliser of the prototype-wise softmax (eqs. (6)-(8))."""
+    Xu, P, W_Q, W_K = _f64(Xu), _f64(P), _f64(W_Q), _f64(W_K)
+    d = P.shape[1]
+    Z = ((P @ W_Q) @ (Xu @ W_K).T) / math.sqrt(d)
+    zmax = Z.max(axis=0)
+    return zmax + np.log(np.exp(Z - zmax[None, :]).sum(axis=0))
 
 
 def sa_user(Xu, P, W_Q, W_K, W_V, eps: float):

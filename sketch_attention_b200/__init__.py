@@ -63,12 +63,12 @@ def load(path: Optional[str] = None):
     lib.sa_forward_workspace.argtypes = [_i, _i64, _i, _i, _i]
     lib.sa_forward.restype = _i
     lib.sa_forward.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
-                               _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+                               _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.sa_backward_workspace.restype = _sz
     lib.sa_backward_workspace.argtypes = [_i, _i64, _i, _i, _i]
     lib.sa_backward.restype = _i
     lib.sa_backward.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
-                                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+                                _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.stca_forward_workspace.restype = _sz
     lib.stca_forward_workspace.argtypes = [_i, _i64, _i, _i, _i, _i]
     lib.stca_forward.restype = _i
@@ -137,9 +137,9 @@ def sa_forward_workspace(B: int, n_total: int, k: int, d: int, dtype: int) -> in
 
 def sa_forward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
                offsets_dev: Optional[torch.Tensor] = None, want_H: bool = False,
-               want_bf16: bool = False, out: Optional[dict] = None,
+               want_bf16: bool = False, want_lse: bool = False, out: Optional[dict] = None,
                workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
-    """Sketches of a ragged batch.  Returns {"S", "mass"[, "H"][, "S_bf16"]}."""
+    """Sketches of a ragged batch.  Returns {"S", "mass"[, "H"][, "S_bf16"][, "lse"]}."""
     lib = load()
     _need_cuda(X, P, W_Q, W_K, W_V)
     off = _host_i64(offsets)
@@ -153,12 +153,14 @@ def sa_forward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
     H = o.get("H") if o.get("H") is not None else (torch.empty(B, k, d, device=dev) if want_H else None)
     Sb = o.get("S_bf16") if o.get("S_bf16") is not None else (
         torch.empty(B, k, d, device=dev, dtype=torch.bfloat16) if want_bf16 else None)
+    lse = o.get("lse") if o.get("lse") is not None else (
+        torch.empty(max(int(off[-1]), 1), device=dev) if want_lse else None)
     ws_bytes = lib.sa_forward_workspace(B, int(off[-1]), k, d, dt)
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     offd = _dev_i64(off, dev, offsets_dev)
     st = lib.sa_forward(_p(X), dt, _hp(off), _p(offd), B, k, d, _p(P), _p(W_Q), _p(W_K), _p(W_V),
-                        float(eps), _p(S), _p(mass), _p(H), _p(Sb), _p(workspace),
+                        float(eps), _p(S), _p(mass), _p(H), _p(Sb), _p(lse), _p(workspace),
                         workspace.numel(), _stream(stream))
     _check("sa_forward", st)
     res = {"S": S, "mass": mass}
@@ -166,6 +168,8 @@ def sa_forward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
         res["H"] = H
     if Sb is not None:
         res["S_bf16"] = Sb
+    if lse is not None:
+        res["lse"] = lse
     return res
 
 
@@ -174,12 +178,12 @@ def sa_backward_workspace(B: int, n_total: int, k: int, d: int, dtype: int) -> i
 
 
 def sa_backward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float, H, mass, dS,
-                dmass=None, *, offsets_dev: Optional[torch.Tensor] = None,
+                dmass=None, lse=None, *, offsets_dev: Optional[torch.Tensor] = None,
                 out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
                 stream=None) -> dict:
     """Gradients {"dX", "dP", "dW_Q", "dW_K", "dW_V"} of <dS, S> + <dmass, mass>."""
     lib = load()
-    _need_cuda(X, P, W_Q, W_K, W_V, H, mass, dS, dmass)
+    _need_cuda(X, P, W_Q, W_K, W_V, H, mass, dS, dmass, lse)
     off = _host_i64(offsets)
     B = len(off) - 1
     k, d = P.shape
@@ -196,7 +200,7 @@ def sa_backward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float, H, mass,
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     offd = _dev_i64(off, dev, offsets_dev)
     st = lib.sa_backward(_p(X), dt, _hp(off), _p(offd), B, k, d, _p(P), _p(W_Q), _p(W_K), _p(W_V),
-                         float(eps), _p(H), _p(mass), _p(dS), _p(dmass), _p(dX), _p(dP), _p(dWQ),
+                         float(eps), _p(H), _p(mass), _p(dS), _p(dmass), _p(lse), _p(dX), _p(dP), _p(dWQ),
                          _p(dWK), _p(dWV), _p(workspace), workspace.numel(), _stream(stream))
     _check("sa_backward", st)
     return {"dX": dX, "dP": dP, "dW_Q": dWQ, "dW_K": dWK, "dW_V": dWV}

@@ -298,8 +298,8 @@ size_t sa_forward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dty
 sa_status sa_forward(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
                      const int64_t* offsets_dev, int B, int k, int d, const float* P,
                      const float* W_Q, const float* W_K, const float* W_V, float eps, float* S,
-                     float* mass, float* H, void* S_bf16, void* workspace, size_t ws_bytes,
-                     sa_stream_t stream) {
+                     float* mass, float* H, void* S_bf16, float* lse, void* workspace,
+                     size_t ws_bytes, sa_stream_t stream) {
   SA_TRY(check_sa_shape(B, k, d, x_dtype));
   SA_TRY(check_offsets(offsets_host, B, "offsets_host"));
   const int64_t n = offsets_host[B];
@@ -314,6 +314,7 @@ sa_status sa_forward(const void* X, sa_dtype x_dtype, const int64_t* offsets_hos
   SA_TRY(check_ptr(mass, "mass"));
   SA_TRY(check_ptr(H, "H", true));
   SA_TRY(check_ptr(S_bf16, "S_bf16", true));
+  SA_TRY(check_ptr(lse, "lse", true));
   if (H == S) return fail(SA_ERR_INVALID_ARG, "H must not alias S");
   const size_t need = layout_fwd(nullptr, B, n, k, d, x_dtype, nullptr);
   if (!workspace || ws_bytes < need)
@@ -321,7 +322,7 @@ sa_status sa_forward(const void* X, sa_dtype x_dtype, const int64_t* offsets_hos
   SA_TRY(check_ptr(workspace, "workspace"));
   SaFwdWork w;
   layout_fwd(workspace, B, n, k, d, x_dtype, &w);
-  SaFwdArgs a{X, x_dtype, offsets_dev, B, n, k, d, P, W_Q, W_K, W_V, eps, S, mass, H, S_bf16};
+  SaFwdArgs a{X, x_dtype, offsets_dev, B, n, k, d, P, W_Q, W_K, W_V, eps, S, mass, H, S_bf16, lse};
   cudaStream_t st = (cudaStream_t)stream;
   SA_TRY(sa_fold(k, d, P, W_Q, W_K, w.T, w.Pf, w.Pb, st));
   if (n > 0) {
@@ -341,8 +342,8 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_ho
                       const int64_t* offsets_dev, int B, int k, int d, const float* P,
                       const float* W_Q, const float* W_K, const float* W_V, float eps,
                       const float* H, const float* mass, const float* dS, const float* dmass,
-                      void* dX, float* dP, float* dW_Q, float* dW_K, float* dW_V,
-                      void* workspace, size_t ws_bytes, sa_stream_t stream) {
+                      const float* lse, void* dX, float* dP, float* dW_Q, float* dW_K,
+                      float* dW_V, void* workspace, size_t ws_bytes, sa_stream_t stream) {
   SA_TRY(check_sa_shape(B, k, d, x_dtype));
   SA_TRY(check_offsets(offsets_host, B, "offsets_host"));
   const int64_t n = offsets_host[B];
@@ -358,6 +359,7 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_ho
   SA_TRY(check_ptr(mass, "mass"));
   SA_TRY(check_ptr(dS, "dS"));
   SA_TRY(check_ptr(dmass, "dmass", true));
+  SA_TRY(check_ptr(lse, "lse", true));
   SA_TRY(check_ptr(dP, "dP"));
   SA_TRY(check_ptr(dW_Q, "dW_Q"));
   SA_TRY(check_ptr(dW_K, "dW_K"));
@@ -369,7 +371,7 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_ho
   SaBwdWork w;
   layout_bwd(workspace, B, n, k, d, &w);
   SaBwdArgs a{X, x_dtype, offsets_dev, B, n, k, d, P, W_Q, W_K, W_V, eps,
-              H, mass, dS, dmass, dX, dP, dW_Q, dW_K, dW_V};
+              H, mass, dS, dmass, lse, dX, dP, dW_Q, dW_K, dW_V};
   cudaStream_t st = (cudaStream_t)stream;
   SA_TRY(sa_fold(k, d, P, W_Q, W_K, w.T, w.Pf, w.Pb, st));
   return sa_simt_backward(a, w, st);

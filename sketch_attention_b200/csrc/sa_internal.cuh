@@ -11,7 +11,7 @@ struct SaFwdArgs {
   int k, d;
   const float *P, *W_Q, *W_K, *W_V;
   float eps;
-  float* S; float* mass; float* H; void* S_bf16;
+  float* S; float* mass; float* H; void* S_bf16; float* lse_out;
 };
 
 // Workspace views of sa_forward.
@@ -33,7 +33,7 @@ struct SaBwdArgs {
   int k, d;
   const float *P, *W_Q, *W_K, *W_V;
   float eps;
-  const float *H, *mass, *dS, *dmass;
+  const float *H, *mass, *dS, *dmass, *lse_in;
   void* dX; float *dP, *dW_Q, *dW_K, *dW_V;
 };
 

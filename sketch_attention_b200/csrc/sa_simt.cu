@@ -30,7 +30,8 @@ __device__ __forceinline__ void load_row_f32(float* dst, const XT* src, int64_t 
 template <class XT, int D>
 __global__ void __launch_bounds__(128) sa_lse_kernel(const XT* __restrict__ X, int64_t n_total,
                                                      const float* __restrict__ Pf, int k,
-                                                     float* __restrict__ lse) {
+                                                     float* __restrict__ lse,
+                                                     float* __restrict__ lse_nat) {
   __shared__ float Ps[32][D];
   const int64_t t = (int64_t)blockIdx.x * 128 + threadIdx.x;
   const bool valid = t < n_total;
@@ -50,7 +51,19 @@ __global__ void __launch_bounds__(128) sa_lse_kernel(const XT* __restrict__ X, i
       else s += exp2f(z - m);
     }
   }
-  if (valid) lse[t] = m + log2f(s);
+  if (valid) {
+    const float l2 = m + log2f(s);
+    lse[t] = l2;
+    if (lse_nat) lse_nat[t] = l2 * kLn2;
+  }
+}
+
+// lse2[t] = lse[t] * log2(e): a caller-provided natural-log lse in base-2 units.
+__global__ void lse_to_log2_kernel(const float* __restrict__ lse, int64_t n,
+                                   float* __restrict__ lse2) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x)
+    lse2[e] = lse[e] * 1.4426950408889634f;
 }
 
 // ---------------------------------------------------------------- pass 2
@@ -420,7 +433,7 @@ sa_status launch_simt_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream
   if (N > 0) {
     SA_TIMED("sa_lse_kernel", st,
              (sa_lse_kernel<XT, D><<<(unsigned)((N + 127) / 128), 128, 0, st>>>(
-                 (const XT*)a.X, N, w.Pf, a.k, w.lse)));
+                 (const XT*)a.X, N, w.Pf, a.k, w.lse, a.lse_out)));
     dim3 grid((a.k + 31) / 32, w.ch.G);
     SA_TIMED("sa_agg_kernel", st,
              (sa_agg_kernel<XT, D><<<grid, 256, 0, st>>>((const XT*)a.X, a.off_dev, a.B, w.ch,
@@ -434,9 +447,15 @@ template <class XT, int D>
 sa_status launch_simt_backward(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st) {
   const int64_t N = a.n_total;
   if (N <= 0) return SA_OK;
-  SA_TIMED("sa_lse_kernel", st,
-           (sa_lse_kernel<XT, D><<<(unsigned)((N + 127) / 128), 128, 0, st>>>(
-               (const XT*)a.X, N, w.Pf, a.k, w.lse)));
+  if (a.lse_in) {
+    SA_TIMED("lse_to_log2_kernel", st,
+             (lse_to_log2_kernel<<<(unsigned)std::min<int64_t>((N + 255) / 256, 8192), 256, 0, st>>>(
+                 a.lse_in, N, w.lse)));
+  } else {
+    SA_TIMED("sa_lse_kernel", st,
+             (sa_lse_kernel<XT, D><<<(unsigned)((N + 127) / 128), 128, 0, st>>>(
+                 (const XT*)a.X, N, w.Pf, a.k, w.lse, nullptr)));
+  }
   SA_TIMED("sa_bwd_token_kernel", st,
            (sa_bwd_token_kernel<XT, D><<<w.ch.G, 256, 0, st>>>(
                (const XT*)a.X, a.off_dev, a.B, w.ch, w.Pf, a.k, w.lse, w.dH, w.dm, w.cbuf,

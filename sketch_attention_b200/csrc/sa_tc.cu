@@ -19,9 +19,10 @@
 //   MMA2   H_slice[j, :] += sum_t p[t, j] [x_t | 1]   (M=128 prototypes, N=144, K=128 tokens)
 // so the k x n assignment matrix never leaves the SM.
 //
-// Warp roles (12 warps): 0 TMA, 1 MMA issue + TMEM owner, 2-3 idle,
-// 4-7 softmax of even tiles (and the H drain at the end of a piece),
-// 8-11 softmax of odd tiles.
+// Warp roles (10 warps): 0 TMA, 1 MMA issue + TMEM owner, 2-5 softmax of
+// even tiles (and the H drain at the end of a piece), 6-9 softmax of odd
+// tiles.  A warp reads TMEM lanes 32 (warp % 4) .. +31, so each group of four
+// consecutive warps covers all 128 lanes.
 #include <algorithm>
 #include <mutex>
 
@@ -38,7 +39,7 @@ constexpr int DD = 128;              // d
 constexpr int NS = 3;                // X pipeline stages
 constexpr int MAXC = 8;              // cluster size limit (k <= 1024)
 constexpr int N2 = DD + 16;          // MMA2 N: d columns + 16 mass columns
-constexpr int THREADS = 384;
+constexpr int THREADS = 320;
 
 // shared-memory layout (offsets from a 1024-aligned base)
 constexpr uint32_t X_BOX = TILE * 32;                  // one [128 x 16] bf16 SW32 box = 4 KB
@@ -73,6 +74,7 @@ struct Params {
   float* Muser;
   float* slotH;
   float* slotM;
+  float* lse;          // optional per-token ln-sum-exp output
   int* err;
 };
 
@@ -90,7 +92,7 @@ __device__ __forceinline__ void for_each_tile(const Params& p, int g, F&& f) {
   }
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __maxnreg__(200)
     sa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmP, Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -215,9 +217,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       // every MMA this thread issued has completed before TMEM is released
       mma_commit(&bars->mma_done);
       mbar_wait_bounded(&bars->mma_done, 0);
-    } else if (warp >= 4) {
+    } else if (warp >= 2) {
       // ------------------------------------------------------------ softmax groups
-      const int wg = (warp - 4) / 4;            // 0: even tiles, 1: odd tiles
+      const int wg = (warp - 2) / 4;            // 0: even tiles, 1: odd tiles
       const int q = warp % 4;                   // TMEM lane quarter
       const int row = q * 32 + lane;            // token within the tile / prototype lane
       const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
@@ -233,13 +235,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           if (!mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort, p.err)) return false;
           tc_fence_after();
           // Two halves of 64 columns; each half is exponentiated against the
-          // running maximum at that point (mh[h]) and kept as bf16 pairs.
-          uint32_t ep[64];
+          // running maximum at that point (mh[h]); the exponentials stay fp32
+          // so the probabilities are rounded to bf16 once.
+          float e[128];
           float mh[2];
           float m = -__builtin_huge_valf(), s = 0.f;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            float z[64];
+            float* z = e + 64 * h;
             tmem_ld32(tmem + lane_addr + (b ? TM_S1 : TM_S0) + 64 * h, z);
             tmem_ld32(tmem + lane_addr + (b ? TM_S1 : TM_S0) + 64 * h + 32, z + 32);
             tmem_wait_ld();
@@ -251,10 +254,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             m = mn;
             mh[h] = mn;
 #pragma unroll
-            for (int j = 0; j < 64; j += 2) {
-              const float e0 = ex2(z[j] - mn), e1 = ex2(z[j + 1] - mn);
-              s += e0 + e1;
-              ep[32 * h + j / 2] = pack_bf16x2(e0, e1);
+            for (int j = 0; j < 64; ++j) {
+              z[j] = ex2(z[j] - mn);
+              s += z[j];
             }
           }
           const float l = valid ? m + lg2(s) : -__builtin_huge_valf();
@@ -272,16 +274,16 @@ __global__ void __launch_bounds__(THREADS, 1)
               bulk_copy_to_peer(map_to_rank(dst, c), src, TILE * 4, map_to_rank(bar, c));
           }
           if (!mbar_wait(&bars->xchg[slot], (t >> 2) & 1, abort, p.err)) return false;
-          uint32_t rr[2] = {0u, 0u};
+          float rh[2] = {0.f, 0.f};
           if (valid) {
             float L = -__builtin_huge_valf();
             for (uint32_t c = 0; c < C; ++c) L = fmaxf(L, xchg[(slot * MAXC + c) * TILE + row]);
             float z = 0.f;
             for (uint32_t c = 0; c < C; ++c) z += ex2(xchg[(slot * MAXC + c) * TILE + row] - L);
             const float lt = L + lg2(z);
-            const float r0 = ex2(mh[0] - lt), r1 = ex2(mh[1] - lt);
-            rr[0] = pack_bf16x2(r0, r0);
-            rr[1] = pack_bf16x2(r1, r1);
+            if (p.lse && rank == 0) p.lse[tb + row] = lt * 0.69314718055994530942f;
+            rh[0] = ex2(mh[0] - lt);
+            rh[1] = ex2(mh[1] - lt);
           }
           named_bar_sync(1 + wg, 128);      // every thread has read the slot
           if (row == 0) mbar_arrive_expect_tx(&bars->xchg[slot], C * TILE * 4);   // re-arm for t+4
@@ -290,12 +292,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t pa = smem_u32(smem + OFF_P + b * 32768) + row * 128;
 #pragma unroll
           for (int blk = 0; blk < 2; ++blk) {
+            const float r = rh[blk];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const int q4 = blk * 32 + c * 4;        // index of the first bf16 pair
+              const float* q8 = e + blk * 64 + c * 8;
               st_shared_v4(pa + blk * 16384 + ((c ^ (row & 7)) << 4),
-                           mul_bf16x2(ep[q4], rr[blk]), mul_bf16x2(ep[q4 + 1], rr[blk]),
-                           mul_bf16x2(ep[q4 + 2], rr[blk]), mul_bf16x2(ep[q4 + 3], rr[blk]));
+                           pack_bf16x2(q8[0] * r, q8[1] * r), pack_bf16x2(q8[2] * r, q8[3] * r),
+                           pack_bf16x2(q8[4] * r, q8[5] * r), pack_bf16x2(q8[6] * r, q8[7] * r));
             }
           }
           fence_proxy_async_smem();
@@ -435,7 +438,8 @@ sa_status sa_tc_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st)
   if (s != SA_OK) return s;
   s = make_map(&tmP, w.Pb, DD, (uint64_t)a.k, 64, TILE, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != SA_OK) return s;
-  Params p{a.off_dev, a.B, w.ch, a.k, a.S, w.Muser, w.slotH, w.slotM, device_status_word()};
+  Params p{a.off_dev, a.B, w.ch, a.k, a.S, w.Muser, w.slotH, w.slotM, a.lse_out,
+           device_status_word()};
   clusters_for(C);   // sets the kernel attributes once per device
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[1];

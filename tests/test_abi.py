@@ -61,7 +61,7 @@ def _fwd(lib, offsets, k=64, d=64, x=0x1000, ws_bytes=1 << 40, eps=1e-6):
     B = len(off) - 1
     p = _fake(0x2000)
     return lib.sa_forward(_fake(x), sab.SA_F32, off.ctypes.data_as(ctypes.c_void_p), p, B, k, d,
-                          p, p, p, p, eps, p, p, None, None, _fake(0x100000), ws_bytes, None)
+                          p, p, p, p, eps, p, p, None, None, None, _fake(0x100000), ws_bytes, None)
 
 
 def test_rejects_bad_arguments_without_touching_the_gpu(lib):

@@ -101,6 +101,25 @@ def test_two_prototype_closed_form_fixes_scale_and_operand_order():
     np.testing.assert_allclose(S[0, 1], (1 - a1) / (1 - a1 + 0.25) * np.array([2.0, -1.0]), rtol=1e-14)
 
 
+def test_token_lse_closed_forms():
+    """k = 1: the log-sum-exp is the single affinity; P = 0: ln k; two
+    prototypes with the closed-form affinities above: ln(e^{s/sqrt 2} + 1)."""
+    rng = np.random.default_rng(12)
+    d = 5
+    X = rng.standard_normal((9, d))
+    P1, WQ, WK = rng.standard_normal((1, d)), rng.standard_normal((d, d)), rng.standard_normal((d, d))
+    z = ((P1 @ WQ) @ (X @ WK).T / math.sqrt(d))[0]
+    np.testing.assert_allclose(oracle.token_lse(X, P1, WQ, WK), z, rtol=1e-13)
+    np.testing.assert_allclose(oracle.token_lse(X, np.zeros((7, d)), WQ, WK), np.log(7.0), rtol=1e-15)
+    s = 1.7
+    P = np.array([[0.0, s], [0.0, 0.0]])
+    lse = oracle.token_lse(np.array([[1.0, 0.0]]), P, np.eye(2), np.array([[0.0, 1.0], [0.0, 0.0]]))
+    np.testing.assert_allclose(lse, [math.log(math.exp(s / math.sqrt(2.0)) + 1.0)], rtol=1e-14)
+    # the assignment is exp(S - lse)
+    A = oracle.assignment(X, P1, WQ, WK)
+    np.testing.assert_allclose(A, 1.0, rtol=1e-15)
+
+
 def test_hard_assignment_limit():
     """Scaling every affinity up drives the prototype-wise softmax to a one-hot
     argmax, so H_j becomes the sum of the tokens whose best prototype is j and
