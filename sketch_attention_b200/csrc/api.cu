@@ -188,12 +188,13 @@ size_t layout_fwd(void* base, int B, int64_t n, int k, int d, sa_dtype dt, SaFwd
   return c.bytes();
 }
 
-size_t layout_bwd(void* base, int B, int64_t n, int k, int d, SaBwdWork* w) {
+size_t layout_bwd(void* base, int B, int64_t n, int k, int d, sa_dtype dt, SaBwdWork* w) {
   const DeviceInfo& di = device_info();
-  int target = 8 * di.sm_count;
+  const bool tc = sa_bwd_tc_supported(dt, k, d);
+  int target = tc ? sa_bwd_tc_dx_chunks() : 8 * di.sm_count;
   target = (int)std::min<int64_t>(target, std::max<int64_t>(1, n / 64));
   Chunking ch = make_chunking(n, target, 1);
-  int targetE = std::max(1, 4 * di.sm_count / ((k + 15) / 16));
+  int targetE = tc ? sa_bwd_tc_e_chunks(k) : std::max(1, 4 * di.sm_count / ((k + 15) / 16));
   targetE = (int)std::min<int64_t>(targetE, std::max<int64_t>(1, n / 256));
   Chunking chE = make_chunking(n, targetE, 1);
   Carve c(base);
@@ -208,7 +209,9 @@ size_t layout_bwd(void* base, int B, int64_t n, int k, int d, SaBwdWork* w) {
   v.dHh = c.take<float>((size_t)B * k * d);
   v.Hhat = c.take<float>((size_t)B * k * d);
   v.dH = c.take<float>((size_t)B * k * d);
+  v.dHb = tc ? c.take<__nv_bfloat16>((size_t)B * k * d) : nullptr;
   v.dm = c.take<float>((size_t)B * k);
+  v.dmc = tc ? c.take<float>((size_t)B * k) : nullptr;
   v.Epart = c.take<float>((size_t)std::max(chE.G, 1) * k * d);
   v.E = c.take<float>((size_t)k * d);
   v.dQ = c.take<float>((size_t)k * d);
@@ -333,9 +336,8 @@ sa_status sa_forward(const void* X, sa_dtype x_dtype, const int64_t* offsets_hos
 }
 
 size_t sa_backward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype) {
-  (void)x_dtype;
   if (B < 1 || k < 1 || d < 1 || n_total < 0) return 0;
-  return layout_bwd(nullptr, B, n_total, k, d, nullptr);
+  return layout_bwd(nullptr, B, n_total, k, d, x_dtype, nullptr);
 }
 
 sa_status sa_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
@@ -364,17 +366,17 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_ho
   SA_TRY(check_ptr(dW_Q, "dW_Q"));
   SA_TRY(check_ptr(dW_K, "dW_K"));
   SA_TRY(check_ptr(dW_V, "dW_V"));
-  const size_t need = layout_bwd(nullptr, B, n, k, d, nullptr);
+  const size_t need = layout_bwd(nullptr, B, n, k, d, x_dtype, nullptr);
   if (!workspace || ws_bytes < need)
     return fail(SA_ERR_WORKSPACE, "workspace needs " + std::to_string(need) + " bytes");
   SA_TRY(check_ptr(workspace, "workspace"));
   SaBwdWork w;
-  layout_bwd(workspace, B, n, k, d, &w);
+  layout_bwd(workspace, B, n, k, d, x_dtype, &w);
   SaBwdArgs a{X, x_dtype, offsets_dev, B, n, k, d, P, W_Q, W_K, W_V, eps,
               H, mass, dS, dmass, lse, dX, dP, dW_Q, dW_K, dW_V};
   cudaStream_t st = (cudaStream_t)stream;
   SA_TRY(sa_fold(k, d, P, W_Q, W_K, w.T, w.Pf, w.Pb, st));
-  return sa_simt_backward(a, w, st);
+  return sa_backward_run(a, w, sa_bwd_tc_supported(x_dtype, k, d), st);
 }
 
 size_t stca_forward_workspace(int B, int64_t C_total, int D, int heads, int d_h, sa_dtype dtype) {

@@ -1,0 +1,597 @@
+// Tensor-core Sketch Attention backward for sm_100a: the chain rule of the SA
+// forward (SequenceO1 Sec. 3.1, eqs. (6)-(9); the pages call SA fully
+// differentiable and print no backward).
+//
+// With A = 2^{z - lse} (z = P' x in base-2 units, lse saved by the forward),
+// dA_tj = dH_j . x_t + dm_j, c_t = sum_j A_tj dA_tj and dZ = A o (dA - c):
+//   dX_t = sum_j A_tj dH_j + ln2 sum_j dZ_tj P'_j
+//        = Y_t + ln2 (W_t - c_t V_t),   Y = A dH,  V = A P',  W = (A o dA) P'
+//   E    = sum_t dZ_t^T x_t   (weight gradients follow from E by small GEMMs)
+// dm is centred per user (dZ and dX do not change when a constant is added to
+// dA); this keeps W - c V free of a large common term.
+//
+// Two kernels:
+//   sa_bwd_dx_tc_kernel  token-parallel: one CTA per token chunk, all k per
+//     tile in chunks of 64 prototypes.  Per chunk: [Z|G] = X [P'_c;dH_c]^T
+//     (M=128 tokens, N=128), then A and A o dA to SMEM (bf16) and
+//     [V|Y] += A [P'_c|dH_c] (N=256), W += (A o dA) P'_c (N=128), all in TMEM;
+//     c_t accumulates in registers.  Needs no knowledge of c beforehand.
+//   sa_bwd_e_tc_kernel   prototype-slice-parallel: one CTA per (128-prototype
+//     slice, token chunk).  Per tile: [Z|G] (N=256), dZ (bf16, SMEM), then
+//     E_slice += dZ^T X (M=128 prototypes, N=128) in TMEM.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "sa_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace sa {
+
+namespace {
+using namespace tc;
+
+constexpr int TILE = 128, DD = 128;
+constexpr float kLn2f = 0.69314718055994530942f;
+
+template <class F>
+__device__ __forceinline__ void for_each_tile(const int64_t* off, int B, const Chunking& ch, int g,
+                                              F&& f) {
+  const int64_t cb = (int64_t)g * ch.T, ce = min(cb + ch.T, ch.n_total);
+  int t = 0, piece = 0;
+  for (int u = user_of_token(off, B, cb); u < B && off[u] < ce; ++u) {
+    const int64_t pb = max(off[u], cb), pe = min(off[u + 1], ce);
+    if (pb >= pe) continue;
+    for (int64_t tb = pb; tb < pe; tb += TILE, ++t)
+      if (!f(t, piece, u, tb, pe, tb == pb, tb + TILE >= pe)) return;
+    ++piece;
+  }
+}
+
+__device__ __forceinline__ void st_row_k_major(uint32_t tile, int row, int q, uint32_t a,
+                                               uint32_t b, uint32_t c, uint32_t d) {
+  // 16-byte chunk q of `row` in a K-major SW128 tile of 128-byte rows
+  st_shared_v4(tile + row * 128 + ((q ^ (row & 7)) << 4), a, b, c, d);
+}
+
+// ============================================================== dX kernel
+constexpr int KC = 64;                       // prototypes per chunk
+constexpr int DX_NXS = 2, DX_NCS = 2;
+constexpr uint32_t XT_BYTES = 32768;         // [128 tokens x 128] bf16: 2 SW128 halves of 16 KB
+constexpr uint32_t CH_BYTES = 32768;         // [P' h0 | dH h0 | P' h1 | dH h1], 8 KB each
+constexpr uint32_t AT_BYTES = 16384;         // [128 tokens x 64] bf16 K-major SW128
+constexpr uint32_t DX_OFF_X = 0;
+constexpr uint32_t DX_OFF_CH = DX_OFF_X + DX_NXS * XT_BYTES;
+constexpr uint32_t DX_OFF_A = DX_OFF_CH + DX_NCS * CH_BYTES;        // 2 x (A tile, A o dA tile)
+constexpr uint32_t DX_OFF_DM = DX_OFF_A + 2 * 2 * AT_BYTES;
+constexpr uint32_t DX_OFF_BAR = DX_OFF_DM + DX_NCS * KC * 4;
+constexpr uint32_t DX_SMEM = DX_OFF_BAR + 256 + 1024;
+constexpr int DX_THREADS = 192;              // warp 0 TMA, 1 MMA, 2-5 one thread per token
+constexpr uint32_t DX_TM_ZG = 0, DX_TM_VY = 128, DX_TM_W = 384;
+
+struct DxBars {
+  uint64_t x_full[DX_NXS], x_empty[DX_NXS], c_full[DX_NCS], c_empty[DX_NCS];
+  uint64_t zg_full, zg_empty, a_full[2], a_empty[2], acc_full, acc_empty, mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct DxParams {
+  const int64_t* off;
+  int B;
+  Chunking ch;
+  int k;
+  const float* lse2;     // [n] per-token log2-sum-exp
+  const float* dmc;      // [B, k] centred dm
+  __nv_bfloat16* dX;     // [n, d]
+  float* cout;           // [n]
+  int* err;
+};
+
+__global__ void __launch_bounds__(DX_THREADS, 1)
+    sa_bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                        const __grid_constant__ CUtensorMap tmH, DxParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  DxBars* bars = (DxBars*)(smem + DX_OFF_BAR);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int g = blockIdx.x;
+  if (g >= p.ch.G) return;
+  const int nch = p.k / KC;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < DX_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
+    for (int s = 0; s < DX_NCS; ++s) { mbar_init(&bars->c_full[s], 1); mbar_init(&bars->c_empty[s], 1); }
+    mbar_init(&bars->zg_full, 1);
+    mbar_init(&bars->zg_empty, 128);
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->a_full[b], 128); mbar_init(&bars->a_empty[b], 1); }
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, 128);
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmP);
+    prefetch_tensormap(&tmH);
+    int cc = 0, issued_t = 0, issued_c = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int u, int64_t tb, int64_t, bool, bool) {
+      const int s = t % DX_NXS;
+      if (t >= DX_NXS && !mbar_wait(&bars->x_empty[s], ((t / DX_NXS) - 1) & 1, abort, p.err)) return false;
+      mbar_arrive_expect_tx(&bars->x_full[s], XT_BYTES);
+      uint8_t* xd = smem + DX_OFF_X + s * XT_BYTES;
+      tma_load_2d(xd, &tmX, &bars->x_full[s], 0, (int)tb);
+      tma_load_2d(xd + XT_BYTES / 2, &tmX, &bars->x_full[s], 64, (int)tb);
+      issued_t = t + 1;
+      for (int c = 0; c < nch; ++c, ++cc) {
+        const int cs = cc % DX_NCS;
+        if (cc >= DX_NCS && !mbar_wait(&bars->c_empty[cs], ((cc / DX_NCS) - 1) & 1, abort, p.err)) return false;
+        mbar_arrive_expect_tx(&bars->c_full[cs], CH_BYTES + KC * 4);
+        uint8_t* cd = smem + DX_OFF_CH + cs * CH_BYTES;
+        const int prow = c * KC, hrow = (int)((int64_t)u * p.k + c * KC);
+        tma_load_2d(cd, &tmP, &bars->c_full[cs], 0, prow);
+        tma_load_2d(cd + 8192, &tmH, &bars->c_full[cs], 0, hrow);
+        tma_load_2d(cd + 16384, &tmP, &bars->c_full[cs], 64, prow);
+        tma_load_2d(cd + 24576, &tmH, &bars->c_full[cs], 64, hrow);
+        bulk_load(smem + DX_OFF_DM + cs * KC * 4, p.dmc + (int64_t)u * p.k + c * KC, KC * 4, &bars->c_full[cs]);
+        issued_c = cc + 1;
+      }
+      return true;
+    });
+    if (*abort) {
+      for (int t = std::max(0, issued_t - DX_NXS); t < issued_t; ++t)
+        mbar_wait_bounded(&bars->x_full[t % DX_NXS], (t / DX_NXS) & 1);
+      for (int c = std::max(0, issued_c - DX_NCS); c < issued_c; ++c)
+        mbar_wait_bounded(&bars->c_full[c % DX_NCS], (c / DX_NCS) & 1);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t id_zg = idesc_bf16(128, 128, false, false);
+    const uint32_t id_vy = idesc_bf16(128, 256, false, true);
+    const uint32_t id_w = idesc_bf16(128, 128, false, true);
+    int ai = 0;   // global chunk index
+    auto avw = [&](int a, int t, int s, bool first, bool last) -> bool {
+      const int cs = a % DX_NCS, b = a & 1;
+      if (!mbar_wait(&bars->a_full[b], (a >> 1) & 1, abort, p.err)) return false;
+      if (first && t > 0 && !mbar_wait(&bars->acc_empty, (t - 1) & 1, abort, p.err)) return false;
+      tc_fence_after();
+      const uint32_t at = smem_u32(smem + DX_OFF_A + b * 2 * AT_BYTES);
+      const uint32_t adt = at + AT_BYTES;
+      const uint32_t cb = smem_u32(smem + DX_OFF_CH + cs * CH_BYTES);
+#pragma unroll
+      for (int ks = 0; ks < KC / 16; ++ks) {
+        const uint32_t acc = (first && ks == 0) ? 0u : 1u;
+        mma_ss(tmem + DX_TM_VY, smem_desc(at + ks * 32, 16, 1024, SWZ_128B),
+               smem_desc(cb + ks * 2048, 8192, 1024, SWZ_128B), id_vy, acc);
+        mma_ss(tmem + DX_TM_W, smem_desc(adt + ks * 32, 16, 1024, SWZ_128B),
+               smem_desc(cb + ks * 2048, 16384, 1024, SWZ_128B), id_w, acc);
+      }
+      mma_commit(&bars->c_empty[cs]);
+      mma_commit(&bars->a_empty[b]);
+      if (last) {
+        mma_commit(&bars->x_empty[s]);
+        mma_commit(&bars->acc_full);
+      }
+      return true;
+    };
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
+      const int s = t % DX_NXS;
+      if (!mbar_wait(&bars->x_full[s], (t / DX_NXS) & 1, abort, p.err)) return false;
+      const uint32_t xa = smem_u32(smem + DX_OFF_X + s * XT_BYTES);
+      for (int c = 0; c < nch; ++c) {
+        const int a = ai + c, cs = a % DX_NCS;
+        if (!mbar_wait(&bars->c_full[cs], (a / DX_NCS) & 1, abort, p.err)) return false;
+        if (a > 0 && !mbar_wait(&bars->zg_empty, (a - 1) & 1, abort, p.err)) return false;
+        tc_fence_after();
+        const uint32_t cb = smem_u32(smem + DX_OFF_CH + cs * CH_BYTES);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tmem + DX_TM_ZG, smem_desc(xa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B),
+                 smem_desc(cb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B), id_zg,
+                 ks > 0 ? 1u : 0u);
+        mma_commit(&bars->zg_full);
+        if (c > 0 && !avw(a - 1, t, s, c - 1 == 0, false)) return false;
+      }
+      if (!avw(ai + nch - 1, t, s, nch == 1, true)) return false;
+      ai += nch;
+      return true;
+    });
+    mma_commit(&bars->mma_done);
+    mbar_wait_bounded(&bars->mma_done, 0);
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ one thread per token
+    const int q = warp % 4;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    int ai = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t pe, bool, bool) {
+      const bool valid = tb + row < pe;
+      const float l2 = valid ? p.lse2[tb + row] : 0.f;
+      float cacc = 0.f;
+      for (int c = 0; c < nch; ++c) {
+        const int a = ai + c, cs = a % DX_NCS, b = a & 1;
+        if (!mbar_wait(&bars->zg_full, a & 1, abort, p.err)) return false;
+        tc_fence_after();
+        float z[64], gv[64];
+        tmem_ld32(tmem + lane_addr + DX_TM_ZG, z);
+        tmem_ld32(tmem + lane_addr + DX_TM_ZG + 32, z + 32);
+        tmem_ld32(tmem + lane_addr + DX_TM_ZG + 64, gv);
+        tmem_ld32(tmem + lane_addr + DX_TM_ZG + 96, gv + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->zg_empty);
+        if (!mbar_wait(&bars->c_full[cs], (a / DX_NCS) & 1, abort, p.err)) return false;
+        if (a >= 2 && !mbar_wait(&bars->a_empty[b], ((a >> 1) - 1) & 1, abort, p.err)) return false;
+        const float4* dm4 = (const float4*)(smem + DX_OFF_DM + cs * KC * 4);
+        const uint32_t at = smem_u32(smem + DX_OFF_A + b * 2 * AT_BYTES);
+        const uint32_t adt = at + AT_BYTES;
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+          const float4 d0 = dm4[2 * q8], d1 = dm4[2 * q8 + 1];
+          const float dmv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+          float av[8], adv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = q8 * 8 + i;
+            const float A = valid ? ex2(z[j] - l2) : 0.f;
+            const float dA = gv[j] + dmv[i];
+            av[i] = A;
+            adv[i] = A * dA;
+            cacc = fmaf(A, dA, cacc);
+          }
+          st_row_k_major(at, row, q8, pack_bf16x2(av[0], av[1]), pack_bf16x2(av[2], av[3]),
+                         pack_bf16x2(av[4], av[5]), pack_bf16x2(av[6], av[7]));
+          st_row_k_major(adt, row, q8, pack_bf16x2(adv[0], adv[1]), pack_bf16x2(adv[2], adv[3]),
+                         pack_bf16x2(adv[4], adv[5]), pack_bf16x2(adv[6], adv[7]));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars->a_full[b]);
+      }
+      ai += nch;
+      // dX_t = Y + ln2 (W - c V)
+      if (!mbar_wait(&bars->acc_full, t & 1, abort, p.err)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int qb = 0; qb < 4; ++qb) {
+        // columns of d block qb: V at VY + (qb/2)*128 + (qb%2)*32, Y 64 further, W at W + 32 qb
+        const uint32_t vcol = DX_TM_VY + (qb >> 1) * 128 + (qb & 1) * 32;
+        float v[32], y[32], w[32];
+        tmem_ld32(tmem + lane_addr + vcol, v);
+        tmem_ld32(tmem + lane_addr + vcol + 64, y);
+        tmem_ld32(tmem + lane_addr + DX_TM_W + 32 * qb, w);
+        tmem_wait_ld();
+        if (valid) {
+          uint32_t o[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            o[i / 2] = pack_bf16x2(y[i] + kLn2f * (w[i] - cacc * v[i]),
+                                   y[i + 1] + kLn2f * (w[i + 1] - cacc * v[i + 1]));
+          uint4* dst = (uint4*)(p.dX + (tb + row) * DD + 32 * qb);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
+      }
+      if (valid) p.cout[tb + row] = cacc;
+      tc_fence_before();
+      mbar_arrive(&bars->acc_empty);
+      return true;
+    });
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================== E kernel
+constexpr int E_NXS = 2;
+constexpr uint32_t E_OFF_PH = 0;              // [P' h0 | dH h0 | P' h1 | dH h1], 16 KB each
+constexpr uint32_t E_OFF_X = 65536;
+constexpr uint32_t E_OFF_DZ = E_OFF_X + E_NXS * XT_BYTES;   // 2 x [128 protos x 128 tokens] MN-major
+constexpr uint32_t E_OFF_DM = E_OFF_DZ + 2 * 32768;
+constexpr uint32_t E_OFF_BAR = E_OFF_DM + TILE * 4;
+constexpr uint32_t E_SMEM = E_OFF_BAR + 256 + 1024;
+constexpr int E_THREADS = 192;
+constexpr uint32_t E_TM_ZG = 0, E_TM_E = 256;
+
+struct EBars {
+  uint64_t p_full, h_full, h_empty, x_full[E_NXS], x_empty[E_NXS];
+  uint64_t zg_full, zg_empty, dz_full[2], dz_empty[2], e_full, mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct EParams {
+  const int64_t* off;
+  int B;
+  Chunking ch;
+  int k;
+  const float* lse2;
+  const float* cin;      // [n] c_t with the centred dm
+  const float* dmc;      // [B, k]
+  float* Epart;          // [G, k, d]
+  int* err;
+};
+
+__global__ void __launch_bounds__(E_THREADS, 1)
+    sa_bwd_e_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                       const __grid_constant__ CUtensorMap tmH, EParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  EBars* bars = (EBars*)(smem + E_OFF_BAR);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int slices = p.k / TILE;
+  const int sl = blockIdx.x % slices, g = blockIdx.x / slices;
+  if (g >= p.ch.G) return;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->p_full, 1);
+    mbar_init(&bars->h_full, 1);
+    mbar_init(&bars->h_empty, 1 + 128);      // the last zg of a piece, and the threads done with its dm
+    for (int s = 0; s < E_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
+    mbar_init(&bars->zg_full, 1);
+    mbar_init(&bars->zg_empty, 128);
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->dz_full[b], 128); mbar_init(&bars->dz_empty[b], 1); }
+    mbar_init(&bars->e_full, 1);
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmP);
+    prefetch_tensormap(&tmH);
+    mbar_arrive_expect_tx(&bars->p_full, 32768);
+    tma_load_2d(smem + E_OFF_PH, &tmP, &bars->p_full, 0, sl * TILE);
+    tma_load_2d(smem + E_OFF_PH + 32768, &tmP, &bars->p_full, 64, sl * TILE);
+    int issued_t = 0, issued_h = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int u, int64_t tb, int64_t, bool first, bool) {
+      if (first) {
+        if (piece > 0 && !mbar_wait(&bars->h_empty, (piece - 1) & 1, abort, p.err)) return false;
+        mbar_arrive_expect_tx(&bars->h_full, 32768 + TILE * 4);
+        const int hrow = (int)((int64_t)u * p.k + sl * TILE);
+        tma_load_2d(smem + E_OFF_PH + 16384, &tmH, &bars->h_full, 0, hrow);
+        tma_load_2d(smem + E_OFF_PH + 49152, &tmH, &bars->h_full, 64, hrow);
+        bulk_load(smem + E_OFF_DM, p.dmc + (int64_t)u * p.k + sl * TILE, TILE * 4, &bars->h_full);
+        issued_h = piece + 1;
+      }
+      const int s = t % E_NXS;
+      if (t >= E_NXS && !mbar_wait(&bars->x_empty[s], ((t / E_NXS) - 1) & 1, abort, p.err)) return false;
+      mbar_arrive_expect_tx(&bars->x_full[s], XT_BYTES);
+      uint8_t* xd = smem + E_OFF_X + s * XT_BYTES;
+      tma_load_2d(xd, &tmX, &bars->x_full[s], 0, (int)tb);
+      tma_load_2d(xd + XT_BYTES / 2, &tmX, &bars->x_full[s], 64, (int)tb);
+      issued_t = t + 1;
+      return true;
+    });
+    if (*abort) {
+      mbar_wait_bounded(&bars->p_full, 0);
+      if (issued_h > 0) mbar_wait_bounded(&bars->h_full, (issued_h - 1) & 1);
+      for (int t = std::max(0, issued_t - E_NXS); t < issued_t; ++t)
+        mbar_wait_bounded(&bars->x_full[t % E_NXS], (t / E_NXS) & 1);
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t id_zg = idesc_bf16(128, 256, false, false);
+    const uint32_t id_e = idesc_bf16(128, 128, true, true);
+    const uint32_t ph = smem_u32(smem + E_OFF_PH);
+    int prev_t = -1, prev_s = 0;
+    auto emma = [&](int t, int s) -> bool {
+      const int b = t & 1;
+      if (!mbar_wait(&bars->dz_full[b], (t >> 1) & 1, abort, p.err)) return false;
+      tc_fence_after();
+      const uint32_t dz = smem_u32(smem + E_OFF_DZ + b * 32768);
+      const uint32_t xa = smem_u32(smem + E_OFF_X + s * XT_BYTES);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ss(tmem + E_TM_E, smem_desc(dz + ks * 2048, 16384, 1024, SWZ_128B),
+               smem_desc(xa + ks * 2048, 16384, 1024, SWZ_128B), id_e, (t > 0 || ks > 0) ? 1u : 0u);
+      mma_commit(&bars->dz_empty[b]);
+      mma_commit(&bars->x_empty[s]);
+      return true;
+    };
+    bool ok = mbar_wait(&bars->p_full, 0, abort, p.err);
+    if (ok) {
+      for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t, int64_t, bool first, bool last) {
+        const int s = t % E_NXS;
+        if (first && !mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return false;
+        if (!mbar_wait(&bars->x_full[s], (t / E_NXS) & 1, abort, p.err)) return false;
+        if (t > 0 && !mbar_wait(&bars->zg_empty, (t - 1) & 1, abort, p.err)) return false;
+        tc_fence_after();
+        const uint32_t xa = smem_u32(smem + E_OFF_X + s * XT_BYTES);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tmem + E_TM_ZG, smem_desc(xa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B),
+                 smem_desc(ph + (ks >> 2) * 32768 + (ks & 3) * 32, 16, 1024, SWZ_128B), id_zg,
+                 ks > 0 ? 1u : 0u);
+        mma_commit(&bars->zg_full);
+        if (last) mma_commit(&bars->h_empty);
+        if (prev_t >= 0 && !emma(prev_t, prev_s)) return false;
+        prev_t = t;
+        prev_s = s;
+        return true;
+      });
+      if (prev_t >= 0 && !*abort && emma(prev_t, prev_s)) mma_commit(&bars->e_full);
+    }
+    mma_commit(&bars->mma_done);
+    mbar_wait_bounded(&bars->mma_done, 0);
+  } else if (warp >= 2) {
+    const int q = warp % 4;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    bool ok = true;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t tb, int64_t pe, bool first, bool last) {
+      const bool valid = tb + row < pe;
+      const float l2 = valid ? p.lse2[tb + row] : 0.f;
+      const float ct = valid ? p.cin[tb + row] : 0.f;
+      if (first && !mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return ok = false;
+      if (!mbar_wait(&bars->zg_full, t & 1, abort, p.err)) return ok = false;
+      tc_fence_after();
+      const int b = t & 1;
+      if (t >= 2 && !mbar_wait(&bars->dz_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return ok = false;
+      const uint32_t dz = smem_u32(smem + E_OFF_DZ + b * 32768) + row * 128;
+      const float4* dm4 = (const float4*)(smem + E_OFF_DM);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float z[64], gv[64];
+        tmem_ld32(tmem + lane_addr + E_TM_ZG + 64 * h, z);
+        tmem_ld32(tmem + lane_addr + E_TM_ZG + 64 * h + 32, z + 32);
+        tmem_ld32(tmem + lane_addr + E_TM_ZG + 128 + 64 * h, gv);
+        tmem_ld32(tmem + lane_addr + E_TM_ZG + 128 + 64 * h + 32, gv + 32);
+        tmem_wait_ld();
+        if (h == 1) {
+          tc_fence_before();
+          mbar_arrive(&bars->zg_empty);
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const float4 d0 = dm4[16 * h + 2 * c8], d1 = dm4[16 * h + 2 * c8 + 1];
+          const float dmv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+          float dzv[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = c8 * 8 + i;
+            const float A = valid ? ex2(z[j] - l2) : 0.f;
+            dzv[i] = A * (gv[j] + dmv[i] - ct);
+          }
+          // MN-major SW128 A operand of E += dZ^T X: M-block h, token row `row`
+          st_shared_v4(dz + h * 16384 + ((c8 ^ (row & 7)) << 4), pack_bf16x2(dzv[0], dzv[1]),
+                       pack_bf16x2(dzv[2], dzv[3]), pack_bf16x2(dzv[4], dzv[5]),
+                       pack_bf16x2(dzv[6], dzv[7]));
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->dz_full[b]);
+      if (last) mbar_arrive(&bars->h_empty);   // this piece's dm is no longer read
+      return true;
+    });
+    if (ok && mbar_wait(&bars->e_full, 0, abort, p.err)) {
+      tc_fence_after();
+      float* dst = p.Epart + ((int64_t)g * p.k + sl * TILE + row) * DD;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_addr + E_TM_E + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *(float4*)(dst + 32 * c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ============================================================== host side
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* q = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      fn = (EncodeFn)q;
+  });
+  return fn;
+}
+
+sa_status map_rows(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {DD, rows};
+  cuuint64_t strides[1] = {DD * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return SA_OK;
+}
+
+// dmc[u, j] = dm[u, j] - mean_j dm[u, :]
+__global__ void center_rows_kernel(const float* __restrict__ dm, int k, float* __restrict__ dmc) {
+  __shared__ float part[256];
+  const int u = blockIdx.x;
+  float s = 0.f;
+  for (int j = threadIdx.x; j < k; j += 256) s += dm[(int64_t)u * k + j];
+  part[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) part[threadIdx.x] += part[threadIdx.x + w];
+    __syncthreads();
+  }
+  const float mean = part[0] / (float)k;
+  for (int j = threadIdx.x; j < k; j += 256) dmc[(int64_t)u * k + j] = dm[(int64_t)u * k + j] - mean;
+}
+}  // namespace
+
+bool sa_bwd_tc_supported(sa_dtype x_dtype, int k, int d) {
+  return x_dtype == SA_BF16 && d == DD && k % TILE == 0 && k >= TILE && k <= 4096;
+}
+
+int sa_bwd_tc_dx_chunks() { return device_info().sm_count; }
+int sa_bwd_tc_e_chunks(int k) { return std::max(1, device_info().sm_count / (k / TILE)); }
+
+sa_status sa_bwd_tc_run(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st) {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(sa_bwd_dx_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DX_SMEM);
+    cudaFuncSetAttribute(sa_bwd_e_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, E_SMEM);
+  });
+  if (a.n_total >= (1LL << 31) || (int64_t)a.B * a.k >= (1LL << 31))
+    return fail(SA_ERR_UNSUPPORTED, "row counts must be < 2^31");
+  SA_TIMED("center_rows_kernel", st, (center_rows_kernel<<<a.B, 256, 0, st>>>(w.dm, a.k, w.dmc)));
+  CUtensorMap tmX, tmP64, tmH64, tmP128, tmH128;
+  sa_status s;
+  if ((s = map_rows(&tmX, a.X, (uint64_t)a.n_total, 128)) != SA_OK) return s;
+  if ((s = map_rows(&tmP64, w.Pb, (uint64_t)a.k, 64)) != SA_OK) return s;
+  if ((s = map_rows(&tmH64, w.dHb, (uint64_t)a.B * a.k, 64)) != SA_OK) return s;
+  if ((s = map_rows(&tmP128, w.Pb, (uint64_t)a.k, 128)) != SA_OK) return s;
+  if ((s = map_rows(&tmH128, w.dHb, (uint64_t)a.B * a.k, 128)) != SA_OK) return s;
+  DxParams dp{a.off_dev, a.B, w.ch, a.k, w.lse, w.dmc, (__nv_bfloat16*)a.dX, w.cbuf, device_status_word()};
+  SA_TIMED("sa_bwd_dx_tc_kernel", st,
+           (sa_bwd_dx_tc_kernel<<<w.ch.G, DX_THREADS, DX_SMEM, st>>>(tmX, tmP64, tmH64, dp)));
+  EParams ep{a.off_dev, a.B, w.chE, a.k, w.lse, w.cbuf, w.dmc, w.Epart, device_status_word()};
+  SA_TIMED("sa_bwd_e_tc_kernel", st,
+           (sa_bwd_e_tc_kernel<<<w.chE.G * (a.k / TILE), E_THREADS, E_SMEM, st>>>(tmX, tmP128, tmH128, ep)));
+  return SA_OK;
+}
+
+}  // namespace sa

@@ -48,7 +48,9 @@ struct SaBwdWork {
   float* dHh;           // [B, k, d]  dS W_V^T
   float* Hhat;          // [B, k, d]
   float* dH;            // [B, k, d]
+  __nv_bfloat16* dHb;   // [B, k, d]  bf16 copy (tensor-core path)
   float* dm;            // [B, k]
+  float* dmc;           // [B, k]     dm centred per user (tensor-core path)
   float* Epart;         // [chE.G, k, d]
   float* E;             // [k, d]
   float* dQ;            // [k, d]
@@ -59,8 +61,14 @@ sa_status sa_fold(int k, int d, const float* P, const float* W_Q, const float* W
                   float* Pf, __nv_bfloat16* Pb, cudaStream_t st);
 sa_status sa_simt_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
 sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
-sa_status sa_simt_backward(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st);
+sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaStream_t st);
 sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st);
+
+// Tensor-core backward (sa_bwd_tc.cu).
+bool sa_bwd_tc_supported(sa_dtype x_dtype, int k, int d);
+int sa_bwd_tc_dx_chunks();
+int sa_bwd_tc_e_chunks(int k);
+sa_status sa_bwd_tc_run(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st);
 
 // Tensor-core forward (sa_tc.cu).
 bool sa_tc_supported(sa_dtype x_dtype, int k, int d);

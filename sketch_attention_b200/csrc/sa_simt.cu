@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(256) sa_reduce_kernel(
 __global__ void __launch_bounds__(256) sa_bwd_prologue_kernel(
     int rows, int D, float eps, const float* __restrict__ H, const float* __restrict__ mass,
     const float* __restrict__ dHh, const float* __restrict__ dmass, float* __restrict__ Hhat,
-    float* __restrict__ dH, float* __restrict__ dm) {
+    float* __restrict__ dH, __nv_bfloat16* __restrict__ dHb, float* __restrict__ dm) {
   const int warp = (blockIdx.x * 256 + threadIdx.x) / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
   const float den = mass[warp] + eps;
@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(256) sa_bwd_prologue_kernel(
     const float hh = H[o] * inv;
     Hhat[o] = hh;
     dH[o] = dHh[o] * inv;
+    if (dHb) dHb[o] = __float2bfloat16_rn(dHh[o] * inv);
     dot = fmaf(dHh[o], hh, dot);
   }
 #pragma unroll
@@ -445,17 +446,6 @@ sa_status launch_simt_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream
 
 template <class XT, int D>
 sa_status launch_simt_backward(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st) {
-  const int64_t N = a.n_total;
-  if (N <= 0) return SA_OK;
-  if (a.lse_in) {
-    SA_TIMED("lse_to_log2_kernel", st,
-             (lse_to_log2_kernel<<<(unsigned)std::min<int64_t>((N + 255) / 256, 8192), 256, 0, st>>>(
-                 a.lse_in, N, w.lse)));
-  } else {
-    SA_TIMED("sa_lse_kernel", st,
-             (sa_lse_kernel<XT, D><<<(unsigned)((N + 127) / 128), 128, 0, st>>>(
-                 (const XT*)a.X, N, w.Pf, a.k, w.lse, nullptr)));
-  }
   SA_TIMED("sa_bwd_token_kernel", st,
            (sa_bwd_token_kernel<XT, D><<<w.ch.G, 256, 0, st>>>(
                (const XT*)a.X, a.off_dev, a.B, w.ch, w.Pf, a.k, w.lse, w.dH, w.dm, w.cbuf,
@@ -465,6 +455,22 @@ sa_status launch_simt_backward(const SaBwdArgs& a, const SaBwdWork& w, cudaStrea
            (sa_bwd_E_kernel<XT, D><<<grid, 256, 0, st>>>((const XT*)a.X, a.off_dev, a.B, w.chE,
                                                         w.Pf, a.k, w.lse, w.dH, w.dm, w.cbuf,
                                                         w.Epart)));
+  return SA_OK;
+}
+
+// lse (base 2) of every token: converted from the caller's saved lse, or recomputed.
+template <class XT, int D>
+sa_status backward_lse(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st) {
+  const int64_t N = a.n_total;
+  if (a.lse_in) {
+    SA_TIMED("lse_to_log2_kernel", st,
+             (lse_to_log2_kernel<<<(unsigned)std::min<int64_t>((N + 255) / 256, 8192), 256, 0, st>>>(
+                 a.lse_in, N, w.lse)));
+  } else {
+    SA_TIMED("sa_lse_kernel", st,
+             (sa_lse_kernel<XT, D><<<(unsigned)((N + 127) / 128), 128, 0, st>>>(
+                 (const XT*)a.X, N, w.Pf, a.k, w.lse, nullptr)));
+  }
   return SA_OK;
 }
 }  // namespace
@@ -514,7 +520,7 @@ sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStre
   return gemm(g, st);
 }
 
-sa_status sa_simt_backward(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st) {
+sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaStream_t st) {
   const int rows = a.B * a.k;
   const int D = a.d;
   // dHh = dS W_V^T
@@ -527,7 +533,8 @@ sa_status sa_simt_backward(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t 
   if (s != SA_OK) return s;
   SA_TIMED("sa_bwd_prologue_kernel", st,
            (sa_bwd_prologue_kernel<<<(rows * 32 + 255) / 256, 256, 0, st>>>(
-               rows, D, a.eps, a.H, a.mass, w.dHh, a.dmass, w.Hhat, w.dH, w.dm)));
+               rows, D, a.eps, a.H, a.mass, w.dHh, a.dmass, w.Hhat, w.dH, tc ? w.dHb : nullptr,
+               w.dm)));
   // dW_V = sum_u Hh_u^T dS_u
   Gemm gv;
   gv.M = D; gv.N = D; gv.K = rows;
@@ -537,8 +544,12 @@ sa_status sa_simt_backward(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t 
   if ((s = gemm(gv, st)) != SA_OK) return s;
   if (a.n_total > 0) {
     const bool bf = a.x_dtype == SA_BF16;
-    if (D == 64) s = bf ? launch_simt_backward<__nv_bfloat16, 64>(a, w, st)
-                        : launch_simt_backward<float, 64>(a, w, st);
+    if (D == 64) s = bf ? backward_lse<__nv_bfloat16, 64>(a, w, st) : backward_lse<float, 64>(a, w, st);
+    else s = bf ? backward_lse<__nv_bfloat16, 128>(a, w, st) : backward_lse<float, 128>(a, w, st);
+    if (s != SA_OK) return s;
+    if (tc) s = sa_bwd_tc_run(a, w, st);
+    else if (D == 64) s = bf ? launch_simt_backward<__nv_bfloat16, 64>(a, w, st)
+                             : launch_simt_backward<float, 64>(a, w, st);
     else s = bf ? launch_simt_backward<__nv_bfloat16, 128>(a, w, st)
                 : launch_simt_backward<float, 128>(a, w, st);
     if (s != SA_OK) return s;

@@ -92,7 +92,7 @@ __device__ __forceinline__ void for_each_tile(const Params& p, int g, F&& f) {
   }
 }
 
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(THREADS, 1)
     sa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmP, Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -235,16 +235,17 @@ __global__ void __maxnreg__(200)
           if (!mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort, p.err)) return false;
           tc_fence_after();
           // Two halves of 64 columns; each half is exponentiated against the
-          // running maximum at that point (mh[h]); the exponentials stay fp32
-          // so the probabilities are rounded to bf16 once.
-          float e[128];
+          // running maximum at that point (mh[h]).  The fp32 exponentials are
+          // parked in the logits' own TMEM columns until the cluster-wide
+          // normaliser is known, so the probabilities are rounded to bf16 once.
+          const uint32_t sbuf = tmem + lane_addr + (b ? TM_S1 : TM_S0);
           float mh[2];
           float m = -__builtin_huge_valf(), s = 0.f;
-#pragma unroll
+#pragma unroll 1
           for (int h = 0; h < 2; ++h) {
-            float* z = e + 64 * h;
-            tmem_ld32(tmem + lane_addr + (b ? TM_S1 : TM_S0) + 64 * h, z);
-            tmem_ld32(tmem + lane_addr + (b ? TM_S1 : TM_S0) + 64 * h + 32, z + 32);
+            float z[64];
+            tmem_ld32(sbuf + 64 * h, z);
+            tmem_ld32(sbuf + 64 * h + 32, z + 32);
             tmem_wait_ld();
             float cm = z[0];
 #pragma unroll
@@ -252,13 +253,16 @@ __global__ void __maxnreg__(200)
             const float mn = fmaxf(m, cm);
             s *= ex2(m - mn);
             m = mn;
-            mh[h] = mn;
+            if (h == 0) mh[0] = mn; else mh[1] = mn;
 #pragma unroll
             for (int j = 0; j < 64; ++j) {
               z[j] = ex2(z[j] - mn);
               s += z[j];
             }
+            tmem_st32f(sbuf + 64 * h, z);
+            tmem_st32f(sbuf + 64 * h + 32, z + 32);
           }
+          tmem_wait_st();
           const float l = valid ? m + lg2(s) : -__builtin_huge_valf();
           // send this CTA's log2-sum-exp of every token to every CTA of the cluster
           float* st = stage + ((t >> 1) & 1) * TILE;
@@ -290,12 +294,16 @@ __global__ void __maxnreg__(200)
           // probabilities p[t, j] = e_j r as bf16 into the MN-major SW128 A tile of MMA2
           if (t >= 2 && !mbar_wait(&bars->p_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return false;
           const uint32_t pa = smem_u32(smem + OFF_P + b * 32768) + row * 128;
-#pragma unroll
+#pragma unroll 1
           for (int blk = 0; blk < 2; ++blk) {
-            const float r = rh[blk];
+            const float r = blk == 0 ? rh[0] : rh[1];
+            float e[64];
+            tmem_ld32(sbuf + 64 * blk, e);
+            tmem_ld32(sbuf + 64 * blk + 32, e + 32);
+            tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
-              const float* q8 = e + blk * 64 + c * 8;
+              const float* q8 = e + c * 8;
               st_shared_v4(pa + blk * 16384 + ((c ^ (row & 7)) << 4),
                            pack_bf16x2(q8[0] * r, q8[1] * r), pack_bf16x2(q8[2] * r, q8[3] * r),
                            pack_bf16x2(q8[4] * r, q8[5] * r), pack_bf16x2(q8[6] * r, q8[7] * r));
