@@ -210,12 +210,14 @@ size_t layout_bwd(void* base, int B, int64_t n, int k, int d, sa_dtype dt, SaBwd
   v.Hhat = c.take<float>((size_t)B * k * d);
   v.dH = c.take<float>((size_t)B * k * d);
   v.dHb = tc ? c.take<__nv_bfloat16>((size_t)B * k * d) : nullptr;
+  v.dHlo = tc ? c.take<__nv_bfloat16>((size_t)B * k * d) : nullptr;
   v.dm = c.take<float>((size_t)B * k);
   v.dmc = tc ? c.take<float>((size_t)B * k) : nullptr;
   v.Epart = c.take<float>((size_t)std::max(chE.G, 1) * k * d);
   v.E = c.take<float>((size_t)k * d);
   v.dQ = c.take<float>((size_t)k * d);
   v.Q = c.take<float>((size_t)k * d);
+  v.gsplit = c.take<float>((size_t)kMaxSplit * d * d);
   if (w) *w = v;
   return c.bytes();
 }

@@ -18,7 +18,15 @@ struct Gemm {
   float alpha = 1.f;
   int batch = 1;
   int64_t sA = 0, sB = 0, sC = 0, sC16 = 0, sCin = 0;                // batch strides
+  // split-K: split_k CTAs share one output tile, each summing a slice of K
+  // into split_ws ([batch * split_k, M, N] fp32); a second kernel adds the
+  // slices in a fixed order and applies alpha, bias and Cin.
+  int split_k = 1;
+  float* split_ws = nullptr;
 };
+
+// Split count for a GEMM with a long K and few output tiles (1 = no split).
+int gemm_split_for(int M, int N, int K, int max_split);
 
 sa_status gemm(const Gemm& g, cudaStream_t stream);
 

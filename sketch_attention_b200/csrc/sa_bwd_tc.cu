@@ -15,7 +15,9 @@
 //     tile in chunks of 64 prototypes.  Per chunk: [Z|G] = X [P'_c;dH_c]^T
 //     (M=128 tokens, N=128), then A and A o dA to SMEM (bf16) and
 //     [V|Y] += A [P'_c|dH_c] (N=256), W += (A o dA) P'_c (N=128), all in TMEM;
-//     c_t accumulates in registers.  Needs no knowledge of c beforehand.
+//     Y also takes A times the bf16 residual of dH (dH = dH_hi + dH_lo), so
+//     only A's rounding is left in Y.  c_t accumulates in registers.  Needs
+//     no knowledge of c beforehand.
 //   sa_bwd_e_tc_kernel   prototype-slice-parallel: one CTA per (128-prototype
 //     slice, token chunk).  Per tile: [Z|G] (N=256), dZ (bf16, SMEM), then
 //     E_slice += dZ^T X (M=128 prototypes, N=128) in TMEM.
@@ -58,7 +60,7 @@ __device__ __forceinline__ void st_row_k_major(uint32_t tile, int row, int q, ui
 constexpr int KC = 64;                       // prototypes per chunk
 constexpr int DX_NXS = 2, DX_NCS = 2;
 constexpr uint32_t XT_BYTES = 32768;         // [128 tokens x 128] bf16: 2 SW128 halves of 16 KB
-constexpr uint32_t CH_BYTES = 32768;         // [P' h0 | dH h0 | P' h1 | dH h1], 8 KB each
+constexpr uint32_t CH_BYTES = 49152;         // [P' h0 | dH h0 | P' h1 | dH h1 | dHlo h0 | dHlo h1], 8 KB each
 constexpr uint32_t AT_BYTES = 16384;         // [128 tokens x 64] bf16 K-major SW128
 constexpr uint32_t DX_OFF_X = 0;
 constexpr uint32_t DX_OFF_CH = DX_OFF_X + DX_NXS * XT_BYTES;
@@ -90,7 +92,8 @@ struct DxParams {
 
 __global__ void __launch_bounds__(DX_THREADS, 1)
     sa_bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
-                        const __grid_constant__ CUtensorMap tmH, DxParams p) {
+                        const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmL,
+                        DxParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   DxBars* bars = (DxBars*)(smem + DX_OFF_BAR);
@@ -126,6 +129,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     prefetch_tensormap(&tmX);
     prefetch_tensormap(&tmP);
     prefetch_tensormap(&tmH);
+    prefetch_tensormap(&tmL);
     int cc = 0, issued_t = 0, issued_c = 0;
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int u, int64_t tb, int64_t, bool, bool) {
       const int s = t % DX_NXS;
@@ -145,6 +149,8 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
         tma_load_2d(cd + 8192, &tmH, &bars->c_full[cs], 0, hrow);
         tma_load_2d(cd + 16384, &tmP, &bars->c_full[cs], 64, prow);
         tma_load_2d(cd + 24576, &tmH, &bars->c_full[cs], 64, hrow);
+        tma_load_2d(cd + 32768, &tmL, &bars->c_full[cs], 0, hrow);
+        tma_load_2d(cd + 40960, &tmL, &bars->c_full[cs], 64, hrow);
         bulk_load(smem + DX_OFF_DM + cs * KC * 4, p.dmc + (int64_t)u * p.k + c * KC, KC * 4, &bars->c_full[cs]);
         issued_c = cc + 1;
       }
@@ -161,6 +167,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     const uint32_t id_zg = idesc_bf16(128, 128, false, false);
     const uint32_t id_vy = idesc_bf16(128, 256, false, true);
     const uint32_t id_w = idesc_bf16(128, 128, false, true);
+    const uint32_t id_lo = idesc_bf16(128, 64, false, true);
     int ai = 0;   // global chunk index
     auto avw = [&](int a, int t, int s, bool first, bool last) -> bool {
       const int cs = a % DX_NCS, b = a & 1;
@@ -177,6 +184,11 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
                smem_desc(cb + ks * 2048, 8192, 1024, SWZ_128B), id_vy, acc);
         mma_ss(tmem + DX_TM_W, smem_desc(adt + ks * 32, 16, 1024, SWZ_128B),
                smem_desc(cb + ks * 2048, 16384, 1024, SWZ_128B), id_w, acc);
+        // Y += A dH_lo: the bf16 residual of dH, so dH is carried to ~16 bits
+        mma_ss(tmem + DX_TM_VY + 64, smem_desc(at + ks * 32, 16, 1024, SWZ_128B),
+               smem_desc(cb + 32768 + ks * 2048, 8192, 1024, SWZ_128B), id_lo, 1u);
+        mma_ss(tmem + DX_TM_VY + 192, smem_desc(at + ks * 32, 16, 1024, SWZ_128B),
+               smem_desc(cb + 40960 + ks * 2048, 8192, 1024, SWZ_128B), id_lo, 1u);
       }
       mma_commit(&bars->c_empty[cs]);
       mma_commit(&bars->a_empty[b]);
@@ -583,11 +595,13 @@ sa_status sa_bwd_tc_run(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st)
   if ((s = map_rows(&tmX, a.X, (uint64_t)a.n_total, 128)) != SA_OK) return s;
   if ((s = map_rows(&tmP64, w.Pb, (uint64_t)a.k, 64)) != SA_OK) return s;
   if ((s = map_rows(&tmH64, w.dHb, (uint64_t)a.B * a.k, 64)) != SA_OK) return s;
+  CUtensorMap tmL64;
+  if ((s = map_rows(&tmL64, w.dHlo, (uint64_t)a.B * a.k, 64)) != SA_OK) return s;
   if ((s = map_rows(&tmP128, w.Pb, (uint64_t)a.k, 128)) != SA_OK) return s;
   if ((s = map_rows(&tmH128, w.dHb, (uint64_t)a.B * a.k, 128)) != SA_OK) return s;
   DxParams dp{a.off_dev, a.B, w.ch, a.k, w.lse, w.dmc, (__nv_bfloat16*)a.dX, w.cbuf, device_status_word()};
   SA_TIMED("sa_bwd_dx_tc_kernel", st,
-           (sa_bwd_dx_tc_kernel<<<w.ch.G, DX_THREADS, DX_SMEM, st>>>(tmX, tmP64, tmH64, dp)));
+           (sa_bwd_dx_tc_kernel<<<w.ch.G, DX_THREADS, DX_SMEM, st>>>(tmX, tmP64, tmH64, tmL64, dp)));
   EParams ep{a.off_dev, a.B, w.chE, a.k, w.lse, w.cbuf, w.dmc, w.Epart, device_status_word()};
   SA_TIMED("sa_bwd_e_tc_kernel", st,
            (sa_bwd_e_tc_kernel<<<w.chE.G * (a.k / TILE), E_THREADS, E_SMEM, st>>>(tmX, tmP128, tmH128, ep)));

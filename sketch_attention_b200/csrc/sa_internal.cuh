@@ -49,13 +49,16 @@ struct SaBwdWork {
   float* Hhat;          // [B, k, d]
   float* dH;            // [B, k, d]
   __nv_bfloat16* dHb;   // [B, k, d]  bf16 copy (tensor-core path)
+  __nv_bfloat16* dHlo;  // [B, k, d]  bf16 residual dH - dHb (tensor-core path)
   float* dm;            // [B, k]
   float* dmc;           // [B, k]     dm centred per user (tensor-core path)
   float* Epart;         // [chE.G, k, d]
   float* E;             // [k, d]
   float* dQ;            // [k, d]
   float* Q;             // [k, d]
+  float* gsplit;        // [kMaxSplit, d, d] split-K partials of the weight-gradient GEMMs
 };
+constexpr int kMaxSplit = 64;
 
 sa_status sa_fold(int k, int d, const float* P, const float* W_Q, const float* W_K, float* T,
                   float* Pf, __nv_bfloat16* Pb, cudaStream_t st);

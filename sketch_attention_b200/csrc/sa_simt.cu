@@ -202,7 +202,8 @@ __global__ void __launch_bounds__(256) sa_reduce_kernel(
 __global__ void __launch_bounds__(256) sa_bwd_prologue_kernel(
     int rows, int D, float eps, const float* __restrict__ H, const float* __restrict__ mass,
     const float* __restrict__ dHh, const float* __restrict__ dmass, float* __restrict__ Hhat,
-    float* __restrict__ dH, __nv_bfloat16* __restrict__ dHb, float* __restrict__ dm) {
+    float* __restrict__ dH, __nv_bfloat16* __restrict__ dHb, __nv_bfloat16* __restrict__ dHlo,
+    float* __restrict__ dm) {
   const int warp = (blockIdx.x * 256 + threadIdx.x) / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
   const float den = mass[warp] + eps;
@@ -213,7 +214,12 @@ __global__ void __launch_bounds__(256) sa_bwd_prologue_kernel(
     const float hh = H[o] * inv;
     Hhat[o] = hh;
     dH[o] = dHh[o] * inv;
-    if (dHb) dHb[o] = __float2bfloat16_rn(dHh[o] * inv);
+    if (dHb) {
+      const float v = dHh[o] * inv;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      dHb[o] = hi;
+      dHlo[o] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    }
     dot = fmaf(dHh[o], hh, dot);
   }
 #pragma unroll
@@ -534,13 +540,15 @@ sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaS
   SA_TIMED("sa_bwd_prologue_kernel", st,
            (sa_bwd_prologue_kernel<<<(rows * 32 + 255) / 256, 256, 0, st>>>(
                rows, D, a.eps, a.H, a.mass, w.dHh, a.dmass, w.Hhat, w.dH, tc ? w.dHb : nullptr,
-               w.dm)));
+               tc ? w.dHlo : nullptr, w.dm)));
   // dW_V = sum_u Hh_u^T dS_u
   Gemm gv;
   gv.M = D; gv.N = D; gv.K = rows;
   gv.A = w.Hhat; gv.lda = D; gv.transA = true;
   gv.B = a.dS; gv.ldb = D;
   gv.C = a.dW_V; gv.ldc = D;
+  gv.split_k = gemm_split_for(D, D, rows, kMaxSplit);
+  gv.split_ws = w.gsplit;
   if ((s = gemm(gv, st)) != SA_OK) return s;
   if (a.n_total > 0) {
     const bool bf = a.x_dtype == SA_BF16;
@@ -583,6 +591,8 @@ sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream
   Gemm g3;
   g3.M = D; g3.N = D; g3.K = k;
   g3.A = a.P; g3.lda = D; g3.transA = true; g3.B = w.dQ; g3.ldb = D; g3.C = a.dW_Q; g3.ldc = D;
+  g3.split_k = gemm_split_for(D, D, k, kMaxSplit);
+  g3.split_ws = w.gsplit;
   if ((s = gemm(g3, st)) != SA_OK) return s;
   // Q = P W_Q;  dW_K = E^T Q / sqrt(d)
   Gemm g4;
@@ -593,6 +603,8 @@ sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream
   g5.M = D; g5.N = D; g5.K = k;
   g5.A = w.E; g5.lda = D; g5.transA = true; g5.B = w.Q; g5.ldb = D; g5.C = a.dW_K; g5.ldc = D;
   g5.alpha = rs;
+  g5.split_k = gemm_split_for(D, D, k, kMaxSplit);
+  g5.split_ws = w.gsplit;
   return gemm(g5, st);
 }
 
