@@ -62,7 +62,7 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                 "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -180,6 +180,39 @@ class TrainStepRunner:
 
 # Per-kernel algorithmic work (flops) per launch, for the roofline of the
 # dominant kernel.  tokens = history tokens of the call.
+KERNEL_SOURCES = {
+    "sa_fwd_tc_kernel": "sa_tc.cu", "sa_bwd_dx_tc_kernel": "sa_bwd_tc.cu",
+    "sa_bwd_e_tc_kernel": "sa_bwd_tc.cu", "stca_attn_tc_kernel": "stca_tc.cu",
+}
+
+
+def source_digest(kernel):
+    import hashlib
+    src = KERNEL_SOURCES.get(kernel)
+    if not src:
+        return None
+    path = os.path.join(ROOT, "sketch_attention_b200", "csrc", src)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(kernel, units):
+    """DRAM bytes of one launch of `kernel` over `units` tokens, scaled from the
+    committed ncu record (profiles/dram_traffic.txt: kernel, bytes per token,
+    source digest); None when there is no record or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for line in f:
+            parts = line.split("#", 1)[0].split()
+            if len(parts) >= 3 and parts[0] == kernel:
+                if parts[2] != source_digest(kernel):
+                    return None
+                return float(parts[1]) * units
+    return None
+
+
 def kernel_model(name, w):
     k, d = w.sa.k, w.sa.d
     n = w.sa.n_total
@@ -218,7 +251,7 @@ def run_ours(args, rank, world, device):
     sab.load()
     from sa_inputs import TRAIN_STEP_WORKLOAD, train_step_workload
     t0 = time.time()
-    w = train_step_workload()
+    w = train_step_workload(users=args.users)
     gen_s = time.time() - t0
     R = TrainStepRunner(w, device, world)
     peaks, peaks_src = load_peaks()
@@ -313,7 +346,8 @@ def run_ours(args, rank, world, device):
                 peak = SMS * FP32_LANES * 2 * mhz * 1e6 / 1e12
                 peak_note = f"fp32 FMA: {SMS} SMs x {FP32_LANES} lanes x 2 x {mhz:.0f} MHz"
             roof = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak,
-                    "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                    "unit": "TFLOP/s", "frac": achieved / peak,
+                    "traffic": measured_traffic(name, w.sa.n_total),
                     "peak_source": peak_note, "avg_launch_ms": tot_ms / cnt,
                     "launches": cnt, "share_of_step": tot_ms / (ms * args.steps)}
     kernels = {n: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
@@ -493,7 +527,7 @@ def run_component(args, rank, world, device):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")

@@ -177,7 +177,7 @@ def test_sa_backward_workload5_sampled(lib, workload_cache):
         gu = lib.sa_backward(dv["X"][lo:hi], [0, hi - lo], dv["P"], dv["W_Q"], dv["W_K"],
                              dv["W_V"], p.eps, fwd["H"][u:u + 1].contiguous(),
                              fwd["mass"][u:u + 1].contiguous(), dS[u:u + 1].contiguous(), None,
-                             fwd["lse"][lo:hi])
+                             fwd["lse"][lo:hi].clone())   # the ABI wants 16-byte aligned buffers
         for n in names:
             total[n] += gu[n].double()
         if u in (0, p.B - 1):
