@@ -104,6 +104,30 @@ sa_status sa_forward(const void* X, sa_dtype x_dtype,
                      float* S, float* mass, float* H, void* S_bf16, float* lse,
                      void* workspace, size_t ws_bytes, sa_stream_t stream);
 
+/*
+ * sa_forward_noalloc -- sa_forward for callers that cannot allocate device
+ * memory (code running inside a memory pool it does not own, plugins whose
+ * host forbids device allocations, work recorded once and replayed).  The
+ * paper has no counterpart: this is an interface variant of sa_forward, with
+ * the same inputs, outputs and results up to rounding, and no workspace.
+ * Scratch lives in a fixed 8 MiB device array inside the library, held by
+ * every GPU that loads it until the process exits.  The call allocates
+ * nothing.
+ * Limits: x_dtype = SA_BF16, d = 128, k a multiple of 128 up to 512,
+ * 1 <= B <= 8; anything else returns SA_ERR_UNSUPPORTED before any GPU work.
+ * Calls share the array: calls that overlap on the GPU (other streams, other
+ * host threads) race and must be serialised.  No scratch word needs to start
+ * at zero.  The first call on each device looks up the array's address, with
+ * that device current; make it before any stream capture.
+ */
+sa_status sa_forward_noalloc(const void* X, sa_dtype x_dtype,
+                             const int64_t* offsets_host, const int64_t* offsets_dev, int B,
+                             int k, int d,
+                             const float* P, const float* W_Q, const float* W_K,
+                             const float* W_V, float eps,
+                             float* S, float* mass, float* H, void* S_bf16, float* lse,
+                             sa_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Sketch Attention backward                                                 */
 /* ------------------------------------------------------------------------ */

@@ -27,7 +27,8 @@ _STATUS = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_
 # Symbols include/sketch_attn.h declares.
 EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_workspace",
            "sa_forward", "sa_backward_workspace", "sa_backward", "stca_forward_workspace",
-           "stca_forward", "stca_fuse", "sa_launch_count", "sa_profile", "sa_profile_read")
+           "stca_forward", "stca_fuse", "sa_launch_count", "sa_profile", "sa_profile_read",
+           "sa_forward_noalloc")
 
 
 class SAError(RuntimeError):
@@ -76,6 +77,9 @@ def load(path: Optional[str] = None):
                                  _i, _i, _i, _i, ctypes.POINTER(StcaLayerC), _vp, _vp, _sz, _vp]
     lib.stca_fuse.restype = _i
     lib.stca_fuse.argtypes = [_vp, _vp, _vp, _vp, _i64, _i, _vp, _vp]
+    lib.sa_forward_noalloc.restype = _i
+    lib.sa_forward_noalloc.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
+                                       _vp, _vp, _vp, _vp, _vp, _vp]
     lib.sa_launch_count.restype = ctypes.c_longlong
     lib.sa_profile.restype = _i
     lib.sa_profile.argtypes = [_i]
@@ -171,6 +175,27 @@ def sa_forward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
     if lse is not None:
         res["lse"] = lse
     return res
+
+
+def sa_forward_noalloc(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
+                       offsets_dev: torch.Tensor, out: dict, stream=None) -> dict:
+    """sa_forward without a workspace, for callers that cannot allocate device
+    memory: every buffer is the caller's (``out`` holds preallocated "S" and
+    "mass", optionally "H", "S_bf16", "lse"; ``offsets_dev`` is a device copy of
+    the offsets), and the library's fixed scratch array stands in for the
+    workspace.  This wrapper allocates nothing on the device."""
+    lib = load()
+    _need_cuda(X, P, W_Q, W_K, W_V, offsets_dev)
+    off = _host_i64(offsets)
+    B = len(off) - 1
+    k, d = P.shape
+    o = {n: out.get(n) for n in ("S", "mass", "H", "S_bf16", "lse")}
+    _need_cuda(*[t for t in o.values() if t is not None])
+    st = lib.sa_forward_noalloc(_p(X), _dtype_code(X), _hp(off), _p(offsets_dev), B, k, d, _p(P),
+                                _p(W_Q), _p(W_K), _p(W_V), float(eps), _p(o["S"]), _p(o["mass"]),
+                                _p(o["H"]), _p(o["S_bf16"]), _p(o["lse"]), _stream(stream))
+    _check("sa_forward_noalloc", st)
+    return {n: t for n, t in o.items() if t is not None}
 
 
 def sa_backward_workspace(B: int, n_total: int, k: int, d: int, dtype: int) -> int:
