@@ -8,7 +8,9 @@
 // H_slice = [A_slice X | A_slice 1] (128 x 144 fp32 in TMEM; the last 16
 // columns hold the mass).  Every CTA of the cluster streams the same 128-token
 // tiles of X through SMEM with TMA (no multicast: each CTA issues its own
-// loads, the copies after the first come from L2).
+// loads, the copies after the first come from L2).  An X tile stays in SMEM
+// from its load until its aggregation MMA, so the number of stages bounds the
+// tiles in flight; the shared-memory budget goes to four stages.
 //
 // Per tile (t = 128 tokens of one user):
 //   MMA1   Z^T[t, j] = X_t . P'_j              (M=128 tokens, N=128 prototypes, K=d)
@@ -36,7 +38,7 @@ using namespace tc;
 
 constexpr int TILE = 128;            // tokens per tile = prototypes per CTA
 constexpr int DD = 128;              // d
-constexpr int NS = 3;                // X pipeline stages
+constexpr int NS = 4;                // X pipeline stages (tiles in flight)
 constexpr int MAXC = 8;              // cluster size limit (k <= 1024)
 constexpr int N2 = DD + 16;          // MMA2 N: d columns + 16 mass columns
 constexpr int THREADS = 320;
@@ -46,10 +48,9 @@ constexpr uint32_t X_BOX = TILE * 32;                  // one [128 x 16] bf16 SW
 constexpr uint32_t X_STAGE = 9 * X_BOX;                // 8 boxes of X + 1 box of ones = 36 KB
 constexpr uint32_t OFF_PQ = 0;                         // P' slice: 2 x [128 x 64] SW128 = 32 KB
 constexpr uint32_t OFF_X = 32768;
-constexpr uint32_t OFF_P = OFF_X + NS * X_STAGE;       // 2 x 32 KB probability tiles
-constexpr uint32_t OFF_XCHG = OFF_P + 2 * 32768;       // [4 slots][MAXC][128] fp32
-constexpr uint32_t OFF_STAGE = OFF_XCHG + 4 * MAXC * TILE * 4;  // [2 wg][2][128] fp32
-constexpr uint32_t OFF_BAR = OFF_STAGE + 2 * 2 * TILE * 4;
+constexpr uint32_t OFF_P = OFF_X + NS * X_STAGE;       // one 32 KB probability tile
+constexpr uint32_t OFF_XCHG = OFF_P + 32768;           // [4 slots][MAXC][128] fp32
+constexpr uint32_t OFF_BAR = OFF_XCHG + 4 * MAXC * TILE * 4;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
 
 // TMEM columns
@@ -57,7 +58,7 @@ constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_H = 256, TM_COLS = 512;
 
 struct Bars {
   uint64_t x_full[NS], x_empty[NS];
-  uint64_t s_full[2], p_full[2], p_empty[2];
+  uint64_t s_full[2], s_empty[2], p_full, p_empty;
   uint64_t h_full, h_empty, pq_full, mma_done;
   uint64_t xchg[4];
   uint32_t tmem_base;
@@ -92,6 +93,41 @@ __device__ __forceinline__ void for_each_tile(const Params& p, int g, F&& f) {
   }
 }
 
+// The same tile sequence as a cursor that can be advanced one tile at a time.
+struct TileCursor {
+  int64_t cb, ce, pb, pe, tb;
+  int u, t, piece;
+  bool done;
+  __device__ void start(const Params& p, int g) {
+    cb = (int64_t)g * p.ch.T;
+    ce = min(cb + p.ch.T, p.ch.n_total);
+    u = user_of_token(p.off, p.B, cb);         // non-empty and overlapping the chunk
+    pb = max(p.off[u], cb);
+    pe = min(p.off[u + 1], ce);
+    tb = pb;
+    t = 0;
+    piece = 0;
+    done = false;
+  }
+  __device__ bool first() const { return tb == pb; }
+  __device__ bool last() const { return tb + TILE >= pe; }
+  __device__ void next(const Params& p) {
+    ++t;
+    tb += TILE;
+    if (tb < pe) return;
+    for (++u; u < p.B && p.off[u] < ce; ++u) {
+      pb = max(p.off[u], cb);
+      pe = min(p.off[u + 1], ce);
+      if (pb < pe) {
+        tb = pb;
+        ++piece;
+        return;
+      }
+    }
+    done = true;
+  }
+};
+
 __global__ void __launch_bounds__(THREADS, 1)
     sa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmP, Params p) {
@@ -109,9 +145,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int s = 0; s < NS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->p_full[b], 128);
-      mbar_init(&bars->p_empty[b], 1);
+      mbar_init(&bars->s_empty[b], 128);
     }
+    mbar_init(&bars->p_full, 128);
+    mbar_init(&bars->p_empty, 1);
     mbar_init(&bars->h_full, 1);
     mbar_init(&bars->h_empty, 128);
     mbar_init(&bars->pq_full, 1);
@@ -120,7 +157,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     bars->abort = 0;
     fence_mbar_init();
     // arm the exchange slots for their first use (tiles 0..3)
-    for (int s = 0; s < 4; ++s) mbar_arrive_expect_tx(&bars->xchg[s], C * TILE * 4);
+    for (int s = 0; s < 4; ++s) mbar_arrive_expect_tx(&bars->xchg[s], (C - 1) * TILE * 4);
   }
   // constant ones block of every stage (MMA2 columns d..d+15 -> prototype mass)
   for (int i = threadIdx.x; i < NS * (int)X_BOX / 4; i += THREADS) {
@@ -164,54 +201,69 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
+      // Two cursors over the same tiles: MMA1 (logits) runs ahead as soon as a
+      // logits buffer is released and the X tile has landed; MMA2 (aggregate)
+      // follows each tile's probabilities.  The barriers are polled, so a tile
+      // waiting on its cluster exchange does not hold back the next logits.
       const uint32_t id1 = idesc_bf16(128, 128, false, false);
       const uint32_t id2 = idesc_bf16(128, N2, true, true);
       const uint32_t pq = smem_u32(smem + OFF_PQ);
       bool ok = mbar_wait(&bars->pq_full, 0, abort, p.err);
-      int piece = -1;
-      int prev_t = -1;
-      bool prev_first = false, prev_last = false;
-      auto mma2 = [&](int t, bool first, bool last) -> bool {
-        const int b = t & 1, s = t % NS;
-        if (first && piece > 0 && !mbar_wait(&bars->h_empty, (piece - 1) & 1, abort, p.err)) return false;
-        if (!mbar_wait(&bars->p_full[b], (t >> 1) & 1, abort, p.err)) return false;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(smem + OFF_P + b * 32768);
-        const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
+      TileCursor c1, c2;
+      c1.start(p, g);
+      c2.start(p, g);
+      long long idle0 = clock64();
+      while (ok && !c2.done) {
+        bool progress = false;
+        if (!c1.done) {
+          const int t = c1.t, s = t % NS, b = t & 1;
+          if ((t < 2 || mbar_test(&bars->s_empty[b], ((t >> 1) - 1) & 1)) &&
+              mbar_test(&bars->x_full[s], (t / NS) & 1)) {
+            tc_fence_after();
+            const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t da = smem_desc(pa + ks * 2048, 16384, 1024, SWZ_128B);
-          const uint64_t db = smem_desc(xa + ks * 512, X_BOX, 256, SWZ_32B);
-          mma_ss(tmem + TM_H, da, db, id2, (first && ks == 0) ? 0u : 1u);
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint64_t da = smem_desc(xa + ks * X_BOX, 16, 256, SWZ_32B);
+              const uint64_t db = smem_desc(pq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B);
+              mma_ss(tmem + (b ? TM_S1 : TM_S0), da, db, id1, ks > 0 ? 1u : 0u);
+            }
+            mma_commit(&bars->s_full[b]);
+            c1.next(p);
+            progress = true;
+          }
         }
-        mma_commit(&bars->p_empty[b]);
-        mma_commit(&bars->x_empty[s]);
-        if (last) mma_commit(&bars->h_full);
-        return true;
-      };
-      if (ok) {
-        for_each_tile(p, g, [&](int t, int, int64_t, int64_t, int64_t, bool first, bool last) {
-          const int s = t % NS, b = t & 1;
-          if (!mbar_wait(&bars->x_full[s], (t / NS) & 1, abort, p.err)) return false;
-          tc_fence_after();
-          const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
+        if (c2.t < c1.t) {
+          const int t = c2.t, b = t & 1, s = t % NS;
+          const bool first = c2.first(), last = c2.last();
+          bool ready = mbar_test(&bars->p_full, t & 1);
+          if (ready && first && c2.piece > 0) ready = mbar_test(&bars->h_empty, (c2.piece - 1) & 1);
+          if (ready) {
+            tc_fence_after();
+            const uint32_t pa = smem_u32(smem + OFF_P);
+            const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t da = smem_desc(xa + ks * X_BOX, 16, 256, SWZ_32B);
-            const uint64_t db = smem_desc(pq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B);
-            mma_ss(tmem + (b ? TM_S1 : TM_S0), da, db, id1, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint64_t da = smem_desc(pa + ks * 2048, 16384, 1024, SWZ_128B);
+              const uint64_t db = smem_desc(xa + ks * 512, X_BOX, 256, SWZ_32B);
+              mma_ss(tmem + TM_H, da, db, id2, (first && ks == 0) ? 0u : 1u);
+            }
+            mma_commit(&bars->p_empty);
+            mma_commit(&bars->x_empty[s]);
+            if (last) mma_commit(&bars->h_full);
+            c2.next(p);
+            progress = true;
           }
-          mma_commit(&bars->s_full[b]);
-          if (prev_t >= 0) {
-            if (prev_first) ++piece;
-            if (!mma2(prev_t, prev_first, prev_last)) return false;
-          }
-          prev_t = t; prev_first = first; prev_last = last;
-          return true;
-        });
-        if (prev_t >= 0 && !*abort) {
-          if (prev_first) ++piece;
-          mma2(prev_t, prev_first, prev_last);
+        }
+        if (progress) {
+          idle0 = clock64();
+        } else if (*abort) {
+          break;
+        } else if (clock64() - idle0 > 4000000000LL) {
+          *abort = 1;
+          if (p.err) atomicOr(p.err, 1);
+          break;
+        } else {
+          __nanosleep(32);      // leave issue slots to the softmax warps sharing this SMSP
         }
       }
       // every MMA this thread issued has completed before TMEM is released
@@ -223,7 +275,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int q = warp % 4;                   // TMEM lane quarter
       const int row = q * 32 + lane;            // token within the tile / prototype lane
       const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-      float* stage = (float*)(smem + OFF_STAGE) + wg * 2 * TILE;
       const float* xchg = (const float*)(smem + OFF_XCHG);
       int piece = -1;
       for_each_tile(p, g, [&](int t, int u, int64_t tb, int64_t pb, int64_t pe, bool first, bool last) {
@@ -234,51 +285,58 @@ __global__ void __launch_bounds__(THREADS, 1)
           // logits of this token over the CTA's 128 prototypes (base-2 units)
           if (!mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort, p.err)) return false;
           tc_fence_after();
-          // Two halves of 64 columns; each half is exponentiated against the
-          // running maximum at that point (mh[h]).  The fp32 exponentials are
-          // parked in the logits' own TMEM columns until the cluster-wide
-          // normaliser is known, so the probabilities are rounded to bf16 once.
+          // Eight chunks of 16 logits, each exponentiated against the running
+          // maximum at that point (mc[c]) and scaled by 2^8, kept as fp16 pairs
+          // (11-bit mantissa, normal range down to 2^-22 of the chunk maximum).
+          // The load of chunk c+1 is in flight while chunk c is processed; the
+          // logits buffer is released as soon as the last chunk has landed.
           const uint32_t sbuf = tmem + lane_addr + (b ? TM_S1 : TM_S0);
-          float mh[2];
+          uint32_t ep[64];
+          float mc[8];
           float m = -__builtin_huge_valf(), s = 0.f;
-#pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            float z[64];
-            tmem_ld32(sbuf + 64 * h, z);
-            tmem_ld32(sbuf + 64 * h + 32, z + 32);
-            tmem_wait_ld();
+          float zbuf[2][16];
+          tmem_ld16(sbuf, zbuf[0]);
+          tmem_wait_ld16(zbuf[0]);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float* z = zbuf[c & 1];
+            if (c < 7) tmem_ld16(sbuf + 16 * (c + 1), zbuf[(c + 1) & 1]);
             float cm = z[0];
 #pragma unroll
-            for (int j = 1; j < 64; ++j) cm = fmaxf(cm, z[j]);
+            for (int j = 1; j < 16; ++j) cm = fmaxf(cm, z[j]);
             const float mn = fmaxf(m, cm);
             s *= ex2(m - mn);
             m = mn;
-            if (h == 0) mh[0] = mn; else mh[1] = mn;
+            mc[c] = mn;
+            const float off = 8.f - mn;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
-              z[j] = ex2(z[j] - mn);
-              s += z[j];
+            for (int j = 0; j < 16; j += 2) {
+              const float e0 = ex2(z[j] + off), e1 = ex2(z[j + 1] + off);
+              s += e0 + e1;
+              ep[8 * c + j / 2] = pack_f16x2(e0, e1);
             }
-            tmem_st32f(sbuf + 64 * h, z);
-            tmem_st32f(sbuf + 64 * h + 32, z + 32);
+            if (c < 7) tmem_wait_ld16(zbuf[(c + 1) & 1]);
+            if (c == 6) {
+              tc_fence_before();
+              mbar_arrive(&bars->s_empty[b]);
+            }
           }
-          tmem_wait_st();
-          const float l = valid ? m + lg2(s) : -__builtin_huge_valf();
-          // send this CTA's log2-sum-exp of every token to every CTA of the cluster
-          float* st = stage + ((t >> 1) & 1) * TILE;
-          st[row] = l;
+          const float l = valid ? m + lg2(s) - 8.f : -__builtin_huge_valf();
+          // this CTA's log2-sum-exp of every token goes into its own row of the
+          // exchange slot, and from there to the same row in every other CTA
+          const int slot = t & 3;
+          float* own = (float*)(smem + OFF_XCHG) + (slot * MAXC + rank) * TILE;
+          own[row] = l;
           fence_proxy_async_smem();
           named_bar_sync(1 + wg, 128);
-          const int slot = t & 3;
           if (row == 0) {
-            const uint32_t src = smem_u32(st);
-            const uint32_t dst = smem_u32(smem + OFF_XCHG + (slot * MAXC + rank) * TILE * 4);
+            const uint32_t src = smem_u32(own);
             const uint32_t bar = smem_u32(&bars->xchg[slot]);
             for (uint32_t c = 0; c < C; ++c)
-              bulk_copy_to_peer(map_to_rank(dst, c), src, TILE * 4, map_to_rank(bar, c));
+              if (c != rank) bulk_copy_to_peer(map_to_rank(src, c), src, TILE * 4, map_to_rank(bar, c));
           }
           if (!mbar_wait(&bars->xchg[slot], (t >> 2) & 1, abort, p.err)) return false;
-          float rh[2] = {0.f, 0.f};
+          float rc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
           if (valid) {
             float L = -__builtin_huge_valf();
             for (uint32_t c = 0; c < C; ++c) L = fmaxf(L, xchg[(slot * MAXC + c) * TILE + row]);
@@ -286,32 +344,27 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (uint32_t c = 0; c < C; ++c) z += ex2(xchg[(slot * MAXC + c) * TILE + row] - L);
             const float lt = L + lg2(z);
             if (p.lse && rank == 0) p.lse[tb + row] = lt * 0.69314718055994530942f;
-            rh[0] = ex2(mh[0] - lt);
-            rh[1] = ex2(mh[1] - lt);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) rc[c] = ex2(mc[c] - 8.f - lt);
           }
           named_bar_sync(1 + wg, 128);      // every thread has read the slot
-          if (row == 0) mbar_arrive_expect_tx(&bars->xchg[slot], C * TILE * 4);   // re-arm for t+4
+          if (row == 0) mbar_arrive_expect_tx(&bars->xchg[slot], (C - 1) * TILE * 4);   // re-arm for t+4
           // probabilities p[t, j] = e_j r as bf16 into the MN-major SW128 A tile of MMA2
-          if (t >= 2 && !mbar_wait(&bars->p_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return false;
-          const uint32_t pa = smem_u32(smem + OFF_P + b * 32768) + row * 128;
-#pragma unroll 1
-          for (int blk = 0; blk < 2; ++blk) {
-            const float r = blk == 0 ? rh[0] : rh[1];
-            float e[64];
-            tmem_ld32(sbuf + 64 * blk, e);
-            tmem_ld32(sbuf + 64 * blk + 32, e + 32);
-            tmem_wait_ld();
+          if (t >= 1 && !mbar_wait(&bars->p_empty, (t - 1) & 1, abort, p.err)) return false;
+          const uint32_t pa = smem_u32(smem + OFF_P) + row * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const float* q8 = e + c * 8;
-              st_shared_v4(pa + blk * 16384 + ((c ^ (row & 7)) << 4),
-                           pack_bf16x2(q8[0] * r, q8[1] * r), pack_bf16x2(q8[2] * r, q8[3] * r),
-                           pack_bf16x2(q8[4] * r, q8[5] * r), pack_bf16x2(q8[6] * r, q8[7] * r));
-            }
+          for (int cc = 0; cc < 16; ++cc) {           // 16-byte chunks of 8 prototypes
+            const float r = rc[cc >> 1];
+            const uint32_t* e4 = ep + 4 * cc;
+            const float2 a0 = unpack_f16x2(e4[0]), a1 = unpack_f16x2(e4[1]);
+            const float2 a2 = unpack_f16x2(e4[2]), a3 = unpack_f16x2(e4[3]);
+            st_shared_v4(pa + (cc >> 3) * 16384 + (((cc & 7) ^ (row & 7)) << 4),
+                         pack_bf16x2(a0.x * r, a0.y * r), pack_bf16x2(a1.x * r, a1.y * r),
+                         pack_bf16x2(a2.x * r, a2.y * r), pack_bf16x2(a3.x * r, a3.y * r));
           }
           fence_proxy_async_smem();
           tc_fence_before();
-          mbar_arrive(&bars->p_full[b]);
+          mbar_arrive(&bars->p_full);
         }
         if (last && wg == 0) {
           // ------------------------------------------------------ drain H of the piece
