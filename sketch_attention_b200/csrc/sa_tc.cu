@@ -21,10 +21,10 @@
 //   MMA2   H_slice[j, :] += sum_t p[t, j] [x_t | 1]   (M=128 prototypes, N=144, K=128 tokens)
 // so the k x n assignment matrix never leaves the SM.
 //
-// Warp roles (10 warps): 0 TMA, 1 MMA issue + TMEM owner, 2-5 softmax of
-// even tiles (and the H drain at the end of a piece), 6-9 softmax of odd
-// tiles.  A warp reads TMEM lanes 32 (warp % 4) .. +31, so each group of four
-// consecutive warps covers all 128 lanes.
+// Warp roles (11 warps): 0 TMA, 1 logits MMAs + TMEM owner, 2 aggregation
+// MMAs, 3-6 softmax of even tiles (and the H drain at the end of a piece),
+// 7-10 softmax of odd tiles.  A warp reads TMEM lanes 32 (warp % 4) .. +31, so
+// each group of four consecutive warps covers all 128 lanes.
 #include <algorithm>
 #include <mutex>
 
@@ -41,7 +41,7 @@ constexpr int DD = 128;              // d
 constexpr int NS = 4;                // X pipeline stages (tiles in flight)
 constexpr int MAXC = 8;              // cluster size limit (k <= 1024)
 constexpr int N2 = DD + 16;          // MMA2 N: d columns + 16 mass columns
-constexpr int THREADS = 320;
+constexpr int THREADS = 352;
 
 // shared-memory layout (offsets from a 1024-aligned base)
 constexpr uint32_t X_BOX = TILE * 32;                  // one [128 x 16] bf16 SW32 box = 4 KB
@@ -93,41 +93,6 @@ __device__ __forceinline__ void for_each_tile(const Params& p, int g, F&& f) {
   }
 }
 
-// The same tile sequence as a cursor that can be advanced one tile at a time.
-struct TileCursor {
-  int64_t cb, ce, pb, pe, tb;
-  int u, t, piece;
-  bool done;
-  __device__ void start(const Params& p, int g) {
-    cb = (int64_t)g * p.ch.T;
-    ce = min(cb + p.ch.T, p.ch.n_total);
-    u = user_of_token(p.off, p.B, cb);         // non-empty and overlapping the chunk
-    pb = max(p.off[u], cb);
-    pe = min(p.off[u + 1], ce);
-    tb = pb;
-    t = 0;
-    piece = 0;
-    done = false;
-  }
-  __device__ bool first() const { return tb == pb; }
-  __device__ bool last() const { return tb + TILE >= pe; }
-  __device__ void next(const Params& p) {
-    ++t;
-    tb += TILE;
-    if (tb < pe) return;
-    for (++u; u < p.B && p.off[u] < ce; ++u) {
-      pb = max(p.off[u], cb);
-      pe = min(p.off[u + 1], ce);
-      if (pb < pe) {
-        tb = pb;
-        ++piece;
-        return;
-      }
-    }
-    done = true;
-  }
-};
-
 __global__ void __launch_bounds__(THREADS, 1)
     sa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                      const __grid_constant__ CUtensorMap tmP, Params p) {
@@ -152,7 +117,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(&bars->h_full, 1);
     mbar_init(&bars->h_empty, 128);
     mbar_init(&bars->pq_full, 1);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->mma_done, 2);        // both MMA-issuing threads
     for (int s = 0; s < 4; ++s) mbar_init(&bars->xchg[s], 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -200,78 +165,62 @@ __global__ void __launch_bounds__(THREADS, 1)
           mbar_wait_bounded(&bars->x_full[t % NS], (t / NS) & 1);
       }
     } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      // Two cursors over the same tiles: MMA1 (logits) runs ahead as soon as a
-      // logits buffer is released and the X tile has landed; MMA2 (aggregate)
-      // follows each tile's probabilities.  The barriers are polled, so a tile
-      // waiting on its cluster exchange does not hold back the next logits.
+      // ------------------------------------------------------------ logits MMAs
+      // MMA1 of a tile is issued as soon as its X tile has landed and the
+      // logits buffer it reuses has been read by the softmax warps.
       const uint32_t id1 = idesc_bf16(128, 128, false, false);
-      const uint32_t id2 = idesc_bf16(128, N2, true, true);
       const uint32_t pq = smem_u32(smem + OFF_PQ);
-      bool ok = mbar_wait(&bars->pq_full, 0, abort, p.err);
-      TileCursor c1, c2;
-      c1.start(p, g);
-      c2.start(p, g);
-      long long idle0 = clock64();
-      while (ok && !c2.done) {
-        bool progress = false;
-        if (!c1.done) {
-          const int t = c1.t, s = t % NS, b = t & 1;
-          if ((t < 2 || mbar_test(&bars->s_empty[b], ((t >> 1) - 1) & 1)) &&
-              mbar_test(&bars->x_full[s], (t / NS) & 1)) {
-            tc_fence_after();
-            const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
+      if (mbar_wait(&bars->pq_full, 0, abort, p.err)) {
+        for_each_tile(p, g, [&](int t, int, int64_t, int64_t, int64_t, bool, bool) {
+          const int s = t % NS, b = t & 1;
+          if (!mbar_wait(&bars->x_full[s], (t / NS) & 1, abort, p.err)) return false;
+          if (t >= 2 && !mbar_wait(&bars->s_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return false;
+          tc_fence_after();
+          const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              const uint64_t da = smem_desc(xa + ks * X_BOX, 16, 256, SWZ_32B);
-              const uint64_t db = smem_desc(pq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B);
-              mma_ss(tmem + (b ? TM_S1 : TM_S0), da, db, id1, ks > 0 ? 1u : 0u);
-            }
-            mma_commit(&bars->s_full[b]);
-            c1.next(p);
-            progress = true;
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t da = smem_desc(xa + ks * X_BOX, 16, 256, SWZ_32B);
+            const uint64_t db = smem_desc(pq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B);
+            mma_ss(tmem + (b ? TM_S1 : TM_S0), da, db, id1, ks > 0 ? 1u : 0u);
           }
-        }
-        if (c2.t < c1.t) {
-          const int t = c2.t, b = t & 1, s = t % NS;
-          const bool first = c2.first(), last = c2.last();
-          bool ready = mbar_test(&bars->p_full, t & 1);
-          if (ready && first && c2.piece > 0) ready = mbar_test(&bars->h_empty, (c2.piece - 1) & 1);
-          if (ready) {
-            tc_fence_after();
-            const uint32_t pa = smem_u32(smem + OFF_P);
-            const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              const uint64_t da = smem_desc(pa + ks * 2048, 16384, 1024, SWZ_128B);
-              const uint64_t db = smem_desc(xa + ks * 512, X_BOX, 256, SWZ_32B);
-              mma_ss(tmem + TM_H, da, db, id2, (first && ks == 0) ? 0u : 1u);
-            }
-            mma_commit(&bars->p_empty);
-            mma_commit(&bars->x_empty[s]);
-            if (last) mma_commit(&bars->h_full);
-            c2.next(p);
-            progress = true;
-          }
-        }
-        if (progress) {
-          idle0 = clock64();
-        } else if (*abort) {
-          break;
-        } else if (clock64() - idle0 > 4000000000LL) {
-          *abort = 1;
-          if (p.err) atomicOr(p.err, 1);
-          break;
-        } else {
-          __nanosleep(32);      // leave issue slots to the softmax warps sharing this SMSP
-        }
+          mma_commit(&bars->s_full[b]);
+          return true;
+        });
       }
       // every MMA this thread issued has completed before TMEM is released
       mma_commit(&bars->mma_done);
       mbar_wait_bounded(&bars->mma_done, 0);
-    } else if (warp >= 2) {
+    } else if (warp == 2 && lane == 0) {
+      // ------------------------------------------------------------ aggregation MMAs
+      // A second issuing thread, so MMA2 of a tile starts the moment its
+      // probabilities are written, independent of the logits of later tiles
+      // (the two streams touch disjoint TMEM and SMEM).
+      const uint32_t id2 = idesc_bf16(128, N2, true, true);
+      int piece = -1;
+      for_each_tile(p, g, [&](int t, int, int64_t, int64_t, int64_t, bool first, bool last) {
+        const int s = t % NS;
+        if (first) ++piece;
+        if (first && piece > 0 && !mbar_wait(&bars->h_empty, (piece - 1) & 1, abort, p.err)) return false;
+        if (!mbar_wait(&bars->p_full, t & 1, abort, p.err)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(smem + OFF_P);
+        const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint64_t da = smem_desc(pa + ks * 2048, 16384, 1024, SWZ_128B);
+          const uint64_t db = smem_desc(xa + ks * 512, X_BOX, 256, SWZ_32B);
+          mma_ss(tmem + TM_H, da, db, id2, (first && ks == 0) ? 0u : 1u);
+        }
+        mma_commit(&bars->p_empty);
+        mma_commit(&bars->x_empty[s]);
+        if (last) mma_commit(&bars->h_full);
+        return true;
+      });
+      mma_commit(&bars->mma_done);
+      mbar_wait_bounded(&bars->mma_done, 0);
+    } else if (warp >= 3) {
       // ------------------------------------------------------------ softmax groups
-      const int wg = (warp - 2) / 4;            // 0: even tiles, 1: odd tiles
+      const int wg = (warp - 3) / 4;            // 0: even tiles, 1: odd tiles
       const int q = warp % 4;                   // TMEM lane quarter
       const int row = q * 32 + lane;            // token within the tile / prototype lane
       const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
