@@ -27,6 +27,8 @@ import time
 import numpy as np
 import torch
 
+from sketch_attention_b200.dist import allreduce_weight_grads
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
@@ -158,8 +160,7 @@ class TrainStepRunner:
                             fwd["H"], fwd["mass"], self.dS, None, fwd["lse"],
                             offsets_dev=self.offd, out=self.go, workspace=self.ws_b)
         if self.world > 1:
-            for name in ("dP", "dW_Q", "dW_K", "dW_V"):
-                torch.distributed.all_reduce(g[name])
+            allreduce_weight_grads(g)
         if ev: ev[2].record()
         sab.stca_forward(self.q, self.cand, self.X, self.rb, self.re, self.layers_r, w.heads, w.d_h,
                          cand_offsets_dev=self.candd, kv_begin_dev=self.rbd, kv_end_dev=self.red,
