@@ -114,7 +114,7 @@ sa_status gemm(const Gemm& g0, cudaStream_t stream) {
   Gemm g = g0;
   if (g.split_k < 1 || !g.split_ws) g.split_k = 1;
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, g.batch * g.split_k);
-  SA_TIMED("gemm_kernel", stream, (gemm_kernel<<<grid, 256, 0, stream>>>(g)));
+  SA_TIMED(g.tag ? g.tag : "gemm_kernel", stream, (gemm_kernel<<<grid, 256, 0, stream>>>(g)));
   if (g.split_k > 1) {
     const int64_t n = (int64_t)g.M * g.N * g.batch;
     SA_TIMED("gemm_split_reduce_kernel", stream,

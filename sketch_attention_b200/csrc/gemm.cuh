@@ -23,6 +23,8 @@ struct Gemm {
   // slices in a fixed order and applies alpha, bias and Cin.
   int split_k = 1;
   float* split_ws = nullptr;
+  // profiler label of the call site (a string literal); NULL = "gemm_kernel"
+  const char* tag = nullptr;
 };
 
 // Split count for a GEMM with a long K and few output tiles (1 = no split).

@@ -58,14 +58,17 @@ __device__ __forceinline__ void st_row_k_major(uint32_t tile, int row, int q, ui
 
 // ============================================================== dX kernel
 constexpr int KC = 64;                       // prototypes per chunk
-constexpr int DX_NXS = 2, DX_NCS = 2;
+// One X stage (only the logits MMAs read X, so it is released after a tile's
+// last logits MMA) and one A buffer (the warpgroup packs a chunk's A values in
+// registers before it waits for the buffer) leave room for three chunk stages.
+constexpr int DX_NXS = 1, DX_NCS = 3, DX_NAB = 1;
 constexpr uint32_t XT_BYTES = 32768;         // [128 tokens x 128] bf16: 2 SW128 halves of 16 KB
 constexpr uint32_t CH_BYTES = 49152;         // [P' h0 | dH h0 | P' h1 | dH h1 | dHlo h0 | dHlo h1], 8 KB each
 constexpr uint32_t AT_BYTES = 16384;         // [128 tokens x 64] bf16 K-major SW128
 constexpr uint32_t DX_OFF_X = 0;
 constexpr uint32_t DX_OFF_CH = DX_OFF_X + DX_NXS * XT_BYTES;
-constexpr uint32_t DX_OFF_A = DX_OFF_CH + DX_NCS * CH_BYTES;        // 2 x (A tile, A o dA tile)
-constexpr uint32_t DX_OFF_DM = DX_OFF_A + 2 * 2 * AT_BYTES;
+constexpr uint32_t DX_OFF_A = DX_OFF_CH + DX_NCS * CH_BYTES;        // DX_NAB x (A tile, A o dA tile)
+constexpr uint32_t DX_OFF_DM = DX_OFF_A + DX_NAB * 2 * AT_BYTES;
 constexpr uint32_t DX_OFF_BAR = DX_OFF_DM + DX_NCS * KC * 4;
 constexpr uint32_t DX_SMEM = DX_OFF_BAR + 256 + 1024;
 constexpr int DX_THREADS = 192;              // warp 0 TMA, 1 MMA, 2-5 one thread per token
@@ -73,7 +76,7 @@ constexpr uint32_t DX_TM_ZG = 0, DX_TM_VY = 128, DX_TM_W = 384;
 
 struct DxBars {
   uint64_t x_full[DX_NXS], x_empty[DX_NXS], c_full[DX_NCS], c_empty[DX_NCS];
-  uint64_t zg_full, zg_empty, a_full[2], a_empty[2], acc_full, acc_empty, mma_done;
+  uint64_t zg_full, zg_empty, a_full[DX_NAB], a_empty[DX_NAB], acc_full, acc_empty, mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -108,7 +111,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     for (int s = 0; s < DX_NCS; ++s) { mbar_init(&bars->c_full[s], 1); mbar_init(&bars->c_empty[s], 1); }
     mbar_init(&bars->zg_full, 1);
     mbar_init(&bars->zg_empty, 128);
-    for (int b = 0; b < 2; ++b) { mbar_init(&bars->a_full[b], 128); mbar_init(&bars->a_empty[b], 1); }
+    for (int b = 0; b < DX_NAB; ++b) { mbar_init(&bars->a_full[b], 128); mbar_init(&bars->a_empty[b], 1); }
     mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->acc_empty, 128);
     mbar_init(&bars->mma_done, 1);
@@ -170,8 +173,8 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     const uint32_t id_lo = idesc_bf16(128, 64, false, true);
     int ai = 0;   // global chunk index
     auto avw = [&](int a, int t, int s, bool first, bool last) -> bool {
-      const int cs = a % DX_NCS, b = a & 1;
-      if (!mbar_wait(&bars->a_full[b], (a >> 1) & 1, abort, p.err)) return false;
+      const int cs = a % DX_NCS, b = a % DX_NAB;
+      if (!mbar_wait(&bars->a_full[b], (a / DX_NAB) & 1, abort, p.err)) return false;
       if (first && t > 0 && !mbar_wait(&bars->acc_empty, (t - 1) & 1, abort, p.err)) return false;
       tc_fence_after();
       const uint32_t at = smem_u32(smem + DX_OFF_A + b * 2 * AT_BYTES);
@@ -192,10 +195,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
       }
       mma_commit(&bars->c_empty[cs]);
       mma_commit(&bars->a_empty[b]);
-      if (last) {
-        mma_commit(&bars->x_empty[s]);
-        mma_commit(&bars->acc_full);
-      }
+      if (last) mma_commit(&bars->acc_full);
       return true;
     };
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
@@ -214,6 +214,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
                  smem_desc(cb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B), id_zg,
                  ks > 0 ? 1u : 0u);
         mma_commit(&bars->zg_full);
+        if (c == nch - 1) mma_commit(&bars->x_empty[s]);   // X is read by the logits MMAs only
         if (c > 0 && !avw(a - 1, t, s, c - 1 == 0, false)) return false;
       }
       if (!avw(ai + nch - 1, t, s, nch == 1, true)) return false;
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
       const float l2 = valid ? p.lse2[tb + row] : 0.f;
       float cacc = 0.f;
       for (int c = 0; c < nch; ++c) {
-        const int a = ai + c, cs = a % DX_NCS, b = a & 1;
+        const int a = ai + c, cs = a % DX_NCS, b = a % DX_NAB;
         if (!mbar_wait(&bars->zg_full, a & 1, abort, p.err)) return false;
         tc_fence_after();
         float z[64], gv[64];
@@ -245,10 +246,10 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
         tc_fence_before();
         mbar_arrive(&bars->zg_empty);
         if (!mbar_wait(&bars->c_full[cs], (a / DX_NCS) & 1, abort, p.err)) return false;
-        if (a >= 2 && !mbar_wait(&bars->a_empty[b], ((a >> 1) - 1) & 1, abort, p.err)) return false;
         const float4* dm4 = (const float4*)(smem + DX_OFF_DM + cs * KC * 4);
         const uint32_t at = smem_u32(smem + DX_OFF_A + b * 2 * AT_BYTES);
         const uint32_t adt = at + AT_BYTES;
+        uint32_t pa[32], pd[32];   // A and A o dA of the chunk, packed bf16 pairs
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) {
           const float4 d0 = dm4[2 * q8], d1 = dm4[2 * q8 + 1];
@@ -263,10 +264,17 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
             adv[i] = A * dA;
             cacc = fmaf(A, dA, cacc);
           }
-          st_row_k_major(at, row, q8, pack_bf16x2(av[0], av[1]), pack_bf16x2(av[2], av[3]),
-                         pack_bf16x2(av[4], av[5]), pack_bf16x2(av[6], av[7]));
-          st_row_k_major(adt, row, q8, pack_bf16x2(adv[0], adv[1]), pack_bf16x2(adv[2], adv[3]),
-                         pack_bf16x2(adv[4], adv[5]), pack_bf16x2(adv[6], adv[7]));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            pa[4 * q8 + i] = pack_bf16x2(av[2 * i], av[2 * i + 1]);
+            pd[4 * q8 + i] = pack_bf16x2(adv[2 * i], adv[2 * i + 1]);
+          }
+        }
+        if (a >= DX_NAB && !mbar_wait(&bars->a_empty[b], ((a / DX_NAB) - 1) & 1, abort, p.err)) return false;
+#pragma unroll
+        for (int q8 = 0; q8 < 8; ++q8) {
+          st_row_k_major(at, row, q8, pa[4 * q8], pa[4 * q8 + 1], pa[4 * q8 + 2], pa[4 * q8 + 3]);
+          st_row_k_major(adt, row, q8, pd[4 * q8], pd[4 * q8 + 1], pd[4 * q8 + 2], pd[4 * q8 + 3]);
         }
         fence_proxy_async_smem();
         mbar_arrive(&bars->a_full[b]);

@@ -489,14 +489,14 @@ sa_status sa_fold(int k, int d, const float* P, const float* W_Q, const float* W
   g1.M = d; g1.N = d; g1.K = d;
   g1.A = W_Q; g1.lda = d;
   g1.B = W_K; g1.ldb = d; g1.transB = true;
-  g1.C = T; g1.ldc = d;
+  g1.C = T; g1.ldc = d; g1.tag = "gemm:fold";
   sa_status s = gemm(g1, st);
   if (s != SA_OK) return s;
   Gemm g2;
   g2.M = k; g2.N = d; g2.K = d;
   g2.A = P; g2.lda = d;
   g2.B = T; g2.ldb = d;
-  g2.C = Pf; g2.ldc = d;
+  g2.C = Pf; g2.ldc = d; g2.tag = "gemm:fold";
   g2.C16 = Pb; g2.ldc16 = d;
   g2.alpha = 1.4426950408889634f / sqrtf((float)d);
   return gemm(g2, st);
@@ -522,7 +522,7 @@ sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStre
   g.A = w.Hhat; g.lda = a.d;
   g.B = a.W_V; g.ldb = a.d;
   g.C = a.S; g.ldc = a.d;
-  g.C16 = (__nv_bfloat16*)a.S_bf16; g.ldc16 = a.d;
+  g.C16 = (__nv_bfloat16*)a.S_bf16; g.ldc16 = a.d; g.tag = "gemm:S_proj";
   return gemm(g, st);
 }
 
@@ -534,7 +534,7 @@ sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaS
   g.M = rows; g.N = D; g.K = D;
   g.A = a.dS; g.lda = D;
   g.B = a.W_V; g.ldb = D; g.transB = true;
-  g.C = w.dHh; g.ldc = D;
+  g.C = w.dHh; g.ldc = D; g.tag = "gemm:dHh";
   sa_status s = gemm(g, st);
   if (s != SA_OK) return s;
   SA_TIMED("sa_bwd_prologue_kernel", st,
@@ -546,7 +546,7 @@ sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaS
   gv.M = D; gv.N = D; gv.K = rows;
   gv.A = w.Hhat; gv.lda = D; gv.transA = true;
   gv.B = a.dS; gv.ldb = D;
-  gv.C = a.dW_V; gv.ldc = D;
+  gv.C = a.dW_V; gv.ldc = D; gv.tag = "gemm:dW_V";
   gv.split_k = gemm_split_for(D, D, rows, kMaxSplit);
   gv.split_ws = w.gsplit;
   if ((s = gemm(gv, st)) != SA_OK) return s;
@@ -580,28 +580,28 @@ sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream
   // dQ = E W_K / sqrt(d)
   Gemm g1;
   g1.M = k; g1.N = D; g1.K = D;
-  g1.A = w.E; g1.lda = D; g1.B = a.W_K; g1.ldb = D; g1.C = w.dQ; g1.ldc = D; g1.alpha = rs;
+  g1.A = w.E; g1.lda = D; g1.B = a.W_K; g1.ldb = D; g1.C = w.dQ; g1.ldc = D; g1.alpha = rs; g1.tag = "gemm:E_grads";
   if ((s = gemm(g1, st)) != SA_OK) return s;
   // dP = dQ W_Q^T
   Gemm g2;
   g2.M = k; g2.N = D; g2.K = D;
-  g2.A = w.dQ; g2.lda = D; g2.B = a.W_Q; g2.ldb = D; g2.transB = true; g2.C = a.dP; g2.ldc = D;
+  g2.A = w.dQ; g2.lda = D; g2.B = a.W_Q; g2.ldb = D; g2.transB = true; g2.C = a.dP; g2.ldc = D; g2.tag = "gemm:E_grads";
   if ((s = gemm(g2, st)) != SA_OK) return s;
   // dW_Q = P^T dQ
   Gemm g3;
   g3.M = D; g3.N = D; g3.K = k;
-  g3.A = a.P; g3.lda = D; g3.transA = true; g3.B = w.dQ; g3.ldb = D; g3.C = a.dW_Q; g3.ldc = D;
+  g3.A = a.P; g3.lda = D; g3.transA = true; g3.B = w.dQ; g3.ldb = D; g3.C = a.dW_Q; g3.ldc = D; g3.tag = "gemm:E_grads";
   g3.split_k = gemm_split_for(D, D, k, kMaxSplit);
   g3.split_ws = w.gsplit;
   if ((s = gemm(g3, st)) != SA_OK) return s;
   // Q = P W_Q;  dW_K = E^T Q / sqrt(d)
   Gemm g4;
   g4.M = k; g4.N = D; g4.K = D;
-  g4.A = a.P; g4.lda = D; g4.B = a.W_Q; g4.ldb = D; g4.C = w.Q; g4.ldc = D;
+  g4.A = a.P; g4.lda = D; g4.B = a.W_Q; g4.ldb = D; g4.C = w.Q; g4.ldc = D; g4.tag = "gemm:E_grads";
   if ((s = gemm(g4, st)) != SA_OK) return s;
   Gemm g5;
   g5.M = D; g5.N = D; g5.K = k;
-  g5.A = w.E; g5.lda = D; g5.transA = true; g5.B = w.Q; g5.ldb = D; g5.C = a.dW_K; g5.ldc = D;
+  g5.A = w.E; g5.lda = D; g5.transA = true; g5.B = w.Q; g5.ldb = D; g5.C = a.dW_K; g5.ldc = D; g5.tag = "gemm:E_grads";
   g5.alpha = rs;
   g5.split_k = gemm_split_for(D, D, k, kMaxSplit);
   g5.split_ws = w.gsplit;

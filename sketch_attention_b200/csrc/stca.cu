@@ -153,7 +153,7 @@ sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
     g1.M = (int)C; g1.N = dh; g1.K = D;
     g1.A = a.out; g1.lda = D; g1.sA = 0;
     g1.B = L.W_Q; g1.ldb = dh; g1.sB = (int64_t)D * dh;
-    g1.C = w.Qh; g1.ldc = HD; g1.sC = dh;
+    g1.C = w.Qh; g1.ldc = HD; g1.sC = dh; g1.tag = "gemm:stca_Qh";
     g1.batch = H;
     if ((s = gemm(g1, st)) != SA_OK) return s;
     // U[c, h, :] = Qh[:, h] W_K^h^T * log2(e)/sqrt(d_h)
@@ -163,7 +163,7 @@ sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
     g2.B = L.W_K; g2.ldb = dh; g2.transB = true; g2.sB = (int64_t)D * dh;
     if (tc) { g2.C16 = w.Ub; g2.ldc16 = (int64_t)H * D; g2.sC16 = D; }
     else { g2.C = w.U; g2.ldc = (int64_t)H * D; g2.sC = D; }
-    g2.alpha = 1.4426950408889634f / sqrtf((float)dh);
+    g2.alpha = 1.4426950408889634f / sqrtf((float)dh); g2.tag = "gemm:stca_U";
     g2.batch = H;
     if ((s = gemm(g2, st)) != SA_OK) return s;
     // Y = attention over the user's keys
@@ -186,7 +186,7 @@ sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
     g3.M = (int)C; g3.N = dh; g3.K = D;
     g3.A = w.Y; g3.lda = (int64_t)H * D; g3.sA = D;
     g3.B = L.W_V; g3.ldb = dh; g3.sB = (int64_t)D * dh;
-    g3.C = w.O; g3.ldc = HD; g3.sC = dh;
+    g3.C = w.O; g3.ldc = HD; g3.sC = dh; g3.tag = "gemm:stca_O";
     g3.batch = H;
     if ((s = gemm(g3, st)) != SA_OK) return s;
     // q <- q + O W_O  (or q + O)
@@ -196,7 +196,7 @@ sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
       g4.A = w.O; g4.lda = HD;
       g4.B = L.W_O; g4.ldb = D;
       g4.C = a.out; g4.ldc = D;
-      g4.Cin = a.out; g4.ldcin = D;
+      g4.Cin = a.out; g4.ldcin = D; g4.tag = "gemm:stca_WO";
       if ((s = gemm(g4, st)) != SA_OK) return s;
     } else {
       SA_TIMED("add_kernel", st, (add_kernel<<<grid_for(nq), 256, 0, st>>>(a.out, w.O, nq)));
@@ -210,13 +210,13 @@ sa_status stca_fuse_run(const float* z_r, const float* z_u, const float* W_F, co
   if (C == 0) return SA_OK;
   Gemm g1;
   g1.M = (int)C; g1.N = D; g1.K = D;
-  g1.A = z_r; g1.lda = D; g1.B = W_F; g1.ldb = D; g1.C = out; g1.ldc = D; g1.bias = b_F;
+  g1.A = z_r; g1.lda = D; g1.B = W_F; g1.ldb = D; g1.C = out; g1.ldc = D; g1.bias = b_F; g1.tag = "gemm:fuse";
   sa_status s = gemm(g1, st);
   if (s != SA_OK) return s;
   Gemm g2;
   g2.M = (int)C; g2.N = D; g2.K = D;
   g2.A = z_u; g2.lda = D; g2.B = W_F + (int64_t)D * D; g2.ldb = D;
-  g2.C = out; g2.ldc = D; g2.Cin = out; g2.ldcin = D;
+  g2.C = out; g2.ldc = D; g2.Cin = out; g2.ldcin = D; g2.tag = "gemm:fuse";
   return gemm(g2, st);
 }
 
