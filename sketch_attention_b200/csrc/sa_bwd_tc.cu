@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
 }
 
 // ============================================================== E kernel
-constexpr int E_NXS = 2;
+constexpr int E_NXS = 3;   // X tiles in flight: each is held from its load until the E MMA of its tile
 constexpr uint32_t E_OFF_PH = 0;              // [P' h0 | dH h0 | P' h1 | dH h1], 16 KB each
 constexpr uint32_t E_OFF_X = 65536;
 constexpr uint32_t E_OFF_DZ = E_OFF_X + E_NXS * XT_BYTES;   // 2 x [128 protos x 128 tokens] MN-major
