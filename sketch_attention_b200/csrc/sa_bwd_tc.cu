@@ -5,19 +5,21 @@
 // With A = 2^{z - lse} (z = P' x in base-2 units, lse saved by the forward),
 // dA_tj = dH_j . x_t + dm_j, c_t = sum_j A_tj dA_tj and dZ = A o (dA - c):
 //   dX_t = sum_j A_tj dH_j + ln2 sum_j dZ_tj P'_j
-//        = Y_t + ln2 (W_t - c_t V_t),   Y = A dH,  V = A P',  W = (A o dA) P'
+//        = Q_t - ln2 c_t V_t,   Q = A dH + ln2 (A o dA) P',  V = A P'
 //   E    = sum_t dZ_t^T x_t   (weight gradients follow from E by small GEMMs)
 // dm is centred per user (dZ and dX do not change when a constant is added to
-// dA); this keeps W - c V free of a large common term.
+// dA); this keeps ln2 (A o dA) P' - ln2 c V free of a large common term.
 //
 // Two kernels:
 //   sa_bwd_dx_tc_kernel  token-parallel: one CTA per token chunk, all k per
 //     tile in chunks of 64 prototypes.  Per chunk: [Z|G] = X [P'_c;dH_c]^T
-//     (M=128 tokens, N=128), then A and A o dA to SMEM (bf16) and
-//     [V|Y] += A [P'_c|dH_c] (N=256), W += (A o dA) P'_c (N=128), all in TMEM;
-//     Y also takes A times the bf16 residual of dH (dH = dH_hi + dH_lo), so
-//     only A's rounding is left in Y.  c_t accumulates in registers.  Needs
-//     no knowledge of c beforehand.
+//     (M=128 tokens, N=128), then A and ln2 A o dA as bf16 into TMEM, and
+//     V += A P'_c,  Q += A dH_c + (ln2 A o dA) P'_c  (the two terms of Q share
+//     one accumulator by concatenating their K; A is the TMEM operand, so the
+//     aggregation MMAs read only P'_c and dH_c from shared memory).  Q also
+//     takes A times the bf16 residual of dH (dH = dH_hi + dH_lo), so only A's
+//     rounding is left in it.  c_t accumulates in registers; at the end of
+//     the tile dX = Q - ln2 c V, so c is not needed beforehand.
 //   sa_bwd_e_tc_kernel   prototype-slice-parallel: one CTA per (128-prototype
 //     slice, token chunk).  Per tile: [Z|G] (N=256), dZ (bf16, SMEM), then
 //     E_slice += dZ^T X (M=128 prototypes, N=128) in TMEM.
@@ -50,33 +52,27 @@ __device__ __forceinline__ void for_each_tile(const int64_t* off, int B, const C
   }
 }
 
-__device__ __forceinline__ void st_row_k_major(uint32_t tile, int row, int q, uint32_t a,
-                                               uint32_t b, uint32_t c, uint32_t d) {
-  // 16-byte chunk q of `row` in a K-major SW128 tile of 128-byte rows
-  st_shared_v4(tile + row * 128 + ((q ^ (row & 7)) << 4), a, b, c, d);
-}
-
 // ============================================================== dX kernel
 constexpr int KC = 64;                       // prototypes per chunk
-// One X stage (only the logits MMAs read X, so it is released after a tile's
-// last logits MMA) and one A buffer (the warpgroup packs a chunk's A values in
-// registers before it waits for the buffer) leave room for three chunk stages.
-constexpr int DX_NXS = 1, DX_NCS = 3, DX_NAB = 1;
+constexpr int DX_NXS = 1, DX_NCS = 4;        // X stages (only the logits MMAs read X), chunk stages
 constexpr uint32_t XT_BYTES = 32768;         // [128 tokens x 128] bf16: 2 SW128 halves of 16 KB
 constexpr uint32_t CH_BYTES = 49152;         // [P' h0 | dH h0 | P' h1 | dH h1 | dHlo h0 | dHlo h1], 8 KB each
-constexpr uint32_t AT_BYTES = 16384;         // [128 tokens x 64] bf16 K-major SW128
 constexpr uint32_t DX_OFF_X = 0;
 constexpr uint32_t DX_OFF_CH = DX_OFF_X + DX_NXS * XT_BYTES;
-constexpr uint32_t DX_OFF_A = DX_OFF_CH + DX_NCS * CH_BYTES;        // DX_NAB x (A tile, A o dA tile)
-constexpr uint32_t DX_OFF_DM = DX_OFF_A + DX_NAB * 2 * AT_BYTES;
+constexpr uint32_t DX_OFF_DM = DX_OFF_CH + DX_NCS * CH_BYTES;
 constexpr uint32_t DX_OFF_BAR = DX_OFF_DM + DX_NCS * KC * 4;
 constexpr uint32_t DX_SMEM = DX_OFF_BAR + 256 + 1024;
 constexpr int DX_THREADS = 192;              // warp 0 TMA, 1 MMA, 2-5 one thread per token
-constexpr uint32_t DX_TM_ZG = 0, DX_TM_VY = 128, DX_TM_W = 384;
+// TMEM columns: [Z|G] of the current chunk; V = A P'; Q = A dH + (ln2 A o dA) P';
+// two buffers of the chunk's A and ln2 A o dA as bf16 pairs (the TMEM operand
+// of the aggregation MMAs: 32 columns each).
+constexpr uint32_t DX_TM_ZG = 0, DX_TM_V = 128, DX_TM_Q = 256, DX_TM_AA = 384;
 
 struct DxBars {
-  uint64_t x_full[DX_NXS], x_empty[DX_NXS], c_full[DX_NCS], c_empty[DX_NCS];
-  uint64_t zg_full, zg_empty, a_full[DX_NAB], a_empty[DX_NAB], acc_full, acc_empty, mma_done;
+  // avq_done[s]: the aggregation MMAs of the chunk in stage s completed, so
+  // both its shared-memory stage and its TMEM A buffer are free again
+  uint64_t x_full[DX_NXS], x_empty[DX_NXS], c_full[DX_NCS], avq_done[DX_NCS];
+  uint64_t zg_full, zg_empty, aa_full[2], acc_full, mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -108,12 +104,11 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < DX_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
-    for (int s = 0; s < DX_NCS; ++s) { mbar_init(&bars->c_full[s], 1); mbar_init(&bars->c_empty[s], 1); }
+    for (int s = 0; s < DX_NCS; ++s) { mbar_init(&bars->c_full[s], 1); mbar_init(&bars->avq_done[s], 1); }
     mbar_init(&bars->zg_full, 1);
     mbar_init(&bars->zg_empty, 128);
-    for (int b = 0; b < DX_NAB; ++b) { mbar_init(&bars->a_full[b], 128); mbar_init(&bars->a_empty[b], 1); }
+    for (int b = 0; b < 2; ++b) mbar_init(&bars->aa_full[b], 128);
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_empty, 128);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -134,17 +129,32 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     prefetch_tensormap(&tmH);
     prefetch_tensormap(&tmL);
     int cc = 0, issued_t = 0, issued_c = 0;
-    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int u, int64_t tb, int64_t, bool, bool) {
-      const int s = t % DX_NXS;
-      if (t >= DX_NXS && !mbar_wait(&bars->x_empty[s], ((t / DX_NXS) - 1) & 1, abort, p.err)) return false;
-      mbar_arrive_expect_tx(&bars->x_full[s], XT_BYTES);
-      uint8_t* xd = smem + DX_OFF_X + s * XT_BYTES;
-      tma_load_2d(xd, &tmX, &bars->x_full[s], 0, (int)tb);
-      tma_load_2d(xd + XT_BYTES / 2, &tmX, &bars->x_full[s], 64, (int)tb);
-      issued_t = t + 1;
+    const int64_t n_total = p.off[p.B];
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int u, int64_t tb, int64_t pe, bool, bool) {
+      // the next X tile (in this user, else the next user's first rows) to L2
+      const int64_t nx = tb + TILE < pe ? tb + TILE : pe;
+      if (nx < n_total) {
+        tma_prefetch_l2_2d(&tmX, 0, (int)nx);
+        tma_prefetch_l2_2d(&tmX, 64, (int)nx);
+      }
+      auto load_x = [&]() -> bool {
+        const int s = t % DX_NXS;
+        if (t >= DX_NXS && !mbar_wait(&bars->x_empty[s], ((t / DX_NXS) - 1) & 1, abort, p.err)) return false;
+        mbar_arrive_expect_tx(&bars->x_full[s], XT_BYTES);
+        uint8_t* xd = smem + DX_OFF_X + s * XT_BYTES;
+        tma_load_2d(xd, &tmX, &bars->x_full[s], 0, (int)tb);
+        tma_load_2d(xd + XT_BYTES / 2, &tmX, &bars->x_full[s], 64, (int)tb);
+        issued_t = t + 1;
+        return true;
+      };
+      // Stages free up in the order the previous tile's MMAs complete: chunks
+      // nch-4 and nch-3 before the tile's X (its last logits MMA), the rest
+      // after; so this tile's first two chunks are loaded before its X.
+      const int x_at = std::min(2, nch);
       for (int c = 0; c < nch; ++c, ++cc) {
+        if (c == x_at && !load_x()) return false;
         const int cs = cc % DX_NCS;
-        if (cc >= DX_NCS && !mbar_wait(&bars->c_empty[cs], ((cc / DX_NCS) - 1) & 1, abort, p.err)) return false;
+        if (cc >= DX_NCS && !mbar_wait(&bars->avq_done[cs], ((cc / DX_NCS) - 1) & 1, abort, p.err)) return false;
         mbar_arrive_expect_tx(&bars->c_full[cs], CH_BYTES + KC * 4);
         uint8_t* cd = smem + DX_OFF_CH + cs * CH_BYTES;
         const int prow = c * KC, hrow = (int)((int64_t)u * p.k + c * KC);
@@ -157,6 +167,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
         bulk_load(smem + DX_OFF_DM + cs * KC * 4, p.dmc + (int64_t)u * p.k + c * KC, KC * 4, &bars->c_full[cs]);
         issued_c = cc + 1;
       }
+      if (x_at == nch && !load_x()) return false;
       return true;
     });
     if (*abort) {
@@ -168,33 +179,30 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     const uint32_t id_zg = idesc_bf16(128, 128, false, false);
-    const uint32_t id_vy = idesc_bf16(128, 256, false, true);
-    const uint32_t id_w = idesc_bf16(128, 128, false, true);
-    const uint32_t id_lo = idesc_bf16(128, 64, false, true);
+    const uint32_t id_acc = idesc_bf16(128, 128, false, true);   // A from TMEM, B MN-major
     int ai = 0;   // global chunk index
-    auto avw = [&](int a, int t, int s, bool first, bool last) -> bool {
-      const int cs = a % DX_NCS, b = a % DX_NAB;
-      if (!mbar_wait(&bars->a_full[b], (a / DX_NAB) & 1, abort, p.err)) return false;
-      if (first && t > 0 && !mbar_wait(&bars->acc_empty, (t - 1) & 1, abort, p.err)) return false;
+    // V += A P'_c;  Q += A dH_c (hi and lo parts) + (ln2 A o dA) P'_c
+    auto avq = [&](int a, bool first, bool last) -> bool {
+      const int cs = a % DX_NCS, b = a & 1;
+      // aa_full also implies that the epilogue of the previous tile has read V and
+      // Q: every thread finishes that epilogue before it writes this tile's A
+      if (!mbar_wait(&bars->aa_full[b], (a >> 1) & 1, abort, p.err)) return false;
       tc_fence_after();
-      const uint32_t at = smem_u32(smem + DX_OFF_A + b * 2 * AT_BYTES);
-      const uint32_t adt = at + AT_BYTES;
+      const uint32_t ta = tmem + DX_TM_AA + 64 * b;    // A in columns 0-31, ln2 A o dA in 32-63
       const uint32_t cb = smem_u32(smem + DX_OFF_CH + cs * CH_BYTES);
 #pragma unroll
       for (int ks = 0; ks < KC / 16; ++ks) {
         const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-        mma_ss(tmem + DX_TM_VY, smem_desc(at + ks * 32, 16, 1024, SWZ_128B),
-               smem_desc(cb + ks * 2048, 8192, 1024, SWZ_128B), id_vy, acc);
-        mma_ss(tmem + DX_TM_W, smem_desc(adt + ks * 32, 16, 1024, SWZ_128B),
-               smem_desc(cb + ks * 2048, 16384, 1024, SWZ_128B), id_w, acc);
-        // Y += A dH_lo: the bf16 residual of dH, so dH is carried to ~16 bits
-        mma_ss(tmem + DX_TM_VY + 64, smem_desc(at + ks * 32, 16, 1024, SWZ_128B),
-               smem_desc(cb + 32768 + ks * 2048, 8192, 1024, SWZ_128B), id_lo, 1u);
-        mma_ss(tmem + DX_TM_VY + 192, smem_desc(at + ks * 32, 16, 1024, SWZ_128B),
-               smem_desc(cb + 40960 + ks * 2048, 8192, 1024, SWZ_128B), id_lo, 1u);
+        const uint64_t bP = smem_desc(cb + ks * 2048, 16384, 1024, SWZ_128B);
+        mma_ts(tmem + DX_TM_V, ta + ks * 8, bP, id_acc, acc);
+        mma_ts(tmem + DX_TM_Q, ta + ks * 8, smem_desc(cb + 8192 + ks * 2048, 16384, 1024, SWZ_128B),
+               id_acc, acc);
+        // the bf16 residual of dH, so dH enters Q to ~16 bits
+        mma_ts(tmem + DX_TM_Q, ta + ks * 8, smem_desc(cb + 32768 + ks * 2048, 8192, 1024, SWZ_128B),
+               id_acc, 1u);
+        mma_ts(tmem + DX_TM_Q, ta + 32 + ks * 8, bP, id_acc, 1u);
       }
-      mma_commit(&bars->c_empty[cs]);
-      mma_commit(&bars->a_empty[b]);
+      mma_commit(&bars->avq_done[cs]);
       if (last) mma_commit(&bars->acc_full);
       return true;
     };
@@ -215,9 +223,9 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
                  ks > 0 ? 1u : 0u);
         mma_commit(&bars->zg_full);
         if (c == nch - 1) mma_commit(&bars->x_empty[s]);   // X is read by the logits MMAs only
-        if (c > 0 && !avw(a - 1, t, s, c - 1 == 0, false)) return false;
+        if (c > 0 && !avq(a - 1, c - 1 == 0, false)) return false;
       }
-      if (!avw(ai + nch - 1, t, s, nch == 1, true)) return false;
+      if (!avq(ai + nch - 1, nch == 1, true)) return false;
       ai += nch;
       return true;
     });
@@ -234,7 +242,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
       const float l2 = valid ? p.lse2[tb + row] : 0.f;
       float cacc = 0.f;
       for (int c = 0; c < nch; ++c) {
-        const int a = ai + c, cs = a % DX_NCS, b = a % DX_NAB;
+        const int a = ai + c, cs = a % DX_NCS, b = a & 1;
         if (!mbar_wait(&bars->zg_full, a & 1, abort, p.err)) return false;
         tc_fence_after();
         float z[64], gv[64];
@@ -247,9 +255,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
         mbar_arrive(&bars->zg_empty);
         if (!mbar_wait(&bars->c_full[cs], (a / DX_NCS) & 1, abort, p.err)) return false;
         const float4* dm4 = (const float4*)(smem + DX_OFF_DM + cs * KC * 4);
-        const uint32_t at = smem_u32(smem + DX_OFF_A + b * 2 * AT_BYTES);
-        const uint32_t adt = at + AT_BYTES;
-        uint32_t pa[32], pd[32];   // A and A o dA of the chunk, packed bf16 pairs
+        uint32_t pa[32], pd[32];   // A and ln2 A o dA of the chunk, bf16 pairs (even prototype low)
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) {
           const float4 d0 = dm4[2 * q8], d1 = dm4[2 * q8 + 1];
@@ -261,7 +267,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
             const float A = valid ? ex2(z[j] - l2) : 0.f;
             const float dA = gv[j] + dmv[i];
             av[i] = A;
-            adv[i] = A * dA;
+            adv[i] = kLn2f * (A * dA);
             cacc = fmaf(A, dA, cacc);
           }
 #pragma unroll
@@ -270,42 +276,38 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
             pd[4 * q8 + i] = pack_bf16x2(adv[2 * i], adv[2 * i + 1]);
           }
         }
-        if (a >= DX_NAB && !mbar_wait(&bars->a_empty[b], ((a / DX_NAB) - 1) & 1, abort, p.err)) return false;
-#pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) {
-          st_row_k_major(at, row, q8, pa[4 * q8], pa[4 * q8 + 1], pa[4 * q8 + 2], pa[4 * q8 + 3]);
-          st_row_k_major(adt, row, q8, pd[4 * q8], pd[4 * q8 + 1], pd[4 * q8 + 2], pd[4 * q8 + 3]);
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&bars->a_full[b]);
+        // TMEM A buffer b was last read by the aggregation MMAs of chunk a-2
+        if (a >= 2 && !mbar_wait(&bars->avq_done[(a - 2) % DX_NCS], ((a - 2) / DX_NCS) & 1, abort, p.err))
+          return false;
+        tc_fence_after();
+        tmem_st32(tmem + lane_addr + DX_TM_AA + 64 * b, pa);
+        tmem_st32(tmem + lane_addr + DX_TM_AA + 64 * b + 32, pd);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->aa_full[b]);
       }
       ai += nch;
-      // dX_t = Y + ln2 (W - c V)
+      // dX_t = Q - ln2 c_t V
       if (!mbar_wait(&bars->acc_full, t & 1, abort, p.err)) return false;
       tc_fence_after();
+      const float lc = kLn2f * cacc;
 #pragma unroll
       for (int qb = 0; qb < 4; ++qb) {
-        // columns of d block qb: V at VY + (qb/2)*128 + (qb%2)*32, Y 64 further, W at W + 32 qb
-        const uint32_t vcol = DX_TM_VY + (qb >> 1) * 128 + (qb & 1) * 32;
-        float v[32], y[32], w[32];
-        tmem_ld32(tmem + lane_addr + vcol, v);
-        tmem_ld32(tmem + lane_addr + vcol + 64, y);
-        tmem_ld32(tmem + lane_addr + DX_TM_W + 32 * qb, w);
+        float v[32], qv[32];
+        tmem_ld32(tmem + lane_addr + DX_TM_V + 32 * qb, v);
+        tmem_ld32(tmem + lane_addr + DX_TM_Q + 32 * qb, qv);
         tmem_wait_ld();
         if (valid) {
           uint32_t o[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2)
-            o[i / 2] = pack_bf16x2(y[i] + kLn2f * (w[i] - cacc * v[i]),
-                                   y[i + 1] + kLn2f * (w[i + 1] - cacc * v[i + 1]));
+            o[i / 2] = pack_bf16x2(fmaf(-lc, v[i], qv[i]), fmaf(-lc, v[i + 1], qv[i + 1]));
           uint4* dst = (uint4*)(p.dX + (tb + row) * DD + 32 * qb);
 #pragma unroll
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
       }
       if (valid) p.cout[tb + row] = cacc;
-      tc_fence_before();
-      mbar_arrive(&bars->acc_empty);
       return true;
     });
   }
