@@ -62,7 +62,8 @@ constexpr uint32_t DX_OFF_CH = DX_OFF_X + DX_NXS * XT_BYTES;
 constexpr uint32_t DX_OFF_DM = DX_OFF_CH + DX_NCS * CH_BYTES;
 constexpr uint32_t DX_OFF_BAR = DX_OFF_DM + DX_NCS * KC * 4;
 constexpr uint32_t DX_SMEM = DX_OFF_BAR + 256 + 1024;
-constexpr int DX_THREADS = 192;              // warp 0 TMA, 1 MMA, 2-5 one thread per token
+constexpr int DX_THREADS = 224;              // warp 0 TMA, 1 logits MMAs, 2-5 one thread per token,
+                                             // 6 aggregation MMAs
 // TMEM columns: [Z|G] of the current chunk; V = A P'; Q = A dH + (ln2 A o dA) P';
 // two buffers of the chunk's A and ln2 A o dA as bf16 pairs (the TMEM operand
 // of the aggregation MMAs: 32 columns each).
@@ -72,7 +73,7 @@ struct DxBars {
   // avq_done[s]: the aggregation MMAs of the chunk in stage s completed, so
   // both its shared-memory stage and its TMEM A buffer are free again
   uint64_t x_full[DX_NXS], x_empty[DX_NXS], c_full[DX_NCS], avq_done[DX_NCS];
-  uint64_t zg_full, zg_empty, aa_full[2], acc_full, mma_done;
+  uint64_t zg_full, zg_empty, aa_full[2], acc_full, mma_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -109,7 +110,8 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     mbar_init(&bars->zg_empty, 128);
     for (int b = 0; b < 2; ++b) mbar_init(&bars->aa_full[b], 128);
     mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->mma_done[0], 1);
+    mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -177,35 +179,9 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
         mbar_wait_bounded(&bars->c_full[c % DX_NCS], (c / DX_NCS) & 1);
     }
   } else if (warp == 1 && lane == 0) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ logits MMA issuer
     const uint32_t id_zg = idesc_bf16(128, 128, false, false);
-    const uint32_t id_acc = idesc_bf16(128, 128, false, true);   // A from TMEM, B MN-major
     int ai = 0;   // global chunk index
-    // V += A P'_c;  Q += A dH_c (hi and lo parts) + (ln2 A o dA) P'_c
-    auto avq = [&](int a, bool first, bool last) -> bool {
-      const int cs = a % DX_NCS, b = a & 1;
-      // aa_full also implies that the epilogue of the previous tile has read V and
-      // Q: every thread finishes that epilogue before it writes this tile's A
-      if (!mbar_wait(&bars->aa_full[b], (a >> 1) & 1, abort, p.err)) return false;
-      tc_fence_after();
-      const uint32_t ta = tmem + DX_TM_AA + 64 * b;    // A in columns 0-31, ln2 A o dA in 32-63
-      const uint32_t cb = smem_u32(smem + DX_OFF_CH + cs * CH_BYTES);
-#pragma unroll
-      for (int ks = 0; ks < KC / 16; ++ks) {
-        const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-        const uint64_t bP = smem_desc(cb + ks * 2048, 16384, 1024, SWZ_128B);
-        mma_ts(tmem + DX_TM_V, ta + ks * 8, bP, id_acc, acc);
-        mma_ts(tmem + DX_TM_Q, ta + ks * 8, smem_desc(cb + 8192 + ks * 2048, 16384, 1024, SWZ_128B),
-               id_acc, acc);
-        // the bf16 residual of dH, so dH enters Q to ~16 bits
-        mma_ts(tmem + DX_TM_Q, ta + ks * 8, smem_desc(cb + 32768 + ks * 2048, 8192, 1024, SWZ_128B),
-               id_acc, 1u);
-        mma_ts(tmem + DX_TM_Q, ta + 32 + ks * 8, bP, id_acc, 1u);
-      }
-      mma_commit(&bars->avq_done[cs]);
-      if (last) mma_commit(&bars->acc_full);
-      return true;
-    };
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
       const int s = t % DX_NXS;
       if (!mbar_wait(&bars->x_full[s], (t / DX_NXS) & 1, abort, p.err)) return false;
@@ -223,15 +199,50 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
                  ks > 0 ? 1u : 0u);
         mma_commit(&bars->zg_full);
         if (c == nch - 1) mma_commit(&bars->x_empty[s]);   // X is read by the logits MMAs only
-        if (c > 0 && !avq(a - 1, c - 1 == 0, false)) return false;
       }
-      if (!avq(ai + nch - 1, nch == 1, true)) return false;
       ai += nch;
       return true;
     });
-    mma_commit(&bars->mma_done);
-    mbar_wait_bounded(&bars->mma_done, 0);
-  } else if (warp >= 2) {
+    mma_commit(&bars->mma_done[0]);
+    mbar_wait_bounded(&bars->mma_done[0], 0);
+  } else if (warp == 6 && lane == 0) {
+    // ------------------------------------------------------------ aggregation MMA issuer
+    // A thread of its own, so its waits overlap the logits thread's issue and
+    // the other way round.  The two threads' MMAs share no TMEM columns.
+    const uint32_t id_acc = idesc_bf16(128, 128, false, true);   // A from TMEM, B MN-major
+    int ai = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int, int, int, int64_t, int64_t, bool, bool) {
+      for (int c = 0; c < nch; ++c) {
+        const int a = ai + c, cs = a % DX_NCS, b = a & 1;
+        // aa_full also implies that the epilogue of the previous tile has read V and
+        // Q: every thread finishes that epilogue before it writes this tile's A
+        if (!mbar_wait(&bars->c_full[cs], (a / DX_NCS) & 1, abort, p.err)) return false;
+        if (!mbar_wait(&bars->aa_full[b], (a >> 1) & 1, abort, p.err)) return false;
+        tc_fence_after();
+        const uint32_t ta = tmem + DX_TM_AA + 64 * b;    // A in columns 0-31, ln2 A o dA in 32-63
+        const uint32_t cb = smem_u32(smem + DX_OFF_CH + cs * CH_BYTES);
+        // V += A P'_c;  Q += A dH_c (hi and lo parts) + (ln2 A o dA) P'_c
+#pragma unroll
+        for (int ks = 0; ks < KC / 16; ++ks) {
+          const uint32_t acc = (c == 0 && ks == 0) ? 0u : 1u;
+          const uint64_t bP = smem_desc(cb + ks * 2048, 16384, 1024, SWZ_128B);
+          mma_ts(tmem + DX_TM_V, ta + ks * 8, bP, id_acc, acc);
+          mma_ts(tmem + DX_TM_Q, ta + ks * 8, smem_desc(cb + 8192 + ks * 2048, 16384, 1024, SWZ_128B),
+                 id_acc, acc);
+          // the bf16 residual of dH, so dH enters Q to ~16 bits
+          mma_ts(tmem + DX_TM_Q, ta + ks * 8, smem_desc(cb + 32768 + ks * 2048, 8192, 1024, SWZ_128B),
+                 id_acc, 1u);
+          mma_ts(tmem + DX_TM_Q, ta + 32 + ks * 8, bP, id_acc, 1u);
+        }
+        mma_commit(&bars->avq_done[cs]);
+        if (c == nch - 1) mma_commit(&bars->acc_full);
+      }
+      ai += nch;
+      return true;
+    });
+    mma_commit(&bars->mma_done[1]);
+    mbar_wait_bounded(&bars->mma_done[1], 0);
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ one thread per token
     const int q = warp % 4;
     const int row = q * 32 + lane;
