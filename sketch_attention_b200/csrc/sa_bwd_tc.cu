@@ -339,7 +339,10 @@ constexpr uint32_t E_OFF_DZ = E_OFF_X + E_NXS * XT_BYTES;   // 2 x [128 protos x
 constexpr uint32_t E_OFF_DM = E_OFF_DZ + 2 * 32768;
 constexpr uint32_t E_OFF_BAR = E_OFF_DM + TILE * 4;
 constexpr uint32_t E_SMEM = E_OFF_BAR + 256 + 1024;
-constexpr int E_THREADS = 192;
+// warp 0 TMA, 1 MMA, 2-5 and 6-9: two warpgroups, group h computing dZ for the
+// prototypes 64h..64h+63 of the slice (so each reads its half of [Z|G] at once
+// and the next tile's logits MMA overlaps all of the dZ work)
+constexpr int E_THREADS = 320;
 constexpr uint32_t E_TM_ZG = 0, E_TM_E = 256;
 
 struct EBars {
@@ -361,7 +364,7 @@ struct EParams {
   int* err;
 };
 
-__global__ void __launch_bounds__(E_THREADS, 1)
+__global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 warps per sub-partition)
     sa_bwd_e_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                        const __grid_constant__ CUtensorMap tmH, EParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -376,11 +379,11 @@ __global__ void __launch_bounds__(E_THREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->p_full, 1);
     mbar_init(&bars->h_full, 1);
-    mbar_init(&bars->h_empty, 1 + 128);      // the last zg of a piece, and the threads done with its dm
+    mbar_init(&bars->h_empty, 1 + 256);      // the last zg of a piece, and the threads done with its dm
     for (int s = 0; s < E_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
     mbar_init(&bars->zg_full, 1);
-    mbar_init(&bars->zg_empty, 128);
-    for (int b = 0; b < 2; ++b) { mbar_init(&bars->dz_full[b], 128); mbar_init(&bars->dz_empty[b], 1); }
+    mbar_init(&bars->zg_empty, 256);
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->dz_full[b], 256); mbar_init(&bars->dz_empty[b], 1); }
     mbar_init(&bars->e_full, 1);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -473,7 +476,7 @@ __global__ void __launch_bounds__(E_THREADS, 1)
     mma_commit(&bars->mma_done);
     mbar_wait_bounded(&bars->mma_done, 0);
   } else if (warp >= 2) {
-    const int q = warp % 4;
+    const int q = warp % 4, h = (warp - 2) / 4;
     const int row = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     bool ok = true;
@@ -485,21 +488,18 @@ __global__ void __launch_bounds__(E_THREADS, 1)
       if (!mbar_wait(&bars->zg_full, t & 1, abort, p.err)) return ok = false;
       tc_fence_after();
       const int b = t & 1;
-      if (t >= 2 && !mbar_wait(&bars->dz_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return ok = false;
       const uint32_t dz = smem_u32(smem + E_OFF_DZ + b * 32768) + row * 128;
       const float4* dm4 = (const float4*)(smem + E_OFF_DM);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      {
         float z[64], gv[64];
         tmem_ld32(tmem + lane_addr + E_TM_ZG + 64 * h, z);
         tmem_ld32(tmem + lane_addr + E_TM_ZG + 64 * h + 32, z + 32);
         tmem_ld32(tmem + lane_addr + E_TM_ZG + 128 + 64 * h, gv);
         tmem_ld32(tmem + lane_addr + E_TM_ZG + 128 + 64 * h + 32, gv + 32);
         tmem_wait_ld();
-        if (h == 1) {
-          tc_fence_before();
-          mbar_arrive(&bars->zg_empty);
-        }
+        tc_fence_before();
+        mbar_arrive(&bars->zg_empty);
+        if (t >= 2 && !mbar_wait(&bars->dz_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return ok = false;
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
           const float4 d0 = dm4[16 * h + 2 * c8], d1 = dm4[16 * h + 2 * c8 + 1];
@@ -526,7 +526,7 @@ __global__ void __launch_bounds__(E_THREADS, 1)
       tc_fence_after();
       float* dst = p.Epart + ((int64_t)g * p.k + sl * TILE + row) * DD;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * h; c < 2 * h + 2; ++c) {
         float v[32];
         tmem_ld32(tmem + lane_addr + E_TM_E + 32 * c, v);
         tmem_wait_ld();
