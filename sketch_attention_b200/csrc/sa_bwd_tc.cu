@@ -250,8 +250,10 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     int ai = 0;
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t pe, bool, bool) {
       const bool valid = tb + row < pe;
-      const float l2 = valid ? p.lse2[tb + row] : 0.f;
-      float cacc = 0.f;
+      // a padding row gets lse = +inf, so its A = 2^(z - inf) = 0 without a select
+      const float l2 = valid ? p.lse2[tb + row] : __builtin_huge_valf();
+      const float2 nl2 = make_float2(-l2, -l2), ln2v = make_float2(kLn2f, kLn2f);
+      float2 c2 = make_float2(0.f, 0.f);   // c_t, as two partial sums (even / odd prototypes)
       for (int c = 0; c < nch; ++c) {
         const int a = ai + c, cs = a % DX_NCS, b = a & 1;
         if (!mbar_wait(&bars->zg_full, a & 1, abort, p.err)) return false;
@@ -267,24 +269,22 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
         if (!mbar_wait(&bars->c_full[cs], (a / DX_NCS) & 1, abort, p.err)) return false;
         const float4* dm4 = (const float4*)(smem + DX_OFF_DM + cs * KC * 4);
         uint32_t pa[32], pd[32];   // A and ln2 A o dA of the chunk, bf16 pairs (even prototype low)
+        // two prototypes per instruction (packed fp32x2 add / mul / fma)
 #pragma unroll
         for (int q8 = 0; q8 < 8; ++q8) {
           const float4 d0 = dm4[2 * q8], d1 = dm4[2 * q8 + 1];
-          const float dmv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-          float av[8], adv[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int j = q8 * 8 + i;
-            const float A = valid ? ex2(z[j] - l2) : 0.f;
-            const float dA = gv[j] + dmv[i];
-            av[i] = A;
-            adv[i] = kLn2f * (A * dA);
-            cacc = fmaf(A, dA, cacc);
-          }
+          const float2 dmp[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
+                                 make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            pa[4 * q8 + i] = pack_bf16x2(av[2 * i], av[2 * i + 1]);
-            pd[4 * q8 + i] = pack_bf16x2(adv[2 * i], adv[2 * i + 1]);
+            const int j = q8 * 8 + 2 * i;
+            const float2 e = __fadd2_rn(make_float2(z[j], z[j + 1]), nl2);
+            const float2 A = make_float2(ex2(e.x), ex2(e.y));
+            const float2 dA = __fadd2_rn(make_float2(gv[j], gv[j + 1]), dmp[i]);
+            c2 = __ffma2_rn(A, dA, c2);
+            const float2 ad = __fmul2_rn(__fmul2_rn(A, dA), ln2v);
+            pa[4 * q8 + i] = pack_bf16x2(A.x, A.y);
+            pd[4 * q8 + i] = pack_bf16x2(ad.x, ad.y);
           }
         }
         // TMEM A buffer b was last read by the aggregation MMAs of chunk a-2
@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
       // dX_t = Q - ln2 c_t V
       if (!mbar_wait(&bars->acc_full, t & 1, abort, p.err)) return false;
       tc_fence_after();
+      const float cacc = c2.x + c2.y;
       const float lc = kLn2f * cacc;
 #pragma unroll
       for (int qb = 0; qb < 4; ++qb) {
@@ -482,8 +483,10 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     bool ok = true;
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t tb, int64_t pe, bool first, bool last) {
       const bool valid = tb + row < pe;
-      const float l2 = valid ? p.lse2[tb + row] : 0.f;
+      // a padding row gets lse = +inf, so its A = 2^(z - inf) = 0 without a select
+      const float l2 = valid ? p.lse2[tb + row] : __builtin_huge_valf();
       const float ct = valid ? p.cin[tb + row] : 0.f;
+      const float2 nl2 = make_float2(-l2, -l2), nct = make_float2(-ct, -ct);
       if (first && !mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return ok = false;
       if (!mbar_wait(&bars->zg_full, t & 1, abort, p.err)) return ok = false;
       tc_fence_after();
@@ -500,21 +503,24 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
         tc_fence_before();
         mbar_arrive(&bars->zg_empty);
         if (t >= 2 && !mbar_wait(&bars->dz_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return ok = false;
+        // two prototypes per instruction (packed fp32x2 add / mul)
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
           const float4 d0 = dm4[16 * h + 2 * c8], d1 = dm4[16 * h + 2 * c8 + 1];
-          const float dmv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
-          float dzv[8];
+          const float2 dmp[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
+                                 make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
+          uint32_t o[4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int j = c8 * 8 + i;
-            const float A = valid ? ex2(z[j] - l2) : 0.f;
-            dzv[i] = A * (gv[j] + dmv[i] - ct);
+          for (int i = 0; i < 4; ++i) {
+            const int j = c8 * 8 + 2 * i;
+            const float2 e = __fadd2_rn(make_float2(z[j], z[j + 1]), nl2);
+            const float2 A = make_float2(ex2(e.x), ex2(e.y));
+            const float2 dA = __fadd2_rn(make_float2(gv[j], gv[j + 1]), dmp[i]);
+            const float2 dzv = __fmul2_rn(A, __fadd2_rn(dA, nct));
+            o[i] = pack_bf16x2(dzv.x, dzv.y);
           }
           // MN-major SW128 A operand of E += dZ^T X: M-block h, token row `row`
-          st_shared_v4(dz + h * 16384 + ((c8 ^ (row & 7)) << 4), pack_bf16x2(dzv[0], dzv[1]),
-                       pack_bf16x2(dzv[2], dzv[3]), pack_bf16x2(dzv[4], dzv[5]),
-                       pack_bf16x2(dzv[6], dzv[7]));
+          st_shared_v4(dz + h * 16384 + ((c8 ^ (row & 7)) << 4), o[0], o[1], o[2], o[3]);
         }
       }
       fence_proxy_async_smem();
