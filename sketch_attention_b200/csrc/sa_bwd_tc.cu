@@ -60,10 +60,11 @@ constexpr uint32_t CH_BYTES = 49152;         // [P' h0 | dH h0 | P' h1 | dH h1 |
 constexpr uint32_t DX_OFF_X = 0;
 constexpr uint32_t DX_OFF_CH = DX_OFF_X + DX_NXS * XT_BYTES;
 constexpr uint32_t DX_OFF_DM = DX_OFF_CH + DX_NCS * CH_BYTES;
-constexpr uint32_t DX_OFF_BAR = DX_OFF_DM + DX_NCS * KC * 4;
+constexpr uint32_t DX_OFF_CP = DX_OFF_DM + DX_NCS * KC * 4;      // [128] partial c of warpgroup 1
+constexpr uint32_t DX_OFF_BAR = DX_OFF_CP + TILE * 4;
 constexpr uint32_t DX_SMEM = DX_OFF_BAR + 256 + 1024;
-constexpr int DX_THREADS = 224;              // warp 0 TMA, 1 logits MMAs, 2-5 one thread per token,
-                                             // 6 aggregation MMAs
+constexpr int DX_THREADS = 352;              // warp 0 TMA, 1 logits MMAs, 2-9 two threads per
+                                             // token, 10 aggregation MMAs
 // TMEM columns: [Z|G] of the current chunk; V = A P'; Q = A dH + (ln2 A o dA) P';
 // two buffers of the chunk's A and ln2 A o dA as bf16 pairs (the TMEM operand
 // of the aggregation MMAs: 32 columns each).
@@ -73,7 +74,7 @@ struct DxBars {
   // avq_done[s]: the aggregation MMAs of the chunk in stage s completed, so
   // both its shared-memory stage and its TMEM A buffer are free again
   uint64_t x_full[DX_NXS], x_empty[DX_NXS], c_full[DX_NCS], avq_done[DX_NCS];
-  uint64_t zg_full, zg_empty, aa_full[2], acc_full, mma_done[2];
+  uint64_t zg_full, zg_empty, aa_full[2], acc_full, cx_full, cx_empty, mma_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -90,7 +91,8 @@ struct DxParams {
   int* err;
 };
 
-__global__ void __launch_bounds__(DX_THREADS, 1)
+// 384: caps registers at 168, as three warps share two of the SM's sub-partitions
+__global__ void __launch_bounds__(384, 1)
     sa_bwd_dx_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                         const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmL,
                         DxParams p) {
@@ -107,8 +109,10 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     for (int s = 0; s < DX_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
     for (int s = 0; s < DX_NCS; ++s) { mbar_init(&bars->c_full[s], 1); mbar_init(&bars->avq_done[s], 1); }
     mbar_init(&bars->zg_full, 1);
-    mbar_init(&bars->zg_empty, 128);
-    for (int b = 0; b < 2; ++b) mbar_init(&bars->aa_full[b], 128);
+    mbar_init(&bars->zg_empty, 256);
+    for (int b = 0; b < 2; ++b) mbar_init(&bars->aa_full[b], 256);
+    mbar_init(&bars->cx_full, 128);
+    mbar_init(&bars->cx_empty, 128);
     mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->mma_done[0], 1);
     mbar_init(&bars->mma_done[1], 1);
@@ -205,7 +209,7 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     });
     mma_commit(&bars->mma_done[0]);
     mbar_wait_bounded(&bars->mma_done[0], 0);
-  } else if (warp == 6 && lane == 0) {
+  } else if (warp == 10 && lane == 0) {
     // ------------------------------------------------------------ aggregation MMA issuer
     // A thread of its own, so its waits overlap the logits thread's issue and
     // the other way round.  The two threads' MMAs share no TMEM columns.
@@ -242,36 +246,37 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
     });
     mma_commit(&bars->mma_done[1]);
     mbar_wait_bounded(&bars->mma_done[1], 0);
-  } else if (warp >= 2 && warp <= 5) {
-    // ------------------------------------------------------------ one thread per token
-    const int q = warp % 4;
+  } else if (warp >= 2 && warp <= 9) {
+    // ------------------------------------------------------------ two threads per token
+    // Warpgroup h (warps 2-5: h = 0, 6-9: h = 1) owns prototypes 32h..32h+31 of every
+    // chunk; its partial c_t is handed to warpgroup 0, which writes dX and c.
+    const int q = warp % 4, h = (warp - 2) / 4;
     const int row = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    float* cpart = (float*)(smem + DX_OFF_CP);
     int ai = 0;
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t pe, bool, bool) {
       const bool valid = tb + row < pe;
       // a padding row gets lse = +inf, so its A = 2^(z - inf) = 0 without a select
       const float l2 = valid ? p.lse2[tb + row] : __builtin_huge_valf();
       const float2 nl2 = make_float2(-l2, -l2), ln2v = make_float2(kLn2f, kLn2f);
-      float2 c2 = make_float2(0.f, 0.f);   // c_t, as two partial sums (even / odd prototypes)
+      float2 c2 = make_float2(0.f, 0.f);   // partial c_t (even / odd prototypes)
       for (int c = 0; c < nch; ++c) {
         const int a = ai + c, cs = a % DX_NCS, b = a & 1;
         if (!mbar_wait(&bars->zg_full, a & 1, abort, p.err)) return false;
         tc_fence_after();
-        float z[64], gv[64];
-        tmem_ld32(tmem + lane_addr + DX_TM_ZG, z);
-        tmem_ld32(tmem + lane_addr + DX_TM_ZG + 32, z + 32);
-        tmem_ld32(tmem + lane_addr + DX_TM_ZG + 64, gv);
-        tmem_ld32(tmem + lane_addr + DX_TM_ZG + 96, gv + 32);
+        float z[32], gv[32];
+        tmem_ld32(tmem + lane_addr + DX_TM_ZG + 32 * h, z);
+        tmem_ld32(tmem + lane_addr + DX_TM_ZG + 64 + 32 * h, gv);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->zg_empty);
         if (!mbar_wait(&bars->c_full[cs], (a / DX_NCS) & 1, abort, p.err)) return false;
-        const float4* dm4 = (const float4*)(smem + DX_OFF_DM + cs * KC * 4);
-        uint32_t pa[32], pd[32];   // A and ln2 A o dA of the chunk, bf16 pairs (even prototype low)
+        const float4* dm4 = (const float4*)(smem + DX_OFF_DM + cs * KC * 4) + 8 * h;
+        uint32_t pa[16], pd[16];   // A and ln2 A o dA, bf16 pairs (even prototype low)
         // two prototypes per instruction (packed fp32x2 add / mul / fma)
 #pragma unroll
-        for (int q8 = 0; q8 < 8; ++q8) {
+        for (int q8 = 0; q8 < 4; ++q8) {
           const float4 d0 = dm4[2 * q8], d1 = dm4[2 * q8 + 1];
           const float2 dmp[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
                                  make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
@@ -291,17 +296,27 @@ __global__ void __launch_bounds__(DX_THREADS, 1)
         if (a >= 2 && !mbar_wait(&bars->avq_done[(a - 2) % DX_NCS], ((a - 2) / DX_NCS) & 1, abort, p.err))
           return false;
         tc_fence_after();
-        tmem_st32(tmem + lane_addr + DX_TM_AA + 64 * b, pa);
-        tmem_st32(tmem + lane_addr + DX_TM_AA + 64 * b + 32, pd);
+        tmem_st16(tmem + lane_addr + DX_TM_AA + 64 * b + 16 * h, pa);
+        tmem_st16(tmem + lane_addr + DX_TM_AA + 64 * b + 32 + 16 * h, pd);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars->aa_full[b]);
       }
       ai += nch;
+      float cacc = c2.x + c2.y;
+      if (h == 1) {
+        // hand the partial c to warpgroup 0 (the slot is free once it has read the last one)
+        if (t > 0 && !mbar_wait(&bars->cx_empty, (t - 1) & 1, abort, p.err)) return false;
+        cpart[row] = cacc;
+        mbar_arrive(&bars->cx_full);
+        return true;
+      }
+      if (!mbar_wait(&bars->cx_full, t & 1, abort, p.err)) return false;
+      cacc += cpart[row];
+      mbar_arrive(&bars->cx_empty);
       // dX_t = Q - ln2 c_t V
       if (!mbar_wait(&bars->acc_full, t & 1, abort, p.err)) return false;
       tc_fence_after();
-      const float cacc = c2.x + c2.y;
       const float lc = kLn2f * cacc;
 #pragma unroll
       for (int qb = 0; qb < 4; ++qb) {
