@@ -28,7 +28,14 @@
 #include <mutex>
 
 #include "sa_internal.cuh"
+#include "exp2_poly.cuh"
 #include "tc_ptx.cuh"
+
+// Pairs (of the 4 in a group of 8 prototypes) whose exponentials the E kernel
+// evaluates on the FMA pipe instead of the MUFU.
+#ifndef SA_E_POLY_PAIRS
+#define SA_E_POLY_PAIRS 0x2
+#endif
 
 namespace sa {
 
@@ -529,7 +536,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
           for (int i = 0; i < 4; ++i) {
             const int j = c8 * 8 + 2 * i;
             const float2 e = __fadd2_rn(make_float2(z[j], z[j + 1]), nl2);
-            const float2 A = make_float2(ex2(e.x), ex2(e.y));
+            const float2 A = ((SA_E_POLY_PAIRS >> i) & 1) ? exp2_poly2(e) : make_float2(ex2(e.x), ex2(e.y));
             const float2 dA = __fadd2_rn(make_float2(gv[j], gv[j + 1]), dmp[i]);
             const float2 dzv = __fmul2_rn(A, __fadd2_rn(dA, nct));
             o[i] = pack_bf16x2(dzv.x, dzv.y);

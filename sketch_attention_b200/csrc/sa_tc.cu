@@ -242,7 +242,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t sbuf = tmem + lane_addr + (b ? TM_S1 : TM_S0);
           uint32_t ep[64];
           float mc[8];
-          float m = -__builtin_huge_valf(), s = 0.f;
+          float m = -__builtin_huge_valf();
+          float2 s2 = make_float2(0.f, 0.f);   // running sum, as two partial sums
           float zbuf[2][16];
           tmem_ld16(sbuf, zbuf[0]);
           tmem_wait_ld16(zbuf[0]);
@@ -254,15 +255,18 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int j = 1; j < 16; ++j) cm = fmaxf(cm, z[j]);
             const float mn = fmaxf(m, cm);
-            s *= ex2(m - mn);
+            const float sc = ex2(m - mn);
+            s2 = __fmul2_rn(s2, make_float2(sc, sc));
             m = mn;
             mc[c] = mn;
-            const float off = 8.f - mn;
+            const float2 off = make_float2(8.f - mn, 8.f - mn);
+            // two logits per instruction (packed fp32x2 add)
 #pragma unroll
             for (int j = 0; j < 16; j += 2) {
-              const float e0 = ex2(z[j] + off), e1 = ex2(z[j + 1] + off);
-              s += e0 + e1;
-              ep[8 * c + j / 2] = pack_f16x2(e0, e1);
+              const float2 zz = __fadd2_rn(make_float2(z[j], z[j + 1]), off);
+              const float2 e = make_float2(ex2(zz.x), ex2(zz.y));
+              s2 = __fadd2_rn(s2, e);
+              ep[8 * c + j / 2] = pack_f16x2(e.x, e.y);
             }
             if (c < 7) tmem_wait_ld16(zbuf[(c + 1) & 1]);
             if (c == 6) {
@@ -270,7 +274,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               mbar_arrive(&bars->s_empty[b]);
             }
           }
-          const float l = valid ? m + lg2(s) - 8.f : -__builtin_huge_valf();
+          const float l = valid ? m + lg2(s2.x + s2.y) - 8.f : -__builtin_huge_valf();
           // this CTA's log2-sum-exp of every token goes into its own row of the
           // exchange slot, and from there to the same row in every other CTA
           const int slot = t & 3;
@@ -303,13 +307,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t pa = smem_u32(smem + OFF_P) + row * 128;
 #pragma unroll
           for (int cc = 0; cc < 16; ++cc) {           // 16-byte chunks of 8 prototypes
-            const float r = rc[cc >> 1];
+            const float2 r = make_float2(rc[cc >> 1], rc[cc >> 1]);
             const uint32_t* e4 = ep + 4 * cc;
-            const float2 a0 = unpack_f16x2(e4[0]), a1 = unpack_f16x2(e4[1]);
-            const float2 a2 = unpack_f16x2(e4[2]), a3 = unpack_f16x2(e4[3]);
+            const float2 a0 = __fmul2_rn(unpack_f16x2(e4[0]), r), a1 = __fmul2_rn(unpack_f16x2(e4[1]), r);
+            const float2 a2 = __fmul2_rn(unpack_f16x2(e4[2]), r), a3 = __fmul2_rn(unpack_f16x2(e4[3]), r);
             st_shared_v4(pa + (cc >> 3) * 16384 + (((cc & 7) ^ (row & 7)) << 4),
-                         pack_bf16x2(a0.x * r, a0.y * r), pack_bf16x2(a1.x * r, a1.y * r),
-                         pack_bf16x2(a2.x * r, a2.y * r), pack_bf16x2(a3.x * r, a3.y * r));
+                         pack_bf16x2(a0.x, a0.y), pack_bf16x2(a1.x, a1.y),
+                         pack_bf16x2(a2.x, a2.y), pack_bf16x2(a3.x, a3.y));
           }
           fence_proxy_async_smem();
           tc_fence_before();
