@@ -1,6 +1,11 @@
-// Tiled SIMT fp32 GEMM: 64 x 64 output tile per CTA, 16-deep k slices staged
-// through shared memory, 4 x 4 outputs per thread.  Arbitrary sizes, strides,
-// transposes and batch; used only for the small projection GEMMs.
+// Tiled SIMT fp32 GEMM: a BM x BN output tile per CTA (BN = 32 when N <= 32,
+// else 64; BM = 64 when 128-row tiles would leave the SMs short of CTAs, else
+// 128), 8 x 4 outputs per thread read from shared memory as float4.  The
+// 16-deep k slices stream through NS shared-memory stages with asynchronous
+// element copies (zero-filled past the edges), NS - 1 slices ahead of the
+// multiply, so global latency is paid about once per CTA rather than once per
+// slice.  Arbitrary sizes, strides, transposes and batch; used only for the
+// small projection GEMMs.
 #include <algorithm>
 
 #include "gemm.cuh"
@@ -8,73 +13,102 @@
 namespace sa {
 
 namespace {
-constexpr int TM = 64, TN = 64, TK = 16;
+constexpr int BK = 16, RM = 8, RN = 4, NS = 3;
 
-__global__ void __launch_bounds__(256) gemm_kernel(Gemm g) {
-  __shared__ float As[TK][TM + 4];
-  __shared__ float Bs[TK][TN + 4];
+__device__ __forceinline__ void cp_async4(float* dst, const float* src, bool pred) {
+  // 4-byte asynchronous copy; with pred false nothing is read and zero is written
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(pred ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// TA / TB: A stored [K, M] / B stored [N, K] (compile-time, so each variant's
+// unrolled copy loops stay small in the instruction cache)
+template <int BM, int BN, bool TA, bool TB>
+__global__ void __launch_bounds__((BM / RM) * (BN / RN), 2) gemm_kernel(Gemm g) {
+  constexpr int NT = (BM / RM) * (BN / RN);
+  constexpr int LA = BM * BK / NT, LB = BK * BN / NT;     // elements copied per thread per slice
+  __shared__ __align__(16) float As[NS][BK][BM + 4];
+  __shared__ __align__(16) float Bs[NS][BK][BN + 4];
   const int b = blockIdx.z / g.split_k, sk = blockIdx.z % g.split_k;
-  const int kper = ((g.K + g.split_k - 1) / g.split_k + TK - 1) / TK * TK;
+  const int kper = ((g.K + g.split_k - 1) / g.split_k + BK - 1) / BK * BK;
   const int kbeg = sk * kper, kend = min(g.K, kbeg + kper);
+  const int nsl = kend > kbeg ? (kend - kbeg + BK - 1) / BK : 0;
   const float* A = g.A + (int64_t)b * g.sA;
   const float* Bm = g.B + (int64_t)b * g.sB;
-  const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4] = {};
-  for (int k0 = kbeg; k0 < kend; k0 += TK) {
-    // 64 x 16 of A and 16 x 64 of B, 4 elements of each per thread.
-    for (int e = threadIdx.x; e < TM * TK; e += 256) {
-      int mm, kk;
-      if (g.transA) { mm = e % TM; kk = e / TM; } else { kk = e % TK; mm = e / TK; }
-      int m = m0 + mm, k = k0 + kk;
-      float v = 0.f;
-      if (m < g.M && k < kend) v = g.transA ? A[(int64_t)k * g.lda + m] : A[(int64_t)m * g.lda + k];
-      As[kk][mm] = v;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int tx = threadIdx.x % (BN / RN), ty = threadIdx.x / (BN / RN);
+  float acc[RM][RN] = {};
+  // element e = threadIdx.x + NT * l of a slice; the operand's contiguous index
+  // runs fastest across threads (coalesced global reads)
+  auto issue = [&](int sl) {
+    if (sl < nsl) {
+      const int k0 = kbeg + sl * BK, st = sl % NS;
+#pragma unroll
+      for (int l = 0; l < LA; ++l) {
+        const int e = threadIdx.x + NT * l;
+        int mm, kk;
+        if (TA) { mm = e % BM; kk = e / BM; } else { kk = e % BK; mm = e / BK; }
+        const int m = m0 + mm, k = k0 + kk;
+        const bool ok = m < g.M && k < kend;
+        cp_async4(&As[st][kk][mm], ok ? (TA ? A + (int64_t)k * g.lda + m : A + (int64_t)m * g.lda + k) : A, ok);
+      }
+#pragma unroll
+      for (int l = 0; l < LB; ++l) {
+        const int e = threadIdx.x + NT * l;
+        int nn, kk;
+        if (TB) { kk = e % BK; nn = e / BK; } else { nn = e % BN; kk = e / BN; }
+        const int n = n0 + nn, k = k0 + kk;
+        const bool ok = n < g.N && k < kend;
+        cp_async4(&Bs[st][kk][nn], ok ? (TB ? Bm + (int64_t)n * g.ldb + k : Bm + (int64_t)k * g.ldb + n) : Bm, ok);
+      }
     }
-    for (int e = threadIdx.x; e < TN * TK; e += 256) {
-      int nn, kk;
-      if (g.transB) { kk = e % TK; nn = e / TK; } else { nn = e % TN; kk = e / TN; }
-      int n = n0 + nn, k = k0 + kk;
-      float v = 0.f;
-      if (n < g.N && k < kend) v = g.transB ? Bm[(int64_t)n * g.ldb + k] : Bm[(int64_t)k * g.ldb + n];
-      Bs[kk][nn] = v;
+    cp_async_commit();   // one group per slice index, empty past the end
+  };
+#pragma unroll
+  for (int sl = 0; sl < NS - 1; ++sl) issue(sl);
+  for (int sl = 0; sl < nsl; ++sl) {
+    cp_async_wait<NS - 2>();   // slice sl has landed (this thread's copies)
+    __syncthreads();           // ... everyone's; and stage (sl - 1) % NS is no longer read
+    issue(sl + NS - 1);
+    const int st = sl % NS;
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      const float4 a0 = *(const float4*)&As[st][kk][ty * RM];
+      const float4 a1 = *(const float4*)&As[st][kk][ty * RM + 4];
+      const float4 b0 = *(const float4*)&Bs[st][kk][tx * RN];
+      const float av[RM] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[RN] = {b0.x, b0.y, b0.z, b0.w};
+#pragma unroll
+      for (int i = 0; i < RM; ++i)
+#pragma unroll
+        for (int j = 0; j < RN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < TK; ++kk) {
-      float a[4], bb[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) bb[j] = Bs[kk][tx + 16 * j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
-    }
-    __syncthreads();
   }
+  cp_async_wait<0>();
   if (g.split_k > 1) {
     float* part = g.split_ws + (int64_t)blockIdx.z * g.M * g.N;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int m = m0 + ty + 16 * i;
+    for (int i = 0; i < RM; ++i) {
+      const int m = m0 + ty * RM + i;
       if (m >= g.M) continue;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int n = n0 + tx + 16 * j;
+      for (int j = 0; j < RN; ++j) {
+        const int n = n0 + tx * RN + j;
         if (n < g.N) part[(int64_t)m * g.N + n] = acc[i][j];
       }
     }
     return;
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    int m = m0 + ty + 16 * i;
+  for (int i = 0; i < RM; ++i) {
+    const int m = m0 + ty * RM + i;
     if (m >= g.M) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      int n = n0 + tx + 16 * j;
+    for (int j = 0; j < RN; ++j) {
+      const int n = n0 + tx * RN + j;
       if (n >= g.N) continue;
       float v = g.alpha * acc[i][j];
       if (g.bias) v += g.bias[n];
@@ -104,8 +138,11 @@ __global__ void gemm_split_reduce_kernel(Gemm g) {
 }  // namespace
 
 int gemm_split_for(int M, int N, int K, int max_split) {
-  const int tiles = ((M + TM - 1) / TM) * ((N + TN - 1) / TN);
-  int s = std::min((K + 511) / 512, std::max(1, 296 / std::max(tiles, 1)));
+  // enough CTAs for about three per SM, and at least four 16-deep k slices per CTA
+  const int bn = N <= 32 ? 32 : 64;
+  const int tiles = std::max(1, ((M + 127) / 128) * ((N + bn - 1) / bn));
+  const int target = 3 * device_info().sm_count;
+  int s = std::min((K + 63) / 64, (target + tiles - 1) / tiles);
   return std::max(1, std::min(s, max_split));
 }
 
@@ -113,8 +150,38 @@ sa_status gemm(const Gemm& g0, cudaStream_t stream) {
   if (g0.M <= 0 || g0.N <= 0 || g0.batch <= 0) return SA_OK;
   Gemm g = g0;
   if (g.split_k < 1 || !g.split_ws) g.split_k = 1;
-  dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, g.batch * g.split_k);
-  SA_TIMED(g.tag ? g.tag : "gemm_kernel", stream, (gemm_kernel<<<grid, 256, 0, stream>>>(g)));
+  const char* tag = g.tag ? g.tag : "gemm_kernel";
+  const int bn = g.N <= 32 ? 32 : 64;
+  const int64_t ctas128 = (int64_t)((g.N + bn - 1) / bn) * ((g.M + 127) / 128) * g.batch * g.split_k;
+  const bool small = ctas128 < 2 * device_info().sm_count;
+  const int bm = small ? 64 : 128;
+  dim3 grid((g.N + bn - 1) / bn, (g.M + bm - 1) / bm, g.batch * g.split_k);
+  const int nt = (bm / RM) * (bn / RN);
+  const int variant = (bm == 64 ? 0 : 4) + (bn == 32 ? 0 : 2) + 0;   // tile shape
+  switch (variant + (g.transA ? 8 : 0) + (g.transB ? 1 : 0)) {
+#define SA_GEMM_CASE(V, BM_, BN_, TA_, TB_)                                               \
+  case V:                                                                                  \
+    SA_TIMED(tag, stream, (gemm_kernel<BM_, BN_, TA_, TB_><<<grid, nt, 0, stream>>>(g))); \
+    break;
+    SA_GEMM_CASE(0, 64, 32, false, false)
+    SA_GEMM_CASE(1, 64, 32, false, true)
+    SA_GEMM_CASE(2, 64, 64, false, false)
+    SA_GEMM_CASE(3, 64, 64, false, true)
+    SA_GEMM_CASE(4, 128, 32, false, false)
+    SA_GEMM_CASE(5, 128, 32, false, true)
+    SA_GEMM_CASE(6, 128, 64, false, false)
+    SA_GEMM_CASE(7, 128, 64, false, true)
+    SA_GEMM_CASE(8, 64, 32, true, false)
+    SA_GEMM_CASE(9, 64, 32, true, true)
+    SA_GEMM_CASE(10, 64, 64, true, false)
+    SA_GEMM_CASE(11, 64, 64, true, true)
+    SA_GEMM_CASE(12, 128, 32, true, false)
+    SA_GEMM_CASE(13, 128, 32, true, true)
+    SA_GEMM_CASE(14, 128, 64, true, false)
+    SA_GEMM_CASE(15, 128, 64, true, true)
+#undef SA_GEMM_CASE
+    default: break;
+  }
   if (g.split_k > 1) {
     const int64_t n = (int64_t)g.M * g.N * g.batch;
     SA_TIMED("gemm_split_reduce_kernel", stream,

@@ -58,7 +58,7 @@ struct SaBwdWork {
   float* Q;             // [k, d]
   float* gsplit;        // [kMaxSplit, d, d] split-K partials of the weight-gradient GEMMs
 };
-constexpr int kMaxSplit = 64;
+constexpr int kMaxSplit = 256;
 
 sa_status sa_fold(int k, int d, const float* P, const float* W_Q, const float* W_K, float* T,
                   float* Pf, __nv_bfloat16* Pb, cudaStream_t st);
