@@ -182,7 +182,7 @@ class TrainStepRunner:
 # Per-kernel algorithmic work (flops) per launch, for the roofline of the
 # dominant kernel.  tokens = history tokens of the call.
 KERNEL_SOURCES = {
-    "sa_fwd_tc_kernel": "sa_tc.cu", "sa_bwd_dx_tc_kernel": "sa_bwd_tc.cu",
+    "sa_lse_tc_kernel": "sa_tc.cu", "sa_agg_tc_kernel": "sa_tc.cu", "sa_bwd_dx_tc_kernel": "sa_bwd_tc.cu",
     "sa_bwd_e_tc_kernel": "sa_bwd_tc.cu", "stca_attn_tc_kernel": "stca_tc.cu",
 }
 
@@ -217,8 +217,12 @@ def measured_traffic(kernel, units):
 def kernel_model(name, w):
     k, d = w.sa.k, w.sa.d
     n = w.sa.n_total
-    if name in ("sa_fwd_tc_kernel",):
-        return "tensor", 4.0 * k * d * n
+    if name == "sa_lse_tc_kernel":
+        # the logits of every token against all k prototypes
+        return "tensor", 2.0 * k * d * n
+    if name == "sa_agg_tc_kernel":
+        # H = A X with its mass (its recomputed logits are not counted)
+        return "tensor", 2.0 * k * d * n
     if name == "sa_lse_kernel":
         return "alu", 2.0 * k * d * n
     if name == "sa_agg_kernel":
@@ -472,7 +476,7 @@ def run_component(args, rank, world, device):
         step = lambda: sab.sa_forward(X, p.offsets, P, WQ, WK, WV, p.eps, offsets_dev=offd, out=out,
                                       workspace=ws)
         units, unit, name = p.n_total, "history-tokens/s", p.name
-        kname, flops = "sa_fwd_tc_kernel", 4.0 * p.k * p.d * p.n_total
+        kname, flops = "sa_agg_tc_kernel", 2.0 * p.k * p.d * p.n_total
     else:
         w = stca_workload(users=args.users or 16)
         q, kvr, kvs = (_dev_bf16(a, device) for a in (w.recent.q, w.recent.kv, w.sketch.kv))

@@ -179,7 +179,7 @@ size_t layout_fwd(void* base, int B, int64_t n, int k, int d, sa_dtype dt, SaFwd
   v.T = c.take<float>((size_t)d * d);
   v.Pf = c.take<float>((size_t)k * d);
   v.Pb = c.take<__nv_bfloat16>((size_t)k * d);
-  v.lse = use_tc(dt, k, d) ? nullptr : c.take<float>((size_t)std::max<int64_t>(n, 1));
+  v.lse = c.take<float>((size_t)std::max<int64_t>(n, 1));
   v.Muser = c.take<float>((size_t)B * k);
   v.slotH = c.take<float>((size_t)std::max(ch.G, 1) * 2 * k * d);
   v.slotM = c.take<float>((size_t)std::max(ch.G, 1) * 2 * k);

@@ -503,11 +503,19 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     const int row = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     bool ok = true;
+    const int64_t n_total = p.off[p.B];
+    float l2_next = 0.f, ct_next = 0.f;   // this row's lse and c for the next tile, loaded a tile ahead
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t tb, int64_t pe, bool first, bool last) {
       const bool valid = tb + row < pe;
+      float l2r = l2_next, ctr = ct_next;
+      if (t == 0 && valid) { l2r = p.lse2[tb + row]; ctr = p.cin[tb + row]; }
+      // the next tile starts 128 rows on, or at the end of this piece (rows of
+      // other users are loaded harmlessly; each tile checks its own validity)
+      const int64_t nb = tb + TILE < pe ? tb + TILE : pe;
+      if (nb + row < n_total) { l2_next = p.lse2[nb + row]; ct_next = p.cin[nb + row]; }
       // a padding row gets lse = +inf, so its A = 2^(z - inf) = 0 without a select
-      const float l2 = valid ? p.lse2[tb + row] : __builtin_huge_valf();
-      const float ct = valid ? p.cin[tb + row] : 0.f;
+      const float l2 = valid ? l2r : __builtin_huge_valf();
+      const float ct = valid ? ctr : 0.f;
       const float2 nl2 = make_float2(-l2, -l2), nct = make_float2(-ct, -ct);
       if (first && !mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return ok = false;
       if (!mbar_wait(&bars->zg_full, t & 1, abort, p.err)) return ok = false;

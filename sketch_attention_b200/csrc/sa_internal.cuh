@@ -20,7 +20,7 @@ struct SaFwdWork {
   float* T;             // [d, d]   W_Q W_K^T
   float* Pf;            // [k, d]   folded prototypes, log2 units, fp32
   __nv_bfloat16* Pb;    // [k, d]   same, bf16 (tensor-core operand)
-  float* lse;           // [n_total] per-token log2-sum-exp (CUDA-core path)
+  float* lse;           // [n_total] per-token log2-sum-exp (NULL: the caller's lse output holds it)
   float* Muser;         // [B, k]   mass of users that lie in one chunk
   float* slotH;         // [G, 2, k, d]
   float* slotM;         // [G, 2, k]

@@ -54,14 +54,15 @@ sa_status scratch_address(void** out) {
 }
 
 // Scratch views inside the array (same roles as sa_forward's workspace).
-size_t layout(void* base, int B, int k, const Chunking& ch, SaFwdWork* w) {
+// n_lse: tokens whose log-sum-exp needs scratch (0 when the caller passes lse)
+size_t layout(void* base, int B, int k, const Chunking& ch, int64_t n_lse, SaFwdWork* w) {
   Carve c(base);
   SaFwdWork v;
   v.ch = ch;
   v.T = c.take<float>((size_t)kD * kD);
   v.Pf = c.take<float>((size_t)k * kD);
   v.Pb = c.take<__nv_bfloat16>((size_t)k * kD);
-  v.lse = nullptr;
+  v.lse = n_lse > 0 ? c.take<float>((size_t)n_lse) : nullptr;
   v.Muser = c.take<float>((size_t)B * k);
   v.slotH = c.take<float>((size_t)std::max(ch.G, 1) * 2 * k * kD);
   v.slotM = c.take<float>((size_t)std::max(ch.G, 1) * 2 * k);
@@ -102,13 +103,15 @@ extern "C" sa_status sa_forward_noalloc(const void* X, sa_dtype x_dtype,
   if (H == S) return fail(SA_ERR_INVALID_ARG, "H must not alias S");
 
   const Chunking ch = make_chunking(n, std::min(kMaxChunks, sa_tc_num_chunks(k)), 1);
-  if (layout(nullptr, B, k, ch, nullptr) > kScratchBytes)
-    return fail(SA_ERR_UNSUPPORTED, "sizes exceed the 8 MiB scratch array");
+  const int64_t n_lse = lse ? 0 : n;
+  if (layout(nullptr, B, k, ch, n_lse, nullptr) > kScratchBytes)
+    return fail(SA_ERR_UNSUPPORTED, "sizes exceed the 8 MiB scratch array (pass lse to take "
+                                    "the per-token log-sum-exp out of it)");
   void* scratch = nullptr;
   sa_status s = scratch_address(&scratch);
   if (s != SA_OK) return s;
   SaFwdWork w;
-  layout(scratch, B, k, ch, &w);
+  layout(scratch, B, k, ch, n_lse, &w);
   SaFwdArgs a{X, x_dtype, offsets_dev, B, n, k, d, P, W_Q, W_K, W_V, eps, S, mass, H, S_bf16, lse};
   cudaStream_t st = (cudaStream_t)stream;
   if ((s = sa_fold(k, d, P, W_Q, W_K, w.T, w.Pf, w.Pb, st)) != SA_OK) return s;

@@ -2,377 +2,517 @@
 // eqs. (6)-(9); the fused streaming operator of Sec. 4.4, re-designed for
 // tcgen05, TMEM and TMA).
 //
-// Work split.  The token stream is cut into G chunks, one per cluster of
-// C = k/128 CTAs.  CTA r of a cluster owns prototypes [128 r, 128 r + 128):
-// its slice of P' (bf16, SMEM-resident) and its accumulator
-// H_slice = [A_slice X | A_slice 1] (128 x 144 fp32 in TMEM; the last 16
-// columns hold the mass).  Every CTA of the cluster streams the same 128-token
-// tiles of X through SMEM with TMA (no multicast: each CTA issues its own
-// loads, the copies after the first come from L2).  An X tile stays in SMEM
-// from its load until its aggregation MMA, so the number of stages bounds the
-// tiles in flight; the shared-memory budget goes to four stages.
+// Two kernels, neither of which ever writes the k x n assignment matrix:
 //
-// Per tile (t = 128 tokens of one user):
-//   MMA1   Z^T[t, j] = X_t . P'_j              (M=128 tokens, N=128 prototypes, K=d)
-//   softmax over all k prototypes of each token: each CTA reduces its 128
-//          logits in registers (one TMEM lane = one token = one thread) to a
-//          log2-sum-exp, sends it to every CTA of the cluster (DSMEM bulk
-//          copies), and rescales its exponentials by 2^{m - lse_total}
-//   MMA2   H_slice[j, :] += sum_t p[t, j] [x_t | 1]   (M=128 prototypes, N=144, K=128 tokens)
-// so the k x n assignment matrix never leaves the SM.
+//   sa_lse_tc_kernel  token-parallel, one CTA per token chunk.  Per 128-token
+//     tile it streams P' in chunks of 128 prototypes: Z_c = X_t P'_c^T
+//     (M=128 tokens, N=128, K=d) into TMEM; two warpgroups (64 prototypes of
+//     each chunk each, one thread per token) keep an online maximum and sum of
+//     2^z, and at the end of the tile combine their halves into the token's
+//     log2-sum-exp over all k prototypes.
 //
-// Warp roles (11 warps): 0 TMA, 1 logits MMAs + TMEM owner, 2 aggregation
-// MMAs, 3-6 softmax of even tiles (and the H drain at the end of a piece),
-// 7-10 softmax of odd tiles.  A warp reads TMEM lanes 32 (warp % 4) .. +31, so
-// each group of four consecutive warps covers all 128 lanes.
+//   sa_agg_tc_kernel  prototype-slice-parallel, one CTA per (128-prototype
+//     slice, token chunk).  Per tile: Z = X_t P'_slice^T into TMEM; two
+//     warpgroups turn their halves into probabilities p = 2^(z - lse) (bf16,
+//     the MN-major A operand of the next MMA) and
+//     H_slice += p^T [X_t | 1]   (M=128 prototypes, N=144, K=128 tokens)
+//     accumulates in TMEM; the last 16 columns hold the mass.  At the end of a
+//     user's piece of the chunk H and the mass go to HBM.
+//
+// The logits are computed twice (once per kernel); in exchange no CTA waits
+// for another, every SM takes part, and a probability tile is written once,
+// already normalised.
 #include <algorithm>
 #include <mutex>
 
+#include "exp2_poly.cuh"
 #include "sa_internal.cuh"
 #include "tc_ptx.cuh"
+
+// Pairs (of the 4 in a group of 8 prototypes) whose exponentials the lse and
+// aggregation kernels evaluate on the FMA pipe instead of the MUFU.
+#ifndef SA_FWD_POLY_PAIRS
+#define SA_FWD_POLY_PAIRS 0x2
+#endif
 
 namespace sa {
 
 namespace {
 using namespace tc;
 
-constexpr int TILE = 128;            // tokens per tile = prototypes per CTA
+constexpr int TILE = 128;            // tokens per tile = prototypes per chunk or slice
 constexpr int DD = 128;              // d
-constexpr int NS = 4;                // X pipeline stages (tiles in flight)
-constexpr int MAXC = 8;              // cluster size limit (k <= 1024)
-constexpr int N2 = DD + 16;          // MMA2 N: d columns + 16 mass columns
-constexpr int THREADS = 352;
+constexpr float kLn2f = 0.69314718055994530942f;
+constexpr float kLog2ef = 1.44269504088896340736f;
 
-// shared-memory layout (offsets from a 1024-aligned base)
-constexpr uint32_t X_BOX = TILE * 32;                  // one [128 x 16] bf16 SW32 box = 4 KB
-constexpr uint32_t X_STAGE = 9 * X_BOX;                // 8 boxes of X + 1 box of ones = 36 KB
-constexpr uint32_t OFF_PQ = 0;                         // P' slice: 2 x [128 x 64] SW128 = 32 KB
-constexpr uint32_t OFF_X = 32768;
-constexpr uint32_t OFF_P = OFF_X + NS * X_STAGE;       // one 32 KB probability tile
-constexpr uint32_t OFF_XCHG = OFF_P + 32768;           // [4 slots][MAXC][128] fp32
-constexpr uint32_t OFF_BAR = OFF_XCHG + 4 * MAXC * TILE * 4;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + barriers + alignment slack
+// Iterates the tiles of chunk g: f(tile_index, piece, user, tile_begin,
+// piece_end, first_tile_of_piece, last_tile_of_piece); stops if f returns false.
+template <class F>
+__device__ __forceinline__ void for_each_tile(const int64_t* off, int B, const Chunking& ch, int g,
+                                              F&& f) {
+  const int64_t cb = (int64_t)g * ch.T, ce = min(cb + ch.T, ch.n_total);
+  int t = 0, piece = 0;
+  for (int u = user_of_token(off, B, cb); u < B && off[u] < ce; ++u) {
+    const int64_t pb = max(off[u], cb), pe = min(off[u + 1], ce);
+    if (pb >= pe) continue;
+    for (int64_t tb = pb; tb < pe; tb += TILE, ++t)
+      if (!f(t, piece, u, tb, pe, tb == pb, tb + TILE >= pe)) return;
+    ++piece;
+  }
+}
 
-// TMEM columns
-constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_H = 256, TM_COLS = 512;
+// 2^e for a pair: on the FMA pipe (fitted cubic) or the MUFU
+template <bool POLY>
+__device__ __forceinline__ float2 exp2_pair(float2 e) {
+  if (POLY) return exp2_poly2(e);
+  return make_float2(ex2(e.x), ex2(e.y));
+}
 
-struct Bars {
-  uint64_t x_full[NS], x_empty[NS];
-  uint64_t s_full[2], s_empty[2], p_full, p_empty;
-  uint64_t h_full, h_empty, pq_full, mma_done;
-  uint64_t xchg[4];
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// maximum of 64 values (four independent chains of three-input maxima)
+__device__ __forceinline__ float max64(const float* z) {
+  float c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float* w = z + 16 * i;
+    float m = max3f(w[0], w[1], w[2]);
+#pragma unroll
+    for (int j = 3; j + 1 < 16; j += 2) m = max3f(m, w[j], w[j + 1]);
+    c[i] = fmaxf(m, w[15]);
+  }
+  return fmaxf(max3f(c[0], c[1], c[2]), c[3]);
+}
+
+// ============================================================== lse kernel
+constexpr int L_NXS = 2, L_NPS = 4;                 // X stages, P' chunk stages
+constexpr uint32_t T_BYTES = TILE * DD * 2;         // [128 x 128] bf16: 2 SW128 halves of 16 KB
+constexpr uint32_t L_OFF_X = 0;
+constexpr uint32_t L_OFF_P = L_OFF_X + L_NXS * T_BYTES;
+constexpr uint32_t L_OFF_XCH = L_OFF_P + L_NPS * T_BYTES;   // [2][128]: warpgroup 1's max and sum
+constexpr uint32_t L_OFF_BAR = L_OFF_XCH + 2 * TILE * 4;
+constexpr uint32_t L_SMEM = L_OFF_BAR + 256 + 1024;
+constexpr int L_THREADS = 320;   // warp 0 TMA, 1 MMA + TMEM owner, 2-5 and 6-9 two warpgroups
+constexpr uint32_t L_TM_Z = 0, L_TM_COLS = 256;    // two [128 x 128] fp32 logits buffers
+
+struct LBars {
+  uint64_t x_full[L_NXS], x_empty[L_NXS], c_full[L_NPS], c_empty[L_NPS];
+  uint64_t z_full[2], z_empty[2], cx_full, cx_empty, mma_done;
   uint32_t tmem_base;
   int abort;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(LBars) <= 256, "barrier block");
 
-struct Params {
+struct LParams {
   const int64_t* off;
   int B;
   Chunking ch;
   int k;
-  float* Huser;
-  float* Muser;
-  float* slotH;
-  float* slotM;
-  float* lse;          // optional per-token ln-sum-exp output
+  float* lse_a;        // [n] required output: the log2-sum-exp times a_scale
+  float a_scale;       // 1 (log2 units) or ln 2 (natural units)
+  float* lse_b;        // [n] optional natural-log copy
   int* err;
 };
 
-// Iterates the tiles of chunk g: calls f(tile_index, user, tile_begin,
-// piece_begin, piece_end, first_tile_of_piece, last_tile_of_piece) in order;
-// stops early if f returns false.
-template <class F>
-__device__ __forceinline__ void for_each_tile(const Params& p, int g, F&& f) {
-  const int64_t cb = (int64_t)g * p.ch.T, ce = min(cb + p.ch.T, p.ch.n_total);
-  int t = 0;
-  for (int u = user_of_token(p.off, p.B, cb); u < p.B && p.off[u] < ce; ++u) {
-    const int64_t pb = max(p.off[u], cb), pe = min(p.off[u + 1], ce);
-    for (int64_t tb = pb; tb < pe; tb += TILE, ++t)
-      if (!f(t, u, tb, pb, pe, tb == pb, tb + TILE >= pe)) return;
-  }
-}
-
-__global__ void __launch_bounds__(THREADS, 1)
-    sa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmX,
-                     const __grid_constant__ CUtensorMap tmP, Params p) {
+__global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 warps share a sub-partition)
+    sa_lse_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                     LParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  Bars* bars = (Bars*)(smem + OFF_BAR);
+  LBars* bars = (LBars*)(smem + L_OFF_BAR);
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint32_t rank = cluster_rank(), C = cluster_size();
-  const int g = (int)cluster_id_x();
-  const bool chunk_ok = g < p.ch.G;
+  const int g = blockIdx.x;
+  if (g >= p.ch.G) return;
+  const int nch = p.k / TILE;
 
-  // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_empty[b], 128);
-    }
-    mbar_init(&bars->p_full, 128);
-    mbar_init(&bars->p_empty, 1);
-    mbar_init(&bars->h_full, 1);
-    mbar_init(&bars->h_empty, 128);
-    mbar_init(&bars->pq_full, 1);
-    mbar_init(&bars->mma_done, 2);        // both MMA-issuing threads
-    for (int s = 0; s < 4; ++s) mbar_init(&bars->xchg[s], 1);
+    for (int s = 0; s < L_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
+    for (int s = 0; s < L_NPS; ++s) { mbar_init(&bars->c_full[s], 1); mbar_init(&bars->c_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->z_full[b], 1); mbar_init(&bars->z_empty[b], 256); }
+    mbar_init(&bars->cx_full, 128);
+    mbar_init(&bars->cx_empty, 128);
+    mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbar_init();
-    // arm the exchange slots for their first use (tiles 0..3)
-    for (int s = 0; s < 4; ++s) mbar_arrive_expect_tx(&bars->xchg[s], (C - 1) * TILE * 4);
   }
-  // constant ones block of every stage (MMA2 columns d..d+15 -> prototype mass)
-  for (int i = threadIdx.x; i < NS * (int)X_BOX / 4; i += THREADS) {
-    const int s = i / (X_BOX / 4), w = i % (X_BOX / 4);
-    ((uint32_t*)(smem + OFF_X + s * X_STAGE + 8 * X_BOX))[w] = 0x3F803F80u;   // bf16 1.0 pairs
-  }
-  fence_proxy_async_smem();
   if (warp == 1) {
-    tmem_alloc(&bars->tmem_base, TM_COLS);
+    tmem_alloc(&bars->tmem_base, L_TM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();          // peers' barriers are initialised before any exchange
   const uint32_t tmem = bars->tmem_base;
 
-  if (chunk_ok) {
-    if (warp == 0 && lane == 0) {
-      // ------------------------------------------------------------ TMA producer
-      prefetch_tensormap(&tmX);
-      prefetch_tensormap(&tmP);
-      mbar_arrive_expect_tx(&bars->pq_full, 2 * 16384);
-      tma_load_2d(smem + OFF_PQ, &tmP, &bars->pq_full, 0, (int)(rank * TILE));
-      tma_load_2d(smem + OFF_PQ + 16384, &tmP, &bars->pq_full, 64, (int)(rank * TILE));
-      int issued = 0;
-      for_each_tile(p, g, [&](int t, int, int64_t tb, int64_t, int64_t, bool, bool) {
-        const int s = t % NS;
-        if (t >= NS && !mbar_wait(&bars->x_empty[s], ((t / NS) - 1) & 1, abort, p.err)) return false;
-        mbar_arrive_expect_tx(&bars->x_full[s], 8 * X_BOX);
-        uint8_t* dst = smem + OFF_X + s * X_STAGE;
-        for (int b = 0; b < 8; ++b) tma_load_2d(dst + b * X_BOX, &tmX, &bars->x_full[s], 16 * b, (int)tb);
-        issued = t + 1;
-        return true;
-      });
-      if (*abort) {
-        // let the loads still in flight land before the CTA can exit
-        mbar_wait_bounded(&bars->pq_full, 0);
-        for (int t = std::max(0, issued - NS); t < issued; ++t)
-          mbar_wait_bounded(&bars->x_full[t % NS], (t / NS) & 1);
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmP);
+    int cc = 0, issued_t = 0, issued_c = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t, bool, bool) {
+      const int s = t % L_NXS;
+      if (t >= L_NXS && !mbar_wait(&bars->x_empty[s], ((t / L_NXS) - 1) & 1, abort, p.err)) return false;
+      mbar_arrive_expect_tx(&bars->x_full[s], T_BYTES);
+      uint8_t* xd = smem + L_OFF_X + s * T_BYTES;
+      tma_load_2d(xd, &tmX, &bars->x_full[s], 0, (int)tb);
+      tma_load_2d(xd + T_BYTES / 2, &tmX, &bars->x_full[s], 64, (int)tb);
+      issued_t = t + 1;
+      for (int c = 0; c < nch; ++c, ++cc) {
+        const int cs = cc % L_NPS;
+        if (cc >= L_NPS && !mbar_wait(&bars->c_empty[cs], ((cc / L_NPS) - 1) & 1, abort, p.err)) return false;
+        mbar_arrive_expect_tx(&bars->c_full[cs], T_BYTES);
+        uint8_t* pd = smem + L_OFF_P + cs * T_BYTES;
+        tma_load_2d(pd, &tmP, &bars->c_full[cs], 0, c * TILE);
+        tma_load_2d(pd + T_BYTES / 2, &tmP, &bars->c_full[cs], 64, c * TILE);
+        issued_c = cc + 1;
       }
-    } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------------------ logits MMAs
-      // MMA1 of a tile is issued as soon as its X tile has landed and the
-      // logits buffer it reuses has been read by the softmax warps.
-      const uint32_t id1 = idesc_bf16(128, 128, false, false);
-      const uint32_t pq = smem_u32(smem + OFF_PQ);
-      if (mbar_wait(&bars->pq_full, 0, abort, p.err)) {
-        for_each_tile(p, g, [&](int t, int, int64_t, int64_t, int64_t, bool, bool) {
-          const int s = t % NS, b = t & 1;
-          if (!mbar_wait(&bars->x_full[s], (t / NS) & 1, abort, p.err)) return false;
-          if (t >= 2 && !mbar_wait(&bars->s_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return false;
-          tc_fence_after();
-          const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
-#pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t da = smem_desc(xa + ks * X_BOX, 16, 256, SWZ_32B);
-            const uint64_t db = smem_desc(pq + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B);
-            mma_ss(tmem + (b ? TM_S1 : TM_S0), da, db, id1, ks > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars->s_full[b]);
-          return true;
-        });
-      }
-      // every MMA this thread issued has completed before TMEM is released
-      mma_commit(&bars->mma_done);
-      mbar_wait_bounded(&bars->mma_done, 0);
-    } else if (warp == 2 && lane == 0) {
-      // ------------------------------------------------------------ aggregation MMAs
-      // A second issuing thread, so MMA2 of a tile starts the moment its
-      // probabilities are written, independent of the logits of later tiles
-      // (the two streams touch disjoint TMEM and SMEM).
-      const uint32_t id2 = idesc_bf16(128, N2, true, true);
-      int piece = -1;
-      for_each_tile(p, g, [&](int t, int, int64_t, int64_t, int64_t, bool first, bool last) {
-        const int s = t % NS;
-        if (first) ++piece;
-        if (first && piece > 0 && !mbar_wait(&bars->h_empty, (piece - 1) & 1, abort, p.err)) return false;
-        if (!mbar_wait(&bars->p_full, t & 1, abort, p.err)) return false;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(smem + OFF_P);
-        const uint32_t xa = smem_u32(smem + OFF_X + s * X_STAGE);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t da = smem_desc(pa + ks * 2048, 16384, 1024, SWZ_128B);
-          const uint64_t db = smem_desc(xa + ks * 512, X_BOX, 256, SWZ_32B);
-          mma_ss(tmem + TM_H, da, db, id2, (first && ks == 0) ? 0u : 1u);
-        }
-        mma_commit(&bars->p_empty);
-        mma_commit(&bars->x_empty[s]);
-        if (last) mma_commit(&bars->h_full);
-        return true;
-      });
-      mma_commit(&bars->mma_done);
-      mbar_wait_bounded(&bars->mma_done, 0);
-    } else if (warp >= 3) {
-      // ------------------------------------------------------------ softmax groups
-      const int wg = (warp - 3) / 4;            // 0: even tiles, 1: odd tiles
-      const int q = warp % 4;                   // TMEM lane quarter
-      const int row = q * 32 + lane;            // token within the tile / prototype lane
-      const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-      const float* xchg = (const float*)(smem + OFF_XCHG);
-      int piece = -1;
-      for_each_tile(p, g, [&](int t, int u, int64_t tb, int64_t pb, int64_t pe, bool first, bool last) {
-        if (first) ++piece;
-        if ((t & 1) == wg) {
-          const int b = t & 1;
-          const bool valid = tb + row < pe;
-          // logits of this token over the CTA's 128 prototypes (base-2 units)
-          if (!mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort, p.err)) return false;
-          tc_fence_after();
-          // Eight chunks of 16 logits, each exponentiated against the running
-          // maximum at that point (mc[c]) and scaled by 2^8, kept as fp16 pairs
-          // (11-bit mantissa, normal range down to 2^-22 of the chunk maximum).
-          // The load of chunk c+1 is in flight while chunk c is processed; the
-          // logits buffer is released as soon as the last chunk has landed.
-          const uint32_t sbuf = tmem + lane_addr + (b ? TM_S1 : TM_S0);
-          uint32_t ep[64];
-          float mc[8];
-          float m = -__builtin_huge_valf();
-          float2 s2 = make_float2(0.f, 0.f);   // running sum, as two partial sums
-          float zbuf[2][16];
-          tmem_ld16(sbuf, zbuf[0]);
-          tmem_wait_ld16(zbuf[0]);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float* z = zbuf[c & 1];
-            if (c < 7) tmem_ld16(sbuf + 16 * (c + 1), zbuf[(c + 1) & 1]);
-            float cm = z[0];
-#pragma unroll
-            for (int j = 1; j < 16; ++j) cm = fmaxf(cm, z[j]);
-            const float mn = fmaxf(m, cm);
-            const float sc = ex2(m - mn);
-            s2 = __fmul2_rn(s2, make_float2(sc, sc));
-            m = mn;
-            mc[c] = mn;
-            const float2 off = make_float2(8.f - mn, 8.f - mn);
-            // two logits per instruction (packed fp32x2 add)
-#pragma unroll
-            for (int j = 0; j < 16; j += 2) {
-              const float2 zz = __fadd2_rn(make_float2(z[j], z[j + 1]), off);
-              const float2 e = make_float2(ex2(zz.x), ex2(zz.y));
-              s2 = __fadd2_rn(s2, e);
-              ep[8 * c + j / 2] = pack_f16x2(e.x, e.y);
-            }
-            if (c < 7) tmem_wait_ld16(zbuf[(c + 1) & 1]);
-            if (c == 6) {
-              tc_fence_before();
-              mbar_arrive(&bars->s_empty[b]);
-            }
-          }
-          const float l = valid ? m + lg2(s2.x + s2.y) - 8.f : -__builtin_huge_valf();
-          // this CTA's log2-sum-exp of every token goes into its own row of the
-          // exchange slot, and from there to the same row in every other CTA
-          const int slot = t & 3;
-          float* own = (float*)(smem + OFF_XCHG) + (slot * MAXC + rank) * TILE;
-          own[row] = l;
-          fence_proxy_async_smem();
-          named_bar_sync(1 + wg, 128);
-          if (row == 0) {
-            const uint32_t src = smem_u32(own);
-            const uint32_t bar = smem_u32(&bars->xchg[slot]);
-            for (uint32_t c = 0; c < C; ++c)
-              if (c != rank) bulk_copy_to_peer(map_to_rank(src, c), src, TILE * 4, map_to_rank(bar, c));
-          }
-          if (!mbar_wait(&bars->xchg[slot], (t >> 2) & 1, abort, p.err)) return false;
-          float rc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          if (valid) {
-            float L = -__builtin_huge_valf();
-            for (uint32_t c = 0; c < C; ++c) L = fmaxf(L, xchg[(slot * MAXC + c) * TILE + row]);
-            float z = 0.f;
-            for (uint32_t c = 0; c < C; ++c) z += ex2(xchg[(slot * MAXC + c) * TILE + row] - L);
-            const float lt = L + lg2(z);
-            if (p.lse && rank == 0) p.lse[tb + row] = lt * 0.69314718055994530942f;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) rc[c] = ex2(mc[c] - 8.f - lt);
-          }
-          named_bar_sync(1 + wg, 128);      // every thread has read the slot
-          if (row == 0) mbar_arrive_expect_tx(&bars->xchg[slot], (C - 1) * TILE * 4);   // re-arm for t+4
-          // probabilities p[t, j] = e_j r as bf16 into the MN-major SW128 A tile of MMA2
-          if (t >= 1 && !mbar_wait(&bars->p_empty, (t - 1) & 1, abort, p.err)) return false;
-          const uint32_t pa = smem_u32(smem + OFF_P) + row * 128;
-#pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {           // 16-byte chunks of 8 prototypes
-            const float2 r = make_float2(rc[cc >> 1], rc[cc >> 1]);
-            const uint32_t* e4 = ep + 4 * cc;
-            const float2 a0 = __fmul2_rn(unpack_f16x2(e4[0]), r), a1 = __fmul2_rn(unpack_f16x2(e4[1]), r);
-            const float2 a2 = __fmul2_rn(unpack_f16x2(e4[2]), r), a3 = __fmul2_rn(unpack_f16x2(e4[3]), r);
-            st_shared_v4(pa + (cc >> 3) * 16384 + (((cc & 7) ^ (row & 7)) << 4),
-                         pack_bf16x2(a0.x, a0.y), pack_bf16x2(a1.x, a1.y),
-                         pack_bf16x2(a2.x, a2.y), pack_bf16x2(a3.x, a3.y));
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          mbar_arrive(&bars->p_full);
-        }
-        if (last && wg == 0) {
-          // ------------------------------------------------------ drain H of the piece
-          if (!mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return false;
-          tc_fence_after();
-          const int64_t ub = p.off[u], ue = p.off[u + 1];
-          const int64_t cb = (int64_t)g * p.ch.T, ce = min(cb + p.ch.T, p.ch.n_total);
-          const int dest = piece_dest(ub, ue, cb, ce);
-          const int j = (int)rank * TILE + row;
-          float* Hrow;
-          float* mrow;
-          if (dest == DEST_USER) {
-            Hrow = p.Huser + ((int64_t)u * p.k + j) * DD;
-            mrow = p.Muser + (int64_t)u * p.k + j;
-          } else {
-            Hrow = p.slotH + (((int64_t)g * 2 + dest) * p.k + j) * DD;
-            mrow = p.slotM + ((int64_t)g * 2 + dest) * p.k + j;
-          }
-          float hv[32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            tmem_ld32(tmem + lane_addr + TM_H + 32 * c, hv);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              *(float4*)(Hrow + 32 * c + i) = make_float4(hv[i], hv[i + 1], hv[i + 2], hv[i + 3]);
-          }
-          const float mass = tmem_ld1(tmem + lane_addr + TM_H + DD);
-          tmem_wait_ld();
-          *mrow = mass;
-          tc_fence_before();
-          mbar_arrive(&bars->h_empty);
-        }
-        return true;
-      });
+      return true;
+    });
+    if (*abort) {
+      for (int t = std::max(0, issued_t - L_NXS); t < issued_t; ++t)
+        mbar_wait_bounded(&bars->x_full[t % L_NXS], (t / L_NXS) & 1);
+      for (int c = std::max(0, issued_c - L_NPS); c < issued_c; ++c)
+        mbar_wait_bounded(&bars->c_full[c % L_NPS], (c / L_NPS) & 1);
     }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ logits MMAs
+    const uint32_t id = idesc_bf16(128, 128, false, false);
+    int ai = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
+      const int s = t % L_NXS;
+      if (!mbar_wait(&bars->x_full[s], (t / L_NXS) & 1, abort, p.err)) return false;
+      const uint32_t xa = smem_u32(smem + L_OFF_X + s * T_BYTES);
+      for (int c = 0; c < nch; ++c) {
+        const int a = ai + c, cs = a % L_NPS, b = a & 1;
+        if (!mbar_wait(&bars->c_full[cs], (a / L_NPS) & 1, abort, p.err)) return false;
+        if (a >= 2 && !mbar_wait(&bars->z_empty[b], ((a >> 1) - 1) & 1, abort, p.err)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(smem + L_OFF_P + cs * T_BYTES);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tmem + L_TM_Z + 128 * b,
+                 smem_desc(xa + (ks >> 2) * (T_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B),
+                 smem_desc(pa + (ks >> 2) * (T_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B), id,
+                 ks > 0 ? 1u : 0u);
+        mma_commit(&bars->z_full[b]);
+        mma_commit(&bars->c_empty[cs]);                     // P' is read by this MMA only
+        if (c == nch - 1) mma_commit(&bars->x_empty[s]);
+      }
+      ai += nch;
+      return true;
+    });
+    mma_commit(&bars->mma_done);
+    mbar_wait_bounded(&bars->mma_done, 0);
+  } else if (warp >= 2 && warp <= 9) {
+    // ------------------------------------------------------------ two threads per token
+    // warpgroup h reads columns 64h..64h+63 of each chunk's logits
+    const int q = warp % 4, h = (warp - 2) / 4;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    float* xch = (float*)(smem + L_OFF_XCH);
+    int ai = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t pe, bool, bool) {
+      float m = -__builtin_huge_valf();
+      float2 s2 = make_float2(0.f, 0.f);
+      for (int c = 0; c < nch; ++c) {
+        const int a = ai + c, b = a & 1;
+        if (!mbar_wait(&bars->z_full[b], (a >> 1) & 1, abort, p.err)) return false;
+        tc_fence_after();
+        float z[64];
+        tmem_ld32(tmem + lane_addr + L_TM_Z + 128 * b + 64 * h, z);
+        tmem_ld32(tmem + lane_addr + L_TM_Z + 128 * b + 64 * h + 32, z + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->z_empty[b]);
+        const float mn = fmaxf(m, max64(z));
+        const float sc = ex2(m - mn);                      // 0 on the first chunk
+        s2 = __fmul2_rn(s2, make_float2(sc, sc));
+        m = mn;
+        const float2 nm = make_float2(-mn, -mn);
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) {
+          const float2 e = __fadd2_rn(make_float2(z[j], z[j + 1]), nm);
+          const float2 v = ((SA_FWD_POLY_PAIRS >> ((j / 2) & 3)) & 1) ? exp2_pair<true>(e) : exp2_pair<false>(e);
+          s2 = __fadd2_rn(s2, v);
+        }
+      }
+      ai += nch;
+      const float s = s2.x + s2.y;
+      if (h == 1) {
+        // hand the half-row statistics to warpgroup 0 (the slot is free once it read the last ones)
+        if (t > 0 && !mbar_wait(&bars->cx_empty, (t - 1) & 1, abort, p.err)) return false;
+        xch[row] = m;
+        xch[TILE + row] = s;
+        mbar_arrive(&bars->cx_full);
+        return true;
+      }
+      if (!mbar_wait(&bars->cx_full, t & 1, abort, p.err)) return false;
+      const float m1 = xch[row], s1 = xch[TILE + row];
+      mbar_arrive(&bars->cx_empty);
+      const float M = fmaxf(m, m1);
+      const float l2 = M + lg2(s * ex2(m - M) + s1 * ex2(m1 - M));
+      if (tb + row < pe) {
+        p.lse_a[tb + row] = l2 * p.a_scale;
+        if (p.lse_b) p.lse_b[tb + row] = l2 * kLn2f;
+      }
+      return true;
+    });
   }
 
-  // ---------------------------------------------------------------- teardown
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TM_COLS);
+    tmem_dealloc(tmem, L_TM_COLS);
   }
-  cluster_sync();          // no peer copies may target this CTA after it exits
 }
 
-struct Cached {
-  bool init = false;
-  int clusters[MAXC + 1] = {};
-};
-std::mutex g_mu;
-Cached g_cache[64];
+// ============================================================== aggregation kernel
+// X stages and probability tiles (an X tile is held from its load to its
+// aggregation MMA, so the stages bound the tiles in flight)
+#ifndef SA_AGG_NS
+#define SA_AGG_NS 3
+#endif
+#ifndef SA_AGG_NP
+#define SA_AGG_NP 2
+#endif
+constexpr int A_NS = SA_AGG_NS, A_NP = SA_AGG_NP;
+constexpr int N2 = DD + 16;                           // MMA2 N: d columns + 16 mass columns
+constexpr uint32_t X_BOX = TILE * 32;                 // one [128 x 16] bf16 SW32 box = 4 KB
+constexpr uint32_t X_STAGE = 9 * X_BOX;               // 8 boxes of X + 1 box of ones = 36 KB
+constexpr uint32_t A_OFF_PQ = 0;                      // P' slice: 2 x [128 x 64] SW128 = 32 KB
+constexpr uint32_t A_OFF_X = T_BYTES;
+constexpr uint32_t A_OFF_P = A_OFF_X + A_NS * X_STAGE;   // A_NP 32 KB probability tiles
+constexpr uint32_t A_OFF_BAR = A_OFF_P + A_NP * T_BYTES;
+constexpr uint32_t A_SMEM = A_OFF_BAR + 256 + 1024;
+constexpr int A_THREADS = 352;   // warp 0 TMA, 1 logits MMAs + TMEM owner, 2 aggregation MMAs,
+                                 // 3-6 and 7-10 two warpgroups (64 prototypes of the slice each)
+constexpr uint32_t A_TM_S = 0, A_TM_H = 256, A_TM_COLS = 512;   // logits 2 x 128, H 144
 
+struct ABars {
+  uint64_t x_full[A_NS], x_empty[A_NS], s_full[2], s_empty[2], p_full[A_NP], p_empty[A_NP];
+  uint64_t h_full, h_empty, pq_full, mma_done[2];
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(ABars) <= 256, "barrier block");
+
+struct AParams {
+  const int64_t* off;
+  int B;
+  Chunking ch;
+  int k;
+  const float* lse;    // [n] per-token log-sum-exp, times in_scale in log2 units
+  float in_scale;
+  float* Huser;        // [B, k, d] users that lie inside one chunk
+  float* Muser;        // [B, k]
+  float* slotH;        // [G, 2, k, d] pieces at chunk boundaries
+  float* slotM;        // [G, 2, k]
+  int* err;
+};
+
+__global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 warps share a sub-partition)
+    sa_agg_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                     AParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  ABars* bars = (ABars*)(smem + A_OFF_BAR);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int slices = p.k / TILE;
+  const int sl = blockIdx.x % slices, g = blockIdx.x / slices;
+  if (g >= p.ch.G) return;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < A_NS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->s_full[b], 1); mbar_init(&bars->s_empty[b], 256); }
+    for (int b = 0; b < A_NP; ++b) { mbar_init(&bars->p_full[b], 256); mbar_init(&bars->p_empty[b], 1); }
+    mbar_init(&bars->h_full, 1);
+    mbar_init(&bars->h_empty, 128);
+    mbar_init(&bars->pq_full, 1);
+    mbar_init(&bars->mma_done[0], 1);
+    mbar_init(&bars->mma_done[1], 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  // constant ones block of every stage (MMA2 columns d..d+15 -> prototype mass)
+  for (int i = threadIdx.x; i < A_NS * (int)X_BOX / 4; i += A_THREADS) {
+    const int s = i / (X_BOX / 4), w = i % (X_BOX / 4);
+    ((uint32_t*)(smem + A_OFF_X + s * X_STAGE + 8 * X_BOX))[w] = 0x3F803F80u;   // bf16 1.0 pairs
+  }
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, A_TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    prefetch_tensormap(&tmX);
+    prefetch_tensormap(&tmP);
+    mbar_arrive_expect_tx(&bars->pq_full, T_BYTES);
+    tma_load_2d(smem + A_OFF_PQ, &tmP, &bars->pq_full, 0, sl * TILE);
+    tma_load_2d(smem + A_OFF_PQ + T_BYTES / 2, &tmP, &bars->pq_full, 64, sl * TILE);
+    int issued = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t, bool, bool) {
+      const int s = t % A_NS;
+      if (t >= A_NS && !mbar_wait(&bars->x_empty[s], ((t / A_NS) - 1) & 1, abort, p.err)) return false;
+      mbar_arrive_expect_tx(&bars->x_full[s], 8 * X_BOX);
+      uint8_t* dst = smem + A_OFF_X + s * X_STAGE;
+      for (int bx = 0; bx < 8; ++bx) tma_load_2d(dst + bx * X_BOX, &tmX, &bars->x_full[s], 16 * bx, (int)tb);
+      issued = t + 1;
+      return true;
+    });
+    if (*abort) {
+      mbar_wait_bounded(&bars->pq_full, 0);
+      for (int t = std::max(0, issued - A_NS); t < issued; ++t)
+        mbar_wait_bounded(&bars->x_full[t % A_NS], (t / A_NS) & 1);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ logits MMAs
+    const uint32_t id1 = idesc_bf16(128, 128, false, false);
+    const uint32_t pq = smem_u32(smem + A_OFF_PQ);
+    if (mbar_wait(&bars->pq_full, 0, abort, p.err)) {
+      for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
+        const int s = t % A_NS, b = t & 1;
+        if (!mbar_wait(&bars->x_full[s], (t / A_NS) & 1, abort, p.err)) return false;
+        if (t >= 2 && !mbar_wait(&bars->s_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return false;
+        tc_fence_after();
+        const uint32_t xa = smem_u32(smem + A_OFF_X + s * X_STAGE);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ss(tmem + A_TM_S + 128 * b, smem_desc(xa + ks * X_BOX, 16, 256, SWZ_32B),
+                 smem_desc(pq + (ks >> 2) * (T_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B), id1,
+                 ks > 0 ? 1u : 0u);
+        mma_commit(&bars->s_full[b]);
+        return true;
+      });
+    }
+    mma_commit(&bars->mma_done[0]);
+    mbar_wait_bounded(&bars->mma_done[0], 0);
+  } else if (warp == 2 && lane == 0) {
+    // ------------------------------------------------------------ aggregation MMAs
+    // A second issuing thread, so the aggregation of a tile starts the moment its
+    // probabilities are written (the two threads' MMAs share no TMEM columns).
+    const uint32_t id2 = idesc_bf16(128, N2, true, true);
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t, int64_t, bool first, bool last) {
+      const int s = t % A_NS, b = t % A_NP;
+      if (first && piece > 0 && !mbar_wait(&bars->h_empty, (piece - 1) & 1, abort, p.err)) return false;
+      if (!mbar_wait(&bars->p_full[b], (t / A_NP) & 1, abort, p.err)) return false;
+      tc_fence_after();
+      const uint32_t pa = smem_u32(smem + A_OFF_P + b * T_BYTES);
+      const uint32_t xa = smem_u32(smem + A_OFF_X + s * X_STAGE);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks)
+        mma_ss(tmem + A_TM_H, smem_desc(pa + ks * 2048, 16384, 1024, SWZ_128B),
+               smem_desc(xa + ks * 512, X_BOX, 256, SWZ_32B), id2, (first && ks == 0) ? 0u : 1u);
+      mma_commit(&bars->p_empty[b]);
+      mma_commit(&bars->x_empty[s]);
+      if (last) mma_commit(&bars->h_full);
+      return true;
+    });
+    mma_commit(&bars->mma_done[1]);
+    mbar_wait_bounded(&bars->mma_done[1], 0);
+  } else if (warp >= 3) {
+    // ------------------------------------------------------------ two threads per token
+    // warpgroup h owns prototypes 64h..64h+63 of the slice: it turns their logits
+    // into probabilities and writes them as M-block h of the MN-major A operand
+    const int q = warp % 4, h = (warp - 3) / 4;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    const int64_t n_total = p.off[p.B];
+    float lse_next = 0.f;      // this row's lse for the next tile, loaded a tile ahead
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int u, int64_t tb, int64_t pe, bool, bool last) {
+      const int b = t & 1;
+      const bool valid = tb + row < pe;
+      const float lse_row = (t == 0 && valid) ? p.lse[tb + row] : lse_next;
+      // the next tile starts 128 rows on, or at the end of this piece (rows of
+      // other users are loaded harmlessly; each tile checks its own validity)
+      const int64_t nb = tb + TILE < pe ? tb + TILE : pe;
+      if (nb + row < n_total) lse_next = p.lse[nb + row];
+      // a row past the piece gets lse = +inf, so its probabilities are 0
+      const float l2 = valid ? lse_row * p.in_scale : __builtin_huge_valf();
+      const float2 nl2 = make_float2(-l2, -l2);
+      if (!mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort, p.err)) return false;
+      tc_fence_after();
+      uint32_t o[32];
+      {
+        float z[64];
+        tmem_ld32(tmem + lane_addr + A_TM_S + 128 * b + 64 * h, z);
+        tmem_ld32(tmem + lane_addr + A_TM_S + 128 * b + 64 * h + 32, z + 32);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->s_empty[b]);
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) {
+          const float2 e = __fadd2_rn(make_float2(z[j], z[j + 1]), nl2);
+          const float2 v = ((SA_FWD_POLY_PAIRS >> ((j / 2) & 3)) & 1) ? exp2_pair<true>(e) : exp2_pair<false>(e);
+          o[j / 2] = pack_bf16x2(v.x, v.y);
+        }
+      }
+      // probability tile pb was last read by the aggregation MMA of tile t - A_NP
+      const int pb = t % A_NP;
+      if (t >= A_NP && !mbar_wait(&bars->p_empty[pb], ((t / A_NP) - 1) & 1, abort, p.err)) return false;
+      const uint32_t pa = smem_u32(smem + A_OFF_P + pb * T_BYTES) + h * 16384 + row * 128;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8)
+        st_shared_v4(pa + ((c8 ^ (row & 7)) << 4), o[4 * c8], o[4 * c8 + 1], o[4 * c8 + 2], o[4 * c8 + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->p_full[pb]);
+      if (last && h == 0) {
+        // ------------------------------------------------------ drain H of the piece
+        if (!mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return false;
+        tc_fence_after();
+        const int64_t ub = p.off[u], ue = p.off[u + 1];
+        const int64_t cb = (int64_t)g * p.ch.T, ce = min(cb + p.ch.T, p.ch.n_total);
+        const int dest = piece_dest(ub, ue, cb, ce);
+        const int j = sl * TILE + row;
+        float* Hrow;
+        float* mrow;
+        if (dest == DEST_USER) {
+          Hrow = p.Huser + ((int64_t)u * p.k + j) * DD;
+          mrow = p.Muser + (int64_t)u * p.k + j;
+        } else {
+          Hrow = p.slotH + (((int64_t)g * 2 + dest) * p.k + j) * DD;
+          mrow = p.slotM + ((int64_t)g * 2 + dest) * p.k + j;
+        }
+        float hv[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_ld32(tmem + lane_addr + A_TM_H + 32 * c, hv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *(float4*)(Hrow + 32 * c + i) = make_float4(hv[i], hv[i + 1], hv[i + 2], hv[i + 3]);
+        }
+        const float mass = tmem_ld1(tmem + lane_addr + A_TM_H + DD);
+        tmem_wait_ld();
+        *mrow = mass;
+        tc_fence_before();
+        mbar_arrive(&bars->h_empty);
+      }
+      return true;
+    });
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, A_TM_COLS);
+  }
+}
+
+// ============================================================== host side
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                               const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                               const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -391,13 +531,14 @@ EncodeFn encode_fn() {
   return fn;
 }
 
-sa_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                   uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+// [outer, 128] bf16 rows; boxes of box_inner x 128 rows
+sa_status make_map(CUtensorMap* map, const void* base, uint64_t outer, uint32_t box_inner,
+                   CUtensorMapSwizzle swz) {
   EncodeFn enc = encode_fn();
   if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint64_t dims[2] = {(cuuint64_t)DD, outer};
+  cuuint64_t strides[1] = {(cuuint64_t)DD * 2};
+  cuuint32_t box[2] = {box_inner, (cuuint32_t)TILE};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -406,70 +547,52 @@ sa_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t 
   return SA_OK;
 }
 
-int clusters_for(int C) {
-  const DeviceInfo& di = device_info();
+std::mutex g_mu;
+bool g_attr_set[64] = {};
+
+void set_attributes() {
+  const int dev = device_info().device & 63;
   std::lock_guard<std::mutex> lock(g_mu);
-  Cached& c = g_cache[di.device & 63];
-  if (!c.init) {
-    cudaFuncSetAttribute(sa_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    cudaFuncSetAttribute(sa_fwd_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    for (int cs = 1; cs <= MAXC; ++cs) {
-      cudaLaunchConfig_t cfg = {};
-      cudaLaunchAttribute at[1];
-      at[0].id = cudaLaunchAttributeClusterDimension;
-      at[0].val.clusterDim.x = cs;
-      at[0].val.clusterDim.y = 1;
-      at[0].val.clusterDim.z = 1;
-      cfg.gridDim = dim3(cs * (di.sm_count / cs), 1, 1);
-      cfg.blockDim = dim3(THREADS, 1, 1);
-      cfg.dynamicSmemBytes = SMEM_BYTES;
-      cfg.attrs = at;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, sa_fwd_tc_kernel, &cfg) != cudaSuccess || n < 1) {
-        cudaGetLastError();
-        n = std::max(1, di.sm_count / cs);
-      }
-      c.clusters[cs] = n;
-    }
-    c.init = true;
-  }
-  return c.clusters[C];
+  if (g_attr_set[dev]) return;
+  cudaFuncSetAttribute(sa_lse_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L_SMEM);
+  cudaFuncSetAttribute(sa_agg_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, A_SMEM);
+  g_attr_set[dev] = true;
 }
 }  // namespace
 
 bool sa_tc_supported(sa_dtype x_dtype, int k, int d) {
-  return x_dtype == SA_BF16 && d == DD && k % TILE == 0 && k / TILE >= 1 && k / TILE <= MAXC;
+  return x_dtype == SA_BF16 && d == DD && k % TILE == 0 && k >= TILE && k <= 4096;
 }
 
-int sa_tc_num_chunks(int k) { return clusters_for(k / TILE); }
+// token chunks of the aggregation kernel: one CTA per (slice, chunk), about one wave
+int sa_tc_num_chunks(int k) { return std::max(1, device_info().sm_count / (k / TILE)); }
 
 sa_status sa_tc_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st) {
-  const int C = a.k / TILE;
   if (a.n_total >= (1LL << 31)) return fail(SA_ERR_UNSUPPORTED, "n_total must be < 2^31");
-  CUtensorMap tmX, tmP;
-  sa_status s = make_map(&tmX, a.X, DD, (uint64_t)a.n_total, 16, TILE, CU_TENSOR_MAP_SWIZZLE_32B);
-  if (s != SA_OK) return s;
-  s = make_map(&tmP, w.Pb, DD, (uint64_t)a.k, 64, TILE, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != SA_OK) return s;
-  Params p{a.off_dev, a.B, w.ch, a.k, a.S, w.Muser, w.slotH, w.slotM, a.lse_out,
-           device_status_word()};
-  clusters_for(C);   // sets the kernel attributes once per device
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = C;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(C * w.ch.G, 1, 1);
-  cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = st;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  cudaError_t le = cudaSuccess;
-  SA_TIMED("sa_fwd_tc_kernel", st, (le = cudaLaunchKernelEx(&cfg, sa_fwd_tc_kernel, tmX, tmP, p)));
-  if (le != cudaSuccess) return cuda_fail(le, "sa_fwd_tc_kernel launch");
+  // the per-token log-sum-exp goes to the workspace (log2 units) or, when the
+  // workspace has none, to the caller's natural-log output
+  float* lse_a = w.lse;
+  float a_scale = 1.f, in_scale = 1.f;
+  float* lse_b = a.lse_out;
+  if (!lse_a) {
+    if (!a.lse_out) return fail(SA_ERR_INVALID_ARG, "the forward needs an lse buffer");
+    lse_a = a.lse_out;
+    lse_b = nullptr;
+    a_scale = kLn2f;
+    in_scale = kLog2ef;
+  }
+  CUtensorMap tmX128, tmX32, tmP;
+  sa_status s;
+  if ((s = make_map(&tmX128, a.X, (uint64_t)a.n_total, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != SA_OK) return s;
+  if ((s = make_map(&tmX32, a.X, (uint64_t)a.n_total, 16, CU_TENSOR_MAP_SWIZZLE_32B)) != SA_OK) return s;
+  if ((s = make_map(&tmP, w.Pb, (uint64_t)a.k, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != SA_OK) return s;
+  set_attributes();
+  const Chunking ch1 = make_chunking(a.n_total, device_info().sm_count, 1);
+  LParams lp{a.off_dev, a.B, ch1, a.k, lse_a, a_scale, lse_b, device_status_word()};
+  SA_TIMED("sa_lse_tc_kernel", st, (sa_lse_tc_kernel<<<ch1.G, L_THREADS, L_SMEM, st>>>(tmX128, tmP, lp)));
+  AParams ap{a.off_dev, a.B, w.ch, a.k, lse_a, in_scale, a.S, w.Muser, w.slotH, w.slotM, device_status_word()};
+  SA_TIMED("sa_agg_tc_kernel", st,
+           (sa_agg_tc_kernel<<<(a.k / TILE) * w.ch.G, A_THREADS, A_SMEM, st>>>(tmX32, tmP, ap)));
   return SA_OK;
 }
 
