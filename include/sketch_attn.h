@@ -115,6 +115,8 @@ sa_status sa_forward(const void* X, sa_dtype x_dtype,
  * nothing.
  * Limits: x_dtype = SA_BF16, d = 128, k a multiple of 128 up to 512,
  * 1 <= B <= 8; anything else returns SA_ERR_UNSUPPORTED before any GPU work.
+ * With lse = NULL the per-token log-sum-exp also takes scratch (4 bytes per
+ * token), which bounds n_total; pass lse to lift that bound.
  * Calls share the array: calls that overlap on the GPU (other streams, other
  * host threads) race and must be serialised.  No scratch word needs to start
  * at zero.  The first call on each device looks up the array's address, with
