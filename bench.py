@@ -50,7 +50,10 @@ def load_peaks():
 # --------------------------------------------------------------------------
 # clocks during the timed region
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons during the timed region: sampling
+    starts (and is confirmed running) on entry, the region is the time between
+    entry and exit, and only samples stamped inside it are summarised."""
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -58,6 +61,7 @@ class ClockSampler:
         self.dev = device_index
         self.proc = None
         self.path = os.path.join("/tmp", f"sa_bench_clocks_{os.getpid()}.csv")
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
@@ -66,18 +70,32 @@ class ClockSampler:
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.QUERY}",
                  "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
+            deadline = time.time() + 5.0            # wait for the first sample (before timing)
+            while time.time() < deadline and os.path.getsize(self.path) == 0:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
+        self.t0 = time.time()
         return self
 
     def __exit__(self, *exc):
+        self.t1 = time.time()
         if self.proc is not None:
+            time.sleep(0.1)                         # let the last sample of the region land
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
             self.f.close()
+
+    @staticmethod
+    def _epoch(ts):
+        import datetime
+        try:
+            return datetime.datetime.strptime(ts, "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
 
     def summary(self):
         if self.proc is None:
@@ -86,16 +104,19 @@ class ClockSampler:
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                if len(parts) >= 10 and parts[2].replace(".", "").isdigit():
                     rows.append(parts)
+        inside = [r for r in rows if (lambda e: e is not None and self.t0 <= e <= self.t1)(self._epoch(r[0]))]
+        if inside:
+            rows = inside
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows]
+        sm = [float(r[2]) for r in rows]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
-                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
-                "samples": len(rows), "reasons": reasons}
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][3]),
+                "power_w_max": max(float(r[4]) for r in rows if r[4].replace(".", "").isdigit()),
+                "samples": len(rows), "samples_in_region": len(inside), "reasons": reasons}
 
 
 # --------------------------------------------------------------------------
