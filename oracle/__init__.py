@@ -21,6 +21,12 @@ Readings where the pages leave a step open (each is an explicit choice):
   to the query (eq. 4 plus the W_O term of eq. 26); no FFN, no LayerNorm.
 * STCA over an empty key range: the attention output is zero.
 * Fusion: a linear map [z_r; z_u] W_F + b_F (Sec. 3.4 leaves the fusion open).
+* Stacked refinement (Sec. 3.3): X^ = A X exactly as eq. (14) writes it (the
+  sum over the user's events, no mass normalisation); LN is a row LayerNorm
+  over d with biased variance, eps and an optional gain and bias; the FFN is
+  SwiGLU with inner width 2d and no biases (eq. (23) counts 6 T w w_f FLOPs
+  with w_f = 2w), SiLU on the first branch.  A user without events gets
+  X^ = 0.
 
 Parity pins (tests/test_oracle_*.py): per-token column sums, total mass,
 permutation invariance, k = 1 mean, uniform assignment at zero logits,
@@ -39,7 +45,8 @@ import numpy as np
 
 __all__ = [
     "sa_forward", "sa_user", "sa_backward", "stca_branch", "stca_branch_reordered",
-    "stca_fuse", "assignment", "token_lse",
+    "stca_fuse", "assignment", "token_lse", "layer_norm", "swiglu_ffn", "sa_refine_user",
+    "sa_refine",
 ]
 
 
@@ -236,4 +243,62 @@ def stca_fuse(z_r, z_u, W_F, b_F=None):
     out = z @ _f64(W_F)
     if b_F is not None:
         out = out + _f64(b_F)[None, :]
+    return out
+
+
+# --------------------------------------------------------------------------
+# Stacked refinement
+# --------------------------------------------------------------------------
+def layer_norm(Y, g=None, b=None, eps: float = 1e-5) -> np.ndarray:
+    """LN over the last axis (Sec. 3.3, eqs. (15)-(16)): (y - mean) / sqrt(var + eps),
+    biased variance, then times the gain g and plus the bias b when given."""
+    Y = _f64(Y)
+    mu = Y.mean(axis=-1, keepdims=True)
+    var = ((Y - mu) ** 2).mean(axis=-1, keepdims=True)
+    out = (Y - mu) / np.sqrt(var + eps)
+    if g is not None:
+        out = out * _f64(g)
+    if b is not None:
+        out = out + _f64(b)
+    return out
+
+
+def swiglu_ffn(Y, W1, W3, W2) -> np.ndarray:
+    """The FFN of eq. (16): (SiLU(Y W1) * (Y W3)) W2 with SiLU(x) = x / (1 + e^-x);
+    W1, W3 [d, 2d], W2 [2d, d] (the SwiGLU of eq. (23) with inner width 2d)."""
+    Y = _f64(Y)
+    a = Y @ _f64(W1)
+    return ((a / (1.0 + np.exp(-a))) * (Y @ _f64(W3))) @ _f64(W2)
+
+
+def sa_refine_user(Xu, P0, layers, ln_eps: float = 1e-5) -> np.ndarray:
+    """One user's stacked refinement (Sec. 3.3), starting from X~(0) = P0 [k, d];
+    per iteration, with that iteration's weights:
+        S  = (X~ W_Q)(X W_K)^T / sqrt(d),  A = softmax over prototypes   (12)-(13)
+        X^ = A X                                                        (14)
+        Xbar = LN(X~ + X^)                                              (15)
+        X~ = LN(Xbar + FFN(Xbar))                                       (16)
+    ``layers``: dicts with W_Q, W_K, W1, W3, W2 and optional ln1_g, ln1_b, ln2_g,
+    ln2_b.  Returns X~ after the last iteration."""
+    Xu = _f64(Xu)
+    Xt = _f64(P0)
+    for L in layers:
+        if Xu.shape[0] == 0:
+            Xhat = np.zeros_like(Xt)
+        else:
+            Xhat = assignment(Xu, Xt, L["W_Q"], L["W_K"]) @ Xu
+        Xbar = layer_norm(Xt + Xhat, L.get("ln1_g"), L.get("ln1_b"), ln_eps)
+        Xt = layer_norm(Xbar + swiglu_ffn(Xbar, L["W1"], L["W3"], L["W2"]), L.get("ln2_g"),
+                        L.get("ln2_b"), ln_eps)
+    return Xt
+
+
+def sa_refine(X, offsets: Sequence[int], P0, layers, ln_eps: float = 1e-5) -> np.ndarray:
+    """Refined sketches of a ragged batch: [B, k, d] fp64."""
+    offsets = np.asarray(offsets, np.int64)
+    B = len(offsets) - 1
+    k, d = np.shape(P0)
+    out = np.zeros((B, k, d))
+    for u in range(B):
+        out[u] = sa_refine_user(X[offsets[u]:offsets[u + 1]], P0, layers, ln_eps)
     return out

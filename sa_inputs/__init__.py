@@ -326,6 +326,27 @@ def stca_layers(rng, n_layers: int, D: int, heads: int, d_h: int, with_wo: bool 
     return out
 
 
+def refine_layers(rng, n_iter: int, d: int, affine: bool = True):
+    """Weights of the stacked refinement, one dict per iteration: W_Q, W_K [d, d]
+    and the SwiGLU FFN W1, W3 [d, 2d] (std 1/sqrt(d)), W2 [2d, d] (std 1/sqrt(2d));
+    with ``affine`` the LN gains ~ 1 + 0.1 N(0, 1) and biases ~ 0.1 N(0, 1)."""
+    out = []
+    for _ in range(n_iter):
+        L = {"W_Q": gauss(rng, (d, d), 1.0 / math.sqrt(d)),
+             "W_K": gauss(rng, (d, d), 1.0 / math.sqrt(d)),
+             "W1": gauss(rng, (d, 2 * d), 1.0 / math.sqrt(d)),
+             "W3": gauss(rng, (d, 2 * d), 1.0 / math.sqrt(d)),
+             "W2": gauss(rng, (2 * d, d), 1.0 / math.sqrt(2 * d))}
+        for key in ("ln1", "ln2"):
+            if affine:
+                L[key + "_g"] = (1.0 + gauss(rng, (d,), 0.1)).astype(np.float32)
+                L[key + "_b"] = gauss(rng, (d,), 0.1)
+            else:
+                L[key + "_g"] = L[key + "_b"] = None
+        out.append(L)
+    return out
+
+
 def suffix_ranges(offsets: np.ndarray, L_r: int = L_RECENT):
     """The recent suffix X_r of each user as a [begin, end) row range (eq. 3);
     a user shorter than L_r contributes its whole history."""
