@@ -162,6 +162,45 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype,
                       void* workspace, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Stacked refinement                                                        */
+/* ------------------------------------------------------------------------ */
+
+/* One refinement iteration's parameters (device pointers, fp32, row-major). */
+typedef struct {
+  const float* W_Q;     /* [d, d]  eq. (12) */
+  const float* W_K;     /* [d, d]  eq. (12) */
+  const float* ln1_g;   /* [d] gain of the LN of eq. (15), or NULL for ones */
+  const float* ln1_b;   /* [d] bias of that LN, or NULL for zeros */
+  const float* W1;      /* [d, 2d] SwiGLU FFN of eq. (16): the SiLU-gated branch */
+  const float* W3;      /* [d, 2d] the linear branch */
+  const float* W2;      /* [2d, d] the output projection */
+  const float* ln2_g;   /* [d] gain of the LN of eq. (16), or NULL for ones */
+  const float* ln2_b;   /* [d] bias of that LN, or NULL for zeros */
+} sa_refine_layer;
+
+size_t sa_refine_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype);
+
+/*
+ * sa_refine_forward -- stacked SA refinement (paper Sec. 3.3, eqs. (12)-(16)),
+ * n_iter iterations starting from the shared prototypes X~(0) = P0 [k, d]:
+ *   A     = softmax over prototypes of (X~ W_Q)(X_u W_K)^T / sqrt(d)   (12)-(13)
+ *   X^    = A X_u                     (14, the sum over the user's events)
+ *   Xbar  = LN(X~ + X^)               (15)
+ *   X~    = LN(Xbar + FFN(Xbar)),  FFN(y) = (SiLU(y W1) * (y W3)) W2   (16)
+ * From the second iteration on the prototypes X~ are per user.  LN normalises
+ * each row over d (mean, biased variance, ln_eps), then applies gain and bias.
+ * Output: sketch [B, k, d] fp32 = X~(n_iter).  X, offsets as in sa_forward;
+ * layers: host array of n_iter structs.  Tensor-core path only: x_dtype =
+ * SA_BF16, d = 128, k a multiple of 128 (else SA_ERR_UNSUPPORTED).  The
+ * caller owns every buffer; asynchronous on `stream`.
+ */
+sa_status sa_refine_forward(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                            const int64_t* offsets_dev, int B, int k, int d, const float* P0,
+                            int n_iter, const sa_refine_layer* layers, float ln_eps,
+                            float* sketch, void* workspace, size_t ws_bytes,
+                            sa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* STCA: stacked target-to-history single-query cross attention             */
 /* ------------------------------------------------------------------------ */
 /* Weights of one STCA layer (device pointers). */

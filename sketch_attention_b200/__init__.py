@@ -28,7 +28,7 @@ _STATUS = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_
 EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_workspace",
            "sa_forward", "sa_backward_workspace", "sa_backward", "stca_forward_workspace",
            "stca_forward", "stca_fuse", "sa_launch_count", "sa_profile", "sa_profile_read",
-           "sa_forward_noalloc")
+           "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward")
 
 
 class SAError(RuntimeError):
@@ -40,6 +40,11 @@ class SAError(RuntimeError):
 class StcaLayerC(ctypes.Structure):
     _fields_ = [("W_Q", ctypes.c_void_p), ("W_K", ctypes.c_void_p),
                 ("W_V", ctypes.c_void_p), ("W_O", ctypes.c_void_p)]
+
+
+class RefineLayerC(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in ("W_Q", "W_K", "ln1_g", "ln1_b", "W1", "W3", "W2",
+                                               "ln2_g", "ln2_b")]
 
 
 _lib = None
@@ -80,6 +85,11 @@ def load(path: Optional[str] = None):
     lib.sa_forward_noalloc.restype = _i
     lib.sa_forward_noalloc.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
                                        _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.sa_refine_workspace.restype = _sz
+    lib.sa_refine_workspace.argtypes = [_i, _i64, _i, _i, _i]
+    lib.sa_refine_forward.restype = _i
+    lib.sa_refine_forward.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _i,
+                                      ctypes.POINTER(RefineLayerC), _f, _vp, _vp, _sz, _vp]
     lib.sa_launch_count.restype = ctypes.c_longlong
     lib.sa_profile.restype = _i
     lib.sa_profile.argtypes = [_i]
@@ -271,6 +281,44 @@ def stca_forward(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin, kv_e
                           _p(kbd), _p(ked), D, heads, d_h, len(layers), arr, _p(res),
                           _p(workspace), workspace.numel(), _stream(stream))
     _check("stca_forward", st)
+    return res
+
+
+REFINE_KEYS = ("W_Q", "W_K", "ln1_g", "ln1_b", "W1", "W3", "W2", "ln2_g", "ln2_b")
+
+
+def sa_refine_workspace(B: int, n_total: int, k: int, d: int, x_dtype: int) -> int:
+    return int(load().sa_refine_workspace(B, n_total, k, d, x_dtype))
+
+
+def sa_refine_forward(X: torch.Tensor, offsets, P0: torch.Tensor, layers: Sequence[dict],
+                      ln_eps: float = 1e-5, *, offsets_dev=None, out: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Stacked SA refinement, len(layers) iterations from the shared prototypes P0
+    [k, d].  ``layers``: dicts with W_Q, W_K [d, d], W1, W3 [d, 2d], W2 [2d, d] and
+    optional ln1_g, ln1_b, ln2_g, ln2_b [d] (fp32 CUDA tensors).  Returns the
+    sketch [B, k, d] fp32."""
+    lib = load()
+    _need_cuda(X, P0)
+    dt = _dtype_code(X)
+    off = _host_i64(offsets)
+    B = len(off) - 1
+    k, d = P0.shape
+    dev = X.device
+    res = out if out is not None else torch.empty(B, k, d, device=dev)
+    arr = (RefineLayerC * len(layers))()
+    for i, L in enumerate(layers):
+        for key in REFINE_KEYS:
+            t = L.get(key)
+            _need_cuda(t)
+            setattr(arr[i], key, t.data_ptr() if t is not None else None)
+    ws_bytes = lib.sa_refine_workspace(B, int(off[-1]), k, d, dt)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    od = _dev_i64(off, dev, offsets_dev)
+    st = lib.sa_refine_forward(_p(X), dt, _hp(off), _p(od), B, k, d, _p(P0), len(layers), arr,
+                               ln_eps, _p(res), _p(workspace), workspace.numel(), _stream(stream))
+    _check("sa_refine_forward", st)
     return res
 
 

@@ -337,6 +337,53 @@ sa_status sa_forward(const void* X, sa_dtype x_dtype, const int64_t* offsets_hos
   return sa_reduce_and_project(a, w, st);
 }
 
+size_t sa_refine_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype) {
+  if (B < 1 || k < 1 || d < 1 || n_total < 0 || !sa_tc_supported(x_dtype, k, d)) return 0;
+  return refine_layout(nullptr, B, n_total, k, d, nullptr, nullptr);
+}
+
+sa_status sa_refine_forward(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                            const int64_t* offsets_dev, int B, int k, int d, const float* P0,
+                            int n_iter, const sa_refine_layer* layers, float ln_eps,
+                            float* sketch, void* workspace, size_t ws_bytes,
+                            sa_stream_t stream) {
+  SA_TRY(check_sa_shape(B, k, d, x_dtype));
+  if (!sa_tc_supported(x_dtype, k, d))
+    return fail(SA_ERR_UNSUPPORTED, "sa_refine_forward needs bf16 X, d = 128 and k a multiple of 128");
+  SA_TRY(check_offsets(offsets_host, B, "offsets_host"));
+  const int64_t n = offsets_host[B];
+  if (n >= (1LL << 31)) return fail(SA_ERR_UNSUPPORTED, "n_total must be < 2^31");
+  if (n_iter < 1) return fail(SA_ERR_INVALID_ARG, "n_iter must be >= 1");
+  if (!layers) return fail(SA_ERR_INVALID_ARG, "layers is NULL");
+  if (!(ln_eps > 0.f)) return fail(SA_ERR_INVALID_ARG, "ln_eps must be > 0");
+  if ((int64_t)B * k >= (1LL << 31)) return fail(SA_ERR_UNSUPPORTED, "B * k must be < 2^31");
+  SA_TRY(check_ptr(X, "X", n == 0));
+  SA_TRY(check_ptr(offsets_dev, "offsets_dev"));
+  SA_TRY(check_ptr(P0, "P0"));
+  SA_TRY(check_ptr(sketch, "sketch"));
+  for (int i = 0; i < n_iter; ++i) {
+    const sa_refine_layer& L = layers[i];
+    SA_TRY(check_ptr(L.W_Q, "layers[].W_Q"));
+    SA_TRY(check_ptr(L.W_K, "layers[].W_K"));
+    SA_TRY(check_ptr(L.W1, "layers[].W1"));
+    SA_TRY(check_ptr(L.W3, "layers[].W3"));
+    SA_TRY(check_ptr(L.W2, "layers[].W2"));
+    SA_TRY(check_ptr(L.ln1_g, "layers[].ln1_g", true));
+    SA_TRY(check_ptr(L.ln1_b, "layers[].ln1_b", true));
+    SA_TRY(check_ptr(L.ln2_g, "layers[].ln2_g", true));
+    SA_TRY(check_ptr(L.ln2_b, "layers[].ln2_b", true));
+  }
+  const size_t need = refine_layout(nullptr, B, n, k, d, nullptr, nullptr);
+  if (!workspace || ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "workspace needs " + std::to_string(need) + " bytes");
+  SA_TRY(check_ptr(workspace, "workspace"));
+  SaFwdWork w;
+  RefineWork r;
+  refine_layout(workspace, B, n, k, d, &w, &r);
+  return sa_refine_run(X, x_dtype, offsets_dev, B, n, k, d, P0, n_iter, layers, ln_eps, sketch, w, r,
+                       (cudaStream_t)stream);
+}
+
 size_t sa_backward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype) {
   if (B < 1 || k < 1 || d < 1 || n_total < 0) return 0;
   return layout_bwd(nullptr, B, n_total, k, d, x_dtype, nullptr);

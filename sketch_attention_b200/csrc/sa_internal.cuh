@@ -12,6 +12,7 @@ struct SaFwdArgs {
   const float *P, *W_Q, *W_K, *W_V;
   float eps;
   float* S; float* mass; float* H; void* S_bf16; float* lse_out;
+  int p_user_rows = 0;   // k: P is [B, k, d], one set of prototypes per user; 0: P is [k, d]
 };
 
 // Workspace views of sa_forward.
@@ -63,6 +64,27 @@ constexpr int kMaxSplit = 256;
 sa_status sa_fold(int k, int d, const float* P, const float* W_Q, const float* W_K, float* T,
                   float* Pf, __nv_bfloat16* Pb, cudaStream_t st);
 sa_status sa_simt_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
+// Stacked refinement (sa_refine.cu): buffers besides the forward's workspace.
+struct RefineWork {
+  float* Huser;   // [B, k, d] the forward's per-user accumulator
+  float* H;       // [B, k, d] A X
+  float* mass;    // [B, k]
+  float* Xbar;    // [B, k, d]
+  float* G1;      // [B, k, 2d]
+  float* G3;      // [B, k, 2d]
+  float* U;       // [B, k, 2d]
+  float* F;       // [B, k, d]
+};
+// Lays out the forward workspace (P' per user) and the refinement buffers;
+// returns the bytes needed.
+size_t refine_layout(void* base, int B, int64_t n, int k, int d, SaFwdWork* w, RefineWork* r);
+sa_status sa_refine_run(const void* X, sa_dtype x_dtype, const int64_t* off_dev, int B, int64_t n,
+                        int k, int d, const float* P0, int n_iter, const sa_refine_layer* layers,
+                        float ln_eps, float* sketch, const SaFwdWork& w, const RefineWork& r,
+                        cudaStream_t st);
+
+// Sums the split-n partials into H (if a.H), the mass and H/(m+eps) (w.Hhat).
+sa_status sa_reduce(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
 sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
 sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaStream_t st);
 sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st);
@@ -75,7 +97,7 @@ sa_status sa_bwd_tc_run(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st)
 
 // Tensor-core forward (sa_tc.cu).
 bool sa_tc_supported(sa_dtype x_dtype, int k, int d);
-int sa_tc_num_chunks(int k);       // number of clusters the persistent launch uses
+int sa_tc_num_chunks(int k);       // token chunks of the aggregation kernel (one CTA per slice and chunk)
 sa_status sa_tc_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
 
 }  // namespace sa

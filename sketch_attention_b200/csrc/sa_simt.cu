@@ -510,12 +510,18 @@ sa_status sa_simt_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t s
             : launch_simt_forward<float, 128>(a, w, st);
 }
 
-sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st) {
+sa_status sa_reduce(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st) {
   dim3 grid((a.k + 7) / 8, a.B);
   SA_TIMED("sa_reduce_kernel", st,
            (sa_reduce_kernel<<<grid, 256, 0, st>>>(a.off_dev, a.B, w.ch, a.k, a.d, a.eps, a.S,
                                                    w.Muser, w.slotH, w.slotM, a.H, a.mass,
                                                    w.Hhat)));
+  return SA_OK;
+}
+
+sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st) {
+  sa_status s = sa_reduce(a, w, st);
+  if (s != SA_OK) return s;
   // S = Hh W_V (and its bf16 copy)
   Gemm g;
   g.M = a.B * a.k; g.N = a.d; g.K = a.d;

@@ -115,6 +115,7 @@ struct LParams {
   float* lse_a;        // [n] required output: the log2-sum-exp times a_scale
   float a_scale;       // 1 (log2 units) or ln 2 (natural units)
   float* lse_b;        // [n] optional natural-log copy
+  int p_user_rows;     // rows of P' per user (k: per-user prototypes), 0: one shared P'
   int* err;
 };
 
@@ -154,8 +155,9 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
     prefetch_tensormap(&tmX);
     prefetch_tensormap(&tmP);
     int cc = 0, issued_t = 0, issued_c = 0;
-    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t, bool, bool) {
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int u, int64_t tb, int64_t, bool, bool) {
       const int s = t % L_NXS;
+      const int prow0 = u * p.p_user_rows;
       if (t >= L_NXS && !mbar_wait(&bars->x_empty[s], ((t / L_NXS) - 1) & 1, abort, p.err)) return false;
       mbar_arrive_expect_tx(&bars->x_full[s], T_BYTES);
       uint8_t* xd = smem + L_OFF_X + s * T_BYTES;
@@ -167,8 +169,8 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
         if (cc >= L_NPS && !mbar_wait(&bars->c_empty[cs], ((cc / L_NPS) - 1) & 1, abort, p.err)) return false;
         mbar_arrive_expect_tx(&bars->c_full[cs], T_BYTES);
         uint8_t* pd = smem + L_OFF_P + cs * T_BYTES;
-        tma_load_2d(pd, &tmP, &bars->c_full[cs], 0, c * TILE);
-        tma_load_2d(pd + T_BYTES / 2, &tmP, &bars->c_full[cs], 64, c * TILE);
+        tma_load_2d(pd, &tmP, &bars->c_full[cs], 0, prow0 + c * TILE);
+        tma_load_2d(pd + T_BYTES / 2, &tmP, &bars->c_full[cs], 64, prow0 + c * TILE);
         issued_c = cc + 1;
       }
       return true;
@@ -296,7 +298,7 @@ constexpr uint32_t A_TM_S = 0, A_TM_H = 256, A_TM_COLS = 512;   // logits 2 x 12
 
 struct ABars {
   uint64_t x_full[A_NS], x_empty[A_NS], s_full[2], s_empty[2], p_full[A_NP], p_empty[A_NP];
-  uint64_t h_full, h_empty, pq_full, mma_done[2];
+  uint64_t h_full, h_empty, pq_full, pq_empty, mma_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -313,6 +315,7 @@ struct AParams {
   float* Muser;        // [B, k]
   float* slotH;        // [G, 2, k, d] pieces at chunk boundaries
   float* slotM;        // [G, 2, k]
+  int p_user_rows;     // rows of P' per user (k: per-user prototypes), 0: one shared P'
   int* err;
 };
 
@@ -335,6 +338,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
     mbar_init(&bars->h_full, 1);
     mbar_init(&bars->h_empty, 128);
     mbar_init(&bars->pq_full, 1);
+    mbar_init(&bars->pq_empty, 1);
     mbar_init(&bars->mma_done[0], 1);
     mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
@@ -359,11 +363,18 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
     // ------------------------------------------------------------ TMA producer
     prefetch_tensormap(&tmX);
     prefetch_tensormap(&tmP);
-    mbar_arrive_expect_tx(&bars->pq_full, T_BYTES);
-    tma_load_2d(smem + A_OFF_PQ, &tmP, &bars->pq_full, 0, sl * TILE);
-    tma_load_2d(smem + A_OFF_PQ + T_BYTES / 2, &tmP, &bars->pq_full, 64, sl * TILE);
-    int issued = 0;
-    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t, bool, bool) {
+    const bool per_user = p.p_user_rows > 0;
+    int issued = 0, pq_issued = 0;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int u, int64_t tb, int64_t, bool first, bool) {
+      // the P' slice: once, or at every user's first tile when the prototypes are per user
+      if (first && (piece == 0 || per_user)) {
+        if (piece > 0 && !mbar_wait(&bars->pq_empty, (piece - 1) & 1, abort, p.err)) return false;
+        mbar_arrive_expect_tx(&bars->pq_full, T_BYTES);
+        const int prow = u * p.p_user_rows + sl * TILE;
+        tma_load_2d(smem + A_OFF_PQ, &tmP, &bars->pq_full, 0, prow);
+        tma_load_2d(smem + A_OFF_PQ + T_BYTES / 2, &tmP, &bars->pq_full, 64, prow);
+        pq_issued = piece + 1;
+      }
       const int s = t % A_NS;
       if (t >= A_NS && !mbar_wait(&bars->x_empty[s], ((t / A_NS) - 1) & 1, abort, p.err)) return false;
       mbar_arrive_expect_tx(&bars->x_full[s], 8 * X_BOX);
@@ -373,7 +384,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
       return true;
     });
     if (*abort) {
-      mbar_wait_bounded(&bars->pq_full, 0);
+      if (pq_issued > 0) mbar_wait_bounded(&bars->pq_full, (pq_issued - 1) & 1);
       for (int t = std::max(0, issued - A_NS); t < issued; ++t)
         mbar_wait_bounded(&bars->x_full[t % A_NS], (t / A_NS) & 1);
     }
@@ -381,9 +392,13 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
     // ------------------------------------------------------------ logits MMAs
     const uint32_t id1 = idesc_bf16(128, 128, false, false);
     const uint32_t pq = smem_u32(smem + A_OFF_PQ);
-    if (mbar_wait(&bars->pq_full, 0, abort, p.err)) {
-      for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
+    const bool per_user = p.p_user_rows > 0;
+    {
+      for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t, int64_t, bool first, bool last) {
         const int s = t % A_NS, b = t & 1;
+        if (first && (piece == 0 || per_user) &&
+            !mbar_wait(&bars->pq_full, (per_user ? piece : 0) & 1, abort, p.err))
+          return false;
         if (!mbar_wait(&bars->x_full[s], (t / A_NS) & 1, abort, p.err)) return false;
         if (t >= 2 && !mbar_wait(&bars->s_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return false;
         tc_fence_after();
@@ -394,6 +409,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
                  smem_desc(pq + (ks >> 2) * (T_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B), id1,
                  ks > 0 ? 1u : 0u);
         mma_commit(&bars->s_full[b]);
+        if (last && per_user) mma_commit(&bars->pq_empty);   // this user's P' slice is done
         return true;
       });
     }
@@ -585,12 +601,14 @@ sa_status sa_tc_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st)
   sa_status s;
   if ((s = make_map(&tmX128, a.X, (uint64_t)a.n_total, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != SA_OK) return s;
   if ((s = make_map(&tmX32, a.X, (uint64_t)a.n_total, 16, CU_TENSOR_MAP_SWIZZLE_32B)) != SA_OK) return s;
-  if ((s = make_map(&tmP, w.Pb, (uint64_t)a.k, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != SA_OK) return s;
+  const uint64_t p_rows = (uint64_t)a.k * (a.p_user_rows > 0 ? (uint64_t)a.B : 1);
+  if ((s = make_map(&tmP, w.Pb, p_rows, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != SA_OK) return s;
   set_attributes();
   const Chunking ch1 = make_chunking(a.n_total, device_info().sm_count, 1);
-  LParams lp{a.off_dev, a.B, ch1, a.k, lse_a, a_scale, lse_b, device_status_word()};
+  LParams lp{a.off_dev, a.B, ch1, a.k, lse_a, a_scale, lse_b, a.p_user_rows, device_status_word()};
   SA_TIMED("sa_lse_tc_kernel", st, (sa_lse_tc_kernel<<<ch1.G, L_THREADS, L_SMEM, st>>>(tmX128, tmP, lp)));
-  AParams ap{a.off_dev, a.B, w.ch, a.k, lse_a, in_scale, a.S, w.Muser, w.slotH, w.slotM, device_status_word()};
+  AParams ap{a.off_dev, a.B, w.ch, a.k, lse_a, in_scale, a.S, w.Muser, w.slotH, w.slotM, a.p_user_rows,
+             device_status_word()};
   SA_TIMED("sa_agg_tc_kernel", st,
            (sa_agg_tc_kernel<<<(a.k / TILE) * w.ch.G, A_THREADS, A_SMEM, st>>>(tmX32, tmP, ap)));
   return SA_OK;
