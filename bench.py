@@ -498,6 +498,24 @@ def run_component(args, rank, world, device):
                                       workspace=ws)
         units, unit, name = p.n_total, "history-tokens/s", p.name
         kname, flops = "sa_agg_tc_kernel", 2.0 * p.k * p.d * p.n_total
+    elif args.workload == "refine":
+        from sa_inputs import refine_layers, rng_for
+        p = sa_workload(5, users=args.users)
+        X = _dev_bf16(p.X, device)
+        offd = torch.from_numpy(p.offsets).to(device)
+        P0 = _f32(p.P, device)
+        layers = [{k: (_f32(v, device) if v is not None else None) for k, v in L.items()}
+                  for L in refine_layers(rng_for(5005), 2, p.d)]
+        out = torch.empty(p.B, p.k, p.d, device=device)
+        ws = torch.empty(sab.sa_refine_workspace(p.B, p.n_total, p.k, p.d, sab.SA_BF16),
+                         dtype=torch.uint8, device=device)
+        step = lambda: sab.sa_refine_forward(X, p.offsets, P0, layers, 1e-5, offsets_dev=offd,
+                                             out=out, workspace=ws)
+        units, unit = p.n_total, "history-tokens/s"
+        name = (f"stacked SA refinement, 2 iterations (per-user prototypes in the second), "
+                f"{p.B} users x mean {p.n_total // max(p.B, 1)} events, k={p.k}, d={p.d}, bf16")
+        # per launch of the dominant kernel: H = A X with its mass (2kd flop per token)
+        kname, flops = "sa_agg_tc_kernel", 2.0 * p.k * p.d * p.n_total
     else:
         w = stca_workload(users=args.users or 16)
         q, kvr, kvs = (_dev_bf16(a, device) for a in (w.recent.q, w.recent.kv, w.sketch.kv))
@@ -558,9 +576,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca"], default="train",
+    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "refine"], default="train",
                     help="train: the full step (default, the headline); sa_fwd: SA forward over "
-                         "32 users x 100K (k=1024); stca: STCA of 16 users x 512 candidates")
+                         "32 users x 100K (k=1024); stca: STCA of 16 users x 512 candidates; "
+                         "refine: stacked SA refinement, 2 iterations, on the train step's users")
     ap.add_argument("--users", type=int, default=None, help="shrink the batch (profiling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -12,55 +12,59 @@
 namespace sa {
 
 namespace {
-constexpr int kMaxPerLane = 32;   // d <= 1024
-
-// out[r, :] = LN(a[ra, :] + b[r, :]) * g + beta, one warp per row; ra = r, or
-// r % a_rows when a holds a_rows rows shared by every user (the first
-// iteration's prototypes).  Mean and biased variance over d.
+// out[r, :] = LN(a[ra, :] + b[r, :]) * g + beta, one warp per row (D = 32 * V
+// features, V per lane as float4s); ra = r, or r % a_rows when a holds a_rows
+// rows shared by every user (the first iteration's prototypes).  Mean and
+// biased variance over D.
+template <int V>
 __global__ void __launch_bounds__(256) residual_ln_kernel(const float* __restrict__ a, int a_rows,
                                                           const float* __restrict__ b,
                                                           const float* __restrict__ g,
                                                           const float* __restrict__ beta, float eps,
-                                                          int64_t rows, int d, float* __restrict__ out) {
+                                                          int64_t rows, float* __restrict__ out) {
+  constexpr int D = 32 * V;
   const int64_t r = ((int64_t)blockIdx.x * 256 + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
   if (r >= rows) return;
   const int64_t ra = a_rows > 0 ? r % a_rows : r;
-  float v[kMaxPerLane];
+  float v[V];
   float sum = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
-    const int c = lane + 32 * i;
-    v[i] = c < d ? a[ra * d + c] + b[r * d + c] : 0.f;
-    sum += v[i];
+  for (int i = 0; i < V; i += 4) {
+    const int c = lane * V + i;
+    const float4 x = *(const float4*)(a + ra * D + c), y = *(const float4*)(b + r * D + c);
+    v[i] = x.x + y.x; v[i + 1] = x.y + y.y; v[i + 2] = x.z + y.z; v[i + 3] = x.w + y.w;
+    sum += (v[i] + v[i + 1]) + (v[i + 2] + v[i + 3]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const float mean = sum / (float)d;
+  const float mean = sum / (float)D;
   float sq = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
-    const int c = lane + 32 * i;
-    const float t = c < d ? v[i] - mean : 0.f;
-    sq += t * t;
-  }
+  for (int i = 0; i < V; ++i) sq += (v[i] - mean) * (v[i] - mean);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-  const float rstd = rsqrtf(sq / (float)d + eps);
+  const float rstd = rsqrtf(sq / (float)D + eps);
 #pragma unroll
-  for (int i = 0; i < kMaxPerLane; ++i) {
-    const int c = lane + 32 * i;
-    if (c < d) out[r * d + c] = (v[i] - mean) * rstd * (g ? g[c] : 1.f) + (beta ? beta[c] : 0.f);
+  for (int i = 0; i < V; i += 4) {
+    const int c = lane * V + i;
+    float4 o;
+    o.x = (v[i] - mean) * rstd * (g ? g[c] : 1.f) + (beta ? beta[c] : 0.f);
+    o.y = (v[i + 1] - mean) * rstd * (g ? g[c + 1] : 1.f) + (beta ? beta[c + 1] : 0.f);
+    o.z = (v[i + 2] - mean) * rstd * (g ? g[c + 2] : 1.f) + (beta ? beta[c + 2] : 0.f);
+    o.w = (v[i + 3] - mean) * rstd * (g ? g[c + 3] : 1.f) + (beta ? beta[c + 3] : 0.f);
+    *(float4*)(out + r * D + c) = o;
   }
 }
 
-// U = SiLU(G1) * G3,  SiLU(x) = x / (1 + e^-x)
-__global__ void __launch_bounds__(256) swiglu_kernel(const float* __restrict__ G1,
-                                                     const float* __restrict__ G3, int64_t n,
-                                                     float* __restrict__ U) {
-  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n; i += (int64_t)gridDim.x * 256) {
-    const float x = G1[i];
-    U[i] = x / (1.f + expf(-x)) * G3[i];
+// U = SiLU(G1) * G3,  SiLU(x) = x / (1 + e^-x); n4 float4s
+__global__ void __launch_bounds__(256) swiglu_kernel(const float4* __restrict__ G1,
+                                                     const float4* __restrict__ G3, int64_t n4,
+                                                     float4* __restrict__ U) {
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n4; i += (int64_t)gridDim.x * 256) {
+    const float4 x = G1[i], y = G3[i];
+    U[i] = make_float4(x.x / (1.f + expf(-x.x)) * y.x, x.y / (1.f + expf(-x.y)) * y.y,
+                       x.z / (1.f + expf(-x.z)) * y.z, x.w / (1.f + expf(-x.w)) * y.w);
   }
 }
 
@@ -117,8 +121,8 @@ sa_status sa_refine_run(const void* X, sa_dtype x_dtype, const int64_t* off_dev,
     if ((s = sa_reduce(a, w, st)) != SA_OK) return s;
     // eq. (15): Xbar = LN(X~ + X^)
     SA_TIMED("residual_ln_kernel", st,
-             (residual_ln_kernel<<<blocks_for(rows * 32, 256), 256, 0, st>>>(
-                 Xt, per_user ? 0 : k, r.H, L.ln1_g, L.ln1_b, ln_eps, rows, d, r.Xbar)));
+             (residual_ln_kernel<4><<<blocks_for(rows * 32, 256), 256, 0, st>>>(
+                 Xt, per_user ? 0 : k, r.H, L.ln1_g, L.ln1_b, ln_eps, rows, r.Xbar)));
     // eq. (16): FFN(Xbar) = (SiLU(Xbar W1) * (Xbar W3)) W2
     Gemm g1;
     g1.M = (int)rows; g1.N = 2 * d; g1.K = d;
@@ -129,7 +133,8 @@ sa_status sa_refine_run(const void* X, sa_dtype x_dtype, const int64_t* off_dev,
     g3.B = L.W3; g3.C = r.G3;
     if ((s = gemm(g3, st)) != SA_OK) return s;
     SA_TIMED("swiglu_kernel", st,
-             (swiglu_kernel<<<blocks_for(rows * 2 * d, 256), 256, 0, st>>>(r.G1, r.G3, rows * 2 * d, r.U)));
+             (swiglu_kernel<<<blocks_for(rows * 2 * d / 4, 256), 256, 0, st>>>(
+                 (const float4*)r.G1, (const float4*)r.G3, rows * 2 * d / 4, (float4*)r.U)));
     Gemm g2;
     g2.M = (int)rows; g2.N = d; g2.K = 2 * d;
     g2.A = r.U; g2.lda = 2 * d; g2.B = L.W2; g2.ldb = d; g2.C = r.F; g2.ldc = d;
@@ -137,8 +142,8 @@ sa_status sa_refine_run(const void* X, sa_dtype x_dtype, const int64_t* off_dev,
     if ((s = gemm(g2, st)) != SA_OK) return s;
     // X~(it+1) = LN(Xbar + FFN), written over X~(it) (no longer read)
     SA_TIMED("residual_ln_kernel", st,
-             (residual_ln_kernel<<<blocks_for(rows * 32, 256), 256, 0, st>>>(
-                 r.Xbar, 0, r.F, L.ln2_g, L.ln2_b, ln_eps, rows, d, sketch)));
+             (residual_ln_kernel<4><<<blocks_for(rows * 32, 256), 256, 0, st>>>(
+                 r.Xbar, 0, r.F, L.ln2_g, L.ln2_b, ln_eps, rows, sketch)));
   }
   return SA_OK;
 }
