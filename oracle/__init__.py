@@ -46,7 +46,7 @@ import numpy as np
 __all__ = [
     "sa_forward", "sa_user", "sa_backward", "stca_branch", "stca_branch_reordered",
     "stca_fuse", "assignment", "token_lse", "layer_norm", "swiglu_ffn", "sa_refine_user",
-    "sa_refine",
+    "sa_refine", "tokenwise_user", "sa_forward_tokenwise",
 ]
 
 
@@ -302,3 +302,38 @@ def sa_refine(X, offsets: Sequence[int], P0, layers, ln_eps: float = 1e-5) -> np
     for u in range(B):
         out[u] = sa_refine_user(X[offsets[u]:offsets[u + 1]], P0, layers, ln_eps)
     return out
+
+
+# --------------------------------------------------------------------------
+# Token-wise normalisation variant (the vanilla-attention baseline)
+# --------------------------------------------------------------------------
+def tokenwise_user(Xu, P, W_Q, W_K, W_V, eps: float):
+    """The affinities of eq. (6) normalised over the user's tokens instead of the
+    prototypes (Sec. 7.1, Table 1; Sec. 2's latent-query, token-wise softmax):
+        A_{j,i} = exp S_{j,i} / sum_i' exp S_{j,i'},  H = A X,  m_j = sum_i A_{j,i}
+    and the output step of sa_user, S = diag(1/(m+eps)) H W_V.  Returns (S, m, H);
+    a user without events gets zeros."""
+    Xu = _f64(Xu)
+    k, d = np.shape(P)
+    if Xu.shape[0] == 0:
+        return np.zeros((k, d)), np.zeros(k), np.zeros((k, d))
+    Z = ((_f64(P) @ _f64(W_Q)) @ (Xu @ _f64(W_K)).T) / math.sqrt(d)   # k x n, eq. (6)
+    Zc = Z - Z.max(axis=1, keepdims=True)
+    E = np.exp(Zc)
+    A = E / E.sum(axis=1, keepdims=True)          # softmax over tokens (rows sum to 1)
+    m = A.sum(axis=1)
+    H = A @ Xu
+    denom = (m + eps)[:, None]
+    Hh = np.divide(H, denom, out=np.zeros_like(H), where=denom > 0)
+    return Hh @ _f64(W_V), m, H
+
+
+def sa_forward_tokenwise(X, offsets: Sequence[int], P, W_Q, W_K, W_V, eps: float):
+    """Token-wise variant over a ragged batch: S [B,k,d], mass [B,k], H [B,k,d]."""
+    offsets = np.asarray(offsets, np.int64)
+    B = len(offsets) - 1
+    k, d = np.shape(P)
+    S, mass, H = np.zeros((B, k, d)), np.zeros((B, k)), np.zeros((B, k, d))
+    for u in range(B):
+        S[u], mass[u], H[u] = tokenwise_user(X[offsets[u]:offsets[u + 1]], P, W_Q, W_K, W_V, eps)
+    return S, mass, H
