@@ -498,6 +498,22 @@ def run_component(args, rank, world, device):
                                       workspace=ws)
         units, unit, name = p.n_total, "history-tokens/s", p.name
         kname, flops = "sa_agg_tc_kernel", 2.0 * p.k * p.d * p.n_total
+    elif args.workload == "tokenwise":
+        p = sa_workload(5, users=args.users)
+        X = _dev_bf16(p.X, device)
+        offd = torch.from_numpy(p.offsets).to(device)
+        P, WQ, WK, WV = (_f32(a, device) for a in (p.P, p.W_Q, p.W_K, p.W_V))
+        out = {"S": torch.empty(p.B, p.k, p.d, device=device),
+               "mass": torch.empty(p.B, p.k, device=device)}
+        ws = torch.empty(sab.sa_forward_tokenwise_workspace(p.B, p.n_total, p.k, p.d, sab.SA_BF16),
+                         dtype=torch.uint8, device=device)
+        step = lambda: sab.sa_forward_tokenwise(X, p.offsets, P, WQ, WK, WV, p.eps, offsets_dev=offd,
+                                                out=out, workspace=ws)
+        units, unit = p.n_total, "history-tokens/s"
+        name = (f"token-wise normalisation variant, {p.B} users x mean "
+                f"{p.n_total // max(p.B, 1)} events, k={p.k}, d={p.d}, bf16")
+        # the attention of the k prototypes over the user's events: S = Q K^T and A V, 4kd per event
+        kname, flops = "stca_attn_tc_kernel", 4.0 * p.k * p.d * p.n_total
     elif args.workload == "refine":
         from sa_inputs import refine_layers, rng_for
         p = sa_workload(5, users=args.users)
@@ -576,10 +592,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "refine"], default="train",
+    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "refine", "tokenwise"], default="train",
                     help="train: the full step (default, the headline); sa_fwd: SA forward over "
                          "32 users x 100K (k=1024); stca: STCA of 16 users x 512 candidates; "
-                         "refine: stacked SA refinement, 2 iterations, on the train step's users")
+                         "refine: stacked SA refinement, 2 iterations, on the train step's users; "
+                         "tokenwise: the token-wise normalisation variant on the train step's users")
     ap.add_argument("--users", type=int, default=None, help="shrink the batch (profiling)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -162,6 +162,29 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype,
                       void* workspace, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Token-wise normalisation variant                                          */
+/* ------------------------------------------------------------------------ */
+
+size_t sa_forward_tokenwise_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype);
+
+/*
+ * sa_forward_tokenwise -- the "vanilla attention" baseline the paper compares
+ * SA with (Sec. 7.1, Table 1; Sec. 2's latent-query, token-wise softmax): the
+ * affinities of eq. (6), normalised over each prototype's tokens instead of
+ * over each token's prototypes:
+ *   A_{j,i} = exp S_{j,i} / sum_{i' of user u} exp S_{j,i'},  H = A X_u,
+ *   m_j = sum_i A_{j,i} (1 for a user with events, 0 without),
+ *   S = diag(1/(m+eps)) H W_V  (the same output step as sa_forward).
+ * Arguments, layouts and ownership as sa_forward (no lse output).  bf16 X and
+ * d = 128 only (else SA_ERR_UNSUPPORTED); any k >= 1.  Asynchronous on stream.
+ */
+sa_status sa_forward_tokenwise(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                               const int64_t* offsets_dev, int B, int k, int d, const float* P,
+                               const float* W_Q, const float* W_K, const float* W_V, float eps,
+                               float* S, float* mass, float* H, void* S_bf16, void* workspace,
+                               size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Stacked refinement                                                        */
 /* ------------------------------------------------------------------------ */
 

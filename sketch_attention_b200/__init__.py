@@ -28,7 +28,8 @@ _STATUS = {0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_UNSUPPORTED", 3: "SA_
 EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_workspace",
            "sa_forward", "sa_backward_workspace", "sa_backward", "stca_forward_workspace",
            "stca_forward", "stca_fuse", "sa_launch_count", "sa_profile", "sa_profile_read",
-           "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward")
+           "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward",
+           "sa_forward_tokenwise_workspace", "sa_forward_tokenwise")
 
 
 class SAError(RuntimeError):
@@ -85,6 +86,11 @@ def load(path: Optional[str] = None):
     lib.sa_forward_noalloc.restype = _i
     lib.sa_forward_noalloc.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
                                        _vp, _vp, _vp, _vp, _vp, _vp]
+    lib.sa_forward_tokenwise_workspace.restype = _sz
+    lib.sa_forward_tokenwise_workspace.argtypes = [_i, _i64, _i, _i, _i]
+    lib.sa_forward_tokenwise.restype = _i
+    lib.sa_forward_tokenwise.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
+                                         _vp, _vp, _vp, _vp, _vp, _sz, _vp]
     lib.sa_refine_workspace.restype = _sz
     lib.sa_refine_workspace.argtypes = [_i, _i64, _i, _i, _i]
     lib.sa_refine_forward.restype = _i
@@ -184,6 +190,41 @@ def sa_forward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
         res["S_bf16"] = Sb
     if lse is not None:
         res["lse"] = lse
+    return res
+
+
+def sa_forward_tokenwise(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
+                         offsets_dev: Optional[torch.Tensor] = None, want_H: bool = False,
+                         want_bf16: bool = False, out: Optional[dict] = None,
+                         workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """The token-wise normalisation variant (softmax over each prototype's tokens).
+    Returns {"S", "mass"[, "H"][, "S_bf16"]}."""
+    lib = load()
+    _need_cuda(X, P, W_Q, W_K, W_V)
+    off = _host_i64(offsets)
+    B = len(off) - 1
+    k, d = P.shape
+    dev = X.device
+    dt = _dtype_code(X)
+    o = dict(out or {})
+    S = o.get("S") if o.get("S") is not None else torch.empty(B, k, d, device=dev)
+    mass = o.get("mass") if o.get("mass") is not None else torch.empty(B, k, device=dev)
+    H = o.get("H") if o.get("H") is not None else (torch.empty(B, k, d, device=dev) if want_H else None)
+    Sb = o.get("S_bf16") if o.get("S_bf16") is not None else (
+        torch.empty(B, k, d, device=dev, dtype=torch.bfloat16) if want_bf16 else None)
+    ws_bytes = lib.sa_forward_tokenwise_workspace(B, int(off[-1]), k, d, dt)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    offd = _dev_i64(off, dev, offsets_dev)
+    st = lib.sa_forward_tokenwise(_p(X), dt, _hp(off), _p(offd), B, k, d, _p(P), _p(W_Q), _p(W_K),
+                                  _p(W_V), float(eps), _p(S), _p(mass), _p(H), _p(Sb),
+                                  _p(workspace), workspace.numel(), _stream(stream))
+    _check("sa_forward_tokenwise", st)
+    res = {"S": S, "mass": mass}
+    if H is not None:
+        res["H"] = H
+    if Sb is not None:
+        res["S_bf16"] = Sb
     return res
 
 

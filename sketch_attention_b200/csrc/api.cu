@@ -337,6 +337,45 @@ sa_status sa_forward(const void* X, sa_dtype x_dtype, const int64_t* offsets_hos
   return sa_reduce_and_project(a, w, st);
 }
 
+size_t sa_forward_tokenwise_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype) {
+  if (B < 1 || k < 1 || d < 1 || n_total < 0 || x_dtype != SA_BF16 || d != 128) return 0;
+  return tokenwise_layout(nullptr, B, k, d, nullptr);
+}
+
+sa_status sa_forward_tokenwise(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                               const int64_t* offsets_dev, int B, int k, int d, const float* P,
+                               const float* W_Q, const float* W_K, const float* W_V, float eps,
+                               float* S, float* mass, float* H, void* S_bf16, void* workspace,
+                               size_t ws_bytes, sa_stream_t stream) {
+  SA_TRY(check_sa_shape(B, k, d, x_dtype));
+  if (x_dtype != SA_BF16 || d != 128)
+    return fail(SA_ERR_UNSUPPORTED, "sa_forward_tokenwise needs bf16 X and d = 128");
+  SA_TRY(check_offsets(offsets_host, B, "offsets_host"));
+  const int64_t n = offsets_host[B];
+  if (n >= (1LL << 31) || (int64_t)B * k >= (1LL << 31))
+    return fail(SA_ERR_UNSUPPORTED, "n_total and B * k must be < 2^31");
+  if (!(eps >= 0.f)) return fail(SA_ERR_INVALID_ARG, "eps must be >= 0");
+  SA_TRY(check_ptr(X, "X", n == 0));
+  SA_TRY(check_ptr(offsets_dev, "offsets_dev"));
+  SA_TRY(check_ptr(P, "P"));
+  SA_TRY(check_ptr(W_Q, "W_Q"));
+  SA_TRY(check_ptr(W_K, "W_K"));
+  SA_TRY(check_ptr(W_V, "W_V"));
+  SA_TRY(check_ptr(S, "S"));
+  SA_TRY(check_ptr(mass, "mass"));
+  SA_TRY(check_ptr(H, "H", true));
+  SA_TRY(check_ptr(S_bf16, "S_bf16", true));
+  if (H == S) return fail(SA_ERR_INVALID_ARG, "H must not alias S");
+  const size_t need = tokenwise_layout(nullptr, B, k, d, nullptr);
+  if (!workspace || ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "workspace needs " + std::to_string(need) + " bytes");
+  SA_TRY(check_ptr(workspace, "workspace"));
+  TokenwiseWork w;
+  tokenwise_layout(workspace, B, k, d, &w);
+  SaFwdArgs a{X, x_dtype, offsets_dev, B, n, k, d, P, W_Q, W_K, W_V, eps, S, mass, H, S_bf16, nullptr};
+  return sa_tokenwise_run(a, w, (cudaStream_t)stream);
+}
+
 size_t sa_refine_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype) {
   if (B < 1 || k < 1 || d < 1 || n_total < 0 || !sa_tc_supported(x_dtype, k, d)) return 0;
   return refine_layout(nullptr, B, n_total, k, d, nullptr, nullptr);

@@ -83,6 +83,20 @@ sa_status sa_refine_run(const void* X, sa_dtype x_dtype, const int64_t* off_dev,
                         float ln_eps, float* sketch, const SaFwdWork& w, const RefineWork& r,
                         cudaStream_t st);
 
+// Token-wise normalisation variant (sa_tokenwise.cu).
+struct TokenwiseWork {
+  float* T;              // [d, d]
+  float* Pf;             // [k, d]
+  __nv_bfloat16* Pb;     // [k, d]
+  __nv_bfloat16* Ub;     // [B, k, d] P' for every user (the attention's queries)
+  float* Y;              // [B, k, d] A X
+  float* Hhat;           // [B, k, d]
+  int64_t* cand;         // [B+1] u k
+  int* prefix;           // [B+1] query tiles before user u
+};
+size_t tokenwise_layout(void* base, int B, int k, int d, TokenwiseWork* w);
+sa_status sa_tokenwise_run(const SaFwdArgs& a, const TokenwiseWork& w, cudaStream_t st);
+
 // Sums the split-n partials into H (if a.H), the mass and H/(m+eps) (w.Hhat).
 sa_status sa_reduce(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
 sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
