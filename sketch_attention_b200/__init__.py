@@ -193,6 +193,10 @@ def sa_forward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
     return res
 
 
+def sa_forward_tokenwise_workspace(B: int, n_total: int, k: int, d: int, x_dtype: int) -> int:
+    return int(load().sa_forward_tokenwise_workspace(B, n_total, k, d, x_dtype))
+
+
 def sa_forward_tokenwise(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float = 1e-6, *,
                          offsets_dev: Optional[torch.Tensor] = None, want_H: bool = False,
                          want_bf16: bool = False, out: Optional[dict] = None,
