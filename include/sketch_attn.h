@@ -161,6 +161,23 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype,
                       const float* lse, void* dX, float* dP, float* dW_Q, float* dW_K, float* dW_V,
                       void* workspace, size_t ws_bytes, sa_stream_t stream);
 
+/*
+ * sa_backward_accumulate -- sa_backward that adds the weight gradients into
+ * dP, dW_Q, dW_K and dW_V instead of overwriting them (dX is written as in
+ * sa_backward).  The weights are shared by all users, so their gradients over
+ * a batch are the sum over any split of its users into groups: call it once
+ * per group (e.g. to overlap the next group's host-to-device copy with this
+ * group's work) after zeroing or a first sa_backward.  Same arguments, layouts
+ * and errors as sa_backward; no counterpart in the paper (an interface form).
+ */
+sa_status sa_backward_accumulate(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                                 const int64_t* offsets_dev, int B, int k, int d, const float* P,
+                                 const float* W_Q, const float* W_K, const float* W_V, float eps,
+                                 const float* H, const float* mass, const float* dS,
+                                 const float* dmass, const float* lse, void* dX, float* dP,
+                                 float* dW_Q, float* dW_K, float* dW_V, void* workspace,
+                                 size_t ws_bytes, sa_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Token-wise normalisation variant                                          */
 /* ------------------------------------------------------------------------ */

@@ -29,7 +29,7 @@ EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_w
            "sa_forward", "sa_backward_workspace", "sa_backward", "stca_forward_workspace",
            "stca_forward", "stca_fuse", "sa_launch_count", "sa_profile", "sa_profile_read",
            "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward",
-           "sa_forward_tokenwise_workspace", "sa_forward_tokenwise")
+           "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate")
 
 
 class SAError(RuntimeError):
@@ -76,6 +76,8 @@ def load(path: Optional[str] = None):
     lib.sa_backward.restype = _i
     lib.sa_backward.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _f,
                                 _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]
+    lib.sa_backward_accumulate.restype = _i
+    lib.sa_backward_accumulate.argtypes = lib.sa_backward.argtypes
     lib.stca_forward_workspace.restype = _sz
     lib.stca_forward_workspace.argtypes = [_i, _i64, _i, _i, _i, _i]
     lib.stca_forward.restype = _i
@@ -260,8 +262,10 @@ def sa_backward_workspace(B: int, n_total: int, k: int, d: int, dtype: int) -> i
 def sa_backward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float, H, mass, dS,
                 dmass=None, lse=None, *, offsets_dev: Optional[torch.Tensor] = None,
                 out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
-                stream=None) -> dict:
-    """Gradients {"dX", "dP", "dW_Q", "dW_K", "dW_V"} of <dS, S> + <dmass, mass>."""
+                stream=None, accumulate: bool = False) -> dict:
+    """Gradients {"dX", "dP", "dW_Q", "dW_K", "dW_V"} of <dS, S> + <dmass, mass>.
+    With ``accumulate`` the weight gradients are added into out's dP, dW_Q, dW_K,
+    dW_V (sa_backward_accumulate), e.g. one call per group of users."""
     lib = load()
     _need_cuda(X, P, W_Q, W_K, W_V, H, mass, dS, dmass, lse)
     off = _host_i64(offsets)
@@ -279,10 +283,13 @@ def sa_backward(X: torch.Tensor, offsets, P, W_Q, W_K, W_V, eps: float, H, mass,
     if workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     offd = _dev_i64(off, dev, offsets_dev)
-    st = lib.sa_backward(_p(X), dt, _hp(off), _p(offd), B, k, d, _p(P), _p(W_Q), _p(W_K), _p(W_V),
-                         float(eps), _p(H), _p(mass), _p(dS), _p(dmass), _p(lse), _p(dX), _p(dP), _p(dWQ),
-                         _p(dWK), _p(dWV), _p(workspace), workspace.numel(), _stream(stream))
-    _check("sa_backward", st)
+    if accumulate and any(o.get(n) is None for n in ("dP", "dW_Q", "dW_K", "dW_V")):
+        raise ValueError("accumulate needs out with dP, dW_Q, dW_K and dW_V")
+    fn = lib.sa_backward_accumulate if accumulate else lib.sa_backward
+    st = fn(_p(X), dt, _hp(off), _p(offd), B, k, d, _p(P), _p(W_Q), _p(W_K), _p(W_V),
+            float(eps), _p(H), _p(mass), _p(dS), _p(dmass), _p(lse), _p(dX), _p(dP), _p(dWQ),
+            _p(dWK), _p(dWV), _p(workspace), workspace.numel(), _stream(stream))
+    _check("sa_backward_accumulate" if accumulate else "sa_backward", st)
     return {"dX": dX, "dP": dP, "dW_Q": dWQ, "dW_K": dWK, "dW_V": dWV}
 
 

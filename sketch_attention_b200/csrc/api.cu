@@ -428,12 +428,16 @@ size_t sa_backward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dt
   return layout_bwd(nullptr, B, n_total, k, d, x_dtype, nullptr);
 }
 
-sa_status sa_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
-                      const int64_t* offsets_dev, int B, int k, int d, const float* P,
-                      const float* W_Q, const float* W_K, const float* W_V, float eps,
-                      const float* H, const float* mass, const float* dS, const float* dmass,
-                      const float* lse, void* dX, float* dP, float* dW_Q, float* dW_K,
-                      float* dW_V, void* workspace, size_t ws_bytes, sa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+sa_status backward_impl(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                        const int64_t* offsets_dev, int B, int k, int d, const float* P,
+                        const float* W_Q, const float* W_K, const float* W_V, float eps,
+                        const float* H, const float* mass, const float* dS, const float* dmass,
+                        const float* lse, void* dX, float* dP, float* dW_Q, float* dW_K,
+                        float* dW_V, void* workspace, size_t ws_bytes, sa_stream_t stream,
+                        bool accumulate) {
   SA_TRY(check_sa_shape(B, k, d, x_dtype));
   SA_TRY(check_offsets(offsets_host, B, "offsets_host"));
   const int64_t n = offsets_host[B];
@@ -462,9 +466,34 @@ sa_status sa_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_ho
   layout_bwd(workspace, B, n, k, d, x_dtype, &w);
   SaBwdArgs a{X, x_dtype, offsets_dev, B, n, k, d, P, W_Q, W_K, W_V, eps,
               H, mass, dS, dmass, lse, dX, dP, dW_Q, dW_K, dW_V};
+  a.accumulate = accumulate;
   cudaStream_t st = (cudaStream_t)stream;
   SA_TRY(sa_fold(k, d, P, W_Q, W_K, w.T, w.Pf, w.Pb, st));
   return sa_backward_run(a, w, sa_bwd_tc_supported(x_dtype, k, d), st);
+}
+}  // namespace
+
+extern "C" {
+
+sa_status sa_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                      const int64_t* offsets_dev, int B, int k, int d, const float* P,
+                      const float* W_Q, const float* W_K, const float* W_V, float eps,
+                      const float* H, const float* mass, const float* dS, const float* dmass,
+                      const float* lse, void* dX, float* dP, float* dW_Q, float* dW_K,
+                      float* dW_V, void* workspace, size_t ws_bytes, sa_stream_t stream) {
+  return backward_impl(X, x_dtype, offsets_host, offsets_dev, B, k, d, P, W_Q, W_K, W_V, eps, H, mass,
+                       dS, dmass, lse, dX, dP, dW_Q, dW_K, dW_V, workspace, ws_bytes, stream, false);
+}
+
+sa_status sa_backward_accumulate(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                                 const int64_t* offsets_dev, int B, int k, int d, const float* P,
+                                 const float* W_Q, const float* W_K, const float* W_V, float eps,
+                                 const float* H, const float* mass, const float* dS,
+                                 const float* dmass, const float* lse, void* dX, float* dP,
+                                 float* dW_Q, float* dW_K, float* dW_V, void* workspace,
+                                 size_t ws_bytes, sa_stream_t stream) {
+  return backward_impl(X, x_dtype, offsets_host, offsets_dev, B, k, d, P, W_Q, W_K, W_V, eps, H, mass,
+                       dS, dmass, lse, dX, dP, dW_Q, dW_K, dW_V, workspace, ws_bytes, stream, true);
 }
 
 size_t stca_forward_workspace(int B, int64_t C_total, int D, int heads, int d_h, sa_dtype dtype) {

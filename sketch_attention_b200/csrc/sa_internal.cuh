@@ -36,6 +36,7 @@ struct SaBwdArgs {
   float eps;
   const float *H, *mass, *dS, *dmass, *lse_in;
   void* dX; float *dP, *dW_Q, *dW_K, *dW_V;
+  bool accumulate = false;   // add the weight gradients into dP, dW_Q, dW_K, dW_V
 };
 
 struct SaBwdWork {

@@ -552,7 +552,8 @@ sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaS
   gv.M = D; gv.N = D; gv.K = rows;
   gv.A = w.Hhat; gv.lda = D; gv.transA = true;
   gv.B = a.dS; gv.ldb = D;
-  gv.C = a.dW_V; gv.ldc = D; gv.tag = "gemm:dW_V";
+  gv.C = a.dW_V; gv.ldc = D;
+  if (a.accumulate) { gv.Cin = a.dW_V; gv.ldcin = D; } gv.tag = "gemm:dW_V";
   gv.split_k = gemm_split_for(D, D, rows, kMaxSplit);
   gv.split_ws = w.gsplit;
   if ((s = gemm(gv, st)) != SA_OK) return s;
@@ -591,12 +592,14 @@ sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream
   // dP = dQ W_Q^T
   Gemm g2;
   g2.M = k; g2.N = D; g2.K = D;
-  g2.A = w.dQ; g2.lda = D; g2.B = a.W_Q; g2.ldb = D; g2.transB = true; g2.C = a.dP; g2.ldc = D; g2.tag = "gemm:E_grads";
+  g2.A = w.dQ; g2.lda = D; g2.B = a.W_Q; g2.ldb = D; g2.transB = true; g2.C = a.dP; g2.ldc = D;
+  if (a.accumulate) { g2.Cin = a.dP; g2.ldcin = D; } g2.tag = "gemm:E_grads";
   if ((s = gemm(g2, st)) != SA_OK) return s;
   // dW_Q = P^T dQ
   Gemm g3;
   g3.M = D; g3.N = D; g3.K = k;
-  g3.A = a.P; g3.lda = D; g3.transA = true; g3.B = w.dQ; g3.ldb = D; g3.C = a.dW_Q; g3.ldc = D; g3.tag = "gemm:E_grads";
+  g3.A = a.P; g3.lda = D; g3.transA = true; g3.B = w.dQ; g3.ldb = D; g3.C = a.dW_Q; g3.ldc = D;
+  if (a.accumulate) { g3.Cin = a.dW_Q; g3.ldcin = D; } g3.tag = "gemm:E_grads";
   g3.split_k = gemm_split_for(D, D, k, kMaxSplit);
   g3.split_ws = w.gsplit;
   if ((s = gemm(g3, st)) != SA_OK) return s;
@@ -607,7 +610,8 @@ sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream
   if ((s = gemm(g4, st)) != SA_OK) return s;
   Gemm g5;
   g5.M = D; g5.N = D; g5.K = k;
-  g5.A = w.E; g5.lda = D; g5.transA = true; g5.B = w.Q; g5.ldb = D; g5.C = a.dW_K; g5.ldc = D; g5.tag = "gemm:E_grads";
+  g5.A = w.E; g5.lda = D; g5.transA = true; g5.B = w.Q; g5.ldb = D; g5.C = a.dW_K; g5.ldc = D;
+  if (a.accumulate) { g5.Cin = a.dW_K; g5.ldcin = D; } g5.tag = "gemm:E_grads";
   g5.alpha = rs;
   g5.split_k = gemm_split_for(D, D, k, kMaxSplit);
   g5.split_ws = w.gsplit;

@@ -190,3 +190,35 @@ def test_sa_backward_workload5_sampled(lib, workload_cache):
     for n in names:
         # the same sums in another order: fp32 reassociation of sums with cancellation
         compare(f"{n} full = sum of users", g[n], total[n].cpu().numpy(), dict(max_rel=1e-3, mean_rel=1e-3))
+
+
+@pytest.mark.parametrize("dtype,k", [("f32", 100), ("bf16", 256)])
+def test_sa_backward_accumulate_over_user_groups(lib, dtype, k):
+    """Weight gradients are sums over users: a first group through sa_backward and
+    a second through sa_backward_accumulate equal one call over the whole batch,
+    and each group's dX rows equal the whole batch's."""
+    p = make_sa_problem((700, 0, 129, 1500, 60), k, 128, dtype, seed=77, with_grad=True)
+    dv = sa_device_inputs(p)
+    fwd = lib.sa_forward(dv["X"], p.offsets, dv["P"], dv["W_Q"], dv["W_K"], dv["W_V"], p.eps,
+                         want_H=True, want_lse=True)
+    dS = dev_f32(p.dS)
+    full = lib.sa_backward(dv["X"], p.offsets, dv["P"], dv["W_Q"], dv["W_K"], dv["W_V"], p.eps,
+                           fwd["H"], fwd["mass"], dS, None, fwd["lse"])
+    names = ["dP", "dW_Q", "dW_K", "dW_V"]
+    acc = {n: torch.empty_like(full[n]) for n in names}
+    off = p.offsets
+    for i, (u0, u1) in enumerate(((0, 2), (2, p.B))):
+        lo, hi = int(off[u0]), int(off[u1])
+        g = lib.sa_backward(dv["X"][lo:hi], off[u0:u1 + 1] - off[u0], dv["P"], dv["W_Q"], dv["W_K"],
+                            dv["W_V"], p.eps, fwd["H"][u0:u1], fwd["mass"][u0:u1], dS[u0:u1], None,
+                            fwd["lse"][lo:hi].clone(), out=dict(acc), accumulate=(i > 0))
+        torch.cuda.synchronize()
+        np.testing.assert_allclose(g["dX"].float().cpu().numpy(), full["dX"][lo:hi].float().cpu().numpy(),
+                                   rtol=1e-2, atol=1e-2 * float(full["dX"].float().abs().max()))
+    for n in names:
+        np.testing.assert_allclose(acc[n].cpu().numpy(), full[n].cpu().numpy(), rtol=1e-3,
+                                   atol=1e-4 * float(full[n].abs().max()))
+    ref = oracle.sa_backward(p.x_f64(), p.offsets, p.P, p.W_Q, p.W_K, p.W_V, p.eps, p.dS)
+    for name, r in zip(["dX", "dP", "dW_Q", "dW_K", "dW_V"], ref):
+        if name != "dX":
+            compare(name, acc[name], r, tol_for(dtype))
