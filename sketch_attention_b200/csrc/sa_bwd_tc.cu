@@ -355,11 +355,18 @@ __global__ void __launch_bounds__(384, 1)
 }
 
 // ============================================================== E kernel
-constexpr int E_NXS = 3;   // X tiles in flight: each is held from its load until the E MMA of its tile
+// X tiles in flight (each is held from its load until the E MMA of its tile) and dZ buffers
+#ifndef SA_E_NXS
+#define SA_E_NXS 3
+#endif
+#ifndef SA_E_NDZ
+#define SA_E_NDZ 2
+#endif
+constexpr int E_NXS = SA_E_NXS, E_NDZ = SA_E_NDZ;
 constexpr uint32_t E_OFF_PH = 0;              // [P' h0 | dH h0 | P' h1 | dH h1], 16 KB each
 constexpr uint32_t E_OFF_X = 65536;
-constexpr uint32_t E_OFF_DZ = E_OFF_X + E_NXS * XT_BYTES;   // 2 x [128 protos x 128 tokens] MN-major
-constexpr uint32_t E_OFF_DM = E_OFF_DZ + 2 * 32768;
+constexpr uint32_t E_OFF_DZ = E_OFF_X + E_NXS * XT_BYTES;   // E_NDZ x [128 protos x 128 tokens] MN-major
+constexpr uint32_t E_OFF_DM = E_OFF_DZ + E_NDZ * 32768;
 constexpr uint32_t E_OFF_BAR = E_OFF_DM + TILE * 4;
 constexpr uint32_t E_SMEM = E_OFF_BAR + 256 + 1024;
 // warp 0 TMA, 1 MMA, 2-5 and 6-9: two warpgroups, group h computing dZ for the
@@ -370,7 +377,7 @@ constexpr uint32_t E_TM_ZG = 0, E_TM_E = 256;
 
 struct EBars {
   uint64_t p_full, h_full, h_empty, x_full[E_NXS], x_empty[E_NXS];
-  uint64_t zg_full, zg_empty, dz_full[2], dz_empty[2], e_full, mma_done;
+  uint64_t zg_full, zg_empty, dz_full[E_NDZ], dz_empty[E_NDZ], e_full, mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -406,7 +413,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     for (int s = 0; s < E_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
     mbar_init(&bars->zg_full, 1);
     mbar_init(&bars->zg_empty, 256);
-    for (int b = 0; b < 2; ++b) { mbar_init(&bars->dz_full[b], 256); mbar_init(&bars->dz_empty[b], 1); }
+    for (int b = 0; b < E_NDZ; ++b) { mbar_init(&bars->dz_full[b], 256); mbar_init(&bars->dz_empty[b], 1); }
     mbar_init(&bars->e_full, 1);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -460,8 +467,8 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     const uint32_t ph = smem_u32(smem + E_OFF_PH);
     int prev_t = -1, prev_s = 0;
     auto emma = [&](int t, int s) -> bool {
-      const int b = t & 1;
-      if (!mbar_wait(&bars->dz_full[b], (t >> 1) & 1, abort, p.err)) return false;
+      const int b = t % E_NDZ;
+      if (!mbar_wait(&bars->dz_full[b], (t / E_NDZ) & 1, abort, p.err)) return false;
       tc_fence_after();
       const uint32_t dz = smem_u32(smem + E_OFF_DZ + b * 32768);
       const uint32_t xa = smem_u32(smem + E_OFF_X + s * XT_BYTES);
@@ -520,7 +527,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
       if (first && !mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return ok = false;
       if (!mbar_wait(&bars->zg_full, t & 1, abort, p.err)) return ok = false;
       tc_fence_after();
-      const int b = t & 1;
+      const int b = t % E_NDZ;
       const uint32_t dz = smem_u32(smem + E_OFF_DZ + b * 32768) + row * 128;
       const float4* dm4 = (const float4*)(smem + E_OFF_DM);
       {
@@ -532,7 +539,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->zg_empty);
-        if (t >= 2 && !mbar_wait(&bars->dz_empty[b], ((t >> 1) - 1) & 1, abort, p.err)) return ok = false;
+        if (t >= E_NDZ && !mbar_wait(&bars->dz_empty[b], ((t / E_NDZ) - 1) & 1, abort, p.err)) return ok = false;
         // two prototypes per instruction (packed fp32x2 add / mul)
 #pragma unroll
         for (int c8 = 0; c8 < 8; ++c8) {
