@@ -19,6 +19,7 @@ CASES = [
     ((385,), 128, 1, False, 2),
     ((2000, 129), 1024, 2, True, 3),
     ((1, 260, 3000), 512, 3, True, 4),
+    ((0, 0), 128, 2, True, 5),            # no events at all: X^ = 0 in every iteration
 ]
 
 
