@@ -18,7 +18,14 @@ Readings where the pages leave a step open (each is an explicit choice):
 * Softmax stabiliser: the per-token maximum over prototypes is subtracted
   ("numerically robust softmax", Sec. 4.4 FlashSA); the result is unchanged.
 * STCA layer body: attention, optional output projection W_O, residual add
-  to the query (eq. 4 plus the W_O term of eq. 26); no FFN, no LayerNorm.
+  to the query (eq. 4 plus the W_O term of eq. 26), no LayerNorm.  The full
+  layer of eqs. (26)-(28) adds two optional SwiGLU FFNs of inner width 2D
+  (no biases, SiLU on the first branch), each with a residual add:
+  - on the history, before the layer's attention: X <- X + FFN_h(X), a
+    per-row, target-independent transform (eq. (27)); the transformed rows
+    are the keys and values of this layer and the input of the next layer's
+    history FFN;
+  - on the query, after the W_O residual: q <- q + FFN_q(q) (eq. (26)).
 * STCA over an empty key range: the attention output is zero.
 * Fusion: a linear map [z_r; z_u] W_F + b_F (Sec. 3.4 leaves the fusion open).
 * Stacked refinement (Sec. 3.3): X^ = A X exactly as eq. (14) writes it (the
@@ -33,7 +40,9 @@ permutation invariance, k = 1 mean, uniform assignment at zero logits,
 identical tokens, a two-prototype closed form that fixes the 1/sqrt(d) scale
 and the operand order, central finite differences for every gradient, STCA at
 L = 1, identical keys, torch SDPA in fp64, the eq. (24) reordering, and the
-analytic FLOP numbers the pages print.  No function here is "parity
+analytic FLOP numbers the pages print; for the full STCA layer, torch's SiLU
+and SDPA in fp64, key-permutation invariance, the layer chaining of the
+history FFN and the reordering with both FFNs.  No function here is "parity
 unpinned".
 """
 from __future__ import annotations
@@ -176,6 +185,20 @@ def _softmax_rows(s: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=1, keepdims=True)
 
 
+def _history_ffn(Xu, lay) -> np.ndarray:
+    """X + FFN_h(X) when the layer has a history FFN (eq. (27)), else X."""
+    if getattr(lay, "hist_W1", None) is None:
+        return Xu
+    return Xu + swiglu_ffn(Xu, lay.hist_W1, lay.hist_W3, lay.hist_W2)
+
+
+def _query_ffn(qu, lay) -> np.ndarray:
+    """q + FFN_q(q) when the layer has a query FFN (eq. (26)), else q."""
+    if getattr(lay, "q_W1", None) is None:
+        return qu
+    return qu + swiglu_ffn(qu, lay.q_W1, lay.q_W3, lay.q_W2)
+
+
 def stca_branch(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: int, d_h: int):
     """Stacked target-to-history single-query cross attention, direct form.
 
@@ -186,7 +209,10 @@ def stca_branch(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: int, d_h: 
     Candidates of user u are rows [cand_offsets[u], cand_offsets[u+1]) of q;
     their keys/values are rows [kv_begin[u], kv_end[u]) of kv.
     ``layers`` is a list of objects with W_Q, W_K, W_V ([heads, D, d_h]) and
-    W_O ([heads*d_h, D] or None).
+    W_O ([heads*d_h, D] or None), and optionally the full layer's FFNs
+    (eqs. (26)-(27)): hist_W1, hist_W3 [D, 2D], hist_W2 [2D, D] applied to
+    the history before the attention, q_W1, q_W3, q_W2 applied to the query
+    after the W_O residual (None = absent).
     """
     out = _f64(q).copy()
     kv = _f64(kv)
@@ -198,6 +224,7 @@ def stca_branch(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: int, d_h: 
         Xu = kv[int(kv_begin[u]):int(kv_end[u])]
         qu = out[c0:c1]
         for lay in layers:
+            Xu = _history_ffn(Xu, lay)
             o = np.zeros((c1 - c0, heads * d_h))
             if Xu.shape[0] > 0:
                 for h in range(heads):
@@ -206,6 +233,7 @@ def stca_branch(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: int, d_h: 
                     alpha = _softmax_rows(scores)
                     o[:, h * d_h:(h + 1) * d_h] = alpha @ (Xu @ Wv)
             qu = qu + (o if lay.W_O is None else o @ _f64(lay.W_O))
+            qu = _query_ffn(qu, lay)
         out[c0:c1] = qu
     return out
 
@@ -225,6 +253,7 @@ def stca_branch_reordered(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: 
         Xu = kv[int(kv_begin[u]):int(kv_end[u])]
         qu = out[c0:c1]
         for lay in layers:
+            Xu = _history_ffn(Xu, lay)
             o = np.zeros((c1 - c0, heads * d_h))
             if Xu.shape[0] > 0:
                 for h in range(heads):
@@ -233,6 +262,7 @@ def stca_branch_reordered(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: 
                     alpha = _softmax_rows(uvec @ Xu.T / math.sqrt(d_h))
                     o[:, h * d_h:(h + 1) * d_h] = (alpha @ Xu) @ Wv
             qu = qu + (o if lay.W_O is None else o @ _f64(lay.W_O))
+            qu = _query_ffn(qu, lay)
         out[c0:c1] = qu
     return out
 

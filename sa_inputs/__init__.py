@@ -281,6 +281,13 @@ class STCALayer:
     W_K: np.ndarray      # f32 [heads, D, d_h]
     W_V: np.ndarray      # f32 [heads, D, d_h]
     W_O: Optional[np.ndarray]   # f32 [heads*d_h, D] or None (identity)
+    # the full layer's SwiGLU FFNs (None = absent): history side, then query side
+    hist_W1: Optional[np.ndarray] = None   # f32 [D, 2D]
+    hist_W3: Optional[np.ndarray] = None   # f32 [D, 2D]
+    hist_W2: Optional[np.ndarray] = None   # f32 [2D, D]
+    q_W1: Optional[np.ndarray] = None      # f32 [D, 2D]
+    q_W3: Optional[np.ndarray] = None      # f32 [D, 2D]
+    q_W2: Optional[np.ndarray] = None      # f32 [2D, D]
 
 
 @dataclasses.dataclass
@@ -324,6 +331,22 @@ def stca_layers(rng, n_layers: int, D: int, heads: int, d_h: int, with_wo: bool 
         W_O = gauss(rng, (heads * d_h, D), std) if with_wo else None
         out.append(STCALayer(W_Q, W_K, W_V, W_O))
     return out
+
+
+def add_stca_ffns(rng, layers, D: int, hist: bool = True, query: bool = True):
+    """Give each STCA layer the full layer's SwiGLU FFNs: W1, W3 [D, 2D] with
+    std 1/sqrt(D) and W2 [2D, D] with std 1/sqrt(2D), history side and/or
+    query side.  Returns the same list."""
+    for lay in layers:
+        if hist:
+            lay.hist_W1 = gauss(rng, (D, 2 * D), 1.0 / math.sqrt(D))
+            lay.hist_W3 = gauss(rng, (D, 2 * D), 1.0 / math.sqrt(D))
+            lay.hist_W2 = gauss(rng, (2 * D, D), 1.0 / math.sqrt(2 * D))
+        if query:
+            lay.q_W1 = gauss(rng, (D, 2 * D), 1.0 / math.sqrt(D))
+            lay.q_W3 = gauss(rng, (D, 2 * D), 1.0 / math.sqrt(D))
+            lay.q_W2 = gauss(rng, (2 * D, D), 1.0 / math.sqrt(2 * D))
+    return layers
 
 
 def refine_layers(rng, n_iter: int, d: int, affine: bool = True):
