@@ -551,6 +551,7 @@ def run_component(args, rank, world, device):
     sab.load()
     from sa_inputs import STCA_WORKLOAD_4, sa_workload, stca_workload
     peaks, peaks_src = load_peaks()
+    extra = []          # (kernel, flops per launch) of other tensor-core kernels to report
     if args.workload == "sa_fwd":
         p = sa_workload(3, users=args.users)
         X = _dev_bf16(p.X, device)
@@ -599,6 +600,46 @@ def run_component(args, rank, world, device):
                 f"{p.B} users x mean {p.n_total // max(p.B, 1)} events, k={p.k}, d={p.d}, bf16")
         # per launch of the dominant kernel: H = A X with its mass (2kd flop per token)
         kname, flops = "sa_agg_tc_kernel", 2.0 * p.k * p.d * p.n_total
+    elif args.workload == "stca_full":
+        from sa_inputs import add_stca_ffns, rng_for
+        w = stca_workload(users=args.users or 16)
+        add_stca_ffns(rng_for(5006), w.layers_r, 128)
+        add_stca_ffns(rng_for(5007), w.layers_u, 128)
+        q, kvr, kvs = (_dev_bf16(a, device) for a in (w.recent.q, w.recent.kv, w.sketch.kv))
+        ffn_keys = ("hist_W1", "hist_W3", "hist_W2", "q_W1", "q_W3", "q_W2")
+        lay = lambda L: dict(W_Q=_f32(L.W_Q, device), W_K=_f32(L.W_K, device), W_V=_f32(L.W_V, device),
+                             W_O=_f32(L.W_O, device), **{k: _f32(getattr(L, k), device) for k in ffn_keys})
+        lr, lu = [lay(L) for L in w.layers_r], [lay(L) for L in w.layers_u]
+        WF, bF = _f32(w.W_F, device), _f32(w.b_F, device)
+        C = int(w.recent.cand_offsets[-1])
+        zr, zu, z = (torch.empty(C, 128, device=device) for _ in range(3))
+        rows_r = int((w.recent.kv_end - w.recent.kv_begin).sum())
+        rows_s = int((w.sketch.kv_end - w.sketch.kv_begin).sum())
+        B = len(w.recent.cand_offsets) - 1
+        ws_r = torch.empty(sab.stca_forward_full_workspace(B, C, rows_r, 128, w.heads, w.d_h, sab.SA_BF16),
+                           dtype=torch.uint8, device=device)
+        ws_s = torch.empty(sab.stca_forward_full_workspace(B, C, rows_s, 128, w.heads, w.d_h, sab.SA_BF16),
+                           dtype=torch.uint8, device=device)
+        dv = lambda a: torch.from_numpy(np.asarray(a, np.int64)).to(device)
+        cd, rbd, red, sbd, sed = (dv(a) for a in (w.recent.cand_offsets, w.recent.kv_begin, w.recent.kv_end,
+                                                  w.sketch.kv_begin, w.sketch.kv_end))
+
+        def step():
+            sab.stca_forward_full(q, w.recent.cand_offsets, kvr, w.recent.kv_begin, w.recent.kv_end,
+                                  lr, w.heads, w.d_h, cand_offsets_dev=cd, kv_begin_dev=rbd,
+                                  kv_end_dev=red, out=zr, workspace=ws_r)
+            sab.stca_forward_full(q, w.sketch.cand_offsets, kvs, w.sketch.kv_begin, w.sketch.kv_end,
+                                  lu, w.heads, w.d_h, cand_offsets_dev=cd, kv_begin_dev=sbd,
+                                  kv_end_dev=sed, out=zu, workspace=ws_s)
+            sab.stca_fuse(zr, zu, WF, bF, out=z)
+        units, unit = C, "candidates/s"
+        name = ("full STCA layers (history-side SwiGLU FFN before and query-side after each attention), "
+                + STCA_WORKLOAD_4)
+        L_avg = 0.5 * (float(np.mean(w.recent.kv_end - w.recent.kv_begin)) + 1024)
+        kname, flops = "stca_attn_tc_kernel", 4.0 * L_avg * 128 * C * w.heads
+        # the history FFN: 12 D^2 flop per key row (eq. (27) with inner width 2D), once per row;
+        # per launch the mean of the two branches' row counts
+        extra.append(("stca_hist_ffn_tc_kernel", 12.0 * 128 * 128 * 0.5 * (rows_r + rows_s)))
     else:
         w = stca_workload(users=args.users or 16)
         q, kvr, kvs = (_dev_bf16(a, device) for a in (w.recent.q, w.recent.kv, w.sketch.kv))
@@ -632,16 +673,19 @@ def run_component(args, rank, world, device):
     prof = sab.profile_read()
     sab.profile(False)
     ms = start.elapsed_time(end) / args.steps
-    roof = None
-    if kname in prof:
-        tot, cnt = prof[kname]
-        ach = flops / (tot / cnt / 1e3) / 1e12
+    def roof_of(kn, fl):
+        if kn not in prof:
+            return None
+        tot, cnt = prof[kn]
+        ach = fl / (tot / cnt / 1e3) / 1e12
         pk = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
-        roof = {"kernel": kname, "bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
+        return {"kernel": kn, "bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
                 "frac": ach / pk, "traffic": None,
                 "peak_source": f"bf16 dense, burst ({peaks_src}): the kernel is timed alone",
                 "avg_launch_ms": tot / cnt}
-    return {"metric": unit, "value": world * units / (ms / 1e3), "unit": unit, "n_gpus": world,
+    roof = roof_of(kname, flops)
+    extra_roofs = {kn: roof_of(kn, fl) for kn, fl in extra}
+    line = {"metric": unit, "value": world * units / (ms / 1e3), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": {"workload": name},
@@ -649,6 +693,9 @@ def run_component(args, rank, world, device):
             "kernels": {n: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
                         for n, v in sorted(prof.items(), key=lambda kv: -kv[1][0])},
             "clocks": clk.summary()}
+    if extra_roofs:
+        line["other_rooflines"] = extra_roofs
+    return line
 
 
 def main():
@@ -659,9 +706,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "refine", "tokenwise"], default="train",
+    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "stca_full", "refine", "tokenwise"],
+                    default="train",
                     help="train: the full step (default, the headline); sa_fwd: SA forward over "
                          "32 users x 100K (k=1024); stca: STCA of 16 users x 512 candidates; "
+                         "stca_full: the same with full layers (history- and query-side FFNs); "
                          "refine: stacked SA refinement, 2 iterations, on the train step's users; "
                          "tokenwise: the token-wise normalisation variant on the train step's users")
     ap.add_argument("--users", type=int, default=None, help="shrink the batch (profiling)")

@@ -281,6 +281,54 @@ sa_status stca_forward(const void* q, sa_dtype dtype,
                        float* out, void* workspace, size_t ws_bytes, sa_stream_t stream);
 
 /*
+ * The full STCA layer (paper Sec. 5.1, eqs. (26)-(28)): the attention layer
+ * above plus two SwiGLU FFNs of inner width 2D (no biases, SiLU(x) =
+ * x / (1 + e^-x) on the first branch), each with a residual add:
+ *   history side (eq. (27)), before the layer's attention, on every key row:
+ *       x <- x + (SiLU(x hist_W1) * (x hist_W3)) hist_W2
+ *     the transformed rows are this layer's keys and values and the input of
+ *     the next layer's history FFN (the transform is target-independent, so
+ *     it runs once per key row, not once per candidate);
+ *   query side (eq. (26)), after the W_O residual:
+ *       q <- q + (SiLU(q q_W1) * (q q_W3)) q_W2
+ * hist_W1, hist_W3, q_W1, q_W3 [D, 2D]; hist_W2, q_W2 [2D, D]; fp32 device
+ * pointers.  Each FFN is either fully given or fully NULL (absent).
+ */
+typedef struct {
+  stca_layer attn;
+  const float* hist_W1;
+  const float* hist_W3;
+  const float* hist_W2;
+  const float* q_W1;
+  const float* q_W3;
+  const float* q_W2;
+} stca_full_layer;
+
+/* kv_total = sum over users of kv_end[u] - kv_begin[u] (the key rows the
+ * history FFNs transform; a range shared by two users counts twice). */
+size_t stca_forward_full_workspace(int B, int64_t C_total, int64_t kv_total, int D, int heads,
+                                   int d_h, sa_dtype dtype);
+
+/*
+ * stca_forward_full -- one STCA branch of full layers.  Arguments as in
+ * stca_forward; layers is a host array of n_layers stca_full_layer.  The
+ * key rows are copied into the workspace (each user's range, in user order)
+ * before the first history FFN, so kv is only read.  With dtype SA_BF16 the
+ * transformed rows are kept in bf16 (they are the attention's keys) and the
+ * history FFN runs on the tensor cores with bf16 weights and fp32
+ * accumulation; with SA_F32 everything is fp32.  The query FFN is fp32.
+ * Errors: as stca_forward, and SA_ERR_INVALID_ARG for a partly given FFN.
+ */
+sa_status stca_forward_full(const void* q, sa_dtype dtype,
+                            const int64_t* cand_offsets_host, const int64_t* cand_offsets_dev,
+                            int B, const void* kv, int64_t kv_rows,
+                            const int64_t* kv_begin_host, const int64_t* kv_end_host,
+                            const int64_t* kv_begin_dev, const int64_t* kv_end_dev,
+                            int D, int heads, int d_h, int n_layers,
+                            const stca_full_layer* layers, float* out, void* workspace,
+                            size_t ws_bytes, sa_stream_t stream);
+
+/*
  * stca_fuse -- linear fusion of the two branches (paper Sec. 3.4 leaves the
  * fusion to a light MLP or gate; this library applies one linear layer):
  *   out = [z_r ; z_u] W_F + b_F

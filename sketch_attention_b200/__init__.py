@@ -6,7 +6,7 @@ is no CPU fallback: if the library is missing or a call fails, an exception
 is raised.
 
 Entry points keep the C names: ``sa_forward``, ``sa_backward``,
-``stca_forward``, ``stca_fuse`` (plus the workspace queries).
+``stca_forward``, ``stca_forward_full``, ``stca_fuse`` (plus the workspace queries).
 """
 from __future__ import annotations
 
@@ -29,7 +29,8 @@ EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_w
            "sa_forward", "sa_backward_workspace", "sa_backward", "stca_forward_workspace",
            "stca_forward", "stca_fuse", "sa_launch_count", "sa_profile", "sa_profile_read",
            "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward",
-           "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate")
+           "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate",
+           "stca_forward_full_workspace", "stca_forward_full")
 
 
 class SAError(RuntimeError):
@@ -41,6 +42,13 @@ class SAError(RuntimeError):
 class StcaLayerC(ctypes.Structure):
     _fields_ = [("W_Q", ctypes.c_void_p), ("W_K", ctypes.c_void_p),
                 ("W_V", ctypes.c_void_p), ("W_O", ctypes.c_void_p)]
+
+
+STCA_FFN_KEYS = ("hist_W1", "hist_W3", "hist_W2", "q_W1", "q_W3", "q_W2")
+
+
+class StcaFullLayerC(ctypes.Structure):
+    _fields_ = [("attn", StcaLayerC)] + [(k, ctypes.c_void_p) for k in STCA_FFN_KEYS]
 
 
 class RefineLayerC(ctypes.Structure):
@@ -83,6 +91,11 @@ def load(path: Optional[str] = None):
     lib.stca_forward.restype = _i
     lib.stca_forward.argtypes = [_vp, _i, _vp, _vp, _i, _vp, _i64, _vp, _vp, _vp, _vp,
                                  _i, _i, _i, _i, ctypes.POINTER(StcaLayerC), _vp, _vp, _sz, _vp]
+    lib.stca_forward_full_workspace.restype = _sz
+    lib.stca_forward_full_workspace.argtypes = [_i, _i64, _i64, _i, _i, _i, _i]
+    lib.stca_forward_full.restype = _i
+    lib.stca_forward_full.argtypes = [_vp, _i, _vp, _vp, _i, _vp, _i64, _vp, _vp, _vp, _vp,
+                                      _i, _i, _i, _i, ctypes.POINTER(StcaFullLayerC), _vp, _vp, _sz, _vp]
     lib.stca_fuse.restype = _i
     lib.stca_fuse.argtypes = [_vp, _vp, _vp, _vp, _i64, _i, _vp, _vp]
     lib.sa_forward_noalloc.restype = _i
@@ -333,6 +346,56 @@ def stca_forward(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin, kv_e
                           _p(kbd), _p(ked), D, heads, d_h, len(layers), arr, _p(res),
                           _p(workspace), workspace.numel(), _stream(stream))
     _check("stca_forward", st)
+    return res
+
+
+def stca_forward_full_workspace(B: int, C_total: int, kv_total: int, D: int, heads: int, d_h: int,
+                                dtype: int) -> int:
+    return int(load().stca_forward_full_workspace(B, C_total, kv_total, D, heads, d_h, dtype))
+
+
+def stca_forward_full(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin, kv_end,
+                      layers: Sequence[dict], heads: int, d_h: int, *,
+                      cand_offsets_dev=None, kv_begin_dev=None, kv_end_dev=None,
+                      out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """One STCA branch of full layers (the attention layer plus the history- and
+    query-side SwiGLU FFNs).  ``layers``: dicts as for stca_forward plus, each
+    optional (absent or None = no such FFN), hist_W1, hist_W3 [D, 2D], hist_W2
+    [2D, D], q_W1, q_W3 [D, 2D], q_W2 [2D, D] (fp32 CUDA tensors).  Returns
+    out [C_total, D] fp32."""
+    lib = load()
+    _need_cuda(q, kv)
+    dt = _dtype_code(q)
+    if kv.dtype != q.dtype:
+        raise TypeError("q and kv must have the same dtype")
+    cand = _host_i64(cand_offsets)
+    kb, ke = _host_i64(kv_begin), _host_i64(kv_end)
+    B = len(cand) - 1
+    D = q.shape[1]
+    dev = q.device
+    C = int(cand[-1])
+    kv_total = int((ke - kb).sum()) if B else 0
+    res = out if out is not None else torch.empty(C, D, device=dev)
+    arr = (StcaFullLayerC * len(layers))()
+    for i, L in enumerate(layers):
+        _need_cuda(L["W_Q"], L["W_K"], L["W_V"], L.get("W_O"), *(L.get(k) for k in STCA_FFN_KEYS))
+        arr[i].attn.W_Q = L["W_Q"].data_ptr()
+        arr[i].attn.W_K = L["W_K"].data_ptr()
+        arr[i].attn.W_V = L["W_V"].data_ptr()
+        arr[i].attn.W_O = L["W_O"].data_ptr() if L.get("W_O") is not None else None
+        for k in STCA_FFN_KEYS:
+            setattr(arr[i], k, L[k].data_ptr() if L.get(k) is not None else None)
+    ws_bytes = lib.stca_forward_full_workspace(B, C, kv_total, D, heads, d_h, dt)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    cd = _dev_i64(cand, dev, cand_offsets_dev)
+    kbd = _dev_i64(kb, dev, kv_begin_dev)
+    ked = _dev_i64(ke, dev, kv_end_dev)
+    st = lib.stca_forward_full(_p(q), dt, _hp(cand), _p(cd), B, _p(kv), kv.shape[0], _hp(kb), _hp(ke),
+                               _p(kbd), _p(ked), D, heads, d_h, len(layers), arr, _p(res),
+                               _p(workspace), workspace.numel(), _stream(stream))
+    _check("stca_forward_full", st)
     return res
 
 

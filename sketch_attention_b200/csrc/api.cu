@@ -502,26 +502,32 @@ size_t stca_forward_workspace(int B, int64_t C_total, int D, int heads, int d_h,
   return layout_stca(nullptr, B, C_total, D, heads, d_h, nullptr);
 }
 
-sa_status stca_forward(const void* q, sa_dtype dtype, const int64_t* cand_offsets_host,
-                       const int64_t* cand_offsets_dev, int B, const void* kv, int64_t kv_rows,
-                       const int64_t* kv_begin_host, const int64_t* kv_end_host,
-                       const int64_t* kv_begin_dev, const int64_t* kv_end_dev, int D, int heads,
-                       int d_h, int n_layers, const stca_layer* layers, float* out,
-                       void* workspace, size_t ws_bytes, sa_stream_t stream) {
+}  // extern "C"
+
+namespace {
+// Checks shared by stca_forward and stca_forward_full; fills a (less the
+// layers) and the number of query tiles and of key rows.
+sa_status stca_check(const void* q, sa_dtype dtype, const int64_t* cand_offsets_host,
+                     const int64_t* cand_offsets_dev, int B, const void* kv, int64_t kv_rows,
+                     const int64_t* kv_begin_host, const int64_t* kv_end_host,
+                     const int64_t* kv_begin_dev, const int64_t* kv_end_dev, int D, int heads,
+                     int d_h, int n_layers, const stca_layer* const* attn, float* out, StcaArgs* a,
+                     int* max_tiles, int64_t* kv_total) {
   if (B < 1) return fail(SA_ERR_INVALID_ARG, "B must be >= 1");
   if (dtype != SA_F32 && dtype != SA_BF16) return fail(SA_ERR_INVALID_ARG, "unknown dtype");
   if (D != 128) return fail(SA_ERR_UNSUPPORTED, "D must be 128");
   if (heads < 1 || d_h < 1 || (int64_t)heads * d_h > 4096)
     return fail(SA_ERR_UNSUPPORTED, "need heads >= 1, d_h >= 1, heads*d_h <= 4096");
-  if (n_layers < 1 || !layers) return fail(SA_ERR_INVALID_ARG, "need n_layers >= 1 and layers");
+  if (n_layers < 1 || !attn) return fail(SA_ERR_INVALID_ARG, "need n_layers >= 1 and layers");
   if (kv_rows < 0) return fail(SA_ERR_INVALID_ARG, "kv_rows must be >= 0");
   SA_TRY(check_offsets(cand_offsets_host, B, "cand_offsets_host"));
   if (!kv_begin_host || !kv_end_host) return fail(SA_ERR_INVALID_ARG, "kv ranges are NULL");
-  int64_t max_rows = 0;
+  int64_t max_rows = 0, kv_sum = 0;
   for (int u = 0; u < B; ++u) {
     if (kv_begin_host[u] < 0 || kv_end_host[u] < kv_begin_host[u] || kv_end_host[u] > kv_rows)
       return fail(SA_ERR_INVALID_ARG, "bad key range of user " + std::to_string(u));
     max_rows = std::max(max_rows, (cand_offsets_host[u + 1] - cand_offsets_host[u]) * heads);
+    kv_sum += kv_end_host[u] - kv_begin_host[u];
   }
   const int64_t C = cand_offsets_host[B];
   SA_TRY(check_ptr(q, "q", C == 0));
@@ -531,28 +537,95 @@ sa_status stca_forward(const void* q, sa_dtype dtype, const int64_t* cand_offset
   SA_TRY(check_ptr(kv_end_dev, "kv_end_dev"));
   SA_TRY(check_ptr(out, "out", C == 0));
   for (int l = 0; l < n_layers; ++l) {
-    SA_TRY(check_ptr(layers[l].W_Q, "layers[].W_Q"));
-    SA_TRY(check_ptr(layers[l].W_K, "layers[].W_K"));
-    SA_TRY(check_ptr(layers[l].W_V, "layers[].W_V"));
-    SA_TRY(check_ptr(layers[l].W_O, "layers[].W_O", true));
-    if (!layers[l].W_O && heads * d_h != D)
+    const stca_layer& L = *attn[l];
+    SA_TRY(check_ptr(L.W_Q, "layers[].W_Q"));
+    SA_TRY(check_ptr(L.W_K, "layers[].W_K"));
+    SA_TRY(check_ptr(L.W_V, "layers[].W_V"));
+    SA_TRY(check_ptr(L.W_O, "layers[].W_O", true));
+    if (!L.W_O && heads * d_h != D)
       return fail(SA_ERR_INVALID_ARG, "W_O = NULL needs heads*d_h == D");
   }
+  const int tq = stca_tc_supported(dtype, D) ? 128 : 32;
+  int64_t tiles = 0;
+  for (int u = 0; u < B; ++u)
+    tiles += ((cand_offsets_host[u + 1] - cand_offsets_host[u]) * heads + tq - 1) / tq;
+  if (tiles > (1LL << 30)) return fail(SA_ERR_UNSUPPORTED, "too many query tiles");
+  *max_tiles = (int)std::max<int64_t>(tiles, 1);
+  *kv_total = kv_sum;
+  *a = StcaArgs{q, dtype, cand_offsets_dev, B, C, kv, kv_rows, kv_begin_dev, kv_end_dev,
+                D, heads, d_h, n_layers, nullptr, out, max_rows};
+  return SA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+sa_status stca_forward(const void* q, sa_dtype dtype, const int64_t* cand_offsets_host,
+                       const int64_t* cand_offsets_dev, int B, const void* kv, int64_t kv_rows,
+                       const int64_t* kv_begin_host, const int64_t* kv_end_host,
+                       const int64_t* kv_begin_dev, const int64_t* kv_end_dev, int D, int heads,
+                       int d_h, int n_layers, const stca_layer* layers, float* out,
+                       void* workspace, size_t ws_bytes, sa_stream_t stream) {
+  if (n_layers < 1 || !layers) return fail(SA_ERR_INVALID_ARG, "need n_layers >= 1 and layers");
+  std::vector<const stca_layer*> attn(n_layers);
+  for (int l = 0; l < n_layers; ++l) attn[l] = &layers[l];
+  StcaArgs a;
+  int max_tiles = 0;
+  int64_t kv_total = 0;
+  SA_TRY(stca_check(q, dtype, cand_offsets_host, cand_offsets_dev, B, kv, kv_rows, kv_begin_host,
+                    kv_end_host, kv_begin_dev, kv_end_dev, D, heads, d_h, n_layers, attn.data(), out,
+                    &a, &max_tiles, &kv_total));
+  const int64_t C = cand_offsets_host[B];
   const size_t need = layout_stca(nullptr, B, C, D, heads, d_h, nullptr);
   if (!workspace || ws_bytes < need)
     return fail(SA_ERR_WORKSPACE, "workspace needs " + std::to_string(need) + " bytes");
   SA_TRY(check_ptr(workspace, "workspace"));
   StcaWork w;
   layout_stca(workspace, B, C, D, heads, d_h, &w);
-  const int tq = stca_tc_supported(dtype, D) ? 128 : 32;
-  int64_t tiles = 0;
-  for (int u = 0; u < B; ++u)
-    tiles += ((cand_offsets_host[u + 1] - cand_offsets_host[u]) * heads + tq - 1) / tq;
-  if (tiles > (1LL << 30)) return fail(SA_ERR_UNSUPPORTED, "too many query tiles");
-  w.max_tiles = (int)std::max<int64_t>(tiles, 1);
-  StcaArgs a{q, dtype, cand_offsets_dev, B, C, kv, kv_rows, kv_begin_dev, kv_end_dev,
-             D, heads, d_h, n_layers, layers, out, max_rows};
+  w.max_tiles = max_tiles;
+  a.layers = layers;
   return stca_run(a, w, (cudaStream_t)stream);
+}
+
+size_t stca_forward_full_workspace(int B, int64_t C_total, int64_t kv_total, int D, int heads,
+                                   int d_h, sa_dtype dtype) {
+  if (B < 1 || C_total < 0 || kv_total < 0 || D < 1 || heads < 1 || d_h < 1) return 0;
+  if (dtype != SA_F32 && dtype != SA_BF16) return 0;
+  return stca_full_layout(nullptr, B, C_total, kv_total, D, heads, d_h, dtype, nullptr);
+}
+
+sa_status stca_forward_full(const void* q, sa_dtype dtype, const int64_t* cand_offsets_host,
+                            const int64_t* cand_offsets_dev, int B, const void* kv, int64_t kv_rows,
+                            const int64_t* kv_begin_host, const int64_t* kv_end_host,
+                            const int64_t* kv_begin_dev, const int64_t* kv_end_dev, int D, int heads,
+                            int d_h, int n_layers, const stca_full_layer* layers, float* out,
+                            void* workspace, size_t ws_bytes, sa_stream_t stream) {
+  if (n_layers < 1 || !layers) return fail(SA_ERR_INVALID_ARG, "need n_layers >= 1 and layers");
+  std::vector<const stca_layer*> attn(n_layers);
+  for (int l = 0; l < n_layers; ++l) {
+    const stca_full_layer& L = layers[l];
+    attn[l] = &L.attn;
+    const int nh = !!L.hist_W1 + !!L.hist_W3 + !!L.hist_W2, nq = !!L.q_W1 + !!L.q_W3 + !!L.q_W2;
+    if ((nh != 0 && nh != 3) || (nq != 0 && nq != 3))
+      return fail(SA_ERR_INVALID_ARG, "layer " + std::to_string(l) + ": an FFN is partly given");
+    for (const float* wp : {L.hist_W1, L.hist_W3, L.hist_W2, L.q_W1, L.q_W3, L.q_W2})
+      SA_TRY(check_ptr(wp, "layers[] FFN weight", true));
+  }
+  StcaArgs a;
+  int max_tiles = 0;
+  int64_t kv_total = 0;
+  SA_TRY(stca_check(q, dtype, cand_offsets_host, cand_offsets_dev, B, kv, kv_rows, kv_begin_host,
+                    kv_end_host, kv_begin_dev, kv_end_dev, D, heads, d_h, n_layers, attn.data(), out,
+                    &a, &max_tiles, &kv_total));
+  const int64_t C = cand_offsets_host[B];
+  const size_t need = stca_full_layout(nullptr, B, C, kv_total, D, heads, d_h, dtype, nullptr);
+  if (!workspace || ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "workspace needs " + std::to_string(need) + " bytes");
+  SA_TRY(check_ptr(workspace, "workspace"));
+  StcaFullWork w;
+  stca_full_layout(workspace, B, C, kv_total, D, heads, d_h, dtype, &w);
+  w.attn.max_tiles = max_tiles;
+  return stca_full_run(a, layers, kv_total, w, (cudaStream_t)stream);
 }
 
 sa_status stca_fuse(const float* z_r, const float* z_u, const float* W_F, const float* b_F,

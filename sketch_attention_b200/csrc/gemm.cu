@@ -155,6 +155,8 @@ sa_status gemm(const Gemm& g0, cudaStream_t stream) {
   const int64_t ctas128 = (int64_t)((g.N + bn - 1) / bn) * ((g.M + 127) / 128) * g.batch * g.split_k;
   const bool small = ctas128 < 2 * device_info().sm_count;
   const int bm = small ? 64 : 128;
+  if ((g.M + bm - 1) / bm > 65535 || (int64_t)g.batch * g.split_k > 65535)
+    return fail(SA_ERR_UNSUPPORTED, std::string(tag) + ": more than 65535 row tiles or batches");
   dim3 grid((g.N + bn - 1) / bn, (g.M + bm - 1) / bm, g.batch * g.split_k);
   const int nt = (bm / RM) * (bn / RN);
   const int variant = (bm == 64 ? 0 : 4) + (bn == 32 ? 0 : 2) + 0;   // tile shape

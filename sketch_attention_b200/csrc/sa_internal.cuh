@@ -100,6 +100,8 @@ sa_status sa_tokenwise_run(const SaFwdArgs& a, const TokenwiseWork& w, cudaStrea
 
 // Sums the split-n partials into H (if a.H), the mass and H/(m+eps) (w.Hhat).
 sa_status sa_reduce(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
+// U = SiLU(G1) * G3 elementwise over n fp32 values (n a multiple of 4, 16-byte aligned)
+sa_status sa_swiglu(const float* G1, const float* G3, int64_t n, float* U, cudaStream_t st);
 sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
 sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaStream_t st);
 sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st);

@@ -73,6 +73,14 @@ unsigned blocks_for(int64_t n, int per_block) {
 }
 }  // namespace
 
+sa_status sa_swiglu(const float* G1, const float* G3, int64_t n, float* U, cudaStream_t st) {
+  if (n <= 0) return SA_OK;
+  SA_TIMED("swiglu_kernel", st,
+           (swiglu_kernel<<<blocks_for(n / 4, 256), 256, 0, st>>>((const float4*)G1, (const float4*)G3,
+                                                                 n / 4, (float4*)U)));
+  return SA_OK;
+}
+
 size_t refine_layout(void* base, int B, int64_t n, int k, int d, SaFwdWork* w, RefineWork* r) {
   Carve c(base);
   SaFwdWork v;
@@ -132,9 +140,7 @@ sa_status sa_refine_run(const void* X, sa_dtype x_dtype, const int64_t* off_dev,
     Gemm g3 = g1;
     g3.B = L.W3; g3.C = r.G3;
     if ((s = gemm(g3, st)) != SA_OK) return s;
-    SA_TIMED("swiglu_kernel", st,
-             (swiglu_kernel<<<blocks_for(rows * 2 * d / 4, 256), 256, 0, st>>>(
-                 (const float4*)r.G1, (const float4*)r.G3, rows * 2 * d / 4, (float4*)r.U)));
+    if ((s = sa_swiglu(r.G1, r.G3, rows * 2 * d, r.U, st)) != SA_OK) return s;
     Gemm g2;
     g2.M = (int)rows; g2.N = d; g2.K = 2 * d;
     g2.A = r.U; g2.lda = 2 * d; g2.B = L.W2; g2.ldb = d; g2.C = r.F; g2.ldc = d;

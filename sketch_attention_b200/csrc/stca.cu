@@ -128,10 +128,9 @@ __global__ void __launch_bounds__(256) stca_attn_simt_kernel(
 unsigned grid_for(int64_t n) { return (unsigned)std::min<int64_t>((n + 255) / 256, 8192); }
 }  // namespace
 
-sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
-  const int D = a.D, H = a.heads, dh = a.d_h, HD = a.heads * a.d_h;
+sa_status stca_begin(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
   const int64_t C = a.C_total;
-  const int64_t nq = C * D;
+  const int64_t nq = C * a.D;
   if (nq > 0) {
     if (a.dtype == SA_BF16)
       SA_TIMED("to_f32_kernel", st,
@@ -141,13 +140,20 @@ sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
                (to_f32_kernel<<<grid_for(nq), 256, 0, st>>>((const float*)a.q, nq, a.out)));
   }
   if (C == 0) return SA_OK;
-  const bool tc = stca_tc_supported(a.dtype, D);
-  const int tq = tc ? 128 : 32;
+  const int tq = stca_tc_supported(a.dtype, a.D) ? 128 : 32;
   SA_TIMED("tile_prefix_kernel", st,
-           (tile_prefix_kernel<<<1, 1, 0, st>>>(a.cand_dev, a.B, H, tq, w.tile_prefix)));
+           (tile_prefix_kernel<<<1, 1, 0, st>>>(a.cand_dev, a.B, a.heads, tq, w.tile_prefix)));
+  return SA_OK;
+}
+
+sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWork& w, cudaStream_t st) {
+  const int D = a.D, H = a.heads, dh = a.d_h, HD = a.heads * a.d_h;
+  const int64_t C = a.C_total;
+  const int64_t nq = C * D;
+  if (C == 0) return SA_OK;
+  const bool tc = stca_tc_supported(a.dtype, D);
   sa_status s;
-  for (int l = 0; l < a.n_layers; ++l) {
-    const stca_layer& L = a.layers[l];
+  {
     // Qh[:, h] = q W_Q^h
     Gemm g1;
     g1.M = (int)C; g1.N = dh; g1.K = D;
@@ -203,6 +209,12 @@ sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
     }
   }
   return SA_OK;
+}
+
+sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
+  sa_status s = stca_begin(a, w, st);
+  for (int l = 0; s == SA_OK && l < a.n_layers; ++l) s = stca_attend_layer(a, a.layers[l], w, st);
+  return s;
 }
 
 sa_status stca_fuse_run(const float* z_r, const float* z_u, const float* W_F, const float* b_F,

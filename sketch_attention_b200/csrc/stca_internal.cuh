@@ -27,6 +27,31 @@ struct StcaWork {
 };
 
 sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st);
+// The two halves of stca_run: q -> out (fp32) and the query-tile prefix, then
+// one attention layer (projections, attention over a.kv, W_O, residual).
+sa_status stca_begin(const StcaArgs& a, const StcaWork& w, cudaStream_t st);
+sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWork& w, cudaStream_t st);
+
+// Full STCA layers (history- and query-side SwiGLU FFNs).
+struct StcaFullWork {
+  StcaWork attn;
+  void* Hk;                 // [kv_total, D] key rows (kv dtype), transformed in place
+  int64_t* kpre;            // [B+1] start of each user's rows in Hk
+  float* G1; float* G3; float* U;   // [max(C, rows of an fp32 history FFN), 2D] fp32
+  __nv_bfloat16* W13t;      // [4 * 128, D] bf16: the tensor-core FFN's first-layer weights
+  __nv_bfloat16* W2t;       // [D, 2D] bf16: its second-layer weights (transposed)
+};
+size_t stca_full_layout(void* base, int B, int64_t C, int64_t kv_total, int D, int heads, int d_h,
+                        sa_dtype dtype, StcaFullWork* w);
+sa_status stca_full_run(const StcaArgs& a, const stca_full_layer* layers, int64_t kv_total,
+                        const StcaFullWork& w, cudaStream_t st);
+
+// x <- x + (SiLU(x W1) * (x W3)) W2 for rows of bf16 x, D = 128, in place, on
+// the tensor cores; W13t / W2t as prepared by stca_ffn_weights_bf16.
+sa_status stca_ffn_weights_bf16(const float* W1, const float* W3, const float* W2,
+                                __nv_bfloat16* W13t, __nv_bfloat16* W2t, cudaStream_t st);
+sa_status stca_hist_ffn_tc(__nv_bfloat16* X, int64_t rows, const __nv_bfloat16* W13t,
+                           const __nv_bfloat16* W2t, cudaStream_t st);
 
 bool stca_tc_supported(sa_dtype dtype, int D);
 sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st);
