@@ -3,19 +3,26 @@
 //   x <- x + (SiLU(x W1) * (x W3)) W2,   W1, W3 [128, 256], W2 [256, 128]
 // in place, with the 256-wide inner activations never leaving the SM.
 //
-// Persistent: one CTA per SM keeps both weight layers resident in shared
-// memory (bf16, 192 KB) and walks 128-row tiles.  A tile's inner width is
+// Persistent: one CTA per SM keeps W1|W3 resident in shared memory (bf16,
+// 128 KB), streams W2 a quarter at a time from L2, and walks 128-row tiles
+// with two X buffers.  A tile's inner width is
 // done in four quarters of 64:
-//   G_q  = X [W1_q | W3_q]     M=128 rows, N=128, K=128   (SS, fp32 in TMEM)
+//   G_q  = X [W1_q | W3_q]     M=128 rows, N=128, K=128   (X from TMEM, fp32 in TMEM)
 //   U_q  = SiLU(G1_q) * G3_q   registers -> bf16 pairs in TMEM
 //   F   += U_q W2_q            M=128, N=128, K=64          (A from TMEM)
 // and x + F goes back to the row as bf16.  G and U are double-buffered, so
 // the tensor pipe computes G_{q+1} while the epilogue warps turn G_q into U_q.
 // SiLU(g) g3 = (g/2) g3 (1 + tanh(g/2)): one MUFU operation per element.
 //
-// Warp roles (10 warps): 0 TMA, 1 MMA issue + TMEM owner, 2-9 two warpgroups
-// of epilogue (warpgroup h takes inner columns 32h..32h+31 of each quarter
-// and output columns 64h..64h+63).
+// Shared memory bandwidth: an N=128 MMA with both operands in shared memory
+// reads 128 bytes per clock, all that an SM's shared memory delivers, so the
+// X tile is moved into TMEM once per tile and every MMA reads only its B
+// operand from shared memory.
+//
+// Warp roles (16 warps): 0 TMA of W1|W3 and the X tiles, 1 first-layer MMA
+// issue + TMEM owner, 2-9 two warpgroups of SiLU gating (warpgroup h takes the
+// quarters of parity h), 10-13 X into TMEM and the residual add and
+// write-back, 14 TMA of the W2 quarters, 15 second-layer MMA issue.
 #include <algorithm>
 #include <cstring>
 #include <mutex>
@@ -28,20 +35,22 @@ namespace sa {
 namespace {
 using namespace tc;
 
-constexpr int DD = 128, TM = 128, THREADS = 320;
+constexpr int DD = 128, TM = 128, THREADS = 512;
 constexpr uint32_t W13_BYTES = 4 * 128 * DD * 2;   // [512 rows][128] bf16, two 64-column atoms
-constexpr uint32_t W2_BYTES = DD * 2 * DD * 2;     // [128 rows][256] bf16, four 64-column atoms
+constexpr uint32_t W2Q_BYTES = DD * 64 * 2;        // one quarter of W2t: [128 rows][64] bf16
 constexpr uint32_t X_BYTES = TM * DD * 2;          // one row tile, two atoms
-constexpr uint32_t OFF_W13 = 0, OFF_W2 = OFF_W13 + W13_BYTES, OFF_X = OFF_W2 + W2_BYTES;
-constexpr uint32_t OFF_BAR = OFF_X + X_BYTES;
+// W1|W3 stay resident; X tiles and W2 quarters (re-read from L2) are double-buffered
+constexpr uint32_t OFF_W13 = 0, OFF_X = OFF_W13 + W13_BYTES, OFF_W2 = OFF_X + 2 * X_BYTES;
+constexpr uint32_t OFF_BAR = OFF_W2 + 2 * W2Q_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-// TMEM columns: G double buffer, U double buffer (bf16 pairs), F accumulator
-constexpr uint32_t TM_G = 0, TM_U = 256, TM_F = 384, TM_COLS = 512;
+// TMEM columns: G double buffer, U double buffer (bf16 pairs), the X tile as the
+// first layer's A operand (bf16 pairs), F accumulator
+constexpr uint32_t TM_G = 0, TM_U = 256, TM_X = 320, TM_F = 384, TM_COLS = 512;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
 struct Bars {
-  uint64_t w_full, x_full, x_empty, g_full[2], g_empty[2], u_full[2], u_empty[2], f_full, f_empty,
-      mma_done;
+  uint64_t w_full, x_full[2], x_empty[2], w2_full[2], w2_empty[2], xt_full, xt_empty, g_full[2],
+      g_empty[2], u_full[2], u_empty[2], f_full, f_empty, mma_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -53,10 +62,19 @@ struct Params {
   int* err;
 };
 
+// SiLU(g1) g3 for a pair of elements: (g1/2) g3 (1 + tanh(g1/2)), one MUFU tanh per
+// element (tanh.approx: relative error about 2^-11, below the bf16 rounding of U).
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+__device__ __forceinline__ uint32_t silu_mul_bf16x2(float a0, float a1, float b0, float b1) {
+  const float2 hx = __fmul2_rn(make_float2(a0, a1), make_float2(0.5f, 0.5f));
+  const float2 th = make_float2(tanh_approx(hx.x), tanh_approx(hx.y));
+  const float2 hg = __fmul2_rn(hx, make_float2(b0, b1));
+  const float2 u = __ffma2_rn(hg, th, hg);
+  return pack_bf16x2(u.x, u.y);
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -71,17 +89,22 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->w_full, 1);
-    mbar_init(&bars->x_full, 1);
-    mbar_init(&bars->x_empty, 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->x_full[b], 1);
+      mbar_init(&bars->x_empty[b], 128);
+      mbar_init(&bars->w2_full[b], 1);
+      mbar_init(&bars->w2_empty[b], 1);
       mbar_init(&bars->g_full[b], 1);
-      mbar_init(&bars->g_empty[b], 256);
-      mbar_init(&bars->u_full[b], 256);
+      mbar_init(&bars->g_empty[b], 128);
+      mbar_init(&bars->u_full[b], 128);
       mbar_init(&bars->u_empty[b], 1);
     }
+    mbar_init(&bars->xt_full, 128);
+    mbar_init(&bars->xt_empty, 1);
     mbar_init(&bars->f_full, 1);
-    mbar_init(&bars->f_empty, 256);
-    mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->f_empty, 128);
+    mbar_init(&bars->mma_done[0], 1);
+    mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -95,26 +118,24 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0 && lane == 0) {
-    // ---------------------------------------------------------------- TMA
+    // ---------------------------------------------------------------- TMA: W1|W3, X tiles
     prefetch_tensormap(&tmX);
     prefetch_tensormap(&tmW13);
-    prefetch_tensormap(&tmW2);
-    mbar_arrive_expect_tx(&bars->w_full, W13_BYTES + W2_BYTES);
+    mbar_arrive_expect_tx(&bars->w_full, W13_BYTES);
     for (int a = 0; a < 2; ++a)
       for (int r = 0; r < 2; ++r)
         tma_load_2d(smem + OFF_W13 + a * (W13_BYTES / 2) + r * (W13_BYTES / 4), &tmW13, &bars->w_full,
                     64 * a, 256 * r);
-    for (int a = 0; a < 4; ++a)
-      tma_load_2d(smem + OFF_W2 + a * (W2_BYTES / 4), &tmW2, &bars->w_full, 64 * a, 0);
     int i = 0, issued = 0;
     for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++i) {
-      if (i > 0 && !mbar_wait(&bars->x_empty, (i - 1) & 1, abort, p.err)) break;
-      mbar_arrive_expect_tx(&bars->x_full, X_BYTES);
-      tma_load_2d(smem + OFF_X, &tmX, &bars->x_full, 0, t * TM);
-      tma_load_2d(smem + OFF_X + X_BYTES / 2, &tmX, &bars->x_full, 64, t * TM);
+      const int s = i & 1;
+      if (i >= 2 && !mbar_wait(&bars->x_empty[s], ((i >> 1) - 1) & 1, abort, p.err)) break;
+      mbar_arrive_expect_tx(&bars->x_full[s], X_BYTES);
+      tma_load_2d(smem + OFF_X + s * X_BYTES, &tmX, &bars->x_full[s], 0, t * TM);
+      tma_load_2d(smem + OFF_X + s * X_BYTES + X_BYTES / 2, &tmX, &bars->x_full[s], 64, t * TM);
       issued = i + 1;
-      // the next tile waits for this one's logits; start its trip to L2 now
-      const int tn = t + (int)gridDim.x;
+      // the tile after next: start its trip to L2
+      const int tn = t + 2 * (int)gridDim.x;
       if (tn < p.ntiles) {
         tma_prefetch_l2_2d(&tmX, 0, tn * TM);
         tma_prefetch_l2_2d(&tmX, 64, tn * TM);
@@ -122,113 +143,190 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (*abort) {
       mbar_wait_bounded(&bars->w_full, 0);
-      if (issued > 0) mbar_wait_bounded(&bars->x_full, (issued - 1) & 1);
+      for (int j = std::max(0, issued - 2); j < issued; ++j)
+        mbar_wait_bounded(&bars->x_full[j & 1], (j >> 1) & 1);
     }
-  } else if (warp == 1 && lane == 0) {
-    // ---------------------------------------------------------------- MMA
-    const uint32_t id = idesc_bf16(128, 128, false, false);
-    const uint32_t xa = smem_u32(smem + OFF_X), w13 = smem_u32(smem + OFF_W13),
-                   w2 = smem_u32(smem + OFF_W2);
-    bool ok = mbar_wait(&bars->w_full, 0, abort, p.err);
-    int i = 0;
-    // G_q = X [W1_q | W3_q]; the quarter's rows of W13t start at 128 q
-    auto gemm1 = [&](int q) -> bool {
-      const int b = q & 1, n = 2 * i + (q >> 1);
-      if (n >= 1 && !mbar_wait(&bars->g_empty[b], (n - 1) & 1, abort, p.err)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
-        mma_ss(tmem + TM_G + 128 * b,
-               smem_desc(xa + (ks >> 2) * (X_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B),
-               smem_desc(w13 + (ks >> 2) * (W13_BYTES / 2) + q * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B),
-               id, ks > 0 ? 1u : 0u);
-      mma_commit(&bars->g_full[b]);
-      return true;
-    };
-    // F += U_q W2_q; atom q of W2t holds inner columns 64q..64q+63
-    auto gemm2 = [&](int q) -> bool {
-      const int b = q & 1, n = 2 * i + (q >> 1);
-      if (!mbar_wait(&bars->u_full[b], n & 1, abort, p.err)) return false;
-      if (q == 0 && i >= 1 && !mbar_wait(&bars->f_empty, (i - 1) & 1, abort, p.err)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        mma_ts(tmem + TM_F, tmem + TM_U + 32 * b + 8 * ks,
-               smem_desc(w2 + q * (W2_BYTES / 4) + ks * 32, 16, 1024, SWZ_128B), id,
-               (q > 0 || ks > 0) ? 1u : 0u);
-      mma_commit(&bars->u_empty[b]);
-      if (q == 3) mma_commit(&bars->f_full);
-      return true;
-    };
-    for (int t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x, ++i) {
-      if (!mbar_wait(&bars->x_full, i & 1, abort, p.err)) break;
-      tc_fence_after();
-      ok = gemm1(0) && gemm1(1) && gemm2(0) && gemm1(2) && gemm2(1) && gemm1(3);
-      if (!ok) break;
-      mma_commit(&bars->x_empty);      // X is read by the first-layer MMAs only
-      ok = gemm2(2) && gemm2(3);
-    }
-    mma_commit(&bars->mma_done);
-    mbar_wait_bounded(&bars->mma_done, 0);
-  } else if (warp >= 2) {
-    // ---------------------------------------------------------------- epilogue
-    const int q4 = warp % 4, h = (warp - 2) / 4;
-    const int row = q4 * 32 + lane;
-    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
-    const float2 half2 = make_float2(0.5f, 0.5f);
-    int i = 0;
+  } else if (warp == 14 && lane == 0) {
+    // ---------------------------------------------------------------- TMA: W2 quarters
+    prefetch_tensormap(&tmW2);
+    int i = 0, issued = 0;
     for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++i) {
       bool ok = true;
       for (int q = 0; q < 4; ++q) {
         const int b = q & 1, n = 2 * i + (q >> 1);
-        if (!mbar_wait(&bars->g_full[b], n & 1, abort, p.err)) { ok = false; break; }
+        if (n >= 1 && !mbar_wait(&bars->w2_empty[b], (n - 1) & 1, abort, p.err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&bars->w2_full[b], W2Q_BYTES);
+        tma_load_2d(smem + OFF_W2 + b * W2Q_BYTES, &tmW2, &bars->w2_full[b], 64 * q, 0);
+        issued = n + 1;
+      }
+      if (!ok) break;
+    }
+    if (*abort)
+      for (int n = std::max(0, issued - 2); n < issued; ++n)
+        mbar_wait_bounded(&bars->w2_full[n & 1], (n >> 1) & 1);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- first-layer MMAs
+    // G_q = X [W1_q | W3_q]; the quarter's rows of W13t start at 128 q.  A thread of
+    // its own, so a G buffer is refilled as soon as its gating warpgroup has read it,
+    // whatever the second-layer MMAs are waiting for.
+    const uint32_t id = idesc_bf16(128, 128, false, false);
+    const uint32_t w13 = smem_u32(smem + OFF_W13);
+    bool ok = mbar_wait(&bars->w_full, 0, abort, p.err);
+    int i = 0;
+    for (int t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x, ++i) {
+      if (!mbar_wait(&bars->xt_full, i & 1, abort, p.err)) break;
+      for (int q = 0; ok && q < 4; ++q) {
+        const int b = q & 1, n = 2 * i + (q >> 1);
+        if (n >= 1 && !mbar_wait(&bars->g_empty[b], (n - 1) & 1, abort, p.err)) { ok = false; break; }
         tc_fence_after();
-        float g1[32], g3[32];
-        tmem_ld32(tmem + lane_addr + TM_G + 128 * b + 32 * h, g1);
-        tmem_ld32(tmem + lane_addr + TM_G + 128 * b + 64 + 32 * h, g3);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&bars->g_empty[b]);
-        uint32_t u[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float2 hx = __fmul2_rn(make_float2(g1[2 * j], g1[2 * j + 1]), half2);
-          const float2 th = make_float2(tanh_approx(hx.x), tanh_approx(hx.y));
-          const float2 hg = __fmul2_rn(hx, make_float2(g3[2 * j], g3[2 * j + 1]));
-          const float2 uu = __ffma2_rn(hg, th, hg);
-          u[j] = pack_bf16x2(uu.x, uu.y);
+        for (int ks = 0; ks < 8; ++ks)
+          mma_ts(tmem + TM_G + 128 * b, tmem + TM_X + 8 * ks,
+                 smem_desc(w13 + (ks >> 2) * (W13_BYTES / 2) + q * 16384 + (ks & 3) * 32, 16, 1024, SWZ_128B),
+                 id, ks > 0 ? 1u : 0u);
+        mma_commit(&bars->g_full[b]);
+      }
+      if (ok) mma_commit(&bars->xt_empty);     // X in TMEM is read by these MMAs only
+    }
+    mma_commit(&bars->mma_done[0]);
+    mbar_wait_bounded(&bars->mma_done[0], 0);
+  } else if (warp == 15 && lane == 0) {
+    // ---------------------------------------------------------------- second-layer MMAs
+    // F += U_q W2_q; W2 slot q % 2 holds W2t's inner columns 64q..64q+63
+    const uint32_t id = idesc_bf16(128, 128, false, false);
+    const uint32_t w2 = smem_u32(smem + OFF_W2);
+    bool ok = true;
+    int i = 0;
+    for (int t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x, ++i) {
+      for (int q = 0; q < 4; ++q) {
+        const int b = q & 1, n = 2 * i + (q >> 1);
+        if (!mbar_wait(&bars->u_full[b], n & 1, abort, p.err) ||
+            !mbar_wait(&bars->w2_full[b], n & 1, abort, p.err) ||
+            (q == 0 && i >= 1 && !mbar_wait(&bars->f_empty, (i - 1) & 1, abort, p.err))) {
+          ok = false;
+          break;
         }
-        // U buffer b was last read by the second-layer MMAs of use n-1
-        if (n >= 1 && !mbar_wait(&bars->u_empty[b], (n - 1) & 1, abort, p.err)) { ok = false; break; }
         tc_fence_after();
-        tmem_st16(tmem + lane_addr + TM_U + 32 * b + 16 * h, u);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          mma_ts(tmem + TM_F, tmem + TM_U + 32 * b + 8 * ks,
+                 smem_desc(w2 + b * W2Q_BYTES + ks * 32, 16, 1024, SWZ_128B), id, (q > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(&bars->u_empty[b]);
+        mma_commit(&bars->w2_empty[b]);
+        if (q == 3) mma_commit(&bars->f_full);
+      }
+    }
+    mma_commit(&bars->mma_done[1]);
+    mbar_wait_bounded(&bars->mma_done[1], 0);
+  } else if (warp >= 2 && warp < 10) {
+    // ---------------------------------------------------------------- SiLU gate
+    // Warpgroup h = 0, 1 takes the quarters q with q % 2 == h (G and U buffer
+    // h), so two quarters are in flight: one warpgroup waits on TMEM while the
+    // other computes.  Each thread owns one row; 32 inner columns per pass.
+    const int q4 = warp % 4, h = (warp - 2) / 4;
+    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    int i = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x, ++i) {
+      for (int q = h; q < 4; q += 2) {
+        const int n = 2 * i + (q >> 1);
+        if (!mbar_wait(&bars->g_full[h], n & 1, abort, p.err)) { ok = false; break; }
+        tc_fence_after();
+        for (int c = 0; c < 2; ++c) {
+          float g1[32], g3[32];
+          tmem_ld32(tmem + lane_addr + TM_G + 128 * h + 32 * c, g1);
+          tmem_ld32(tmem + lane_addr + TM_G + 128 * h + 64 + 32 * c, g3);
+          tmem_wait_ld();
+          if (c == 1) {
+            tc_fence_before();
+            mbar_arrive(&bars->g_empty[h]);
+          }
+          uint32_t u[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) u[j] = silu_mul_bf16x2(g1[2 * j], g1[2 * j + 1], g3[2 * j], g3[2 * j + 1]);
+          // U buffer h was last read by the second-layer MMAs of use n-1
+          if (c == 0 && n >= 1 && !mbar_wait(&bars->u_empty[h], (n - 1) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          tmem_st16(tmem + lane_addr + TM_U + 32 * h + 16 * c, u);
+        }
+        if (!ok) break;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars->u_full[b]);
+        mbar_arrive(&bars->u_full[h]);
       }
-      if (!ok || !mbar_wait(&bars->f_full, i & 1, abort, p.err)) break;
+    }
+  } else if (warp >= 10 && warp < 14) {
+    // ---------------------------------------------------------------- X to TMEM, x + F
+    // Each thread owns one row.  It moves the row of the next tile from shared
+    // memory (swizzled) into TMEM as the first layer's A operand, so the MMAs
+    // read only W1|W3 from shared memory, then writes x + F of this tile.
+    const int q4 = warp % 4;
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
+    // tile j's row: 16 pieces of 16 bytes (8 bf16), piece 8a + c at atom a, chunk c ^ (row % 8)
+    auto stage_x = [&](int j) -> bool {
+      const int s = j & 1;
+      if (!mbar_wait(&bars->x_full[s], (j >> 1) & 1, abort, p.err)) return false;
+      if (j >= 1 && !mbar_wait(&bars->xt_empty, (j - 1) & 1, abort, p.err)) return false;
+      const uint32_t base = smem_u32(smem + OFF_X + s * X_BYTES) + row * 128;
+      uint32_t v[64];
+#pragma unroll
+      for (int pc = 0; pc < 16; ++pc) {
+        const uint32_t addr = base + (pc >> 3) * (X_BYTES / 2) + (((pc & 7) ^ (row & 7)) << 4);
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v[4 * pc]), "=r"(v[4 * pc + 1]), "=r"(v[4 * pc + 2]), "=r"(v[4 * pc + 3])
+                     : "r"(addr));
+      }
+      mbar_arrive(&bars->x_empty[s]);
       tc_fence_after();
-      float f[64];
-      tmem_ld32(tmem + lane_addr + TM_F + 64 * h, f);
-      tmem_ld32(tmem + lane_addr + TM_F + 64 * h + 32, f + 32);
-      tmem_wait_ld();
+      tmem_st32(tmem + lane_addr + TM_X, v);
+      tmem_st32(tmem + lane_addr + TM_X + 32, v + 32);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bars->f_empty);
+      mbar_arrive(&bars->xt_full);
+      return true;
+    };
+    int i = 0;
+    bool ok = blockIdx.x < p.ntiles && stage_x(0);
+    for (int t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x, ++i) {
+      // the next tile's X goes in as soon as this tile's first-layer MMAs are done
+      if (t + (int)gridDim.x < p.ntiles && !stage_x(i + 1)) break;
       const int64_t grow = (int64_t)t * TM + row;
-      if (grow < p.rows) {
-        uint4* px = (uint4*)(p.X + grow * DD + 64 * h);
+      const bool valid = grow < p.rows;
+      const uint4* px = (const uint4*)(p.X + (valid ? grow : 0) * DD);
+      uint32_t xr[64];                  // the row as bf16 pairs
 #pragma unroll
-        for (int v = 0; v < 8; ++v) {
-          uint4 x = px[v];
-          uint32_t* xw = (uint32_t*)&x;
+      for (int v = 0; v < 16; ++v) {
+        const uint4 x = valid ? px[v] : make_uint4(0, 0, 0, 0);
+        xr[4 * v] = x.x; xr[4 * v + 1] = x.y; xr[4 * v + 2] = x.z; xr[4 * v + 3] = x.w;
+      }
+      if (!mbar_wait(&bars->f_full, i & 1, abort, p.err)) break;
+      tc_fence_after();
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 xb = *(__nv_bfloat162*)&xw[e];
-            const float2 xf = __bfloat1622float2(xb);
-            xw[e] = pack_bf16x2(xf.x + f[8 * v + 2 * e], xf.y + f[8 * v + 2 * e + 1]);
-          }
-          px[v] = x;
+      for (int c = 0; c < 8; ++c) {
+        float f[16];
+        tmem_ld16(tmem + lane_addr + TM_F + 16 * c, f);
+        tmem_wait_ld16(f);
+        if (c == 7) {
+          tc_fence_before();
+          mbar_arrive(&bars->f_empty);
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32
+          const float lo = __uint_as_float(xr[8 * c + e] << 16);
+          const float hi = __uint_as_float(xr[8 * c + e] & 0xFFFF0000u);
+          xr[8 * c + e] = pack_bf16x2(lo + f[2 * e], hi + f[2 * e + 1]);
+        }
+      }
+      if (valid) {
+        uint4* po = (uint4*)(p.X + grow * DD);
+#pragma unroll
+        for (int v = 0; v < 16; ++v)
+          po[v] = make_uint4(xr[4 * v], xr[4 * v + 1], xr[4 * v + 2], xr[4 * v + 3]);
       }
     }
   }
