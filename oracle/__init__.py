@@ -55,7 +55,7 @@ import numpy as np
 __all__ = [
     "sa_forward", "sa_user", "sa_backward", "stca_branch", "stca_branch_reordered",
     "stca_fuse", "assignment", "token_lse", "layer_norm", "swiglu_ffn", "sa_refine_user",
-    "sa_refine", "tokenwise_user", "sa_forward_tokenwise",
+    "sa_refine", "tokenwise_user", "sa_forward_tokenwise", "stca_branch_grads",
 ]
 
 
@@ -265,6 +265,71 @@ def stca_branch_reordered(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: 
             qu = _query_ffn(qu, lay)
         out[c0:c1] = qu
     return out
+
+
+STCA_WEIGHTS = ("W_Q", "W_K", "W_V", "W_O", "hist_W1", "hist_W3", "hist_W2", "q_W1", "q_W3", "q_W2")
+
+
+def stca_branch_grads(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: int, d_h: int, dout):
+    """Gradients of sum(dout * stca_branch(...)) with respect to q, kv and every weight of
+    every layer, by reverse-mode differentiation (torch autograd, fp64, CPU) of the same
+    definition as ``stca_branch`` written with torch operations: per user, the layer's
+    history FFN (if any), the attention of eq. (4) per head, W_O and the residual, the
+    query FFN (if any).  A key row shared by several users' ranges collects the gradient
+    of every use.  Returns {"dq": [C, D], "dkv": [rows, D], "layers": [{name: grad}]}
+    with None for an absent weight."""
+    import torch
+
+    t = lambda a: torch.tensor(_f64(a), dtype=torch.float64)
+    qv = t(q).requires_grad_(True)
+    kvv = t(kv).requires_grad_(True)
+    W = []
+    for lay in layers:
+        W.append({k: (t(getattr(lay, k)).requires_grad_(True) if getattr(lay, k, None) is not None else None)
+                  for k in STCA_WEIGHTS})
+
+    def ffn(x, W1, W3, W2):
+        a = x @ W1
+        return ((a / (1.0 + torch.exp(-a))) * (x @ W3)) @ W2
+
+    cand_offsets = np.asarray(cand_offsets, np.int64)
+    outs = []
+    for u in range(len(cand_offsets) - 1):
+        c0, c1 = int(cand_offsets[u]), int(cand_offsets[u + 1])
+        if c1 == c0:
+            continue
+        Xu = kvv[int(kv_begin[u]):int(kv_end[u])]
+        qu = qv[c0:c1]
+        for w in W:
+            if w["hist_W1"] is not None:
+                Xu = Xu + ffn(Xu, w["hist_W1"], w["hist_W3"], w["hist_W2"])
+            if Xu.shape[0] > 0:
+                o = []
+                for h in range(heads):
+                    s = (qu @ w["W_Q"][h]) @ (Xu @ w["W_K"][h]).T / math.sqrt(d_h)
+                    o.append(torch.softmax(s, dim=1) @ (Xu @ w["W_V"][h]))
+                o = torch.cat(o, dim=1)
+            else:
+                o = torch.zeros(c1 - c0, heads * d_h, dtype=torch.float64)
+            qu = qu + (o if w["W_O"] is None else o @ w["W_O"])
+            if w["q_W1"] is not None:
+                qu = qu + ffn(qu, w["q_W1"], w["q_W3"], w["q_W2"])
+        outs.append((c0, c1, qu))
+    total = sum((o * t(dout)[c0:c1]).sum() for c0, c1, o in outs) if outs else qv.sum() * 0.0
+    leaves = [qv, kvv] + [v for w in W for v in w.values() if v is not None]
+    grads = torch.autograd.grad(total, leaves, allow_unused=True)
+    g = iter(grads)
+    res = {"dq": next(g), "dkv": next(g), "layers": []}
+    for w in W:
+        res["layers"].append({k: (next(g) if v is not None else None) for k, v in w.items()})
+    zero = lambda x, like: torch.zeros_like(like) if x is None else x
+    res["dq"] = zero(res["dq"], qv).numpy()
+    res["dkv"] = zero(res["dkv"], kvv).numpy()
+    for li, w in enumerate(W):
+        for k, v in w.items():
+            if v is not None:
+                res["layers"][li][k] = zero(res["layers"][li][k], v).numpy()
+    return res
 
 
 def stca_fuse(z_r, z_u, W_F, b_F=None):
