@@ -328,6 +328,51 @@ sa_status stca_forward_full(const void* q, sa_dtype dtype,
                             const stca_full_layer* layers, float* out, void* workspace,
                             size_t ws_bytes, sa_stream_t stream);
 
+/* Gradients of one full STCA layer's weights (fp32 device buffers, shaped as the
+ * weights; written, not accumulated).  dW_O is ignored when the layer's W_O is NULL,
+ * and an absent FFN's gradients are ignored. */
+typedef struct {
+  float* dW_Q;
+  float* dW_K;
+  float* dW_V;
+  float* dW_O;
+  float* hist_dW1;
+  float* hist_dW3;
+  float* hist_dW2;
+  float* q_dW1;
+  float* q_dW3;
+  float* q_dW2;
+} stca_full_layer_grad;
+
+/* Workspace of stca_backward_full; the host offsets are those of the call. */
+size_t stca_backward_full_workspace(int B, const int64_t* cand_offsets_host,
+                                    const int64_t* kv_begin_host, const int64_t* kv_end_host,
+                                    int D, int heads, int d_h, int n_layers, sa_dtype dtype);
+
+/*
+ * stca_backward_full -- the backward of stca_forward_full: given dout [C_total, D]
+ * fp32, the gradient of the branch output, writes
+ *   dq   [C_total, D] fp32 (or NULL): the gradient with respect to q;
+ *   dkv  [kv_rows, D] fp32 (or NULL): the gradient with respect to kv (a row in no
+ *        user's range gets 0; a row in several ranges sums their gradients);
+ *   grads[l]: every weight gradient of layer l.
+ * Inputs as stca_forward_full.  The layers are recomputed in fp32 (bf16 inputs are
+ * widened, not rounded further) and each user's attention is evaluated with its
+ * C_u*heads x L_u score matrix in the workspace, so the workspace grows with the
+ * largest user.  Deterministic: users are processed in order.
+ * Errors: as stca_forward_full, and SA_ERR_INVALID_ARG for a NULL gradient buffer
+ * of a weight that is present.
+ */
+sa_status stca_backward_full(const void* q, sa_dtype dtype,
+                             const int64_t* cand_offsets_host, const int64_t* cand_offsets_dev,
+                             int B, const void* kv, int64_t kv_rows,
+                             const int64_t* kv_begin_host, const int64_t* kv_end_host,
+                             const int64_t* kv_begin_dev, const int64_t* kv_end_dev,
+                             int D, int heads, int d_h, int n_layers,
+                             const stca_full_layer* layers, const float* dout, float* dq,
+                             float* dkv, const stca_full_layer_grad* grads, void* workspace,
+                             size_t ws_bytes, sa_stream_t stream);
+
 /*
  * stca_fuse -- linear fusion of the two branches (paper Sec. 3.4 leaves the
  * fusion to a light MLP or gate; this library applies one linear layer):

@@ -30,7 +30,8 @@ EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_w
            "stca_forward", "stca_fuse", "sa_launch_count", "sa_profile", "sa_profile_read",
            "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward",
            "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate",
-           "stca_forward_full_workspace", "stca_forward_full")
+           "stca_forward_full_workspace", "stca_forward_full", "stca_backward_full_workspace",
+           "stca_backward_full")
 
 
 class SAError(RuntimeError):
@@ -49,6 +50,13 @@ STCA_FFN_KEYS = ("hist_W1", "hist_W3", "hist_W2", "q_W1", "q_W3", "q_W2")
 
 class StcaFullLayerC(ctypes.Structure):
     _fields_ = [("attn", StcaLayerC)] + [(k, ctypes.c_void_p) for k in STCA_FFN_KEYS]
+
+
+STCA_GRAD_KEYS = ("dW_Q", "dW_K", "dW_V", "dW_O", "hist_dW1", "hist_dW3", "hist_dW2", "q_dW1", "q_dW3", "q_dW2")
+
+
+class StcaFullLayerGradC(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in STCA_GRAD_KEYS]
 
 
 class RefineLayerC(ctypes.Structure):
@@ -96,6 +104,12 @@ def load(path: Optional[str] = None):
     lib.stca_forward_full.restype = _i
     lib.stca_forward_full.argtypes = [_vp, _i, _vp, _vp, _i, _vp, _i64, _vp, _vp, _vp, _vp,
                                       _i, _i, _i, _i, ctypes.POINTER(StcaFullLayerC), _vp, _vp, _sz, _vp]
+    lib.stca_backward_full_workspace.restype = _sz
+    lib.stca_backward_full_workspace.argtypes = [_i, _vp, _vp, _vp, _i, _i, _i, _i, _i]
+    lib.stca_backward_full.restype = _i
+    lib.stca_backward_full.argtypes = [_vp, _i, _vp, _vp, _i, _vp, _i64, _vp, _vp, _vp, _vp,
+                                       _i, _i, _i, _i, ctypes.POINTER(StcaFullLayerC), _vp, _vp, _vp,
+                                       ctypes.POINTER(StcaFullLayerGradC), _vp, _sz, _vp]
     lib.stca_fuse.restype = _i
     lib.stca_fuse.argtypes = [_vp, _vp, _vp, _vp, _i64, _i, _vp, _vp]
     lib.sa_forward_noalloc.restype = _i
@@ -397,6 +411,78 @@ def stca_forward_full(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin,
                                _p(workspace), workspace.numel(), _stream(stream))
     _check("stca_forward_full", st)
     return res
+
+
+def _full_layers_c(layers):
+    arr = (StcaFullLayerC * len(layers))()
+    for i, L in enumerate(layers):
+        _need_cuda(L["W_Q"], L["W_K"], L["W_V"], L.get("W_O"), *(L.get(k) for k in STCA_FFN_KEYS))
+        arr[i].attn.W_Q = L["W_Q"].data_ptr()
+        arr[i].attn.W_K = L["W_K"].data_ptr()
+        arr[i].attn.W_V = L["W_V"].data_ptr()
+        arr[i].attn.W_O = L["W_O"].data_ptr() if L.get("W_O") is not None else None
+        for k in STCA_FFN_KEYS:
+            setattr(arr[i], k, L[k].data_ptr() if L.get(k) is not None else None)
+    return arr
+
+
+def stca_backward_full_workspace(cand_offsets, kv_begin, kv_end, D: int, heads: int, d_h: int,
+                                 n_layers: int, dtype: int) -> int:
+    cand, kb, ke = _host_i64(cand_offsets), _host_i64(kv_begin), _host_i64(kv_end)
+    return int(load().stca_backward_full_workspace(len(cand) - 1, _hp(cand), _hp(kb), _hp(ke), D, heads, d_h,
+                                                   n_layers, dtype))
+
+
+def stca_backward_full(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin, kv_end,
+                       layers: Sequence[dict], heads: int, d_h: int, dout: torch.Tensor, *,
+                       cand_offsets_dev=None, kv_begin_dev=None, kv_end_dev=None,
+                       out: Optional[dict] = None, workspace: Optional[torch.Tensor] = None,
+                       stream=None) -> dict:
+    """Backward of stca_forward_full.  ``dout`` [C_total, D] fp32.  Returns {"dq": [C, D],
+    "dkv": [kv_rows, D], "layers": [dict of weight gradients per layer]} (fp32; the
+    gradient keys are dW_Q, dW_K, dW_V, dW_O and hist_dW1.. / q_dW1.. for the FFNs that
+    the layer has).  ``out`` may supply any of these buffers."""
+    lib = load()
+    _need_cuda(q, kv, dout)
+    dt = _dtype_code(q)
+    if kv.dtype != q.dtype:
+        raise TypeError("q and kv must have the same dtype")
+    cand = _host_i64(cand_offsets)
+    kb, ke = _host_i64(kv_begin), _host_i64(kv_end)
+    B = len(cand) - 1
+    D = q.shape[1]
+    dev = q.device
+    C = int(cand[-1])
+    out = dict(out or {})
+    dq = out.get("dq") if out.get("dq") is not None else torch.empty(C, D, device=dev)
+    dkv = out.get("dkv") if out.get("dkv") is not None else torch.empty(kv.shape[0], D, device=dev)
+    lg_out = out.get("layers") or [{} for _ in layers]
+    grads = []
+    garr = (StcaFullLayerGradC * len(layers))()
+    for i, L in enumerate(layers):
+        g = {}
+        have = {"dW_Q": "W_Q", "dW_K": "W_K", "dW_V": "W_V", "dW_O": "W_O", "hist_dW1": "hist_W1",
+                "hist_dW3": "hist_W3", "hist_dW2": "hist_W2", "q_dW1": "q_W1", "q_dW3": "q_W3", "q_dW2": "q_W2"}
+        for gk, wk in have.items():
+            if L.get(wk) is None:
+                continue
+            buf = lg_out[i].get(gk) if lg_out[i].get(gk) is not None else torch.empty_like(L[wk])
+            _need_cuda(buf)
+            g[gk] = buf
+            setattr(garr[i], gk, buf.data_ptr())
+        grads.append(g)
+    arr = _full_layers_c(layers)
+    ws_bytes = lib.stca_backward_full_workspace(B, _hp(cand), _hp(kb), _hp(ke), D, heads, d_h, len(layers), dt)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    cd = _dev_i64(cand, dev, cand_offsets_dev)
+    kbd = _dev_i64(kb, dev, kv_begin_dev)
+    ked = _dev_i64(ke, dev, kv_end_dev)
+    st = lib.stca_backward_full(_p(q), dt, _hp(cand), _p(cd), B, _p(kv), kv.shape[0], _hp(kb), _hp(ke),
+                                _p(kbd), _p(ked), D, heads, d_h, len(layers), arr, _p(dout), _p(dq), _p(dkv),
+                                garr, _p(workspace), workspace.numel(), _stream(stream))
+    _check("stca_backward_full", st)
+    return {"dq": dq, "dkv": dkv, "layers": grads}
 
 
 REFINE_KEYS = ("W_Q", "W_K", "ln1_g", "ln1_b", "W1", "W3", "W2", "ln2_g", "ln2_b")

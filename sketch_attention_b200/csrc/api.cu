@@ -512,7 +512,7 @@ sa_status stca_check(const void* q, sa_dtype dtype, const int64_t* cand_offsets_
                      const int64_t* kv_begin_host, const int64_t* kv_end_host,
                      const int64_t* kv_begin_dev, const int64_t* kv_end_dev, int D, int heads,
                      int d_h, int n_layers, const stca_layer* const* attn, float* out, StcaArgs* a,
-                     int* max_tiles, int64_t* kv_total) {
+                     int* max_tiles, int64_t* kv_total, bool out_optional = false) {
   if (B < 1) return fail(SA_ERR_INVALID_ARG, "B must be >= 1");
   if (dtype != SA_F32 && dtype != SA_BF16) return fail(SA_ERR_INVALID_ARG, "unknown dtype");
   if (D != 128) return fail(SA_ERR_UNSUPPORTED, "D must be 128");
@@ -535,7 +535,7 @@ sa_status stca_check(const void* q, sa_dtype dtype, const int64_t* cand_offsets_
   SA_TRY(check_ptr(cand_offsets_dev, "cand_offsets_dev"));
   SA_TRY(check_ptr(kv_begin_dev, "kv_begin_dev"));
   SA_TRY(check_ptr(kv_end_dev, "kv_end_dev"));
-  SA_TRY(check_ptr(out, "out", C == 0));
+  SA_TRY(check_ptr(out, "out", C == 0 || out_optional));
   for (int l = 0; l < n_layers; ++l) {
     const stca_layer& L = *attn[l];
     SA_TRY(check_ptr(L.W_Q, "layers[].W_Q"));
@@ -626,6 +626,85 @@ sa_status stca_forward_full(const void* q, sa_dtype dtype, const int64_t* cand_o
   stca_full_layout(workspace, B, C, kv_total, D, heads, d_h, dtype, &w);
   w.attn.max_tiles = max_tiles;
   return stca_full_run(a, layers, kv_total, w, (cudaStream_t)stream);
+}
+
+}  // extern "C"
+
+namespace {
+// Shape of a backward call from its host offsets (no validation beyond sizes).
+StcaBwdShape bwd_shape(int B, const int64_t* cand, const int64_t* kb, const int64_t* ke, int D, int heads,
+                       int d_h, int n_layers) {
+  StcaBwdShape sh{};
+  sh.C = cand[B];
+  for (int u = 0; u < B; ++u) {
+    sh.kv_total += ke[u] - kb[u];
+    sh.max_rows_x_keys = std::max(sh.max_rows_x_keys, (cand[u + 1] - cand[u]) * heads * (ke[u] - kb[u]));
+  }
+  sh.D = D; sh.heads = heads; sh.d_h = d_h; sh.n_layers = n_layers;
+  return sh;
+}
+}  // namespace
+
+extern "C" {
+
+size_t stca_backward_full_workspace(int B, const int64_t* cand_offsets_host, const int64_t* kv_begin_host,
+                                    const int64_t* kv_end_host, int D, int heads, int d_h, int n_layers,
+                                    sa_dtype dtype) {
+  if (B < 1 || !cand_offsets_host || !kv_begin_host || !kv_end_host || D < 1 || heads < 1 || d_h < 1 ||
+      n_layers < 1 || (dtype != SA_F32 && dtype != SA_BF16))
+    return 0;
+  for (int u = 0; u < B; ++u)
+    if (kv_end_host[u] < kv_begin_host[u] || cand_offsets_host[u + 1] < cand_offsets_host[u]) return 0;
+  return stca_bwd_layout(nullptr, bwd_shape(B, cand_offsets_host, kv_begin_host, kv_end_host, D, heads, d_h,
+                                            n_layers), nullptr);
+}
+
+sa_status stca_backward_full(const void* q, sa_dtype dtype, const int64_t* cand_offsets_host,
+                             const int64_t* cand_offsets_dev, int B, const void* kv, int64_t kv_rows,
+                             const int64_t* kv_begin_host, const int64_t* kv_end_host,
+                             const int64_t* kv_begin_dev, const int64_t* kv_end_dev, int D, int heads,
+                             int d_h, int n_layers, const stca_full_layer* layers, const float* dout,
+                             float* dq, float* dkv, const stca_full_layer_grad* grads, void* workspace,
+                             size_t ws_bytes, sa_stream_t stream) {
+  if (n_layers < 1 || !layers) return fail(SA_ERR_INVALID_ARG, "need n_layers >= 1 and layers");
+  if (!grads) return fail(SA_ERR_INVALID_ARG, "grads is NULL");
+  std::vector<const stca_layer*> attn(n_layers);
+  for (int l = 0; l < n_layers; ++l) {
+    const stca_full_layer& L = layers[l];
+    const stca_full_layer_grad& G = grads[l];
+    attn[l] = &L.attn;
+    const int nh = !!L.hist_W1 + !!L.hist_W3 + !!L.hist_W2, nq = !!L.q_W1 + !!L.q_W3 + !!L.q_W2;
+    if ((nh != 0 && nh != 3) || (nq != 0 && nq != 3))
+      return fail(SA_ERR_INVALID_ARG, "layer " + std::to_string(l) + ": an FFN is partly given");
+    const float* need[] = {G.dW_Q, G.dW_K, G.dW_V};
+    for (const float* g : need) SA_TRY(check_ptr(g, "grads[] attention weight gradient"));
+    if (L.attn.W_O) SA_TRY(check_ptr(G.dW_O, "grads[].dW_O"));
+    if (nh) for (const float* g : {G.hist_dW1, G.hist_dW3, G.hist_dW2}) SA_TRY(check_ptr(g, "grads[] history FFN gradient"));
+    if (nq) for (const float* g : {G.q_dW1, G.q_dW3, G.q_dW2}) SA_TRY(check_ptr(g, "grads[] query FFN gradient"));
+  }
+  StcaArgs a;
+  int max_tiles = 0;
+  int64_t kv_total = 0;
+  SA_TRY(stca_check(q, dtype, cand_offsets_host, cand_offsets_dev, B, kv, kv_rows, kv_begin_host,
+                    kv_end_host, kv_begin_dev, kv_end_dev, D, heads, d_h, n_layers, attn.data(), nullptr,
+                    &a, &max_tiles, &kv_total, true));
+  const int64_t C = cand_offsets_host[B];
+  SA_TRY(check_ptr(dout, "dout", C == 0));
+  SA_TRY(check_ptr(dq, "dq", true));
+  SA_TRY(check_ptr(dkv, "dkv", true));
+  const StcaBwdShape sh = bwd_shape(B, cand_offsets_host, kv_begin_host, kv_end_host, D, heads, d_h, n_layers);
+  if (sh.max_rows_x_keys >= (1LL << 31) || sh.kv_total >= (1LL << 31) || C * heads >= (1LL << 31))
+    return fail(SA_ERR_UNSUPPORTED, "a user's score matrix or the row counts must be < 2^31 elements");
+  const size_t need = stca_bwd_layout(nullptr, sh, nullptr);
+  if (!workspace || ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "workspace needs " + std::to_string(need) + " bytes");
+  SA_TRY(check_ptr(workspace, "workspace"));
+  StcaBwdWork w;
+  stca_bwd_layout(workspace, sh, &w);
+  std::vector<int64_t> kpre(B + 1, 0);
+  for (int u = 0; u < B; ++u) kpre[u + 1] = kpre[u] + (kv_end_host[u] - kv_begin_host[u]);
+  StcaBwdHost hst{cand_offsets_host, kv_begin_host, kv_end_host, kpre.data(), kv_total};
+  return stca_backward_run(a, hst, layers, grads, dout, dq, dkv, w, (cudaStream_t)stream);
 }
 
 sa_status stca_fuse(const float* z_r, const float* z_u, const float* W_F, const float* b_F,

@@ -46,6 +46,30 @@ size_t stca_full_layout(void* base, int B, int64_t C, int64_t kv_total, int D, i
 sa_status stca_full_run(const StcaArgs& a, const stca_full_layer* layers, int64_t kv_total,
                         const StcaFullWork& w, cudaStream_t st);
 
+// Backward of a branch of full layers (fp32, GEMM-based).
+struct StcaBwdShape {
+  int64_t C, kv_total, max_rows_x_keys;   // max over users of C_u * heads * (kv_end - kv_begin)
+  int D, heads, d_h, n_layers;
+};
+struct StcaBwdHost {                      // host copies of the offsets, read while issuing
+  const int64_t* cand;                    // [B+1]
+  const int64_t* kv_begin;                // [B]
+  const int64_t* kv_end;                  // [B]
+  const int64_t* kpre;                    // [B+1] start of each user's rows among the gathered rows
+  int64_t kv_total;
+};
+struct StcaBwdWork {
+  float *qin, *qmid, *Qh, *U, *Y, *O;     // per layer (qin: n_layers + 1 states)
+  float* Xk;                              // [n_layers + 1, kv_total, D] key-row states
+  float *G1, *G3, *Uf, *dUf;              // [max(C, kv_total), 2D]
+  float *S, *dS;                          // one user's score matrix and its gradient
+  float *dq, *dqmid, *dO, *dY, *dU, *dQh, *dX;
+};
+size_t stca_bwd_layout(void* base, const StcaBwdShape& sh, StcaBwdWork* w);
+sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stca_full_layer* layers,
+                            const stca_full_layer_grad* grads, const float* dout, float* dq_out, float* dkv,
+                            const StcaBwdWork& w, cudaStream_t st);
+
 // x <- x + (SiLU(x W1) * (x W3)) W2 for rows of bf16 x, D = 128, in place, on
 // the tensor cores; W13t / W2t as prepared by stca_ffn_weights_bf16.
 sa_status stca_ffn_weights_bf16(const float* W1, const float* W3, const float* W2,
