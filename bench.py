@@ -640,6 +640,50 @@ def run_component(args, rank, world, device):
         # the history FFN: 12 D^2 flop per key row (eq. (27) with inner width 2D), once per row;
         # per launch the mean of the two branches' row counts
         extra.append(("stca_hist_ffn_tc_kernel", 12.0 * 128 * 128 * 0.5 * (rows_r + rows_s)))
+    elif args.workload == "stca_bwd":
+        from sa_inputs import add_stca_ffns, rng_for
+        w = stca_workload(users=args.users or 16)
+        add_stca_ffns(rng_for(5006), w.layers_r, 128)
+        add_stca_ffns(rng_for(5007), w.layers_u, 128)
+        q, kvr, kvs = (_dev_bf16(a, device) for a in (w.recent.q, w.recent.kv, w.sketch.kv))
+        wkeys = ("W_Q", "W_K", "W_V", "W_O", "hist_W1", "hist_W3", "hist_W2", "q_W1", "q_W3", "q_W2")
+        lay = lambda L: {k: _f32(getattr(L, k), device) for k in wkeys}
+        lr, lu = [lay(L) for L in w.layers_r], [lay(L) for L in w.layers_u]
+        C = int(w.recent.cand_offsets[-1])
+        gen = torch.Generator(device="cpu").manual_seed(5008)
+        dzr, dzu = (torch.randn(C, 128, generator=gen).to(device) for _ in range(2))
+        dv = lambda a: torch.from_numpy(np.asarray(a, np.int64)).to(device)
+        cd, rbd, red, sbd, sed = (dv(a) for a in (w.recent.cand_offsets, w.recent.kv_begin, w.recent.kv_end,
+                                                  w.sketch.kv_begin, w.sketch.kv_end))
+        nlay = len(lr)
+        ws_r = torch.empty(sab.stca_backward_full_workspace(w.recent.cand_offsets, w.recent.kv_begin,
+                                                            w.recent.kv_end, 128, w.heads, w.d_h, nlay, sab.SA_BF16),
+                           dtype=torch.uint8, device=device)
+        ws_s = torch.empty(sab.stca_backward_full_workspace(w.sketch.cand_offsets, w.sketch.kv_begin,
+                                                            w.sketch.kv_end, 128, w.heads, w.d_h, nlay, sab.SA_BF16),
+                           dtype=torch.uint8, device=device)
+        gr = sab.stca_backward_full(q, w.recent.cand_offsets, kvr, w.recent.kv_begin, w.recent.kv_end, lr, w.heads,
+                                    w.d_h, dzr, cand_offsets_dev=cd, kv_begin_dev=rbd, kv_end_dev=red, workspace=ws_r)
+        gs = sab.stca_backward_full(q, w.sketch.cand_offsets, kvs, w.sketch.kv_begin, w.sketch.kv_end, lu, w.heads,
+                                    w.d_h, dzu, cand_offsets_dev=cd, kv_begin_dev=sbd, kv_end_dev=sed, workspace=ws_s)
+
+        def step():
+            sab.stca_backward_full(q, w.recent.cand_offsets, kvr, w.recent.kv_begin, w.recent.kv_end, lr, w.heads,
+                                   w.d_h, dzr, cand_offsets_dev=cd, kv_begin_dev=rbd, kv_end_dev=red, out=gr,
+                                   workspace=ws_r)
+            sab.stca_backward_full(q, w.sketch.cand_offsets, kvs, w.sketch.kv_begin, w.sketch.kv_end, lu, w.heads,
+                                   w.d_h, dzu, cand_offsets_dev=cd, kv_begin_dev=sbd, kv_end_dev=sed, out=gs,
+                                   workspace=ws_s)
+        units, unit = C, "candidates/s"
+        name = ("backward of full STCA layers (both FFNs, both branches), " + STCA_WORKLOAD_4)
+        # the per-user attention GEMMs: S and Y in the recompute, S, dP, dU and the two dX
+        # products in the backward, 14 R_u L_u D flop per user and layer (fp32, CUDA cores)
+        rows_x_keys = sum(float(w.recent.cand_offsets[u + 1] - w.recent.cand_offsets[u]) * w.heads *
+                          float(w.recent.kv_end[u] - w.recent.kv_begin[u]) +
+                          float(w.sketch.cand_offsets[u + 1] - w.sketch.cand_offsets[u]) * w.heads *
+                          float(w.sketch.kv_end[u] - w.sketch.kv_begin[u])
+                          for u in range(len(w.recent.cand_offsets) - 1))
+        kname, attn_flops_step = "gemm:stca_bwd_attn", 14.0 * rows_x_keys * 128 * nlay
     else:
         w = stca_workload(users=args.users or 16)
         q, kvr, kvs = (_dev_bf16(a, device) for a in (w.recent.q, w.recent.kv, w.sketch.kv))
@@ -673,11 +717,21 @@ def run_component(args, rank, world, device):
     prof = sab.profile_read()
     sab.profile(False)
     ms = start.elapsed_time(end) / args.steps
+    if args.workload == "stca_bwd":
+        # flops per launch of the dominant (fp32 GEMM) call site: the step's total over its launches
+        flops = attn_flops_step / max(prof.get(kname, (0, 1))[1] / args.steps, 1)
+
     def roof_of(kn, fl):
         if kn not in prof:
             return None
         tot, cnt = prof[kn]
         ach = fl / (tot / cnt / 1e3) / 1e12
+        if args.workload == "stca_bwd":
+            pk = 148 * 128 * 2 * 1965e6 / 1e12
+            return {"kernel": kn, "bound": "alu", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
+                    "frac": ach / pk, "traffic": None,
+                    "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz (unit counts, max clock)",
+                    "avg_launch_ms": tot / cnt}
         pk = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
         return {"kernel": kn, "bound": "tensor", "achieved": ach, "peak": pk, "unit": "TFLOP/s",
                 "frac": ach / pk, "traffic": None,
@@ -687,7 +741,7 @@ def run_component(args, rank, world, device):
     extra_roofs = {kn: roof_of(kn, fl) for kn, fl in extra}
     line = {"metric": unit, "value": world * units / (ms / 1e3), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32" if args.workload == "stca_bwd" else "bf16",
             "data": "synthetic", "config": {"workload": name},
             "roofline": roof,
             "kernels": {n: {"ms_per_step": v[0] / args.steps, "launches_per_step": v[1] / args.steps}
@@ -706,11 +760,13 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "stca_full", "refine", "tokenwise"],
+    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "stca_full", "stca_bwd", "refine",
+                                           "tokenwise"],
                     default="train",
                     help="train: the full step (default, the headline); sa_fwd: SA forward over "
                          "32 users x 100K (k=1024); stca: STCA of 16 users x 512 candidates; "
                          "stca_full: the same with full layers (history- and query-side FFNs); "
+                         "stca_bwd: the backward of those full layers; "
                          "refine: stacked SA refinement, 2 iterations, on the train step's users; "
                          "tokenwise: the token-wise normalisation variant on the train step's users")
     ap.add_argument("--users", type=int, default=None, help="shrink the batch (profiling)")

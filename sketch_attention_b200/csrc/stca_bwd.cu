@@ -102,7 +102,27 @@ unsigned grid_for(int64_t n) { return (unsigned)std::max<int64_t>(1, std::min<in
 bool has_hist(const stca_full_layer& L) { return L.hist_W1 != nullptr; }
 bool has_query(const stca_full_layer& L) { return L.q_W1 != nullptr; }
 
-sa_status mm(Gemm g, cudaStream_t st) { return gemm(g, st); }
+// The stream and the split-K partials shared by every GEMM of one call (they run
+// in stream order).
+struct Ctx {
+  cudaStream_t st;
+  float* split;
+};
+
+// GEMM with split-K when its output tiles alone leave most SMs idle (the weight
+// gradients and the per-user P X, dS X products have small outputs and long K)
+sa_status mm(Gemm g, const Ctx& cx) {
+  if (g.M > 0 && g.N > 0) {
+    const int64_t out = (int64_t)g.M * g.N * g.batch;
+    int split = gemm_split_for(g.M, g.N * g.batch, g.K, kMaxSplit);
+    split = (int)std::min<int64_t>(split, (int64_t)(kStcaBwdSplitFloats / (size_t)std::max<int64_t>(out, 1)));
+    if (split > 1) {
+      g.split_k = split;
+      g.split_ws = cx.split;
+    }
+  }
+  return gemm(g, cx.st);
+}
 
 // C = alpha A B (+ Cin) for plain row-major operands
 Gemm plain(int M, int N, int K, const float* A, int64_t lda, bool ta, const float* B, int64_t ldb, bool tb,
@@ -122,45 +142,47 @@ struct Ffn {
 
 // y = x + FFN(x) over `rows` rows
 sa_status ffn_fwd(const float* x, int64_t rows, int D, const Ffn& f, float* G1, float* G3, float* U, float* y,
-                  cudaStream_t st) {
+                  const Ctx& cx) {
+  cudaStream_t st = cx.st;
   if (rows == 0) return SA_OK;
   sa_status s;
-  if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W1, 2 * D, false, G1, 2 * D, "gemm:stca_bwd_ffn"), st)) != SA_OK) return s;
-  if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W3, 2 * D, false, G3, 2 * D, "gemm:stca_bwd_ffn"), st)) != SA_OK) return s;
+  if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W1, 2 * D, false, G1, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
+  if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W3, 2 * D, false, G3, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
   if ((s = sa_swiglu(G1, G3, rows * 2 * D, U, st)) != SA_OK) return s;
   Gemm g = plain((int)rows, D, 2 * D, U, 2 * D, false, f.W2, D, false, y, D, "gemm:stca_bwd_ffn");
   g.Cin = x; g.ldcin = D;
-  return mm(g, st);
+  return mm(g, cx);
 }
 
 // given dy (the gradient of y = x + FFN(x)), dx = dy + dG1 W1^T + dG3 W3^T and the
 // weight gradients; dx may alias dy
 sa_status ffn_bwd(const float* x, int64_t rows, int D, const Ffn& f, const float* dy, float* dx, float* G1,
-                  float* G3, float* U, float* dU, cudaStream_t st) {
+                  float* G3, float* U, float* dU, const Ctx& cx) {
+  cudaStream_t st = cx.st;
   sa_status s;
   if (rows == 0) {
     for (float* w : {f.dW1, f.dW3, f.dW2})
       SA_CUDA(cudaMemsetAsync(w, 0, sizeof(float) * 2 * D * D, st));
     return SA_OK;
   }
-  if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W1, 2 * D, false, G1, 2 * D, "gemm:stca_bwd_ffn"), st)) != SA_OK) return s;
-  if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W3, 2 * D, false, G3, 2 * D, "gemm:stca_bwd_ffn"), st)) != SA_OK) return s;
+  if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W1, 2 * D, false, G1, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
+  if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W3, 2 * D, false, G3, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
   if ((s = sa_swiglu(G1, G3, rows * 2 * D, U, st)) != SA_OK) return s;
   // dW2 = U^T dy;  dU = dy W2^T
-  if ((s = mm(plain(2 * D, D, (int)rows, U, 2 * D, true, dy, D, false, f.dW2, D, "gemm:stca_bwd_ffn"), st)) != SA_OK) return s;
-  if ((s = mm(plain((int)rows, 2 * D, D, dy, D, false, f.W2, D, true, dU, 2 * D, "gemm:stca_bwd_ffn"), st)) != SA_OK) return s;
+  if ((s = mm(plain(2 * D, D, (int)rows, U, 2 * D, true, dy, D, false, f.dW2, D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
+  if ((s = mm(plain((int)rows, 2 * D, D, dy, D, false, f.W2, D, true, dU, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
   // dG1 over U (no longer needed), dG3 over G1 (each element read before it is written)
   SA_TIMED("swiglu_bwd_kernel", st,
            (swiglu_bwd_kernel<<<grid_for(rows * 2 * D), 256, 0, st>>>(G1, G3, dU, rows * 2 * D, U, G1)));
   // now U = dG1, G1 = dG3
-  if ((s = mm(plain(D, 2 * D, (int)rows, x, D, true, U, 2 * D, false, f.dW1, 2 * D, "gemm:stca_bwd_ffn"), st)) != SA_OK) return s;
-  if ((s = mm(plain(D, 2 * D, (int)rows, x, D, true, G1, 2 * D, false, f.dW3, 2 * D, "gemm:stca_bwd_ffn"), st)) != SA_OK) return s;
+  if ((s = mm(plain(D, 2 * D, (int)rows, x, D, true, U, 2 * D, false, f.dW1, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
+  if ((s = mm(plain(D, 2 * D, (int)rows, x, D, true, G1, 2 * D, false, f.dW3, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
   Gemm g1 = plain((int)rows, D, 2 * D, U, 2 * D, false, f.W1, 2 * D, true, dx, D, "gemm:stca_bwd_ffn");
   g1.Cin = dy; g1.ldcin = D;
-  if ((s = mm(g1, st)) != SA_OK) return s;
+  if ((s = mm(g1, cx)) != SA_OK) return s;
   Gemm g3 = plain((int)rows, D, 2 * D, G1, 2 * D, false, f.W3, 2 * D, true, dx, D, "gemm:stca_bwd_ffn");
   g3.Cin = dx; g3.ldcin = D;
-  return mm(g3, st);
+  return mm(g3, cx);
 }
 }  // namespace
 
@@ -191,6 +213,7 @@ size_t stca_bwd_layout(void* base, const StcaBwdShape& sh, StcaBwdWork* w) {
   v.dU = c.take<float>(C * H * D);
   v.dQh = c.take<float>(C * HD);
   v.dX = c.take<float>(R * D);
+  v.gsplit = c.take<float>(kStcaBwdSplitFloats);
   if (w) *w = v;
   return c.bytes();
 }
@@ -203,6 +226,7 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
   const size_t CD = (size_t)C * D, CHD = (size_t)C * HD, CHD2 = (size_t)C * H * D, RD = (size_t)R * D;
   const float inv_sqrt = 1.f / std::sqrt((float)dh);
   sa_status s;
+  const Ctx cx{st, w.gsplit};
   // ---------------------------------------------------------------- inputs, widened
   if (C > 0) {
     if (a.dtype == SA_BF16)
@@ -235,7 +259,7 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
     float* O = w.O + (size_t)l * CHD;
     if (has_hist(L)) {
       Ffn f{L.hist_W1, L.hist_W3, L.hist_W2, nullptr, nullptr, nullptr};
-      if ((s = ffn_fwd(Xs(l), R, D, f, w.G1, w.G3, w.Uf, Xs(l + 1), st)) != SA_OK) return s;
+      if ((s = ffn_fwd(Xs(l), R, D, f, w.G1, w.G3, w.Uf, Xs(l + 1), cx)) != SA_OK) return s;
     } else if (R > 0) {
       SA_CUDA(cudaMemcpyAsync(Xs(l + 1), Xs(l), sizeof(float) * RD, cudaMemcpyDeviceToDevice, st));
     }
@@ -244,10 +268,10 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
     // Qh[:, h] = q W_Q^h;  U[c*H + h] = Qh[:, h] W_K^h^T / sqrt(d_h)
     Gemm g1 = plain((int)C, dh, D, qin, D, false, L.attn.W_Q, dh, false, Qh, HD, "gemm:stca_bwd_proj");
     g1.batch = H; g1.sB = (int64_t)D * dh; g1.sC = dh;
-    if ((s = mm(g1, st)) != SA_OK) return s;
+    if ((s = mm(g1, cx)) != SA_OK) return s;
     Gemm g2 = plain((int)C, D, dh, Qh, HD, false, L.attn.W_K, dh, true, U, (int64_t)H * D, "gemm:stca_bwd_proj");
     g2.batch = H; g2.sA = dh; g2.sB = (int64_t)D * dh; g2.sC = D; g2.alpha = inv_sqrt;
-    if ((s = mm(g2, st)) != SA_OK) return s;
+    if ((s = mm(g2, cx)) != SA_OK) return s;
     // per user: S = U_u X_u^T, P = softmax, Y_u = P X_u
     for (int u = 0; u < B; ++u) {
       const int64_t r0 = hst.cand[u] * H, ru = (hst.cand[u + 1] - hst.cand[u]) * H;
@@ -259,18 +283,18 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
         continue;
       }
       const float* Xu = X + (size_t)hst.kpre[u] * D;
-      if ((s = mm(plain((int)ru, (int)lu, D, U + (size_t)r0 * D, D, false, Xu, D, true, w.S, lu, "gemm:stca_bwd_attn"), st)) != SA_OK) return s;
+      if ((s = mm(plain((int)ru, (int)lu, D, U + (size_t)r0 * D, D, false, Xu, D, true, w.S, lu, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
       SA_TIMED("softmax_rows_kernel", st, (softmax_rows_kernel<<<(unsigned)ru, 256, 0, st>>>(w.S, lu)));
-      if ((s = mm(plain((int)ru, D, (int)lu, w.S, lu, false, Xu, D, false, Yu, D, "gemm:stca_bwd_attn"), st)) != SA_OK) return s;
+      if ((s = mm(plain((int)ru, D, (int)lu, w.S, lu, false, Xu, D, false, Yu, D, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
     }
     // O[:, h] = Y_h W_V^h;  qmid = q + O W_O (or q + O)
     Gemm g3 = plain((int)C, dh, D, Y, (int64_t)H * D, false, L.attn.W_V, dh, false, O, HD, "gemm:stca_bwd_proj");
     g3.batch = H; g3.sA = D; g3.sB = (int64_t)D * dh; g3.sC = dh;
-    if ((s = mm(g3, st)) != SA_OK) return s;
+    if ((s = mm(g3, cx)) != SA_OK) return s;
     if (L.attn.W_O) {
       Gemm g4 = plain((int)C, D, HD, O, HD, false, L.attn.W_O, D, false, qmid, D, "gemm:stca_bwd_proj");
       g4.Cin = qin; g4.ldcin = D;
-      if ((s = mm(g4, st)) != SA_OK) return s;
+      if ((s = mm(g4, cx)) != SA_OK) return s;
     } else {
       SA_CUDA(cudaMemcpyAsync(qmid, qin, sizeof(float) * CD, cudaMemcpyDeviceToDevice, st));
       SA_TIMED("add_rows_kernel", st, (add_rows_kernel<<<grid_for(CD), 256, 0, st>>>(O, CD, qmid)));
@@ -278,7 +302,7 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
     float* qout = w.qin + (size_t)(l + 1) * CD;
     if (has_query(L)) {
       Ffn f{L.q_W1, L.q_W3, L.q_W2, nullptr, nullptr, nullptr};
-      if ((s = ffn_fwd(qmid, C, D, f, w.G1, w.G3, w.Uf, qout, st)) != SA_OK) return s;
+      if ((s = ffn_fwd(qmid, C, D, f, w.G1, w.G3, w.Uf, qout, cx)) != SA_OK) return s;
     } else {
       SA_CUDA(cudaMemcpyAsync(qout, qmid, sizeof(float) * CD, cudaMemcpyDeviceToDevice, st));
     }
@@ -299,16 +323,16 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
     // query FFN: dqmid = dq + FFN_q backward
     if (has_query(L)) {
       Ffn f{L.q_W1, L.q_W3, L.q_W2, Gd.q_dW1, Gd.q_dW3, Gd.q_dW2};
-      if ((s = ffn_bwd(qmid, C, D, f, w.dq, w.dqmid, w.G1, w.G3, w.Uf, w.dUf, st)) != SA_OK) return s;
+      if ((s = ffn_bwd(qmid, C, D, f, w.dq, w.dqmid, w.G1, w.G3, w.Uf, w.dUf, cx)) != SA_OK) return s;
     } else if (C > 0) {
       SA_CUDA(cudaMemcpyAsync(w.dqmid, w.dq, sizeof(float) * CD, cudaMemcpyDeviceToDevice, st));
     }
     // W_O: dO = dqmid W_O^T, dW_O = O^T dqmid; the residual passes dqmid to q
     if (L.attn.W_O) {
-      if ((s = mm(plain((int)C, HD, D, w.dqmid, D, false, L.attn.W_O, D, true, w.dO, HD, "gemm:stca_bwd_proj"), st)) != SA_OK) return s;
+      if ((s = mm(plain((int)C, HD, D, w.dqmid, D, false, L.attn.W_O, D, true, w.dO, HD, "gemm:stca_bwd_proj"), cx)) != SA_OK) return s;
       if (Gd.dW_O) {
         if (C > 0) {
-          if ((s = mm(plain(HD, D, (int)C, O, HD, true, w.dqmid, D, false, Gd.dW_O, D, "gemm:stca_bwd_proj"), st)) != SA_OK) return s;
+          if ((s = mm(plain(HD, D, (int)C, O, HD, true, w.dqmid, D, false, Gd.dW_O, D, "gemm:stca_bwd_proj"), cx)) != SA_OK) return s;
         } else {
           SA_CUDA(cudaMemsetAsync(Gd.dW_O, 0, sizeof(float) * HD * D, st));
         }
@@ -319,11 +343,11 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
     // dY_h = dO_h W_V^h^T;  dW_V^h = Y_h^T dO_h
     Gemm gy = plain((int)C, D, dh, w.dO, HD, false, L.attn.W_V, dh, true, w.dY, (int64_t)H * D, "gemm:stca_bwd_proj");
     gy.batch = H; gy.sA = dh; gy.sB = (int64_t)D * dh; gy.sC = D;
-    if ((s = mm(gy, st)) != SA_OK) return s;
+    if ((s = mm(gy, cx)) != SA_OK) return s;
     if (C > 0) {
       Gemm gv = plain(D, dh, (int)C, Y, (int64_t)H * D, true, w.dO, HD, false, Gd.dW_V, dh, "gemm:stca_bwd_proj");
       gv.batch = H; gv.sA = D; gv.sB = dh; gv.sC = (int64_t)D * dh;
-      if ((s = mm(gv, st)) != SA_OK) return s;
+      if ((s = mm(gv, cx)) != SA_OK) return s;
     } else {
       SA_CUDA(cudaMemsetAsync(Gd.dW_V, 0, sizeof(float) * H * D * dh, st));
     }
@@ -341,37 +365,37 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
       const float* Uu = U + (size_t)r0 * D;
       const float* dYu = w.dY + (size_t)r0 * D;
       float* dXu = w.dX + (size_t)hst.kpre[u] * D;
-      if ((s = mm(plain((int)ru, (int)lu, D, Uu, D, false, Xu, D, true, w.S, lu, "gemm:stca_bwd_attn"), st)) != SA_OK) return s;
+      if ((s = mm(plain((int)ru, (int)lu, D, Uu, D, false, Xu, D, true, w.S, lu, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
       SA_TIMED("softmax_rows_kernel", st, (softmax_rows_kernel<<<(unsigned)ru, 256, 0, st>>>(w.S, lu)));
-      if ((s = mm(plain((int)ru, (int)lu, D, dYu, D, false, Xu, D, true, w.dS, lu, "gemm:stca_bwd_attn"), st)) != SA_OK) return s;
+      if ((s = mm(plain((int)ru, (int)lu, D, dYu, D, false, Xu, D, true, w.dS, lu, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
       SA_TIMED("softmax_bwd_kernel", st, (softmax_bwd_kernel<<<(unsigned)ru, 256, 0, st>>>(
                                              w.S, w.dS, lu, dYu, Y + (size_t)r0 * D, D)));
-      if ((s = mm(plain((int)ru, D, (int)lu, w.dS, lu, false, Xu, D, false, dUu, D, "gemm:stca_bwd_attn"), st)) != SA_OK) return s;
+      if ((s = mm(plain((int)ru, D, (int)lu, w.dS, lu, false, Xu, D, false, dUu, D, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
       Gemm gk = plain((int)lu, D, (int)ru, w.dS, lu, true, Uu, D, false, dXu, D, "gemm:stca_bwd_attn");
       gk.Cin = dXu; gk.ldcin = D;
-      if ((s = mm(gk, st)) != SA_OK) return s;
+      if ((s = mm(gk, cx)) != SA_OK) return s;
       Gemm gvv = plain((int)lu, D, (int)ru, w.S, lu, true, dYu, D, false, dXu, D, "gemm:stca_bwd_attn");
       gvv.Cin = dXu; gvv.ldcin = D;
-      if ((s = mm(gvv, st)) != SA_OK) return s;
+      if ((s = mm(gvv, cx)) != SA_OK) return s;
     }
     // dQh_h = dU_h W_K^h / sqrt(d_h);  dW_K^h = dU_h^T Qh_h / sqrt(d_h)
     Gemm gq = plain((int)C, dh, D, w.dU, (int64_t)H * D, false, L.attn.W_K, dh, false, w.dQh, HD, "gemm:stca_bwd_proj");
     gq.batch = H; gq.sA = D; gq.sB = (int64_t)D * dh; gq.sC = dh; gq.alpha = inv_sqrt;
-    if ((s = mm(gq, st)) != SA_OK) return s;
+    if ((s = mm(gq, cx)) != SA_OK) return s;
     if (C > 0) {
       Gemm gk = plain(D, dh, (int)C, w.dU, (int64_t)H * D, true, Qh, HD, false, Gd.dW_K, dh, "gemm:stca_bwd_proj");
       gk.batch = H; gk.sA = D; gk.sB = dh; gk.sC = (int64_t)D * dh; gk.alpha = inv_sqrt;
-      if ((s = mm(gk, st)) != SA_OK) return s;
+      if ((s = mm(gk, cx)) != SA_OK) return s;
       // dW_Q^h = q^T dQh_h
       Gemm gw = plain(D, dh, (int)C, qin, D, true, w.dQh, HD, false, Gd.dW_Q, dh, "gemm:stca_bwd_proj");
       gw.batch = H; gw.sB = dh; gw.sC = (int64_t)D * dh;
-      if ((s = mm(gw, st)) != SA_OK) return s;
+      if ((s = mm(gw, cx)) != SA_OK) return s;
       // dq = dqmid + sum_h dQh_h W_Q^h^T
       for (int h = 0; h < H; ++h) {
         Gemm gd = plain((int)C, D, dh, w.dQh + h * dh, HD, false, L.attn.W_Q + (size_t)h * D * dh, dh, true, w.dq, D,
                         "gemm:stca_bwd_proj");
         gd.Cin = h == 0 ? w.dqmid : w.dq; gd.ldcin = D;
-        if ((s = mm(gd, st)) != SA_OK) return s;
+        if ((s = mm(gd, cx)) != SA_OK) return s;
       }
     } else {
       SA_CUDA(cudaMemsetAsync(Gd.dW_K, 0, sizeof(float) * H * D * dh, st));
@@ -380,7 +404,7 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
     // history FFN: the gradient reaches the layer's input rows
     if (has_hist(L)) {
       Ffn f{L.hist_W1, L.hist_W3, L.hist_W2, Gd.hist_dW1, Gd.hist_dW3, Gd.hist_dW2};
-      if ((s = ffn_bwd(Xs(l), R, D, f, w.dX, w.dX, w.G1, w.G3, w.Uf, w.dUf, st)) != SA_OK) return s;
+      if ((s = ffn_bwd(Xs(l), R, D, f, w.dX, w.dX, w.G1, w.G3, w.Uf, w.dUf, cx)) != SA_OK) return s;
     }
   }
   // ---------------------------------------------------------------- outputs

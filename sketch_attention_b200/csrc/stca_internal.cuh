@@ -64,7 +64,9 @@ struct StcaBwdWork {
   float *G1, *G3, *Uf, *dUf;              // [max(C, kv_total), 2D]
   float *S, *dS;                          // one user's score matrix and its gradient
   float *dq, *dqmid, *dO, *dY, *dU, *dQh, *dX;
+  float* gsplit;                          // split-K partials of the GEMMs with small outputs
 };
+constexpr size_t kStcaBwdSplitFloats = (size_t)16 << 20;
 size_t stca_bwd_layout(void* base, const StcaBwdShape& sh, StcaBwdWork* w);
 sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stca_full_layer* layers,
                             const stca_full_layer_grad* grads, const float* dout, float* dq_out, float* dkv,
