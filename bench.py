@@ -200,17 +200,27 @@ class TrainStepRunner:
             phases.append(ev)
         return self.z, g
 
-    def make_pipelined_e2e(self, groups: int):
+    def make_pipelined_e2e(self, groups: int, events: bool = False):
         """The end-to-end step through the public API with host buffers, in user
         groups: group g+1's rows of X, q and dS cross PCIe (a side stream) while
         group g computes; every group's calls are the public ones (the backward
         of groups after the first adds into the weight gradients), and each
-        group's result is read back as soon as it is ready.  Returns (step,
-        h2d bytes, d2h bytes)."""
+        group's result is read back as soon as it is ready.  With ``events`` the
+        host ships each event's item id and action type (5 bytes) instead of its
+        row, and the rows are gathered on the device from the resident bf16
+        embedding tables (sa_gather_events) before the group's forward.
+        Returns (step, h2d bytes, d2h bytes)."""
         from sketch_attention_b200.dist import shard_users
         sab, w, dev = self.sab, self.w, self.dev
-        hX = torch.empty(self.X.shape, dtype=torch.bfloat16, pin_memory=True)
-        hX.copy_(self.X)
+        if events:
+            hI = torch.from_numpy(w.sa.item_ids).pin_memory()
+            hA = torch.from_numpy(w.sa.action_ids).pin_memory()
+            dI, dA = torch.empty_like(hI, device=dev), torch.empty_like(hA, device=dev)
+            item_t = torch.from_numpy(w.item_table.view(np.int16)).to(dev).view(torch.bfloat16)
+            act_t = torch.from_numpy(w.action_table.view(np.int16)).to(dev).view(torch.bfloat16)
+        else:
+            hX = torch.empty(self.X.shape, dtype=torch.bfloat16, pin_memory=True)
+            hX.copy_(self.X)
         hq = torch.empty(self.q.shape, dtype=torch.bfloat16, pin_memory=True)
         hq.copy_(self.q)
         hdS = torch.empty(self.dS.shape, dtype=torch.float32, pin_memory=True)
@@ -245,7 +255,11 @@ class TrainStepRunner:
             copy_stream.wait_stream(main)          # the previous step's reads of these buffers are done
             with torch.cuda.stream(copy_stream):
                 for g in plan:
-                    self.X[g["lo"]:g["hi"]].copy_(hX[g["lo"]:g["hi"]], non_blocking=True)
+                    if events:
+                        dI[g["lo"]:g["hi"]].copy_(hI[g["lo"]:g["hi"]], non_blocking=True)
+                        dA[g["lo"]:g["hi"]].copy_(hA[g["lo"]:g["hi"]], non_blocking=True)
+                    else:
+                        self.X[g["lo"]:g["hi"]].copy_(hX[g["lo"]:g["hi"]], non_blocking=True)
                     self.q[g["c0"]:g["c1"]].copy_(hq[g["c0"]:g["c1"]], non_blocking=True)
                     self.dS[g["u0"]:g["u1"]].copy_(hdS[g["u0"]:g["u1"]], non_blocking=True)
                     g["ev"].record(copy_stream)
@@ -253,6 +267,8 @@ class TrainStepRunner:
                 main.wait_event(g["ev"])
                 u0, u1, lo, hi, c0, c1 = g["u0"], g["u1"], g["lo"], g["hi"], g["c0"], g["c1"]
                 Xg = self.X[lo:hi]
+                if events:
+                    sab.sa_gather_events(item_t, act_t, dI[lo:hi], dA[lo:hi], out=Xg)
                 f = sab.sa_forward(Xg, g["off"], self.P, self.WQ, self.WK, self.WV, w.sa.eps,
                                    offsets_dev=g["offd"], workspace=self.ws_f,
                                    out={"S": fo["S"][u0:u1], "mass": fo["mass"][u0:u1],
@@ -278,7 +294,8 @@ class TrainStepRunner:
             for n in hg:
                 hg[n].copy_(go[n], non_blocking=True)
 
-        h2d = hX.numel() * 2 + hq.numel() * 2 + hdS.numel() * 4
+        rows_bytes = (hI.numel() * 4 + hA.numel()) if events else hX.numel() * 2
+        h2d = rows_bytes + hq.numel() * 2 + hdS.numel() * 4
         return step, h2d, self.results_nbytes()
 
     def results_nbytes(self):
@@ -397,11 +414,9 @@ def run_ours(args, rank, world, device):
     ph_ms = ph.mean(axis=0) if len(ph) else np.zeros(3)
 
     # ---- end to end through the public API with host buffers
-    e2e = None
-    if not args.no_e2e:
-        e2e_step, h2d, d2h = R.make_pipelined_e2e(E2E_GROUPS)
+    def time_e2e(events):
+        e2e_step, h2d, d2h = R.make_pipelined_e2e(E2E_GROUPS, events=events)
         torch.cuda.synchronize()
-
         for _ in range(max(1, args.warmup)):
             e2e_step()
         torch.cuda.synchronize()
@@ -416,9 +431,18 @@ def run_ours(args, rank, world, device):
         if world > 1:
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
-        e2e = {"value": world * R.tokens / (e2e_ms / 1e3), "unit": "history-tokens/s",
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "user_groups": E2E_GROUPS}
+        return {"value": world * R.tokens / (e2e_ms / 1e3), "unit": "history-tokens/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "user_groups": E2E_GROUPS}
+
+    e2e = e2e_ids = None
+    if not args.no_e2e:
+        e2e = time_e2e(False)
+        if R.w.item_table is not None:
+            # the same step shipping 5-byte event ids; the bf16 embedding tables are
+            # resident parameters, the rows are gathered on the device
+            e2e_ids = time_e2e(True)
+            e2e_ids["inputs"] = "item ids (int32) + action types (uint8) per event, q, dS; tables resident"
 
     # ---- roofline of the dominant kernel
     roof = None
@@ -466,6 +490,7 @@ def run_ours(args, rank, world, device):
         "kernels": kernels,
         "gpu_launches": int(launches),
         "e2e": e2e,
+        "e2e_event_ids": e2e_ids,
         "clocks": clk.summary(),
         "input_generation_s": gen_s,
     }

@@ -240,6 +240,22 @@ sa_status sa_refine_forward(const void* X, sa_dtype x_dtype, const int64_t* offs
                             float* sketch, void* workspace, size_t ws_bytes,
                             sa_stream_t stream);
 
+/*
+ * sa_gather_events -- the events' input rows on the device: for i < n
+ *   X[i] = item_table[item_ids[i]] + action_table[action_ids[i]]
+ * (an item embedding plus the embedding of the feedback type, the workloads'
+ * events; paper Sec. 3.5, the sum that eq. (20)'s fusion adds a SwiGLU term
+ * to), so that a step ships 5 bytes of ids per event instead of its row.
+ * item_table [vocab, d] and action_table [n_actions, d] bf16, 16-byte aligned;
+ * item_ids int32 [n] (4-byte aligned), action_ids uint8 [n]; X [n, d] bf16 out.
+ * The sum is formed in fp32 and rounded to nearest even.  d a multiple of 8.
+ * An id outside its table gives a zero row and makes the next
+ * sa_poll_device_status return SA_ERR_INVALID_ARG (no out-of-bounds read).
+ */
+sa_status sa_gather_events(const void* item_table, int64_t vocab, const void* action_table,
+                           int n_actions, const int32_t* item_ids, const uint8_t* action_ids,
+                           int64_t n, int d, void* X, sa_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* STCA: stacked target-to-history single-query cross attention             */
 /* ------------------------------------------------------------------------ */

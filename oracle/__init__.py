@@ -55,7 +55,7 @@ import numpy as np
 __all__ = [
     "sa_forward", "sa_user", "sa_backward", "stca_branch", "stca_branch_reordered",
     "stca_fuse", "assignment", "token_lse", "layer_norm", "swiglu_ffn", "sa_refine_user",
-    "sa_refine", "tokenwise_user", "sa_forward_tokenwise", "stca_branch_grads",
+    "sa_refine", "tokenwise_user", "sa_forward_tokenwise", "stca_branch_grads", "event_rows",
 ]
 
 
@@ -330,6 +330,13 @@ def stca_branch_grads(q, cand_offsets, kv, kv_begin, kv_end, layers, heads: int,
             if v is not None:
                 res["layers"][li][k] = zero(res["layers"][li][k], v).numpy()
     return res
+
+
+def event_rows(item_table, action_table, item_ids, action_ids) -> np.ndarray:
+    """Event embeddings x_i = item_table[id_i] + action_table[a_i] (the workloads'
+    events: an item embedding plus the embedding of the feedback type, the plain
+    sum that eq. (20)'s fusion adds a SwiGLU term to), exact in fp64."""
+    return _f64(item_table)[np.asarray(item_ids, np.int64)] + _f64(action_table)[np.asarray(action_ids, np.int64)]
 
 
 def stca_fuse(z_r, z_u, W_F, b_F=None):

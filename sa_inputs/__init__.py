@@ -107,11 +107,15 @@ class EventTables:
         action = gauss(rng, (N_ACTIONS, d), 0.02)
         return EventTables(item, action, ZipfSampler(rng, vocab))
 
-    def events(self, rng, n: int) -> np.ndarray:
-        """n event embeddings item[id] + action[a], fp32 (not yet rounded)."""
+    def events(self, rng, n: int, with_ids: bool = False):
+        """n event embeddings item[id] + action[a], fp32 (not yet rounded); with
+        ``with_ids`` also the item ids (int32) and action types (uint8) drawn."""
         ids = self.zipf.sample(rng, n)
         acts = rng.integers(0, N_ACTIONS, n)
-        return self.item[ids] + self.action[acts]
+        rows = self.item[ids] + self.action[acts]
+        if with_ids:
+            return rows, ids.astype(np.int32), acts.astype(np.uint8)
+        return rows
 
     def targets(self, rng, n: int) -> np.ndarray:
         return self.item[self.zipf.sample(rng, n)].copy()
@@ -132,6 +136,8 @@ class SAProblem:
     W_V: np.ndarray
     eps: float = 1e-6
     dS: Optional[np.ndarray] = None   # f32 [B, k, d] upstream gradient
+    item_ids: Optional[np.ndarray] = None     # int32 [N] the events' item ids (when kept)
+    action_ids: Optional[np.ndarray] = None   # uint8 [N] their action types
 
     @property
     def B(self) -> int:
@@ -238,11 +244,13 @@ SA_WORKLOADS = {
 
 
 def sa_workload(cfg: int, vocab: int = 1_000_000, users: Optional[int] = None,
-                with_tables: bool = False):
+                with_tables: bool = False, keep_ids: bool = False):
     """SA inputs for workload ``cfg`` (1, 2, 3 or 5).
 
     ``users`` truncates the batch to its first users (same random stream for
     the lengths and weights, so the first users match the full batch's).
+    ``keep_ids`` also records each event's item id and action type (the same
+    draws, so X is unchanged).
     """
     rng = rng_for(1000 + cfg)
     if cfg == 1:
@@ -262,11 +270,20 @@ def sa_workload(cfg: int, vocab: int = 1_000_000, users: Optional[int] = None,
     offsets = np.zeros(len(lengths) + 1, np.int64)
     offsets[1:] = np.cumsum(lengths)
     X = np.empty((int(offsets[-1]), d), np.uint16 if dtype == "bf16" else np.float32)
+    keep = keep_ids and kind == "events"
+    item_ids = np.empty(int(offsets[-1]), np.int32) if keep else None
+    action_ids = np.empty(int(offsets[-1]), np.uint8) if keep else None
     for u, n in enumerate(lengths):
-        rows = gauss(rng, (n, d), 1.0 / math.sqrt(d)) if kind == "gauss" else tables.events(rng, n)
+        if kind == "gauss":
+            rows = gauss(rng, (n, d), 1.0 / math.sqrt(d))
+        elif keep:
+            rows, item_ids[offsets[u]:offsets[u + 1]], action_ids[offsets[u]:offsets[u + 1]] = \
+                tables.events(rng, n, with_ids=True)
+        else:
+            rows = tables.events(rng, n)
         X[offsets[u]:offsets[u + 1]] = _pack(dtype, rows)
     dS = gauss(rng, (len(lengths), k, d), 1.0) if cfg == 5 else None
-    prob = SAProblem(SA_WORKLOADS[cfg], dtype, offsets, X, P, W_Q, W_K, W_V, 1e-6, dS)
+    prob = SAProblem(SA_WORKLOADS[cfg], dtype, offsets, X, P, W_Q, W_K, W_V, 1e-6, dS, item_ids, action_ids)
     if with_tables:
         return prob, tables, rng
     return prob
@@ -331,6 +348,18 @@ def stca_layers(rng, n_layers: int, D: int, heads: int, d_h: int, with_wo: bool 
         W_O = gauss(rng, (heads * d_h, D), std) if with_wo else None
         out.append(STCALayer(W_Q, W_K, W_V, W_O))
     return out
+
+
+def event_problem(n: int, vocab: int, d: int, seed: int, n_actions: int = N_ACTIONS):
+    """Seeded inputs of the event-embedding gather: bf16 item and action tables
+    (bits, std 0.02 like the workloads' tables), Zipf(1.1) item ids (int32) and
+    uniform action types (uint8) for n events."""
+    rng = rng_for(seed)
+    item = bf16_bits(gauss(rng, (vocab, d), 0.02))
+    action = bf16_bits(gauss(rng, (n_actions, d), 0.02))
+    ids = ZipfSampler(rng, vocab).sample(rng, n).astype(np.int32)
+    acts = rng.integers(0, n_actions, n).astype(np.uint8)
+    return item, action, ids, acts
 
 
 def add_stca_ffns(rng, layers, D: int, hist: bool = True, query: bool = True):
@@ -431,6 +460,8 @@ class TrainStep:
     layers_u: list
     W_F: np.ndarray
     b_F: np.ndarray
+    item_table: Optional[np.ndarray] = None     # bf16 bits [vocab, d]: the events' item embeddings
+    action_table: Optional[np.ndarray] = None   # bf16 bits [N_ACTIONS, d]
 
 
 TRAIN_STEP_WORKLOAD = ("train step bf16 B=64 n~lognormal(mean 85K) d=128 k=1024: sa_fwd+sa_bwd, "
@@ -440,7 +471,7 @@ TRAIN_STEP_WORKLOAD = ("train step bf16 B=64 n~lognormal(mean 85K) d=128 k=1024:
 
 def train_step_workload(vocab: int = 1_000_000, users: Optional[int] = None,
                         cands: int = 256) -> TrainStep:
-    sa, tables, rng = sa_workload(5, vocab=vocab, users=users, with_tables=True)
+    sa, tables, rng = sa_workload(5, vocab=vocab, users=users, with_tables=True, keep_ids=True)
     D, heads, d_h = sa.d, 4, 32
     layers_r = stca_layers(rng, 2, D, heads, d_h)
     layers_u = stca_layers(rng, 2, D, heads, d_h)
@@ -449,4 +480,5 @@ def train_step_workload(vocab: int = 1_000_000, users: Optional[int] = None,
     cand_off = np.arange(sa.B + 1, dtype=np.int64) * cands
     q = bf16_bits(tables.targets(rng, int(cand_off[-1])))
     rb, re = suffix_ranges(sa.offsets)
-    return TrainStep(sa, cand_off, q, rb, re, heads, d_h, layers_r, layers_u, W_F, b_F)
+    return TrainStep(sa, cand_off, q, rb, re, heads, d_h, layers_r, layers_u, W_F, b_F,
+                     bf16_bits(tables.item), bf16_bits(tables.action))

@@ -31,7 +31,7 @@ EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_w
            "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward",
            "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate",
            "stca_forward_full_workspace", "stca_forward_full", "stca_backward_full_workspace",
-           "stca_backward_full")
+           "stca_backward_full", "sa_gather_events")
 
 
 class SAError(RuntimeError):
@@ -110,6 +110,8 @@ def load(path: Optional[str] = None):
     lib.stca_backward_full.argtypes = [_vp, _i, _vp, _vp, _i, _vp, _i64, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, ctypes.POINTER(StcaFullLayerC), _vp, _vp, _vp,
                                        ctypes.POINTER(StcaFullLayerGradC), _vp, _sz, _vp]
+    lib.sa_gather_events.restype = _i
+    lib.sa_gather_events.argtypes = [_vp, _i64, _vp, _i, _vp, _vp, _i64, _i, _vp, _vp]
     lib.stca_fuse.restype = _i
     lib.stca_fuse.argtypes = [_vp, _vp, _vp, _vp, _i64, _i, _vp, _vp]
     lib.sa_forward_noalloc.restype = _i
@@ -411,6 +413,24 @@ def stca_forward_full(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin,
                                _p(workspace), workspace.numel(), _stream(stream))
     _check("stca_forward_full", st)
     return res
+
+
+def sa_gather_events(item_table: torch.Tensor, action_table: torch.Tensor, item_ids: torch.Tensor,
+                     action_ids: torch.Tensor, *, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """X[i] = item_table[item_ids[i]] + action_table[action_ids[i]] (bf16 tables and
+    output, int32 / uint8 ids, CUDA tensors).  Returns X [n, d] bf16."""
+    lib = load()
+    _need_cuda(item_table, action_table, item_ids, action_ids)
+    if item_table.dtype != torch.bfloat16 or action_table.dtype != torch.bfloat16:
+        raise TypeError("the tables must be bf16")
+    if item_ids.dtype != torch.int32 or action_ids.dtype != torch.uint8:
+        raise TypeError("item_ids must be int32 and action_ids uint8")
+    n, d = item_ids.numel(), item_table.shape[1]
+    X = out if out is not None else torch.empty(n, d, dtype=torch.bfloat16, device=item_table.device)
+    st = lib.sa_gather_events(_p(item_table), item_table.shape[0], _p(action_table), action_table.shape[0],
+                              _p(item_ids), _p(action_ids), n, d, _p(X), _stream(stream))
+    _check("sa_gather_events", st)
+    return X
 
 
 def _full_layers_c(layers):

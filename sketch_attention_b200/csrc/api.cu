@@ -290,6 +290,7 @@ sa_status sa_poll_device_status(sa_stream_t stream) {
     int zero = 0;
     cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice);
     if (v & DEV_ERR_TIMEOUT) return fail(SA_ERR_TIMEOUT, "a device-side wait expired");
+    if (v & DEV_ERR_INDEX) return fail(SA_ERR_INVALID_ARG, "an embedding id was out of range (its row was zeroed)");
     return fail(SA_ERR_CUDA, "device error word " + std::to_string(v));
   }
   return SA_OK;
@@ -646,6 +647,21 @@ StcaBwdShape bwd_shape(int B, const int64_t* cand, const int64_t* kb, const int6
 }  // namespace
 
 extern "C" {
+
+sa_status sa_gather_events(const void* item_table, int64_t vocab, const void* action_table, int n_actions,
+                           const int32_t* item_ids, const uint8_t* action_ids, int64_t n, int d, void* X,
+                           sa_stream_t stream) {
+  if (n < 0 || vocab < 1 || n_actions < 1 || n_actions > 256) return fail(SA_ERR_INVALID_ARG, "bad sizes");
+  if (d < 8 || d % 8 != 0) return fail(SA_ERR_UNSUPPORTED, "d must be a positive multiple of 8");
+  SA_TRY(check_ptr(item_table, "item_table"));
+  SA_TRY(check_ptr(action_table, "action_table"));
+  // the ids are read element by element: any alignment of their type will do
+  if (n > 0 && (!item_ids || !action_ids)) return fail(SA_ERR_INVALID_ARG, "item_ids or action_ids is NULL");
+  if (((uintptr_t)item_ids & 3) != 0) return fail(SA_ERR_INVALID_ARG, "item_ids is not 4-byte aligned");
+  SA_TRY(check_ptr(X, "X", n == 0));
+  return gather_events_run(item_table, vocab, action_table, n_actions, item_ids, action_ids, n, d, X,
+                           (cudaStream_t)stream);
+}
 
 size_t stca_backward_full_workspace(int B, const int64_t* cand_offsets_host, const int64_t* kv_begin_host,
                                     const int64_t* kv_end_host, int D, int heads, int d_h, int n_layers,

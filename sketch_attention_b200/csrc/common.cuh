@@ -47,7 +47,7 @@ void prof_end(const char* name, cudaStream_t st);
 
 // Device error word (defined in api.cu): kernels whose bounded waits expire
 // OR in a code; sa_poll_device_status reads and clears it.
-enum : int { DEV_ERR_TIMEOUT = 1 };
+enum : int { DEV_ERR_TIMEOUT = 1, DEV_ERR_INDEX = 2 };
 int* device_status_word();
 
 // ---------------------------------------------------------------- device info

@@ -100,6 +100,10 @@ sa_status sa_tokenwise_run(const SaFwdArgs& a, const TokenwiseWork& w, cudaStrea
 
 // Sums the split-n partials into H (if a.H), the mass and H/(m+eps) (w.Hhat).
 sa_status sa_reduce(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
+// x_i = item[id_i] + action[a_i] for n bf16 rows of width d (a multiple of 8)
+sa_status gather_events_run(const void* item, int64_t vocab, const void* action, int n_actions,
+                            const int32_t* ids, const uint8_t* acts, int64_t n, int d, void* X,
+                            cudaStream_t st);
 // U = SiLU(G1) * G3 elementwise over n fp32 values (n a multiple of 4, 16-byte aligned)
 sa_status sa_swiglu(const float* G1, const float* G3, int64_t n, float* U, cudaStream_t st);
 sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
