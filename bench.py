@@ -591,6 +591,7 @@ def run_component(args, rank, world, device):
                                       workspace=ws)
         units, unit, name = p.n_total, "history-tokens/s", p.name
         kname, flops = "sa_agg_tc_kernel", 2.0 * p.k * p.d * p.n_total
+        fwd_k = p.k
     elif args.workload == "tokenwise":
         p = sa_workload(5, users=args.users)
         X = _dev_bf16(p.X, device)
@@ -774,6 +775,22 @@ def run_component(args, rank, world, device):
             "clocks": clk.summary()}
     if extra_roofs:
         line["other_rooflines"] = extra_roofs
+    if args.workload == "sa_fwd" and "sa_lse_tc_kernel" in prof and "sa_agg_tc_kernel" in prof:
+        # the forward as a whole (its two kernels): 4kd flop and 2k exponentials per token
+        # credited, against the burst bf16 peak and the measured exponential rate of the
+        # kernels' MUFU / FMA mix
+        fwd_s = (prof["sa_lse_tc_kernel"][0] + prof["sa_agg_tc_kernel"][0]) / args.steps / 1e3
+        rate_mix, rate_mufu = sab.measure_exp2_rate(1), sab.measure_exp2_rate(0)
+        pk = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+        tf = 4.0 * fwd_k * 128 * units / fwd_s / 1e12
+        ex = 2.0 * fwd_k * units / fwd_s
+        line["forward_rooflines"] = {
+            "kernels_ms": fwd_s * 1e3,
+            "tensor": {"achieved": tf, "peak": pk, "unit": "TFLOP/s", "frac": tf / pk,
+                       "peak_source": f"bf16 dense, burst ({peaks_src})"},
+            "exp": {"achieved": ex, "peak": rate_mix, "unit": "exp2/s", "frac": ex / rate_mix,
+                    "peak_source": "measured on this GPU in this run (sa_measure_exp2_rate, the kernels' "
+                                   "mix: 3/4 MUFU ex2, 1/4 FMA cubic)", "mufu_only_rate": rate_mufu}}
     return line
 
 

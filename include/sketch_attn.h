@@ -401,6 +401,14 @@ sa_status stca_fuse(const float* z_r, const float* z_u, const float* W_F, const 
 /* ------------------------------------------------------------------------ */
 /* Measurement support (not part of the method)                              */
 /* ------------------------------------------------------------------------ */
+/*
+ * Exponentials per second on the current GPU (all SMs, synchronous): mode 0 with
+ * every 2^x on the MUFU (ex2.approx), mode 1 with the SA forward kernels' mix
+ * (one pair in four by a cubic on the FMA pipe).  The co-roofline of the
+ * forward: each of its two kernels evaluates k exponentials per token.
+ */
+sa_status sa_measure_exp2_rate(int mode, double* per_second, sa_stream_t stream);
+
 /* Number of kernels this library has launched in this process. */
 long long sa_launch_count(void);
 

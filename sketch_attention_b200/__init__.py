@@ -31,7 +31,7 @@ EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_w
            "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward",
            "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate",
            "stca_forward_full_workspace", "stca_forward_full", "stca_backward_full_workspace",
-           "stca_backward_full", "sa_gather_events")
+           "stca_backward_full", "sa_gather_events", "sa_measure_exp2_rate")
 
 
 class SAError(RuntimeError):
@@ -110,6 +110,8 @@ def load(path: Optional[str] = None):
     lib.stca_backward_full.argtypes = [_vp, _i, _vp, _vp, _i, _vp, _i64, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, ctypes.POINTER(StcaFullLayerC), _vp, _vp, _vp,
                                        ctypes.POINTER(StcaFullLayerGradC), _vp, _sz, _vp]
+    lib.sa_measure_exp2_rate.restype = _i
+    lib.sa_measure_exp2_rate.argtypes = [_i, ctypes.POINTER(ctypes.c_double), _vp]
     lib.sa_gather_events.restype = _i
     lib.sa_gather_events.argtypes = [_vp, _i64, _vp, _i, _vp, _vp, _i64, _i, _vp, _vp]
     lib.stca_fuse.restype = _i
@@ -413,6 +415,14 @@ def stca_forward_full(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin,
                                _p(workspace), workspace.numel(), _stream(stream))
     _check("stca_forward_full", st)
     return res
+
+
+def measure_exp2_rate(mode: int = 1, stream=None) -> float:
+    """Exponentials per second on the current GPU: mode 0 all on the MUFU, mode 1 the
+    SA forward kernels' mix (one pair in four on the FMA pipe)."""
+    out = ctypes.c_double(0.0)
+    _check("sa_measure_exp2_rate", load().sa_measure_exp2_rate(mode, ctypes.byref(out), _stream(stream)))
+    return out.value
 
 
 def sa_gather_events(item_table: torch.Tensor, action_table: torch.Tensor, item_ids: torch.Tensor,

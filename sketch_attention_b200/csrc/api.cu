@@ -648,6 +648,11 @@ StcaBwdShape bwd_shape(int B, const int64_t* cand, const int64_t* kb, const int6
 
 extern "C" {
 
+sa_status sa_measure_exp2_rate(int mode, double* per_second, sa_stream_t stream) {
+  if ((mode != 0 && mode != 1) || !per_second) return fail(SA_ERR_INVALID_ARG, "mode must be 0 or 1, per_second non-NULL");
+  return measure_exp2_rate(mode, per_second, (cudaStream_t)stream);
+}
+
 sa_status sa_gather_events(const void* item_table, int64_t vocab, const void* action_table, int n_actions,
                            const int32_t* item_ids, const uint8_t* action_ids, int64_t n, int d, void* X,
                            sa_stream_t stream) {
