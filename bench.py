@@ -494,6 +494,13 @@ def run_ours(args, rank, world, device):
         "clocks": clk.summary(),
         "input_generation_s": gen_s,
     }
+    from sketch_attention_b200 import flops as flop_model
+    hl = flop_model.headline(100_000)
+    line["analytic_context"] = {
+        "train_flop_reduction_vs_direct_stca": round(hl["train_ratio"], 2),
+        "infer_flop_reduction_vs_direct_stca": round(hl["infer_ratio"], 2),
+        "note": "the pages' GEMM-FLOP ratios at 100K events (Sec. 5.4, eqs. 28-34), recomputed by "
+                "sketch_attention_b200.flops; analytic context, not a hardware target"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, 30_000)
     return line
