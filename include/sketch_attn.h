@@ -409,6 +409,15 @@ sa_status stca_fuse(const float* z_r, const float* z_u, const float* W_F, const 
  */
 sa_status sa_measure_exp2_rate(int mode, double* per_second, sa_stream_t stream);
 
+/*
+ * Self-test of the device-side failure path (no fault): launches one thread that
+ * waits on an mbarrier nothing arrives at, with the bounded wait every kernel of
+ * the library uses, for about budget_cycles SM clocks (1 .. 4e9).  On expiry the
+ * wait sets the device error word and the kernel returns, so the next
+ * sa_poll_device_status returns SA_ERR_TIMEOUT and the context stays usable.
+ */
+sa_status sa_selftest_bounded_wait(long long budget_cycles, sa_stream_t stream);
+
 /* Number of kernels this library has launched in this process. */
 long long sa_launch_count(void);
 

@@ -31,7 +31,7 @@ EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_w
            "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward",
            "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate",
            "stca_forward_full_workspace", "stca_forward_full", "stca_backward_full_workspace",
-           "stca_backward_full", "sa_gather_events", "sa_measure_exp2_rate")
+           "stca_backward_full", "sa_gather_events", "sa_measure_exp2_rate", "sa_selftest_bounded_wait")
 
 
 class SAError(RuntimeError):
@@ -110,6 +110,8 @@ def load(path: Optional[str] = None):
     lib.stca_backward_full.argtypes = [_vp, _i, _vp, _vp, _i, _vp, _i64, _vp, _vp, _vp, _vp,
                                        _i, _i, _i, _i, ctypes.POINTER(StcaFullLayerC), _vp, _vp, _vp,
                                        ctypes.POINTER(StcaFullLayerGradC), _vp, _sz, _vp]
+    lib.sa_selftest_bounded_wait.restype = _i
+    lib.sa_selftest_bounded_wait.argtypes = [ctypes.c_longlong, _vp]
     lib.sa_measure_exp2_rate.restype = _i
     lib.sa_measure_exp2_rate.argtypes = [_i, ctypes.POINTER(ctypes.c_double), _vp]
     lib.sa_gather_events.restype = _i
@@ -415,6 +417,12 @@ def stca_forward_full(q: torch.Tensor, cand_offsets, kv: torch.Tensor, kv_begin,
                                _p(workspace), workspace.numel(), _stream(stream))
     _check("stca_forward_full", st)
     return res
+
+
+def selftest_bounded_wait(budget_cycles: int = 2_000_000, stream=None) -> None:
+    """Launch a kernel whose only wait cannot complete (bounded to ~budget_cycles);
+    the next poll_device_status() raises SAError with SA_ERR_TIMEOUT."""
+    _check("sa_selftest_bounded_wait", load().sa_selftest_bounded_wait(budget_cycles, _stream(stream)))
 
 
 def measure_exp2_rate(mode: int = 1, stream=None) -> float:

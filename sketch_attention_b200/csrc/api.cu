@@ -653,6 +653,11 @@ sa_status sa_measure_exp2_rate(int mode, double* per_second, sa_stream_t stream)
   return measure_exp2_rate(mode, per_second, (cudaStream_t)stream);
 }
 
+sa_status sa_selftest_bounded_wait(long long budget_cycles, sa_stream_t stream) {
+  if (budget_cycles < 1 || budget_cycles > 4000000000LL) return fail(SA_ERR_INVALID_ARG, "budget out of range");
+  return selftest_bounded_wait(budget_cycles, (cudaStream_t)stream);
+}
+
 sa_status sa_gather_events(const void* item_table, int64_t vocab, const void* action_table, int n_actions,
                            const int32_t* item_ids, const uint8_t* action_ids, int64_t n, int d, void* X,
                            sa_stream_t stream) {

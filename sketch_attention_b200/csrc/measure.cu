@@ -36,7 +36,25 @@ __global__ void __launch_bounds__(kThreads) exp2_rate_kernel(float* __restrict__
   for (int j = 0; j < kPairs; ++j) s += v[j].x + v[j].y;
   sink[(int64_t)blockIdx.x * kThreads + threadIdx.x] = s;
 }
+// One thread waits on an mbarrier that nothing arrives at, with the bounded wait
+// every kernel of the library uses; on expiry the wait sets the abort flag and the
+// device error word and returns, and so does the kernel (no trap, no fault).
+__global__ void bounded_wait_kernel(long long budget, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  tc::mbar_init(&bar, 1);
+  abort_flag = 0;
+  tc::fence_mbar_init();
+  tc::mbar_wait(&bar, 0, &abort_flag, err, budget);
+}
 }  // namespace
+
+sa_status selftest_bounded_wait(long long budget_cycles, cudaStream_t st) {
+  bounded_wait_kernel<<<1, 32, 0, st>>>(budget_cycles, device_status_word());
+  SA_CUDA(cudaGetLastError());
+  return SA_OK;
+}
 
 sa_status measure_exp2_rate(int mode, double* per_second, cudaStream_t st) {
   const int blocks = device_info().sm_count * 4;

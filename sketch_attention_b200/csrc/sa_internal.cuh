@@ -103,6 +103,8 @@ sa_status sa_reduce(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);
 // exponentials per second over the whole GPU: mode 0 all on the MUFU, mode 1 the
 // SA forward's mix (one pair in four on the FMA pipe)
 sa_status measure_exp2_rate(int mode, double* per_second, cudaStream_t st);
+// a kernel whose only mbarrier wait cannot complete: exercises the bounded-wait path
+sa_status selftest_bounded_wait(long long budget_cycles, cudaStream_t st);
 // x_i = item[id_i] + action[a_i] for n bf16 rows of width d (a multiple of 8)
 sa_status gather_events_run(const void* item, int64_t vocab, const void* action, int n_actions,
                             const int32_t* ids, const uint8_t* acts, int64_t n, int d, void* X,
