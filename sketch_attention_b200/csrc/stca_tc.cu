@@ -18,6 +18,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "exp2_poly.cuh"
 #include "stca_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -208,13 +209,24 @@ __global__ void __launch_bounds__(THREADS, 1)
       // P buffer b was last read by PV(j-2)
       if (j >= 2 && !mbar_wait(&bars->pv_done[b], ((j >> 1) - 1) & 1, abort, p.err)) { ok = false; break; }
       uint32_t pw[64];
-      float ls = 0.f;
+      float2 ls2 = make_float2(0.f, 0.f);
+      const float2 nm = make_float2(-m, -m);
 #pragma unroll
       for (int i = 0; i < 128; i += 2) {
-        const float e0 = ex2(sv[i] - m), e1 = ex2(sv[i + 1] - m);
-        ls += e0 + e1;
-        pw[i / 2] = pack_bf16x2(e0, e1);
+        // one pair in four on the FMA pipe (fitted cubic), the rest on the MUFU
+        const float2 e = __fadd2_rn(make_float2(sv[i], sv[i + 1]), nm);
+        float2 v;
+        if ((i / 2) % 4 == 1) {
+          v = exp2_poly2(e);                 // clamps at 2^-125: a masked key (-inf) must give 0
+          v.x = e.x < -125.f ? 0.f : v.x;
+          v.y = e.y < -125.f ? 0.f : v.y;
+        } else {
+          v = make_float2(ex2(e.x), ex2(e.y));
+        }
+        ls2 = __fadd2_rn(ls2, v);
+        pw[i / 2] = pack_bf16x2(v.x, v.y);
       }
+      const float ls = ls2.x + ls2.y;
       l += ls;
       tmem_st32(tmem + lane_addr + (b ? TM_P1 : TM_P0), pw);
       tmem_st32(tmem + lane_addr + (b ? TM_P1 : TM_P0) + 32, pw + 32);
