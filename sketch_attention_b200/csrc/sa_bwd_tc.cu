@@ -30,6 +30,7 @@
 #include "sa_internal.cuh"
 #include "exp2_poly.cuh"
 #include "tc_ptx.cuh"
+#include "tma_map.cuh"
 
 // Pairs (of the 4 in a group of 8 prototypes) whose exponentials the E kernel
 // evaluates on the FMA pipe instead of the MUFU.
@@ -589,36 +590,9 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
 }
 
 // ============================================================== host side
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* q = nullptr;
-    cudaDriverEntryPointQueryResult r;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
-        r == cudaDriverEntryPointSuccess)
-      fn = (EncodeFn)q;
-  });
-  return fn;
-}
 
 sa_status map_rows(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
-  EncodeFn enc = encode_fn();
-  if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  cuuint64_t dims[2] = {DD, rows};
-  cuuint64_t strides[1] = {DD * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
-  return SA_OK;
+  return tma_map_bf16(map, base, DD, rows, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // dmc[u, j] = dm[u, j] - mean_j dm[u, :]

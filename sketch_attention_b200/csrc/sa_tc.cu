@@ -28,6 +28,7 @@
 #include "exp2_poly.cuh"
 #include "sa_internal.cuh"
 #include "tc_ptx.cuh"
+#include "tma_map.cuh"
 
 // Pairs (of the 4 in a group of 8 prototypes) whose exponentials the lse and
 // aggregation kernels evaluate on the FMA pipe instead of the MUFU.
@@ -529,38 +530,11 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
 }
 
 // ============================================================== host side
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = (EncodeFn)p;
-  });
-  return fn;
-}
 
 // [outer, 128] bf16 rows; boxes of box_inner x 128 rows
 sa_status make_map(CUtensorMap* map, const void* base, uint64_t outer, uint32_t box_inner,
                    CUtensorMapSwizzle swz) {
-  EncodeFn enc = encode_fn();
-  if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  cuuint64_t dims[2] = {(cuuint64_t)DD, outer};
-  cuuint64_t strides[1] = {(cuuint64_t)DD * 2};
-  cuuint32_t box[2] = {box_inner, (cuuint32_t)TILE};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
-  return SA_OK;
+  return tma_map_bf16(map, base, DD, outer, box_inner, TILE, swz);
 }
 
 std::mutex g_mu;

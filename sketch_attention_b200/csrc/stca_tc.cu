@@ -21,6 +21,7 @@
 #include "exp2_poly.cuh"
 #include "stca_internal.cuh"
 #include "tc_ptx.cuh"
+#include "tma_map.cuh"
 
 namespace sa {
 
@@ -261,36 +262,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* q = nullptr;
-    cudaDriverEntryPointQueryResult r;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
-        r == cudaDriverEntryPointSuccess)
-      fn = (EncodeFn)q;
-  });
-  return fn;
-}
 
 sa_status make_map(CUtensorMap* map, const void* base, uint64_t rows) {
-  EncodeFn enc = encode_fn();
-  if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  cuuint64_t dims[2] = {DD, rows};
-  cuuint64_t strides[1] = {DD * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
-  return SA_OK;
+  return tma_map_bf16(map, base, DD, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 }  // namespace
 
