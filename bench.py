@@ -508,27 +508,31 @@ def run_ours(args, rank, world, device):
 
 # --------------------------------------------------------------------------
 # the oracle on the host cores (CPU baseline and the reference arm)
-def _oracle_sample(w, n_tokens=None):
-    """One bounded sample of the step: user 0's forward and backward (its first
-    n_tokens events) plus STCA of its 256 candidates on both branches and the
-    fusion, all by the fp64 oracle."""
+def _oracle_sample(w, n_tokens=None, users=(0,)):
+    """One bounded sample of the step: for each listed user, its forward and
+    backward (its first n_tokens events) plus STCA of its 256 candidates on both
+    branches and the fusion, all by the fp64 oracle.  Returns (events, seconds)."""
     import oracle
     from sa_inputs import bf16_to_f64
     sa = w.sa
-    lo, hi = int(sa.offsets[0]), int(sa.offsets[1])
-    if n_tokens is not None:
-        hi = min(hi, lo + n_tokens)
-    X = sa.x_f64(lo, hi)
-    t0 = time.perf_counter()
-    S, m, H = oracle.sa_forward(X, [0, hi - lo], sa.P, sa.W_Q, sa.W_K, sa.W_V, sa.eps)
-    oracle.sa_backward(X, [0, hi - lo], sa.P, sa.W_Q, sa.W_K, sa.W_V, sa.eps, sa.dS[:1])
-    c0, c1 = int(w.cand_offsets[0]), int(w.cand_offsets[1])
-    q = bf16_to_f64(w.q[c0:c1])
-    rb = max(lo, hi - 10_000)
-    zr = oracle.stca_branch(q, [0, c1 - c0], X, [rb - lo], [hi - lo], w.layers_r, w.heads, w.d_h)
-    zu = oracle.stca_branch(q, [0, c1 - c0], S[0], [0], [sa.k], w.layers_u, w.heads, w.d_h)
-    oracle.stca_fuse(zr, zu, w.W_F, w.b_F)
-    return hi - lo, time.perf_counter() - t0
+    events, secs = 0, 0.0
+    for u in users:
+        lo, hi = int(sa.offsets[u]), int(sa.offsets[u + 1])
+        if n_tokens is not None:
+            hi = min(hi, lo + n_tokens)
+        X = sa.x_f64(lo, hi)
+        t0 = time.perf_counter()
+        S, m, H = oracle.sa_forward(X, [0, hi - lo], sa.P, sa.W_Q, sa.W_K, sa.W_V, sa.eps)
+        oracle.sa_backward(X, [0, hi - lo], sa.P, sa.W_Q, sa.W_K, sa.W_V, sa.eps, sa.dS[u:u + 1])
+        c0, c1 = int(w.cand_offsets[u]), int(w.cand_offsets[u + 1])
+        q = bf16_to_f64(w.q[c0:c1])
+        rb = max(lo, hi - 10_000)
+        zr = oracle.stca_branch(q, [0, c1 - c0], X, [rb - lo], [hi - lo], w.layers_r, w.heads, w.d_h)
+        zu = oracle.stca_branch(q, [0, c1 - c0], S[0], [0], [sa.k], w.layers_u, w.heads, w.d_h)
+        oracle.stca_fuse(zr, zu, w.W_F, w.b_F)
+        secs += time.perf_counter() - t0
+        events += hi - lo
+    return events, secs
 
 
 def _cores():
@@ -540,11 +544,13 @@ def _cores():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, n_tokens=None):
-    n, secs = _oracle_sample(w, n_tokens)
+def cpu_baseline(w, n_tokens=None, n_users=10):
+    users = tuple(range(min(n_users, w.sa.B)))
+    n, secs = _oracle_sample(w, n_tokens, users)
     return {"value": n / secs, "unit": "history-tokens/s", "cores": _cores(), "kind": "oracle",
-            "sample": f"user 0 ({n} events) forward+backward, STCA on its 256 candidates "
-                      f"(both branches), fusion; fp64 numpy, {secs:.1f} s"}
+            "sample": f"users 0-{users[-1]}, the first {n_tokens} events of each ({n} events): "
+                      f"forward+backward, STCA on each user's 256 candidates (both branches), "
+                      f"fusion; fp64 numpy, {secs:.1f} s"}
 
 
 def run_reference(args):
