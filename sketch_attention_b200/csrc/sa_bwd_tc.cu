@@ -620,11 +620,10 @@ int sa_bwd_tc_dx_chunks() { return device_info().sm_count; }
 int sa_bwd_tc_e_chunks(int k) { return std::max(1, device_info().sm_count / (k / TILE)); }
 
 sa_status sa_bwd_tc_run(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st) {
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(sa_bwd_dx_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DX_SMEM);
-    cudaFuncSetAttribute(sa_bwd_e_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, E_SMEM);
-  });
+  static unsigned long long done_dx = 0, done_e = 0;
+  static std::mutex mu;
+  set_smem_limit_once((const void*)sa_bwd_dx_tc_kernel, DX_SMEM, &done_dx, mu);
+  set_smem_limit_once((const void*)sa_bwd_e_tc_kernel, E_SMEM, &done_e, mu);
   if (a.n_total >= (1LL << 31) || (int64_t)a.B * a.k >= (1LL << 31))
     return fail(SA_ERR_UNSUPPORTED, "row counts must be < 2^31");
   SA_TIMED("center_rows_kernel", st, (center_rows_kernel<<<a.B, 256, 0, st>>>(w.dm, a.k, w.dmc)));

@@ -377,10 +377,9 @@ sa_status stca_hist_ffn_tc(__nv_bfloat16* X, int64_t rows, const __nv_bfloat16* 
                            const __nv_bfloat16* W2t, cudaStream_t st) {
   if (rows <= 0) return SA_OK;
   if (rows >= (1LL << 31) - TM) return fail(SA_ERR_UNSUPPORTED, "history rows must be < 2^31 - 128");
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(stca_hist_ffn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
+  static unsigned long long done = 0;
+  static std::mutex mu;
+  set_smem_limit_once((const void*)stca_hist_ffn_tc_kernel, SMEM_BYTES, &done, mu);
   CUtensorMap tmX, tmW13, tmW2;
   sa_status s;
   if ((s = make_map(&tmX, X, DD, (uint64_t)rows, TM)) != SA_OK) return s;

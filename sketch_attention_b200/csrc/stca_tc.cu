@@ -263,6 +263,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 
+// ============================================================== host side
 sa_status make_map(CUtensorMap* map, const void* base, uint64_t rows) {
   return tma_map_bf16(map, base, DD, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
@@ -271,10 +272,9 @@ sa_status make_map(CUtensorMap* map, const void* base, uint64_t rows) {
 bool stca_tc_supported(sa_dtype dtype, int D) { return dtype == SA_BF16 && D == DD; }
 
 sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
-  static std::once_flag once;
-  std::call_once(once, [] {
-    cudaFuncSetAttribute(stca_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  });
+  static unsigned long long done = 0;
+  static std::mutex mu;
+  set_smem_limit_once((const void*)stca_attn_tc_kernel, SMEM_BYTES, &done, mu);
   if (a.kv_rows >= (1LL << 31) || a.C_total * a.heads >= (1LL << 31))
     return fail(SA_ERR_UNSUPPORTED, "row counts must be < 2^31");
   CUtensorMap tmU, tmK;

@@ -1,4 +1,4 @@
-// Tensor maps (TMA descriptors) of the tensor-core kernels: bf16 row-major
+// Tensor maps (TMA descriptors) of the tensor-core kernels, and their shared-memory limit: bf16 row-major
 // matrices [outer, inner] copied in boxes of box_inner x box_outer elements.
 // cuTensorMapEncodeTiled is taken from the driver once per process.  The
 // encoder checks the base (16-byte aligned), the row pitch (a multiple of 16
@@ -44,6 +44,16 @@ inline sa_status tma_map_bf16(CUtensorMap* map, const void* base, uint64_t inner
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
   return SA_OK;
+}
+
+// A kernel's dynamic shared-memory limit is an attribute of the device's context: set it once
+// per device (bit `device` of *done), under `mu`.
+inline void set_smem_limit_once(const void* kernel, int bytes, unsigned long long* done, std::mutex& mu) {
+  const int dev = device_info().device & 63;
+  std::lock_guard<std::mutex> lock(mu);
+  if (*done & (1ull << dev)) return;
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  *done |= 1ull << dev;
 }
 
 }  // namespace sa
