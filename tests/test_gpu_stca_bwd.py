@@ -127,3 +127,21 @@ def test_stca_backward_rejects_missing_gradient_buffer(lib):
                                        None, None, garr, ws.data_ptr(), ws.numel(), None)
     assert st == 1      # SA_ERR_INVALID_ARG
     assert b"gradient" in lib.load().sa_last_error()
+
+
+@pytest.mark.parametrize("which", ["recent", "sketch"])
+def test_stca_backward_full_size_one_user(lib, which):
+    """The bench's STCA-backward shapes for one user (512 candidates x 4 heads, a 10K
+    suffix or a 1024-row sketch, two full layers): every gradient against the oracle.
+    The weight gradients of a batch are sums of such per-user terms."""
+    from sa_inputs import make_stca_problem
+    prob = make_stca_problem(1, (512,), (10_000,), 1024, 128, 4, 32, 2, "bf16", seed=620)
+    add_stca_ffns(rng_for(621), prob.layers_r, 128)
+    add_stca_ffns(rng_for(622), prob.layers_u, 128)
+    br = prob.recent if which == "recent" else prob.sketch
+    layers = prob.layers_r if which == "recent" else prob.layers_u
+    dout = gauss(rng_for(623), (512, 128), 1.0)
+    p = dict(layers=layers, cand=br.cand_offsets, q=br.q, kv=br.kv, kb=br.kv_begin, ke=br.kv_end, dout=dout,
+             heads=4, d_h=32, dtype="bf16")
+    errs = _check(lib, p)
+    print(which, {k: round(v["max_rel"], 8) for k, v in errs.items()})
