@@ -634,14 +634,15 @@ sa_status stca_forward_full(const void* q, sa_dtype dtype, const int64_t* cand_o
 namespace {
 // Shape of a backward call from its host offsets (no validation beyond sizes).
 StcaBwdShape bwd_shape(int B, const int64_t* cand, const int64_t* kb, const int64_t* ke, int D, int heads,
-                       int d_h, int n_layers) {
+                       int d_h, int n_layers, sa_dtype dtype) {
   StcaBwdShape sh{};
   sh.C = cand[B];
   for (int u = 0; u < B; ++u) {
     sh.kv_total += ke[u] - kb[u];
-    sh.max_rows_x_keys = std::max(sh.max_rows_x_keys, (cand[u + 1] - cand[u]) * heads * (ke[u] - kb[u]));
+    sh.max_rows_x_keys =
+        std::max(sh.max_rows_x_keys, (cand[u + 1] - cand[u]) * heads * score_pitch(ke[u] - kb[u]));
   }
-  sh.D = D; sh.heads = heads; sh.d_h = d_h; sh.n_layers = n_layers;
+  sh.D = D; sh.heads = heads; sh.d_h = d_h; sh.n_layers = n_layers; sh.dtype = dtype;
   return sh;
 }
 }  // namespace
@@ -682,7 +683,7 @@ size_t stca_backward_full_workspace(int B, const int64_t* cand_offsets_host, con
   for (int u = 0; u < B; ++u)
     if (kv_end_host[u] < kv_begin_host[u] || cand_offsets_host[u + 1] < cand_offsets_host[u]) return 0;
   return stca_bwd_layout(nullptr, bwd_shape(B, cand_offsets_host, kv_begin_host, kv_end_host, D, heads, d_h,
-                                            n_layers), nullptr);
+                                            n_layers, dtype), nullptr);
 }
 
 sa_status stca_backward_full(const void* q, sa_dtype dtype, const int64_t* cand_offsets_host,
@@ -718,7 +719,7 @@ sa_status stca_backward_full(const void* q, sa_dtype dtype, const int64_t* cand_
   SA_TRY(check_ptr(dout, "dout", C == 0));
   SA_TRY(check_ptr(dq, "dq", true));
   SA_TRY(check_ptr(dkv, "dkv", true));
-  const StcaBwdShape sh = bwd_shape(B, cand_offsets_host, kv_begin_host, kv_end_host, D, heads, d_h, n_layers);
+  const StcaBwdShape sh = bwd_shape(B, cand_offsets_host, kv_begin_host, kv_end_host, D, heads, d_h, n_layers, dtype);
   if (sh.max_rows_x_keys >= (1LL << 31) || sh.kv_total >= (1LL << 31) || C * heads >= (1LL << 31))
     return fail(SA_ERR_UNSUPPORTED, "a user's score matrix or the row counts must be < 2^31 elements");
   const size_t need = stca_bwd_layout(nullptr, sh, nullptr);

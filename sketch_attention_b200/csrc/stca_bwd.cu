@@ -11,8 +11,10 @@
 //   dP = dY X^T,  dS = P o (dP - rowsum(dY o Y)),  dU = dS X,
 //   dX += dS^T U + P^T dY        (K = V = X)
 // then the head projections, W_O and the two SwiGLU FFNs by their chain
-// rules.  Every contraction is the projection GEMM; users are processed in
-// order on the stream, so the results are deterministic.
+// rules.  With bf16 inputs the six attention products per user and layer run
+// on the tensor cores (tc_gemm.cu) with bf16 copies of U, X, dY, P and dS; with
+// fp32 inputs, and for every other contraction, the fp32 projection GEMM.
+// Users are processed in order on the stream, so the results are deterministic.
 #include <algorithm>
 #include <cmath>
 
@@ -42,10 +44,13 @@ __global__ void add_rows_kernel(const float* __restrict__ src, int64_t n, float*
     dst[e] += src[e];
 }
 
-// softmax of each row of S [rows, L] in place (one block per row)
-__global__ void __launch_bounds__(256) softmax_rows_kernel(float* __restrict__ S, int64_t L) {
+// softmax of each row of S [rows, L] (row pitch ld) in place, and its bf16 split
+// Pb + Plo (same pitch) when given; one block per row
+__global__ void __launch_bounds__(256) softmax_rows_kernel(float* __restrict__ S, int64_t L, int64_t ld,
+                                                          __nv_bfloat16* __restrict__ Pb,
+                                                          __nv_bfloat16* __restrict__ Plo) {
   __shared__ float red[8];
-  float* row = S + (int64_t)blockIdx.x * L;
+  float* row = S + (int64_t)blockIdx.x * ld;
   const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
   float m = -INFINITY;
   for (int64_t j = threadIdx.x; j < L; j += 256) m = fmaxf(m, row[j]);
@@ -67,13 +72,24 @@ __global__ void __launch_bounds__(256) softmax_rows_kernel(float* __restrict__ S
   s = 0.f;
   for (int i = 0; i < 8; ++i) s += red[i];
   const float inv = 1.f / s;
-  for (int64_t j = threadIdx.x; j < L; j += 256) row[j] *= inv;
+  for (int64_t j = threadIdx.x; j < L; j += 256) {
+    const float v = row[j] * inv;
+    row[j] = v;
+    if (Pb) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      Pb[(int64_t)blockIdx.x * ld + j] = hi;
+      Plo[(int64_t)blockIdx.x * ld + j] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    }
+  }
 }
 
-// dS = P o (dP - sum_d dY[r, d] Y[r, d]) in place over dP (one block per row)
+// dS = P o (dP - sum_d dY[r, d] Y[r, d]) in place over dP (row pitch ld), and its bf16
+// split dSb + dSlo (same pitch) when given; one block per row
 __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* __restrict__ P, float* __restrict__ dP,
-                                                          int64_t L, const float* __restrict__ dY,
-                                                          const float* __restrict__ Y, int D) {
+                                                          int64_t L, int64_t ld, const float* __restrict__ dY,
+                                                          const float* __restrict__ Y, int D,
+                                                          __nv_bfloat16* __restrict__ dSb,
+                                                          __nv_bfloat16* __restrict__ dSlo) {
   __shared__ float red[8];
   const int64_t r = blockIdx.x;
   float v = 0.f;
@@ -83,7 +99,27 @@ __global__ void __launch_bounds__(256) softmax_bwd_kernel(const float* __restric
   __syncthreads();
   float c = 0.f;
   for (int i = 0; i < 8; ++i) c += red[i];
-  for (int64_t j = threadIdx.x; j < L; j += 256) dP[r * L + j] = P[r * L + j] * (dP[r * L + j] - c);
+  for (int64_t j = threadIdx.x; j < L; j += 256) {
+    const float v = P[r * ld + j] * (dP[r * ld + j] - c);
+    dP[r * ld + j] = v;
+    if (dSb) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      dSb[r * ld + j] = hi;
+      dSlo[r * ld + j] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    }
+  }
+}
+
+// x = hi + lo with both in bf16 (hi the rounding of x, lo the rounding of the rest):
+// products over hi and lo carry x to about 16 bits
+__global__ void split_kernel(const float* __restrict__ in, int64_t n, __nv_bfloat16* __restrict__ hi,
+                             __nv_bfloat16* __restrict__ lo) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float x = in[e];
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    hi[e] = h;
+    lo[e] = __float2bfloat16_rn(x - __bfloat162float(h));
+  }
 }
 
 // dG1 = dU o G3 o SiLU'(G1), dG3 = dU o SiLU(G1); SiLU'(g) = s (1 + g (1 - s)), s = 1/(1+e^-g).
@@ -139,6 +175,27 @@ struct Ffn {
   const float *W1, *W3, *W2;
   float *dW1, *dW3, *dW2;
 };
+
+// a bf16 split x = hi + lo of an fp32 operand
+struct Split {
+  const __nv_bfloat16 *hi, *lo;
+  Split at(int64_t off) const { return {hi + off, lo + off}; }
+};
+
+// C[M, N] = A B (+ Cin) on the tensor cores over split operands (about 16 significant
+// bits each): A K-major or (a_mn) M-major, B K-major or (b_mn) N-major
+sa_status tc(int M, int N, int K, Split A, int64_t lda, bool a_mn, Split B, int64_t ldb, bool b_mn, float* C,
+             int64_t ldc, const float* Cin, const Ctx& cx) {
+  cudaStream_t st = cx.st;
+  TcGemm g;
+  g.part = cx.split; g.part_floats = kStcaBwdSplitFloats;
+  g.M = M; g.N = N; g.K = K;
+  g.A = A.hi; g.A_lo = A.lo; g.lda = lda; g.a_mn = a_mn;
+  g.B = B.hi; g.B_lo = B.lo; g.ldb = ldb; g.b_mn = b_mn;
+  g.C = C; g.ldc = ldc; g.Cin = Cin; g.ldcin = ldc;
+  g.tag = "tc_gemm:stca_bwd_attn";
+  return tc_gemm(g, st);
+}
 
 // y = x + FFN(x) over `rows` rows
 sa_status ffn_fwd(const float* x, int64_t rows, int D, const Ffn& f, float* G1, float* G3, float* U, float* y,
@@ -206,6 +263,17 @@ size_t stca_bwd_layout(void* base, const StcaBwdShape& sh, StcaBwdWork* w) {
   const size_t sl = (size_t)std::max<int64_t>(sh.max_rows_x_keys, 1);
   v.S = c.take<float>(sl);
   v.dS = c.take<float>(sl);
+  const bool tc = sh.dtype == SA_BF16;        // bf16 inputs: the attention products on the tensor cores
+  v.Ub = c.take<__nv_bfloat16>(tc ? NL * C * H * D : 1);
+  v.Ulo = c.take<__nv_bfloat16>(tc ? NL * C * H * D : 1);
+  v.Xkb = c.take<__nv_bfloat16>(tc ? NL * R * D : 1);
+  v.Xklo = c.take<__nv_bfloat16>(tc ? NL * R * D : 1);
+  v.dYb = c.take<__nv_bfloat16>(tc ? C * H * D : 1);
+  v.dYlo = c.take<__nv_bfloat16>(tc ? C * H * D : 1);
+  v.Pb = c.take<__nv_bfloat16>(tc ? sl : 1);
+  v.Plo = c.take<__nv_bfloat16>(tc ? sl : 1);
+  v.dSb = c.take<__nv_bfloat16>(tc ? sl : 1);
+  v.dSlo = c.take<__nv_bfloat16>(tc ? sl : 1);
   v.dq = c.take<float>(C * D);
   v.dqmid = c.take<float>(C * D);
   v.dO = c.take<float>(C * HD);
@@ -227,6 +295,7 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
   const float inv_sqrt = 1.f / std::sqrt((float)dh);
   sa_status s;
   const Ctx cx{st, w.gsplit};
+  const bool tcp = a.dtype == SA_BF16;       // the attention products on the tensor cores
   // ---------------------------------------------------------------- inputs, widened
   if (C > 0) {
     if (a.dtype == SA_BF16)
@@ -264,6 +333,10 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
       SA_CUDA(cudaMemcpyAsync(Xs(l + 1), Xs(l), sizeof(float) * RD, cudaMemcpyDeviceToDevice, st));
     }
     const float* X = Xs(l + 1);
+    const Split Xb{w.Xkb + (size_t)l * RD, w.Xklo + (size_t)l * RD};   // its bf16 split (tensor-core path)
+    if (tcp && R > 0)
+      SA_TIMED("split_kernel", st, (split_kernel<<<grid_for(RD), 256, 0, st>>>(X, RD, w.Xkb + (size_t)l * RD,
+                                                                               w.Xklo + (size_t)l * RD)));
     if (C == 0) continue;
     // Qh[:, h] = q W_Q^h;  U[c*H + h] = Qh[:, h] W_K^h^T / sqrt(d_h)
     Gemm g1 = plain((int)C, dh, D, qin, D, false, L.attn.W_Q, dh, false, Qh, HD, "gemm:stca_bwd_proj");
@@ -272,6 +345,10 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
     Gemm g2 = plain((int)C, D, dh, Qh, HD, false, L.attn.W_K, dh, true, U, (int64_t)H * D, "gemm:stca_bwd_proj");
     g2.batch = H; g2.sA = dh; g2.sB = (int64_t)D * dh; g2.sC = D; g2.alpha = inv_sqrt;
     if ((s = mm(g2, cx)) != SA_OK) return s;
+    const Split Ub{w.Ub + (size_t)l * CHD2, w.Ulo + (size_t)l * CHD2};
+    if (tcp)
+      SA_TIMED("split_kernel", st, (split_kernel<<<grid_for(CHD2), 256, 0, st>>>(U, CHD2, w.Ub + (size_t)l * CHD2,
+                                                                                 w.Ulo + (size_t)l * CHD2)));
     // per user: S = U_u X_u^T, P = softmax, Y_u = P X_u
     for (int u = 0; u < B; ++u) {
       const int64_t r0 = hst.cand[u] * H, ru = (hst.cand[u + 1] - hst.cand[u]) * H;
@@ -283,9 +360,18 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
         continue;
       }
       const float* Xu = X + (size_t)hst.kpre[u] * D;
-      if ((s = mm(plain((int)ru, (int)lu, D, U + (size_t)r0 * D, D, false, Xu, D, true, w.S, lu, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
-      SA_TIMED("softmax_rows_kernel", st, (softmax_rows_kernel<<<(unsigned)ru, 256, 0, st>>>(w.S, lu)));
-      if ((s = mm(plain((int)ru, D, (int)lu, w.S, lu, false, Xu, D, false, Yu, D, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
+      const int64_t lp = score_pitch(lu);
+      if (tcp) {
+        const Split Xbu = Xb.at((int64_t)hst.kpre[u] * D), Ubu = Ub.at(r0 * D), Pb{w.Pb, w.Plo};
+        if ((s = tc((int)ru, (int)lu, D, Ubu, D, false, Xbu, D, false, w.S, lp, nullptr, cx)) != SA_OK) return s;
+        SA_TIMED("softmax_rows_kernel", st, (softmax_rows_kernel<<<(unsigned)ru, 256, 0, st>>>(w.S, lu, lp, w.Pb,
+                                                                                                w.Plo)));
+        if ((s = tc((int)ru, D, (int)lu, Pb, lp, false, Xbu, D, true, Yu, D, nullptr, cx)) != SA_OK) return s;
+      } else {
+        if ((s = mm(plain((int)ru, (int)lu, D, U + (size_t)r0 * D, D, false, Xu, D, true, w.S, lp, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
+        SA_TIMED("softmax_rows_kernel", st, (softmax_rows_kernel<<<(unsigned)ru, 256, 0, st>>>(w.S, lu, lp, nullptr, nullptr)));
+        if ((s = mm(plain((int)ru, D, (int)lu, w.S, lp, false, Xu, D, false, Yu, D, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
+      }
     }
     // O[:, h] = Y_h W_V^h;  qmid = q + O W_O (or q + O)
     Gemm g3 = plain((int)C, dh, D, Y, (int64_t)H * D, false, L.attn.W_V, dh, false, O, HD, "gemm:stca_bwd_proj");
@@ -344,6 +430,8 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
     Gemm gy = plain((int)C, D, dh, w.dO, HD, false, L.attn.W_V, dh, true, w.dY, (int64_t)H * D, "gemm:stca_bwd_proj");
     gy.batch = H; gy.sA = dh; gy.sB = (int64_t)D * dh; gy.sC = D;
     if ((s = mm(gy, cx)) != SA_OK) return s;
+    if (tcp && C > 0)
+      SA_TIMED("split_kernel", st, (split_kernel<<<grid_for(CHD2), 256, 0, st>>>(w.dY, CHD2, w.dYb, w.dYlo)));
     if (C > 0) {
       Gemm gv = plain(D, dh, (int)C, Y, (int64_t)H * D, true, w.dO, HD, false, Gd.dW_V, dh, "gemm:stca_bwd_proj");
       gv.batch = H; gv.sA = D; gv.sB = dh; gv.sC = (int64_t)D * dh;
@@ -365,16 +453,36 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
       const float* Uu = U + (size_t)r0 * D;
       const float* dYu = w.dY + (size_t)r0 * D;
       float* dXu = w.dX + (size_t)hst.kpre[u] * D;
-      if ((s = mm(plain((int)ru, (int)lu, D, Uu, D, false, Xu, D, true, w.S, lu, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
-      SA_TIMED("softmax_rows_kernel", st, (softmax_rows_kernel<<<(unsigned)ru, 256, 0, st>>>(w.S, lu)));
-      if ((s = mm(plain((int)ru, (int)lu, D, dYu, D, false, Xu, D, true, w.dS, lu, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
+      const int64_t lp = score_pitch(lu);
+      if (tcp) {
+        const Split Xbu{w.Xkb + (size_t)l * RD + (size_t)hst.kpre[u] * D,
+                        w.Xklo + (size_t)l * RD + (size_t)hst.kpre[u] * D};
+        const Split Ubu{w.Ub + (size_t)l * CHD2 + (size_t)r0 * D, w.Ulo + (size_t)l * CHD2 + (size_t)r0 * D};
+        const Split dYbu{w.dYb + (size_t)r0 * D, w.dYlo + (size_t)r0 * D};
+        const Split Pb{w.Pb, w.Plo}, dSb{w.dSb, w.dSlo};
+        if ((s = tc((int)ru, (int)lu, D, Ubu, D, false, Xbu, D, false, w.S, lp, nullptr, cx)) != SA_OK) return s;
+        SA_TIMED("softmax_rows_kernel", st, (softmax_rows_kernel<<<(unsigned)ru, 256, 0, st>>>(w.S, lu, lp, w.Pb,
+                                                                                                w.Plo)));
+        // dP = dY X^T, then dS = P o (dP - <dY, Y>)
+        if ((s = tc((int)ru, (int)lu, D, dYbu, D, false, Xbu, D, false, w.dS, lp, nullptr, cx)) != SA_OK) return s;
+        SA_TIMED("softmax_bwd_kernel", st, (softmax_bwd_kernel<<<(unsigned)ru, 256, 0, st>>>(
+                                               w.S, w.dS, lu, lp, dYu, Y + (size_t)r0 * D, D, w.dSb, w.dSlo)));
+        // dU = dS X;  dX += dS^T U + P^T dY  (the transposed score matrices are M-major operands)
+        if ((s = tc((int)ru, D, (int)lu, dSb, lp, false, Xbu, D, true, dUu, D, nullptr, cx)) != SA_OK) return s;
+        if ((s = tc((int)lu, D, (int)ru, dSb, lp, true, Ubu, D, true, dXu, D, dXu, cx)) != SA_OK) return s;
+        if ((s = tc((int)lu, D, (int)ru, Pb, lp, true, dYbu, D, true, dXu, D, dXu, cx)) != SA_OK) return s;
+        continue;
+      }
+      if ((s = mm(plain((int)ru, (int)lu, D, Uu, D, false, Xu, D, true, w.S, lp, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
+      SA_TIMED("softmax_rows_kernel", st, (softmax_rows_kernel<<<(unsigned)ru, 256, 0, st>>>(w.S, lu, lp, nullptr, nullptr)));
+      if ((s = mm(plain((int)ru, (int)lu, D, dYu, D, false, Xu, D, true, w.dS, lp, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
       SA_TIMED("softmax_bwd_kernel", st, (softmax_bwd_kernel<<<(unsigned)ru, 256, 0, st>>>(
-                                             w.S, w.dS, lu, dYu, Y + (size_t)r0 * D, D)));
-      if ((s = mm(plain((int)ru, D, (int)lu, w.dS, lu, false, Xu, D, false, dUu, D, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
-      Gemm gk = plain((int)lu, D, (int)ru, w.dS, lu, true, Uu, D, false, dXu, D, "gemm:stca_bwd_attn");
+                                             w.S, w.dS, lu, lp, dYu, Y + (size_t)r0 * D, D, nullptr, nullptr)));
+      if ((s = mm(plain((int)ru, D, (int)lu, w.dS, lp, false, Xu, D, false, dUu, D, "gemm:stca_bwd_attn"), cx)) != SA_OK) return s;
+      Gemm gk = plain((int)lu, D, (int)ru, w.dS, lp, true, Uu, D, false, dXu, D, "gemm:stca_bwd_attn");
       gk.Cin = dXu; gk.ldcin = D;
       if ((s = mm(gk, cx)) != SA_OK) return s;
-      Gemm gvv = plain((int)lu, D, (int)ru, w.S, lu, true, dYu, D, false, dXu, D, "gemm:stca_bwd_attn");
+      Gemm gvv = plain((int)lu, D, (int)ru, w.S, lp, true, dYu, D, false, dXu, D, "gemm:stca_bwd_attn");
       gvv.Cin = dXu; gvv.ldcin = D;
       if ((s = mm(gvv, cx)) != SA_OK) return s;
     }

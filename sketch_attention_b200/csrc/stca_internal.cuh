@@ -46,11 +46,32 @@ size_t stca_full_layout(void* base, int B, int64_t C, int64_t kv_total, int D, i
 sa_status stca_full_run(const StcaArgs& a, const stca_full_layer* layers, int64_t kv_total,
                         const StcaFullWork& w, cudaStream_t st);
 
+// bf16 tensor-core GEMM: C[M, N] = alpha A B (+ Cin), fp32 out.  A is K-major
+// (A[m lda + k]) or, with a_mn, M-major (A[k lda + m]); B is K-major (B[n ldb + k])
+// or, with b_mn, N-major (B[k ldb + n]).  lda, ldb multiples of 8; A, B 16-byte aligned.
+struct TcGemm {
+  int M = 0, N = 0, K = 0;
+  const __nv_bfloat16* A = nullptr; int64_t lda = 0; bool a_mn = false;
+  const __nv_bfloat16* B = nullptr; int64_t ldb = 0; bool b_mn = false;
+  const __nv_bfloat16* A_lo = nullptr;     // optional lo parts of split operands (same layout)
+  const __nv_bfloat16* B_lo = nullptr;
+  float* part = nullptr;                   // optional split-K workspace of part_floats floats
+  size_t part_floats = 0;
+  float* C = nullptr; int64_t ldc = 0;
+  const float* Cin = nullptr; int64_t ldcin = 0;
+  float alpha = 1.f;
+  const char* tag = nullptr;
+};
+sa_status tc_gemm(const TcGemm& g, cudaStream_t st);
+
 // Backward of a branch of full layers (fp32, GEMM-based).
 struct StcaBwdShape {
-  int64_t C, kv_total, max_rows_x_keys;   // max over users of C_u * heads * (kv_end - kv_begin)
+  int64_t C, kv_total, max_rows_x_keys;   // max over users of C_u * heads * pitch(kv_end - kv_begin)
   int D, heads, d_h, n_layers;
+  sa_dtype dtype;
 };
+// row pitch of a user's score matrix: its key count rounded up to 8 (16-byte rows in bf16)
+inline int64_t score_pitch(int64_t keys) { return (keys + 7) / 8 * 8; }
 struct StcaBwdHost {                      // host copies of the offsets, read while issuing
   const int64_t* cand;                    // [B+1]
   const int64_t* kv_begin;                // [B]
@@ -65,6 +86,8 @@ struct StcaBwdWork {
   float *S, *dS;                          // one user's score matrix and its gradient
   float *dq, *dqmid, *dO, *dY, *dU, *dQh, *dX;
   float* gsplit;                          // split-K partials of the GEMMs with small outputs
+  // bf16 operands of the tensor-core attention products (bf16 inputs only)
+  __nv_bfloat16 *Ub, *Ulo, *Xkb, *Xklo, *dYb, *dYlo, *Pb, *Plo, *dSb, *dSlo;
 };
 constexpr size_t kStcaBwdSplitFloats = (size_t)16 << 20;
 size_t stca_bwd_layout(void* base, const StcaBwdShape& sh, StcaBwdWork* w);

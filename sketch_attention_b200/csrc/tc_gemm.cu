@@ -1,0 +1,260 @@
+// bf16 GEMM on the sm_100a tensor cores for the STCA backward's attention
+// products: C[M, N] = alpha A B (+ Cin), fp32 accumulation and output.
+// An operand may come as a split pair x = hi + lo (both bf16, lo the rounding of
+// x - hi): the K loop then runs again over hi x lo and lo x hi into the same
+// accumulator (lo x lo, below 2^-16 of the product, is dropped), which carries
+// fp32 operands to about 16 significant bits on the bf16 tensor cores.
+//
+// A is [M, K], stored K-major (A[m lda + k]) or M-major (A[k lda + m]); B is
+// [K, N], stored K-major (B[n ldb + k]) or N-major (B[k ldb + n]).  One CTA per
+// 128 x 128 output tile: TMA brings 64-deep K slices of both operands into a
+// four-stage ring (128-byte swizzle; a K-major operand is one 64 x 128 box, an
+// MN-major one two 64 x 64 boxes), one thread issues the MMAs (M = 128,
+// N = 128, K = 16) into a TMEM accumulator, and four warps write the tile.
+// Edges are zero-filled by the TMA and masked in the epilogue.  A deep K over few
+// output tiles is split across CTAs (grid z): each writes its raw partial tile to a
+// workspace slice and a second kernel adds the slices in order (deterministic).
+#include <algorithm>
+#include <mutex>
+
+#include "stca_internal.cuh"
+#include "tc_ptx.cuh"
+#include "tma_map.cuh"
+
+namespace sa {
+
+namespace {
+using namespace tc;
+
+constexpr int TM = 128, TN = 128, TK = 64, NST = 4, THREADS = 192;
+constexpr uint32_t OP_BYTES = TM * TK * 2;                 // 16 KB per operand per stage
+constexpr uint32_t STAGE = 2 * OP_BYTES;
+constexpr uint32_t OFF_BAR = NST * STAGE;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
+constexpr uint32_t TM_COLS = 128;
+
+struct Bars {
+  uint64_t full[NST], empty[NST], done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+struct Params {
+  int M, N, K;
+  int ph_alo, ph_blo;     // the K-loop pass that reads A's (B's) lo part; -1: none
+  float* C;
+  int64_t ldc;
+  const float* Cin;
+  int64_t ldcin;
+  float alpha;
+  int kt_per;             // K slices (of TK) per split; the split index is blockIdx.z
+  float* part;            // split > 1: raw partial tiles, [split][M][N]
+  int* err;
+};
+
+// the smem descriptor of K-step ks (16 deep) of a 64-deep operand slice
+__device__ __forceinline__ uint64_t op_desc(uint32_t base, int ks, bool mn) {
+  return mn ? smem_desc(base + ks * 2048, OP_BYTES / 2, 1024, SWZ_128B)   // two 64-wide MN atoms
+            : smem_desc(base + ks * 32, 16, 1024, SWZ_128B);              // 128 rows, K along the row
+}
+
+template <bool AMN, bool BMN>
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAl,
+                   const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBl, Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  Bars* bars = (Bars*)(smem + OFF_BAR);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
+  const int kt0 = blockIdx.z * p.kt_per;
+  const int nk = min(p.kt_per, (p.K + TK - 1) / TK - kt0);        // >= 1 (the host sizes the split)
+  const int nit = nk * (1 + (p.ph_alo >= 0) + (p.ph_blo >= 0));   // K slices over all passes
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) { mbar_init(&bars->full[s], 1); mbar_init(&bars->empty[s], 1); }
+    mbar_init(&bars->done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars->tmem_base, TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    if (p.ph_alo >= 0) prefetch_tensormap(&tmAl);
+    if (p.ph_blo >= 0) prefetch_tensormap(&tmBl);
+    int issued = 0;
+    for (int it = 0; it < nit; ++it) {
+      const int s = it % NST, ph = it / nk, k0 = (kt0 + it % nk) * TK;
+      const CUtensorMap* ma = ph == p.ph_alo ? &tmAl : &tmA;
+      const CUtensorMap* mb = ph == p.ph_blo ? &tmBl : &tmB;
+      if (it >= NST && !mbar_wait(&bars->empty[s], ((it / NST) - 1) & 1, abort, p.err)) break;
+      mbar_arrive_expect_tx(&bars->full[s], STAGE);
+      uint8_t* a = smem + s * STAGE;
+      uint8_t* b = a + OP_BYTES;
+      if (AMN) {
+        tma_load_2d(a, ma, &bars->full[s], m0, k0);
+        tma_load_2d(a + OP_BYTES / 2, ma, &bars->full[s], m0 + 64, k0);
+      } else {
+        tma_load_2d(a, ma, &bars->full[s], k0, m0);
+      }
+      if (BMN) {
+        tma_load_2d(b, mb, &bars->full[s], n0, k0);
+        tma_load_2d(b + OP_BYTES / 2, mb, &bars->full[s], n0 + 64, k0);
+      } else {
+        tma_load_2d(b, mb, &bars->full[s], k0, n0);
+      }
+      issued = it + 1;
+    }
+    if (*abort)
+      for (int it = std::max(0, issued - NST); it < issued; ++it)
+        mbar_wait_bounded(&bars->full[it % NST], (it / NST) & 1);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA
+    const uint32_t id = idesc_bf16(128, 128, AMN, BMN);
+    for (int it = 0; it < nit; ++it) {
+      const int s = it % NST;
+      if (!mbar_wait(&bars->full[s], (it / NST) & 1, abort, p.err)) break;
+      tc_fence_after();
+      const uint32_t a = smem_u32(smem + s * STAGE), b = a + OP_BYTES;
+#pragma unroll
+      for (int ks = 0; ks < TK / 16; ++ks)
+        mma_ss(tmem, op_desc(a, ks, AMN), op_desc(b, ks, BMN), id, (it > 0 || ks > 0) ? 1u : 0u);
+      mma_commit(&bars->empty[s]);
+    }
+    mma_commit(&bars->done);
+    mbar_wait_bounded(&bars->done, 0);
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue: one row per thread
+    const int q = warp % 4;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    if (mbar_wait(&bars->done, 0, abort, p.err)) {
+      tc_fence_after();
+      const int m = m0 + row;
+#pragma unroll 1
+      for (int c = 0; c < TN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_addr + 32 * c, v);
+        tmem_wait_ld();
+        if (m >= p.M) continue;
+        const int nb = n0 + 32 * c;
+        if (p.part) {
+          float* dst = p.part + ((int64_t)blockIdx.z * p.M + m) * p.N + nb;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (nb + i < p.N) dst[i] = v[i];
+          continue;
+        }
+        float* dst = p.C + (int64_t)m * p.ldc + nb;
+        const float* cin = p.Cin ? p.Cin + (int64_t)m * p.ldcin + nb : nullptr;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          if (nb + i < p.N) {
+            float x = p.alpha * v[i];
+            if (cin) x += cin[i];
+            dst[i] = x;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TM_COLS);
+  }
+}
+
+// C = alpha sum_z part[z] (+ Cin), the slices added in order
+__global__ void tc_gemm_reduce_kernel(const float* __restrict__ part, int splits, int M, int N, float* C,
+                                      int64_t ldc, const float* Cin, int64_t ldcin, float alpha) {
+  const int64_t mn = (int64_t)M * N;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < mn; e += (int64_t)gridDim.x * blockDim.x) {
+    float v = 0.f;
+    for (int z = 0; z < splits; ++z) v += part[z * mn + e];
+    const int64_t m = e / N, n = e % N;
+    v *= alpha;
+    if (Cin) v += Cin[m * ldcin + n];
+    C[m * ldc + n] = v;
+  }
+}
+
+template <bool AMN, bool BMN>
+void set_limit() {
+  static unsigned long long done = 0;
+  static std::mutex mu;
+  set_smem_limit_once((const void*)tc_gemm_kernel<AMN, BMN>, SMEM_BYTES, &done, mu);
+}
+}  // namespace
+
+sa_status tc_gemm(const TcGemm& g, cudaStream_t st) {
+  if (g.M <= 0 || g.N <= 0) return SA_OK;
+  if (g.K <= 0) return fail(SA_ERR_INVALID_ARG, "tc_gemm: K must be positive");
+  if (g.lda % 8 || g.ldb % 8) return fail(SA_ERR_INVALID_ARG, "tc_gemm: leading dimensions must be multiples of 8");
+  if ((g.M + TM - 1) / TM > 65535) return fail(SA_ERR_UNSUPPORTED, "tc_gemm: too many row tiles");
+  CUtensorMap tmA, tmAl, tmB, tmBl;
+  // A: K-major [M rows of lda] or M-major [K rows of lda]; B: K-major [N rows] or N-major [K rows]
+  // (the extents are the matrix's, the pitch its leading dimension, so a tail reads as zero)
+  auto map_a = [&](CUtensorMap* m, const __nv_bfloat16* x) {
+    return g.a_mn ? tma_map_bf16(m, x, (uint64_t)g.M, (uint64_t)g.K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, g.lda)
+                  : tma_map_bf16(m, x, (uint64_t)g.K, (uint64_t)g.M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, g.lda);
+  };
+  auto map_b = [&](CUtensorMap* m, const __nv_bfloat16* x) {
+    return g.b_mn ? tma_map_bf16(m, x, (uint64_t)g.N, (uint64_t)g.K, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B, g.ldb)
+                  : tma_map_bf16(m, x, (uint64_t)g.K, (uint64_t)g.N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B, g.ldb);
+  };
+  sa_status s;
+  if ((s = map_a(&tmA, g.A)) != SA_OK || (s = map_b(&tmB, g.B)) != SA_OK) return s;
+  tmAl = tmA;
+  tmBl = tmB;
+  if (g.A_lo && (s = map_a(&tmAl, g.A_lo)) != SA_OK) return s;
+  if (g.B_lo && (s = map_b(&tmBl, g.B_lo)) != SA_OK) return s;
+  // passes: hi x hi, then hi x lo (B split), then lo x hi (A split)
+  const int ph_blo = g.B_lo ? 1 : -1;
+  const int ph_alo = g.A_lo ? (g.B_lo ? 2 : 1) : -1;
+  // split K while the output tiles fill less than the SMs, keeping >= 8 K slices a split
+  const int tiles = ((g.N + TN - 1) / TN) * ((g.M + TM - 1) / TM), nk = (g.K + TK - 1) / TK;
+  const int kSMs = device_info().sm_count;
+  int split = 1;
+  if (g.part && tiles < kSMs) {
+    split = std::min({(kSMs + tiles - 1) / tiles, std::max(1, nk / 8), 64});
+    split = (int)std::min<int64_t>(split, (int64_t)(g.part_floats / ((size_t)g.M * g.N)));
+    split = std::max(split, 1);
+  }
+  const int kt_per = (nk + split - 1) / split;
+  split = (nk + kt_per - 1) / kt_per;            // every split gets >= 1 slice
+  Params p{g.M, g.N, g.K, ph_alo, ph_blo, g.C, g.ldc, g.Cin, g.ldcin, g.alpha, kt_per,
+           split > 1 ? g.part : nullptr, device_status_word()};
+  dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, split);
+  const char* tag = g.tag ? g.tag : "tc_gemm_kernel";
+  if (g.a_mn) {
+    if (g.b_mn) { set_limit<true, true>(); SA_TIMED(tag, st, (tc_gemm_kernel<true, true><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p))); }
+    else { set_limit<true, false>(); SA_TIMED(tag, st, (tc_gemm_kernel<true, false><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p))); }
+  } else {
+    if (g.b_mn) { set_limit<false, true>(); SA_TIMED(tag, st, (tc_gemm_kernel<false, true><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p))); }
+    else { set_limit<false, false>(); SA_TIMED(tag, st, (tc_gemm_kernel<false, false><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p))); }
+  }
+  if (split > 1) {
+    const int64_t mn = (int64_t)g.M * g.N;
+    const unsigned blocks = (unsigned)std::min<int64_t>((mn + 255) / 256, 4 * kSMs);
+    SA_TIMED("tc_gemm_reduce_kernel", st,
+             (tc_gemm_reduce_kernel<<<blocks, 256, 0, st>>>(g.part, split, g.M, g.N, g.C, g.ldc, g.Cin, g.ldcin,
+                                                            g.alpha)));
+  }
+  return SA_OK;
+}
+
+}  // namespace sa

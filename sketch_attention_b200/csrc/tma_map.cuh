@@ -31,12 +31,15 @@ inline TmaEncodeFn tma_encode_fn() {
   return fn;
 }
 
+// pitch: elements between consecutive rows (default: inner); elements past `inner`
+// or `outer` read as zero
 inline sa_status tma_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
-                              uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+                              uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz,
+                              uint64_t pitch = 0) {
   TmaEncodeFn enc = tma_encode_fn();
   if (!enc) return fail(SA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {inner * 2};
+  cuuint64_t strides[1] = {(pitch ? pitch : inner) * 2};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,

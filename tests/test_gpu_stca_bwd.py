@@ -1,7 +1,9 @@
 """GPU parity of stca_backward_full (the STCA backward through the attention, W_O
 and both SwiGLU FFNs of the full layer) against the fp64 oracle's reverse-mode
-gradients, through the C ABI.  The library recomputes in fp32 (bf16 inputs are
-read exactly), so every gradient tensor is held to the fp32 bound."""
+gradients, through the C ABI.  With fp32 inputs everything runs in fp32 and
+every gradient tensor is held to the fp32 bound; with bf16 inputs the attention
+products run on the tensor cores over hi + lo bf16 splits of their fp32 operands
+and the bound derived for that arithmetic applies."""
 import math
 
 import numpy as np
@@ -9,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import compare, dev_f32, dev_x, tol_for
+from helpers import TOL_SPLIT_BWD, compare, dev_f32, dev_x, tol_for
 from sa_inputs import STCALayer, add_stca_ffns, bf16_bits, bf16_to_f64, gauss, rng_for
 
 pytestmark = pytest.mark.gpu
@@ -61,7 +63,7 @@ def _check(lib, p):
     got = _run(lib, p)
     ref = oracle.stca_branch_grads(_widen(p, p["q"]), p["cand"], _widen(p, p["kv"]), p["kb"], p["ke"],
                                    p["layers"], p["heads"], p["d_h"], p["dout"])
-    tol = tol_for("f32")
+    tol = tol_for("f32") if p["dtype"] == "f32" else TOL_SPLIT_BWD
     errs = {"dq": compare("dq", got["dq"], ref["dq"], tol), "dkv": compare("dkv", got["dkv"], ref["dkv"], tol)}
     for li, (gl, rl) in enumerate(zip(got["layers"], ref["layers"])):
         for gk, buf in gl.items():
@@ -75,6 +77,8 @@ CASES = [
     ((7, 9), 600, (0, 250), (300, 600), 128, 4, 32, 2, "f32", False, True, False),
     ((33, 2), 500, (0, 0), (500, 0), 128, 2, 64, 1, "bf16", True, False, True),
     ((4, 4, 4), 260, (0, 100, 200), (150, 250, 260), 128, 4, 32, 2, "f32", True, False, False),
+    # key ranges of 1, 7 and 65 rows: tiles far past the matrix edges on the tensor cores
+    ((1, 2, 3), 80, (0, 1, 8), (1, 8, 73), 128, 4, 32, 2, "bf16", True, True, True),
 ]
 
 
@@ -83,7 +87,7 @@ def test_stca_backward_small(lib, case):
     cands, rows, kb, ke, D, heads, d_h, nl, dtype, wo, hist, query = case
     p = _problem(500 + rows, cands, rows, kb, ke, D, heads, d_h, nl, dtype, wo, hist, query)
     errs = _check(lib, p)
-    print(case, {k: round(v["max_rel"], 8) for k, v in errs.items()})
+    print(case, {k: (round(v["max_rel"], 6), round(v["mean_rel"], 6)) for k, v in errs.items()})
 
 
 def test_stca_backward_overlapping_ranges_and_unused_rows(lib):
@@ -108,7 +112,7 @@ def test_stca_backward_larger(lib):
     per head group), two full layers."""
     p = _problem(613, (128, 64), 6500, (0, 2500), (2500, 6500), 128, 4, 32, 2, "bf16", kv_scale=0.5)
     errs = _check(lib, p)
-    print({k: round(v["max_rel"], 8) for k, v in errs.items()})
+    print({k: (round(v["max_rel"], 6), round(v["mean_rel"], 6)) for k, v in errs.items()})
 
 
 def test_stca_backward_rejects_missing_gradient_buffer(lib):
@@ -144,4 +148,4 @@ def test_stca_backward_full_size_one_user(lib, which):
     p = dict(layers=layers, cand=br.cand_offsets, q=br.q, kv=br.kv, kb=br.kv_begin, ke=br.kv_end, dout=dout,
              heads=4, d_h=32, dtype="bf16")
     errs = _check(lib, p)
-    print(which, {k: round(v["max_rel"], 8) for k, v in errs.items()})
+    print(which, {k: (round(v["max_rel"], 6), round(v["mean_rel"], 6)) for k, v in errs.items()})
