@@ -727,6 +727,11 @@ def run_component(args, rank, world, device):
                           float(w.sketch.kv_end[u] - w.sketch.kv_begin[u])
                           for u in range(len(w.recent.cand_offsets) - 1))
         kname, attn_flops_step = "tc_gemm:stca_bwd_attn", 14.0 * rows_x_keys * 128 * nlay
+        # the FFN products (history FFN on every key row, query FFN on every candidate row, both
+        # branches): 12 D^2 flop per row in the recompute and 32 D^2 in the backward, per layer
+        ffn_rows = (float(np.sum(w.recent.kv_end - w.recent.kv_begin)) +
+                    float(np.sum(w.sketch.kv_end - w.sketch.kv_begin)) + 2.0 * C)
+        ffn_flops_step = 44.0 * 128 * 128 * ffn_rows * nlay
     else:
         w = stca_workload(users=args.users or 16)
         q, kvr, kvs = (_dev_bf16(a, device) for a in (w.recent.q, w.recent.kv, w.sketch.kv))
@@ -763,6 +768,8 @@ def run_component(args, rank, world, device):
     if args.workload == "stca_bwd":
         # flops per launch of the dominant (tensor-core GEMM) call site: the step's total over its launches
         flops = attn_flops_step / max(prof.get(kname, (0, 1))[1] / args.steps, 1)
+        extra.append(("tc_gemm:stca_bwd_ffn",
+                      ffn_flops_step / max(prof.get("tc_gemm:stca_bwd_ffn", (0, 1))[1] / args.steps, 1)))
 
     def roof_of(kn, fl):
         if kn not in prof:

@@ -375,7 +375,11 @@ size_t stca_backward_full_workspace(int B, const int64_t* cand_offsets_host,
  * Inputs as stca_forward_full.  The layers are recomputed in fp32 (bf16 inputs are
  * widened, not rounded further) and each user's attention is evaluated with its
  * C_u*heads x L_u score matrix in the workspace, so the workspace grows with the
- * largest user.  Deterministic: users are processed in order.
+ * largest user.  With SA_BF16 inputs the attention products run on the tensor
+ * cores with each fp32 operand split into two bf16 parts (hi + lo, about 16
+ * significant bits; three MMA passes per product), with SA_F32 inputs on fp32
+ * CUDA cores.  Deterministic: users are processed in order and split-K partial
+ * sums are added in a fixed order.
  * Errors: as stca_forward_full, and SA_ERR_INVALID_ARG for a NULL gradient buffer
  * of a weight that is present.
  */

@@ -133,16 +133,51 @@ __global__ void swiglu_bwd_kernel(const float* G1, const float* G3, const float*
   }
 }
 
+__device__ __forceinline__ void put_split(float v, __nv_bfloat16* hi, __nv_bfloat16* lo, int64_t e) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi[e] = h;
+  lo[e] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+// U = SiLU(G1) * G3, written only as its hi + lo split
+__global__ void swiglu_split_kernel(const float* __restrict__ G1, const float* __restrict__ G3, int64_t n,
+                                    __nv_bfloat16* __restrict__ hi, __nv_bfloat16* __restrict__ lo) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float g = G1[e];
+    put_split(g / (1.f + expf(-g)) * G3[e], hi, lo, e);
+  }
+}
+
+// dG1 and dG3 as swiglu_bwd_kernel computes them, written only as hi + lo splits
+__global__ void swiglu_bwd_split_kernel(const float* __restrict__ G1, const float* __restrict__ G3,
+                                        const float* __restrict__ dU, int64_t n, __nv_bfloat16* __restrict__ d1_hi,
+                                        __nv_bfloat16* __restrict__ d1_lo, __nv_bfloat16* __restrict__ d3_hi,
+                                        __nv_bfloat16* __restrict__ d3_lo) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float g = G1[e], s = 1.f / (1.f + expf(-g));
+    put_split(dU[e] * G3[e] * s * (1.f + g * (1.f - s)), d1_hi, d1_lo, e);
+    put_split(dU[e] * g * s, d3_hi, d3_lo, e);
+  }
+}
+
 unsigned grid_for(int64_t n) { return (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 1 << 16)); }
 
 bool has_hist(const stca_full_layer& L) { return L.hist_W1 != nullptr; }
 bool has_query(const stca_full_layer& L) { return L.q_W1 != nullptr; }
 
-// The stream and the split-K partials shared by every GEMM of one call (they run
-// in stream order).
+// bf16 hi + lo scratch for the FFN products' operands on the tensor cores: x [rows, D],
+// two [rows, 2D] slots and the three weights (2 D^2 each)
+struct FfnScratch {
+  __nv_bfloat16 *x_hi, *x_lo, *a_hi, *a_lo, *b_hi, *b_lo, *w_hi, *w_lo;
+};
+
+// The stream, the split-K partials and the split scratch shared by every GEMM of one
+// call (they run in stream order); tcp: bf16 inputs, products on the tensor cores.
 struct Ctx {
   cudaStream_t st;
   float* split;
+  bool tcp;
+  FfnScratch fs;
 };
 
 // GEMM with split-K when its output tiles alone leave most SMs idle (the weight
@@ -185,7 +220,7 @@ struct Split {
 // C[M, N] = A B (+ Cin) on the tensor cores over split operands (about 16 significant
 // bits each): A K-major or (a_mn) M-major, B K-major or (b_mn) N-major
 sa_status tc(int M, int N, int K, Split A, int64_t lda, bool a_mn, Split B, int64_t ldb, bool b_mn, float* C,
-             int64_t ldc, const float* Cin, const Ctx& cx) {
+             int64_t ldc, const float* Cin, const Ctx& cx, const char* tag = "tc_gemm:stca_bwd_attn") {
   cudaStream_t st = cx.st;
   TcGemm g;
   g.part = cx.split; g.part_floats = kStcaBwdSplitFloats;
@@ -193,9 +228,28 @@ sa_status tc(int M, int N, int K, Split A, int64_t lda, bool a_mn, Split B, int6
   g.A = A.hi; g.A_lo = A.lo; g.lda = lda; g.a_mn = a_mn;
   g.B = B.hi; g.B_lo = B.lo; g.ldb = ldb; g.b_mn = b_mn;
   g.C = C; g.ldc = ldc; g.Cin = Cin; g.ldcin = ldc;
-  g.tag = "tc_gemm:stca_bwd_attn";
+  g.tag = tag;
   return tc_gemm(g, st);
 }
+
+// hi + lo split of n fp32 values into the given scratch
+sa_status split_to(const float* x, int64_t n, __nv_bfloat16* hi, __nv_bfloat16* lo, Split* out, cudaStream_t st) {
+  SA_TIMED("split_kernel", st, (split_kernel<<<grid_for(n), 256, 0, st>>>(x, n, hi, lo)));
+  *out = {hi, lo};
+  return SA_OK;
+}
+
+// the FFN's three weights split into the weight scratch: W1, W3 [D, 2D], W2 [2D, D]
+sa_status split_weights(const Ffn& f, int D, Split w[3], const Ctx& cx) {
+  const float* W[3] = {f.W1, f.W3, f.W2};
+  const int64_t n = 2LL * D * D;
+  sa_status s;
+  for (int i = 0; i < 3; ++i)
+    if ((s = split_to(W[i], n, cx.fs.w_hi + i * n, cx.fs.w_lo + i * n, &w[i], cx.st)) != SA_OK) return s;
+  return SA_OK;
+}
+
+constexpr const char* kFfnTag = "tc_gemm:stca_bwd_ffn";
 
 // y = x + FFN(x) over `rows` rows
 sa_status ffn_fwd(const float* x, int64_t rows, int D, const Ffn& f, float* G1, float* G3, float* U, float* y,
@@ -203,6 +257,19 @@ sa_status ffn_fwd(const float* x, int64_t rows, int D, const Ffn& f, float* G1, 
   cudaStream_t st = cx.st;
   if (rows == 0) return SA_OK;
   sa_status s;
+  if (cx.tcp) {
+    Split w[3], xs, us;
+    const int R = (int)rows;
+    if ((s = split_weights(f, D, w, cx)) != SA_OK) return s;
+    if ((s = split_to(x, rows * D, cx.fs.x_hi, cx.fs.x_lo, &xs, st)) != SA_OK) return s;
+    if ((s = tc(R, 2 * D, D, xs, D, false, w[0], 2 * D, true, G1, 2 * D, nullptr, cx, kFfnTag)) != SA_OK) return s;
+    if ((s = tc(R, 2 * D, D, xs, D, false, w[1], 2 * D, true, G3, 2 * D, nullptr, cx, kFfnTag)) != SA_OK) return s;
+    const int64_t n2 = rows * 2 * D;
+    SA_TIMED("swiglu_split_kernel", st,
+             (swiglu_split_kernel<<<grid_for(n2), 256, 0, st>>>(G1, G3, n2, cx.fs.a_hi, cx.fs.a_lo)));
+    us = {cx.fs.a_hi, cx.fs.a_lo};
+    return tc(R, D, 2 * D, us, 2 * D, false, w[2], D, true, y, D, x, cx, kFfnTag);
+  }
   if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W1, 2 * D, false, G1, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
   if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W3, 2 * D, false, G3, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
   if ((s = sa_swiglu(G1, G3, rows * 2 * D, U, st)) != SA_OK) return s;
@@ -221,6 +288,31 @@ sa_status ffn_bwd(const float* x, int64_t rows, int D, const Ffn& f, const float
     for (float* w : {f.dW1, f.dW3, f.dW2})
       SA_CUDA(cudaMemsetAsync(w, 0, sizeof(float) * 2 * D * D, st));
     return SA_OK;
+  }
+  if (cx.tcp) {
+    Split w[3], xs, as, bs;
+    const int R = (int)rows;
+    const int64_t n1 = rows * D, n2 = rows * 2 * D;
+    if ((s = split_weights(f, D, w, cx)) != SA_OK) return s;
+    if ((s = split_to(x, n1, cx.fs.x_hi, cx.fs.x_lo, &xs, st)) != SA_OK) return s;
+    if ((s = tc(R, 2 * D, D, xs, D, false, w[0], 2 * D, true, G1, 2 * D, nullptr, cx, kFfnTag)) != SA_OK) return s;
+    if ((s = tc(R, 2 * D, D, xs, D, false, w[1], 2 * D, true, G3, 2 * D, nullptr, cx, kFfnTag)) != SA_OK) return s;
+    // U (split only) = SiLU(G1) * G3;  dW2 = U^T dy (U read M-major);  dU = dy W2^T (W2 read K-major)
+    SA_TIMED("swiglu_split_kernel", st,
+             (swiglu_split_kernel<<<grid_for(n2), 256, 0, st>>>(G1, G3, n2, cx.fs.a_hi, cx.fs.a_lo)));
+    as = {cx.fs.a_hi, cx.fs.a_lo};
+    if ((s = split_to(dy, n1, cx.fs.b_hi, cx.fs.b_lo, &bs, st)) != SA_OK) return s;
+    if ((s = tc(2 * D, D, R, as, 2 * D, true, bs, D, true, f.dW2, D, nullptr, cx, kFfnTag)) != SA_OK) return s;
+    if ((s = tc(R, 2 * D, D, bs, D, false, w[2], D, false, dU, 2 * D, nullptr, cx, kFfnTag)) != SA_OK) return s;
+    // dG1 (slot a) and dG3 (slot b), split only: dW1 = x^T dG1, dW3 = x^T dG3,
+    // dx = dy + dG1 W1^T + dG3 W3^T
+    SA_TIMED("swiglu_bwd_split_kernel", st,
+             (swiglu_bwd_split_kernel<<<grid_for(n2), 256, 0, st>>>(G1, G3, dU, n2, cx.fs.a_hi, cx.fs.a_lo,
+                                                                    cx.fs.b_hi, cx.fs.b_lo)));
+    if ((s = tc(D, 2 * D, R, xs, D, true, as, 2 * D, true, f.dW1, 2 * D, nullptr, cx, kFfnTag)) != SA_OK) return s;
+    if ((s = tc(D, 2 * D, R, xs, D, true, bs, 2 * D, true, f.dW3, 2 * D, nullptr, cx, kFfnTag)) != SA_OK) return s;
+    if ((s = tc(R, D, 2 * D, as, 2 * D, false, w[0], 2 * D, false, dx, D, dy, cx, kFfnTag)) != SA_OK) return s;
+    return tc(R, D, 2 * D, bs, 2 * D, false, w[1], 2 * D, false, dx, D, dx, cx, kFfnTag);
   }
   if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W1, 2 * D, false, G1, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
   if ((s = mm(plain((int)rows, 2 * D, D, x, D, false, f.W3, 2 * D, false, G3, 2 * D, "gemm:stca_bwd_ffn"), cx)) != SA_OK) return s;
@@ -274,6 +366,10 @@ size_t stca_bwd_layout(void* base, const StcaBwdShape& sh, StcaBwdWork* w) {
   v.Plo = c.take<__nv_bfloat16>(tc ? sl : 1);
   v.dSb = c.take<__nv_bfloat16>(tc ? sl : 1);
   v.dSlo = c.take<__nv_bfloat16>(tc ? sl : 1);
+  const size_t rows_max = std::max(C, R);
+  for (__nv_bfloat16** p : {&v.fx_hi, &v.fx_lo}) *p = c.take<__nv_bfloat16>(tc ? rows_max * D : 1);
+  for (__nv_bfloat16** p : {&v.fa_hi, &v.fa_lo, &v.fb_hi, &v.fb_lo}) *p = c.take<__nv_bfloat16>(tc ? rows_max * 2 * D : 1);
+  for (__nv_bfloat16** p : {&v.fw_hi, &v.fw_lo}) *p = c.take<__nv_bfloat16>(tc ? 6 * D * D : 1);
   v.dq = c.take<float>(C * D);
   v.dqmid = c.take<float>(C * D);
   v.dO = c.take<float>(C * HD);
@@ -294,8 +390,8 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
   const size_t CD = (size_t)C * D, CHD = (size_t)C * HD, CHD2 = (size_t)C * H * D, RD = (size_t)R * D;
   const float inv_sqrt = 1.f / std::sqrt((float)dh);
   sa_status s;
-  const Ctx cx{st, w.gsplit};
-  const bool tcp = a.dtype == SA_BF16;       // the attention products on the tensor cores
+  const bool tcp = a.dtype == SA_BF16;       // the attention and FFN products on the tensor cores
+  const Ctx cx{st, w.gsplit, tcp, {w.fx_hi, w.fx_lo, w.fa_hi, w.fa_lo, w.fb_hi, w.fb_lo, w.fw_hi, w.fw_lo}};
   // ---------------------------------------------------------------- inputs, widened
   if (C > 0) {
     if (a.dtype == SA_BF16)

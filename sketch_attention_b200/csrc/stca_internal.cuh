@@ -88,6 +88,7 @@ struct StcaBwdWork {
   float* gsplit;                          // split-K partials of the GEMMs with small outputs
   // bf16 operands of the tensor-core attention products (bf16 inputs only)
   __nv_bfloat16 *Ub, *Ulo, *Xkb, *Xklo, *dYb, *dYlo, *Pb, *Plo, *dSb, *dSlo;
+  __nv_bfloat16 *fx_hi, *fx_lo, *fa_hi, *fa_lo, *fb_hi, *fb_lo, *fw_hi, *fw_lo;   // FFN operand splits
 };
 constexpr size_t kStcaBwdSplitFloats = (size_t)16 << 20;
 size_t stca_bwd_layout(void* base, const StcaBwdShape& sh, StcaBwdWork* w);

@@ -8,7 +8,7 @@
 // A is [M, K], stored K-major (A[m lda + k]) or M-major (A[k lda + m]); B is
 // [K, N], stored K-major (B[n ldb + k]) or N-major (B[k ldb + n]).  One CTA per
 // 128 x 128 output tile: TMA brings 64-deep K slices of both operands into a
-// four-stage ring (128-byte swizzle; a K-major operand is one 64 x 128 box, an
+// three-stage ring (128-byte swizzle; a K-major operand is one 64 x 128 box, an
 // MN-major one two 64 x 64 boxes), one thread issues the MMAs (M = 128,
 // N = 128, K = 16) into a TMEM accumulator, and four warps write the tile.
 // Edges are zero-filled by the TMA and masked in the epilogue.  A deep K over few
@@ -26,12 +26,15 @@ namespace sa {
 namespace {
 using namespace tc;
 
-constexpr int TM = 128, TN = 128, TK = 64, NST = 4, THREADS = 192;
+constexpr int TM = 128, TN = 128, TK = 64, NST = 3, THREADS = 192;
 constexpr uint32_t OP_BYTES = TM * TK * 2;                 // 16 KB per operand per stage
 constexpr uint32_t STAGE = 2 * OP_BYTES;
 constexpr uint32_t OFF_BAR = NST * STAGE;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 128 + 1024;
 constexpr uint32_t TM_COLS = 128;
+// two CTAs per SM (2 x ~99.5 KB of shared memory, 2 x 128 TMEM columns): one CTA's
+// epilogue overlaps the other's loads and MMAs, which matters for the short-K products
+static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
 
 struct Bars {
   uint64_t full[NST], empty[NST], done;
@@ -59,7 +62,7 @@ __device__ __forceinline__ uint64_t op_desc(uint32_t base, int ks, bool mn) {
 }
 
 template <bool AMN, bool BMN>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAl,
                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBl, Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -135,37 +138,40 @@ __global__ void __launch_bounds__(THREADS, 1)
     mma_commit(&bars->done);
     mbar_wait_bounded(&bars->done, 0);
   } else if (warp >= 2) {
-    // ---------------------------------------------------------------- epilogue: one row per thread
+    // ---------------------------------------------------------------- epilogue
+    // warp q owns TMEM lanes (tile rows) 32q..32q+31; each 32 x 32 block goes from
+    // TMEM (a row per thread) through a padded shared-memory block (the operand ring is
+    // idle once every MMA has completed) so that each store writes 128 contiguous bytes
+    // of one row
     const int q = warp % 4;
-    const int row = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    float* blk = (float*)smem + q * (32 * 33);
     if (mbar_wait(&bars->done, 0, abort, p.err)) {
       tc_fence_after();
-      const int m = m0 + row;
 #pragma unroll 1
       for (int c = 0; c < TN / 32; ++c) {
         float v[32];
         tmem_ld32(tmem + lane_addr + 32 * c, v);
         tmem_wait_ld();
-        if (m >= p.M) continue;
-        const int nb = n0 + 32 * c;
-        if (p.part) {
-          float* dst = p.part + ((int64_t)blockIdx.z * p.M + m) * p.N + nb;
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (nb + i < p.N) dst[i] = v[i];
-          continue;
-        }
-        float* dst = p.C + (int64_t)m * p.ldc + nb;
-        const float* cin = p.Cin ? p.Cin + (int64_t)m * p.ldcin + nb : nullptr;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          if (nb + i < p.N) {
-            float x = p.alpha * v[i];
-            if (cin) x += cin[i];
-            dst[i] = x;
+        for (int i = 0; i < 32; ++i) blk[lane * 33 + i] = v[i];
+        __syncwarp();
+        const int n = n0 + 32 * c + lane;
+#pragma unroll 4
+        for (int r = 0; r < 32; ++r) {
+          const int m = m0 + q * 32 + r;
+          if (m < p.M && n < p.N) {
+            float x = blk[r * 33 + lane];
+            if (p.part) {
+              p.part[((int64_t)blockIdx.z * p.M + m) * p.N + n] = x;
+            } else {
+              x *= p.alpha;
+              if (p.Cin) x += p.Cin[(int64_t)m * p.ldcin + n];
+              p.C[(int64_t)m * p.ldc + n] = x;
+            }
           }
         }
+        __syncwarp();
       }
     }
   }
