@@ -61,7 +61,8 @@ __device__ __forceinline__ uint64_t op_desc(uint32_t base, int ks, bool mn) {
             : smem_desc(base + ks * 32, 16, 1024, SWZ_128B);              // 128 rows, K along the row
 }
 
-template <bool AMN, bool BMN>
+// CIN: the launch adds Cin in its epilogue (no split K)
+template <bool AMN, bool BMN, bool CIN>
 __global__ void __launch_bounds__(THREADS, 2)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAl,
                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmBl, Params p) {
@@ -143,9 +144,23 @@ __global__ void __launch_bounds__(THREADS, 2)
     // TMEM (a row per thread) through a padded shared-memory block (the operand ring is
     // idle once every MMA has completed) so that each store writes 128 contiguous bytes
     // of one row
+    // The added input Cin of a block is loaded as 32 independent row loads before the
+    // block's stores (the first block's while the MMAs still run), so its latency is paid
+    // once per block rather than once per row.  Cin may alias C: each element is read
+    // and then written by the same thread.
     const int q = warp % 4;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     float* blk = (float*)smem + q * (32 * 33);
+    float cv[CIN ? 32 : 1];
+    auto load_cin = [&](int c) {
+      const int n = n0 + 32 * c + lane;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        const int m = m0 + q * 32 + r;
+        cv[r] = (m < p.M && n < p.N) ? p.Cin[(int64_t)m * p.ldcin + n] : 0.f;
+      }
+    };
+    if constexpr (CIN) load_cin(0);
     if (mbar_wait(&bars->done, 0, abort, p.err)) {
       tc_fence_after();
 #pragma unroll 1
@@ -157,21 +172,30 @@ __global__ void __launch_bounds__(THREADS, 2)
         for (int i = 0; i < 32; ++i) blk[lane * 33 + i] = v[i];
         __syncwarp();
         const int n = n0 + 32 * c + lane;
+        if constexpr (CIN) {
+#pragma unroll
+          for (int r = 0; r < 32; ++r) {
+            const int m = m0 + q * 32 + r;
+            if (m < p.M && n < p.N) p.C[(int64_t)m * p.ldc + n] = p.alpha * blk[r * 33 + lane] + cv[r];
+          }
+        } else {
 #pragma unroll 4
-        for (int r = 0; r < 32; ++r) {
-          const int m = m0 + q * 32 + r;
-          if (m < p.M && n < p.N) {
-            float x = blk[r * 33 + lane];
-            if (p.part) {
-              p.part[((int64_t)blockIdx.z * p.M + m) * p.N + n] = x;
-            } else {
-              x *= p.alpha;
-              if (p.Cin) x += p.Cin[(int64_t)m * p.ldcin + n];
-              p.C[(int64_t)m * p.ldc + n] = x;
+          for (int r = 0; r < 32; ++r) {
+            const int m = m0 + q * 32 + r;
+            if (m < p.M && n < p.N) {
+              float x = blk[r * 33 + lane];
+              if (p.part) {
+                p.part[((int64_t)blockIdx.z * p.M + m) * p.N + n] = x;
+              } else {
+                p.C[(int64_t)m * p.ldc + n] = p.alpha * x;
+              }
             }
           }
         }
         __syncwarp();
+        if constexpr (CIN) {
+          if (c + 1 < TN / 32) load_cin(c + 1);
+        }
       }
     }
   }
@@ -198,11 +222,26 @@ __global__ void tc_gemm_reduce_kernel(const float* __restrict__ part, int splits
   }
 }
 
-template <bool AMN, bool BMN>
+template <bool AMN, bool BMN, bool CIN>
 void set_limit() {
   static unsigned long long done = 0;
   static std::mutex mu;
-  set_smem_limit_once((const void*)tc_gemm_kernel<AMN, BMN>, SMEM_BYTES, &done, mu);
+  set_smem_limit_once((const void*)tc_gemm_kernel<AMN, BMN, CIN>, SMEM_BYTES, &done, mu);
+}
+
+template <bool AMN, bool BMN, bool CIN>
+sa_status launch(const char* tag, dim3 grid, cudaStream_t st, const CUtensorMap& tmA, const CUtensorMap& tmAl,
+                 const CUtensorMap& tmB, const CUtensorMap& tmBl, const Params& p) {
+  set_limit<AMN, BMN, CIN>();
+  SA_TIMED(tag, st, (tc_gemm_kernel<AMN, BMN, CIN><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p)));
+  return SA_OK;
+}
+
+template <bool AMN, bool BMN>
+sa_status launch(bool cin, const char* tag, dim3 grid, cudaStream_t st, const CUtensorMap& tmA,
+                 const CUtensorMap& tmAl, const CUtensorMap& tmB, const CUtensorMap& tmBl, const Params& p) {
+  return cin ? launch<AMN, BMN, true>(tag, grid, st, tmA, tmAl, tmB, tmBl, p)
+             : launch<AMN, BMN, false>(tag, grid, st, tmA, tmAl, tmB, tmBl, p);
 }
 }  // namespace
 
@@ -246,13 +285,12 @@ sa_status tc_gemm(const TcGemm& g, cudaStream_t st) {
            split > 1 ? g.part : nullptr, device_status_word()};
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, split);
   const char* tag = g.tag ? g.tag : "tc_gemm_kernel";
-  if (g.a_mn) {
-    if (g.b_mn) { set_limit<true, true>(); SA_TIMED(tag, st, (tc_gemm_kernel<true, true><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p))); }
-    else { set_limit<true, false>(); SA_TIMED(tag, st, (tc_gemm_kernel<true, false><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p))); }
-  } else {
-    if (g.b_mn) { set_limit<false, true>(); SA_TIMED(tag, st, (tc_gemm_kernel<false, true><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p))); }
-    else { set_limit<false, false>(); SA_TIMED(tag, st, (tc_gemm_kernel<false, false><<<grid, THREADS, SMEM_BYTES, st>>>(tmA, tmAl, tmB, tmBl, p))); }
-  }
+  const bool cin = split == 1 && g.Cin != nullptr;
+  if ((s = g.a_mn ? (g.b_mn ? launch<true, true>(cin, tag, grid, st, tmA, tmAl, tmB, tmBl, p)
+                            : launch<true, false>(cin, tag, grid, st, tmA, tmAl, tmB, tmBl, p))
+                  : (g.b_mn ? launch<false, true>(cin, tag, grid, st, tmA, tmAl, tmB, tmBl, p)
+                            : launch<false, false>(cin, tag, grid, st, tmA, tmAl, tmB, tmBl, p))) != SA_OK)
+    return s;
   if (split > 1) {
     const int64_t mn = (int64_t)g.M * g.N;
     const unsigned blocks = (unsigned)std::min<int64_t>((mn + 255) / 256, 4 * kSMs);
