@@ -1,5 +1,5 @@
-// bf16 GEMM on the sm_100a tensor cores for the STCA backward's attention
-// products: C[M, N] = alpha A B (+ Cin), fp32 accumulation and output.
+// bf16 GEMM on the sm_100a tensor cores for the STCA backward's attention and
+// SwiGLU FFN products: C[M, N] = alpha A B (+ Cin), fp32 accumulation and output.
 // An operand may come as a split pair x = hi + lo (both bf16, lo the rounding of
 // x - hi): the K loop then runs again over hi x lo and lo x hi into the same
 // accumulator (lo x lo, below 2^-16 of the product, is dropped), which carries
@@ -10,7 +10,9 @@
 // 128 x 128 output tile: TMA brings 64-deep K slices of both operands into a
 // three-stage ring (128-byte swizzle; a K-major operand is one 64 x 128 box, an
 // MN-major one two 64 x 64 boxes), one thread issues the MMAs (M = 128,
-// N = 128, K = 16) into a TMEM accumulator, and four warps write the tile.
+// N = 128, K = 16) into a TMEM accumulator, and four warps write the tile through
+// shared memory (row-contiguous stores).  Two CTAs share an SM, so one CTA's
+// epilogue overlaps the other's loads and MMAs.
 // Edges are zero-filled by the TMA and masked in the epilogue.  A deep K over few
 // output tiles is split across CTAs (grid z): each writes its raw partial tile to a
 // workspace slice and a second kernel adds the slices in order (deterministic).
