@@ -591,6 +591,10 @@ def run_component(args, rank, world, device):
         _b.build()
     sab.load()
     from sa_inputs import STCA_WORKLOAD_4, sa_workload, stca_workload
+
+    def stca_label(w):
+        # the STCA workload's name with its actual user count (--users)
+        return STCA_WORKLOAD_4.replace("B=16", f"B={len(w.recent.cand_offsets) - 1}")
     peaks, peaks_src = load_peaks()
     extra = []          # (kernel, flops per launch) of other tensor-core kernels to report
     if args.workload == "sa_fwd":
@@ -676,7 +680,7 @@ def run_component(args, rank, world, device):
             sab.stca_fuse(zr, zu, WF, bF, out=z)
         units, unit = C, "candidates/s"
         name = ("full STCA layers (history-side SwiGLU FFN before and query-side after each attention), "
-                + STCA_WORKLOAD_4)
+                + stca_label(w))
         L_avg = 0.5 * (float(np.mean(w.recent.kv_end - w.recent.kv_begin)) + 1024)
         kname, flops = "stca_attn_tc_kernel", 4.0 * L_avg * 128 * C * w.heads
         # the history FFN: 12 D^2 flop per key row (eq. (27) with inner width 2D), once per row;
@@ -717,7 +721,7 @@ def run_component(args, rank, world, device):
                                    w.d_h, dzu, cand_offsets_dev=cd, kv_begin_dev=sbd, kv_end_dev=sed, out=gs,
                                    workspace=ws_s)
         units, unit = C, "candidates/s"
-        name = ("backward of full STCA layers (both FFNs, both branches), " + STCA_WORKLOAD_4)
+        name = ("backward of full STCA layers (both FFNs, both branches), " + stca_label(w))
         # the per-user attention GEMMs: S and Y in the recompute, S, dP, dU and the two dX
         # products in the backward, 14 R_u L_u D flop per user and layer (tensor cores, each
         # fp32 operand split into hi + lo bf16 parts: three MMA passes per algorithmic flop)
@@ -748,7 +752,7 @@ def run_component(args, rank, world, device):
             sab.stca_forward(q, w.sketch.cand_offsets, kvs, w.sketch.kv_begin, w.sketch.kv_end,
                              lu, w.heads, w.d_h, out=zu)
             sab.stca_fuse(zr, zu, WF, bF, out=z)
-        units, unit, name = C, "candidates/s", STCA_WORKLOAD_4
+        units, unit, name = C, "candidates/s", stca_label(w)
         L_avg = 0.5 * (float(np.mean(w.recent.kv_end - w.recent.kv_begin)) + 1024)
         kname, flops = "stca_attn_tc_kernel", 4.0 * L_avg * 128 * C * w.heads
     for _ in range(args.warmup):
