@@ -91,3 +91,22 @@ def test_stca_rejects_bad_ranges(lib):
                           kb.ctypes.data_as(ctypes.c_void_p), ke.ctypes.data_as(ctypes.c_void_p),
                           p, p, 96, 4, 32, 1, lay, p, p, 1 << 40, None)
     assert st == 2
+
+
+def test_stca_backward_workspace_query(lib):
+    """Host-only sizing of stca_backward_full's workspace: the bf16 path adds the operand
+    splits of its tensor-core products; the score scratch is one user's (the largest),
+    so a second, small user adds only its rows; an inverted range answers 0."""
+    def ws(cands, kb, ke, dtype, n_layers=2):
+        cand = np.concatenate([[0], np.cumsum(cands)]).astype(np.int64)
+        return sab.stca_backward_full_workspace(cand, np.asarray(kb, np.int64), np.asarray(ke, np.int64),
+                                                128, 4, 32, n_layers, dtype)
+    one_f32 = ws([512], [0], [10_000], sab.SA_F32)
+    one_bf16 = ws([512], [0], [10_000], sab.SA_BF16)
+    score_f32 = 512 * 4 * 10_000 * 4                    # one user's S, fp32
+    assert one_f32 >= 2 * score_f32                      # S and dS
+    assert one_bf16 >= one_f32 + 2 * score_f32          # + P and dS as bf16 hi + lo pairs (4 B a score each)
+    two_f32 = ws([512, 4], [0, 10_000], [10_000, 10_010], sab.SA_F32)
+    assert one_f32 < two_f32 < one_f32 + score_f32 // 8
+    assert ws([512], [0], [10_000], sab.SA_F32, n_layers=3) > one_f32
+    assert ws([4], [10], [5], sab.SA_F32) == 0           # kv_end < kv_begin
