@@ -12,7 +12,7 @@
 // Limits (larger sizes return SA_ERR_UNSUPPORTED before any GPU work): bf16
 // X, d = 128, k a multiple of 128 with k <= 512, B <= 8 users, any n_total
 // < 2^31.  Fewer token chunks are used than sa_forward uses (at most 8
-// clusters), so it is slower than sa_forward on large batches.
+// token chunks), so it is slower than sa_forward on large batches.
 //
 // Every call shares the array and it keeps the last call's contents.  Nothing
 // in it needs to start at zero: every word a call reads was written earlier
