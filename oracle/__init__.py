@@ -339,6 +339,18 @@ def event_rows(item_table, action_table, item_ids, action_ids) -> np.ndarray:
     return _f64(item_table)[np.asarray(item_ids, np.int64)] + _f64(action_table)[np.asarray(action_ids, np.int64)]
 
 
+def event_rows_fused(item_table, action_table, item_ids, action_ids, W1, W3, W2) -> np.ndarray:
+    """Action-side SwiGLU fusion (Sec. 3.6 / App. D, eq. (20)):
+        x_i = e_i + FFN_SwiGLU([e_i ; a_i]),   e_i = item_table[id_i], a_i = action_table[type_i]
+    with FFN_SwiGLU(z) = (SiLU(z W1) * (z W3)) W2 on the concatenated 2d-wide
+    feature, mapped back to the item embedding's width d so the residual add is
+    defined; W1, W3 [2d, w_f], W2 [w_f, d] (the workloads take w_f = 2d, eq. (23)'s
+    inner width for an FFN of width d), no biases."""
+    e = _f64(item_table)[np.asarray(item_ids, np.int64)]
+    a = _f64(action_table)[np.asarray(action_ids, np.int64)]
+    return e + swiglu_ffn(np.concatenate([e, a], axis=1), W1, W3, W2)
+
+
 def stca_fuse(z_r, z_u, W_F, b_F=None):
     """Linear fusion of the two branches: [z_r ; z_u] W_F + b_F (Sec. 3.4)."""
     z = np.concatenate([_f64(z_r), _f64(z_u)], axis=1)
