@@ -291,6 +291,9 @@ sa_status sa_poll_device_status(sa_stream_t stream) {
     cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice);
     if (v & DEV_ERR_TIMEOUT) return fail(SA_ERR_TIMEOUT, "a device-side wait expired");
     if (v & DEV_ERR_INDEX) return fail(SA_ERR_INVALID_ARG, "an embedding id was out of range (its row was zeroed)");
+    if (v & DEV_ERR_RANGE)
+      return fail(SA_ERR_UNSUPPORTED, "a value of the full STCA layer's fp16 operands exceeded the fp16 range "
+                                      "(|x| > 65504); scale the inputs down or use fp32 inputs");
     return fail(SA_ERR_CUDA, "device error word " + std::to_string(v));
   }
   return SA_OK;
@@ -672,6 +675,35 @@ sa_status sa_gather_events(const void* item_table, int64_t vocab, const void* ac
   SA_TRY(check_ptr(X, "X", n == 0));
   return gather_events_run(item_table, vocab, action_table, n_actions, item_ids, action_ids, n, d, X,
                            (cudaStream_t)stream);
+}
+
+size_t sa_gather_events_fused_workspace(int n_actions, int d, int d_ff) {
+  if (n_actions < 1 || n_actions > 16 || d != 128 || d_ff != 2 * d) return 0;
+  return events_ffn_layout(nullptr, n_actions, nullptr);
+}
+
+sa_status sa_gather_events_fused(const void* item_table, int64_t vocab, const void* action_table, int n_actions,
+                                 const int32_t* item_ids, const uint8_t* action_ids, int64_t n, int d,
+                                 const float* W1, const float* W3, const float* W2, int d_ff, void* X,
+                                 void* workspace, size_t ws_bytes, sa_stream_t stream) {
+  if (n < 0 || vocab < 1 || n_actions < 1) return fail(SA_ERR_INVALID_ARG, "bad sizes");
+  if (d != 128 || d_ff != 2 * d || n_actions > 16)
+    return fail(SA_ERR_UNSUPPORTED, "the fused event rows take d = 128, d_ff = 256 and 1..16 action types");
+  SA_TRY(check_ptr(item_table, "item_table"));
+  SA_TRY(check_ptr(action_table, "action_table"));
+  if (n > 0 && (!item_ids || !action_ids)) return fail(SA_ERR_INVALID_ARG, "item_ids or action_ids is NULL");
+  if (((uintptr_t)item_ids & 3) != 0) return fail(SA_ERR_INVALID_ARG, "item_ids is not 4-byte aligned");
+  SA_TRY(check_ptr(W1, "W1"));
+  SA_TRY(check_ptr(W3, "W3"));
+  SA_TRY(check_ptr(W2, "W2"));
+  SA_TRY(check_ptr(X, "X", n == 0));
+  const size_t need = events_ffn_layout(nullptr, n_actions, nullptr);
+  if (!workspace || ws_bytes < need || !aligned16(workspace))
+    return fail(SA_ERR_WORKSPACE, "workspace too small or unaligned: need " + std::to_string(need) + " bytes");
+  EventsFfnWork w;
+  events_ffn_layout(workspace, n_actions, &w);
+  return events_ffn_run((const __nv_bfloat16*)item_table, vocab, (const __nv_bfloat16*)action_table, n_actions,
+                        item_ids, action_ids, n, W1, W3, W2, (__nv_bfloat16*)X, w, (cudaStream_t)stream);
 }
 
 size_t stca_backward_full_workspace(int B, const int64_t* cand_offsets_host, const int64_t* kv_begin_host,

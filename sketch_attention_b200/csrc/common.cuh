@@ -5,6 +5,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 #include <string>
 
@@ -47,7 +48,9 @@ void prof_end(const char* name, cudaStream_t st);
 
 // Device error word (defined in api.cu): kernels whose bounded waits expire
 // OR in a code; sa_poll_device_status reads and clears it.
-enum : int { DEV_ERR_TIMEOUT = 1, DEV_ERR_INDEX = 2 };
+// bits of the device status word: a bounded wait expired; an embedding id was out of
+// range; a value stored as fp16 exceeded the fp16 range (|x| > 65504)
+enum : int { DEV_ERR_TIMEOUT = 1, DEV_ERR_INDEX = 2, DEV_ERR_RANGE = 4 };
 int* device_status_word();
 
 // ---------------------------------------------------------------- device info

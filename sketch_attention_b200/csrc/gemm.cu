@@ -21,6 +21,16 @@ __device__ __forceinline__ void cp_async4(float* dst, const float* src, bool pre
                "l"(src), "r"(pred ? 4 : 0) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// the 16-bit copy of an output: bf16, or fp16 with |v| > 65504 flagged on the device
+__device__ __forceinline__ void store16(const Gemm& g, int64_t i, float v) {
+  if (g.c16_half) {
+    if (!(fabsf(v) <= 65504.f) && g.err) atomicOr(g.err, DEV_ERR_RANGE);
+    reinterpret_cast<__half*>(g.C16)[i] = __float2half_rn(v);
+  } else {
+    g.C16[i] = __float2bfloat16_rn(v);
+  }
+}
+
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
@@ -114,7 +124,7 @@ __global__ void __launch_bounds__((BM / RM) * (BN / RN), 2) gemm_kernel(Gemm g) 
       if (g.bias) v += g.bias[n];
       if (g.Cin) v += g.Cin[(int64_t)b * g.sCin + (int64_t)m * g.ldcin + n];
       if (g.C) g.C[(int64_t)b * g.sC + (int64_t)m * g.ldc + n] = v;
-      if (g.C16) g.C16[(int64_t)b * g.sC16 + (int64_t)m * g.ldc16 + n] = __float2bfloat16_rn(v);
+      if (g.C16) store16(g, (int64_t)b * g.sC16 + (int64_t)m * g.ldc16 + n, v);
     }
   }
 }
@@ -132,7 +142,7 @@ __global__ void gemm_split_reduce_kernel(Gemm g) {
     if (g.bias) v += g.bias[n];
     if (g.Cin) v += g.Cin[(int64_t)b * g.sCin + (int64_t)m * g.ldcin + n];
     if (g.C) g.C[(int64_t)b * g.sC + (int64_t)m * g.ldc + n] = v;
-    if (g.C16) g.C16[(int64_t)b * g.sC16 + (int64_t)m * g.ldc16 + n] = __float2bfloat16_rn(v);
+    if (g.C16) store16(g, (int64_t)b * g.sC16 + (int64_t)m * g.ldc16 + n, v);
   }
 }
 }  // namespace

@@ -13,6 +13,8 @@ struct Gemm {
   const float* B = nullptr; int64_t ldb = 0; bool transB = false;   // B[k*ldb+n] or B[n*ldb+k]
   float* C = nullptr; int64_t ldc = 0;                               // fp32 out (may be NULL)
   __nv_bfloat16* C16 = nullptr; int64_t ldc16 = 0;                   // optional bf16 copy
+  bool c16_half = false;    // C16 holds fp16 values instead of bf16; |v| > 65504 sets the range bit in *err
+  int* err = nullptr;
   const float* Cin = nullptr; int64_t ldcin = 0;                     // optional addend
   const float* bias = nullptr;                                        // optional [N]
   float alpha = 1.f;

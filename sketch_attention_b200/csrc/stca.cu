@@ -167,7 +167,10 @@ sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWo
     g2.M = (int)C; g2.N = D; g2.K = dh;
     g2.A = w.Qh; g2.lda = HD; g2.sA = dh;
     g2.B = L.W_K; g2.ldb = dh; g2.transB = true; g2.sB = (int64_t)D * dh;
-    if (tc) { g2.C16 = w.Ub; g2.ldc16 = (int64_t)H * D; g2.sC16 = D; }
+    if (tc) {
+      g2.C16 = w.Ub; g2.ldc16 = (int64_t)H * D; g2.sC16 = D;
+      g2.c16_half = a.kv_f16; g2.err = device_status_word();
+    }
     else { g2.C = w.U; g2.ldc = (int64_t)H * D; g2.sC = D; }
     g2.alpha = 1.4426950408889634f / sqrtf((float)dh); g2.tag = "gemm:stca_U";
     g2.batch = H;

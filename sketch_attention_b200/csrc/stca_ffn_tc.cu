@@ -1,16 +1,23 @@
 // History-side SwiGLU FFN of the full STCA layer on the sm_100a tensor cores
-// (SequenceO1 Sec. 5.1, eq. (27)): for every bf16 key row x (D = 128)
+// (SequenceO1 Sec. 5.1, eq. (27)): for every fp16 key row x (D = 128)
 //   x <- x + (SiLU(x W1) * (x W3)) W2,   W1, W3 [128, 256], W2 [256, 128]
 // in place, with the 256-wide inner activations never leaving the SM.
 //
-// Persistent: one CTA per SM keeps W1|W3 resident in shared memory (bf16,
+// Every operand is fp16 (11 significant bits), not bf16 (8): the weights, the
+// inner activations and the stored rows are computed or converted values, and
+// bf16 roundings of all three put the layer's output about 3.6e-3 (mean
+// relative) from the exact one, fp16 roundings about 8 times less.  The rows of
+// this path stay far inside the fp16 range; a stored row value above 65504 sets
+// the range bit of the device status word.
+//
+// Persistent: one CTA per SM keeps W1|W3 resident in shared memory (fp16,
 // 128 KB), streams W2 a quarter at a time from L2, and walks 128-row tiles
 // with two X buffers.  A tile's inner width is
 // done in four quarters of 64:
 //   G_q  = X [W1_q | W3_q]     M=128 rows, N=128, K=128   (X from TMEM, fp32 in TMEM)
-//   U_q  = SiLU(G1_q) * G3_q   registers -> bf16 pairs in TMEM
+//   U_q  = SiLU(G1_q) * G3_q   registers -> fp16 pairs in TMEM
 //   F   += U_q W2_q            M=128, N=128, K=64          (A from TMEM)
-// and x + F goes back to the row as bf16.  G and U are double-buffered, so
+// and x + F goes back to the row as fp16.  G and U are double-buffered, so
 // the tensor pipe computes G_{q+1} while the epilogue warps turn G_q into U_q.
 // SiLU(g) g3 = (g/2) g3 (1 + tanh(g/2)): one MUFU operation per element.
 //
@@ -18,6 +25,14 @@
 // reads 128 bytes per clock, all that an SM's shared memory delivers, so the
 // X tile is moved into TMEM once per tile and every MMA reads only its B
 // operand from shared memory.
+//
+// The same kernel builds the events' input rows with the action-side SwiGLU
+// fusion of Sec. 3.6 / App. D, eq. (20): x = e + FFN([e; a]) for e = item
+// embedding, a = action embedding.  The action part of the first layer,
+// a [W1_a | W3_a], takes one of n_actions values, so it is a per-action bias of
+// G (precomputed, kept in shared memory in place of the X tiles); the rows are
+// gathered from the item table by id instead of read by TMA, and the result
+// goes to a separate bf16 output.
 //
 // Warp roles (16 warps): 0 TMA of W1|W3 and the X tiles, 1 first-layer MMA
 // issue + TMEM owner, 2-9 two warpgroups of SiLU gating (warpgroup h takes the
@@ -37,15 +52,15 @@ namespace {
 using namespace tc;
 
 constexpr int DD = 128, TM = 128, THREADS = 512;
-constexpr uint32_t W13_BYTES = 4 * 128 * DD * 2;   // [512 rows][128] bf16, two 64-column atoms
-constexpr uint32_t W2Q_BYTES = DD * 64 * 2;        // one quarter of W2t: [128 rows][64] bf16
+constexpr uint32_t W13_BYTES = 4 * 128 * DD * 2;   // [512 rows][128] fp16, two 64-column atoms
+constexpr uint32_t W2Q_BYTES = DD * 64 * 2;        // one quarter of W2t: [128 rows][64] fp16
 constexpr uint32_t X_BYTES = TM * DD * 2;          // one row tile, two atoms
 // W1|W3 stay resident; X tiles and W2 quarters (re-read from L2) are double-buffered
 constexpr uint32_t OFF_W13 = 0, OFF_X = OFF_W13 + W13_BYTES, OFF_W2 = OFF_X + 2 * X_BYTES;
 constexpr uint32_t OFF_BAR = OFF_W2 + 2 * W2Q_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
 // TMEM columns: G double buffer, U double buffer (bf16 pairs), the X tile as the
-// first layer's A operand (bf16 pairs), F accumulator
+// first layer's A operand (fp16 pairs), F accumulator
 constexpr uint32_t TM_G = 0, TM_U = 256, TM_X = 320, TM_F = 384, TM_COLS = 512;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
@@ -57,27 +72,41 @@ struct Bars {
 };
 
 struct Params {
-  __nv_bfloat16* X;
+  __half* X;           // rows transformed in place (history FFN)
   int64_t rows;
   int ntiles;
   int* err;
+  // event rows (eq. (20)): Xout[i] = bf16(item[ids[i]] + FFN([item[ids[i]]; action[acts[i]]]))
+  const __nv_bfloat16* item;
+  int64_t vocab;
+  const int32_t* ids;
+  const uint8_t* acts;
+  int n_actions;
+  const float* cb;     // [n_actions][512]: per quarter q, a W1_a[:, 64q..] then a W3_a[:, 64q..]
+  __nv_bfloat16* Xout;
 };
+constexpr int kMaxActions = 16;
+constexpr int CB_STRIDE = 516;   // floats per action in shared memory (4 banks apart per action)
+static_assert(kMaxActions * CB_STRIDE * 4 <= 2 * X_BYTES, "bias table fits the X stages");
 
 // SiLU(g1) g3 for a pair of elements: (g1/2) g3 (1 + tanh(g1/2)), one MUFU tanh per
-// element (tanh.approx: relative error about 2^-11, below the bf16 rounding of U).
+// element (tanh.approx: relative error about 2^-11, the size of the fp16 rounding of U).
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ uint32_t silu_mul_bf16x2(float a0, float a1, float b0, float b1) {
+__device__ __forceinline__ uint32_t silu_mul_f16x2(float a0, float a1, float b0, float b1) {
   const float2 hx = __fmul2_rn(make_float2(a0, a1), make_float2(0.5f, 0.5f));
   const float2 th = make_float2(tanh_approx(hx.x), tanh_approx(hx.y));
   const float2 hg = __fmul2_rn(hx, make_float2(b0, b1));
   const float2 u = __ffma2_rn(hg, th, hg);
-  return pack_bf16x2(u.x, u.y);
+  return pack_f16x2(u.x, u.y);
 }
 
+// EV: event rows of eq. (20) (gathered inputs, per-action bias, bf16 output);
+// else the history FFN of eq. (27), in place on fp16 rows
+template <bool EV>
 __global__ void __launch_bounds__(THREADS, 1)
     stca_hist_ffn_tc_kernel(const __grid_constant__ CUtensorMap tmX,
                             const __grid_constant__ CUtensorMap tmW13,
@@ -109,6 +138,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     bars->abort = 0;
     fence_mbar_init();
   }
+  if (EV) {
+    // the per-action bias of G (the X stages are free: rows are gathered, not loaded)
+    float* cbs = (float*)(smem + OFF_X);
+    for (int e = threadIdx.x; e < p.n_actions * 512; e += THREADS)
+      cbs[(e / 512) * CB_STRIDE + e % 512] = p.cb[e];
+  }
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, TM_COLS);
     tmem_relinquish();
@@ -120,7 +155,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------------------------------------------------------- TMA: W1|W3, X tiles
-    prefetch_tensormap(&tmX);
+    if (!EV) prefetch_tensormap(&tmX);
     prefetch_tensormap(&tmW13);
     mbar_arrive_expect_tx(&bars->w_full, W13_BYTES);
     for (int a = 0; a < 2; ++a)
@@ -128,7 +163,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_load_2d(smem + OFF_W13 + a * (W13_BYTES / 2) + r * (W13_BYTES / 4), &tmW13, &bars->w_full,
                     64 * a, 256 * r);
     int i = 0, issued = 0;
-    for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++i) {
+    for (int t = blockIdx.x; !EV && t < p.ntiles; t += gridDim.x, ++i) {
       const int s = i & 1;
       if (i >= 2 && !mbar_wait(&bars->x_empty[s], ((i >> 1) - 1) & 1, abort, p.err)) break;
       mbar_arrive_expect_tx(&bars->x_full[s], X_BYTES);
@@ -170,7 +205,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // G_q = X [W1_q | W3_q]; the quarter's rows of W13t start at 128 q.  A thread of
     // its own, so a G buffer is refilled as soon as its gating warpgroup has read it,
     // whatever the second-layer MMAs are waiting for.
-    const uint32_t id = idesc_bf16(128, 128, false, false);
+    const uint32_t id = idesc_f16(128, 128, false, false);
     const uint32_t w13 = smem_u32(smem + OFF_W13);
     bool ok = mbar_wait(&bars->w_full, 0, abort, p.err);
     int i = 0;
@@ -194,7 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 15 && lane == 0) {
     // ---------------------------------------------------------------- second-layer MMAs
     // F += U_q W2_q; W2 slot q % 2 holds W2t's inner columns 64q..64q+63
-    const uint32_t id = idesc_bf16(128, 128, false, false);
+    const uint32_t id = idesc_f16(128, 128, false, false);
     const uint32_t w2 = smem_u32(smem + OFF_W2);
     bool ok = true;
     int i = 0;
@@ -229,6 +264,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     int i = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x, ++i) {
+      // eq. (20): this row's action bias (a row past the end or with a bad type takes action 0;
+      // its output is dropped or zeroed by the write-back warps)
+      const float* cbr = nullptr;
+      if (EV) {
+        const int64_t grow = (int64_t)t * TM + q4 * 32 + lane;
+        const int a = grow < p.rows ? (int)p.acts[grow] : 0;
+        cbr = (const float*)(smem + OFF_X) + (a < p.n_actions ? a : 0) * CB_STRIDE;
+      }
       for (int q = h; q < 4; q += 2) {
         const int n = 2 * i + (q >> 1);
         if (!mbar_wait(&bars->g_full[h], n & 1, abort, p.err)) { ok = false; break; }
@@ -242,9 +285,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_before();
             mbar_arrive(&bars->g_empty[h]);
           }
+          if (EV) {
+            const float4* b1 = (const float4*)(cbr + 128 * q + 32 * c);
+            const float4* b3 = (const float4*)(cbr + 128 * q + 64 + 32 * c);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 x1 = b1[j], x3 = b3[j];
+              g1[4 * j] += x1.x; g1[4 * j + 1] += x1.y; g1[4 * j + 2] += x1.z; g1[4 * j + 3] += x1.w;
+              g3[4 * j] += x3.x; g3[4 * j + 1] += x3.y; g3[4 * j + 2] += x3.z; g3[4 * j + 3] += x3.w;
+            }
+          }
           uint32_t u[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) u[j] = silu_mul_bf16x2(g1[2 * j], g1[2 * j + 1], g3[2 * j], g3[2 * j + 1]);
+          for (int j = 0; j < 16; ++j) u[j] = silu_mul_f16x2(g1[2 * j], g1[2 * j + 1], g3[2 * j], g3[2 * j + 1]);
           // U buffer h was last read by the second-layer MMAs of use n-1
           if (c == 0 && n >= 1 && !mbar_wait(&bars->u_empty[h], (n - 1) & 1, abort, p.err)) {
             ok = false;
@@ -268,20 +321,52 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int row = q4 * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     // tile j's row: 16 pieces of 16 bytes (8 bf16), piece 8a + c at atom a, chunk c ^ (row % 8)
+    float vmax = 0.f;                   // largest |x + F| (or, for events, |e|) seen by this thread
+    // EV: the item row of tile j's row (zeros past the end or for an id outside the table)
+    auto event_row = [&](int j, uint4* v) {
+      const int64_t grow = (int64_t)(blockIdx.x + j * (int)gridDim.x) * TM + row;
+      bool ok = grow < p.rows;
+      int64_t id = 0;
+      if (ok) {
+        id = p.ids[grow];
+        ok = id >= 0 && id < p.vocab && (int)p.acts[grow] < p.n_actions;
+      }
+      const uint4* src = (const uint4*)(p.item + id * DD);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) v[c] = ok ? src[c] : make_uint4(0, 0, 0, 0);
+      return ok;
+    };
     auto stage_x = [&](int j) -> bool {
       const int s = j & 1;
-      if (!mbar_wait(&bars->x_full[s], (j >> 1) & 1, abort, p.err)) return false;
-      if (j >= 1 && !mbar_wait(&bars->xt_empty, (j - 1) & 1, abort, p.err)) return false;
-      const uint32_t base = smem_u32(smem + OFF_X + s * X_BYTES) + row * 128;
       uint32_t v[64];
+      if (EV) {
+        if (j >= 1 && !mbar_wait(&bars->xt_empty, (j - 1) & 1, abort, p.err)) return false;
+        uint4 e[16];
+        event_row(j, e);
 #pragma unroll
-      for (int pc = 0; pc < 16; ++pc) {
-        const uint32_t addr = base + (pc >> 3) * (X_BYTES / 2) + (((pc & 7) ^ (row & 7)) << 4);
-        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(v[4 * pc]), "=r"(v[4 * pc + 1]), "=r"(v[4 * pc + 2]), "=r"(v[4 * pc + 3])
-                     : "r"(addr));
+        for (int c = 0; c < 16; ++c) {
+          const uint32_t w[4] = {e[c].x, e[c].y, e[c].z, e[c].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            // bf16 -> fp32 exactly (the bf16 bits are the high half), then to fp16
+            const float lo = __uint_as_float(w[k] << 16), hi = __uint_as_float(w[k] & 0xFFFF0000u);
+            vmax = fmaxf(vmax, fmaxf(fabsf(lo), fabsf(hi)));
+            v[4 * c + k] = pack_f16x2(lo, hi);
+          }
+        }
+      } else {
+        if (!mbar_wait(&bars->x_full[s], (j >> 1) & 1, abort, p.err)) return false;
+        if (j >= 1 && !mbar_wait(&bars->xt_empty, (j - 1) & 1, abort, p.err)) return false;
+        const uint32_t base = smem_u32(smem + OFF_X + s * X_BYTES) + row * 128;
+#pragma unroll
+        for (int pc = 0; pc < 16; ++pc) {
+          const uint32_t addr = base + (pc >> 3) * (X_BYTES / 2) + (((pc & 7) ^ (row & 7)) << 4);
+          asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                       : "=r"(v[4 * pc]), "=r"(v[4 * pc + 1]), "=r"(v[4 * pc + 2]), "=r"(v[4 * pc + 3])
+                       : "r"(addr));
+        }
+        mbar_arrive(&bars->x_empty[s]);
       }
-      mbar_arrive(&bars->x_empty[s]);
       tc_fence_after();
       tmem_st32(tmem + lane_addr + TM_X, v);
       tmem_st32(tmem + lane_addr + TM_X + 32, v + 32);
@@ -297,12 +382,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (t + (int)gridDim.x < p.ntiles && !stage_x(i + 1)) break;
       const int64_t grow = (int64_t)t * TM + row;
       const bool valid = grow < p.rows;
-      const uint4* px = (const uint4*)(p.X + (valid ? grow : 0) * DD);
-      uint32_t xr[64];                  // the row as bf16 pairs
+      uint32_t xr[64];                  // the row as fp16 pairs (events: as bf16 pairs)
+      bool ev_ok = true;
+      if (EV) {
+        uint4 e[16];
+        ev_ok = event_row(i, e);        // the item row again (in L2 since it was staged)
+        if (valid && !ev_ok && p.err) atomicOr(p.err, DEV_ERR_INDEX);
 #pragma unroll
-      for (int v = 0; v < 16; ++v) {
-        const uint4 x = valid ? px[v] : make_uint4(0, 0, 0, 0);
-        xr[4 * v] = x.x; xr[4 * v + 1] = x.y; xr[4 * v + 2] = x.z; xr[4 * v + 3] = x.w;
+        for (int v = 0; v < 16; ++v) {
+          xr[4 * v] = e[v].x; xr[4 * v + 1] = e[v].y; xr[4 * v + 2] = e[v].z; xr[4 * v + 3] = e[v].w;
+        }
+      } else {
+        const uint4* px = (const uint4*)(p.X + (valid ? grow : 0) * DD);
+#pragma unroll
+        for (int v = 0; v < 16; ++v) {
+          const uint4 x = valid ? px[v] : make_uint4(0, 0, 0, 0);
+          xr[4 * v] = x.x; xr[4 * v + 1] = x.y; xr[4 * v + 2] = x.z; xr[4 * v + 3] = x.w;
+        }
       }
       if (!mbar_wait(&bars->f_full, i & 1, abort, p.err)) break;
       tc_fence_after();
@@ -317,19 +413,31 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32
-          const float lo = __uint_as_float(xr[8 * c + e] << 16);
-          const float hi = __uint_as_float(xr[8 * c + e] & 0xFFFF0000u);
-          xr[8 * c + e] = pack_bf16x2(lo + f[2 * e], hi + f[2 * e + 1]);
+          if (EV) {
+            // x = e + F, rounded once to bf16; a bad id or type gives a zero row
+            const uint32_t w = xr[8 * c + e];
+            const float y0 = __uint_as_float(w << 16) + f[2 * e];
+            const float y1 = __uint_as_float(w & 0xFFFF0000u) + f[2 * e + 1];
+            xr[8 * c + e] = ev_ok ? pack_bf16x2(y0, y1) : 0u;
+          } else {
+            __half2 hx;
+            memcpy(&hx, &xr[8 * c + e], 4);
+            const float2 x = __half22float2(hx);
+            const float y0 = x.x + f[2 * e], y1 = x.y + f[2 * e + 1];
+            vmax = fmaxf(vmax, fmaxf(fabsf(y0), fabsf(y1)));
+            xr[8 * c + e] = pack_f16x2(y0, y1);
+          }
         }
       }
       if (valid) {
-        uint4* po = (uint4*)(p.X + grow * DD);
+        uint4* po = EV ? (uint4*)(p.Xout + grow * DD) : (uint4*)(p.X + grow * DD);
 #pragma unroll
         for (int v = 0; v < 16; ++v)
           po[v] = make_uint4(xr[4 * v], xr[4 * v + 1], xr[4 * v + 2], xr[4 * v + 3]);
       }
     }
+    // NaN fails the comparison too
+    if (!(vmax <= 65504.f) && p.err) atomicOr(p.err, DEV_ERR_RANGE);
   }
 
   tc_fence_before();
@@ -342,55 +450,122 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 // W13t[128 q + r][k] = W1[k][64 q + r] (r < 64), W3[k][64 q + r - 64] (r >= 64);
 // W2t[n][j] = W2[j][n]
-__global__ void ffn_weights_bf16_kernel(const float* __restrict__ W1, const float* __restrict__ W3,
-                                        const float* __restrict__ W2, __nv_bfloat16* __restrict__ W13t,
-                                        __nv_bfloat16* __restrict__ W2t) {
+__global__ void ffn_weights_f16_kernel(const float* __restrict__ W1, const float* __restrict__ W3,
+                                       const float* __restrict__ W2, __half* __restrict__ W13t,
+                                       __half* __restrict__ W2t, int* __restrict__ err) {
+  float v = 0.f;
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e < 4 * 128 * DD) {
     const int r = e / DD, k = e % DD;
     const int q = r / 128, rr = r % 128;
     const float* src = rr < 64 ? W1 : W3;
-    W13t[e] = __float2bfloat16_rn(src[k * 2 * DD + 64 * q + (rr & 63)]);
+    v = src[k * 2 * DD + 64 * q + (rr & 63)];
+    W13t[e] = __float2half_rn(v);
   } else if (e < 4 * 128 * DD + DD * 2 * DD) {
     const int f = e - 4 * 128 * DD;
     const int n = f / (2 * DD), j = f % (2 * DD);
-    W2t[f] = __float2bfloat16_rn(W2[j * DD + n]);
+    v = W2[j * DD + n];
+    W2t[f] = __float2half_rn(v);
   }
+  if (!(fabsf(v) <= 65504.f) && err) atomicOr(err, DEV_ERR_RANGE);
 }
 
 
-// bf16 matrix [outer][inner], boxes of 64 x box_outer, 128-byte swizzle
+// fp16 matrix [outer][inner], boxes of 64 x box_outer, 128-byte swizzle
 sa_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint32_t box_outer) {
-  return tma_map_bf16(map, base, inner, outer, 64, box_outer, CU_TENSOR_MAP_SWIZZLE_128B);
+  return tma_map_2byte(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, base, inner, outer, 64, box_outer,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
 }
 }  // namespace
 
-sa_status stca_ffn_weights_bf16(const float* W1, const float* W3, const float* W2, __nv_bfloat16* W13t,
-                                __nv_bfloat16* W2t, cudaStream_t st) {
+sa_status stca_ffn_weights_f16(const float* W1, const float* W3, const float* W2, __half* W13t, __half* W2t,
+                               cudaStream_t st) {
   constexpr int n = 4 * 128 * DD + DD * 2 * DD;
-  SA_TIMED("ffn_weights_bf16_kernel", st,
-           (ffn_weights_bf16_kernel<<<(n + 255) / 256, 256, 0, st>>>(W1, W3, W2, W13t, W2t)));
+  SA_TIMED("ffn_weights_f16_kernel", st,
+           (ffn_weights_f16_kernel<<<(n + 255) / 256, 256, 0, st>>>(W1, W3, W2, W13t, W2t,
+                                                                     device_status_word())));
   return SA_OK;
 }
 
-sa_status stca_hist_ffn_tc(__nv_bfloat16* X, int64_t rows, const __nv_bfloat16* W13t,
-                           const __nv_bfloat16* W2t, cudaStream_t st) {
-  if (rows <= 0) return SA_OK;
-  if (rows >= (1LL << 31) - TM) return fail(SA_ERR_UNSUPPORTED, "history rows must be < 2^31 - 128");
-  static unsigned long long done = 0;
-  static std::mutex mu;
-  set_smem_limit_once((const void*)stca_hist_ffn_tc_kernel, SMEM_BYTES, &done, mu);
+namespace {
+std::mutex g_mu;
+unsigned long long g_done[2] = {0, 0};
+
+sa_status ffn_launch(bool ev, const Params& p0, const void* x_map_base, const __half* W13t, const __half* W2t,
+                     cudaStream_t st) {
+  if (ev) set_smem_limit_once((const void*)stca_hist_ffn_tc_kernel<true>, SMEM_BYTES, &g_done[1], g_mu);
+  else set_smem_limit_once((const void*)stca_hist_ffn_tc_kernel<false>, SMEM_BYTES, &g_done[0], g_mu);
   CUtensorMap tmX, tmW13, tmW2;
   sa_status s;
-  if ((s = make_map(&tmX, X, DD, (uint64_t)rows, TM)) != SA_OK) return s;
   if ((s = make_map(&tmW13, W13t, DD, 4 * 128, 256)) != SA_OK) return s;
   if ((s = make_map(&tmW2, W2t, 2 * DD, DD, 128)) != SA_OK) return s;
-  const int ntiles = (int)((rows + TM - 1) / TM);
-  const int grid = std::min(ntiles, device_info().sm_count);
-  Params p{X, rows, ntiles, device_status_word()};
-  SA_TIMED("stca_hist_ffn_tc_kernel", st,
-           (stca_hist_ffn_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmX, tmW13, tmW2, p)));
+  if (ev) tmX = tmW13;                  // not read: event rows are gathered by id
+  else if ((s = make_map(&tmX, x_map_base, DD, (uint64_t)p0.rows, TM)) != SA_OK) return s;
+  Params p = p0;
+  p.ntiles = (int)((p.rows + TM - 1) / TM);
+  p.err = device_status_word();
+  const int grid = std::min(p.ntiles, device_info().sm_count);
+  if (ev)
+    SA_TIMED("events_ffn_tc_kernel", st,
+             (stca_hist_ffn_tc_kernel<true><<<grid, THREADS, SMEM_BYTES, st>>>(tmX, tmW13, tmW2, p)));
+  else
+    SA_TIMED("stca_hist_ffn_tc_kernel", st,
+             (stca_hist_ffn_tc_kernel<false><<<grid, THREADS, SMEM_BYTES, st>>>(tmX, tmW13, tmW2, p)));
   return SA_OK;
+}
+
+// cb[a][128 q + c] = (action[a] W1[D:, :])[64 q + c] for c < 64, (action[a] W3[D:, :])[64 q + c - 64] else
+__global__ void __launch_bounds__(512) action_bias_kernel(const __nv_bfloat16* __restrict__ action,
+                                                          const float* __restrict__ W1,
+                                                          const float* __restrict__ W3, float* __restrict__ cb) {
+  const int a = blockIdx.x, e = threadIdx.x;
+  const int q = e / 128, c = e % 128;
+  const float* W = (c < 64 ? W1 : W3) + (int64_t)DD * 2 * DD + 64 * q + (c & 63);
+  float acc = 0.f;
+  for (int k = 0; k < DD; ++k) acc = fmaf(__bfloat162float(action[(int64_t)a * DD + k]), W[(int64_t)k * 2 * DD], acc);
+  cb[a * 512 + e] = acc;
+}
+}  // namespace
+
+sa_status stca_hist_ffn_tc(__half* X, int64_t rows, const __half* W13t, const __half* W2t, cudaStream_t st) {
+  if (rows <= 0) return SA_OK;
+  if (rows >= (1LL << 31) - TM) return fail(SA_ERR_UNSUPPORTED, "history rows must be < 2^31 - 128");
+  Params p{};
+  p.X = X;
+  p.rows = rows;
+  return ffn_launch(false, p, X, W13t, W2t, st);
+}
+
+size_t events_ffn_layout(void* base, int n_actions, EventsFfnWork* w) {
+  Carve c(base);
+  EventsFfnWork v;
+  v.W13t = c.take<__half>((size_t)4 * DD * DD);
+  v.W2t = c.take<__half>((size_t)2 * DD * DD);
+  v.cb = c.take<float>((size_t)std::max(n_actions, 1) * 512);
+  if (w) *w = v;
+  return c.bytes();
+}
+
+sa_status events_ffn_run(const __nv_bfloat16* item, int64_t vocab, const __nv_bfloat16* action, int n_actions,
+                         const int32_t* ids, const uint8_t* acts, int64_t n, const float* W1, const float* W3,
+                         const float* W2, __nv_bfloat16* X, const EventsFfnWork& w, cudaStream_t st) {
+  if (n <= 0) return SA_OK;
+  if (n >= (1LL << 31) - TM) return fail(SA_ERR_UNSUPPORTED, "events must be < 2^31 - 128");
+  if (n_actions < 1 || n_actions > kMaxActions)
+    return fail(SA_ERR_UNSUPPORTED, "the fused event rows take 1..16 action types");
+  sa_status s;
+  if ((s = stca_ffn_weights_f16(W1, W3, W2, w.W13t, w.W2t, st)) != SA_OK) return s;
+  SA_TIMED("action_bias_kernel", st, (action_bias_kernel<<<n_actions, 512, 0, st>>>(action, W1, W3, w.cb)));
+  Params p{};
+  p.rows = n;
+  p.item = item;
+  p.vocab = vocab;
+  p.ids = ids;
+  p.acts = acts;
+  p.n_actions = n_actions;
+  p.cb = w.cb;
+  p.Xout = X;
+  return ffn_launch(true, p, nullptr, w.W13t, w.W2t, st);
 }
 
 }  // namespace sa

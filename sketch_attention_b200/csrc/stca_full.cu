@@ -5,9 +5,13 @@
 // The history transform does not depend on the target, so it runs once per
 // key row (the amortisation the pages' eq. (33) counts for grouped requests)
 // on a private copy of each user's key range, which then serves as the
-// layer's keys and values.  bf16 keys: the fused tensor-core FFN of
-// stca_ffn_tc.cu; fp32 keys and the (small) query side: the projection GEMM.
+// layer's keys and values.  bf16 keys: the copy is fp16 (the rows it holds after
+// a transform are computed values, kept to 11 significant bits rather than
+// bf16's 8), transformed by the fused tensor-core FFN of stca_ffn_tc.cu, and
+// every layer's attention reads it with fp16 operands; fp32 keys and the (small)
+// query side: the projection GEMM.
 #include <algorithm>
+#include <cstring>
 
 #include "sa_internal.cuh"
 #include "stca_internal.cuh"
@@ -42,6 +46,37 @@ __global__ void gather_ranges_kernel(const uint4* __restrict__ kv, const int64_t
     }
     Hk[e] = kv[(kvb[lo] + (r - kpre[lo])) * pieces_per_row + c];
   }
+}
+
+// Hk[kpre[u] + j] = fp16(kv[kvb[u] + j]) for bf16 rows: 8 elements (16 bytes) per thread;
+// a value above the fp16 range sets the range bit of the device status word.
+__global__ void gather_ranges_f16_kernel(const uint4* __restrict__ kv, const int64_t* __restrict__ kvb,
+                                         const int64_t* __restrict__ kpre, int B, int pieces_per_row,
+                                         int64_t total_pieces, uint4* __restrict__ Hk, int* __restrict__ err) {
+  float vmax = 0.f;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total_pieces;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / pieces_per_row;
+    const int c = (int)(e % pieces_per_row);
+    int lo = 0, hi = B - 1;                // user: largest u with kpre[u] <= r
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (kpre[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    const uint4 x = kv[(kvb[lo] + (r - kpre[lo])) * pieces_per_row + c];
+    const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32
+      const float a = __uint_as_float(in[i] << 16), b = __uint_as_float(in[i] & 0xFFFF0000u);
+      vmax = fmaxf(vmax, fmaxf(fabsf(a), fabsf(b)));
+      const __half2 h = __floats2half2_rn(a, b);
+      memcpy(&out[i], &h, 4);
+    }
+    Hk[e] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+  if (!(vmax <= 65504.f) && err) atomicOr(err, DEV_ERR_RANGE);
 }
 
 unsigned grid_for(int64_t n) { return (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 1 << 16)); }
@@ -92,8 +127,8 @@ size_t stca_full_layout(void* base, int B, int64_t C, int64_t kv_total, int D, i
   v.G1 = c.take<float>(grows * 2 * D);
   v.G3 = c.take<float>(grows * 2 * D);
   v.U = c.take<float>(grows * 2 * D);
-  v.W13t = c.take<__nv_bfloat16>((size_t)4 * D * D);
-  v.W2t = c.take<__nv_bfloat16>((size_t)2 * D * D);
+  v.W13t = c.take<__half>((size_t)4 * D * D);
+  v.W2t = c.take<__half>((size_t)2 * D * D);
   if (w) *w = v;
   return c.bytes();
 }
@@ -112,19 +147,35 @@ sa_status stca_full_run(const StcaArgs& a0, const stca_full_layer* layers, int64
              (range_prefix_kernel<<<1, 1, 0, st>>>(a.kvb_dev, a.kve_dev, a.B, w.kpre)));
     const int ppr = a.D * esz / 16;
     const int64_t pieces = kv_total * ppr;
-    if (pieces > 0)
-      SA_TIMED("gather_ranges_kernel", st,
-               (gather_ranges_kernel<<<grid_for(pieces), 256, 0, st>>>(
-                   (const uint4*)a.kv, a.kvb_dev, w.kpre, a.B, ppr, pieces, (uint4*)w.Hk)));
+    if (pieces > 0) {
+      if (a.dtype == SA_BF16)
+        SA_TIMED("gather_ranges_f16_kernel", st,
+                 (gather_ranges_f16_kernel<<<grid_for(pieces), 256, 0, st>>>(
+                     (const uint4*)a.kv, a.kvb_dev, w.kpre, a.B, ppr, pieces, (uint4*)w.Hk,
+                     device_status_word())));
+      else
+        SA_TIMED("gather_ranges_kernel", st,
+                 (gather_ranges_kernel<<<grid_for(pieces), 256, 0, st>>>(
+                     (const uint4*)a.kv, a.kvb_dev, w.kpre, a.B, ppr, pieces, (uint4*)w.Hk)));
+    }
+    if (a.dtype == SA_BF16) {
+      // every layer attends over the fp16 copy (a layer without a history FFN reads the
+      // rows it was given, converted exactly within the fp16 range)
+      a.kv = w.Hk;
+      a.kv_rows = kv_total;
+      a.kvb_dev = w.kpre;
+      a.kve_dev = w.kpre + 1;
+      a.kv_f16 = true;
+    }
   }
   for (int l = 0; l < a.n_layers; ++l) {
     const stca_full_layer& L = layers[l];
     if (has_hist(L)) {
       // eq. (27): the layer's keys and values become x + FFN_h(x)
       if (a.dtype == SA_BF16) {
-        if ((s = stca_ffn_weights_bf16(L.hist_W1, L.hist_W3, L.hist_W2, w.W13t, w.W2t, st)) != SA_OK)
+        if ((s = stca_ffn_weights_f16(L.hist_W1, L.hist_W3, L.hist_W2, w.W13t, w.W2t, st)) != SA_OK)
           return s;
-        if ((s = stca_hist_ffn_tc((__nv_bfloat16*)w.Hk, kv_total, w.W13t, w.W2t, st)) != SA_OK) return s;
+        if ((s = stca_hist_ffn_tc((__half*)w.Hk, kv_total, w.W13t, w.W2t, st)) != SA_OK) return s;
       } else {
         if ((s = ffn_residual_gemm((float*)w.Hk, kv_total, a.D, L.hist_W1, L.hist_W3, L.hist_W2, w.G1,
                                    w.G3, w.U, "gemm:stca_hist_ffn", st)) != SA_OK)

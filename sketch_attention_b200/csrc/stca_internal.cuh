@@ -14,12 +14,15 @@ struct StcaArgs {
   const stca_layer* layers;   // host array
   float* out;
   int64_t max_rows_per_user;  // max over users of C_u * heads (host-computed)
+  // bf16 dtype only: kv rows (and the attention's query operand) are fp16 rather than
+  // bf16 (the full layer's transformed key rows, computed values kept to 11 bits)
+  bool kv_f16 = false;
 };
 
 struct StcaWork {
   float* Qh;           // [C, heads*d_h]
   float* U;            // [C*heads, D]   fp32 (CUDA-core attention)
-  __nv_bfloat16* Ub;   // [C*heads, D]   bf16 (tensor-core attention)
+  __nv_bfloat16* Ub;   // [C*heads, D]   bf16 or, with kv_f16, fp16 (tensor-core attention)
   float* Y;            // [C*heads, D]
   float* O;            // [C, heads*d_h]
   int* tile_prefix;    // [B+1]
@@ -35,11 +38,11 @@ sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWo
 // Full STCA layers (history- and query-side SwiGLU FFNs).
 struct StcaFullWork {
   StcaWork attn;
-  void* Hk;                 // [kv_total, D] key rows (kv dtype), transformed in place
+  void* Hk;                 // [kv_total, D] key rows (fp32 inputs: fp32; bf16 inputs: fp16), transformed in place
   int64_t* kpre;            // [B+1] start of each user's rows in Hk
   float* G1; float* G3; float* U;   // [max(C, rows of an fp32 history FFN), 2D] fp32
-  __nv_bfloat16* W13t;      // [4 * 128, D] bf16: the tensor-core FFN's first-layer weights
-  __nv_bfloat16* W2t;       // [D, 2D] bf16: its second-layer weights (transposed)
+  __half* W13t;             // [4 * 128, D] fp16: the tensor-core FFN's first-layer weights
+  __half* W2t;              // [D, 2D] fp16: its second-layer weights (transposed)
 };
 size_t stca_full_layout(void* base, int B, int64_t C, int64_t kv_total, int D, int heads, int d_h,
                         sa_dtype dtype, StcaFullWork* w);
@@ -96,12 +99,24 @@ sa_status stca_backward_run(const StcaArgs& a, const StcaBwdHost& hst, const stc
                             const stca_full_layer_grad* grads, const float* dout, float* dq_out, float* dkv,
                             const StcaBwdWork& w, cudaStream_t st);
 
-// x <- x + (SiLU(x W1) * (x W3)) W2 for rows of bf16 x, D = 128, in place, on
-// the tensor cores; W13t / W2t as prepared by stca_ffn_weights_bf16.
-sa_status stca_ffn_weights_bf16(const float* W1, const float* W3, const float* W2,
-                                __nv_bfloat16* W13t, __nv_bfloat16* W2t, cudaStream_t st);
-sa_status stca_hist_ffn_tc(__nv_bfloat16* X, int64_t rows, const __nv_bfloat16* W13t,
-                           const __nv_bfloat16* W2t, cudaStream_t st);
+// x <- x + (SiLU(x W1) * (x W3)) W2 for rows of fp16 x, D = 128, in place, on
+// the tensor cores; W13t / W2t (fp16) as prepared by stca_ffn_weights_f16.
+sa_status stca_ffn_weights_f16(const float* W1, const float* W3, const float* W2, __half* W13t, __half* W2t,
+                               cudaStream_t st);
+sa_status stca_hist_ffn_tc(__half* X, int64_t rows, const __half* W13t, const __half* W2t, cudaStream_t st);
+
+// Event rows with the action-side SwiGLU fusion (eq. (20)), d = 128, inner width 256:
+// X[i] = bf16(e + (SiLU(z W1) * (z W3)) W2), e = item[ids[i]], z = [e; action[acts[i]]];
+// W1, W3 [2d, 2d], W2 [2d, d] fp32.  Workspace: the fp16 weights and the per-action bias.
+struct EventsFfnWork {
+  __half* W13t;
+  __half* W2t;
+  float* cb;   // [n_actions, 512]
+};
+size_t events_ffn_layout(void* base, int n_actions, EventsFfnWork* w);
+sa_status events_ffn_run(const __nv_bfloat16* item, int64_t vocab, const __nv_bfloat16* action, int n_actions,
+                         const int32_t* ids, const uint8_t* acts, int64_t n, const float* W1, const float* W3,
+                         const float* W2, __nv_bfloat16* X, const EventsFfnWork& w, cudaStream_t st);
 
 bool stca_tc_supported(sa_dtype dtype, int D);
 sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st);

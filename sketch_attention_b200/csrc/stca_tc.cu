@@ -51,6 +51,8 @@ struct Params {
   int* err;
 };
 
+// F16: the query and key operands are fp16 (and so are the probabilities), else bf16
+template <bool F16>
 __global__ void __launch_bounds__(THREADS, 1)
     stca_attn_tc_kernel(const __grid_constant__ CUtensorMap tmU,
                         const __grid_constant__ CUtensorMap tmK, Params p) {
@@ -126,8 +128,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA
-    const uint32_t idS = idesc_bf16(128, 128, false, false);
-    const uint32_t idO = idesc_bf16(128, 128, false, true);
+    const uint32_t idS = F16 ? idesc_f16(128, 128, false, false) : idesc_bf16(128, 128, false, false);
+    const uint32_t idO = F16 ? idesc_f16(128, 128, false, true) : idesc_bf16(128, 128, false, true);
     const uint32_t qa = smem_u32(smem + OFF_Q);
     auto pv = [&](int j) -> bool {
       const int b = j & 1, s = j % NSK;
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           v = make_float2(ex2(e.x), ex2(e.y));
         }
         ls2 = __fadd2_rn(ls2, v);
-        pw[i / 2] = pack_bf16x2(v.x, v.y);
+        pw[i / 2] = F16 ? pack_f16x2(v.x, v.y) : pack_bf16x2(v.x, v.y);
       }
       const float ls = ls2.x + ls2.y;
       l += ls;
@@ -264,31 +266,37 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 
 // ============================================================== host side
-sa_status make_map(CUtensorMap* map, const void* base, uint64_t rows) {
-  return tma_map_bf16(map, base, DD, rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+sa_status make_map(CUtensorMap* map, const void* base, uint64_t rows, bool f16) {
+  return tma_map_2byte(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, DD,
+                       rows, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 }  // namespace
 
 bool stca_tc_supported(sa_dtype dtype, int D) { return dtype == SA_BF16 && D == DD; }
 
 sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
-  static unsigned long long done = 0;
+  static unsigned long long done = 0, done16 = 0;
   static std::mutex mu;
-  set_smem_limit_once((const void*)stca_attn_tc_kernel, SMEM_BYTES, &done, mu);
+  set_smem_limit_once((const void*)stca_attn_tc_kernel<false>, SMEM_BYTES, &done, mu);
+  set_smem_limit_once((const void*)stca_attn_tc_kernel<true>, SMEM_BYTES, &done16, mu);
   if (a.kv_rows >= (1LL << 31) || a.C_total * a.heads >= (1LL << 31))
     return fail(SA_ERR_UNSUPPORTED, "row counts must be < 2^31");
   CUtensorMap tmU, tmK;
-  sa_status s = make_map(&tmU, w.Ub, (uint64_t)(a.C_total * a.heads));
+  sa_status s = make_map(&tmU, w.Ub, (uint64_t)(a.C_total * a.heads), a.kv_f16);
   if (s != SA_OK) return s;
   if (a.kv_rows > 0) {
-    s = make_map(&tmK, a.kv, (uint64_t)a.kv_rows);
+    s = make_map(&tmK, a.kv, (uint64_t)a.kv_rows, a.kv_f16);
     if (s != SA_OK) return s;
   } else {
     memset(&tmK, 0, sizeof(tmK));     // never read: every key range is empty
   }
   Params p{w.tile_prefix, a.cand_dev, a.kvb_dev, a.kve_dev, a.B, a.heads, w.Y, device_status_word()};
-  SA_TIMED("stca_attn_tc_kernel", st,
-           (stca_attn_tc_kernel<<<w.max_tiles, THREADS, SMEM_BYTES, st>>>(tmU, tmK, p)));
+  if (a.kv_f16)
+    SA_TIMED("stca_attn_tc_kernel", st,
+             (stca_attn_tc_kernel<true><<<w.max_tiles, THREADS, SMEM_BYTES, st>>>(tmU, tmK, p)));
+  else
+    SA_TIMED("stca_attn_tc_kernel", st,
+             (stca_attn_tc_kernel<false><<<w.max_tiles, THREADS, SMEM_BYTES, st>>>(tmU, tmK, p)));
   return SA_OK;
 }
 

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import compare, dev_f32, dev_x, tol_for, tol_full_stca
+from helpers import compare, dev_f32, dev_x, tol_for
 from sa_inputs import add_stca_ffns, bf16_bits, make_stca_problem, rng_for, stca_workload
 
 pytestmark = pytest.mark.gpu
@@ -94,7 +94,7 @@ def _make(case, seed):
 @pytest.mark.parametrize("which", ["recent", "sketch"])
 def test_stca_full_small(lib, case, which):
     prob = _make(case, 300 + case[3])
-    e = compare(f"stca_full {which}", _run(lib, prob, which), _ref(prob, which), tol_full_stca(prob.dtype))
+    e = compare(f"stca_full {which}", _run(lib, prob, which), _ref(prob, which), tol_for(prob.dtype))
     print(f"stca_full {which} {case}: {e}")
 
 
@@ -108,7 +108,7 @@ def test_stca_full_large_history_values(lib, dtype):
     kv_in = bf16_bits(kv.astype(np.float32)) if dtype == "bf16" else kv.astype(np.float32)
     got = _run(lib, prob, "recent", kv=kv_in)
     ref = _ref(prob, "recent", kv=kv_in)
-    print("stca_full recent x40", dtype, compare("stca_full recent x40", got, ref, tol_full_stca(dtype)))
+    print("stca_full recent x40", dtype, compare("stca_full recent x40", got, ref, tol_for(dtype)))
 
 
 def test_stca_full_all_ranges_empty(lib):
@@ -169,4 +169,21 @@ def test_stca_full_workload4_sampled(lib, w4full, which):
     br, _ = _branch(w4full, which)
     for u, ref in _ref(w4full, which, users=(0, 15)).items():
         c0, c1 = int(br.cand_offsets[u]), int(br.cand_offsets[u + 1])
-        print(which, u, compare(f"stca_full {which}[{u}]", got[c0:c1], ref, tol_full_stca("bf16")))
+        print(which, u, compare(f"stca_full {which}[{u}]", got[c0:c1], ref, tol_for("bf16")))
+
+
+def test_stca_full_reports_fp16_range(lib):
+    """bf16 rows beyond the fp16 range (|x| > 65504) cannot be held by the full
+    layer's fp16 key copy: the call's status poll reports SA_ERR_UNSUPPORTED,
+    and the next call on normal rows runs clean."""
+    prob = _make((2, (5, 6), (50, 70), 16, 4, 32, 1, "bf16", "hist"), 470)
+    br, layers = _branch(prob, "sketch")
+    big = bf16_bits((prob.widen(br.kv) * 1e5).astype(np.float32))
+    lib.stca_forward_full(dev_x(br.q, "bf16"), br.cand_offsets, dev_x(big, "bf16"), br.kv_begin, br.kv_end,
+                          _layers_dev(layers), prob.heads, prob.d_h)
+    torch.cuda.synchronize()
+    with pytest.raises(lib.SAError) as ei:
+        lib.poll_device_status()
+    assert ei.value.status == 2 and "fp16" in str(ei.value)
+    out = _run(lib, prob, "sketch")
+    compare("stca_full after a range error", out, _ref(prob, "sketch"), tol_for("bf16"))
