@@ -244,8 +244,9 @@ sa_status sa_refine_forward(const void* X, sa_dtype x_dtype, const int64_t* offs
  * sa_gather_events -- the events' input rows on the device: for i < n
  *   X[i] = item_table[item_ids[i]] + action_table[action_ids[i]]
  * (an item embedding plus the embedding of the feedback type, the workloads'
- * events; paper Sec. 3.5, the sum that eq. (20)'s fusion adds a SwiGLU term
- * to), so that a step ships 5 bytes of ids per event instead of its row.
+ * events; paper Sec. 3.6, the plain sum next to eq. (20)'s fused rows of
+ * sa_gather_events_fused), so that a step ships 5 bytes of ids per event
+ * instead of its row.
  * item_table [vocab, d] and action_table [n_actions, d] bf16, 16-byte aligned;
  * item_ids int32 [n] (4-byte aligned), action_ids uint8 [n]; X [n, d] bf16 out.
  * The sum is formed in fp32 and rounded to nearest even.  d a multiple of 8.
@@ -255,6 +256,29 @@ sa_status sa_refine_forward(const void* X, sa_dtype x_dtype, const int64_t* offs
 sa_status sa_gather_events(const void* item_table, int64_t vocab, const void* action_table,
                            int n_actions, const int32_t* item_ids, const uint8_t* action_ids,
                            int64_t n, int d, void* X, sa_stream_t stream);
+
+size_t sa_gather_events_fused_workspace(int n_actions, int d, int d_ff);
+
+/*
+ * sa_gather_events_fused -- the events' input rows with the action-side SwiGLU
+ * fusion (paper Sec. 3.6 / App. D, eq. (20)): for i < n, with
+ * e = item_table[item_ids[i]], a = action_table[action_ids[i]] and z = [e ; a],
+ *   X[i] = e + (SiLU(z W1) * (z W3)) W2
+ * W1, W3 [2d, d_ff] and W2 [d_ff, d] fp32 row-major device arrays (no biases);
+ * the FFN maps the 2d-wide concatenation back to width d for the residual.
+ * d = 128, d_ff = 256 and 1..16 action types (else SA_ERR_UNSUPPORTED).
+ * Tables bf16, ids as in sa_gather_events, X [n, d] bf16 out (rounded once to
+ * nearest even).  The tensor-core products take fp16 operands (the weights,
+ * e and the inner activations), fp32 accumulation; the action half of the
+ * first layer is computed once per action type into the workspace.
+ * Workspace: sa_gather_events_fused_workspace bytes, 16-byte aligned, caller
+ * owned.  An id or action type outside its table gives a zero row and makes
+ * the next sa_poll_device_status return SA_ERR_INVALID_ARG.
+ */
+sa_status sa_gather_events_fused(const void* item_table, int64_t vocab, const void* action_table,
+                                 int n_actions, const int32_t* item_ids, const uint8_t* action_ids,
+                                 int64_t n, int d, const float* W1, const float* W3, const float* W2,
+                                 int d_ff, void* X, void* workspace, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* STCA: stacked target-to-history single-query cross attention             */

@@ -362,6 +362,15 @@ def event_problem(n: int, vocab: int, d: int, seed: int, n_actions: int = N_ACTI
     return item, action, ids, acts
 
 
+def event_ffn_weights(rng, d: int, d_ff: int = None, scale: float = 1.0):
+    """Weights of the action-side SwiGLU fusion of the event rows: W1, W3 [2d, d_ff]
+    with std scale/sqrt(2d) and W2 [d_ff, d] with std 1/sqrt(d_ff) (variance 1 over
+    the fan-in; d_ff = 2d by default), fp32."""
+    d_ff = 2 * d if d_ff is None else d_ff
+    return (gauss(rng, (2 * d, d_ff), scale / math.sqrt(2 * d)), gauss(rng, (2 * d, d_ff), scale / math.sqrt(2 * d)),
+            gauss(rng, (d_ff, d), 1.0 / math.sqrt(d_ff)))
+
+
 def add_stca_ffns(rng, layers, D: int, hist: bool = True, query: bool = True):
     """Give each STCA layer the full layer's SwiGLU FFNs: W1, W3 [D, 2D] with
     std 1/sqrt(D) and W2 [2D, D] with std 1/sqrt(2D), history side and/or

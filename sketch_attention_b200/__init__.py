@@ -31,7 +31,8 @@ EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_w
            "sa_forward_noalloc", "sa_refine_workspace", "sa_refine_forward",
            "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate",
            "stca_forward_full_workspace", "stca_forward_full", "stca_backward_full_workspace",
-           "stca_backward_full", "sa_gather_events", "sa_measure_exp2_rate", "sa_selftest_bounded_wait")
+           "stca_backward_full", "sa_gather_events", "sa_gather_events_fused",
+           "sa_gather_events_fused_workspace", "sa_measure_exp2_rate", "sa_selftest_bounded_wait")
 
 
 class SAError(RuntimeError):
@@ -116,6 +117,11 @@ def load(path: Optional[str] = None):
     lib.sa_measure_exp2_rate.argtypes = [_i, ctypes.POINTER(ctypes.c_double), _vp]
     lib.sa_gather_events.restype = _i
     lib.sa_gather_events.argtypes = [_vp, _i64, _vp, _i, _vp, _vp, _i64, _i, _vp, _vp]
+    lib.sa_gather_events_fused_workspace.restype = _sz
+    lib.sa_gather_events_fused_workspace.argtypes = [_i, _i, _i]
+    lib.sa_gather_events_fused.restype = _i
+    lib.sa_gather_events_fused.argtypes = [_vp, _i64, _vp, _i, _vp, _vp, _i64, _i, _vp, _vp, _vp, _i, _vp, _vp,
+                                           _sz, _vp]
     lib.stca_fuse.restype = _i
     lib.stca_fuse.argtypes = [_vp, _vp, _vp, _vp, _i64, _i, _vp, _vp]
     lib.sa_forward_noalloc.restype = _i
@@ -448,6 +454,37 @@ def sa_gather_events(item_table: torch.Tensor, action_table: torch.Tensor, item_
     st = lib.sa_gather_events(_p(item_table), item_table.shape[0], _p(action_table), action_table.shape[0],
                               _p(item_ids), _p(action_ids), n, d, _p(X), _stream(stream))
     _check("sa_gather_events", st)
+    return X
+
+
+def sa_gather_events_fused_workspace(n_actions: int, d: int = 128, d_ff: int = 256) -> int:
+    return int(load().sa_gather_events_fused_workspace(n_actions, d, d_ff))
+
+
+def sa_gather_events_fused(item_table: torch.Tensor, action_table: torch.Tensor, item_ids: torch.Tensor,
+                           action_ids: torch.Tensor, W1: torch.Tensor, W3: torch.Tensor, W2: torch.Tensor, *,
+                           out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """X[i] = e + (SiLU(z W1) * (z W3)) W2 with e = item_table[item_ids[i]],
+    z = [e ; action_table[action_ids[i]]] (eq. (20)); bf16 tables and output,
+    int32 / uint8 ids, fp32 weights W1, W3 [2d, d_ff], W2 [d_ff, d].  Returns X [n, d]."""
+    lib = load()
+    _need_cuda(item_table, action_table, item_ids, action_ids, W1, W3, W2)
+    if item_table.dtype != torch.bfloat16 or action_table.dtype != torch.bfloat16:
+        raise TypeError("the tables must be bf16")
+    if item_ids.dtype != torch.int32 or action_ids.dtype != torch.uint8:
+        raise TypeError("item_ids must be int32 and action_ids uint8")
+    n, d = item_ids.numel(), item_table.shape[1]
+    d_ff = W2.shape[0]
+    na = action_table.shape[0]
+    X = out if out is not None else torch.empty(n, d, dtype=torch.bfloat16, device=item_table.device)
+    if workspace is None:
+        workspace = torch.empty(max(sa_gather_events_fused_workspace(na, d, d_ff), 16), dtype=torch.uint8,
+                                device=item_table.device)
+    st = lib.sa_gather_events_fused(_p(item_table), item_table.shape[0], _p(action_table), na, _p(item_ids),
+                                    _p(action_ids), n, d, _p(W1), _p(W3), _p(W2), d_ff, _p(X), _p(workspace),
+                                    workspace.numel(), _stream(stream))
+    _check("sa_gather_events_fused", st)
     return X
 
 

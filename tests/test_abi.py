@@ -110,3 +110,25 @@ def test_stca_backward_workspace_query(lib):
     assert one_f32 < two_f32 < one_f32 + score_f32 // 8
     assert ws([512], [0], [10_000], sab.SA_F32, n_layers=3) > one_f32
     assert ws([4], [10], [5], sab.SA_F32) == 0           # kv_end < kv_begin
+
+
+def test_fused_event_rows_host_checks(lib):
+    """Host-only checks of sa_gather_events_fused: its workspace holds the fp16 weights
+    (3 x 256 x 128 x 2 bytes) and the per-action bias; sizes outside d = 128, d_ff = 2d
+    and 1..16 action types answer 0 / SA_ERR_UNSUPPORTED, a short workspace
+    SA_ERR_WORKSPACE, all before any GPU work."""
+    w8 = sab.sa_gather_events_fused_workspace(8, 128, 256)
+    assert w8 >= 3 * 256 * 128 * 2 + 8 * 512 * 4
+    assert sab.sa_gather_events_fused_workspace(9, 128, 256) > w8
+    assert sab.sa_gather_events_fused_workspace(8, 64, 128) == 0
+    assert sab.sa_gather_events_fused_workspace(17, 128, 256) == 0
+    p = _fake(0x10000)
+    ids = _fake(0x20000)
+    st = lib.sa_gather_events_fused(p, 1000, p, 8, ids, p, 10, 64, p, p, p, 128, p, p, 1 << 30, None)
+    assert st == 2
+    st = lib.sa_gather_events_fused(p, 1000, p, 17, ids, p, 10, 128, p, p, p, 256, p, p, 1 << 30, None)
+    assert st == 2
+    st = lib.sa_gather_events_fused(p, 1000, p, 8, ids, p, 10, 128, p, p, p, 256, p, p, w8 - 16, None)
+    assert st == 5
+    st = lib.sa_gather_events_fused(p, 1000, p, 8, _fake(0x20002), p, 10, 128, p, p, p, 256, p, p, w8, None)
+    assert st == 1
