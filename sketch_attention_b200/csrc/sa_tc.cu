@@ -5,10 +5,11 @@
 // Two kernels, neither of which ever writes the k x n assignment matrix:
 //
 //   sa_lse_tc_kernel  token-parallel, one CTA per token chunk.  Per 128-token
-//     tile it streams P' in chunks of 128 prototypes: Z_c = X_t P'_c^T
-//     (M=128 tokens, N=128, K=d) into TMEM; two warpgroups (64 prototypes of
+//     tile (moved into TMEM, the MMA's A operand) it streams P' in chunks of 128
+//     prototypes: Z_c = X_t P'_c^T
+//     (M=128 tokens, N=128, K=d) into TMEM; four warpgroups (32 prototypes of
 //     each chunk each, one thread per token) keep an online maximum and sum of
-//     2^z, and at the end of the tile combine their halves into the token's
+//     2^z, and at the end of the tile combine their quarters into the token's
 //     log2-sum-exp over all k prototypes.
 //
 //   sa_agg_tc_kernel  prototype-slice-parallel, one CTA per (128-prototype
@@ -78,34 +79,23 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-// maximum of 64 values (four independent chains of three-input maxima)
-__device__ __forceinline__ float max64(const float* z) {
-  float c[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float* w = z + 16 * i;
-    float m = max3f(w[0], w[1], w[2]);
-#pragma unroll
-    for (int j = 3; j + 1 < 16; j += 2) m = max3f(m, w[j], w[j + 1]);
-    c[i] = fmaxf(m, w[15]);
-  }
-  return fmaxf(max3f(c[0], c[1], c[2]), c[3]);
-}
-
 // ============================================================== lse kernel
 constexpr int L_NXS = 2, L_NPS = 4;                 // X stages, P' chunk stages
 constexpr uint32_t T_BYTES = TILE * DD * 2;         // [128 x 128] bf16: 2 SW128 halves of 16 KB
 constexpr uint32_t L_OFF_X = 0;
 constexpr uint32_t L_OFF_P = L_OFF_X + L_NXS * T_BYTES;
-constexpr uint32_t L_OFF_XCH = L_OFF_P + L_NPS * T_BYTES;   // [2][128]: warpgroup 1's max and sum
-constexpr uint32_t L_OFF_BAR = L_OFF_XCH + 2 * TILE * 4;
+constexpr uint32_t L_OFF_XCH = L_OFF_P + L_NPS * T_BYTES;   // [3][2][128]: warpgroups 1-3's max and sum
+constexpr uint32_t L_OFF_BAR = L_OFF_XCH + 6 * TILE * 4;
 constexpr uint32_t L_SMEM = L_OFF_BAR + 256 + 1024;
-constexpr int L_THREADS = 320;   // warp 0 TMA, 1 MMA + TMEM owner, 2-5 and 6-9 two warpgroups
-constexpr uint32_t L_TM_Z = 0, L_TM_COLS = 256;    // two [128 x 128] fp32 logits buffers
+constexpr int L_THREADS = 704;   // warp 0 TMA, 1 MMA + TMEM owner, 2-5 and 6-9 two warpgroups,
+                                 // 10-13 X tiles from shared memory into TMEM
+// TMEM columns: two [128 x 128] fp32 logits buffers, two X tiles (bf16 pairs: the
+// MMA's A operand, so the logits MMAs read only P' from shared memory)
+constexpr uint32_t L_TM_Z = 0, L_TM_X = 256, L_TM_COLS = 512;
 
 struct LBars {
   uint64_t x_full[L_NXS], x_empty[L_NXS], c_full[L_NPS], c_empty[L_NPS];
-  uint64_t z_full[2], z_empty[2], cx_full, cx_empty, mma_done;
+  uint64_t z_full[2], z_empty[2], xt_full[2], xt_empty[2], cx_full, cx_empty, mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -123,7 +113,7 @@ struct LParams {
   int* err;
 };
 
-__global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 warps share a sub-partition)
+__global__ void __launch_bounds__(L_THREADS, 1)
     sa_lse_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                      LParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -136,10 +126,15 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
   const int nch = p.k / TILE;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < L_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
+    for (int s = 0; s < L_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 128); }
     for (int s = 0; s < L_NPS; ++s) { mbar_init(&bars->c_full[s], 1); mbar_init(&bars->c_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&bars->z_full[b], 1); mbar_init(&bars->z_empty[b], 256); }
-    mbar_init(&bars->cx_full, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->z_full[b], 1);
+      mbar_init(&bars->z_empty[b], 512);
+      mbar_init(&bars->xt_full[b], 128);
+      mbar_init(&bars->xt_empty[b], 1);
+    }
+    mbar_init(&bars->cx_full, 384);
     mbar_init(&bars->cx_empty, 128);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
@@ -187,12 +182,12 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ logits MMAs
+    // Z_c = X_t P'_c^T with X_t from TMEM (A) and P'_c from shared memory (B)
     const uint32_t id = idesc_bf16(128, 128, false, false);
     int ai = 0;
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
-      const int s = t % L_NXS;
-      if (!mbar_wait(&bars->x_full[s], (t / L_NXS) & 1, abort, p.err)) return false;
-      const uint32_t xa = smem_u32(smem + L_OFF_X + s * T_BYTES);
+      const int xb = t & 1;
+      if (!mbar_wait(&bars->xt_full[xb], (t >> 1) & 1, abort, p.err)) return false;
       for (int c = 0; c < nch; ++c) {
         const int a = ai + c, cs = a % L_NPS, b = a & 1;
         if (!mbar_wait(&bars->c_full[cs], (a / L_NPS) & 1, abort, p.err)) return false;
@@ -201,22 +196,21 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
         const uint32_t pa = smem_u32(smem + L_OFF_P + cs * T_BYTES);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          mma_ss(tmem + L_TM_Z + 128 * b,
-                 smem_desc(xa + (ks >> 2) * (T_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B),
+          mma_ts(tmem + L_TM_Z + 128 * b, tmem + L_TM_X + 64 * xb + 8 * ks,
                  smem_desc(pa + (ks >> 2) * (T_BYTES / 2) + (ks & 3) * 32, 16, 1024, SWZ_128B), id,
                  ks > 0 ? 1u : 0u);
         mma_commit(&bars->z_full[b]);
         mma_commit(&bars->c_empty[cs]);                     // P' is read by this MMA only
-        if (c == nch - 1) mma_commit(&bars->x_empty[s]);
       }
+      mma_commit(&bars->xt_empty[xb]);                      // X in TMEM is read by these MMAs only
       ai += nch;
       return true;
     });
     mma_commit(&bars->mma_done);
     mbar_wait_bounded(&bars->mma_done, 0);
-  } else if (warp >= 2 && warp <= 9) {
-    // ------------------------------------------------------------ two threads per token
-    // warpgroup h reads columns 64h..64h+63 of each chunk's logits
+  } else if (warp >= 2 && warp <= 17) {
+    // ------------------------------------------------------------ four threads per token
+    // warpgroup h reads columns 32h..32h+31 of each chunk's logits
     const int q = warp % 4, h = (warp - 2) / 4;
     const int row = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
@@ -229,19 +223,21 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
         const int a = ai + c, b = a & 1;
         if (!mbar_wait(&bars->z_full[b], (a >> 1) & 1, abort, p.err)) return false;
         tc_fence_after();
-        float z[64];
-        tmem_ld32(tmem + lane_addr + L_TM_Z + 128 * b + 64 * h, z);
-        tmem_ld32(tmem + lane_addr + L_TM_Z + 128 * b + 64 * h + 32, z + 32);
+        float z[32];
+        tmem_ld32(tmem + lane_addr + L_TM_Z + 128 * b + 32 * h, z);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->z_empty[b]);
-        const float mn = fmaxf(m, max64(z));
+        float mz = max3f(z[0], z[1], z[2]);
+#pragma unroll
+        for (int j = 3; j + 1 < 32; j += 2) mz = max3f(mz, z[j], z[j + 1]);
+        const float mn = fmaxf(m, fmaxf(mz, z[31]));
         const float sc = ex2(m - mn);                      // 0 on the first chunk
         s2 = __fmul2_rn(s2, make_float2(sc, sc));
         m = mn;
         const float2 nm = make_float2(-mn, -mn);
 #pragma unroll
-        for (int j = 0; j < 64; j += 2) {
+        for (int j = 0; j < 32; j += 2) {
           const float2 e = __fadd2_rn(make_float2(z[j], z[j + 1]), nm);
           const float2 v = ((SA_FWD_POLY_PAIRS >> ((j / 2) & 3)) & 1) ? exp2_pair<true>(e) : exp2_pair<false>(e);
           s2 = __fadd2_rn(s2, v);
@@ -249,23 +245,55 @@ __global__ void __launch_bounds__(384, 1)   // 384: at most 168 registers (3 war
       }
       ai += nch;
       const float s = s2.x + s2.y;
-      if (h == 1) {
-        // hand the half-row statistics to warpgroup 0 (the slot is free once it read the last ones)
+      if (h > 0) {
+        // hand the quarter-row statistics to warpgroup 0 (the slot is free once it read the last ones)
         if (t > 0 && !mbar_wait(&bars->cx_empty, (t - 1) & 1, abort, p.err)) return false;
-        xch[row] = m;
-        xch[TILE + row] = s;
+        xch[(h - 1) * 2 * TILE + row] = m;
+        xch[(h - 1) * 2 * TILE + TILE + row] = s;
         mbar_arrive(&bars->cx_full);
         return true;
       }
       if (!mbar_wait(&bars->cx_full, t & 1, abort, p.err)) return false;
-      const float m1 = xch[row], s1 = xch[TILE + row];
+      float mm[3], ss[3];
+#pragma unroll
+      for (int w = 0; w < 3; ++w) { mm[w] = xch[w * 2 * TILE + row]; ss[w] = xch[w * 2 * TILE + TILE + row]; }
       mbar_arrive(&bars->cx_empty);
-      const float M = fmaxf(m, m1);
-      const float l2 = M + lg2(s * ex2(m - M) + s1 * ex2(m1 - M));
+      const float M = fmaxf(fmaxf(m, mm[0]), fmaxf(mm[1], mm[2]));
+      const float l2 = M + lg2(s * ex2(m - M) + ss[0] * ex2(mm[0] - M) + ss[1] * ex2(mm[1] - M) + ss[2] * ex2(mm[2] - M));
       if (tb + row < pe) {
         p.lse_a[tb + row] = l2 * p.a_scale;
         if (p.lse_b) p.lse_b[tb + row] = l2 * kLn2f;
       }
+      return true;
+    });
+  } else if (warp >= 18) {
+    // ------------------------------------------------------------ X tile into TMEM
+    // Each thread moves its token's row (16 pieces of 16 bytes; piece 8a + c of the
+    // row sits in 128-byte-swizzled half a at chunk c ^ (row % 8)) into TMEM as bf16
+    // pairs, the A operand of the tile's logits MMAs.
+    const int q = warp % 4;
+    const int row = q * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
+      const int s = t % L_NXS, xb = t & 1;
+      if (!mbar_wait(&bars->x_full[s], (t / L_NXS) & 1, abort, p.err)) return false;
+      if (t >= 2 && !mbar_wait(&bars->xt_empty[xb], ((t >> 1) - 1) & 1, abort, p.err)) return false;
+      const uint32_t base = smem_u32(smem + L_OFF_X + s * T_BYTES) + row * 128;
+      uint32_t v[64];
+#pragma unroll
+      for (int pc = 0; pc < 16; ++pc) {
+        const uint32_t addr = base + (pc >> 3) * (T_BYTES / 2) + (((pc & 7) ^ (row & 7)) << 4);
+        asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v[4 * pc]), "=r"(v[4 * pc + 1]), "=r"(v[4 * pc + 2]), "=r"(v[4 * pc + 3])
+                     : "r"(addr));
+      }
+      mbar_arrive(&bars->x_empty[s]);
+      tc_fence_after();
+      tmem_st32(tmem + lane_addr + L_TM_X + 64 * xb, v);
+      tmem_st32(tmem + lane_addr + L_TM_X + 64 * xb + 32, v + 32);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->xt_full[xb]);
       return true;
     });
   }
