@@ -14,14 +14,13 @@
 //
 //   sa_agg_tc_kernel  prototype-slice-parallel, one CTA per (128-prototype
 //     slice, token chunk), transposed so the prototypes are the TMEM lanes:
-//     per tile Z = P'_slice X_t^T (P' resident in TMEM as the A operand); two
+//     per tile Z = P'_slice X_t^T into one of three TMEM buffers; two
 //     warpgroups (64 tokens each, one thread per prototype) turn Z into
-//     probabilities p = 2^(z - lse) and write them back over Z as bf16 pairs,
-//     the TMEM A operand of
-//     H_slice += p [X_t | 1]   (M=128 prototypes, N=144, K=128 tokens)
-//     which accumulates in TMEM; the last 16 columns hold the mass.  The X tile
-//     is the only shared-memory operand.  At the end of a user's piece of the
-//     chunk H and the mass go to HBM.
+//     probabilities p = 2^(z - lse), sum them into the prototype's mass, and
+//     write them back over Z as bf16 pairs, the TMEM A operand of
+//     H_slice += p X_t   (M=128 prototypes, N=d, K=128 tokens)
+//     which accumulates in TMEM.  At the end of a user's piece of the chunk H
+//     and the mass go to HBM.
 //
 // The logits are computed twice (once per kernel); in exchange no CTA waits
 // for another, every SM takes part, and a probability tile is written once,
@@ -307,36 +306,39 @@ __global__ void __launch_bounds__(L_THREADS, 1)
 }
 
 // ============================================================== aggregation kernel
-// Transposed so that both MMAs take their A operand from TMEM: the prototypes
-// of the slice are the MMA rows (TMEM lanes), the tokens the columns.
-//   Z_t = P'_slice X_t^T   (M=128 prototypes, N=128 tokens, K=d; P' resident in TMEM)
-//   p   = 2^(Z_t - lse)     fp32 -> bf16 pairs, written over the first half of the
-//                           warpgroup's own Z columns (each warpgroup owns 64 tokens)
-//   H  += p [X_t | 1]      (M=128 prototypes, N=144, K=128 tokens; p from TMEM)
-// The X tile is the only shared-memory operand: B of both MMAs (K-major for the
-// logits, MN-major for the aggregation), so per tile the SM's shared memory
-// serves one TMA write and two operand reads of X, nothing else.
+// Transposed: the prototypes of the slice are the MMA rows (TMEM lanes), the
+// tokens the columns, so the probabilities are written where the logits were
+// and feed the aggregation MMA from TMEM:
+//   Z_t = P'_slice X_t^T   (M=128 prototypes, N=128 tokens, K=d; both operands in shared memory)
+//   p   = 2^(Z_t - lse)     fp32 -> bf16 pairs over the first half of the warpgroup's own
+//                           Z columns (each warpgroup owns 64 tokens); the fp32 values
+//                           are summed in registers into the prototype's mass
+//   H  += p X_t            (M=128 prototypes, N=d, K=128 tokens; p from TMEM, X MN-major)
+// A tile's logits -> probabilities -> aggregation chain crosses three mbarrier
+// hand-offs, so three logits buffers are kept in flight; that takes every TMEM
+// column (3 x 128 + H 128), which is why P' is a shared-memory operand here and
+// the mass is not an extra block of MMA columns.
 #ifndef SA_AGG_NS
 #define SA_AGG_NS 4
 #endif
 constexpr int A_NS = SA_AGG_NS;                       // X stages (a tile is held until its aggregation)
-constexpr int N2 = DD + 16;                           // MMA2 N: d columns + 16 mass columns
+constexpr int A_NZ = 3;                               // logits/probability buffers
 constexpr uint32_t X_BOX = TILE * 32;                 // one [128 x 16] bf16 SW32 box = 4 KB
-constexpr uint32_t X_STAGE = 9 * X_BOX;               // 8 boxes of X + 1 box of ones = 36 KB
-constexpr uint32_t A_OFF_X = 0;
+constexpr uint32_t X_STAGE = 8 * X_BOX;               // 32 KB
+constexpr uint32_t A_OFF_PQ = 0;                      // P' slice: 2 x [128 x 64] SW128 = 32 KB
+constexpr uint32_t A_OFF_X = T_BYTES;
 constexpr uint32_t A_OFF_LSE = A_OFF_X + A_NS * X_STAGE;   // [A_NS][128] fp32: -lse of the stage's tokens
-constexpr uint32_t A_OFF_BAR = A_OFF_LSE + A_NS * TILE * 4;
+constexpr uint32_t A_OFF_M = A_OFF_LSE + A_NS * TILE * 4;  // [2 slots][2 warpgroups][128] partial masses
+constexpr uint32_t A_OFF_BAR = A_OFF_M + 2 * 2 * TILE * 4;
 constexpr uint32_t A_SMEM = A_OFF_BAR + 256 + 1024;
 constexpr int A_THREADS = 480;   // warp 0 TMA + lse tiles, 1 logits MMAs + TMEM owner, 2 aggregation
-                                 // MMAs, 3-6 P' staging and H drain, 7-10 and 11-14 two softmax
-                                 // warpgroups (64 tokens of each tile each)
-// TMEM columns: two logits/probability buffers, H (144), the P' slice (bf16 pairs)
-constexpr uint32_t A_TM_Z = 0, A_TM_H = 256, A_TM_PQ = 448, A_TM_COLS = 512;
+                                 // MMAs, 3-6 H drain, 7-10 and 11-14 two softmax warpgroups
+constexpr uint32_t A_TM_Z = 0, A_TM_H = 384, A_TM_COLS = 512;
 static_assert(A_SMEM <= 232448, "shared memory per CTA");
 
 struct ABars {
-  uint64_t x_full[A_NS], x_empty[A_NS], z_full[2], p_full[2], z_free[2];
-  uint64_t h_full, h_empty, pq_full, pq_empty, mma_done[2];
+  uint64_t x_full[A_NS], x_empty[A_NS], z_full[A_NZ], p_full[A_NZ], z_free[A_NZ];
+  uint64_t h_full, h_empty, pq_full, pq_empty, m_full[2], m_empty[2], mma_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -349,7 +351,6 @@ struct AParams {
   int k;
   const float* lse;    // [n] per-token log-sum-exp, times in_scale in log2 units
   float in_scale;
-  const __nv_bfloat16* Pb;   // folded prototypes, bf16 [rows, d]
   float* Huser;        // [B, k, d] users that lie inside one chunk
   float* Muser;        // [B, k]
   float* slotH;        // [G, 2, k, d] pieces at chunk boundaries
@@ -359,7 +360,8 @@ struct AParams {
 };
 
 __global__ void __launch_bounds__(A_THREADS, 1)
-    sa_agg_tc_kernel(const __grid_constant__ CUtensorMap tmX, AParams p) {
+    sa_agg_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
+                     AParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   ABars* bars = (ABars*)(smem + A_OFF_BAR);
@@ -372,26 +374,21 @@ __global__ void __launch_bounds__(A_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < A_NS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < A_NZ; ++b) {
       mbar_init(&bars->z_full[b], 1);
       mbar_init(&bars->p_full[b], 256);
       mbar_init(&bars->z_free[b], 1);
     }
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars->m_full[b], 256); mbar_init(&bars->m_empty[b], 128); }
     mbar_init(&bars->h_full, 1);
     mbar_init(&bars->h_empty, 128);
-    mbar_init(&bars->pq_full, 128);
+    mbar_init(&bars->pq_full, 1);
     mbar_init(&bars->pq_empty, 1);
     mbar_init(&bars->mma_done[0], 1);
     mbar_init(&bars->mma_done[1], 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  // constant ones block of every stage (MMA2 columns d..d+15 -> prototype mass)
-  for (int i = threadIdx.x; i < A_NS * (int)X_BOX / 4; i += A_THREADS) {
-    const int s = i / (X_BOX / 4), w = i % (X_BOX / 4);
-    ((uint32_t*)(smem + A_OFF_X + s * X_STAGE + 8 * X_BOX))[w] = 0x3F803F80u;   // bf16 1.0 pairs
-  }
-  fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(&bars->tmem_base, A_TM_COLS);
     tmem_relinquish();
@@ -403,14 +400,34 @@ __global__ void __launch_bounds__(A_THREADS, 1)
   const int64_t n_total = p.off[p.B];
 
   if (warp == 0) {
-    // ------------------------------------------------------------ X tiles (TMA) and -lse tiles
-    // The warp copies the tile's per-token -lse (+inf past the piece: p = 0) into the
+    // ------------------------------------------------------------ P' slices, X tiles, -lse tiles
+    // The warp copies the tile's per-token -lse (-inf past the piece: p = 0) into the
     // stage's slot before lane 0 arrives on x_full; the values are loaded a tile ahead.
-    if (lane == 0) prefetch_tensormap(&tmX);
-    int issued = 0;
+    // Lane 0 takes every wait and tells the warp (a uniform decision: no lane may be
+    // left behind at the __syncwarp below).
+    if (lane == 0) {
+      prefetch_tensormap(&tmX);
+      prefetch_tensormap(&tmP);
+    }
+    int issued = 0, pq_issued = 0;
     float cur[4], nxt[4];
-    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t tb, int64_t pe, bool, bool) {
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int u, int64_t tb, int64_t pe, bool first, bool) {
       const int s = t % A_NS;
+      bool ok = true;
+      if (first && (piece == 0 || per_user)) {
+        // the P' slice: once, or at every user's first tile when the prototypes are per user
+        if (lane == 0) {
+          if (piece > 0) ok = mbar_wait(&bars->pq_empty, (piece - 1) & 1, abort, p.err);
+          if (ok) {
+            mbar_arrive_expect_tx(&bars->pq_full, T_BYTES);
+            const int prow = u * p.p_user_rows + sl * TILE;
+            tma_load_2d(smem + A_OFF_PQ, &tmP, &bars->pq_full, 0, prow);
+            tma_load_2d(smem + A_OFF_PQ + T_BYTES / 2, &tmP, &bars->pq_full, 64, prow);
+            pq_issued = piece + 1;
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return false;
+      }
       if (t == 0) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -427,9 +444,6 @@ __global__ void __launch_bounds__(A_THREADS, 1)
         const int64_t tok = nb + 32 * i + lane;
         if (tok < n_total) nxt[i] = p.lse[tok];
       }
-      // lane 0 waits for the stage and tells the warp (a uniform decision: no lane may be
-      // left behind at the __syncwarp below)
-      bool ok = true;
       if (t >= A_NS && lane == 0) ok = mbar_wait(&bars->x_empty[s], ((t / A_NS) - 1) & 1, abort, p.err);
       if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return false;
       float* ls = (float*)(smem + A_OFF_LSE) + s * TILE;
@@ -440,33 +454,36 @@ __global__ void __launch_bounds__(A_THREADS, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bars->x_full[s], 8 * X_BOX);
+        mbar_arrive_expect_tx(&bars->x_full[s], X_STAGE);
         uint8_t* dst = smem + A_OFF_X + s * X_STAGE;
         for (int bx = 0; bx < 8; ++bx) tma_load_2d(dst + bx * X_BOX, &tmX, &bars->x_full[s], 16 * bx, (int)tb);
       }
       issued = t + 1;
       return true;
     });
-    if (*abort && lane == 0)
+    if (*abort && lane == 0) {
+      if (pq_issued > 0) mbar_wait_bounded(&bars->pq_full, (pq_issued - 1) & 1);
       for (int t = std::max(0, issued - A_NS); t < issued; ++t)
         mbar_wait_bounded(&bars->x_full[t % A_NS], (t / A_NS) & 1);
+    }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ logits MMAs
     const uint32_t id1 = idesc_bf16(128, 128, false, false);
+    const uint64_t dp = smem_desc(smem_u32(smem + A_OFF_PQ), 16, 1024, SWZ_128B);
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t, int64_t, bool first, bool last) {
-      const int s = t % A_NS, b = t & 1;
+      const int s = t % A_NS, b = t % A_NZ;
       if (first && (piece == 0 || per_user) &&
           !mbar_wait(&bars->pq_full, (per_user ? piece : 0) & 1, abort, p.err))
         return false;
       if (!mbar_wait(&bars->x_full[s], (t / A_NS) & 1, abort, p.err)) return false;
-      // buffer b was last read (as probabilities) by the aggregation of tile t - 2
-      if (t >= 2 && !mbar_wait(&bars->z_free[b], ((t >> 1) - 1) & 1, abort, p.err)) return false;
+      // buffer b was last read (as probabilities) by the aggregation of tile t - A_NZ
+      if (t >= A_NZ && !mbar_wait(&bars->z_free[b], ((t / A_NZ) - 1) & 1, abort, p.err)) return false;
       tc_fence_after();
-      const uint32_t xa = smem_u32(smem + A_OFF_X + s * X_STAGE);
+      const uint64_t dx = smem_desc(smem_u32(smem + A_OFF_X + s * X_STAGE), 16, 256, SWZ_32B);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
-        mma_ts(tmem + A_TM_Z + 128 * b, tmem + A_TM_PQ + 8 * ks, smem_desc(xa + ks * X_BOX, 16, 256, SWZ_32B),
-               id1, ks > 0 ? 1u : 0u);
+        mma_ss(tmem + A_TM_Z + 128 * b, dp + (uint64_t)((((ks >> 2) * (T_BYTES / 2)) + (ks & 3) * 32) >> 4),
+               dx + (uint64_t)((ks * X_BOX) >> 4), id1, ks > 0 ? 1u : 0u);
       mma_commit(&bars->z_full[b]);
       if (last && per_user) mma_commit(&bars->pq_empty);   // this user's P' slice is done
       return true;
@@ -475,18 +492,18 @@ __global__ void __launch_bounds__(A_THREADS, 1)
     mbar_wait_bounded(&bars->mma_done[0], 0);
   } else if (warp == 2 && lane == 0) {
     // ------------------------------------------------------------ aggregation MMAs
-    const uint32_t id2 = idesc_bf16(128, N2, false, true);
+    const uint32_t id2 = idesc_bf16(128, DD, false, true);
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t, int64_t, bool first, bool last) {
-      const int s = t % A_NS, b = t & 1;
+      const int s = t % A_NS, b = t % A_NZ;
       if (first && piece > 0 && !mbar_wait(&bars->h_empty, (piece - 1) & 1, abort, p.err)) return false;
-      if (!mbar_wait(&bars->p_full[b], (t >> 1) & 1, abort, p.err)) return false;
+      if (!mbar_wait(&bars->p_full[b], (t / A_NZ) & 1, abort, p.err)) return false;
       tc_fence_after();
-      const uint32_t xa = smem_u32(smem + A_OFF_X + s * X_STAGE);
+      const uint64_t dx = smem_desc(smem_u32(smem + A_OFF_X + s * X_STAGE), X_BOX, 256, SWZ_32B);
       // tokens 16 ks .. 16 ks + 15: warpgroup ks / 4 wrote their pairs at its column base
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
         mma_ts(tmem + A_TM_H, tmem + A_TM_Z + 128 * b + 64 * (ks >> 2) + 8 * (ks & 3),
-               smem_desc(xa + ks * 512, X_BOX, 256, SWZ_32B), id2, (first && ks == 0) ? 0u : 1u);
+               dx + (uint64_t)((ks * 512) >> 4), id2, (first && ks == 0) ? 0u : 1u);
       mma_commit(&bars->x_empty[s]);
       mma_commit(&bars->z_free[b]);
       if (last) mma_commit(&bars->h_full);
@@ -495,28 +512,14 @@ __global__ void __launch_bounds__(A_THREADS, 1)
     mma_commit(&bars->mma_done[1]);
     mbar_wait_bounded(&bars->mma_done[1], 0);
   } else if (warp >= 3 && warp <= 6) {
-    // ------------------------------------------------------------ P' into TMEM, H out of it
+    // ------------------------------------------------------------ H and the mass out of the SM
     const int q = warp % 4;
     const int row = q * 32 + lane;                     // prototype of the slice = TMEM lane
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
     const int64_t cb = (int64_t)g * p.ch.T, ce = min(cb + p.ch.T, p.ch.n_total);
-    auto stage = [&](int u) {
-      const uint4* src = (const uint4*)(p.Pb + ((int64_t)u * p.p_user_rows + sl * TILE + row) * DD);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 x = src[8 * c + i];
-          v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
-        }
-        tmem_st32(tmem + lane_addr + A_TM_PQ + 32 * c, v);
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      mbar_arrive(&bars->pq_full);
-    };
-    auto drain = [&](int piece, int u) -> bool {
+    const float* msl = (const float*)(smem + A_OFF_M);
+    for_each_tile(p.off, p.B, p.ch, g, [&](int, int piece, int u, int64_t, int64_t, bool, bool last) {
+      if (!last) return true;
       if (!mbar_wait(&bars->h_full, piece & 1, abort, p.err)) return false;
       tc_fence_after();
       const int dest = piece_dest(p.off[u], p.off[u + 1], cb, ce);
@@ -530,48 +533,38 @@ __global__ void __launch_bounds__(A_THREADS, 1)
         Hrow = p.slotH + (((int64_t)g * 2 + dest) * p.k + j) * DD;
         mrow = p.slotM + ((int64_t)g * 2 + dest) * p.k + j;
       }
-      float hv[32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        tmem_ld32(tmem + lane_addr + A_TM_H + 32 * c, hv);
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        float hv[16];
+        tmem_ld16(tmem + lane_addr + A_TM_H + 16 * c, hv);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *(float4*)(Hrow + 32 * c + i) = make_float4(hv[i], hv[i + 1], hv[i + 2], hv[i + 3]);
+        for (int i = 0; i < 16; i += 4)
+          *(float4*)(Hrow + 16 * c + i) = make_float4(hv[i], hv[i + 1], hv[i + 2], hv[i + 3]);
       }
-      const float mass = tmem_ld1(tmem + lane_addr + A_TM_H + DD);
-      tmem_wait_ld();
-      *mrow = mass;
       tc_fence_before();
       mbar_arrive(&bars->h_empty);
-      return true;
-    };
-    int npieces = 0, prev_u = 0;
-    bool ok = true;
-    for_each_tile(p.off, p.B, p.ch, g, [&](int, int piece, int u, int64_t, int64_t, bool first, bool) {
-      if (!first) return true;
-      if (piece == 0 || per_user) {
-        // a new user's prototypes replace the slice once the last user's logits MMAs are done
-        if (piece > 0 && !mbar_wait(&bars->pq_empty, (piece - 1) & 1, abort, p.err)) { ok = false; return false; }
-        stage(u);
-      }
-      if (piece > 0 && !drain(piece - 1, prev_u)) { ok = false; return false; }
-      prev_u = u;
-      npieces = piece + 1;
+      // the piece's mass: the two softmax warpgroups' sums of this prototype's probabilities
+      const int slot = piece & 1;
+      if (!mbar_wait(&bars->m_full[slot], (piece >> 1) & 1, abort, p.err)) return false;
+      *mrow = msl[(slot * 2 + 0) * TILE + row] + msl[(slot * 2 + 1) * TILE + row];
+      mbar_arrive(&bars->m_empty[slot]);
       return true;
     });
-    if (ok && npieces > 0) drain(npieces - 1, prev_u);
   } else if (warp >= 7) {
     // ------------------------------------------------------------ probabilities
     // warpgroup h owns tokens 64h..64h+63 of each tile (TMEM columns of the buffer);
     // each thread one prototype (TMEM lane)
     const int q = warp % 4, h = (warp - 7) / 4;
+    const int row = q * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
-    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int, int, int64_t, int64_t, bool, bool) {
-      const int s = t % A_NS, b = t & 1;
+    float* msl = (float*)(smem + A_OFF_M);
+    float2 msum = make_float2(0.f, 0.f);
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t, int64_t, bool, bool last) {
+      const int s = t % A_NS, b = t % A_NZ;
       // the stage's -lse values were written before its x_full arrival
       if (!mbar_wait(&bars->x_full[s], (t / A_NS) & 1, abort, p.err)) return false;
-      if (!mbar_wait(&bars->z_full[b], (t >> 1) & 1, abort, p.err)) return false;
+      if (!mbar_wait(&bars->z_full[b], (t / A_NZ) & 1, abort, p.err)) return false;
       tc_fence_after();
       const uint32_t zc = tmem + lane_addr + A_TM_Z + 128 * b + 64 * h;
       const float4* nl = (const float4*)((const float*)(smem + A_OFF_LSE) + s * TILE + 64 * h);
@@ -590,6 +583,7 @@ __global__ void __launch_bounds__(A_THREADS, 1)
           const float2 e1 = __fadd2_rn(make_float2(z[j + 2], z[j + 3]), make_float2(l.z, l.w));
           const float2 v0 = ((SA_FWD_POLY_PAIRS >> ((j / 2) & 3)) & 1) ? exp2_pair<true>(e0) : exp2_pair<false>(e0);
           const float2 v1 = ((SA_FWD_POLY_PAIRS >> ((j / 2 + 1) & 3)) & 1) ? exp2_pair<true>(e1) : exp2_pair<false>(e1);
+          msum = __fadd2_rn(msum, __fadd2_rn(v0, v1));
           o[j / 2] = pack_bf16x2(v0.x, v0.y);
           o[j / 2 + 1] = pack_bf16x2(v1.x, v1.y);
         }
@@ -598,6 +592,15 @@ __global__ void __launch_bounds__(A_THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars->p_full[b]);
+      if (last) {
+        // hand this warpgroup's part of the prototype's mass to the drain (slot piece % 2,
+        // free once the drain of piece - 2 has read it)
+        const int slot = piece & 1;
+        if (piece >= 2 && !mbar_wait(&bars->m_empty[slot], ((piece >> 1) - 1) & 1, abort, p.err)) return false;
+        msl[(slot * 2 + h) * TILE + row] = msum.x + msum.y;
+        mbar_arrive(&bars->m_full[slot]);
+        msum = make_float2(0.f, 0.f);
+      }
       return true;
     });
   }
@@ -662,10 +665,10 @@ sa_status sa_tc_forward(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st)
   const Chunking ch1 = make_chunking(a.n_total, device_info().sm_count, 1);
   LParams lp{a.off_dev, a.B, ch1, a.k, lse_a, a_scale, lse_b, a.p_user_rows, device_status_word()};
   SA_TIMED("sa_lse_tc_kernel", st, (sa_lse_tc_kernel<<<ch1.G, L_THREADS, L_SMEM, st>>>(tmX128, tmP, lp)));
-  AParams ap{a.off_dev, a.B, w.ch, a.k, lse_a, in_scale, w.Pb, a.S, w.Muser, w.slotH, w.slotM,
-             a.p_user_rows, device_status_word()};
+  AParams ap{a.off_dev, a.B, w.ch, a.k, lse_a, in_scale, a.S, w.Muser, w.slotH, w.slotM, a.p_user_rows,
+             device_status_word()};
   SA_TIMED("sa_agg_tc_kernel", st,
-           (sa_agg_tc_kernel<<<(a.k / TILE) * w.ch.G, A_THREADS, A_SMEM, st>>>(tmX32, ap)));
+           (sa_agg_tc_kernel<<<(a.k / TILE) * w.ch.G, A_THREADS, A_SMEM, st>>>(tmX32, tmP, ap)));
   return SA_OK;
 }
 
