@@ -407,6 +407,62 @@ def sa_refine_user(Xu, P0, layers, ln_eps: float = 1e-5) -> np.ndarray:
     return Xt
 
 
+REFINE_WEIGHTS = ("W_Q", "W_K", "W1", "W3", "W2", "ln1_g", "ln1_b", "ln2_g", "ln2_b")
+
+
+def sa_refine_grads(X, offsets: Sequence[int], P0, layers, dout, ln_eps: float = 1e-5):
+    """Gradients of sum(dout * sa_refine(...)) with respect to X, P0 and every weight of
+    every iteration, by reverse-mode differentiation (torch autograd, fp64, CPU) of the
+    same definition as ``sa_refine_user`` written with torch operations: per user and
+    iteration, S = (X~ W_Q)(X W_K)^T / sqrt(d), the softmax over prototypes, X^ = A X,
+    Xbar = LN(X~ + X^), X~ = LN(Xbar + FFN(Xbar)) (eqs. (12)-(16)).  The weights are
+    shared by the users, so their gradients are sums over users.  Returns
+    {"dX": [n, d], "dP0": [k, d], "layers": [{name: grad or None}]}."""
+    import torch
+
+    t = lambda a: torch.tensor(_f64(a), dtype=torch.float64)
+    Xv = t(X).requires_grad_(True)
+    P0v = t(P0).requires_grad_(True)
+    W = [{k: (t(L[k]).requires_grad_(True) if L.get(k) is not None else None) for k in REFINE_WEIGHTS}
+         for L in layers]
+
+    def ln(y, g, b):
+        mu = y.mean(dim=-1, keepdim=True)
+        var = ((y - mu) ** 2).mean(dim=-1, keepdim=True)
+        out = (y - mu) / torch.sqrt(var + ln_eps)
+        if g is not None:
+            out = out * g
+        if b is not None:
+            out = out + b
+        return out
+
+    d = Xv.shape[1]
+    offsets = np.asarray(offsets, np.int64)
+    total = P0v.sum() * 0.0
+    dt = t(dout)
+    for u in range(len(offsets) - 1):
+        Xu = Xv[int(offsets[u]):int(offsets[u + 1])]
+        Xt = P0v
+        for w in W:
+            if Xu.shape[0] > 0:
+                S = (Xt @ w["W_Q"]) @ (Xu @ w["W_K"]).T / math.sqrt(d)
+                Xhat = torch.softmax(S, dim=0) @ Xu
+            else:
+                Xhat = torch.zeros_like(Xt)
+            Xbar = ln(Xt + Xhat, w["ln1_g"], w["ln1_b"])
+            a = Xbar @ w["W1"]
+            Xt = ln(Xbar + ((a / (1.0 + torch.exp(-a))) * (Xbar @ w["W3"])) @ w["W2"], w["ln2_g"], w["ln2_b"])
+        total = total + (Xt * dt[u]).sum()
+    leaves = [Xv, P0v] + [v for w in W for v in w.values() if v is not None]
+    grads = torch.autograd.grad(total, leaves, allow_unused=True)
+    g = iter(grads)
+    z = lambda v, r: (torch.zeros_like(v) if r is None else r).numpy()
+    res = {"dX": z(Xv, next(g)), "dP0": z(P0v, next(g)), "layers": []}
+    for w in W:
+        res["layers"].append({k: (z(v, next(g)) if v is not None else None) for k, v in w.items()})
+    return res
+
+
 def sa_refine(X, offsets: Sequence[int], P0, layers, ln_eps: float = 1e-5) -> np.ndarray:
     """Refined sketches of a ragged batch: [B, k, d] fp64."""
     offsets = np.asarray(offsets, np.int64)
