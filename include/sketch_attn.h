@@ -240,6 +240,48 @@ sa_status sa_refine_forward(const void* X, sa_dtype x_dtype, const int64_t* offs
                             float* sketch, void* workspace, size_t ws_bytes,
                             sa_stream_t stream);
 
+/* Gradients of one refinement iteration's parameters (fp32 device buffers shaped as
+ * the parameters; written, not accumulated; sums over the users).  A gradient whose
+ * parameter is NULL in the layer is not written (its pointer may be NULL). */
+typedef struct {
+  float* dW_Q;
+  float* dW_K;
+  float* dln1_g;
+  float* dln1_b;
+  float* dW1;
+  float* dW3;
+  float* dW2;
+  float* dln2_g;
+  float* dln2_b;
+} sa_refine_layer_grad;
+
+size_t sa_refine_backward_workspace(int B, int64_t n_total, int k, int d, int n_iter, sa_dtype x_dtype);
+
+/*
+ * sa_refine_backward -- the backward of sa_refine_forward (paper Sec. 3.3, eqs.
+ * (12)-(16), trained end to end): given dsketch [B, k, d] fp32, the gradient of
+ * the returned sketch, writes
+ *   dX   [n_total, d] fp32: the gradient with respect to the events' rows;
+ *   dP0  [k, d] fp32: the gradient with respect to the shared prototypes;
+ *   grads[i]: the gradients of iteration i's parameters.
+ * Inputs as sa_refine_forward (bf16 X, d = 128, k a multiple of 128 up to 4096,
+ * n_iter <= 8).  The forward is recomputed with its intermediates kept in the
+ * workspace.  Per iteration, from the last: the LayerNorm and SwiGLU backward
+ * (the FFN products on the tensor cores over hi + lo bf16 splits), then the SA
+ * backward of X^ = A X_u with every user's own prototypes (the tensor-core
+ * kernels of sa_backward, run user by user, dX accumulated in fp32): dA = dX^ . x,
+ * c = sum_j A dA, dZ = A (dA - c), dX += A dX^ + dZ (X~ W_Q W_K^T)/sqrt(d),
+ * E_u = dZ^T X_u, dX~ += E_u W_K W_Q^T / sqrt(d), and the W_Q, W_K gradients
+ * summed over users.  Workspace: sa_refine_backward_workspace bytes, 16-byte
+ * aligned, caller owned.  Asynchronous on `stream`.
+ */
+sa_status sa_refine_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                             const int64_t* offsets_dev, int B, int k, int d, const float* P0,
+                             int n_iter, const sa_refine_layer* layers, float ln_eps,
+                             const float* dsketch, float* dX, float* dP0,
+                             const sa_refine_layer_grad* grads, void* workspace, size_t ws_bytes,
+                             sa_stream_t stream);
+
 /*
  * sa_gather_events -- the events' input rows on the device: for i < n
  *   X[i] = item_table[item_ids[i]] + action_table[action_ids[i]]
@@ -432,7 +474,7 @@ sa_status stca_fuse(const float* z_r, const float* z_u, const float* W_F, const 
 /*
  * Exponentials per second on the current GPU (all SMs, synchronous): mode 0 with
  * every 2^x on the MUFU (ex2.approx), mode 1 with the SA forward kernels' mix
- * (one pair in four by a cubic on the FMA pipe).  The co-roofline of the
+ * (one pair in eight by a cubic on the FMA pipe).  The co-roofline of the
  * forward: each of its two kernels evaluates k exponentials per token.
  */
 sa_status sa_measure_exp2_rate(int mode, double* per_second, sa_stream_t stream);

@@ -32,7 +32,8 @@ EXPORTS = ("sa_version", "sa_last_error", "sa_poll_device_status", "sa_forward_w
            "sa_forward_tokenwise_workspace", "sa_forward_tokenwise", "sa_backward_accumulate",
            "stca_forward_full_workspace", "stca_forward_full", "stca_backward_full_workspace",
            "stca_backward_full", "sa_gather_events", "sa_gather_events_fused",
-           "sa_gather_events_fused_workspace", "sa_measure_exp2_rate", "sa_selftest_bounded_wait")
+           "sa_gather_events_fused_workspace", "sa_measure_exp2_rate", "sa_selftest_bounded_wait",
+           "sa_refine_backward_workspace", "sa_refine_backward")
 
 
 class SAError(RuntimeError):
@@ -63,6 +64,13 @@ class StcaFullLayerGradC(ctypes.Structure):
 class RefineLayerC(ctypes.Structure):
     _fields_ = [(k, ctypes.c_void_p) for k in ("W_Q", "W_K", "ln1_g", "ln1_b", "W1", "W3", "W2",
                                                "ln2_g", "ln2_b")]
+
+
+REFINE_GRAD_KEYS = ("dW_Q", "dW_K", "dln1_g", "dln1_b", "dW1", "dW3", "dW2", "dln2_g", "dln2_b")
+
+
+class RefineLayerGradC(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in REFINE_GRAD_KEYS]
 
 
 _lib = None
@@ -137,6 +145,11 @@ def load(path: Optional[str] = None):
     lib.sa_refine_forward.restype = _i
     lib.sa_refine_forward.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _i,
                                       ctypes.POINTER(RefineLayerC), _f, _vp, _vp, _sz, _vp]
+    lib.sa_refine_backward_workspace.restype = _sz
+    lib.sa_refine_backward_workspace.argtypes = [_i, _i64, _i, _i, _i, _i]
+    lib.sa_refine_backward.restype = _i
+    lib.sa_refine_backward.argtypes = [_vp, _i, _vp, _vp, _i, _i, _i, _vp, _i, ctypes.POINTER(RefineLayerC), _f,
+                                       _vp, _vp, _vp, ctypes.POINTER(RefineLayerGradC), _vp, _sz, _vp]
     lib.sa_launch_count.restype = ctypes.c_longlong
     lib.sa_profile.restype = _i
     lib.sa_profile.argtypes = [_i]
@@ -596,6 +609,51 @@ def sa_refine_forward(X: torch.Tensor, offsets, P0: torch.Tensor, layers: Sequen
                                ln_eps, _p(res), _p(workspace), workspace.numel(), _stream(stream))
     _check("sa_refine_forward", st)
     return res
+
+
+def sa_refine_backward_workspace(B: int, n_total: int, k: int, d: int, n_iter: int, dtype: int) -> int:
+    return int(load().sa_refine_backward_workspace(B, n_total, k, d, n_iter, dtype))
+
+
+def sa_refine_backward(X: torch.Tensor, offsets, P0: torch.Tensor, layers: Sequence[dict], dsketch: torch.Tensor,
+                       ln_eps: float = 1e-5, *, offsets_dev=None, out: Optional[dict] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Gradients of <dsketch, sa_refine_forward(X, offsets, P0, layers)>: returns
+    {"dX": [n, d] fp32, "dP0": [k, d] fp32, "layers": [{"dW_Q", "dW_K", "dW1", "dW3", "dW2",
+    and "dln1_g", ... for the LayerNorm parameters the layer has}]}."""
+    lib = load()
+    _need_cuda(X, P0, dsketch)
+    dt = _dtype_code(X)
+    off = _host_i64(offsets)
+    B = len(off) - 1
+    k, d = P0.shape
+    n = int(off[-1])
+    dev = X.device
+    o = dict(out or {})
+    dX = o.get("dX") if o.get("dX") is not None else torch.empty(max(n, 1), d, device=dev)
+    dP0 = o.get("dP0") if o.get("dP0") is not None else torch.empty(k, d, device=dev)
+    arr = (RefineLayerC * len(layers))()
+    garr = (RefineLayerGradC * len(layers))()
+    gl = []
+    for i, L in enumerate(layers):
+        g = {}
+        for key in REFINE_KEYS:
+            t = L.get(key)
+            _need_cuda(t)
+            setattr(arr[i], key, t.data_ptr() if t is not None else None)
+            if t is not None:
+                g["d" + key] = torch.empty_like(t)
+                setattr(garr[i], "d" + key, g["d" + key].data_ptr())
+        gl.append(g)
+    ws_bytes = lib.sa_refine_backward_workspace(B, n, k, d, len(layers), dt)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    od = _dev_i64(off, dev, offsets_dev)
+    st = lib.sa_refine_backward(_p(X), dt, _hp(off), _p(od), B, k, d, _p(P0), len(layers), arr, ln_eps,
+                                _p(dsketch), _p(dX), _p(dP0), garr, _p(workspace), workspace.numel(),
+                                _stream(stream))
+    _check("sa_refine_backward", st)
+    return {"dX": dX[:n], "dP0": dP0, "layers": gl}
 
 
 def stca_fuse(z_r: torch.Tensor, z_u: torch.Tensor, W_F: torch.Tensor, b_F=None, *,

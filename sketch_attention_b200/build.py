@@ -11,7 +11,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsketchattn.so")
-SOURCES = ["api.cu", "gemm.cu", "sa_simt.cu", "sa_tc.cu", "sa_bwd_tc.cu", "sa_refine.cu", "sa_tokenwise.cu", "sa_noalloc.cu", "stca.cu",
+SOURCES = ["api.cu", "gemm.cu", "sa_simt.cu", "sa_tc.cu", "sa_bwd_tc.cu", "sa_refine.cu", "sa_refine_bwd.cu", "sa_tokenwise.cu", "sa_noalloc.cu", "stca.cu",
            "stca_tc.cu", "stca_full.cu", "stca_ffn_tc.cu", "stca_bwd.cu", "events.cu", "measure.cu", "tc_gemm.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -224,15 +224,7 @@ size_t layout_bwd(void* base, int B, int64_t n, int k, int d, sa_dtype dt, SaBwd
 
 size_t layout_stca(void* base, int B, int64_t C, int D, int heads, int d_h, StcaWork* w) {
   Carve c(base);
-  StcaWork v;
-  const size_t rows = (size_t)std::max<int64_t>(C, 1);
-  v.Qh = c.take<float>(rows * heads * d_h);
-  v.U = c.take<float>(rows * heads * D);
-  v.Ub = c.take<__nv_bfloat16>(rows * heads * D);
-  v.Y = c.take<float>(rows * heads * D);
-  v.O = c.take<float>(rows * heads * d_h);
-  v.tile_prefix = c.take<int>((size_t)B + 1);
-  v.max_tiles = 0;
+  StcaWork v = stca_attn_carve(c, B, C, D, heads, d_h);
   if (w) *w = v;
   return c.bytes();
 }
@@ -425,6 +417,61 @@ sa_status sa_refine_forward(const void* X, sa_dtype x_dtype, const int64_t* offs
   refine_layout(workspace, B, n, k, d, &w, &r);
   return sa_refine_run(X, x_dtype, offsets_dev, B, n, k, d, P0, n_iter, layers, ln_eps, sketch, w, r,
                        (cudaStream_t)stream);
+}
+
+size_t sa_refine_backward_workspace(int B, int64_t n_total, int k, int d, int n_iter, sa_dtype x_dtype) {
+  if (B < 1 || n_total < 0 || n_iter < 1 || n_iter > 8 || !sa_tc_supported(x_dtype, k, d)) return 0;
+  return refine_bwd_layout(nullptr, B, n_total, k, d, n_iter, nullptr);
+}
+
+sa_status sa_refine_backward(const void* X, sa_dtype x_dtype, const int64_t* offsets_host,
+                             const int64_t* offsets_dev, int B, int k, int d, const float* P0,
+                             int n_iter, const sa_refine_layer* layers, float ln_eps,
+                             const float* dsketch, float* dX, float* dP0,
+                             const sa_refine_layer_grad* grads, void* workspace, size_t ws_bytes,
+                             sa_stream_t stream) {
+  SA_TRY(check_sa_shape(B, k, d, x_dtype));
+  if (!sa_tc_supported(x_dtype, k, d))
+    return fail(SA_ERR_UNSUPPORTED, "sa_refine_backward needs bf16 X, d = 128 and k a multiple of 128");
+  SA_TRY(check_offsets(offsets_host, B, "offsets_host"));
+  const int64_t n = offsets_host[B];
+  if (n >= (1LL << 31)) return fail(SA_ERR_UNSUPPORTED, "n_total must be < 2^31");
+  if (n_iter < 1 || n_iter > 8) return fail(SA_ERR_UNSUPPORTED, "n_iter must be 1..8");
+  if (!layers || !grads) return fail(SA_ERR_INVALID_ARG, "layers or grads is NULL");
+  if (!(ln_eps > 0.f)) return fail(SA_ERR_INVALID_ARG, "ln_eps must be > 0");
+  if ((int64_t)B * k >= (1LL << 31)) return fail(SA_ERR_UNSUPPORTED, "B * k must be < 2^31");
+  SA_TRY(check_ptr(X, "X", n == 0));
+  SA_TRY(check_ptr(offsets_dev, "offsets_dev"));
+  SA_TRY(check_ptr(P0, "P0"));
+  SA_TRY(check_ptr(dsketch, "dsketch"));
+  SA_TRY(check_ptr(dX, "dX", n == 0));
+  SA_TRY(check_ptr(dP0, "dP0"));
+  for (int i = 0; i < n_iter; ++i) {
+    const sa_refine_layer& L = layers[i];
+    const sa_refine_layer_grad& G = grads[i];
+    SA_TRY(check_ptr(L.W_Q, "layers[].W_Q"));
+    SA_TRY(check_ptr(L.W_K, "layers[].W_K"));
+    SA_TRY(check_ptr(L.W1, "layers[].W1"));
+    SA_TRY(check_ptr(L.W3, "layers[].W3"));
+    SA_TRY(check_ptr(L.W2, "layers[].W2"));
+    SA_TRY(check_ptr(G.dW_Q, "grads[].dW_Q"));
+    SA_TRY(check_ptr(G.dW_K, "grads[].dW_K"));
+    SA_TRY(check_ptr(G.dW1, "grads[].dW1"));
+    SA_TRY(check_ptr(G.dW3, "grads[].dW3"));
+    SA_TRY(check_ptr(G.dW2, "grads[].dW2"));
+    const float* opt[4] = {L.ln1_g, L.ln1_b, L.ln2_g, L.ln2_b};
+    float* const gopt[4] = {G.dln1_g, G.dln1_b, G.dln2_g, G.dln2_b};
+    for (int j = 0; j < 4; ++j) {
+      SA_TRY(check_ptr(opt[j], "a LayerNorm parameter", true));
+      if (opt[j]) SA_TRY(check_ptr(gopt[j], "the gradient of a LayerNorm parameter"));
+    }
+  }
+  const size_t need = refine_bwd_layout(nullptr, B, n, k, d, n_iter, nullptr);
+  if (!workspace || ws_bytes < need)
+    return fail(SA_ERR_WORKSPACE, "workspace needs " + std::to_string(need) + " bytes");
+  SA_TRY(check_ptr(workspace, "workspace"));
+  return sa_refine_backward_run(X, offsets_host, offsets_dev, B, n, k, d, P0, n_iter, layers, ln_eps, dsketch,
+                                dX, dP0, grads, workspace, (cudaStream_t)stream);
 }
 
 size_t sa_backward_workspace(int B, int64_t n_total, int k, int d, sa_dtype x_dtype) {

@@ -4,7 +4,7 @@
 //
 // Every thread keeps 16 independent values v <- 2^(v - 1) (bounded in (1/2, 1]),
 // so the loop is limited by exponential throughput, not latency.  Mode 0: all
-// on the MUFU (ex2.approx); mode 1: the forward kernels' mix, one pair in four
+// on the MUFU (ex2.approx); mode 1: the forward kernels' mix, one pair in eight
 // by the cubic on the FMA pipe (exp2_poly.cuh).
 #include <algorithm>
 
@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(kThreads) exp2_rate_kernel(float* __restrict__
 #pragma unroll
     for (int j = 0; j < kPairs; ++j) {
       const float2 e = __fadd2_rn(v[j], m1);
-      v[j] = (MODE == 1 && (j & 3) == 1) ? exp2_poly2(e) : make_float2(tc::ex2(e.x), tc::ex2(e.y));
+      v[j] = (MODE == 1 && (j & 7) == 1) ? exp2_poly2(e) : make_float2(tc::ex2(e.x), tc::ex2(e.y));
     }
   }
   float s = 0.f;

@@ -35,7 +35,7 @@
 // Pairs (of the 4 in a group of 8 prototypes) whose exponentials the E kernel
 // evaluates on the FMA pipe instead of the MUFU.
 #ifndef SA_E_POLY_PAIRS
-#define SA_E_POLY_PAIRS 0x2
+#define SA_E_POLY_PAIRS 0x0
 #endif
 
 namespace sa {
@@ -94,9 +94,11 @@ struct DxParams {
   int k;
   const float* lse2;     // [n] per-token log2-sum-exp
   const float* dmc;      // [B, k] centred dm
-  __nv_bfloat16* dX;     // [n, d]
+  __nv_bfloat16* dX;     // [n, d] (unless dX32)
   float* cout;           // [n]
   int* err;
+  float* dX32;           // optional [n, d] fp32 output instead of dX, added to when acc32
+  int acc32;
 };
 
 // 384: caps registers at 168, as three warps share two of the SM's sub-partitions
@@ -332,7 +334,19 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld32(tmem + lane_addr + DX_TM_V + 32 * qb, v);
         tmem_ld32(tmem + lane_addr + DX_TM_Q + 32 * qb, qv);
         tmem_wait_ld();
-        if (valid) {
+        if (valid && p.dX32) {
+          float4* dst = (float4*)(p.dX32 + (tb + row) * DD + 32 * qb);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 o = make_float4(fmaf(-lc, v[4 * i], qv[4 * i]), fmaf(-lc, v[4 * i + 1], qv[4 * i + 1]),
+                                   fmaf(-lc, v[4 * i + 2], qv[4 * i + 2]), fmaf(-lc, v[4 * i + 3], qv[4 * i + 3]));
+            if (p.acc32) {
+              const float4 a0 = dst[i];
+              o.x += a0.x; o.y += a0.y; o.z += a0.z; o.w += a0.w;
+            }
+            dst[i] = o;
+          }
+        } else if (valid) {
           uint32_t o[16];
 #pragma unroll
           for (int i = 0; i < 32; i += 2)
@@ -636,7 +650,8 @@ sa_status sa_bwd_tc_run(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st)
   if ((s = map_rows(&tmL64, w.dHlo, (uint64_t)a.B * a.k, 64)) != SA_OK) return s;
   if ((s = map_rows(&tmP128, w.Pb, (uint64_t)a.k, 128)) != SA_OK) return s;
   if ((s = map_rows(&tmH128, w.dHb, (uint64_t)a.B * a.k, 128)) != SA_OK) return s;
-  DxParams dp{a.off_dev, a.B, w.ch, a.k, w.lse, w.dmc, (__nv_bfloat16*)a.dX, w.cbuf, device_status_word()};
+  DxParams dp{a.off_dev, a.B, w.ch, a.k, w.lse, w.dmc, (__nv_bfloat16*)a.dX, w.cbuf, device_status_word(),
+              a.dX32, a.dX_acc ? 1 : 0};
   SA_TIMED("sa_bwd_dx_tc_kernel", st,
            (sa_bwd_dx_tc_kernel<<<w.ch.G, DX_THREADS, DX_SMEM, st>>>(tmX, tmP64, tmH64, tmL64, dp)));
   EParams ep{a.off_dev, a.B, w.chE, a.k, w.lse, w.cbuf, w.dmc, w.Epart, device_status_word()};

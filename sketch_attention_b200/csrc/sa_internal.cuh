@@ -37,6 +37,8 @@ struct SaBwdArgs {
   const float *H, *mass, *dS, *dmass, *lse_in;
   void* dX; float *dP, *dW_Q, *dW_K, *dW_V;
   bool accumulate = false;   // add the weight gradients into dP, dW_Q, dW_K, dW_V
+  float* dX32 = nullptr;     // tensor-core path: dX as fp32 [n, d] instead of dX (added to when dX_acc)
+  bool dX_acc = false;
 };
 
 struct SaBwdWork {
@@ -84,6 +86,14 @@ sa_status sa_refine_run(const void* X, sa_dtype x_dtype, const int64_t* off_dev,
                         float ln_eps, float* sketch, const SaFwdWork& w, const RefineWork& r,
                         cudaStream_t st);
 
+// Backward of the stacked refinement (sa_refine_bwd.cu).
+size_t refine_bwd_layout(void* base, int B, int64_t n, int k, int d, int n_iter, void* views);
+sa_status sa_refine_backward_run(const void* X, const int64_t* off_host, const int64_t* off_dev, int B,
+                                 int64_t n, int k, int d, const float* P0, int n_iter,
+                                 const sa_refine_layer* layers, float ln_eps, const float* dsketch,
+                                 float* dX, float* dP0, const sa_refine_layer_grad* grads, void* workspace,
+                                 cudaStream_t st);
+
 // Token-wise normalisation variant (sa_tokenwise.cu).
 struct TokenwiseWork {
   float* T;              // [d, d]
@@ -109,6 +119,12 @@ sa_status selftest_bounded_wait(long long budget_cycles, cudaStream_t st);
 sa_status gather_events_run(const void* item, int64_t vocab, const void* action, int n_actions,
                             const int32_t* ids, const uint8_t* acts, int64_t n, int d, void* X,
                             cudaStream_t st);
+// out[r] = LN(a[r or r % a_rows] + b[r]) * g + beta over rows of d = 128 (a_rows > 0: a holds
+// a_rows rows shared by every block of a_rows output rows); g, beta nullable
+sa_status sa_residual_ln(const float* a, int a_rows, const float* b, const float* g, const float* beta, float eps,
+                         int64_t rows, int d, float* out, cudaStream_t st);
+// out[e] = sum_{g < G} part[g][e] in a fixed order (zeros when G = 0)
+sa_status sa_sum_slices(const float* part, int G, int64_t n, float* out, cudaStream_t st);
 // U = SiLU(G1) * G3 elementwise over n fp32 values (n a multiple of 4, 16-byte aligned)
 sa_status sa_swiglu(const float* G1, const float* G3, int64_t n, float* U, cudaStream_t st);
 sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st);

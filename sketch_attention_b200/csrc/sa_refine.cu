@@ -73,6 +73,15 @@ unsigned blocks_for(int64_t n, int per_block) {
 }
 }  // namespace
 
+sa_status sa_residual_ln(const float* a, int a_rows, const float* b, const float* g, const float* beta, float eps,
+                         int64_t rows, int d, float* out, cudaStream_t st) {
+  if (rows <= 0) return SA_OK;
+  if (d != 128) return fail(SA_ERR_UNSUPPORTED, "the LayerNorm kernels take d = 128");
+  SA_TIMED("residual_ln_kernel", st,
+           (residual_ln_kernel<4><<<blocks_for(rows * 32, 256), 256, 0, st>>>(a, a_rows, b, g, beta, eps, rows, out)));
+  return SA_OK;
+}
+
 sa_status sa_swiglu(const float* G1, const float* G3, int64_t n, float* U, cudaStream_t st) {
   if (n <= 0) return SA_OK;
   SA_TIMED("swiglu_kernel", st,

@@ -572,6 +572,17 @@ sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaS
   return sa_bwd_weight_grads(a, w, st);
 }
 
+sa_status sa_sum_slices(const float* part, int G, int64_t n, float* out, cudaStream_t st) {
+  if (n <= 0) return SA_OK;
+  if (G <= 0) {
+    SA_CUDA(cudaMemsetAsync(out, 0, n * sizeof(float), st));
+    return SA_OK;
+  }
+  SA_TIMED("sum_slices_kernel", st,
+           (sum_slices_kernel<<<(unsigned)std::min<int64_t>((n + 255) / 256, 4096), 256, 0, st>>>(part, G, n, out)));
+  return SA_OK;
+}
+
 sa_status sa_bwd_weight_grads(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st) {
   const int D = a.d, k = a.k;
   const int64_t n = (int64_t)k * D;

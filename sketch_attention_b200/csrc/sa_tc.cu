@@ -33,10 +33,13 @@
 #include "tc_ptx.cuh"
 #include "tma_map.cuh"
 
-// Pairs (of the 4 in a group of 8 prototypes) whose exponentials the lse and
-// aggregation kernels evaluate on the FMA pipe instead of the MUFU.
-#ifndef SA_FWD_POLY_PAIRS
-#define SA_FWD_POLY_PAIRS 0x2
+// Pairs (bit i: pair i of each group of 8 pairs) whose exponentials the lse and
+// the aggregation kernel evaluate on the FMA pipe instead of the MUFU.
+#ifndef SA_LSE_POLY
+#define SA_LSE_POLY 0x02
+#endif
+#ifndef SA_AGG_POLY
+#define SA_AGG_POLY 0x02
 #endif
 
 namespace sa {
@@ -86,8 +89,8 @@ constexpr uint32_t L_OFF_P = L_OFF_X + L_NXS * T_BYTES;
 constexpr uint32_t L_OFF_XCH = L_OFF_P + L_NPS * T_BYTES;   // [3][2][128]: warpgroups 1-3's max and sum
 constexpr uint32_t L_OFF_BAR = L_OFF_XCH + 6 * TILE * 4;
 constexpr uint32_t L_SMEM = L_OFF_BAR + 256 + 1024;
-constexpr int L_THREADS = 704;   // warp 0 TMA, 1 MMA + TMEM owner, 2-5 and 6-9 two warpgroups,
-                                 // 10-13 X tiles from shared memory into TMEM
+constexpr int L_THREADS = 704;   // warp 0 TMA, 1 MMA + TMEM owner, 2-17 four softmax warpgroups,
+                                 // 18-21 X tiles from shared memory into TMEM
 // TMEM columns: two [128 x 128] fp32 logits buffers, two X tiles (bf16 pairs: the
 // MMA's A operand, so the logits MMAs read only P' from shared memory)
 constexpr uint32_t L_TM_Z = 0, L_TM_X = 256, L_TM_COLS = 512;
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(L_THREADS, 1)
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
           const float2 e = __fadd2_rn(make_float2(z[j], z[j + 1]), nm);
-          const float2 v = ((SA_FWD_POLY_PAIRS >> ((j / 2) & 3)) & 1) ? exp2_pair<true>(e) : exp2_pair<false>(e);
+          const float2 v = ((SA_LSE_POLY >> ((j / 2) & 7)) & 1) ? exp2_pair<true>(e) : exp2_pair<false>(e);
           s2 = __fadd2_rn(s2, v);
         }
       }
@@ -581,8 +584,8 @@ __global__ void __launch_bounds__(A_THREADS, 1)
           const float4 l = nl[8 * c + j / 4];
           const float2 e0 = __fadd2_rn(make_float2(z[j], z[j + 1]), make_float2(l.x, l.y));
           const float2 e1 = __fadd2_rn(make_float2(z[j + 2], z[j + 3]), make_float2(l.z, l.w));
-          const float2 v0 = ((SA_FWD_POLY_PAIRS >> ((j / 2) & 3)) & 1) ? exp2_pair<true>(e0) : exp2_pair<false>(e0);
-          const float2 v1 = ((SA_FWD_POLY_PAIRS >> ((j / 2 + 1) & 3)) & 1) ? exp2_pair<true>(e1) : exp2_pair<false>(e1);
+          const float2 v0 = ((SA_AGG_POLY >> ((j / 2) & 7)) & 1) ? exp2_pair<true>(e0) : exp2_pair<false>(e0);
+          const float2 v1 = ((SA_AGG_POLY >> ((j / 2 + 1) & 7)) & 1) ? exp2_pair<true>(e1) : exp2_pair<false>(e1);
           msum = __fadd2_rn(msum, __fadd2_rn(v0, v1));
           o[j / 2] = pack_bf16x2(v0.x, v0.y);
           o[j / 2 + 1] = pack_bf16x2(v1.x, v1.y);

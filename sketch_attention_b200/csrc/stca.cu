@@ -4,6 +4,9 @@
 // Per layer:  Qh = q W_Q^h;  U_h = Qh W_K^h^T * log2(e)/sqrt(d_h)  (GEMMs)
 //             Y_h = softmax_i(U_h . x_i) x  over the user's keys  (attention)
 //             O_h = Y_h W_V^h;  q <- q + concat_h(O_h) W_O          (GEMMs)
+// With bf16 inputs the projections run on the tensor cores with the heads' weights
+// folded (two GEMMs per layer, see stca_attend_layer); fp32 inputs keep the CUDA-core
+// GEMMs and attention.
 // Query rows of the attention are (candidate, head) pairs, so the history is
 // read once per tile of 32 (CUDA cores) or 128 (tensor cores) rows.
 #include <algorithm>
@@ -126,7 +129,97 @@ __global__ void __launch_bounds__(256) stca_attn_simt_kernel(
 }
 
 unsigned grid_for(int64_t n) { return (unsigned)std::min<int64_t>((n + 255) / 256, 8192); }
+
+// The heads' folded weights of one layer as hi + lo bf16 splits:
+//   M[k][h D + n] = sum_j W_Q^h[k][j] W_K^h[n][j] * scale        ([D, heads D])
+//   N[h D + k][n] = sum_j W_V^h[k][j] W_O[h d_h + j][n]          ([heads D, D]; with W_O NULL
+//                   (the identity) N[h D + k][n] = W_V^h[k][n - h d_h] inside head h's columns)
+// One block per (head, matrix, 16 rows of k); the contraction over j runs in slices of 32
+// staged in shared memory (the block's rows of W_Q^h or W_V^h, and W_K^h transposed or head
+// h's rows of W_O); D = 128, each thread 8 outputs.
+__global__ void __launch_bounds__(256) fold_heads_kernel(const float* __restrict__ W_Q, const float* __restrict__ W_K,
+                                                         const float* __restrict__ W_V, const float* __restrict__ W_O,
+                                                         int heads, int d_h, float scale,
+                                                         __nv_bfloat16* __restrict__ Mhi, __nv_bfloat16* __restrict__ Mlo,
+                                                         __nv_bfloat16* __restrict__ Nhi, __nv_bfloat16* __restrict__ Nlo) {
+  constexpr int D = 128, KR = 16, JS = 32;
+  __shared__ float a[KR][JS + 1];       // a[r][j]: W_Q^h (or W_V^h) row k0 + r, slice columns
+  __shared__ float bt[JS][D + 1];       // bt[j][n]: W_K^h[n][j] (or W_O[h d_h + j][n])
+  const int h = blockIdx.x, which = blockIdx.y, k0 = blockIdx.z * KR;
+  const bool isM = which == 0;
+  const float* Arows = (isM ? W_Q : W_V) + (int64_t)h * D * d_h;
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  if (isM || W_O) {
+    for (int j0 = 0; j0 < d_h; j0 += JS) {
+      const int js = min(JS, d_h - j0);
+      __syncthreads();
+      for (int e = threadIdx.x; e < KR * JS; e += 256) {
+        const int r = e / JS, j = e % JS;
+        a[r][j] = j < js ? Arows[(int64_t)(k0 + r) * d_h + j0 + j] : 0.f;
+      }
+      for (int e = threadIdx.x; e < JS * D; e += 256) {
+        const int j = e / D, n = e % D;
+        float x = 0.f;
+        if (j < js) x = isM ? W_K[((int64_t)h * D + n) * d_h + j0 + j] : W_O[((int64_t)h * d_h + j0 + j) * D + n];
+        bt[j][n] = x;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = threadIdx.x + 256 * i, r = e / D, n = e % D;
+        for (int j = 0; j < js; ++j) v[i] = fmaf(a[r][j], bt[j][n], v[i]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = threadIdx.x + 256 * i, r = e / D, n = e % D, k = k0 + r;
+    float x = v[i];
+    if (isM) {
+      x *= scale;
+    } else if (!W_O) {
+      x = (n >= h * d_h && n < (h + 1) * d_h) ? Arows[(int64_t)k * d_h + (n - h * d_h)] : 0.f;
+    }
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+    if (isM) {
+      const int64_t o = (int64_t)k * heads * D + h * D + n;
+      Mhi[o] = hi;
+      Mlo[o] = lo;
+    } else {
+      const int64_t o = ((int64_t)h * D + k) * D + n;
+      Nhi[o] = hi;
+      Nlo[o] = lo;
+    }
+  }
+}
 }  // namespace
+
+StcaWork stca_attn_carve(Carve& c, int B, int64_t C, int D, int heads, int d_h) {
+  StcaWork v;
+  const size_t rows = (size_t)std::max<int64_t>(C, 1);
+  const size_t HD = (size_t)heads * D;
+  v.Qh = c.take<float>(rows * heads * d_h);
+  v.U = c.take<float>(rows * HD);
+  v.Ub = c.take<__nv_bfloat16>(rows * HD);
+  v.Y = c.take<float>(rows * HD);
+  v.O = c.take<float>(rows * heads * d_h);
+  v.tile_prefix = c.take<int>((size_t)B + 1);
+  v.max_tiles = 0;
+  v.Mhi = c.take<__nv_bfloat16>((size_t)D * HD);
+  v.Mlo = c.take<__nv_bfloat16>((size_t)D * HD);
+  v.Nhi = c.take<__nv_bfloat16>(HD * D);
+  v.Nlo = c.take<__nv_bfloat16>(HD * D);
+  v.qhi = c.take<__nv_bfloat16>(rows * D);
+  v.qlo = c.take<__nv_bfloat16>(rows * D);
+  v.Yhi = c.take<__nv_bfloat16>(rows * HD);
+  v.Ylo = c.take<__nv_bfloat16>(rows * HD);
+  v.part_floats = 4 * rows * D;
+  v.part = c.take<float>(v.part_floats);
+  return v;
+}
 
 sa_status stca_begin(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
   const int64_t C = a.C_total;
@@ -146,6 +239,25 @@ sa_status stca_begin(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
   return SA_OK;
 }
 
+// The tensor-core path (bf16 inputs, D = 128): the heads' projections folded into two
+// weight matrices per layer, so each layer is two GEMMs on the tensor cores over hi + lo
+// bf16 splits of their fp32 operands (about 16 significant bits, see tc_gemm):
+//   U = q M,   M = [W_Q^h W_K^h^T log2(e)/sqrt(d_h)]_h   [D, heads D]   (16-bit output: the
+//              attention's query operand, one row of D per (candidate, head))
+//   q <- q + Y N,   N = [W_V^h W_O^h]_h                 [heads D, D]   (Y: the attention's
+//              output, [C, heads D])
+// (the associativity of eqs. (24)-(26): (q W_Q^h) W_K^h^T = q (W_Q^h W_K^h^T) and
+// sum_h (Y_h W_V^h) W_O^h = Y N).
+sa_status tc_projections_prepare(const StcaArgs& a, const stca_layer& L, const StcaWork& w, cudaStream_t st) {
+  const int D = a.D, H = a.heads, dh = a.d_h;
+  if (D != 128) return fail(SA_ERR_UNSUPPORTED, "the tensor-core projections take D = 128");
+  SA_TIMED("fold_heads_kernel", st,
+           (fold_heads_kernel<<<dim3(H, 2, D / 16), 256, 0, st>>>(L.W_Q, L.W_K, L.W_V, L.W_O, H, dh,
+                                                                  1.4426950408889634f / sqrtf((float)dh), w.Mhi,
+                                                                  w.Mlo, w.Nhi, w.Nlo)));
+  return SA_OK;
+}
+
 sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWork& w, cudaStream_t st) {
   const int D = a.D, H = a.heads, dh = a.d_h, HD = a.heads * a.d_h;
   const int64_t C = a.C_total;
@@ -153,6 +265,25 @@ sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWo
   if (C == 0) return SA_OK;
   const bool tc = stca_tc_supported(a.dtype, D);
   sa_status s;
+  if (tc) {
+    if ((s = tc_projections_prepare(a, L, w, st)) != SA_OK) return s;
+    if ((s = split_hi_lo(a.out, nq, w.qhi, w.qlo, st)) != SA_OK) return s;
+    TcGemm gu;                                // U = q M -> the attention's 16-bit queries
+    gu.M = (int)C; gu.N = H * D; gu.K = D;
+    gu.A = w.qhi; gu.A_lo = w.qlo; gu.lda = D;
+    gu.B = w.Mhi; gu.B_lo = w.Mlo; gu.ldb = (int64_t)H * D; gu.b_mn = true;
+    gu.C16 = w.Ub; gu.ldc16 = (int64_t)H * D; gu.c16_half = a.kv_f16;
+    gu.tag = "tc_gemm:stca_U";
+    if ((s = tc_gemm(gu, st)) != SA_OK) return s;
+    if ((s = stca_tc_attention(a, w, st, true)) != SA_OK) return s;
+    TcGemm go;                                // q <- q + Y N
+    go.M = (int)C; go.N = D; go.K = H * D;
+    go.A = w.Yhi; go.A_lo = w.Ylo; go.lda = (int64_t)H * D;
+    go.B = w.Nhi; go.B_lo = w.Nlo; go.ldb = D; go.b_mn = true;
+    go.C = a.out; go.ldc = D; go.Cin = a.out; go.ldcin = D;
+    go.tag = "tc_gemm:stca_O";
+    return tc_gemm(go, st);
+  }
   {
     // Qh[:, h] = q W_Q^h
     Gemm g1;
@@ -167,29 +298,21 @@ sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWo
     g2.M = (int)C; g2.N = D; g2.K = dh;
     g2.A = w.Qh; g2.lda = HD; g2.sA = dh;
     g2.B = L.W_K; g2.ldb = dh; g2.transB = true; g2.sB = (int64_t)D * dh;
-    if (tc) {
-      g2.C16 = w.Ub; g2.ldc16 = (int64_t)H * D; g2.sC16 = D;
-      g2.c16_half = a.kv_f16; g2.err = device_status_word();
-    }
-    else { g2.C = w.U; g2.ldc = (int64_t)H * D; g2.sC = D; }
+    g2.C = w.U; g2.ldc = (int64_t)H * D; g2.sC = D;
     g2.alpha = 1.4426950408889634f / sqrtf((float)dh); g2.tag = "gemm:stca_U";
     g2.batch = H;
     if ((s = gemm(g2, st)) != SA_OK) return s;
-    // Y = attention over the user's keys
-    if (tc) {
-      if ((s = stca_tc_attention(a, w, st)) != SA_OK) return s;
-    } else {
-      if (a.dtype == SA_BF16)
-        SA_TIMED("stca_attn_simt_kernel", st,
-                 (stca_attn_simt_kernel<__nv_bfloat16><<<w.max_tiles, 256, 0, st>>>(
-                     w.U, (const __nv_bfloat16*)a.kv, a.cand_dev, a.kvb_dev, a.kve_dev,
-                     w.tile_prefix, a.B, H, w.Y)));
-      else
-        SA_TIMED("stca_attn_simt_kernel", st,
-                 (stca_attn_simt_kernel<float><<<w.max_tiles, 256, 0, st>>>(
-                     w.U, (const float*)a.kv, a.cand_dev, a.kvb_dev, a.kve_dev, w.tile_prefix,
-                     a.B, H, w.Y)));
-    }
+    // Y = attention over the user's keys (CUDA cores)
+    if (a.dtype == SA_BF16)
+      SA_TIMED("stca_attn_simt_kernel", st,
+               (stca_attn_simt_kernel<__nv_bfloat16><<<w.max_tiles, 256, 0, st>>>(
+                   w.U, (const __nv_bfloat16*)a.kv, a.cand_dev, a.kvb_dev, a.kve_dev,
+                   w.tile_prefix, a.B, H, w.Y)));
+    else
+      SA_TIMED("stca_attn_simt_kernel", st,
+               (stca_attn_simt_kernel<float><<<w.max_tiles, 256, 0, st>>>(
+                   w.U, (const float*)a.kv, a.cand_dev, a.kvb_dev, a.kve_dev, w.tile_prefix,
+                   a.B, H, w.Y)));
     // O[:, h] = Y[:, h, :] W_V^h
     Gemm g3;
     g3.M = (int)C; g3.N = dh; g3.K = D;

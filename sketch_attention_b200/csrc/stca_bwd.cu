@@ -335,6 +335,43 @@ sa_status ffn_bwd(const float* x, int64_t rows, int D, const Ffn& f, const float
 }
 }  // namespace
 
+FfnBwdScratch ffn_bwd_scratch_carve(Carve& c, int64_t rows, int D) {
+  FfnBwdScratch f;
+  const size_t r = (size_t)std::max<int64_t>(rows, 1);
+  f.G1 = c.take<float>(r * 2 * D);
+  f.G3 = c.take<float>(r * 2 * D);
+  f.U = c.take<float>(r * 2 * D);
+  f.dU = c.take<float>(r * 2 * D);
+  f.split = c.take<float>(kStcaBwdSplitFloats);
+  f.x_hi = c.take<__nv_bfloat16>(r * D);
+  f.x_lo = c.take<__nv_bfloat16>(r * D);
+  f.a_hi = c.take<__nv_bfloat16>(r * 2 * D);
+  f.a_lo = c.take<__nv_bfloat16>(r * 2 * D);
+  f.b_hi = c.take<__nv_bfloat16>(r * 2 * D);
+  f.b_lo = c.take<__nv_bfloat16>(r * 2 * D);
+  f.w_hi = c.take<__nv_bfloat16>((size_t)6 * D * D);
+  f.w_lo = c.take<__nv_bfloat16>((size_t)6 * D * D);
+  return f;
+}
+
+sa_status ffn_residual_backward_tc(const float* x, int64_t rows, int D, const float* W1, const float* W3,
+                                   const float* W2, const float* dy, float* dx, float* dW1, float* dW3, float* dW2,
+                                   const FfnBwdScratch& f, cudaStream_t st) {
+  Ctx cx;
+  cx.st = st;
+  cx.split = f.split;
+  cx.tcp = true;
+  cx.fs = {f.x_hi, f.x_lo, f.a_hi, f.a_lo, f.b_hi, f.b_lo, f.w_hi, f.w_lo};
+  Ffn fn{W1, W3, W2, dW1, dW3, dW2};
+  return ffn_bwd(x, rows, D, fn, dy, dx, f.G1, f.G3, f.U, f.dU, cx);
+}
+
+sa_status split_hi_lo(const float* x, int64_t n, __nv_bfloat16* hi, __nv_bfloat16* lo, cudaStream_t st) {
+  if (n <= 0) return SA_OK;
+  SA_TIMED("split_kernel", st, (split_kernel<<<grid_for(n), 256, 0, st>>>(x, n, hi, lo)));
+  return SA_OK;
+}
+
 size_t stca_bwd_layout(void* base, const StcaBwdShape& sh, StcaBwdWork* w) {
   Carve c(base);
   StcaBwdWork v;

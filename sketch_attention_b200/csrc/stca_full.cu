@@ -113,13 +113,7 @@ size_t stca_full_layout(void* base, int B, int64_t C, int64_t kv_total, int D, i
   StcaFullWork v;
   // the attention part: the same carve as the plain branch
   const size_t rows = (size_t)std::max<int64_t>(C, 1);
-  v.attn.Qh = c.take<float>(rows * heads * d_h);
-  v.attn.U = c.take<float>(rows * heads * D);
-  v.attn.Ub = c.take<__nv_bfloat16>(rows * heads * D);
-  v.attn.Y = c.take<float>(rows * heads * D);
-  v.attn.O = c.take<float>(rows * heads * d_h);
-  v.attn.tile_prefix = c.take<int>((size_t)B + 1);
-  v.attn.max_tiles = 0;
+  v.attn = stca_attn_carve(c, B, C, D, heads, d_h);
   const size_t kt = (size_t)std::max<int64_t>(kv_total, 1);
   v.Hk = c.take<uint8_t>(kt * D * (dtype == SA_BF16 ? 2 : 4));
   v.kpre = c.take<int64_t>((size_t)B + 1);

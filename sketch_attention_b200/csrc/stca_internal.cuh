@@ -27,7 +27,16 @@ struct StcaWork {
   float* O;            // [C, heads*d_h]
   int* tile_prefix;    // [B+1]
   int max_tiles;       // upper bound on the number of query tiles
+  // tensor-core projections (bf16 inputs): the heads' folded weights
+  //   M = [W_Q^h W_K^h^T log2(e)/sqrt(d_h)]_h  [D, heads*D]  and  N = [W_V^h W_O^h]_h  [heads*D, D]
+  // and hi + lo bf16 splits of them, of the query state q [C, D] and of Y [C, heads*D]
+  __nv_bfloat16 *Mhi, *Mlo, *Nhi, *Nlo, *qhi, *qlo, *Yhi, *Ylo;
+  float* part;         // split-K partials of the output projection
+  size_t part_floats;
 };
+
+// Carves the attention part of an STCA workspace (B users, C candidates) from c.
+StcaWork stca_attn_carve(Carve& c, int B, int64_t C, int D, int heads, int d_h);
 
 sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st);
 // The two halves of stca_run: q -> out (fp32) and the query-tile prefix, then
@@ -60,12 +69,29 @@ struct TcGemm {
   const __nv_bfloat16* B_lo = nullptr;
   float* part = nullptr;                   // optional split-K workspace of part_floats floats
   size_t part_floats = 0;
-  float* C = nullptr; int64_t ldc = 0;
+  float* C = nullptr; int64_t ldc = 0;   // fp32 output (may be NULL when C16 is given)
   const float* Cin = nullptr; int64_t ldcin = 0;
   float alpha = 1.f;
+  // optional 16-bit copy of the output: bf16, or (c16_half) fp16 with |v| > 65504 flagged
+  // in the device status word
+  __nv_bfloat16* C16 = nullptr; int64_t ldc16 = 0; bool c16_half = false;
   const char* tag = nullptr;
+  int min_split_slices = 8;   // split K only while every split keeps this many 64-deep K slices
 };
 sa_status tc_gemm(const TcGemm& g, cudaStream_t st);
+// Backward of y = x + (SiLU(x W1) * (x W3)) W2 (inner width 2D) over `rows` fp32 rows on the
+// tensor cores with hi + lo split operands: dx = dy + the FFN's input gradient (dx may alias
+// dy), dW1, dW3 [D, 2D] and dW2 [2D, D] overwritten.
+struct FfnBwdScratch {
+  float *G1, *G3, *U, *dU, *split;
+  __nv_bfloat16 *x_hi, *x_lo, *a_hi, *a_lo, *b_hi, *b_lo, *w_hi, *w_lo;
+};
+FfnBwdScratch ffn_bwd_scratch_carve(Carve& c, int64_t rows, int D);
+sa_status ffn_residual_backward_tc(const float* x, int64_t rows, int D, const float* W1, const float* W3,
+                                   const float* W2, const float* dy, float* dx, float* dW1, float* dW3, float* dW2,
+                                   const FfnBwdScratch& f, cudaStream_t st);
+// x = hi + lo: hi = bf16(x), lo = bf16(x - hi), for n fp32 values
+sa_status split_hi_lo(const float* x, int64_t n, __nv_bfloat16* hi, __nv_bfloat16* lo, cudaStream_t st);
 
 // Backward of a branch of full layers (fp32, GEMM-based).
 struct StcaBwdShape {
@@ -119,6 +145,7 @@ sa_status events_ffn_run(const __nv_bfloat16* item, int64_t vocab, const __nv_bf
                          const float* W2, __nv_bfloat16* X, const EventsFfnWork& w, cudaStream_t st);
 
 bool stca_tc_supported(sa_dtype dtype, int D);
-sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st);
+// Y = attention over each user's keys into w.Y (fp32), or (split_y) into w.Yhi / w.Ylo
+sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st, bool split_y = false);
 
 }  // namespace sa

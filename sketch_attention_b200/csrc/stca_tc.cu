@@ -28,6 +28,12 @@ namespace sa {
 namespace {
 using namespace tc;
 
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 constexpr int TQ = 128, TKB = 128, DD = 128, NSK = 3, THREADS = 256;
 constexpr uint32_t TILE_BYTES = TQ * DD * 2;                       // 32 KB
 constexpr uint32_t OFF_Q = 0, OFF_KV = TILE_BYTES, OFF_BAR = OFF_KV + NSK * TILE_BYTES;
@@ -47,7 +53,9 @@ struct Params {
   const int64_t* kvb;
   const int64_t* kve;
   int B, heads;
-  float* Y;
+  float* Y;              // fp32 output, or (Y NULL) hi + lo bf16 splits of it
+  __nv_bfloat16* Yhi;
+  __nv_bfloat16* Ylo;
   int* err;
 };
 
@@ -77,7 +85,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     // no keys: the attention output is zero
     for (int e = threadIdx.x; e < TQ * DD; e += THREADS) {
       const int64_t row = r0 + e / DD;
-      if (row < rend) p.Y[row * DD + e % DD] = 0.f;
+      if (row < rend) {
+        if (p.Y) {
+          p.Y[row * DD + e % DD] = 0.f;
+        } else {
+          p.Yhi[row * DD + e % DD] = __float2bfloat16_rn(0.f);
+          p.Ylo[row * DD + e % DD] = __float2bfloat16_rn(0.f);
+        }
+      }
     }
     return;
   }
@@ -183,9 +198,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < 128; ++i)
           if (kbase + i >= ke) sv[i] = -__builtin_huge_valf();
       }
-      float bm = sv[0];
+      // block maximum: eight independent chains of three-input maxima
+      float bm;
+      {
+        float c[8];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) bm = fmaxf(bm, sv[i]);
+        for (int q8 = 0; q8 < 8; ++q8) {
+          const float* w = sv + 16 * q8;
+          float m3 = max3f(w[0], w[1], w[2]);
+#pragma unroll
+          for (int j = 3; j + 1 < 16; j += 2) m3 = max3f(m3, w[j], w[j + 1]);
+          c[q8] = fmaxf(m3, w[15]);
+        }
+        bm = fmaxf(max3f(c[0], c[1], c[2]), max3f(c[3], c[4], max3f(c[5], c[6], c[7])));
+      }
       const bool raise = bm > m + kRescale;
       if (__any_sync(0xffffffffu, raise)) {
         const float mn = fmaxf(m, bm);
@@ -212,7 +238,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // P buffer b was last read by PV(j-2)
       if (j >= 2 && !mbar_wait(&bars->pv_done[b], ((j >> 1) - 1) & 1, abort, p.err)) { ok = false; break; }
       uint32_t pw[64];
-      float2 ls2 = make_float2(0.f, 0.f);
+      float2 lsa[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 nm = make_float2(-m, -m);
 #pragma unroll
       for (int i = 0; i < 128; i += 2) {
@@ -226,9 +252,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         } else {
           v = make_float2(ex2(e.x), ex2(e.y));
         }
-        ls2 = __fadd2_rn(ls2, v);
+        lsa[(i / 2) & 3] = __fadd2_rn(lsa[(i / 2) & 3], v);   // four independent sums
         pw[i / 2] = F16 ? pack_f16x2(v.x, v.y) : pack_bf16x2(v.x, v.y);
       }
+      const float2 ls2 = __fadd2_rn(__fadd2_rn(lsa[0], lsa[1]), __fadd2_rn(lsa[2], lsa[3]));
       const float ls = ls2.x + ls2.y;
       l += ls;
       tmem_st32(tmem + lane_addr + (b ? TM_P1 : TM_P0), pw);
@@ -246,11 +273,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         float o[32];
         tmem_ld32(tmem + lane_addr + TM_O + 32 * c, o);
         tmem_wait_ld();
-        if (grow < rend) {
+        if (grow < rend && p.Y) {
           float* dst = p.Y + grow * DD + 32 * c;
 #pragma unroll
           for (int i = 0; i < 32; i += 4)
             *(float4*)(dst + i) = make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+        } else if (grow < rend) {
+          // the output projection's operand: y = hi + lo, hi = bf16(y), lo = bf16(y - hi)
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float y0 = o[i] * inv, y1 = o[i + 1] * inv;
+            hi[i / 2] = pack_bf16x2(y0, y1);
+            lo[i / 2] = pack_bf16x2(y0 - __uint_as_float(hi[i / 2] << 16), y1 - __uint_as_float(hi[i / 2] & 0xFFFF0000u));
+          }
+          uint4* dh = (uint4*)(p.Yhi + grow * DD + 32 * c);
+          uint4* dl = (uint4*)(p.Ylo + grow * DD + 32 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            dh[i] = make_uint4(hi[4 * i], hi[4 * i + 1], hi[4 * i + 2], hi[4 * i + 3]);
+            dl[i] = make_uint4(lo[4 * i], lo[4 * i + 1], lo[4 * i + 2], lo[4 * i + 3]);
+          }
         }
       }
     }
@@ -274,7 +317,7 @@ sa_status make_map(CUtensorMap* map, const void* base, uint64_t rows, bool f16) 
 
 bool stca_tc_supported(sa_dtype dtype, int D) { return dtype == SA_BF16 && D == DD; }
 
-sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
+sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t st, bool split_y) {
   static unsigned long long done = 0, done16 = 0;
   static std::mutex mu;
   set_smem_limit_once((const void*)stca_attn_tc_kernel<false>, SMEM_BYTES, &done, mu);
@@ -290,7 +333,8 @@ sa_status stca_tc_attention(const StcaArgs& a, const StcaWork& w, cudaStream_t s
   } else {
     memset(&tmK, 0, sizeof(tmK));     // never read: every key range is empty
   }
-  Params p{w.tile_prefix, a.cand_dev, a.kvb_dev, a.kve_dev, a.B, a.heads, w.Y, device_status_word()};
+  Params p{w.tile_prefix, a.cand_dev, a.kvb_dev, a.kve_dev, a.B, a.heads, split_y ? nullptr : w.Y,
+           split_y ? w.Yhi : nullptr, split_y ? w.Ylo : nullptr, device_status_word()};
   if (a.kv_f16)
     SA_TIMED("stca_attn_tc_kernel", st,
              (stca_attn_tc_kernel<true><<<w.max_tiles, THREADS, SMEM_BYTES, st>>>(tmU, tmK, p)));

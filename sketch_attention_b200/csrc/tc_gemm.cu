@@ -1,5 +1,6 @@
-// bf16 GEMM on the sm_100a tensor cores for the STCA backward's attention and
-// SwiGLU FFN products: C[M, N] = alpha A B (+ Cin), fp32 accumulation and output.
+// bf16 GEMM on the sm_100a tensor cores for the STCA projections and the STCA
+// backward's attention and SwiGLU FFN products: C[M, N] = alpha A B (+ Cin), fp32
+// accumulation, fp32 and/or 16-bit output.
 // An operand may come as a split pair x = hi + lo (both bf16, lo the rounding of
 // x - hi): the K loop then runs again over hi x lo and lo x hi into the same
 // accumulator (lo x lo, below 2^-16 of the product, is dropped), which carries
@@ -55,7 +56,20 @@ struct Params {
   int kt_per;             // K slices (of TK) per split; the split index is blockIdx.z
   float* part;            // split > 1: raw partial tiles, [split][M][N]
   int* err;
+  __nv_bfloat16* C16;     // optional 16-bit output (bf16, or fp16 when c16_half)
+  int64_t ldc16;
+  int c16_half;
 };
+
+// the 16-bit copy of an output element; an fp16 value beyond its range is flagged
+__device__ __forceinline__ void store_c16(const Params& p, int64_t m, int n, float v) {
+  if (p.c16_half) {
+    if (!(fabsf(v) <= 65504.f)) atomicOr(p.err, DEV_ERR_RANGE);
+    reinterpret_cast<__half*>(p.C16)[m * p.ldc16 + n] = __float2half_rn(v);
+  } else {
+    p.C16[m * p.ldc16 + n] = __float2bfloat16_rn(v);
+  }
+}
 
 // the smem descriptor of K-step ks (16 deep) of a 64-deep operand slice
 __device__ __forceinline__ uint64_t op_desc(uint32_t base, int ks, bool mn) {
@@ -178,7 +192,11 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
           for (int r = 0; r < 32; ++r) {
             const int m = m0 + q * 32 + r;
-            if (m < p.M && n < p.N) p.C[(int64_t)m * p.ldc + n] = p.alpha * blk[r * 33 + lane] + cv[r];
+            if (m < p.M && n < p.N) {
+              const float v = p.alpha * blk[r * 33 + lane] + cv[r];
+              if (p.C) p.C[(int64_t)m * p.ldc + n] = v;
+              if (p.C16) store_c16(p, m, n, v);
+            }
           }
         } else {
 #pragma unroll 4
@@ -189,7 +207,8 @@ __global__ void __launch_bounds__(THREADS, 2)
               if (p.part) {
                 p.part[((int64_t)blockIdx.z * p.M + m) * p.N + n] = x;
               } else {
-                p.C[(int64_t)m * p.ldc + n] = p.alpha * x;
+                if (p.C) p.C[(int64_t)m * p.ldc + n] = p.alpha * x;
+                if (p.C16) store_c16(p, m, n, p.alpha * x);
               }
             }
           }
@@ -211,16 +230,17 @@ __global__ void __launch_bounds__(THREADS, 2)
 }
 
 // C = alpha sum_z part[z] (+ Cin), the slices added in order
-__global__ void tc_gemm_reduce_kernel(const float* __restrict__ part, int splits, int M, int N, float* C,
-                                      int64_t ldc, const float* Cin, int64_t ldcin, float alpha) {
-  const int64_t mn = (int64_t)M * N;
+__global__ void tc_gemm_reduce_kernel(const float* __restrict__ part, int splits, Params p) {
+  const int64_t mn = (int64_t)p.M * p.N;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < mn; e += (int64_t)gridDim.x * blockDim.x) {
     float v = 0.f;
     for (int z = 0; z < splits; ++z) v += part[z * mn + e];
-    const int64_t m = e / N, n = e % N;
-    v *= alpha;
-    if (Cin) v += Cin[m * ldcin + n];
-    C[m * ldc + n] = v;
+    const int64_t m = e / p.N;
+    const int n = (int)(e % p.N);
+    v *= p.alpha;
+    if (p.Cin) v += p.Cin[m * p.ldcin + n];
+    if (p.C) p.C[m * p.ldc + n] = v;
+    if (p.C16) store_c16(p, m, n, v);
   }
 }
 
@@ -277,14 +297,15 @@ sa_status tc_gemm(const TcGemm& g, cudaStream_t st) {
   const int kSMs = device_info().sm_count;
   int split = 1;
   if (g.part && tiles < kSMs) {
-    split = std::min({(kSMs + tiles - 1) / tiles, std::max(1, nk / 8), 64});
+    split = std::min({(kSMs + tiles - 1) / tiles, std::max(1, nk / std::max(1, g.min_split_slices)), 64});
     split = (int)std::min<int64_t>(split, (int64_t)(g.part_floats / ((size_t)g.M * g.N)));
     split = std::max(split, 1);
   }
   const int kt_per = (nk + split - 1) / split;
   split = (nk + kt_per - 1) / kt_per;            // every split gets >= 1 slice
+  if (!g.C && !g.C16) return fail(SA_ERR_INVALID_ARG, "tc_gemm: no output");
   Params p{g.M, g.N, g.K, ph_alo, ph_blo, g.C, g.ldc, g.Cin, g.ldcin, g.alpha, kt_per,
-           split > 1 ? g.part : nullptr, device_status_word()};
+           split > 1 ? g.part : nullptr, device_status_word(), g.C16, g.ldc16, g.c16_half ? 1 : 0};
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, split);
   const char* tag = g.tag ? g.tag : "tc_gemm_kernel";
   const bool cin = split == 1 && g.Cin != nullptr;
@@ -296,9 +317,9 @@ sa_status tc_gemm(const TcGemm& g, cudaStream_t st) {
   if (split > 1) {
     const int64_t mn = (int64_t)g.M * g.N;
     const unsigned blocks = (unsigned)std::min<int64_t>((mn + 255) / 256, 4 * kSMs);
-    SA_TIMED("tc_gemm_reduce_kernel", st,
-             (tc_gemm_reduce_kernel<<<blocks, 256, 0, st>>>(g.part, split, g.M, g.N, g.C, g.ldc, g.Cin, g.ldcin,
-                                                            g.alpha)));
+    Params pr = p;
+    pr.part = nullptr;
+    SA_TIMED("tc_gemm_reduce_kernel", st, (tc_gemm_reduce_kernel<<<blocks, 256, 0, st>>>(g.part, split, pr)));
   }
   return SA_OK;
 }
