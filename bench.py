@@ -893,6 +893,29 @@ def run_component(args, rank, world, device):
                 f"{p.B} users x mean {p.n_total // max(p.B, 1)} events, k={p.k}, d={p.d}, bf16")
         # per launch of the dominant kernel: H = A X with its mass (2kd flop per token)
         kname, flops = "sa_agg_tc_kernel", 2.0 * p.k * p.d * p.n_total
+    elif args.workload == "refine_bwd":
+        from sa_inputs import refine_layers, rng_for
+        p = sa_workload(5, users=args.users)
+        X = _dev_bf16(p.X, device)
+        offd = torch.from_numpy(p.offsets).to(device)
+        P0 = _f32(p.P, device)
+        n_iter = 2
+        layers = [{k: (_f32(v, device) if v is not None else None) for k, v in L.items()}
+                  for L in refine_layers(rng_for(5005), n_iter, p.d)]
+        gen = torch.Generator(device="cpu").manual_seed(5009)
+        dsk = torch.randn(p.B, p.k, p.d, generator=gen).to(device)
+        ws = torch.empty(sab.sa_refine_backward_workspace(p.B, p.n_total, p.k, p.d, n_iter, sab.SA_BF16),
+                         dtype=torch.uint8, device=device)
+        rb_out = {"dX": torch.empty(p.n_total, p.d, device=device), "dP0": torch.empty(p.k, p.d, device=device)}
+        step = lambda: sab.sa_refine_backward(X, p.offsets, P0, layers, dsk, 1e-5, offsets_dev=offd,
+                                              out=rb_out, workspace=ws)
+        units, unit = p.n_total, "history-tokens/s"
+        name = (f"backward of the stacked SA refinement (forward recomputed), {n_iter} iterations, "
+                f"{p.B} users x mean {p.n_total // max(p.B, 1)} events, k={p.k}, d={p.d}, bf16")
+        # the dX kernel's credited 8kd flop per token and iteration, spread over its per-user launches
+        kname, refine_dx_flops_step = "sa_bwd_dx_tc_kernel", 8.0 * p.k * p.d * p.n_total * n_iter
+        extra_step = [("sa_bwd_e_tc_kernel", 2.0 * p.k * p.d * p.n_total * n_iter),
+                      ("sa_agg_tc_kernel", 2.0 * p.k * p.d * p.n_total * n_iter)]
     elif args.workload == "stca_full":
         from sa_inputs import add_stca_ffns, rng_for
         w = stca_workload(users=args.users or 16)
@@ -1016,6 +1039,11 @@ def run_component(args, rank, world, device):
     prof = sab.profile_read()
     sab.profile(False)
     ms = start.elapsed_time(end) / args.steps
+    if args.workload == "refine_bwd":
+        # per-user launches: flops per launch = the step's credited total over its launches
+        per_launch = lambda kn, fl: fl / max(prof.get(kn, (0, 1))[1] / args.steps, 1)
+        flops = per_launch(kname, refine_dx_flops_step)
+        extra.extend((kn, per_launch(kn, fl)) for kn, fl in extra_step)
     if args.workload == "stca_bwd":
         # flops per launch of the dominant (tensor-core GEMM) call site: the step's total over its launches
         flops = attn_flops_step / max(prof.get(kname, (0, 1))[1] / args.steps, 1)
@@ -1082,7 +1110,7 @@ def main():
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-configuration records (SA forward at 32 x 100K, 8 users and the "
                          "small fp32 case; STCA at 16 users x 512 candidates)")
-    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "stca_full", "stca_bwd", "refine",
+    ap.add_argument("--workload", choices=["train", "sa_fwd", "stca", "stca_full", "stca_bwd", "refine", "refine_bwd",
                                            "tokenwise"],
                     default="train",
                     help="train: the full step (default, the headline); sa_fwd: SA forward over "
