@@ -28,14 +28,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
   asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
+// One bounded probe of the phase.  try_wait without a suspend-time hint (the
+// hardware's own limit): measured faster than a 1 ms hint in the SA forward
+// kernels (lse 0.489 -> 0.462 ms, aggregation 0.712 -> 0.660 ms on 16 users of
+// 100K events) and neutral elsewhere.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar_addr), "r"(parity), "r"(1000000u)
+      : "r"(bar_addr), "r"(parity)
       : "memory");
   return ok != 0;
 }
