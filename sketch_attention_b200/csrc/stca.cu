@@ -18,12 +18,6 @@ namespace sa {
 namespace {
 constexpr float kInf = __builtin_huge_valf();
 
-template <class T>
-__global__ void to_f32_kernel(const T* __restrict__ in, int64_t n, float* __restrict__ out) {
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
-       e += (int64_t)gridDim.x * blockDim.x)
-    out[e] = load_as_f32(in, e);
-}
 
 __global__ void add_kernel(float* __restrict__ y, const float* __restrict__ x, int64_t n) {
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
@@ -31,17 +25,39 @@ __global__ void add_kernel(float* __restrict__ y, const float* __restrict__ x, i
     y[e] += x[e];
 }
 
-// prefix[u] = number of query tiles of users < u; a user has
-// ceil(C_u * heads / tq) tiles.
-__global__ void tile_prefix_kernel(const int64_t* __restrict__ cand, int B, int heads, int tq,
-                                   int* __restrict__ prefix) {
-  if (blockIdx.x != 0 || threadIdx.x != 0) return;
-  int acc = 0;
-  prefix[0] = 0;
-  for (int u = 0; u < B; ++u) {
-    const int64_t rows = (cand[u + 1] - cand[u]) * heads;
-    acc += (int)((rows + tq - 1) / tq);
-    prefix[u + 1] = acc;
+// The start of an STCA call: q -> out (fp32) and, when qhi is given, q's hi + lo
+// bf16 split; block 0 also writes prefix[u] = the number of query tiles of users < u (a
+// user has ceil(C_u * heads / tq) tiles): per-user counts in parallel, then a scan over
+// shared memory, 256 users at a time.
+template <class T>
+__global__ void __launch_bounds__(256) stca_begin_kernel(const T* __restrict__ q, int64_t n, float* __restrict__ out,
+                                                         __nv_bfloat16* __restrict__ qhi, __nv_bfloat16* __restrict__ qlo,
+                                                         const int64_t* __restrict__ cand, int B, int heads, int tq,
+                                                         int* __restrict__ prefix) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const float v = load_as_f32(q, e);
+    out[e] = v;
+    if (qhi) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      qhi[e] = hi;
+      qlo[e] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    }
+  }
+  if (blockIdx.x != 0 || !prefix) return;
+  __shared__ int cnt[256];
+  int base = 0;
+  if (threadIdx.x == 0) prefix[0] = 0;
+  for (int u0 = 0; u0 < B; u0 += 256) {
+    const int u = u0 + threadIdx.x;
+    cnt[threadIdx.x] = u < B ? (int)(((cand[u + 1] - cand[u]) * heads + tq - 1) / tq) : 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int i = 0; i < 256 && u0 + i < B; ++i) {
+        base += cnt[i];
+        prefix[u0 + i + 1] = base;
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -224,18 +240,19 @@ StcaWork stca_attn_carve(Carve& c, int B, int64_t C, int D, int heads, int d_h) 
 sa_status stca_begin(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
   const int64_t C = a.C_total;
   const int64_t nq = C * a.D;
-  if (nq > 0) {
-    if (a.dtype == SA_BF16)
-      SA_TIMED("to_f32_kernel", st,
-               (to_f32_kernel<<<grid_for(nq), 256, 0, st>>>((const __nv_bfloat16*)a.q, nq, a.out)));
-    else
-      SA_TIMED("to_f32_kernel", st,
-               (to_f32_kernel<<<grid_for(nq), 256, 0, st>>>((const float*)a.q, nq, a.out)));
-  }
-  if (C == 0) return SA_OK;
-  const int tq = stca_tc_supported(a.dtype, a.D) ? 128 : 32;
-  SA_TIMED("tile_prefix_kernel", st,
-           (tile_prefix_kernel<<<1, 1, 0, st>>>(a.cand_dev, a.B, a.heads, tq, w.tile_prefix)));
+  if (nq == 0) return SA_OK;
+  const bool tc = stca_tc_supported(a.dtype, a.D);
+  const int tq = tc ? 128 : 32;
+  __nv_bfloat16* qhi = tc ? w.qhi : nullptr;
+  __nv_bfloat16* qlo = tc ? w.qlo : nullptr;
+  if (a.dtype == SA_BF16)
+    SA_TIMED("stca_begin_kernel", st,
+             (stca_begin_kernel<<<grid_for(nq), 256, 0, st>>>((const __nv_bfloat16*)a.q, nq, a.out, qhi, qlo,
+                                                              a.cand_dev, a.B, a.heads, tq, w.tile_prefix)));
+  else
+    SA_TIMED("stca_begin_kernel", st,
+             (stca_begin_kernel<<<grid_for(nq), 256, 0, st>>>((const float*)a.q, nq, a.out, qhi, qlo, a.cand_dev,
+                                                              a.B, a.heads, tq, w.tile_prefix)));
   return SA_OK;
 }
 
@@ -258,7 +275,8 @@ sa_status tc_projections_prepare(const StcaArgs& a, const stca_layer& L, const S
   return SA_OK;
 }
 
-sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWork& w, cudaStream_t st) {
+sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWork& w, cudaStream_t st,
+                            bool q_split, bool split_out) {
   const int D = a.D, H = a.heads, dh = a.d_h, HD = a.heads * a.d_h;
   const int64_t C = a.C_total;
   const int64_t nq = C * D;
@@ -267,7 +285,7 @@ sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWo
   sa_status s;
   if (tc) {
     if ((s = tc_projections_prepare(a, L, w, st)) != SA_OK) return s;
-    if ((s = split_hi_lo(a.out, nq, w.qhi, w.qlo, st)) != SA_OK) return s;
+    if (!q_split && (s = split_hi_lo(a.out, nq, w.qhi, w.qlo, st)) != SA_OK) return s;
     TcGemm gu;                                // U = q M -> the attention's 16-bit queries
     gu.M = (int)C; gu.N = H * D; gu.K = D;
     gu.A = w.qhi; gu.A_lo = w.qlo; gu.lda = D;
@@ -281,6 +299,7 @@ sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWo
     go.A = w.Yhi; go.A_lo = w.Ylo; go.lda = (int64_t)H * D;
     go.B = w.Nhi; go.B_lo = w.Nlo; go.ldb = D; go.b_mn = true;
     go.C = a.out; go.ldc = D; go.Cin = a.out; go.ldcin = D;
+    if (split_out) { go.Chi = w.qhi; go.Clo = w.qlo; go.ldcs = D; }   // the next layer's q split
     go.tag = "tc_gemm:stca_O";
     return tc_gemm(go, st);
   }
@@ -339,7 +358,9 @@ sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWo
 
 sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st) {
   sa_status s = stca_begin(a, w, st);
-  for (int l = 0; s == SA_OK && l < a.n_layers; ++l) s = stca_attend_layer(a, a.layers[l], w, st);
+  // stca_begin split q; each output projection splits the q it writes for the next layer
+  for (int l = 0; s == SA_OK && l < a.n_layers; ++l)
+    s = stca_attend_layer(a, a.layers[l], w, st, true, l + 1 < a.n_layers);
   return s;
 }
 

@@ -162,6 +162,7 @@ sa_status stca_full_run(const StcaArgs& a0, const stca_full_layer* layers, int64
       a.kv_f16 = true;
     }
   }
+  bool split_ready = true;
   for (int l = 0; l < a.n_layers; ++l) {
     const stca_full_layer& L = layers[l];
     if (has_hist(L)) {
@@ -180,7 +181,11 @@ sa_status stca_full_run(const StcaArgs& a0, const stca_full_layer* layers, int64
       a.kvb_dev = w.kpre;
       a.kve_dev = w.kpre + 1;
     }
-    if ((s = stca_attend_layer(a, L.attn, w.attn, st)) != SA_OK) return s;
+    // q's split is ready from stca_begin for the first layer, and from the previous
+    // layer's output projection when that layer has no query FFN (which changes q)
+    const bool split_out = !has_query(L) && l + 1 < a.n_layers;
+    if ((s = stca_attend_layer(a, L.attn, w.attn, st, split_ready, split_out)) != SA_OK) return s;
+    split_ready = split_out;
     // eq. (26): q <- q + FFN_q(q)
     if (has_query(L) &&
         (s = ffn_residual_gemm(a.out, a.C_total, a.D, L.q_W1, L.q_W3, L.q_W2, w.G1, w.G3, w.U,

@@ -41,8 +41,12 @@ StcaWork stca_attn_carve(Carve& c, int B, int64_t C, int D, int heads, int d_h);
 sa_status stca_run(const StcaArgs& a, const StcaWork& w, cudaStream_t st);
 // The two halves of stca_run: q -> out (fp32) and the query-tile prefix, then
 // one attention layer (projections, attention over a.kv, W_O, residual).
+// With bf16 inputs stca_begin also writes q's hi + lo split (w.qhi, w.qlo); a layer reads
+// that split when q_split is true (else it splits q itself) and, with split_out, has its
+// output projection write the split of the new q for the next layer.
 sa_status stca_begin(const StcaArgs& a, const StcaWork& w, cudaStream_t st);
-sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWork& w, cudaStream_t st);
+sa_status stca_attend_layer(const StcaArgs& a, const stca_layer& L, const StcaWork& w, cudaStream_t st,
+                            bool q_split = false, bool split_out = false);
 
 // Full STCA layers (history- and query-side SwiGLU FFNs).
 struct StcaFullWork {
@@ -75,6 +79,8 @@ struct TcGemm {
   // optional 16-bit copy of the output: bf16, or (c16_half) fp16 with |v| > 65504 flagged
   // in the device status word
   __nv_bfloat16* C16 = nullptr; int64_t ldc16 = 0; bool c16_half = false;
+  // optional hi + lo bf16 split of the output (the operand of a following split GEMM)
+  __nv_bfloat16* Chi = nullptr; __nv_bfloat16* Clo = nullptr; int64_t ldcs = 0;
   const char* tag = nullptr;
   int min_split_slices = 8;   // split K only while every split keeps this many 64-deep K slices
 };

@@ -59,9 +59,17 @@ struct Params {
   __nv_bfloat16* C16;     // optional 16-bit output (bf16, or fp16 when c16_half)
   int64_t ldc16;
   int c16_half;
+  __nv_bfloat16* Chi;     // optional hi + lo bf16 split of the output: hi = bf16(c), lo = bf16(c - hi)
+  __nv_bfloat16* Clo;
+  int64_t ldcs;
 };
 
 // the 16-bit copy of an output element; an fp16 value beyond its range is flagged
+__device__ __forceinline__ void store_split(const Params& p, int64_t m, int n, float v) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+  p.Chi[m * p.ldcs + n] = hi;
+  p.Clo[m * p.ldcs + n] = __float2bfloat16_rn(v - __bfloat162float(hi));
+}
 __device__ __forceinline__ void store_c16(const Params& p, int64_t m, int n, float v) {
   if (p.c16_half) {
     if (!(fabsf(v) <= 65504.f)) atomicOr(p.err, DEV_ERR_RANGE);
@@ -196,6 +204,7 @@ __global__ void __launch_bounds__(THREADS, 2)
               const float v = p.alpha * blk[r * 33 + lane] + cv[r];
               if (p.C) p.C[(int64_t)m * p.ldc + n] = v;
               if (p.C16) store_c16(p, m, n, v);
+              if (p.Chi) store_split(p, m, n, v);
             }
           }
         } else {
@@ -209,6 +218,7 @@ __global__ void __launch_bounds__(THREADS, 2)
               } else {
                 if (p.C) p.C[(int64_t)m * p.ldc + n] = p.alpha * x;
                 if (p.C16) store_c16(p, m, n, p.alpha * x);
+                if (p.Chi) store_split(p, m, n, p.alpha * x);
               }
             }
           }
@@ -241,6 +251,7 @@ __global__ void tc_gemm_reduce_kernel(const float* __restrict__ part, int splits
     if (p.Cin) v += p.Cin[m * p.ldcin + n];
     if (p.C) p.C[m * p.ldc + n] = v;
     if (p.C16) store_c16(p, m, n, v);
+    if (p.Chi) store_split(p, m, n, v);
   }
 }
 
@@ -305,7 +316,8 @@ sa_status tc_gemm(const TcGemm& g, cudaStream_t st) {
   split = (nk + kt_per - 1) / kt_per;            // every split gets >= 1 slice
   if (!g.C && !g.C16) return fail(SA_ERR_INVALID_ARG, "tc_gemm: no output");
   Params p{g.M, g.N, g.K, ph_alo, ph_blo, g.C, g.ldc, g.Cin, g.ldcin, g.alpha, kt_per,
-           split > 1 ? g.part : nullptr, device_status_word(), g.C16, g.ldc16, g.c16_half ? 1 : 0};
+           split > 1 ? g.part : nullptr, device_status_word(), g.C16, g.ldc16, g.c16_half ? 1 : 0,
+           g.Chi, g.Clo, g.ldcs};
   dim3 grid((g.N + TN - 1) / TN, (g.M + TM - 1) / TM, split);
   const char* tag = g.tag ? g.tag : "tc_gemm_kernel";
   const bool cin = split == 1 && g.Cin != nullptr;
