@@ -99,6 +99,7 @@ struct DxParams {
   int* err;
   float* dX32;           // optional [n, d] fp32 output instead of dX, added to when acc32
   int acc32;
+  int p_user_rows;       // rows of P' per user (k: per-user prototypes), 0: one shared P'
 };
 
 // 384: caps registers at 168, as three warps share two of the SM's sub-partitions
@@ -173,7 +174,8 @@ __global__ void __launch_bounds__(384, 1)
         if (cc >= DX_NCS && !mbar_wait(&bars->avq_done[cs], ((cc / DX_NCS) - 1) & 1, abort, p.err)) return false;
         mbar_arrive_expect_tx(&bars->c_full[cs], CH_BYTES + KC * 4);
         uint8_t* cd = smem + DX_OFF_CH + cs * CH_BYTES;
-        const int prow = c * KC, hrow = (int)((int64_t)u * p.k + c * KC);
+        const int hrow = (int)((int64_t)u * p.k + c * KC);
+        const int prow = (int)((int64_t)u * p.p_user_rows + c * KC);
         tma_load_2d(cd, &tmP, &bars->c_full[cs], 0, prow);
         tma_load_2d(cd + 8192, &tmH, &bars->c_full[cs], 0, hrow);
         tma_load_2d(cd + 16384, &tmP, &bars->c_full[cs], 64, prow);
@@ -392,7 +394,7 @@ constexpr uint32_t E_TM_ZG = 0, E_TM_E = 256;
 
 struct EBars {
   uint64_t p_full, h_full, h_empty, x_full[E_NXS], x_empty[E_NXS];
-  uint64_t zg_full, zg_empty, dz_full[E_NDZ], dz_empty[E_NDZ], e_full, mma_done;
+  uint64_t zg_full, zg_empty, dz_full[E_NDZ], dz_empty[E_NDZ], e_full, e_empty, mma_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -407,8 +409,16 @@ struct EParams {
   const float* dmc;      // [B, k]
   float* Epart;          // [G, k, d]
   int* err;
+  // per-user prototypes: P' slice reloaded with each user's dH slice, and E written at
+  // the end of every user's piece (to the user's rows, or a slot of the chunk when the
+  // user spans chunks) instead of once per chunk
+  int per_user;
+  float* Euser;          // [B, k, d]
+  float* slotE;          // [G, 2, k, d]
 };
 
+// PU: per-user prototypes and per-user E (EParams::per_user)
+template <bool PU>
 __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 warps per sub-partition)
     sa_bwd_e_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                        const __grid_constant__ CUtensorMap tmH, EParams p) {
@@ -430,6 +440,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     mbar_init(&bars->zg_empty, 256);
     for (int b = 0; b < E_NDZ; ++b) { mbar_init(&bars->dz_full[b], 256); mbar_init(&bars->dz_empty[b], 1); }
     mbar_init(&bars->e_full, 1);
+    mbar_init(&bars->e_empty, 256);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -447,15 +458,22 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     prefetch_tensormap(&tmX);
     prefetch_tensormap(&tmP);
     prefetch_tensormap(&tmH);
-    mbar_arrive_expect_tx(&bars->p_full, 32768);
-    tma_load_2d(smem + E_OFF_PH, &tmP, &bars->p_full, 0, sl * TILE);
-    tma_load_2d(smem + E_OFF_PH + 32768, &tmP, &bars->p_full, 64, sl * TILE);
+    if (!PU) {
+      mbar_arrive_expect_tx(&bars->p_full, 32768);
+      tma_load_2d(smem + E_OFF_PH, &tmP, &bars->p_full, 0, sl * TILE);
+      tma_load_2d(smem + E_OFF_PH + 32768, &tmP, &bars->p_full, 64, sl * TILE);
+    }
     int issued_t = 0, issued_h = 0;
     for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int u, int64_t tb, int64_t, bool first, bool) {
       if (first) {
         if (piece > 0 && !mbar_wait(&bars->h_empty, (piece - 1) & 1, abort, p.err)) return false;
-        mbar_arrive_expect_tx(&bars->h_full, 32768 + TILE * 4);
+        mbar_arrive_expect_tx(&bars->h_full, (PU ? 65536 : 32768) + TILE * 4);
         const int hrow = (int)((int64_t)u * p.k + sl * TILE);
+        if (PU) {
+          // this user's P' slice (the first two 16 KB blocks of the pair layout)
+          tma_load_2d(smem + E_OFF_PH, &tmP, &bars->h_full, 0, hrow);
+          tma_load_2d(smem + E_OFF_PH + 32768, &tmP, &bars->h_full, 64, hrow);
+        }
         tma_load_2d(smem + E_OFF_PH + 16384, &tmH, &bars->h_full, 0, hrow);
         tma_load_2d(smem + E_OFF_PH + 49152, &tmH, &bars->h_full, 64, hrow);
         bulk_load(smem + E_OFF_DM, p.dmc + (int64_t)u * p.k + sl * TILE, TILE * 4, &bars->h_full);
@@ -471,7 +489,7 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
       return true;
     });
     if (*abort) {
-      mbar_wait_bounded(&bars->p_full, 0);
+      if (!PU) mbar_wait_bounded(&bars->p_full, 0);
       if (issued_h > 0) mbar_wait_bounded(&bars->h_full, (issued_h - 1) & 1);
       for (int t = std::max(0, issued_t - E_NXS); t < issued_t; ++t)
         mbar_wait_bounded(&bars->x_full[t % E_NXS], (t / E_NXS) & 1);
@@ -480,22 +498,28 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     const uint32_t id_zg = idesc_bf16(128, 256, false, false);
     const uint32_t id_e = idesc_bf16(128, 128, true, true);
     const uint32_t ph = smem_u32(smem + E_OFF_PH);
-    int prev_t = -1, prev_s = 0;
-    auto emma = [&](int t, int s) -> bool {
+    int prev_t = -1, prev_s = 0, prev_piece = 0;
+    bool prev_first = false, prev_last = false;
+    auto emma = [&](int t, int s, int piece, bool first, bool last) -> bool {
       const int b = t % E_NDZ;
+      // per user: E starts afresh at each piece, once the previous piece's E is drained
+      if (PU && first && piece > 0 && !mbar_wait(&bars->e_empty, (piece - 1) & 1, abort, p.err))
+        return false;
       if (!mbar_wait(&bars->dz_full[b], (t / E_NDZ) & 1, abort, p.err)) return false;
       tc_fence_after();
       const uint32_t dz = smem_u32(smem + E_OFF_DZ + b * 32768);
       const uint32_t xa = smem_u32(smem + E_OFF_X + s * XT_BYTES);
+      const bool fresh = PU ? first : t == 0;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
         mma_ss(tmem + E_TM_E, smem_desc(dz + ks * 2048, 16384, 1024, SWZ_128B),
-               smem_desc(xa + ks * 2048, 16384, 1024, SWZ_128B), id_e, (t > 0 || ks > 0) ? 1u : 0u);
+               smem_desc(xa + ks * 2048, 16384, 1024, SWZ_128B), id_e, (!fresh || ks > 0) ? 1u : 0u);
       mma_commit(&bars->dz_empty[b]);
       mma_commit(&bars->x_empty[s]);
+      if (PU && last) mma_commit(&bars->e_full);
       return true;
     };
-    bool ok = mbar_wait(&bars->p_full, 0, abort, p.err);
+    bool ok = PU || mbar_wait(&bars->p_full, 0, abort, p.err);
     if (ok) {
       for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t, int64_t, bool first, bool last) {
         const int s = t % E_NXS;
@@ -511,12 +535,16 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
                  ks > 0 ? 1u : 0u);
         mma_commit(&bars->zg_full);
         if (last) mma_commit(&bars->h_empty);
-        if (prev_t >= 0 && !emma(prev_t, prev_s)) return false;
+        if (prev_t >= 0 && !emma(prev_t, prev_s, prev_piece, prev_first, prev_last)) return false;
         prev_t = t;
         prev_s = s;
+        prev_piece = piece;
+        prev_first = first;
+        prev_last = last;
         return true;
       });
-      if (prev_t >= 0 && !*abort && emma(prev_t, prev_s)) mma_commit(&bars->e_full);
+      if (prev_t >= 0 && !*abort && emma(prev_t, prev_s, prev_piece, prev_first, prev_last) && !PU)
+        mma_commit(&bars->e_full);
     }
     mma_commit(&bars->mma_done);
     mbar_wait_bounded(&bars->mma_done, 0);
@@ -527,7 +555,21 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     bool ok = true;
     const int64_t n_total = p.off[p.B];
     float l2_next = 0.f, ct_next = 0.f;   // this row's lse and c for the next tile, loaded a tile ahead
-    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int, int64_t tb, int64_t pe, bool first, bool last) {
+    const int64_t cb = (int64_t)g * p.ch.T, ce = min(cb + p.ch.T, p.ch.n_total);
+    // this thread's 64 columns of the prototype's row of E, into dst
+    auto write_e = [&](float* dst) {
+      tc_fence_after();
+#pragma unroll
+      for (int c = 2 * h; c < 2 * h + 2; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_addr + E_TM_E + 32 * c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *(float4*)(dst + 32 * c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+      }
+    };
+    for_each_tile(p.off, p.B, p.ch, g, [&](int t, int piece, int u, int64_t tb, int64_t pe, bool first, bool last) {
       const bool valid = tb + row < pe;
       float l2r = l2_next, ctr = ct_next;
       if (t == 0 && valid) { l2r = p.lse2[tb + row]; ctr = p.cin[tb + row]; }
@@ -578,21 +620,21 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
       fence_proxy_async_smem();
       mbar_arrive(&bars->dz_full[b]);
       if (last) mbar_arrive(&bars->h_empty);   // this piece's dm is no longer read
+      if (PU && last) {
+        // the user's E over this piece: to the user's rows, or to a slot of the chunk when
+        // the user spans chunks (added up by e_user_reduce_kernel); then E may start afresh
+        if (!mbar_wait(&bars->e_full, piece & 1, abort, p.err)) return ok = false;
+        const int dest = piece_dest(p.off[u], p.off[u + 1], cb, ce);
+        const int j = sl * TILE + row;
+        write_e(dest == DEST_USER ? p.Euser + ((int64_t)u * p.k + j) * DD
+                                  : p.slotE + (((int64_t)g * 2 + dest) * p.k + j) * DD);
+        tc_fence_before();
+        mbar_arrive(&bars->e_empty);
+      }
       return true;
     });
-    if (ok && mbar_wait(&bars->e_full, 0, abort, p.err)) {
-      tc_fence_after();
-      float* dst = p.Epart + ((int64_t)g * p.k + sl * TILE + row) * DD;
-#pragma unroll
-      for (int c = 2 * h; c < 2 * h + 2; ++c) {
-        float v[32];
-        tmem_ld32(tmem + lane_addr + E_TM_E + 32 * c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *(float4*)(dst + 32 * c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-      }
-    }
+    if (ok && !PU && mbar_wait(&bars->e_full, 0, abort, p.err))
+      write_e(p.Epart + ((int64_t)g * p.k + sl * TILE + row) * DD);
   }
 
   tc_fence_before();
@@ -607,6 +649,29 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
 
 sa_status map_rows(CUtensorMap* map, const void* base, uint64_t rows, uint32_t box_rows) {
   return tma_map_bf16(map, base, DD, rows, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Per-user E of users that span E chunks: E_u = its first chunk's slot 1 + the middle
+// chunks' slot 0 + its last chunk's slot 0, added in that order; users inside one chunk
+// were written by the E kernel, users without tokens get zeros.
+__global__ void e_user_reduce_kernel(const int64_t* __restrict__ off, Chunking ch, int k,
+                                     const float* __restrict__ slotE, float* __restrict__ Euser) {
+  const int u = blockIdx.y;
+  const int64_t ub = off[u], ue = off[u + 1];
+  const int64_t kd = (int64_t)k * DD;
+  float* dst = Euser + (int64_t)u * kd;
+  if (ue <= ub) {
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < kd; e += (int64_t)gridDim.x * blockDim.x)
+      dst[e] = 0.f;
+    return;
+  }
+  const int64_t gf = ub / ch.T, gl = (ue - 1) / ch.T;
+  if (gf == gl) return;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < kd; e += (int64_t)gridDim.x * blockDim.x) {
+    float v = slotE[((int64_t)gf * 2 + 1) * kd + e];
+    for (int64_t g = gf + 1; g <= gl; ++g) v += slotE[((int64_t)g * 2 + 0) * kd + e];
+    dst[e] = v;
+  }
 }
 
 // dmc[u, j] = dm[u, j] - mean_j dm[u, :]
@@ -634,29 +699,41 @@ int sa_bwd_tc_dx_chunks() { return device_info().sm_count; }
 int sa_bwd_tc_e_chunks(int k) { return std::max(1, device_info().sm_count / (k / TILE)); }
 
 sa_status sa_bwd_tc_run(const SaBwdArgs& a, const SaBwdWork& w, cudaStream_t st) {
-  static unsigned long long done_dx = 0, done_e = 0;
+  static unsigned long long done_dx = 0, done_e = 0, done_e_pu = 0;
   static std::mutex mu;
   set_smem_limit_once((const void*)sa_bwd_dx_tc_kernel, DX_SMEM, &done_dx, mu);
-  set_smem_limit_once((const void*)sa_bwd_e_tc_kernel, E_SMEM, &done_e, mu);
+  set_smem_limit_once((const void*)sa_bwd_e_tc_kernel<false>, E_SMEM, &done_e, mu);
+  set_smem_limit_once((const void*)sa_bwd_e_tc_kernel<true>, E_SMEM, &done_e_pu, mu);
   if (a.n_total >= (1LL << 31) || (int64_t)a.B * a.k >= (1LL << 31))
     return fail(SA_ERR_UNSUPPORTED, "row counts must be < 2^31");
   SA_TIMED("center_rows_kernel", st, (center_rows_kernel<<<a.B, 256, 0, st>>>(w.dm, a.k, w.dmc)));
   CUtensorMap tmX, tmP64, tmH64, tmP128, tmH128;
   sa_status s;
+  // per-user prototypes: P' has B k rows, user u's at u k
+  const uint64_t p_rows = a.per_user ? (uint64_t)a.B * a.k : (uint64_t)a.k;
+  if (a.per_user && (!w.Euser || !w.slotE)) return fail(SA_ERR_INVALID_ARG, "per-user backward: no E outputs");
   if ((s = map_rows(&tmX, a.X, (uint64_t)a.n_total, 128)) != SA_OK) return s;
-  if ((s = map_rows(&tmP64, w.Pb, (uint64_t)a.k, 64)) != SA_OK) return s;
+  if ((s = map_rows(&tmP64, w.Pb, p_rows, 64)) != SA_OK) return s;
   if ((s = map_rows(&tmH64, w.dHb, (uint64_t)a.B * a.k, 64)) != SA_OK) return s;
   CUtensorMap tmL64;
   if ((s = map_rows(&tmL64, w.dHlo, (uint64_t)a.B * a.k, 64)) != SA_OK) return s;
-  if ((s = map_rows(&tmP128, w.Pb, (uint64_t)a.k, 128)) != SA_OK) return s;
+  if ((s = map_rows(&tmP128, w.Pb, p_rows, 128)) != SA_OK) return s;
   if ((s = map_rows(&tmH128, w.dHb, (uint64_t)a.B * a.k, 128)) != SA_OK) return s;
   DxParams dp{a.off_dev, a.B, w.ch, a.k, w.lse, w.dmc, (__nv_bfloat16*)a.dX, w.cbuf, device_status_word(),
-              a.dX32, a.dX_acc ? 1 : 0};
+              a.dX32, a.dX_acc ? 1 : 0, a.per_user ? a.k : 0};
   SA_TIMED("sa_bwd_dx_tc_kernel", st,
            (sa_bwd_dx_tc_kernel<<<w.ch.G, DX_THREADS, DX_SMEM, st>>>(tmX, tmP64, tmH64, tmL64, dp)));
-  EParams ep{a.off_dev, a.B, w.chE, a.k, w.lse, w.cbuf, w.dmc, w.Epart, device_status_word()};
-  SA_TIMED("sa_bwd_e_tc_kernel", st,
-           (sa_bwd_e_tc_kernel<<<w.chE.G * (a.k / TILE), E_THREADS, E_SMEM, st>>>(tmX, tmP128, tmH128, ep)));
+  EParams ep{a.off_dev, a.B, w.chE, a.k, w.lse, w.cbuf, w.dmc, w.Epart, device_status_word(),
+             a.per_user ? 1 : 0, w.Euser, w.slotE};
+  if (a.per_user)
+    SA_TIMED("sa_bwd_e_tc_kernel", st,
+             (sa_bwd_e_tc_kernel<true><<<w.chE.G * (a.k / TILE), E_THREADS, E_SMEM, st>>>(tmX, tmP128, tmH128, ep)));
+  else
+    SA_TIMED("sa_bwd_e_tc_kernel", st,
+             (sa_bwd_e_tc_kernel<false><<<w.chE.G * (a.k / TILE), E_THREADS, E_SMEM, st>>>(tmX, tmP128, tmH128, ep)));
+  if (a.per_user)
+    SA_TIMED("e_user_reduce_kernel", st,
+             (e_user_reduce_kernel<<<dim3(64, a.B), 256, 0, st>>>(a.off_dev, w.chE, a.k, w.slotE, w.Euser)));
   return SA_OK;
 }
 

@@ -39,6 +39,10 @@ struct SaBwdArgs {
   bool accumulate = false;   // add the weight gradients into dP, dW_Q, dW_K, dW_V
   float* dX32 = nullptr;     // tensor-core path: dX as fp32 [n, d] instead of dX (added to when dX_acc)
   bool dX_acc = false;
+  // tensor-core path with per-user prototypes (the refinement's later iterations): user u's
+  // folded prototypes are rows u k.. of w.Pb, and E is kept per user (w.Euser) instead of
+  // summed over the batch
+  bool per_user = false;
 };
 
 struct SaBwdWork {
@@ -57,6 +61,8 @@ struct SaBwdWork {
   float* dm;            // [B, k]
   float* dmc;           // [B, k]     dm centred per user (tensor-core path)
   float* Epart;         // [chE.G, k, d]
+  float* Euser;         // per_user: [B, k, d] each user's E
+  float* slotE;         // per_user: [chE.G, 2, k, d] pieces of users that span E chunks
   float* E;             // [k, d]
   float* dQ;            // [k, d]
   float* Q;             // [k, d]

@@ -16,8 +16,9 @@
 //   dX_u += A^T dX^ + ln2 dZ^T P'_u (the tensor-core dX kernel, P'_u the user's folded prototypes),
 //   E_u = sum_t dZ_t^T x_t (the tensor-core E kernel),
 //   dQ_u = E_u W_K / sqrt(d),  dW_Q += X~_u^T dQ_u,  dW_K += E_u^T (X~_u W_Q) / sqrt(d).
-// The SA kernels take one set of prototypes per launch, so they run user by
-// user; dX accumulates over the iterations in fp32.  After the first iteration
+// The SA backward kernels run once per iteration for the whole batch with
+// per-user prototypes (user u's folded P' rows) and keep E per user; dX
+// accumulates over the iterations in fp32.  After the first iteration
 // dP0 = sum_u dX~_u.
 #include <algorithm>
 #include <vector>
@@ -47,11 +48,10 @@ struct RB {
   float *Euser, *dQ, *Qall;                // [B, k, d]
   __nv_bfloat16 *dHb, *dHlo;               // [B k, d]
   float *cbuf;                             // [n]
-  float *dmz, *dmc;                        // [k] zeros, centred (zeros)
-  float* Epart;                            // [G_E, k, d]
+  float *dmz, *dmc;                        // [B, k] zeros (no mass term), centred (zeros)
+  float* slotE;                            // [G_E, 2, k, d] E of users spanning E chunks
   float* lnpart;                           // [LN blocks, 2, d]
   float* gsplit;                           // split-K partials of the weight-gradient GEMMs
-  int64_t* ou;                             // [2 B] per-user device offsets {0, n_u}
   FfnBwdScratch fb;
 };
 
@@ -91,12 +91,11 @@ size_t layout(void* base, int B, int64_t n, int k, int d, int n_iter, RB* out) {
   v.dHb = c.take<__nv_bfloat16>(bkd);
   v.dHlo = c.take<__nv_bfloat16>(bkd);
   v.cbuf = c.take<float>(nn);
-  v.dmz = c.take<float>((size_t)k);
-  v.dmc = c.take<float>((size_t)k);
-  v.Epart = c.take<float>((size_t)std::max(sa_bwd_tc_e_chunks(k), 1) * k * d);
+  v.dmz = c.take<float>(rows);
+  v.dmc = c.take<float>(rows);
+  v.slotE = c.take<float>((size_t)std::max(sa_bwd_tc_e_chunks(k), 1) * 2 * k * d);
   v.lnpart = c.take<float>((rows + LN_ROWS - 1) / LN_ROWS * 2 * d);
   v.gsplit = c.take<float>((size_t)kMaxSplit * d * d);
-  v.ou = c.take<int64_t>((size_t)2 * B);
   v.fb = ffn_bwd_scratch_carve(c, (int64_t)rows, d);
   if (out) *out = v;
   return c.bytes();
@@ -283,14 +282,7 @@ sa_status sa_refine_backward_run(const void* X, const int64_t* off_host, const i
   }
 
   // ---------------------------------------------------------------- backward
-  {
-    std::vector<int64_t> ou(2 * (size_t)B);
-    for (int u = 0; u < B; ++u) { ou[2 * u] = 0; ou[2 * u + 1] = off_host[u + 1] - off_host[u]; }
-    SA_CUDA(cudaMemcpyAsync(v.ou, ou.data(), sizeof(int64_t) * 2 * B, cudaMemcpyHostToDevice, st));
-    // the copy reads `ou` before this function returns and frees it
-    SA_CUDA(cudaStreamSynchronize(st));
-  }
-  SA_CUDA(cudaMemsetAsync(v.dmz, 0, sizeof(float) * k, st));
+  SA_CUDA(cudaMemsetAsync(v.dmz, 0, sizeof(float) * rows, st));
   SA_CUDA(cudaMemcpyAsync(v.dXt, dsketch, sizeof(float) * bkd, cudaMemcpyDeviceToDevice, st));
   for (int it = n_iter - 1; it >= 0; --it) {
     const sa_refine_layer& L = layers[it];
@@ -306,39 +298,37 @@ sa_status sa_refine_backward_run(const void* X, const int64_t* off_host, const i
     if ((s = ln_backward(v.Xin[it], v.H[it], L.ln1_g, v.dXbar, ln_eps, rows, d, v.dY1, L.ln1_g ? G.dln1_g : nullptr,
                          L.ln1_b ? G.dln1_b : nullptr, v.lnpart, st)) != SA_OK)
       return s;
-    // eq. (14): X^ = A X_u, user by user with the user's own prototypes
+    // eq. (14): X^ = A X_u with each user's own prototypes (one launch of each SA
+    // backward kernel for the batch; E kept per user)
     SA_TIMED("split_bf16_kernel", st, (split_bf16_kernel<<<grid_for(bkd), 256, 0, st>>>(v.dY1, bkd, v.dHb, v.dHlo)));
-    for (int u = 0; u < B; ++u) {
-      const int64_t nu = off_host[u + 1] - off_host[u];
-      float* Eu = v.Euser + (int64_t)u * kd;
-      if (nu == 0) {
-        SA_CUDA(cudaMemsetAsync(Eu, 0, sizeof(float) * kd, st));
-        continue;
-      }
+    if (n == 0) {
+      SA_CUDA(cudaMemsetAsync(v.Euser, 0, sizeof(float) * bkd, st));
+    } else {
       SaBwdArgs ab{};
-      ab.X = (const __nv_bfloat16*)X + off_host[u] * d;
+      ab.X = X;
       ab.x_dtype = SA_BF16;
-      ab.off_dev = v.ou + 2 * u;
-      ab.B = 1;
-      ab.n_total = nu;
+      ab.off_dev = off_dev;
+      ab.B = B;
+      ab.n_total = n;
       ab.k = k;
       ab.d = d;
       ab.dX = nullptr;
-      ab.dX32 = dX + off_host[u] * d;
+      ab.dX32 = dX;
       ab.dX_acc = it < n_iter - 1;
+      ab.per_user = true;
       SaBwdWork wb{};
-      wb.ch = make_chunking(nu, sa_bwd_tc_dx_chunks(), 1);
-      wb.chE = make_chunking(nu, sa_bwd_tc_e_chunks(k), 1);
-      wb.Pb = v.Pb[it] + (int64_t)u * kd;
-      wb.lse = v.lse[it] + off_host[u];
-      wb.cbuf = v.cbuf + off_host[u];
-      wb.dHb = v.dHb + (int64_t)u * kd;
-      wb.dHlo = v.dHlo + (int64_t)u * kd;
+      wb.ch = make_chunking(n, sa_bwd_tc_dx_chunks(), 1);
+      wb.chE = make_chunking(n, sa_bwd_tc_e_chunks(k), 1);
+      wb.Pb = v.Pb[it];
+      wb.lse = v.lse[it];
+      wb.cbuf = v.cbuf;
+      wb.dHb = v.dHb;
+      wb.dHlo = v.dHlo;
       wb.dm = v.dmz;
       wb.dmc = v.dmc;
-      wb.Epart = v.Epart;
+      wb.Euser = v.Euser;
+      wb.slotE = v.slotE;
       if ((s = sa_bwd_tc_run(ab, wb, st)) != SA_OK) return s;
-      if ((s = sa_sum_slices(v.Epart, wb.chE.G, kd, Eu, st)) != SA_OK) return s;
     }
     // dQ = E W_K / sqrt(d);  dX~ = dY1 + dQ W_Q^T
     Gemm gq = plain((int)rows, d, d, v.Euser, d, false, L.W_K, d, false, v.dQ, d, "gemm:refine_grads");
