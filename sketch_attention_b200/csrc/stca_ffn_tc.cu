@@ -322,27 +322,39 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lane_addr = (uint32_t)(q4 * 32) << 16;
     // tile j's row: 16 pieces of 16 bytes (8 bf16), piece 8a + c at atom a, chunk c ^ (row % 8)
     float vmax = 0.f;                   // largest |x + F| (or, for events, |e|) seen by this thread
-    // EV: the item row of tile j's row (zeros past the end or for an id outside the table)
-    auto event_row = [&](int j, uint4* v) {
-      const int64_t grow = (int64_t)(blockIdx.x + j * (int)gridDim.x) * TM + row;
-      bool ok = grow < p.rows;
-      int64_t id = 0;
-      if (ok) {
+    // EV: each row's table index runs ahead of the tiles: the raw id and type of tile
+    // i + 2 are loaded while tile i is finished, validated (-1: past the end, an id
+    // outside the table or a bad type) and the item row prefetched to L2 one tile later,
+    // then gathered into TMEM when tile i + 1 is staged; the write-back gathers it again
+    // (from L2) to add F.
+    auto ev_raw = [&](int j, int32_t& id, int& act) {
+      const int64_t grow = (int64_t)(blockIdx.x + (int64_t)j * gridDim.x) * TM + row;
+      id = -1;
+      act = 0;
+      if (grow < p.rows) {
         id = p.ids[grow];
-        ok = id >= 0 && id < p.vocab && (int)p.acts[grow] < p.n_actions;
+        act = p.acts[grow];
       }
-      const uint4* src = (const uint4*)(p.item + id * DD);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) v[c] = ok ? src[c] : make_uint4(0, 0, 0, 0);
-      return ok;
     };
-    auto stage_x = [&](int j) -> bool {
+    auto ev_valid = [&](int32_t id, int act) -> int64_t {
+      return (id >= 0 && (int64_t)id < p.vocab && act < p.n_actions) ? (int64_t)id : -1;
+    };
+    auto ev_prefetch = [&](int64_t id) {
+      if (id >= 0) {
+        const char* a = (const char*)(p.item + id * DD);
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a + 128));
+      }
+    };
+    auto stage_x = [&](int j, int64_t id) -> bool {
       const int s = j & 1;
       uint32_t v[64];
       if (EV) {
         if (j >= 1 && !mbar_wait(&bars->xt_empty, (j - 1) & 1, abort, p.err)) return false;
         uint4 e[16];
-        event_row(j, e);
+        const uint4* src = (const uint4*)(p.item + (id >= 0 ? id : 0) * DD);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) e[c] = id >= 0 ? src[c] : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           const uint32_t w[4] = {e[c].x, e[c].y, e[c].z, e[c].w};
@@ -376,22 +388,44 @@ __global__ void __launch_bounds__(THREADS, 1)
       return true;
     };
     int i = 0;
-    bool ok = blockIdx.x < p.ntiles && stage_x(0);
+    int64_t id0 = -1, id1 = -1;            // tiles i and i + 1 (validated)
+    int32_t raw2 = -1;                     // tile i + 2 (loaded, not yet validated)
+    int act2 = 0;
+    if (EV) {
+      int32_t r;
+      int a;
+      ev_raw(0, r, a);
+      id0 = ev_valid(r, a);
+      ev_raw(1, r, a);
+      id1 = ev_valid(r, a);
+      ev_prefetch(id1);
+      ev_raw(2, raw2, act2);
+    }
+    bool ok = blockIdx.x < p.ntiles && stage_x(0, id0);
     for (int t = blockIdx.x; ok && t < p.ntiles; t += gridDim.x, ++i) {
+      int64_t id2 = -1;
+      if (EV) {
+        id2 = ev_valid(raw2, act2);
+        ev_prefetch(id2);
+        ev_raw(i + 3, raw2, act2);
+      }
       // the next tile's X goes in as soon as this tile's first-layer MMAs are done
-      if (t + (int)gridDim.x < p.ntiles && !stage_x(i + 1)) break;
+      if (t + (int)gridDim.x < p.ntiles && !stage_x(i + 1, id1)) break;
       const int64_t grow = (int64_t)t * TM + row;
       const bool valid = grow < p.rows;
-      uint32_t xr[64];                  // the row as fp16 pairs (events: as bf16 pairs)
-      bool ev_ok = true;
+      uint32_t xr[64];                  // the row as fp16 pairs (events: the bf16 item row)
+      const bool ev_ok = !EV || id0 >= 0;
       if (EV) {
-        uint4 e[16];
-        ev_ok = event_row(i, e);        // the item row again (in L2 since it was staged)
         if (valid && !ev_ok && p.err) atomicOr(p.err, DEV_ERR_INDEX);
+        // the item row again (in L2: it was staged a tile ago)
+        const uint4* px = (const uint4*)(p.item + (ev_ok ? id0 : 0) * DD);
 #pragma unroll
         for (int v = 0; v < 16; ++v) {
-          xr[4 * v] = e[v].x; xr[4 * v + 1] = e[v].y; xr[4 * v + 2] = e[v].z; xr[4 * v + 3] = e[v].w;
+          const uint4 x = (valid && ev_ok) ? px[v] : make_uint4(0, 0, 0, 0);
+          xr[4 * v] = x.x; xr[4 * v + 1] = x.y; xr[4 * v + 2] = x.z; xr[4 * v + 3] = x.w;
         }
+        id0 = id1;
+        id1 = id2;
       } else {
         const uint4* px = (const uint4*)(p.X + (valid ? grow : 0) * DD);
 #pragma unroll
