@@ -184,6 +184,12 @@ size_t layout_fwd(void* base, int B, int64_t n, int k, int d, sa_dtype dt, SaFwd
   v.slotH = c.take<float>((size_t)std::max(ch.G, 1) * 2 * k * d);
   v.slotM = c.take<float>((size_t)std::max(ch.G, 1) * 2 * k);
   v.Hhat = c.take<float>((size_t)B * k * d);
+  if (dt == SA_BF16 && d == 128) {
+    v.Hhi = c.take<__nv_bfloat16>((size_t)B * k * d);
+    v.Hlo = c.take<__nv_bfloat16>((size_t)B * k * d);
+    v.Vhi = c.take<__nv_bfloat16>((size_t)d * d);
+    v.Vlo = c.take<__nv_bfloat16>((size_t)d * d);
+  }
   if (w) *w = v;
   return c.bytes();
 }
@@ -218,6 +224,14 @@ size_t layout_bwd(void* base, int B, int64_t n, int k, int d, sa_dtype dt, SaBwd
   v.dQ = c.take<float>((size_t)k * d);
   v.Q = c.take<float>((size_t)k * d);
   v.gsplit = c.take<float>((size_t)kMaxSplit * d * d);
+  if (tc) {
+    v.dShi = c.take<__nv_bfloat16>((size_t)B * k * d);
+    v.dSlo = c.take<__nv_bfloat16>((size_t)B * k * d);
+    v.Hhi = c.take<__nv_bfloat16>((size_t)B * k * d);
+    v.Hlo = c.take<__nv_bfloat16>((size_t)B * k * d);
+    v.Vhi = c.take<__nv_bfloat16>((size_t)d * d);
+    v.Vlo = c.take<__nv_bfloat16>((size_t)d * d);
+  }
   if (w) *w = v;
   return c.bytes();
 }

@@ -26,6 +26,12 @@ struct SaFwdWork {
   float* slotH;         // [G, 2, k, d]
   float* slotM;         // [G, 2, k]
   float* Hhat;          // [B, k, d] H/(m+eps)
+  // the output projection on the tensor cores (bf16 inputs, d = 128; NULL: the fp32 GEMM):
+  // hi + lo bf16 splits of Hhat [B, k, d] and of W_V [d, d]
+  __nv_bfloat16* Hhi = nullptr;
+  __nv_bfloat16* Hlo = nullptr;
+  __nv_bfloat16* Vhi = nullptr;
+  __nv_bfloat16* Vlo = nullptr;
 };
 
 struct SaBwdArgs {
@@ -61,6 +67,14 @@ struct SaBwdWork {
   float* dm;            // [B, k]
   float* dmc;           // [B, k]     dm centred per user (tensor-core path)
   float* Epart;         // [chE.G, k, d]
+  // the projection GEMMs on the tensor cores (bf16 inputs, d = 128; NULL: fp32 GEMMs): hi + lo
+  // bf16 splits of dS and Hhat [B, k, d] and of W_V [d, d]
+  __nv_bfloat16* dShi = nullptr;
+  __nv_bfloat16* dSlo = nullptr;
+  __nv_bfloat16* Hhi = nullptr;
+  __nv_bfloat16* Hlo = nullptr;
+  __nv_bfloat16* Vhi = nullptr;
+  __nv_bfloat16* Vlo = nullptr;
   float* Euser;         // per_user: [B, k, d] each user's E
   float* slotE;         // per_user: [chE.G, 2, k, d] pieces of users that span E chunks
   float* E;             // [k, d]

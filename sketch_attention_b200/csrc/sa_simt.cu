@@ -12,6 +12,7 @@
 #include <algorithm>
 
 #include "sa_internal.cuh"
+#include "stca_internal.cuh"
 
 namespace sa {
 
@@ -153,7 +154,8 @@ __global__ void __launch_bounds__(256) sa_reduce_kernel(
     const int64_t* __restrict__ off, int B, Chunking ch, int k, int D, float eps,
     const float* __restrict__ Huser, const float* __restrict__ Muser,
     const float* __restrict__ slotH, const float* __restrict__ slotM,
-    float* __restrict__ Hout, float* __restrict__ mass_out, float* __restrict__ Hhat) {
+    float* __restrict__ Hout, float* __restrict__ mass_out, float* __restrict__ Hhat,
+    __nv_bfloat16* __restrict__ Hhi, __nv_bfloat16* __restrict__ Hlo) {
   constexpr int RB = 8;
   __shared__ float inv[RB];
   const int u = blockIdx.y;
@@ -193,7 +195,14 @@ __global__ void __launch_bounds__(256) sa_reduce_kernel(
     }
     const int64_t o = ((int64_t)u * k + j) * D + c;
     if (Hout) Hout[o] = h;
-    Hhat[o] = h * inv[jj];
+    const float hh = h * inv[jj];
+    Hhat[o] = hh;
+    if (Hhi) {
+      // the output projection's split operand: hh = hi + lo
+      const __nv_bfloat16 hi = __float2bfloat16_rn(hh);
+      Hhi[o] = hi;
+      Hlo[o] = __float2bfloat16_rn(hh - __bfloat162float(hi));
+    }
   }
 }
 
@@ -203,7 +212,7 @@ __global__ void __launch_bounds__(256) sa_bwd_prologue_kernel(
     int rows, int D, float eps, const float* __restrict__ H, const float* __restrict__ mass,
     const float* __restrict__ dHh, const float* __restrict__ dmass, float* __restrict__ Hhat,
     float* __restrict__ dH, __nv_bfloat16* __restrict__ dHb, __nv_bfloat16* __restrict__ dHlo,
-    float* __restrict__ dm) {
+    float* __restrict__ dm, __nv_bfloat16* __restrict__ Hhi, __nv_bfloat16* __restrict__ Hlo) {
   const int warp = (blockIdx.x * 256 + threadIdx.x) / 32, lane = threadIdx.x % 32;
   if (warp >= rows) return;
   const float den = mass[warp] + eps;
@@ -213,6 +222,11 @@ __global__ void __launch_bounds__(256) sa_bwd_prologue_kernel(
     const int64_t o = (int64_t)warp * D + c;
     const float hh = H[o] * inv;
     Hhat[o] = hh;
+    if (Hhi) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(hh);
+      Hhi[o] = hi;
+      Hlo[o] = __float2bfloat16_rn(hh - __bfloat162float(hi));
+    }
     dH[o] = dHh[o] * inv;
     if (dHb) {
       const float v = dHh[o] * inv;
@@ -515,13 +529,27 @@ sa_status sa_reduce(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st) {
   SA_TIMED("sa_reduce_kernel", st,
            (sa_reduce_kernel<<<grid, 256, 0, st>>>(a.off_dev, a.B, w.ch, a.k, a.d, a.eps, a.S,
                                                    w.Muser, w.slotH, w.slotM, a.H, a.mass,
-                                                   w.Hhat)));
+                                                   w.Hhat, w.Vhi ? w.Hhi : nullptr,
+                                                   w.Vhi ? w.Hlo : nullptr)));
   return SA_OK;
 }
 
 sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStream_t st) {
   sa_status s = sa_reduce(a, w, st);
   if (s != SA_OK) return s;
+  if (w.Hhi && w.Vhi) {
+    // S = Hh W_V on the tensor cores over hi + lo splits of both (three passes, about 16
+    // significant bits), with its bf16 copy
+    if ((s = split_hi_lo(a.W_V, (int64_t)a.d * a.d, w.Vhi, w.Vlo, st)) != SA_OK) return s;
+    TcGemm t;
+    t.M = a.B * a.k; t.N = a.d; t.K = a.d;
+    t.A = w.Hhi; t.A_lo = w.Hlo; t.lda = a.d;
+    t.B = w.Vhi; t.B_lo = w.Vlo; t.ldb = a.d; t.b_mn = true;
+    t.C = a.S; t.ldc = a.d;
+    t.C16 = (__nv_bfloat16*)a.S_bf16; t.ldc16 = a.d;
+    t.tag = "tc_gemm:S_proj";
+    return tc_gemm(t, st);
+  }
   // S = Hh W_V (and its bf16 copy)
   Gemm g;
   g.M = a.B * a.k; g.N = a.d; g.K = a.d;
@@ -535,28 +563,55 @@ sa_status sa_reduce_and_project(const SaFwdArgs& a, const SaFwdWork& w, cudaStre
 sa_status sa_backward_run(const SaBwdArgs& a, const SaBwdWork& w, bool tc, cudaStream_t st) {
   const int rows = a.B * a.k;
   const int D = a.d;
+  // the two W_V products on the tensor cores over hi + lo splits (three passes, about 16
+  // significant bits) when the workspace has the split buffers, else fp32 GEMMs
+  const bool tcp = tc && w.dShi && w.Hhi && w.Vhi;
+  sa_status s;
   // dHh = dS W_V^T
-  Gemm g;
-  g.M = rows; g.N = D; g.K = D;
-  g.A = a.dS; g.lda = D;
-  g.B = a.W_V; g.ldb = D; g.transB = true;
-  g.C = w.dHh; g.ldc = D; g.tag = "gemm:dHh";
-  sa_status s = gemm(g, st);
-  if (s != SA_OK) return s;
+  if (tcp) {
+    if ((s = split_hi_lo(a.dS, (int64_t)rows * D, w.dShi, w.dSlo, st)) != SA_OK) return s;
+    if ((s = split_hi_lo(a.W_V, (int64_t)D * D, w.Vhi, w.Vlo, st)) != SA_OK) return s;
+    TcGemm t;
+    t.M = rows; t.N = D; t.K = D;
+    t.A = w.dShi; t.A_lo = w.dSlo; t.lda = D;
+    t.B = w.Vhi; t.B_lo = w.Vlo; t.ldb = D;      // B[n][k] = W_V[n][k]: K-major
+    t.C = w.dHh; t.ldc = D; t.tag = "tc_gemm:dHh";
+    if ((s = tc_gemm(t, st)) != SA_OK) return s;
+  } else {
+    Gemm g;
+    g.M = rows; g.N = D; g.K = D;
+    g.A = a.dS; g.lda = D;
+    g.B = a.W_V; g.ldb = D; g.transB = true;
+    g.C = w.dHh; g.ldc = D; g.tag = "gemm:dHh";
+    if ((s = gemm(g, st)) != SA_OK) return s;
+  }
   SA_TIMED("sa_bwd_prologue_kernel", st,
            (sa_bwd_prologue_kernel<<<(rows * 32 + 255) / 256, 256, 0, st>>>(
                rows, D, a.eps, a.H, a.mass, w.dHh, a.dmass, w.Hhat, w.dH, tc ? w.dHb : nullptr,
-               tc ? w.dHlo : nullptr, w.dm)));
+               tc ? w.dHlo : nullptr, w.dm, tcp ? w.Hhi : nullptr, tcp ? w.Hlo : nullptr)));
   // dW_V = sum_u Hh_u^T dS_u
-  Gemm gv;
-  gv.M = D; gv.N = D; gv.K = rows;
-  gv.A = w.Hhat; gv.lda = D; gv.transA = true;
-  gv.B = a.dS; gv.ldb = D;
-  gv.C = a.dW_V; gv.ldc = D;
-  if (a.accumulate) { gv.Cin = a.dW_V; gv.ldcin = D; } gv.tag = "gemm:dW_V";
-  gv.split_k = gemm_split_for(D, D, rows, kMaxSplit);
-  gv.split_ws = w.gsplit;
-  if ((s = gemm(gv, st)) != SA_OK) return s;
+  if (tcp) {
+    TcGemm t;
+    t.M = D; t.N = D; t.K = rows;
+    t.A = w.Hhi; t.A_lo = w.Hlo; t.lda = D; t.a_mn = true;      // A[k][m] = Hhat[k][m]
+    t.B = w.dShi; t.B_lo = w.dSlo; t.ldb = D; t.b_mn = true;    // B[k][n] = dS[k][n]
+    t.C = a.dW_V; t.ldc = D;
+    if (a.accumulate) { t.Cin = a.dW_V; t.ldcin = D; }
+    t.part = w.gsplit; t.part_floats = (size_t)kMaxSplit * D * D;
+    t.tag = "tc_gemm:dW_V";
+    if ((s = tc_gemm(t, st)) != SA_OK) return s;
+  } else {
+    Gemm gv;
+    gv.M = D; gv.N = D; gv.K = rows;
+    gv.A = w.Hhat; gv.lda = D; gv.transA = true;
+    gv.B = a.dS; gv.ldb = D;
+    gv.C = a.dW_V; gv.ldc = D;
+    if (a.accumulate) { gv.Cin = a.dW_V; gv.ldcin = D; }
+    gv.tag = "gemm:dW_V";
+    gv.split_k = gemm_split_for(D, D, rows, kMaxSplit);
+    gv.split_ws = w.gsplit;
+    if ((s = gemm(gv, st)) != SA_OK) return s;
+  }
   if (a.n_total > 0) {
     const bool bf = a.x_dtype == SA_BF16;
     if (D == 64) s = bf ? backward_lse<__nv_bfloat16, 64>(a, w, st) : backward_lse<float, 64>(a, w, st);

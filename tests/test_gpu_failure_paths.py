@@ -6,7 +6,8 @@ import pytest
 import torch
 
 from helpers import dev_f32, dev_x
-from sa_inputs import add_stca_ffns, make_sa_problem, make_stca_problem, refine_layers, rng_for
+from sa_inputs import (add_stca_ffns, event_ffn_weights, event_problem, make_sa_problem, make_stca_problem,
+                       refine_layers, rng_for)
 
 pytestmark = pytest.mark.gpu
 
@@ -120,3 +121,47 @@ def test_refine_and_tokenwise_stay_inside_their_workspaces(lib):
     torch.cuda.synchronize()
     lib.poll_device_status()
     assert _intact(big, ws_b)
+
+
+def test_refine_backward_stays_inside_its_buffers(lib):
+    """The batched refinement backward (per-user prototypes in both SA backward kernels, E
+    drained per user piece into user rows or chunk slots) writes only its workspace and its
+    outputs."""
+    p = make_sa_problem((900, 0, 300, 2500), 256, 128, "bf16", seed=807, x_kind="events")
+    X = dev_x(p.X, p.dtype)
+    layers = [{k: (dev_f32(v) if v is not None else None) for k, v in L.items()}
+              for L in refine_layers(rng_for(808), 2, 128)]
+    ws_b = lib.sa_refine_backward_workspace(p.B, p.n_total, p.k, p.d, 2, lib.SA_BF16)
+    big, ws = _padded(ws_b)
+    outs = {"dX": _padded_like((p.n_total, p.d), torch.float32), "dP0": _padded_like((p.k, p.d), torch.float32)}
+    dsk = dev_f32(np.random.default_rng(9).standard_normal((p.B, p.k, p.d)).astype(np.float32))
+    lib.sa_refine_backward(X, p.offsets, dev_f32(p.P), layers, dsk, out={k: v[1] for k, v in outs.items()},
+                           workspace=ws)
+    torch.cuda.synchronize()
+    lib.poll_device_status()
+    assert _intact(big, ws_b)
+    for k, (b, t) in outs.items():
+        assert _intact(b, t.numel() * t.element_size()), k
+
+
+def test_event_rows_stay_inside_their_buffers(lib):
+    """Both event-row entry points (the plain sum and eq. (20)'s fused FFN) write only their
+    output rows and, for the fused form, its workspace; a ragged last tile (n not a multiple
+    of 128) included."""
+    item, action, ids, acts = event_problem(1000, 4096, 128, seed=809)
+    t = lambda b: torch.from_numpy(b.view(np.int16)).cuda().view(torch.bfloat16)
+    dev = (t(item), t(action), torch.from_numpy(ids).cuda(), torch.from_numpy(acts).cuda())
+    xbig, X = _padded_like((len(ids), 128), torch.bfloat16)
+    lib.sa_gather_events(*dev, out=X)
+    torch.cuda.synchronize()
+    lib.poll_device_status()
+    assert _intact(xbig, X.numel() * 2)
+    W1, W3, W2 = (dev_f32(w) for w in event_ffn_weights(rng_for(810), 128))
+    ws_b = lib.sa_gather_events_fused_workspace(action.shape[0], 128, 256)
+    wbig, ws = _padded(ws_b)
+    xbig, X = _padded_like((len(ids), 128), torch.bfloat16)
+    lib.sa_gather_events_fused(*dev, W1, W3, W2, out=X, workspace=ws)
+    torch.cuda.synchronize()
+    lib.poll_device_status()
+    assert _intact(wbig, ws_b)
+    assert _intact(xbig, X.numel() * 2)
