@@ -16,7 +16,7 @@ Readings where the pages leave a step open (each is an explicit choice):
   H = A X (the pages' X-tilde) is returned as well.  A prototype whose
   m_j + eps is zero (eps = 0 and no mass) gets S_j = 0.
 * Softmax stabiliser: the per-token maximum over prototypes is subtracted
-  ("numerically robust softmax", Sec. 4.4 FlashSA); the result is unchanged.
+  (Sec. 4.4 asks FlashSA for a numerically stable softmax); the result is unchanged.
 * STCA layer body: attention, optional output projection W_O, residual add
   to the query (eq. 4 plus the W_O term of eq. 26), no LayerNorm.  The full
   layer of eqs. (26)-(28) adds two optional SwiGLU FFNs of inner width 2D
