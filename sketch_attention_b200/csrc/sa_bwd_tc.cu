@@ -386,10 +386,16 @@ constexpr uint32_t E_OFF_DZ = E_OFF_X + E_NXS * XT_BYTES;   // E_NDZ x [128 prot
 constexpr uint32_t E_OFF_DM = E_OFF_DZ + E_NDZ * 32768;
 constexpr uint32_t E_OFF_BAR = E_OFF_DM + TILE * 4;
 constexpr uint32_t E_SMEM = E_OFF_BAR + 256 + 1024;
-// warp 0 TMA, 1 MMA, 2-5 and 6-9: two warpgroups, group h computing dZ for the
-// prototypes 64h..64h+63 of the slice (so each reads its half of [Z|G] at once
-// and the next tile's logits MMA overlaps all of the dZ work)
-constexpr int E_THREADS = 320;
+// warp 0 TMA, 1 MMA, then E_NWG warpgroups, group h computing dZ for the
+// prototypes E_PW h .. E_PW h + E_PW-1 of the slice (so each reads its share of [Z|G]
+// at once and the next tile's logits MMA overlaps all of the dZ work)
+#ifndef SA_E_NWG
+#define SA_E_NWG 2
+#endif
+constexpr int E_NWG = SA_E_NWG, E_PW = TILE / E_NWG;
+static_assert(E_NWG == 2 || E_NWG == 4, "two or four dZ warpgroups");
+constexpr int E_THREADS = 64 + 128 * E_NWG;
+constexpr int E_BOUND = E_NWG == 2 ? 384 : E_THREADS;   // 384 with two: caps registers at 168
 constexpr uint32_t E_TM_ZG = 0, E_TM_E = 256;
 
 struct EBars {
@@ -419,7 +425,7 @@ struct EParams {
 
 // PU: per-user prototypes and per-user E (EParams::per_user)
 template <bool PU>
-__global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 warps per sub-partition)
+__global__ void __launch_bounds__(E_BOUND, 1)
     sa_bwd_e_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmP,
                        const __grid_constant__ CUtensorMap tmH, EParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -434,13 +440,14 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
   if (threadIdx.x == 0) {
     mbar_init(&bars->p_full, 1);
     mbar_init(&bars->h_full, 1);
-    mbar_init(&bars->h_empty, 1 + 256);      // the last zg of a piece, and the threads done with its dm
+    constexpr int NT = 128 * E_NWG;          // dZ threads
+    mbar_init(&bars->h_empty, 1 + NT);       // the last zg of a piece, and the threads done with its dm
     for (int s = 0; s < E_NXS; ++s) { mbar_init(&bars->x_full[s], 1); mbar_init(&bars->x_empty[s], 1); }
     mbar_init(&bars->zg_full, 1);
-    mbar_init(&bars->zg_empty, 256);
-    for (int b = 0; b < E_NDZ; ++b) { mbar_init(&bars->dz_full[b], 256); mbar_init(&bars->dz_empty[b], 1); }
+    mbar_init(&bars->zg_empty, NT);
+    for (int b = 0; b < E_NDZ; ++b) { mbar_init(&bars->dz_full[b], NT); mbar_init(&bars->dz_empty[b], 1); }
     mbar_init(&bars->e_full, 1);
-    mbar_init(&bars->e_empty, 256);
+    mbar_init(&bars->e_empty, NT);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -556,11 +563,11 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
     const int64_t n_total = p.off[p.B];
     float l2_next = 0.f, ct_next = 0.f;   // this row's lse and c for the next tile, loaded a tile ahead
     const int64_t cb = (int64_t)g * p.ch.T, ce = min(cb + p.ch.T, p.ch.n_total);
-    // this thread's 64 columns of the prototype's row of E, into dst
+    // this thread's E_PW columns of the prototype's row of E, into dst
     auto write_e = [&](float* dst) {
       tc_fence_after();
 #pragma unroll
-      for (int c = 2 * h; c < 2 * h + 2; ++c) {
+      for (int c = E_PW / 32 * h; c < E_PW / 32 * (h + 1); ++c) {
         float v[32];
         tmem_ld32(tmem + lane_addr + E_TM_E + 32 * c, v);
         tmem_wait_ld();
@@ -588,19 +595,21 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
       const uint32_t dz = smem_u32(smem + E_OFF_DZ + b * 32768) + row * 128;
       const float4* dm4 = (const float4*)(smem + E_OFF_DM);
       {
-        float z[64], gv[64];
-        tmem_ld32(tmem + lane_addr + E_TM_ZG + 64 * h, z);
-        tmem_ld32(tmem + lane_addr + E_TM_ZG + 64 * h + 32, z + 32);
-        tmem_ld32(tmem + lane_addr + E_TM_ZG + 128 + 64 * h, gv);
-        tmem_ld32(tmem + lane_addr + E_TM_ZG + 128 + 64 * h + 32, gv + 32);
+        float z[E_PW], gv[E_PW];
+#pragma unroll
+        for (int c = 0; c < E_PW / 32; ++c) {
+          tmem_ld32(tmem + lane_addr + E_TM_ZG + E_PW * h + 32 * c, z + 32 * c);
+          tmem_ld32(tmem + lane_addr + E_TM_ZG + 128 + E_PW * h + 32 * c, gv + 32 * c);
+        }
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->zg_empty);
         if (t >= E_NDZ && !mbar_wait(&bars->dz_empty[b], ((t / E_NDZ) - 1) & 1, abort, p.err)) return ok = false;
         // two prototypes per instruction (packed fp32x2 add / mul)
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const float4 d0 = dm4[16 * h + 2 * c8], d1 = dm4[16 * h + 2 * c8 + 1];
+        for (int c8 = 0; c8 < E_PW / 8; ++c8) {
+          const int p0 = E_PW * h + 8 * c8;   // the first of these eight prototypes in the slice
+          const float4 d0 = dm4[p0 / 4], d1 = dm4[p0 / 4 + 1];
           const float2 dmp[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
                                  make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
           uint32_t o[4];
@@ -613,8 +622,8 @@ __global__ void __launch_bounds__(384, 1)   // 384: caps registers at 168 (3 war
             const float2 dzv = __fmul2_rn(A, __fadd2_rn(dA, nct));
             o[i] = pack_bf16x2(dzv.x, dzv.y);
           }
-          // MN-major SW128 A operand of E += dZ^T X: M-block h, token row `row`
-          st_shared_v4(dz + h * 16384 + ((c8 ^ (row & 7)) << 4), o[0], o[1], o[2], o[3]);
+          // MN-major SW128 A operand of E += dZ^T X: M-block p0/64, token row `row`
+          st_shared_v4(dz + (p0 / 64) * 16384 + ((((p0 % 64) / 8) ^ (row & 7)) << 4), o[0], o[1], o[2], o[3]);
         }
       }
       fence_proxy_async_smem();
