@@ -34,7 +34,13 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-constexpr int TQ = 128, TKB = 128, DD = 128, NSK = 3, THREADS = 256;
+#ifndef STCA_NSK
+#define STCA_NSK 3                   // key/value tile stages
+#endif
+#ifndef STCA_POLY_MASK
+#define STCA_POLY_MASK 0x22          // key pairs (of each eight) whose exponential runs on the FMA pipe
+#endif
+constexpr int TQ = 128, TKB = 128, DD = 128, NSK = STCA_NSK, THREADS = 256;
 constexpr uint32_t TILE_BYTES = TQ * DD * 2;                       // 32 KB
 constexpr uint32_t OFF_Q = 0, OFF_KV = TILE_BYTES, OFF_BAR = OFF_KV + NSK * TILE_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
@@ -242,10 +248,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const float2 nm = make_float2(-m, -m);
 #pragma unroll
       for (int i = 0; i < 128; i += 2) {
-        // one pair in four on the FMA pipe (fitted cubic), the rest on the MUFU
+        // the pairs STCA_POLY_MASK selects on the FMA pipe (fitted cubic), the rest on the MUFU
         const float2 e = __fadd2_rn(make_float2(sv[i], sv[i + 1]), nm);
         float2 v;
-        if ((i / 2) % 4 == 1) {
+        if ((STCA_POLY_MASK >> ((i / 2) % 8)) & 1) {
           v = exp2_poly2(e);                 // clamps at 2^-125: a masked key (-inf) must give 0
           v.x = e.x < -125.f ? 0.f : v.x;
           v.y = e.y < -125.f ? 0.f : v.y;
