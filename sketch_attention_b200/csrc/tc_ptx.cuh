@@ -84,8 +84,8 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Plain bulk copy global -> this CTA's shared memory (no multicast; the
-// launching CTA's own address in the shared::cluster window), completing on `bar`.
+// Plain bulk copy global -> this CTA's own shared memory (the destination is the
+// launching CTA's address in the shared::cluster window), completing on `bar`.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
                                           uint64_t* bar) {
   asm volatile(
